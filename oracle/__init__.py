@@ -1,0 +1,226 @@
+"""fp64 CPU oracle for query-aware block-sparse attention.
+
+TEST INFRASTRUCTURE, NOT PRODUCT CODE.  Only the tests, ``__graft_entry__.smoke()`` and
+the CPU-baseline leg of ``bench.py`` may import this package.  The arithmetic lives in
+``lsa_oracle.c`` (plain C, double precision, one loop nest per definition); this module
+only compiles it with gcc and marshals torch CPU tensors into it.  It shares nothing with
+the CUDA library in ``query_aware_block_b200``.
+
+Parity status of each function (what pins it is in tests/test_oracle_pins.py):
+  summaries, block_scores, select, decode_attn, blockquery_select, blockquery_attn,
+  blasst_prefill -- all pinned (textbook special cases, brute force, library routines,
+  closed forms and invariants).
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+import subprocess
+import threading
+
+import numpy as np
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "lsa_oracle.c")
+_LIB_PATH = os.path.join(_HERE, "liblsa_oracle.so")
+_lib = None
+_lock = threading.Lock()
+
+F32, BF16 = 0, 1
+
+
+def build(force: bool = False) -> str:
+    """Compile lsa_oracle.c into liblsa_oracle.so (gcc, -O2, OpenMP, no fast-math)."""
+    if (not force and os.path.exists(_LIB_PATH)
+            and os.path.getmtime(_LIB_PATH) >= os.path.getmtime(_SRC)):
+        return _LIB_PATH
+    tmp = _LIB_PATH + f".tmp{os.getpid()}"
+    cmd = ["gcc", "-O2", "-std=c11", "-fopenmp", "-fPIC", "-shared", "-Wall", "-Wextra",
+           "-fno-fast-math", "-o", tmp, _SRC, "-lm"]
+    subprocess.run(cmd, check=True)
+    os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            build()
+            _lib = ctypes.CDLL(_LIB_PATH)
+            _lib.oracle_num_threads.restype = ctypes.c_int
+    return _lib
+
+
+def _p(t: torch.Tensor | None):
+    if t is None:
+        return ctypes.c_void_p(0)
+    assert t.device.type == "cpu" and t.is_contiguous(), "oracle takes contiguous CPU tensors"
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _dt(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return F32
+    if t.dtype == torch.bfloat16:
+        return BF16
+    raise TypeError(f"oracle inputs are float32 or bfloat16, got {t.dtype}")
+
+
+def _i32(t):
+    return t.to(torch.int32).contiguous()
+
+
+def num_threads() -> int:
+    return int(_load().oracle_num_threads())
+
+
+def set_num_threads(n: int) -> None:
+    _load().oracle_set_num_threads(ctypes.c_int(n))
+
+
+def _scale(scale, D):
+    return 1.0 / math.sqrt(D) if (scale is None or scale <= 0) else float(scale)
+
+
+def summaries(k, seqlens, blk=64):
+    """k [B,Hkv,T_cap,D] -> fp64 summaries [B,Hkv,ceil(T_cap/blk),D] (zeros past each T_b)."""
+    k = k.contiguous()
+    B, Hkv, T_cap, D = k.shape
+    NB_cap = -(-T_cap // blk)
+    out = torch.zeros(B, Hkv, NB_cap, D, dtype=torch.float64)
+    sl = _i32(seqlens)
+    _load().oracle_summaries(_p(k), _dt(k), B, Hkv, T_cap, D, _p(sl), blk, _p(out))
+    return out
+
+
+def block_scores(q, summ, seqlens, blk=64, scale=None):
+    """q [B,Hq,D], fp64 summ [B,Hkv,NB_cap,D] -> fp64 group scores [B,Hkv,NB_cap]."""
+    q = q.contiguous()
+    summ = summ.to(torch.float64).contiguous()
+    B, Hq, D = q.shape
+    _, Hkv, NB_cap, _ = summ.shape
+    G = Hq // Hkv
+    out = torch.empty(B, Hkv, NB_cap, dtype=torch.float64)
+    sl = _i32(seqlens)
+    _load().oracle_block_scores(_p(q), _dt(q), _p(summ), B, Hkv, G, D, NB_cap, _p(sl), blk,
+                                ctypes.c_double(_scale(scale, D)), _p(out))
+    return out
+
+
+def select(scores, seqlens, topk, n_sink, n_local, blk=64):
+    """fp64 scores [B,Hkv,NB_cap] -> (idx [B,Hkv,topk] ascending, -1 pad; nsel [B,Hkv])."""
+    scores = scores.to(torch.float64).contiguous()
+    B, Hkv, NB_cap = scores.shape
+    idx = torch.empty(B, Hkv, topk, dtype=torch.int32)
+    nsel = torch.empty(B, Hkv, dtype=torch.int32)
+    sl = _i32(seqlens)
+    _load().oracle_select(_p(scores), B, Hkv, NB_cap, _p(sl), blk, topk, n_sink, n_local,
+                          _p(idx), _p(nsel))
+    return idx, nsel
+
+
+def decode_attn(q, k, v, seqlens, idx, nsel, blk=64, scale=None):
+    """Sparse decode attention over the listed blocks -> (o fp64 [B,Hq,D], lse fp64 [B,Hq])."""
+    q, k, v = q.contiguous(), k.contiguous(), v.contiguous()
+    assert q.dtype == k.dtype == v.dtype
+    B, Hq, D = q.shape
+    _, Hkv, T_cap, _ = k.shape
+    G = Hq // Hkv
+    idx = _i32(idx)
+    nsel = _i32(nsel)
+    topk = idx.shape[-1]
+    o = torch.empty(B, Hq, D, dtype=torch.float64)
+    lse = torch.empty(B, Hq, dtype=torch.float64)
+    sl = _i32(seqlens)
+    _load().oracle_decode_attn(_p(q), _p(k), _p(v), _dt(q), B, Hkv, G, D, T_cap, _p(sl), blk,
+                               _p(idx), _p(nsel), topk, ctypes.c_double(_scale(scale, D)),
+                               _p(o), _p(lse))
+    return o, lse
+
+
+def decode(q, k, v, seqlens, topk, n_sink, n_local, blk=64, scale=None):
+    """The whole decode path in the oracle: summaries -> scores -> select -> attention."""
+    summ = summaries(k, seqlens, blk)
+    s = block_scores(q, summ, seqlens, blk, scale)
+    idx, nsel = select(s, seqlens, topk, n_sink, n_local, blk)
+    o, lse = decode_attn(q, k, v, seqlens, idx, nsel, blk, scale)
+    return dict(summ=summ, scores=s, idx=idx, nsel=nsel, o=o, lse=lse)
+
+
+def blockquery_select(q, summ, active, T_prefix, topk, n_sink=0, n_local=0, blk=64,
+                      scale=None, return_sel=False):
+    """Per-active-token top-k and the union per (b, kv group).
+
+    q [B,Hq,Tq,D]; fp64 summ [B,Hkv,NB_cap,D]; active [B,Tq] (uint8/bool).
+    Returns union_idx [B,Hkv,NBp] (ascending, -1 pad), union_cnt [B,Hkv] and, if asked,
+    each token's own selection [B,Tq,Hkv,topk]."""
+    q = q.contiguous()
+    summ = summ.to(torch.float64).contiguous()
+    B, Hq, Tq, D = q.shape
+    _, Hkv, NB_cap, _ = summ.shape
+    G = Hq // Hkv
+    NBp = -(-T_prefix // blk)
+    act = active.to(torch.uint8).contiguous()
+    uidx = torch.empty(B, Hkv, NBp, dtype=torch.int32)
+    ucnt = torch.empty(B, Hkv, dtype=torch.int32)
+    sel = torch.empty(B, Tq, Hkv, topk, dtype=torch.int32) if return_sel else None
+    _load().oracle_blockquery_select(_p(q), _dt(q), _p(summ), B, Hkv, G, D, Tq, T_prefix,
+                                     NB_cap, blk, topk, n_sink, n_local,
+                                     ctypes.c_double(_scale(scale, D)), _p(act), _p(uidx),
+                                     _p(ucnt), _p(sel))
+    return (uidx, ucnt, sel) if return_sel else (uidx, ucnt)
+
+
+def blockquery_attn(q, k, v, active, o_cache, lse_cache, union_idx, union_cnt, T_prefix,
+                    blk=64, scale=None):
+    """Active rows attend over the union blocks; stable rows copy the cache.
+
+    -> (o fp64 [B,Hq,Tq,D], lse fp64 [B,Hq,Tq])."""
+    q, k, v = q.contiguous(), k.contiguous(), v.contiguous()
+    B, Hq, Tq, D = q.shape
+    _, Hkv, T_cap, _ = k.shape
+    G = Hq // Hkv
+    act = active.to(torch.uint8).contiguous()
+    oc = o_cache.to(q.dtype).contiguous()
+    lc = lse_cache.to(torch.float32).contiguous()
+    ui = _i32(union_idx)
+    uc = _i32(union_cnt)
+    NBp = -(-T_prefix // blk)
+    assert ui.shape[-1] == NBp
+    o = torch.empty(B, Hq, Tq, D, dtype=torch.float64)
+    lse = torch.empty(B, Hq, Tq, dtype=torch.float64)
+    _load().oracle_blockquery_attn(_p(q), _p(k), _p(v), _dt(q), B, Hkv, G, D, Tq, T_prefix,
+                                   T_cap, blk, ctypes.c_double(_scale(scale, D)), _p(act),
+                                   _p(oc), _p(lc), _p(ui), _p(uc), _p(o), _p(lse))
+    return o, lse
+
+
+def blasst_prefill(q, k, v, units, lam, tq=128, tk=64, scale=None, forced_bits=None):
+    """BLASST causal prefill on a list of (b, h, a) work units.
+
+    q [B,Hq,L,D]; k, v [B,Hkv,L,D]; units int [n,3].
+    Returns dict(o [n,tq,D] fp64, lse [n,tq] fp64, bits [n,words] uint32 as int64,
+    gap [n,nkv] fp64) where words = ceil(ceil(L/tk)/32)."""
+    q, k, v = q.contiguous(), k.contiguous(), v.contiguous()
+    B, Hq, L, D = q.shape
+    Hkv = k.shape[1]
+    units = _i32(torch.as_tensor(units).reshape(-1, 3))
+    n = units.shape[0]
+    nkv = -(-L // tk)
+    words = -(-nkv // 32)
+    o = torch.empty(n, tq, D, dtype=torch.float64)
+    lse = torch.empty(n, tq, dtype=torch.float64)
+    bits = torch.empty(n, words, dtype=torch.int32)
+    gap = torch.empty(n, nkv, dtype=torch.float64)
+    fb = None
+    if forced_bits is not None:
+        fb = np.asarray(torch.as_tensor(forced_bits).to(torch.int64).reshape(n, words))
+        fb = torch.from_numpy((fb & 0xFFFFFFFF).astype(np.uint32).view(np.int32).copy())
+    _load().oracle_blasst_prefill(_p(q), _p(k), _p(v), _dt(q), B, Hq, Hkv, L, D,
+                                  ctypes.c_double(_scale(scale, D)), ctypes.c_double(float(lam)),
+                                  tq, tk, n, _p(units), _p(fb), words, _p(o), _p(lse),
+                                  _p(bits), _p(gap))
+    return dict(o=o, lse=lse, bits=bits.to(torch.int64) & 0xFFFFFFFF, gap=gap)

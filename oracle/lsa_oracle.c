@@ -1,0 +1,509 @@
+/*
+ * lsa_oracle.c -- plain fp64 CPU oracle for query-aware block-sparse attention.
+ *
+ * TEST INFRASTRUCTURE, NOT PRODUCT CODE.  Only the test suite, the smoke check of
+ * __graft_entry__ and the CPU-baseline leg of bench.py may load this library.  It
+ * shares no code, header, table or helper with the CUDA library under
+ * query_aware_block_b200/; neither side includes or links the other.
+ *
+ * Every quantity is computed in double precision from the exact input bits
+ * (bf16 and fp32 inputs are widened exactly to double).  The functions are the
+ * plain definitions of what the method computes, in the order the source pages
+ * describe them, with no blocking, fusion or reordering:
+ *
+ *   oracle_summaries         mean-pooled key summary of each 64-token block
+ *                            [Prism, "1. 문제 정의" and "2. 핵심 이론적 발견":
+ *                             training-free block importance uses mean pooling]
+ *   oracle_block_scores      query-aware block score, shared by a GQA group
+ *                            [NSA news article, "기존 스파스 어텐션 접근법의 한계 분석":
+ *                             query-aware selection scores chunks; "기술 구현의 실제적
+ *                             도전과 해결": GQA compatibility decides memory access]
+ *   oracle_select            top-n selection with forced initial and local blocks
+ *                            [NSA, "NSA 구조": l'=64, n=16 including 1 initial + 2 local]
+ *   oracle_decode_attn       exact softmax attention over the selected tokens, original
+ *                            positions kept [FASA, "2. 방법론", Focused Attention Computation]
+ *   oracle_blockquery_select per active token top-n, union across the query block
+ *                            [LoSA, "1. 문제 정의" (the union sets the traffic) and
+ *                             "2. 방법론" (selection for active tokens only)]
+ *   oracle_blockquery_attn   attention of active rows over the union; stable rows reuse
+ *                            the cached output and statistics [LoSA, "2. 방법론"]
+ *   oracle_blasst_prefill    causal online-softmax attention over KV tiles in ascending
+ *                            order, skipping a tile whose row maxima all trail the running
+ *                            maxima by more than ln(lambda)
+ *                            [BLASST, "2. 방법론", "핵심 아이디어" and "알고리즘 및 커널 설계"]
+ *
+ * Readings taken where the pages are silent (each also listed in the design doc):
+ *   - a partial last block is averaged over its valid tokens only;
+ *   - the GQA group score is the sum over the group's query heads of scale * q_h . kbar;
+ *   - ties in the top-n go to the lower block index;
+ *   - the forced blocks are counted inside the n selected blocks;
+ *   - the BLASST test quantifies over rows: skip iff every row's
+ *     (tile row max - running row max) < ln(lambda); strict '<' as printed.
+ *
+ * Parallelism: OpenMP over independent (batch, kv head) / (batch, head, q tile) units
+ * only; each unit is computed by one thread exactly as a serial loop would.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+enum { ORC_F32 = 0, ORC_BF16 = 1 };
+
+/* Exact widening of one input element to double. */
+static double elem(const void* p, int dtype, size_t i) {
+  if (dtype == ORC_F32) return (double)((const float*)p)[i];
+  uint32_t u = (uint32_t)((const uint16_t*)p)[i] << 16;
+  float f;
+  memcpy(&f, &u, sizeof f);
+  return (double)f;
+}
+
+static int ceil_div(int a, int b) { return (a + b - 1) / b; }
+
+int oracle_num_threads(void) {
+#ifdef _OPENMP
+  return omp_get_max_threads();
+#else
+  return 1;
+#endif
+}
+
+void oracle_set_num_threads(int n) {
+#ifdef _OPENMP
+  if (n > 0) omp_set_num_threads(n);
+#else
+  (void)n;
+#endif
+}
+
+/* ------------------------------------------------------------------------------------
+ * Mean-pooled block summaries.
+ *   summ[b,g,j,:] = (1/n_j) * sum_{t in block j, t < T_b} k[b,g,t,:]
+ * k: [B,Hkv,T_cap,D]; summ: [B,Hkv,NB_cap,D] with NB_cap = ceil(T_cap/blk).
+ * Blocks at or beyond NB_b = ceil(T_b/blk) are written as zeros.
+ * ---------------------------------------------------------------------------------- */
+void oracle_summaries(const void* k, int dtype, int B, int Hkv, int T_cap, int D,
+                      const int32_t* seqlens, int blk, double* summ) {
+  const int NB_cap = ceil_div(T_cap, blk);
+#pragma omp parallel for collapse(2) schedule(dynamic)
+  for (int b = 0; b < B; ++b) {
+    for (int g = 0; g < Hkv; ++g) {
+      const int T = seqlens[b];
+      const int NB = ceil_div(T, blk);
+      for (int j = 0; j < NB_cap; ++j) {
+        double* out = summ + (((size_t)b * Hkv + g) * NB_cap + j) * D;
+        for (int d = 0; d < D; ++d) out[d] = 0.0;
+        if (j >= NB) continue;
+        const int t0 = j * blk;
+        const int t1 = (t0 + blk < T) ? t0 + blk : T;
+        for (int t = t0; t < t1; ++t) {
+          const size_t row = (((size_t)b * Hkv + g) * T_cap + t) * D;
+          for (int d = 0; d < D; ++d) out[d] += elem(k, dtype, row + d);
+        }
+        const double n = (double)(t1 - t0);
+        for (int d = 0; d < D; ++d) out[d] /= n;
+      }
+    }
+  }
+}
+
+/* ------------------------------------------------------------------------------------
+ * Group block scores for one query per sequence (decode).
+ *   scores[b,g,j] = scale * sum_{h in group g} q[b,h,:] . summ[b,g,j,:]   (j < NB_b)
+ * q: [B,Hq,D] with Hq = Hkv*G, query head h belongs to group h / G.
+ * Entries j >= NB_b are -inf.
+ * ---------------------------------------------------------------------------------- */
+void oracle_block_scores(const void* q, int dtype, const double* summ, int B, int Hkv, int G,
+                         int D, int NB_cap, const int32_t* seqlens, int blk, double scale,
+                         double* scores) {
+#pragma omp parallel for collapse(2) schedule(dynamic)
+  for (int b = 0; b < B; ++b) {
+    for (int g = 0; g < Hkv; ++g) {
+      const int NB = ceil_div(seqlens[b], blk);
+      for (int j = 0; j < NB_cap; ++j) {
+        double* s = scores + ((size_t)b * Hkv + g) * NB_cap + j;
+        if (j >= NB) {
+          *s = -INFINITY;
+          continue;
+        }
+        const double* kb = summ + (((size_t)b * Hkv + g) * NB_cap + j) * D;
+        double acc = 0.0;
+        for (int hh = 0; hh < G; ++hh) {
+          const int h = g * G + hh;
+          const size_t qrow = ((size_t)b * Hkv * G + h) * D;
+          double dot = 0.0;
+          for (int d = 0; d < D; ++d) dot += elem(q, dtype, qrow + d) * kb[d];
+          acc += dot;
+        }
+        *s = scale * acc;
+      }
+    }
+  }
+}
+
+/* Candidate ordering for the top-n: higher score first, ties to the lower block index. */
+typedef struct {
+  double score;
+  int j;
+} cand_t;
+
+static int cand_cmp(const void* pa, const void* pb) {
+  const cand_t* a = (const cand_t*)pa;
+  const cand_t* b = (const cand_t*)pb;
+  if (a->score > b->score) return -1;
+  if (a->score < b->score) return 1;
+  return (a->j < b->j) ? -1 : (a->j > b->j);
+}
+
+/* Select from one row of NB scores; writes `topk` ascending indices padded with -1 and
+ * returns the count.  The forced set F = {0..n_sink-1} U {NB-n_local..NB-1} (clipped to
+ * [0,NB)) is always kept and counted inside topk; the remaining topk-|F| slots go to
+ * the highest-scoring blocks outside F.  If NB <= topk every block is kept. */
+static int select_row(const double* s, int NB, int topk, int n_sink, int n_local,
+                      int32_t* idx_out, unsigned char* chosen, cand_t* cands) {
+  for (int j = 0; j < NB; ++j) chosen[j] = 0;
+  if (NB <= topk) {
+    for (int j = 0; j < NB; ++j) chosen[j] = 1;
+  } else {
+    int nforced = 0;
+    for (int j = 0; j < n_sink && j < NB; ++j)
+      if (!chosen[j]) { chosen[j] = 1; ++nforced; }
+    for (int j = NB - n_local; j < NB; ++j)
+      if (j >= 0 && !chosen[j]) { chosen[j] = 1; ++nforced; }
+    int nc = 0;
+    for (int j = 0; j < NB; ++j)
+      if (!chosen[j]) { cands[nc].score = s[j]; cands[nc].j = j; ++nc; }
+    qsort(cands, (size_t)nc, sizeof(cand_t), cand_cmp);
+    const int nfree = topk - nforced;
+    for (int r = 0; r < nfree && r < nc; ++r) chosen[cands[r].j] = 1;
+  }
+  int cnt = 0;
+  for (int j = 0; j < NB; ++j)
+    if (chosen[j]) idx_out[cnt++] = j;
+  for (int r = cnt; r < topk; ++r) idx_out[r] = -1;
+  return cnt;
+}
+
+/* ------------------------------------------------------------------------------------
+ * Decode selection: idx[b,g,:] (ascending, -1 padded), nsel[b,g].
+ * ---------------------------------------------------------------------------------- */
+void oracle_select(const double* scores, int B, int Hkv, int NB_cap, const int32_t* seqlens,
+                   int blk, int topk, int n_sink, int n_local, int32_t* idx, int32_t* nsel) {
+#pragma omp parallel for collapse(2) schedule(dynamic)
+  for (int b = 0; b < B; ++b) {
+    for (int g = 0; g < Hkv; ++g) {
+      const int NB = ceil_div(seqlens[b], blk);
+      unsigned char* chosen = (unsigned char*)malloc((size_t)(NB > 0 ? NB : 1));
+      cand_t* cands = (cand_t*)malloc(sizeof(cand_t) * (size_t)(NB > 0 ? NB : 1));
+      const size_t u = (size_t)b * Hkv + g;
+      nsel[u] = select_row(scores + u * NB_cap, NB, topk, n_sink, n_local, idx + u * topk,
+                           chosen, cands);
+      free(cands);
+      free(chosen);
+    }
+  }
+}
+
+/* Softmax attention of one query row over an explicit token list.
+ * logit_t = scale * q . k_t;  o = sum_t softmax(logit)_t v_t;  lse = log sum_t exp(logit_t).
+ * With no tokens: o = 0, lse = -inf. */
+static void attend_row(const void* q, const void* k, const void* v, int dtype, size_t qrow,
+                       size_t kvbase, int D, const int* toks, int ntok, double scale,
+                       double* logits, double* o, double* lse) {
+  for (int d = 0; d < D; ++d) o[d] = 0.0;
+  if (ntok == 0) {
+    *lse = -INFINITY;
+    return;
+  }
+  double m = -INFINITY;
+  for (int i = 0; i < ntok; ++i) {
+    const size_t krow = kvbase + (size_t)toks[i] * D;
+    double dot = 0.0;
+    for (int d = 0; d < D; ++d) dot += elem(q, dtype, qrow + d) * elem(k, dtype, krow + d);
+    logits[i] = scale * dot;
+    if (logits[i] > m) m = logits[i];
+  }
+  double l = 0.0;
+  for (int i = 0; i < ntok; ++i) {
+    const double p = exp(logits[i] - m);
+    l += p;
+    const size_t vrow = kvbase + (size_t)toks[i] * D;
+    for (int d = 0; d < D; ++d) o[d] += p * elem(v, dtype, vrow + d);
+  }
+  for (int d = 0; d < D; ++d) o[d] /= l;
+  *lse = m + log(l);
+}
+
+/* ------------------------------------------------------------------------------------
+ * Sparse decode attention over the selected blocks.
+ * q [B,Hq,D]; k,v [B,Hkv,T_cap,D]; idx [B,Hkv,topk] (-1 = unused slot); nsel [B,Hkv].
+ * Token set of group g: {t : floor(t/blk) in idx[b,g,:nsel], t < T_b}.
+ * o [B,Hq,D], lse [B,Hq].
+ * ---------------------------------------------------------------------------------- */
+void oracle_decode_attn(const void* q, const void* k, const void* v, int dtype, int B, int Hkv,
+                        int G, int D, int T_cap, const int32_t* seqlens, int blk,
+                        const int32_t* idx, const int32_t* nsel, int topk, double scale,
+                        double* o, double* lse) {
+  const int Hq = Hkv * G;
+#pragma omp parallel for collapse(2) schedule(dynamic)
+  for (int b = 0; b < B; ++b) {
+    for (int g = 0; g < Hkv; ++g) {
+      const int T = seqlens[b];
+      const size_t u = (size_t)b * Hkv + g;
+      int* toks = (int*)malloc(sizeof(int) * (size_t)(topk * blk + 1));
+      double* logits = (double*)malloc(sizeof(double) * (size_t)(topk * blk + 1));
+      int ntok = 0;
+      for (int r = 0; r < nsel[u]; ++r) {
+        const int j = idx[u * topk + r];
+        if (j < 0) continue;
+        for (int t = j * blk; t < j * blk + blk && t < T; ++t) toks[ntok++] = t;
+      }
+      const size_t kvbase = u * (size_t)T_cap * D;
+      for (int hh = 0; hh < G; ++hh) {
+        const int h = g * G + hh;
+        const size_t qrow = ((size_t)b * Hq + h) * D;
+        attend_row(q, k, v, dtype, qrow, kvbase, D, toks, ntok, scale, logits,
+                   o + ((size_t)b * Hq + h) * D, lse + (size_t)b * Hq + h);
+      }
+      free(logits);
+      free(toks);
+    }
+  }
+}
+
+/* ------------------------------------------------------------------------------------
+ * Block-query selection (diffusion-LM step).
+ * q [B,Hq,Tq,D]; summ [B,Hkv,NB_cap,D] (double); active [B,Tq] (1 = active token).
+ * For every active token i and group g: the scores over the NBp = ceil(T_prefix/blk)
+ * prefix blocks are scale * sum_{h in g} q[b,h,i,:] . summ[b,g,j,:]; the token keeps its
+ * top-`topk` blocks (forced set as in oracle_select).  union_idx[b,g,:] lists the union
+ * over active tokens in ascending order (capacity NBp, -1 padded); union_cnt[b,g] its size.
+ * sel (optional) receives each token's own selection [B,Tq,Hkv,topk] (-1 rows if stable).
+ * ---------------------------------------------------------------------------------- */
+void oracle_blockquery_select(const void* q, int dtype, const double* summ, int B, int Hkv,
+                              int G, int D, int Tq, int T_prefix, int NB_cap, int blk,
+                              int topk, int n_sink, int n_local, double scale,
+                              const uint8_t* active, int32_t* union_idx, int32_t* union_cnt,
+                              int32_t* sel) {
+  const int Hq = Hkv * G;
+  const int NBp = ceil_div(T_prefix, blk);
+#pragma omp parallel for collapse(2) schedule(dynamic)
+  for (int b = 0; b < B; ++b) {
+    for (int g = 0; g < Hkv; ++g) {
+      const size_t u = (size_t)b * Hkv + g;
+      const int nb1 = NBp > 0 ? NBp : 1;
+      unsigned char* in_union = (unsigned char*)calloc((size_t)nb1, 1);
+      unsigned char* chosen = (unsigned char*)malloc((size_t)nb1);
+      cand_t* cands = (cand_t*)malloc(sizeof(cand_t) * (size_t)nb1);
+      double* s = (double*)malloc(sizeof(double) * (size_t)nb1);
+      int32_t* mine = (int32_t*)malloc(sizeof(int32_t) * (size_t)(topk > 0 ? topk : 1));
+      for (int i = 0; i < Tq; ++i) {
+        int32_t* sel_row = sel ? sel + (((size_t)b * Tq + i) * Hkv + g) * topk : NULL;
+        if (!active[(size_t)b * Tq + i]) {
+          if (sel_row)
+            for (int r = 0; r < topk; ++r) sel_row[r] = -1;
+          continue;
+        }
+        for (int j = 0; j < NBp; ++j) {
+          const double* kb = summ + (((size_t)b * Hkv + g) * NB_cap + j) * D;
+          double acc = 0.0;
+          for (int hh = 0; hh < G; ++hh) {
+            const int h = g * G + hh;
+            const size_t qrow = (((size_t)b * Hq + h) * Tq + i) * D;
+            double dot = 0.0;
+            for (int d = 0; d < D; ++d) dot += elem(q, dtype, qrow + d) * kb[d];
+            acc += dot;
+          }
+          s[j] = scale * acc;
+        }
+        const int cnt = select_row(s, NBp, topk, n_sink, n_local, mine, chosen, cands);
+        for (int r = 0; r < cnt; ++r) in_union[mine[r]] = 1;
+        if (sel_row)
+          for (int r = 0; r < topk; ++r) sel_row[r] = mine[r];
+      }
+      int c = 0;
+      for (int j = 0; j < NBp; ++j)
+        if (in_union[j]) union_idx[u * NBp + c++] = j;
+      for (int r = c; r < NBp; ++r) union_idx[u * NBp + r] = -1;
+      union_cnt[u] = c;
+      free(mine);
+      free(s);
+      free(cands);
+      free(chosen);
+      free(in_union);
+    }
+  }
+}
+
+/* ------------------------------------------------------------------------------------
+ * Block-query attention.
+ * Active row (b, h, i): softmax attention over every prefix token t < T_prefix whose block
+ * is in union_idx[b, h/G, :union_cnt] (no mask inside the prefix).
+ * Stable row: o and lse are the cached values, unchanged.
+ * q, o_cache: [B,Hq,Tq,D]; lse_cache: [B,Hq,Tq]; union_idx: [B,Hkv,NBp].
+ * ---------------------------------------------------------------------------------- */
+void oracle_blockquery_attn(const void* q, const void* k, const void* v, int dtype, int B,
+                            int Hkv, int G, int D, int Tq, int T_prefix, int T_cap, int blk,
+                            double scale, const uint8_t* active, const void* o_cache,
+                            const float* lse_cache, const int32_t* union_idx,
+                            const int32_t* union_cnt, double* o, double* lse) {
+  const int Hq = Hkv * G;
+  const int NBp = ceil_div(T_prefix, blk);
+#pragma omp parallel for collapse(2) schedule(dynamic)
+  for (int b = 0; b < B; ++b) {
+    for (int g = 0; g < Hkv; ++g) {
+      const size_t u = (size_t)b * Hkv + g;
+      const int cnt = union_cnt[u];
+      int* toks = (int*)malloc(sizeof(int) * ((size_t)cnt * blk + 1));
+      double* logits = (double*)malloc(sizeof(double) * ((size_t)cnt * blk + 1));
+      int ntok = 0;
+      for (int r = 0; r < cnt; ++r) {
+        const int j = union_idx[u * NBp + r];
+        if (j < 0) continue;
+        for (int t = j * blk; t < j * blk + blk && t < T_prefix; ++t) toks[ntok++] = t;
+      }
+      const size_t kvbase = u * (size_t)T_cap * D;
+      for (int hh = 0; hh < G; ++hh) {
+        const int h = g * G + hh;
+        for (int i = 0; i < Tq; ++i) {
+          const size_t row = ((size_t)b * Hq + h) * Tq + i;
+          if (active[(size_t)b * Tq + i]) {
+            attend_row(q, k, v, dtype, row * D, kvbase, D, toks, ntok, scale, logits,
+                       o + row * D, lse + row);
+          } else {
+            for (int d = 0; d < D; ++d) o[row * D + d] = elem(o_cache, dtype, row * D + d);
+            lse[row] = (double)lse_cache[row];
+          }
+        }
+      }
+      free(logits);
+      free(toks);
+    }
+  }
+}
+
+/* ------------------------------------------------------------------------------------
+ * BLASST causal prefill, for a list of work units (b, h, a): query head h of sequence b,
+ * query tile a = rows [tq*a, min(tq*a+tq, L)).  KV tiles c = 0,1,... of tk keys are visited
+ * in ascending order up to the causal diagonal.  For each tile:
+ *   S_it = scale * q_i . k_t, with S_it = -inf where t > i or t >= L;
+ *   r_i  = max_t S_it  (the tile's row max);   gap = max over the tile's rows of (r_i - m_i)
+ *   where m_i is the running row max (-inf before the first tile; (-inf) - x = -inf);
+ *   skip  iff gap < ln(lambda)      (lambda = 0 gives ln = -inf: never skip);
+ *   else  m' = max(m, r); l = l e^{m-m'} + sum_t e^{S-m'}; acc = acc e^{m-m'} + sum_t e^{S-m'} v_t.
+ * Finally o = acc / l and lse = m + ln l.
+ * If forced_bits is given, the skip decision of tile c is read from it (bit c of the
+ * unit's row) instead, so the output can be evaluated on another implementation's
+ * decisions; the gap is still reported.
+ * Outputs per unit u: o[u, tq, D], lse[u, tq] (rows >= L are left 0 / -inf),
+ * skip_bits[u, words] (bit c set iff tile c was skipped), gap[u, nkv] (NaN if unvisited).
+ * q [B,Hq,L,D]; k,v [B,Hkv,L,D]; head h reads kv head h / (Hq/Hkv).
+ * ---------------------------------------------------------------------------------- */
+void oracle_blasst_prefill(const void* q, const void* k, const void* v, int dtype, int B, int Hq,
+                           int Hkv, int L, int D, double scale, double lambda, int tq, int tk,
+                           int n_units, const int32_t* units, const uint32_t* forced_bits,
+                           int words, double* o, double* lse, uint32_t* skip_bits,
+                           double* gap_out) {
+  (void)B;
+  const int G = Hq / Hkv;
+  const int nkv = ceil_div(L, tk);
+  const double ln_lambda = (lambda > 0.0) ? log(lambda) : -INFINITY;
+#pragma omp parallel for schedule(dynamic)
+  for (int uidx = 0; uidx < n_units; ++uidx) {
+    const int b = units[3 * uidx + 0];
+    const int h = units[3 * uidx + 1];
+    const int a = units[3 * uidx + 2];
+    const int g = h / G;
+    const int i0 = a * tq;
+    const int i1 = (i0 + tq < L) ? i0 + tq : L;
+    const int nrows = i1 - i0;
+    double* m = (double*)malloc(sizeof(double) * (size_t)tq);
+    double* l = (double*)malloc(sizeof(double) * (size_t)tq);
+    double* r = (double*)malloc(sizeof(double) * (size_t)tq);
+    double* S = (double*)malloc(sizeof(double) * (size_t)tq * tk);
+    double* acc = o + (size_t)uidx * tq * D;
+    double* lse_u = lse + (size_t)uidx * tq;
+    uint32_t* bits = skip_bits + (size_t)uidx * words;
+    for (int w = 0; w < words; ++w) bits[w] = 0u;
+    for (int c = 0; c < nkv; ++c) gap_out[(size_t)uidx * nkv + c] = NAN;
+    for (int ii = 0; ii < tq; ++ii) {
+      m[ii] = -INFINITY;
+      l[ii] = 0.0;
+      for (int d = 0; d < D; ++d) acc[(size_t)ii * D + d] = 0.0;
+      lse_u[ii] = -INFINITY;
+    }
+    const size_t qbase = ((size_t)b * Hq + h) * (size_t)L * D;
+    const size_t kvbase = ((size_t)b * Hkv + g) * (size_t)L * D;
+    const int last_key = i1 - 1; /* the largest key any row of this tile may see */
+    const int n_visit = last_key / tk + 1;
+    for (int c = 0; c < n_visit; ++c) {
+      const int t0 = c * tk;
+      /* logits and row maxima of this tile */
+      for (int ii = 0; ii < nrows; ++ii) {
+        const int i = i0 + ii;
+        r[ii] = -INFINITY;
+        for (int tt = 0; tt < tk; ++tt) {
+          const int t = t0 + tt;
+          double sv = -INFINITY;
+          if (t <= i && t < L) {
+            double dot = 0.0;
+            for (int d = 0; d < D; ++d)
+              dot += elem(q, dtype, qbase + (size_t)i * D + d) *
+                     elem(k, dtype, kvbase + (size_t)t * D + d);
+            sv = scale * dot;
+          }
+          S[(size_t)ii * tk + tt] = sv;
+          if (sv > r[ii]) r[ii] = sv;
+        }
+      }
+      /* the skip test: every row negligible */
+      double gap = -INFINITY;
+      for (int ii = 0; ii < nrows; ++ii) {
+        double gi;
+        if (r[ii] == -INFINITY) gi = -INFINITY;
+        else if (m[ii] == -INFINITY) gi = INFINITY;
+        else gi = r[ii] - m[ii];
+        if (gi > gap) gap = gi;
+      }
+      gap_out[(size_t)uidx * nkv + c] = gap;
+      int skip;
+      if (forced_bits) skip = (int)((forced_bits[(size_t)uidx * words + c / 32] >> (c % 32)) & 1u);
+      else skip = gap < ln_lambda;
+      if (skip) {
+        bits[c / 32] |= 1u << (c % 32);
+        continue;
+      }
+      /* online-softmax update */
+      for (int ii = 0; ii < nrows; ++ii) {
+        const double mn = (r[ii] > m[ii]) ? r[ii] : m[ii];
+        if (mn == -INFINITY) continue; /* row has seen no key yet */
+        const double alpha = (m[ii] == -INFINITY) ? 0.0 : exp(m[ii] - mn);
+        l[ii] *= alpha;
+        double* arow = acc + (size_t)ii * D;
+        for (int d = 0; d < D; ++d) arow[d] *= alpha;
+        for (int tt = 0; tt < tk; ++tt) {
+          const double sv = S[(size_t)ii * tk + tt];
+          if (sv == -INFINITY) continue;
+          const double p = exp(sv - mn);
+          l[ii] += p;
+          const size_t vrow = kvbase + (size_t)(t0 + tt) * D;
+          for (int d = 0; d < D; ++d) arow[d] += p * elem(v, dtype, vrow + d);
+        }
+        m[ii] = mn;
+      }
+    }
+    for (int ii = 0; ii < nrows; ++ii) {
+      double* arow = acc + (size_t)ii * D;
+      for (int d = 0; d < D; ++d) arow[d] /= l[ii];
+      lse_u[ii] = m[ii] + log(l[ii]);
+    }
+    free(S);
+    free(r);
+    free(l);
+    free(m);
+  }
+}

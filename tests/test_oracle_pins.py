@@ -1,0 +1,468 @@
+"""Pins for the fp64 oracle: every check here ties the oracle to something other than
+itself -- textbook special cases, closed forms, brute-force enumeration, library routines
+(torch scaled_dot_product_attention / logsumexp / topk in fp64) and invariants of the
+method -- so that a dropped term, a wrong sign or index, or a transposed operand in
+oracle/lsa_oracle.c fails at least one of them.  CPU only."""
+import itertools
+import json
+import math
+import os
+
+import pytest
+import torch
+import torch.nn.functional as F
+
+import oracle
+import synth
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _bf(x):
+    return x.to(torch.bfloat16)
+
+
+# ---------------------------------------------------------------- rotary generator ----
+
+def test_rope_preserves_norm_and_is_relative():
+    g = torch.Generator().manual_seed(0)
+    D = 64
+    x = torch.randn(5, D, generator=g, dtype=torch.float64)
+    pos = torch.tensor([0, 3, 17, 1000, 65535])
+    y = synth.rope(x, pos, 1e4)
+    assert torch.allclose(y.norm(dim=-1), x.norm(dim=-1), rtol=0, atol=1e-12)
+    # R(m) q . R(n) k depends only on m - n
+    q = torch.randn(D, generator=g, dtype=torch.float64)
+    k = torch.randn(D, generator=g, dtype=torch.float64)
+    d1 = (synth.rope(q[None], torch.tensor([10]), 1e4) * synth.rope(k[None], torch.tensor([4]), 1e4)).sum()
+    d2 = (synth.rope(q[None], torch.tensor([106]), 1e4) * synth.rope(k[None], torch.tensor([100]), 1e4)).sum()
+    assert abs(float(d1 - d2)) < 1e-10
+    # position 0 is the identity
+    assert torch.allclose(synth.rope(q[None], torch.tensor([0]), 1e4)[0], q, atol=0)
+
+
+# ---------------------------------------------------------------------- summaries ----
+
+def test_summary_of_constant_keys_is_exact():
+    B, Hkv, T, D = 2, 3, 200, 16
+    c = torch.randn(B, Hkv, 1, D).expand(B, Hkv, T, D).contiguous()
+    s = oracle.summaries(c, torch.tensor([200, 77]))
+    # NB_cap = 4; sequence 0 has 4 blocks (last one 8 tokens), sequence 1 has 2 blocks
+    for j in range(4):
+        assert torch.equal(s[0, :, j], c[0, :, 0].double())
+    for j in range(2):
+        assert torch.equal(s[1, :, j], c[1, :, 0].double())
+    assert torch.count_nonzero(s[1, :, 2:]) == 0
+
+
+def test_summary_partial_block_closed_form():
+    # keys k_t = t in every dim: the mean of block j is (t0 + t1 - 1) / 2 over valid tokens
+    T_cap, T = 256, 150
+    k = torch.arange(T_cap, dtype=torch.float32).view(1, 1, T_cap, 1).expand(1, 1, T_cap, 4).contiguous()
+    s = oracle.summaries(k, torch.tensor([T]))
+    expect = [(0 + 63) / 2, (64 + 127) / 2, (128 + 149) / 2, 0.0]
+    assert s[0, 0, :, 0].tolist() == expect
+
+
+def test_summary_is_dirichlet_low_pass_of_rotated_constant():
+    # Mean pooling of a rotated constant over n positions scales each rotary pair's
+    # magnitude by |sin(n w / 2) / (n sin(w / 2))| (Dirichlet kernel) -- the low-pass
+    # effect of mean pooling on RoPE dims [Prism, "2. 핵심 이론적 발견"].
+    D, theta, T = 32, 1e4, 64 + 40
+    c = torch.randn(D, dtype=torch.float64, generator=torch.Generator().manual_seed(3))
+    keys = synth.rope(c.expand(T, D), torch.arange(T), theta).to(torch.float32)
+    s = oracle.summaries(keys.view(1, 1, T, D).contiguous(), torch.tensor([T]))
+    half = D // 2
+    cf = c.to(torch.float32).double()
+    for j, n in ((0, 64), (1, 40)):
+        for p in range(half):
+            w = theta ** (-2.0 * p / D)
+            ratio = abs(math.sin(n * w / 2) / (n * math.sin(w / 2)))
+            mag_c = math.hypot(cf[p], cf[p + half])
+            mag_s = math.hypot(s[0, 0, j, p], s[0, 0, j, p + half])
+            assert abs(mag_s - ratio * mag_c) < 2e-6 * (1 + mag_c), (j, p)
+    # the highest-frequency pair is strongly attenuated, the lowest is not
+    assert math.hypot(s[0, 0, 0, 0], s[0, 0, 0, half]) < 0.05 * math.hypot(cf[0], cf[half])
+    assert math.hypot(s[0, 0, 0, half - 1], s[0, 0, 0, D - 1]) > 0.99 * math.hypot(cf[half - 1], cf[D - 1])
+
+
+def test_summary_bf16_widening_is_exact():
+    k = torch.randn(1, 1, 64, 8).to(torch.bfloat16)
+    s = oracle.summaries(k, torch.tensor([64]))
+    exact = k.double().sum(dim=2) / 64.0
+    assert torch.allclose(s[0, :, 0], exact[0], rtol=0, atol=1e-15)
+
+
+# ------------------------------------------------------------------------- scores ----
+
+def test_group_score_is_sum_of_single_head_scores():
+    # a group score with G heads equals the sum of the scores of each head on its own;
+    # catches a dropped head or a wrong head -> group mapping (h belongs to group h // G)
+    g = torch.Generator().manual_seed(5)
+    B, Hkv, G, D, T = 2, 3, 4, 16, 320
+    q = torch.randn(B, Hkv * G, D, generator=g)
+    summ = torch.randn(B, Hkv, 5, D, generator=g, dtype=torch.float64)
+    sl = torch.tensor([320, 130])
+    full = oracle.block_scores(q, summ, sl, scale=0.25)
+    acc = torch.zeros_like(full)
+    for hh in range(G):
+        qh = q.view(B, Hkv, G, D)[:, :, hh].contiguous()  # one head per group
+        acc += oracle.block_scores(qh, summ, sl, scale=0.25)
+    valid = torch.isfinite(full)
+    assert torch.allclose(full[valid], acc[valid], rtol=1e-13, atol=1e-13)
+    assert valid[1].sum() == Hkv * 3  # 130 tokens -> 3 blocks
+    assert torch.isinf(full[1, :, 3:]).all() and (full[1, :, 3:] < 0).all()
+
+
+def test_score_sign_and_scale():
+    # a block whose summary points along the summed query scores highest (Cauchy-Schwarz);
+    # the anti-aligned block scores lowest; the score scales linearly with `scale`
+    D, G = 8, 2
+    q = torch.tensor([[1.0, 2, 0, 0, 0, 0, 0, 1], [0.0, 1, 1, 0, 0, 0, 0, 0]]).view(1, G, D)
+    u = q.sum(dim=1)[0].double()
+    u = u / u.norm()
+    summ = torch.randn(1, 1, 6, D, dtype=torch.float64, generator=torch.Generator().manual_seed(1))
+    summ = summ / summ.norm(dim=-1, keepdim=True)
+    summ[0, 0, 2] = u
+    summ[0, 0, 4] = -u
+    s1 = oracle.block_scores(q, summ, torch.tensor([6 * 64]), scale=1.0)[0, 0]
+    s3 = oracle.block_scores(q, summ, torch.tensor([6 * 64]), scale=3.0)[0, 0]
+    assert int(s1.argmax()) == 2 and int(s1.argmin()) == 4
+    assert abs(float(s1[2]) - float(q.sum(dim=1)[0].double().norm())) < 1e-12
+    assert torch.allclose(s3, 3 * s1, rtol=1e-14, atol=0)
+
+
+# ----------------------------------------------------------------------- selection ----
+
+def _brute_best_sum(s, NB, k, forced):
+    free = [j for j in range(NB) if j not in forced]
+    best = -math.inf
+    for comb in itertools.combinations(free, k - len(forced)):
+        best = max(best, sum(s[j] for j in comb))
+    return best
+
+
+@pytest.mark.parametrize("NB,k,ns,nl", [(10, 5, 1, 2), (12, 6, 0, 0), (9, 4, 2, 1), (11, 3, 1, 2)])
+def test_select_matches_brute_force(NB, k, ns, nl):
+    g = torch.Generator().manual_seed(NB * 100 + k)
+    for trial in range(20):
+        s = torch.randn(1, 1, NB, generator=g, dtype=torch.float64)
+        idx, nsel = oracle.select(s, torch.tensor([NB * 64]), k, ns, nl)
+        chosen = [int(j) for j in idx[0, 0] if j >= 0]
+        assert int(nsel[0, 0]) == k == len(chosen)
+        assert chosen == sorted(chosen)
+        forced = set(range(ns)) | set(range(NB - nl, NB))
+        assert forced <= set(chosen)
+        got = sum(float(s[0, 0, j]) for j in chosen if j not in forced)
+        assert abs(got - _brute_best_sum(s[0, 0].tolist(), NB, k, forced)) < 1e-12
+
+
+def test_select_agrees_with_torch_topk():
+    g = torch.Generator().manual_seed(9)
+    NB, k = 1024, 16
+    s = torch.randn(1, 1, NB, generator=g, dtype=torch.float64)
+    idx, _ = oracle.select(s, torch.tensor([NB * 64]), k, 1, 2)
+    masked = s[0, 0].clone()
+    masked[[0, NB - 2, NB - 1]] = -math.inf
+    top = torch.topk(masked, k - 3).indices.tolist()
+    assert idx[0, 0].tolist() == sorted(top + [0, NB - 2, NB - 1])
+
+
+def test_select_ties_go_to_lower_index_and_small_nb_takes_all():
+    s = torch.zeros(1, 1, 8, dtype=torch.float64)
+    s[0, 0, 5] = 1.0
+    idx, nsel = oracle.select(s, torch.tensor([8 * 64]), 4, 0, 0)
+    assert idx[0, 0].tolist() == [0, 1, 2, 5]
+    idx, nsel = oracle.select(s, torch.tensor([3 * 64 + 1]), 6, 1, 2)  # NB = 4 <= 6
+    assert idx[0, 0].tolist() == [0, 1, 2, 3, -1, -1] and int(nsel[0, 0]) == 4
+    idx, nsel = oracle.select(s, torch.tensor([0]), 4, 1, 2)  # empty sequence
+    assert idx[0, 0].tolist() == [-1] * 4 and int(nsel[0, 0]) == 0
+
+
+def test_nsa_token_accounting_golden():
+    # The NSA page gives, for 64K decoding, 5,632 tokens touched instead of 65,536 with
+    # compression block 32 / stride 16, 16 selected blocks of 64 *including* the initial
+    # block and 2 local blocks, and a 512-token window.  The selection count that makes
+    # the total come out is 16 blocks (forced inside n), which is what the oracle keeps.
+    with open(os.path.join(GOLDEN, "nsa_decode_token_accounting.json")) as f:
+        gold = json.load(f)
+    T = gold["context"]
+    NB = T // gold["selection_block"]
+    s = torch.randn(1, 1, NB, dtype=torch.float64, generator=torch.Generator().manual_seed(2))
+    _, nsel = oracle.select(s, torch.tensor([T]), gold["selected_blocks"], 1, 2)
+    compressed = T // gold["compression_stride"]
+    total = compressed + int(nsel[0, 0]) * gold["selection_block"] + gold["window"]
+    assert total == gold["tokens_accessed"]
+
+
+# ------------------------------------------------------------------ decode attention ----
+
+def _sdpa64(q, k, v, mask=None):
+    """Library routine: fp64 scaled dot-product attention (default scale 1/sqrt(D))."""
+    return F.scaled_dot_product_attention(q.double(), k.double(), v.double(), attn_mask=mask)
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_decode_with_all_blocks_equals_dense(dtype):
+    B, Hkv, G, D = 2, 2, 3, 32
+    case = synth.decode_case(B, Hkv, G, D, T_cap=300, seqlens=[300, 190], dtype=dtype,
+                             topk=8, n_sink=1, n_local=2, seed=11, poison_tail=True)
+    r = oracle.decode(case.q, case.k, case.v, case.seqlens, case.topk, 1, 2)
+    assert r["nsel"].tolist() == [[5, 5], [3, 3]]
+    for b in range(B):
+        T = int(case.seqlens[b])
+        for h in range(Hkv * G):
+            g = h // G
+            ref = _sdpa64(case.q[b, h][None, None], case.k[b, g, :T][None], case.v[b, g, :T][None])
+            assert torch.allclose(r["o"][b, h], ref[0, 0], rtol=0, atol=1e-12)
+            logits = case.q[b, h].double() @ case.k[b, g, :T].double().T / math.sqrt(D)
+            assert abs(float(r["lse"][b, h] - torch.logsumexp(logits, 0))) < 1e-12
+
+
+def test_decode_subset_equals_masked_dense_and_ignores_tail():
+    B, Hkv, G, D, T = 1, 2, 2, 64, 1000  # last block partial (1000 = 15*64 + 40)
+    case = synth.decode_case(B, Hkv, G, D, T_cap=1024, seqlens=T, dtype=torch.bfloat16,
+                             topk=5, n_sink=1, n_local=2, seed=12, poison_tail=True)
+    r = oracle.decode(case.q, case.k, case.v, case.seqlens, 5, 1, 2)
+    assert torch.isfinite(r["o"]).all()
+    for g in range(Hkv):
+        blocks = [int(j) for j in r["idx"][0, g] if j >= 0]
+        assert blocks[0] == 0 and blocks[-2:] == [14, 15]
+        mask = torch.zeros(T, dtype=torch.bool)
+        for j in blocks:
+            mask[j * 64:min(j * 64 + 64, T)] = True
+        for hh in range(G):
+            h = g * G + hh
+            ref = _sdpa64(case.q[0, h][None, None], case.k[0, g, :T][None], case.v[0, g, :T][None],
+                          mask=mask[None, None])
+            assert torch.allclose(r["o"][0, h], ref[0, 0], rtol=0, atol=1e-12)
+
+
+def test_decode_uniform_keys_give_mean_of_values():
+    D = 16
+    k = torch.zeros(1, 1, 128, D)
+    k[0, 0, 64:] = torch.randn(D)  # all keys of block 1 equal
+    v = torch.randn(1, 1, 128, D)
+    q = torch.randn(1, 1, D)
+    o, lse = oracle.decode_attn(q, k, v, torch.tensor([128]), torch.tensor([[[1]]]),
+                                torch.tensor([[1]]))
+    assert torch.allclose(o[0, 0], v[0, 0, 64:].double().mean(0), rtol=0, atol=1e-14)
+    logit = float(q[0, 0].double() @ k[0, 0, 64].double()) / 4.0
+    assert abs(float(lse[0, 0]) - (logit + math.log(64))) < 1e-12
+
+
+def test_decode_split_merge_associativity():
+    # attention over blocks S = S1 U S2 equals the log-sum-exp merge of the two halves
+    case = synth.decode_case(1, 1, 4, 32, 640, 640, torch.float32, 6, 0, 0, seed=13)
+    idx = torch.tensor([[[0, 2, 3, 5, 7, 9]]])
+    full_o, full_l = oracle.decode_attn(case.q, case.k, case.v, case.seqlens, idx, torch.tensor([[6]]))
+    o1, l1 = oracle.decode_attn(case.q, case.k, case.v, case.seqlens, idx[..., :2].contiguous(), torch.tensor([[2]]))
+    o2, l2 = oracle.decode_attn(case.q, case.k, case.v, case.seqlens, idx[..., 2:].contiguous(), torch.tensor([[4]]))
+    lm = torch.logaddexp(l1, l2)
+    om = o1 * torch.exp(l1 - lm)[..., None] + o2 * torch.exp(l2 - lm)[..., None]
+    assert torch.allclose(lm, full_l, rtol=0, atol=1e-12)
+    assert torch.allclose(om, full_o, rtol=0, atol=1e-12)
+
+
+def test_decode_block_permutation_invariance_without_rope():
+    # with no rotary embedding and no forced blocks, permuting the KV blocks permutes the
+    # selection and leaves the output unchanged
+    B, Hkv, G, D, NB = 1, 2, 2, 16, 12
+    case = synth.decode_case(B, Hkv, G, D, NB * 64, NB * 64, torch.float32, 4, 0, 0,
+                             theta=1e30, seed=14)  # theta -> inf: all angles ~ 0
+    perm = torch.randperm(NB, generator=torch.Generator().manual_seed(4))
+    kp = case.k.view(B, Hkv, NB, 64, D)[:, :, perm].reshape(case.k.shape).contiguous()
+    vp = case.v.view(B, Hkv, NB, 64, D)[:, :, perm].reshape(case.v.shape).contiguous()
+    r0 = oracle.decode(case.q, case.k, case.v, case.seqlens, 4, 0, 0)
+    r1 = oracle.decode(case.q, kp, vp, case.seqlens, 4, 0, 0)
+    inv = torch.argsort(perm)
+    for g in range(Hkv):
+        a = sorted(int(j) for j in r0["idx"][0, g])
+        b = sorted(int(perm[int(j)]) for j in r1["idx"][0, g])
+        assert a == b
+        assert sorted(int(inv[j]) for j in a) == [int(j) for j in r1["idx"][0, g]]
+    assert torch.allclose(r0["o"], r1["o"], rtol=0, atol=1e-12)
+
+
+# --------------------------------------------------------------------- block-query ----
+
+def _bq_run(case, topk=None):
+    sl = torch.full((case.k.shape[0],), case.T_prefix, dtype=torch.int32)
+    summ = oracle.summaries(case.k[:, :, :case.T_prefix].contiguous(), sl)
+    ui, uc, sel = oracle.blockquery_select(case.q, summ, case.active, case.T_prefix,
+                                           topk or case.topk, case.n_sink, case.n_local,
+                                           return_sel=True)
+    o, lse = oracle.blockquery_attn(case.q, case.k, case.v, case.active, case.o_cache,
+                                    case.lse_cache, ui, uc, case.T_prefix)
+    return summ, ui, uc, sel, o, lse
+
+
+def test_blockquery_union_is_union_of_token_selections():
+    case = synth.blockquery_case(B=2, Hkv=2, G=2, D=32, Tq=8, T_prefix=1024, n_active=3,
+                                 topk=4, seed=21)
+    summ, ui, uc, sel, o, lse = _bq_run(case)
+    NB = 16
+    for b in range(2):
+        A = int(case.active[b].sum())
+        for g in range(2):
+            want = set()
+            for i in range(8):
+                row = [int(j) for j in sel[b, i, g] if j >= 0]
+                if case.active[b, i]:
+                    assert len(row) == 4
+                    want |= set(row)
+                else:
+                    assert row == []
+            got = [int(j) for j in ui[b, g] if j >= 0]
+            assert got == sorted(want) and int(uc[b, g]) == len(got)
+            assert len(got) <= min(NB, 4 * A)
+
+
+def test_blockquery_token_selection_brute_force():
+    # each active token's own selection maximises the summed block scores (tiny NB)
+    case = synth.blockquery_case(B=1, Hkv=1, G=2, D=16, Tq=4, T_prefix=10 * 64, n_active=4,
+                                 topk=3, seed=22)
+    summ, ui, uc, sel, o, lse = _bq_run(case)
+    for i in range(4):
+        qi = case.q[:, :, i].contiguous()  # [1, G, D]
+        s = oracle.block_scores(qi, summ, torch.tensor([640]))[0, 0].tolist()
+        chosen = [int(j) for j in sel[0, i, 0]]
+        assert abs(sum(s[j] for j in chosen) - _brute_best_sum(s, 10, 3, set())) < 1e-12
+
+
+def test_blockquery_identical_queries_union_equals_topk():
+    case = synth.blockquery_case(B=1, Hkv=2, G=2, D=32, Tq=8, T_prefix=2048, n_active=8,
+                                 topk=5, seed=23, same_query=True)
+    _, ui, uc, _, _, _ = _bq_run(case)
+    assert uc.tolist() == [[5, 5]]
+
+
+def test_blockquery_all_stable_is_cache_bit_exact():
+    case = synth.blockquery_case(B=1, Hkv=2, G=2, D=32, Tq=8, T_prefix=1024, n_active=0,
+                                 topk=4, seed=24)
+    _, ui, uc, _, o, lse = _bq_run(case)
+    assert uc.tolist() == [[0, 0]]
+    assert torch.equal(o, case.o_cache.double()) and torch.equal(lse, case.lse_cache.double())
+
+
+def test_blockquery_all_blocks_equals_dense_prefix_attention():
+    case = synth.blockquery_case(B=1, Hkv=2, G=2, D=32, Tq=6, T_prefix=400, T_cap=512,
+                                 n_active=4, topk=16, seed=25)
+    _, ui, uc, _, o, lse = _bq_run(case)
+    assert uc.tolist() == [[7, 7]]
+    for h in range(4):
+        g = h // 2
+        ref = _sdpa64(case.q[0, h][None], case.k[0, g, :400][None], case.v[0, g, :400][None])[0]
+        for i in range(6):
+            if case.active[0, i]:
+                assert torch.allclose(o[0, h, i], ref[i], rtol=0, atol=1e-12)
+            else:
+                assert torch.equal(o[0, h, i], case.o_cache[0, h, i].double())
+
+
+# ------------------------------------------------------------------------- BLASST ----
+
+def _dense_causal(q, k, v):
+    return F.scaled_dot_product_attention(q.double(), k.double(), v.double(), is_causal=True)
+
+
+def _all_units(B, Hq, L, tq=128):
+    return [(b, h, a) for b in range(B) for h in range(Hq) for a in range(-(-L // tq))]
+
+
+def _assemble(r, units, B, Hq, L, D, tq=128):
+    out = torch.zeros(B, Hq, L, D, dtype=torch.float64)
+    for u, (b, h, a) in enumerate(units):
+        n = min(tq, L - a * tq)
+        out[b, h, a * tq:a * tq + n] = r["o"][u, :n]
+    return out
+
+
+@pytest.mark.parametrize("L", [256, 300])
+def test_blasst_lambda_zero_is_dense_causal(L):
+    case = synth.prefill_case(B=1, Hq=4, Hkv=2, L=L, D=32, lam=0.0, seed=31)
+    units = _all_units(1, 4, L)
+    r = oracle.blasst_prefill(case.q, case.k, case.v, units, 0.0)
+    assert int(r["bits"].sum()) == 0
+    o = _assemble(r, units, 1, 4, L, 32)
+    kx = case.k.repeat_interleave(2, dim=1)
+    vx = case.v.repeat_interleave(2, dim=1)
+    ref = _dense_causal(case.q, kx, vx)
+    assert torch.allclose(o, ref, rtol=0, atol=1e-12)
+    logits = case.q.double() @ kx.double().transpose(-1, -2) / math.sqrt(32)
+    logits = logits.masked_fill(torch.triu(torch.ones(L, L, dtype=torch.bool), 1), -math.inf)
+    lse_ref = torch.logsumexp(logits, -1)
+    for u, (b, h, a) in enumerate(units):
+        n = min(128, L - a * 128)
+        assert torch.allclose(r["lse"][u, :n], lse_ref[b, h, a * 128:a * 128 + n], rtol=0, atol=1e-12)
+
+
+def _sharp_case(L=512, seed=32, sink=7.0):
+    return synth.prefill_case(B=1, Hq=2, Hkv=1, L=L, D=32, lam=1e-3, sink=sink, seed=seed)
+
+
+def test_blasst_skips_equal_masked_dense_and_respect_error_bound():
+    case = _sharp_case()
+    L, lam = 512, 0.05
+    units = _all_units(1, 2, L)
+    r = oracle.blasst_prefill(case.q, case.k, case.v, units, lam)
+    nskip = int(sum(bin(int(w)).count("1") for w in r["bits"].flatten()))
+    nvis = sum((min(a * 128 + 128, L) - 1) // 64 + 1 for (_, _, a) in units)
+    assert 0 < nskip < nvis - len(units), "the sink case must skip some tiles, not all"
+    ln_lam = math.log(lam)
+    kx = case.k.repeat_interleave(2, dim=1).double()
+    vx = case.v.repeat_interleave(2, dim=1).double()
+    dense = _dense_causal(case.q, kx, vx)
+    for u, (b, h, a) in enumerate(units):
+        words = int(r["bits"][u, 0])
+        nvisit = (min(a * 128 + 128, L) - 1) // 64 + 1
+        assert words & 1 == 0  # the first visited tile is never skipped
+        for c in range(nvisit):
+            skipped = (words >> c) & 1
+            assert skipped == (r["gap"][u, c] < ln_lam)
+        # output = dense softmax restricted to the keys of the non-skipped tiles
+        rows = torch.arange(a * 128, a * 128 + 128)
+        keep = torch.zeros(128, L, dtype=torch.bool)
+        for c in range(nvisit):
+            if not (words >> c) & 1:
+                keep[:, c * 64:(c + 1) * 64] = True
+        keep &= rows[:, None] >= torch.arange(L)[None, :]
+        ref = F.scaled_dot_product_attention(case.q[b, h, a * 128:a * 128 + 128].double()[None],
+                                             kx[b, h][None], vx[b, h][None], attn_mask=keep[None])[0]
+        assert torch.allclose(r["o"][u], ref, rtol=0, atol=1e-12)
+        # error bound against dense: each dropped weight is < lambda relative to the
+        # final row max, so |o - dense| <= 2 max|v| * n_dropped * lambda
+        dropped = (~keep & (rows[:, None] >= torch.arange(L)[None, :])).sum(1).double()
+        bound = 2 * vx[b, h].abs().max() * dropped * lam
+        err = (r["o"][u] - dense[b, h, a * 128:a * 128 + 128]).abs().max(dim=1).values
+        assert (err <= bound + 1e-12).all()
+
+
+def test_blasst_constructed_negligible_tile_is_skipped():
+    # keys of tile 1 have logits far below tile 0's for every row -> tile 1 (and only it)
+    # is skipped, and the rows that see tile 1 attend to tile 0 only
+    D, L = 16, 128
+    q = torch.zeros(1, 1, L, D)
+    q[..., 0] = 4.0
+    k = torch.zeros(1, 1, L, D)
+    k[0, 0, :64, 0] = 4.0     # logits 16/4 = 4 for tile 0
+    k[0, 0, 64:, 0] = -4.0    # logits -4 for tile 1: gap -8 < ln(1e-3) = -6.9
+    v = torch.randn(1, 1, L, D)
+    r = oracle.blasst_prefill(q, k, v, [(0, 0, 0)], 1e-3, scale=0.25)
+    assert int(r["bits"][0, 0]) == 0b10
+    assert abs(float(r["gap"][0, 1]) + 8.0) < 1e-12
+    assert torch.allclose(r["o"][0, 64:], v[0, 0, :64].double().mean(0).expand(64, D), atol=1e-12)
+    r2 = oracle.blasst_prefill(q, k, v, [(0, 0, 0)], 1e-4, scale=0.25)  # ln 1e-4 = -9.2 < -8
+    assert int(r2["bits"][0, 0]) == 0
+
+
+def test_blasst_forced_bits_follow_the_given_decisions():
+    case = _sharp_case(L=256, seed=33)
+    units = _all_units(1, 2, 256)
+    free = oracle.blasst_prefill(case.q, case.k, case.v, units, 0.0)
+    forced = torch.zeros_like(free["bits"])
+    forced[:, 0] = 0b0100  # skip tile 2 wherever it is visited
+    r = oracle.blasst_prefill(case.q, case.k, case.v, units, 0.0, forced_bits=forced)
+    for u, (b, h, a) in enumerate(units):
+        nvisit = (min(a * 128 + 128, 256) - 1) // 64 + 1
+        assert int(r["bits"][u, 0]) == (0b0100 if nvisit > 2 else 0)
