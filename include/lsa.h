@@ -1,0 +1,215 @@
+/*
+ * lsa.h -- C ABI of liblsa.so: query-aware block-sparse softmax attention over a long KV
+ * cache, for NVIDIA B200 (sm_100a).
+ *
+ * The hot path: per-block key summaries -> block scoring shared by a GQA group and top-n
+ * selection with forced initial/local blocks (or, for a block of queries, the union of
+ * the tokens' selections) -> online-softmax attention over only the selected KV blocks;
+ * plus a causal prefill that skips whole KV tiles by a softmax threshold (BLASST).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * Memory.   Every tensor argument is a raw DEVICE pointer to a contiguous row-major array
+ *           in the stated layout, aligned to 16 bytes.  The caller owns all memory; the
+ *           library allocates nothing, keeps no per-call state and never frees.
+ * Streams.  All work is enqueued on `stream` (a cudaStream_t; 0 = legacy default
+ *           stream).  Calls return as soon as the work is enqueued; nothing synchronises
+ *           the host.  Calls are thread-safe.
+ * Shapes.   B = batch, Hkv = KV heads, G = query heads per KV head (query head h belongs
+ *           to KV group h / G), Hq = Hkv * G, D = head dim, blk = KV block size.
+ *           KV cache k, v: [B, Hkv, T_cap, D].  seqlens[b] = valid tokens of sequence b
+ *           (0 <= seqlens[b] <= T_cap), a device int32 array.  A sequence has
+ *           NB_b = ceil(seqlens[b] / blk) blocks; NB_cap = ceil(T_cap / blk).
+ *           Summaries summ: [B, Hkv, NB_cap, D] float32.
+ * Types.    dtype = LSA_F32 or LSA_BF16 for q, k, v and o.  lse, summaries and scores are
+ *           always float32; indices int32.
+ * Support.  D in {64, 128}; blk == 64; G <= 16.  bf16 everywhere; fp32 in summaries,
+ *           selection and decode.  Anything else returns LSA_ERR_UNSUPPORTED.
+ * Scale.    scale <= 0 means 1/sqrt(D).
+ * Errors.   Every argument is validated on the host before anything is launched; on
+ *           error nothing is enqueued and the status is returned.  LSA_ERR_CUDA means a
+ *           launch failed; lsa_last_cuda_error() returns that cudaError_t for the
+ *           calling thread.  Device-side values (seqlens, idx) are trusted: they must obey
+ *           the documented ranges.
+ */
+#ifndef LSA_H_
+#define LSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define LSA_API __attribute__((visibility("default")))
+#else
+#define LSA_API
+#endif
+
+#define LSA_OK 0
+#define LSA_ERR_INVALID_ARG 1
+#define LSA_ERR_UNSUPPORTED 2
+#define LSA_ERR_CUDA 3
+#define LSA_ERR_DEVICE_STATUS 4
+
+#define LSA_F32 0
+#define LSA_BF16 1
+
+/* Human-readable name of a status code (static storage). */
+LSA_API const char* lsa_status_string(int status);
+
+/* cudaError_t of the last failed launch on the calling thread (0 if none). */
+LSA_API int lsa_last_cuda_error(void);
+
+/* Library version: major * 10000 + minor * 100 + patch. */
+LSA_API int lsa_version(void);
+
+/*
+ * lsa_build_summaries -- mean-pooled key summary of each KV block.
+ *
+ * Defined by: Prism, "1. 문제 정의" (training-free block importance uses mean pooling of
+ * the keys of a block) and "2. 핵심 이론적 발견" (mean pooling acts as a low-pass filter).
+ *
+ *   summ[b, g, j, :] = (1 / n_j) * sum_{t = j*blk}^{min(j*blk + blk, seqlens[b]) - 1} k[b, g, t, :]
+ *
+ * with n_j the number of valid tokens of block j (a partial last block is averaged over
+ * its valid tokens only).  Accumulation is float32.
+ *
+ * k        [B, Hkv, T_cap, D] (dtype), read only.
+ * summ     [B, Hkv, NB_cap, D] float32, written for the blocks in range only.
+ * nb_begin, nb_end: block range per sequence, clipped to [0, NB_b).  nb_begin < 0 means
+ *          NB_b + nb_begin (the last -nb_begin blocks); nb_end < 0 means NB_b.  (0, -1)
+ *          rebuilds every block; (-1, -1) refreshes only the last block after a token
+ *          was appended.  Blocks outside the range are not touched.
+ */
+LSA_API int lsa_build_summaries(const void* k, int dtype, int B, int Hkv, int T_cap, int D,
+                        const int32_t* seqlens, int blk, int nb_begin, int nb_end,
+                        float* summ, cudaStream_t stream);
+
+/*
+ * lsa_select_blocks -- query-aware block scores and top-n selection, one selection per
+ * KV head shared by its G query heads.
+ *
+ * Defined by: NSA news article, "NSA 구조" (selection blocks of l' = 64 tokens; n = 16
+ * blocks selected, the initial block and 2 local blocks included) and "기존 스파스 어텐션
+ * 접근법의 한계 분석" / "기술 구현의 실제적 도전과 해결" (query-aware chunk scoring;
+ * GQA-compatible selection decides memory-access efficiency).
+ *
+ *   score[b, g, j] = scale * sum_{h in group g} q[b, h, :] . summ[b, g, j, :]    (j < NB_b)
+ *   F = {0 .. n_sink-1} U {NB_b - n_local .. NB_b - 1}  (clipped, deduplicated)
+ *   selected = F U (the topk - |F| highest-scoring blocks outside F; ties -> lower j)
+ *   if NB_b <= topk, every block is selected.
+ *
+ * q          [B, Hq, D] (dtype).  summ [B, Hkv, NB_cap, D] float32.
+ * idx        [B, Hkv, topk] int32 out: selected block indices ascending, padded with -1.
+ * nsel       [B, Hkv] int32 out: number of selected blocks (min(topk, NB_b)).
+ * scores_out [B, Hkv, NB_cap] float32 out, or NULL: the block scores, written only for
+ *            sequences with NB_b > topk and only for j < NB_b (other entries untouched).
+ * Requires 1 <= topk <= 64, n_sink >= 0, n_local >= 0, n_sink + n_local <= topk.
+ */
+LSA_API int lsa_select_blocks(const void* q, int dtype, const float* summ, int B, int Hkv, int G,
+                      int D, int NB_cap, const int32_t* seqlens, int blk, int topk,
+                      int n_sink, int n_local, float scale, int32_t* idx, int32_t* nsel,
+                      float* scores_out, cudaStream_t stream);
+
+/*
+ * lsa_sparse_attn_decode -- softmax attention of one query token per head over only the
+ * tokens of the selected KV blocks (original positions kept), split over the selected
+ * blocks with a log-sum-exp merge.
+ *
+ * Defined by: NSA news article, "NSA 구조" and "처리 속도" (decoding touches only the
+ * selected blocks' tokens); FASA, "2. 방법론", Focused Attention Computation (exact
+ * full-dimension attention over the selected tokens, positions preserved).
+ *
+ *   tokens(b, g) = { t : floor(t / blk) in selected(b, g), t < seqlens[b] }
+ *   o[b, h, :]   = sum_t softmax_t(scale * q[b,h,:] . k[b,g,t,:]) v[b,g,t,:]
+ *   lse[b, h]    = log sum_t exp(scale * q[b,h,:] . k[b,g,t,:])        (g = h / G)
+ * An empty token set gives o = 0 and lse = -inf.
+ *
+ * Two modes:
+ *   given selection (idx != NULL): idx [B, Hkv, topk] and nsel [B, Hkv] as written by
+ *       lsa_select_blocks (entries in [0, NB_b), the first nsel valid; -1 ignored).
+ *   fused selection (idx == NULL): selection as in lsa_select_blocks is computed inside
+ *       the same launch from summ (required) with n_sink / n_local; the selected indices
+ *       are written to idx_out [B, Hkv, topk] (ascending, -1 padded) when it is non-NULL.
+ * q [B, Hq, D]; k, v [B, Hkv, T_cap, D]; o [B, Hq, D] (dtype); lse [B, Hq] float32 or NULL.
+ * K/V rows at or beyond seqlens[b] are never used (they may hold any bits, NaN included).
+ */
+LSA_API int lsa_sparse_attn_decode(const void* q, const void* k, const void* v, int dtype, int B,
+                           int Hkv, int G, int D, int T_cap, const int32_t* seqlens,
+                           int blk, const int32_t* idx, const int32_t* nsel, int topk,
+                           float scale, const float* summ, int n_sink, int n_local,
+                           int32_t* idx_out, void* o, float* lse, cudaStream_t stream);
+
+/*
+ * lsa_sparse_attn_blockquery -- one denoising step of a block of Tq query tokens
+ * (block-wise diffusion LM) against a cached prefix of T_prefix tokens.
+ *
+ * Defined by: LoSA, "1. 문제 정의" (the union of the KV positions selected by the
+ * queries of a block sets memory traffic and latency) and "2. 방법론" (only active tokens
+ * select and attend, sparsely; stable tokens reuse the previous step's prefix-attention
+ * output and statistics; the union is taken over active tokens only).
+ *
+ * For every active token i (active[b, i] != 0) and KV group g:
+ *   s_i(j)    = scale * sum_{h in g} q[b, h, i, :] . summ[b, g, j, :]   over prefix blocks
+ *               j < NBp = ceil(T_prefix / blk)
+ *   S(i, g)   = top-`topk_per_query` of s_i with forced blocks as in lsa_select_blocks
+ *   U(b, g)   = union over active i of S(i, g), deduplicated, ascending
+ *   every active row (b, h in g, i) attends over all tokens t < T_prefix of the blocks in
+ *   U(b, g) (no mask inside the prefix): o = softmax-weighted v, lse = log-sum-exp.
+ * Stable rows (active == 0): o[b,h,i,:] = o_cache[b,h,i,:] and lse = lse_cache, bit-exact
+ * (o_cache / lse_cache may alias o / lse, in which case stable rows are left as they are).
+ *
+ * q [B, Hq, Tq, D] bf16; k, v [B, Hkv, T_cap, D] bf16 (T_prefix <= T_cap);
+ * summ [B, Hkv, NB_cap, D] float32; active [B, Tq] uint8;
+ * o_cache [B, Hq, Tq, D] bf16; lse_cache [B, Hq, Tq] float32; o, lse: same shapes, out.
+ * union_idx [B, Hkv, NBp] int32 out or NULL (ascending, -1 padded);
+ * union_cnt [B, Hkv] int32 out or NULL.
+ * Requires 1 <= Tq <= 64, 1 <= topk_per_query <= 64.
+ */
+LSA_API int lsa_sparse_attn_blockquery(const void* q, const void* k, const void* v, int dtype,
+                               int B, int Hkv, int G, int D, int Tq, int T_prefix,
+                               int T_cap, const float* summ, int blk, int topk_per_query,
+                               int n_sink, int n_local, float scale, const uint8_t* active,
+                               const void* o_cache, const float* lse_cache, void* o,
+                               float* lse, int32_t* union_idx, int32_t* union_cnt,
+                               cudaStream_t stream);
+
+/*
+ * lsa_blasst_prefill -- causal softmax attention that skips whole KV tiles whose
+ * softmax weight is negligible (BLASST).
+ *
+ * Defined by: BLASST, "2. 방법론" -- "핵심 아이디어: 온라인 Softmax 통계 활용" (compare each
+ * block's local maximum with the running maximum of the blockwise online softmax; skip
+ * the exponentials, the V-block load and the P.V product of a block that trails by more
+ * than the threshold) and "알고리즘 및 커널 설계" (the test block_max - running_max < ln(lambda)).
+ *
+ * For query head h (KV head h / (Hq / Hkv)) and query tile a (rows [128a, 128a + 128)),
+ * KV tiles c = 0, 1, ... of 64 keys are visited in ascending order up to the diagonal:
+ *   S = scale * Q K_c^T with the causal mask; r_i = max_t S_it; m_i = running row max
+ *   skip tile c  iff  max over the tile's rows of (r_i - m_i) < ln(lambda)
+ *   otherwise the usual online-softmax update of (m, l, acc) with tile c.
+ * lambda = 0 never skips (plain causal attention).  The first tile is never skipped.
+ * Outputs o = acc / l, lse = m + ln l.
+ *
+ * q [B, Hq, L, D] bf16; k, v [B, Hkv, L, D] bf16; o [B, Hq, L, D] bf16 out;
+ * lse [B, Hq, L] float32 out or NULL;
+ * skip_bits [B, Hq, ceil(L/128), ceil(ceil(L/64)/32)] uint32 out or NULL: bit c of a
+ *     (b, h, a) row is set iff tile c was skipped;
+ * skipped_tiles: one uint64 counter or NULL, incremented by the number of skipped tiles
+ *     (the caller zeroes it).
+ * Requires D == 128, Hq % Hkv == 0, L >= 1.
+ */
+LSA_API int lsa_blasst_prefill(const void* q, const void* k, const void* v, int dtype, int B, int Hq,
+                       int Hkv, int L, int D, float scale, float lambda, void* o, float* lse,
+                       uint32_t* skip_bits, unsigned long long* skipped_tiles,
+                       cudaStream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LSA_H_ */

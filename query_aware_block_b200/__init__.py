@@ -1,0 +1,152 @@
+"""Thin Python binding of liblsa.so (query-aware block-sparse attention for B200).
+
+The functions carry the names of the C ABI in include/lsa.h and only marshal arguments:
+shapes are read from the torch tensors, pointers and the current CUDA stream are passed
+through ctypes, and a non-zero status raises LsaError.  Every step of the computation runs
+in the library's CUDA kernels; there is no fallback of any kind.  If liblsa.so has not been
+built (``python -m query_aware_block_b200._build``), importing this package raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "liblsa.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"{LIB_PATH} is missing: build it with `python -m query_aware_block_b200._build`")
+
+_lib = ctypes.CDLL(LIB_PATH)
+
+LSA_OK, LSA_ERR_INVALID_ARG, LSA_ERR_UNSUPPORTED, LSA_ERR_CUDA, LSA_ERR_DEVICE_STATUS = 0, 1, 2, 3, 4
+LSA_F32, LSA_BF16 = 0, 1
+BLK = 64
+
+EXPORTED = ("lsa_status_string", "lsa_last_cuda_error", "lsa_version", "lsa_build_summaries",
+            "lsa_select_blocks", "lsa_sparse_attn_decode", "lsa_sparse_attn_blockquery",
+            "lsa_blasst_prefill")
+
+_vp, _i, _f = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+_lib.lsa_status_string.restype = ctypes.c_char_p
+_lib.lsa_status_string.argtypes = [_i]
+_lib.lsa_last_cuda_error.restype = _i
+_lib.lsa_version.restype = _i
+_lib.lsa_build_summaries.argtypes = [_vp, _i, _i, _i, _i, _i, _vp, _i, _i, _i, _vp, _vp]
+_lib.lsa_select_blocks.argtypes = [_vp, _i, _vp, _i, _i, _i, _i, _i, _vp, _i, _i, _i, _i, _f,
+                                   _vp, _vp, _vp, _vp]
+_lib.lsa_sparse_attn_decode.argtypes = [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp, _i, _vp, _vp,
+                                        _i, _f, _vp, _i, _i, _vp, _vp, _vp, _vp]
+_lib.lsa_sparse_attn_blockquery.argtypes = [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _vp,
+                                            _i, _i, _i, _i, _f, _vp, _vp, _vp, _vp, _vp, _vp,
+                                            _vp, _vp]
+_lib.lsa_blasst_prefill.argtypes = [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _f, _vp, _vp, _vp,
+                                    _vp, _vp]
+for _n in EXPORTED[3:]:
+    getattr(_lib, _n).restype = _i
+
+
+class LsaError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        msg = _lib.lsa_status_string(status).decode()
+        if status == LSA_ERR_CUDA:
+            msg += f" (cudaError {_lib.lsa_last_cuda_error()})"
+        super().__init__(f"{where}: {msg}")
+        self.status = status
+
+
+def library():
+    """The loaded ctypes library (for tests of the raw ABI)."""
+    return _lib
+
+
+def lsa_version() -> int:
+    return int(_lib.lsa_version())
+
+
+def _ptr(t):
+    return None if t is None else t.data_ptr()
+
+
+def _dtype(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return LSA_BF16
+    if t.dtype == torch.float32:
+        return LSA_F32
+    return -1  # rejected by the library as unsupported
+
+
+def _stream(stream):
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    return getattr(stream, "cuda_stream", stream)
+
+
+def _check(status: int, where: str):
+    if status != LSA_OK:
+        raise LsaError(status, where)
+
+
+def lsa_build_summaries(k, seqlens, summ, nb_begin=0, nb_end=-1, blk=BLK, stream=None):
+    """k [B,Hkv,T_cap,D] -> summ [B,Hkv,ceil(T_cap/blk),D] float32 (in place)."""
+    B, Hkv, T_cap, D = k.shape
+    _check(_lib.lsa_build_summaries(_ptr(k), _dtype(k), B, Hkv, T_cap, D, _ptr(seqlens), blk,
+                                    nb_begin, nb_end, _ptr(summ), _stream(stream)),
+           "lsa_build_summaries")
+    return summ
+
+
+def lsa_select_blocks(q, summ, seqlens, topk, n_sink, n_local, idx, nsel, scale=0.0,
+                      scores_out=None, blk=BLK, stream=None):
+    """q [B,Hq,D], summ [B,Hkv,NB_cap,D] -> idx [B,Hkv,topk], nsel [B,Hkv] (in place)."""
+    B, Hq, D = q.shape
+    _, Hkv, NB_cap, _ = summ.shape
+    _check(_lib.lsa_select_blocks(_ptr(q), _dtype(q), _ptr(summ), B, Hkv, Hq // Hkv, D, NB_cap,
+                                  _ptr(seqlens), blk, topk, n_sink, n_local, float(scale),
+                                  _ptr(idx), _ptr(nsel), _ptr(scores_out), _stream(stream)),
+           "lsa_select_blocks")
+    return idx, nsel
+
+
+def lsa_sparse_attn_decode(q, k, v, seqlens, o, topk, idx=None, nsel=None, summ=None,
+                           n_sink=0, n_local=0, idx_out=None, lse=None, scale=0.0, blk=BLK,
+                           stream=None):
+    """Sparse decode attention.  Given selection: idx, nsel.  Fused selection: summ."""
+    B, Hq, D = q.shape
+    _, Hkv, T_cap, _ = k.shape
+    _check(_lib.lsa_sparse_attn_decode(_ptr(q), _ptr(k), _ptr(v), _dtype(q), B, Hkv, Hq // Hkv,
+                                       D, T_cap, _ptr(seqlens), blk, _ptr(idx), _ptr(nsel),
+                                       topk, float(scale), _ptr(summ), n_sink, n_local,
+                                       _ptr(idx_out), _ptr(o), _ptr(lse), _stream(stream)),
+           "lsa_sparse_attn_decode")
+    return o
+
+
+def lsa_sparse_attn_blockquery(q, k, v, summ, T_prefix, topk_per_query, active, o_cache,
+                               lse_cache, o, lse, n_sink=0, n_local=0, union_idx=None,
+                               union_cnt=None, scale=0.0, blk=BLK, stream=None):
+    """Block-query step: q [B,Hq,Tq,D] against the prefix of k, v [B,Hkv,T_cap,D]."""
+    B, Hq, Tq, D = q.shape
+    _, Hkv, T_cap, _ = k.shape
+    _check(_lib.lsa_sparse_attn_blockquery(_ptr(q), _ptr(k), _ptr(v), _dtype(q), B, Hkv,
+                                           Hq // Hkv, D, Tq, T_prefix, T_cap, _ptr(summ), blk,
+                                           topk_per_query, n_sink, n_local, float(scale),
+                                           _ptr(active), _ptr(o_cache), _ptr(lse_cache),
+                                           _ptr(o), _ptr(lse), _ptr(union_idx), _ptr(union_cnt),
+                                           _stream(stream)),
+           "lsa_sparse_attn_blockquery")
+    return o, lse
+
+
+def lsa_blasst_prefill(q, k, v, o, lam, lse=None, skip_bits=None, skipped_tiles=None,
+                       scale=0.0, stream=None):
+    """BLASST causal prefill: q [B,Hq,L,D], k, v [B,Hkv,L,D] -> o (in place)."""
+    B, Hq, L, D = q.shape
+    Hkv = k.shape[1]
+    _check(_lib.lsa_blasst_prefill(_ptr(q), _ptr(k), _ptr(v), _dtype(q), B, Hq, Hkv, L, D,
+                                   float(scale), float(lam), _ptr(o), _ptr(lse), _ptr(skip_bits),
+                                   _ptr(skipped_tiles), _stream(stream)),
+           "lsa_blasst_prefill")
+    return o

@@ -1,0 +1,158 @@
+// lsa_api.cu -- the exported C ABI (include/lsa.h): host-side validation, then launch.
+// Nothing is launched when an argument is invalid; the library allocates nothing.
+#include <math.h>
+#include <stdint.h>
+
+#include "../../include/lsa.h"
+#include "lsa_internal.h"
+
+namespace {
+
+thread_local int g_last_cuda_error = 0;
+
+int cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return LSA_OK;
+  g_last_cuda_error = (int)e;
+  return LSA_ERR_CUDA;
+}
+
+bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+
+int ceil_div(int a, int b) { return (a + b - 1) / b; }
+
+float resolve_scale(float scale, int D) { return scale > 0.f ? scale : 1.0f / sqrtf((float)D); }
+
+// Shape checks shared by the attention entry points.
+int check_common(int dtype, int B, int Hkv, int G, int D, int blk) {
+  if (B < 0 || Hkv < 0 || G < 1) return LSA_ERR_INVALID_ARG;
+  if (dtype != LSA_F32 && dtype != LSA_BF16) return LSA_ERR_UNSUPPORTED;
+  if (D != 64 && D != 128) return LSA_ERR_UNSUPPORTED;
+  if (blk != 64) return LSA_ERR_UNSUPPORTED;
+  if (G > 16) return LSA_ERR_UNSUPPORTED;
+  return LSA_OK;
+}
+
+constexpr int kMaxTcap = 1 << 21;  // 2M tokens: 32768 blocks per sequence
+
+}  // namespace
+
+extern "C" {
+
+const char* lsa_status_string(int status) {
+  switch (status) {
+    case LSA_OK: return "LSA_OK";
+    case LSA_ERR_INVALID_ARG: return "LSA_ERR_INVALID_ARG: an argument is out of range or a required pointer is NULL/misaligned";
+    case LSA_ERR_UNSUPPORTED: return "LSA_ERR_UNSUPPORTED: dtype, head dim, block size or size not supported";
+    case LSA_ERR_CUDA: return "LSA_ERR_CUDA: a kernel launch failed (see lsa_last_cuda_error)";
+    case LSA_ERR_DEVICE_STATUS: return "LSA_ERR_DEVICE_STATUS: a kernel reported an error status";
+    default: return "unknown lsa status";
+  }
+}
+
+int lsa_last_cuda_error(void) { return g_last_cuda_error; }
+
+int lsa_version(void) { return 100; }
+
+int lsa_build_summaries(const void* k, int dtype, int B, int Hkv, int T_cap, int D,
+                        const int32_t* seqlens, int blk, int nb_begin, int nb_end,
+                        float* summ, cudaStream_t stream) {
+  int st = check_common(dtype, B, Hkv, 1, D, blk);
+  if (st != LSA_OK) return st;
+  if (T_cap < 0 || T_cap > kMaxTcap) return T_cap < 0 ? LSA_ERR_INVALID_ARG : LSA_ERR_UNSUPPORTED;
+  if (B == 0 || Hkv == 0 || T_cap == 0) return LSA_OK;
+  if (!k || !seqlens || !summ) return LSA_ERR_INVALID_ARG;
+  if (!aligned16(k) || !aligned16(summ)) return LSA_ERR_INVALID_ARG;
+  const int NB_cap = ceil_div(T_cap, blk);
+  // the widest block range any sequence can have
+  int range_max;
+  if (nb_begin >= 0) {
+    const int hi = nb_end >= 0 ? (nb_end < NB_cap ? nb_end : NB_cap) : NB_cap;
+    range_max = hi - nb_begin;
+  } else {
+    range_max = -nb_begin < NB_cap ? -nb_begin : NB_cap;
+  }
+  if (range_max <= 0) return LSA_OK;
+  return cuda_status(lsa::launch_build_summaries(k, dtype, B, Hkv, T_cap, D, seqlens, nb_begin,
+                                                 nb_end, range_max, summ, stream));
+}
+
+int lsa_select_blocks(const void* q, int dtype, const float* summ, int B, int Hkv, int G,
+                      int D, int NB_cap, const int32_t* seqlens, int blk, int topk,
+                      int n_sink, int n_local, float scale, int32_t* idx, int32_t* nsel,
+                      float* scores_out, cudaStream_t stream) {
+  int st = check_common(dtype, B, Hkv, G, D, blk);
+  if (st != LSA_OK) return st;
+  if (topk < 1 || topk > 64 || n_sink < 0 || n_local < 0 || n_sink + n_local > topk)
+    return LSA_ERR_INVALID_ARG;
+  if (NB_cap < 0) return LSA_ERR_INVALID_ARG;
+  if (NB_cap > kMaxTcap / 64) return LSA_ERR_UNSUPPORTED;
+  if (B == 0 || Hkv == 0) return LSA_OK;
+  if (!q || !summ || !seqlens || !idx || !nsel) return LSA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(summ)) return LSA_ERR_INVALID_ARG;
+  lsa::DecodeArgs a = {};
+  a.q = q; a.dtype = dtype; a.summ = summ;
+  a.B = B; a.Hkv = Hkv; a.G = G; a.D = D; a.T_cap = NB_cap * blk; a.NB_cap = NB_cap;
+  a.seqlens = seqlens; a.topk = topk; a.n_sink = n_sink; a.n_local = n_local;
+  a.scale = resolve_scale(scale, D);
+  a.idx_out = idx; a.nsel_out = nsel; a.scores_out = scores_out;
+  a.mode = lsa::MODE_SELECT;
+  return cuda_status(lsa::launch_decode(a, stream));
+}
+
+int lsa_sparse_attn_decode(const void* q, const void* k, const void* v, int dtype, int B,
+                           int Hkv, int G, int D, int T_cap, const int32_t* seqlens,
+                           int blk, const int32_t* idx, const int32_t* nsel, int topk,
+                           float scale, const float* summ, int n_sink, int n_local,
+                           int32_t* idx_out, void* o, float* lse, cudaStream_t stream) {
+  int st = check_common(dtype, B, Hkv, G, D, blk);
+  if (st != LSA_OK) return st;
+  if (topk < 1 || topk > 64) return LSA_ERR_INVALID_ARG;
+  if (T_cap < 0) return LSA_ERR_INVALID_ARG;
+  if (T_cap > kMaxTcap) return LSA_ERR_UNSUPPORTED;
+  if (B == 0 || Hkv == 0) return LSA_OK;
+  if (!q || !k || !v || !seqlens || !o) return LSA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return LSA_ERR_INVALID_ARG;
+  const bool fused = idx == nullptr;
+  if (fused) {
+    if (!summ || !aligned16(summ)) return LSA_ERR_INVALID_ARG;
+    if (n_sink < 0 || n_local < 0 || n_sink + n_local > topk) return LSA_ERR_INVALID_ARG;
+  } else if (!nsel) {
+    return LSA_ERR_INVALID_ARG;
+  }
+  lsa::DecodeArgs a = {};
+  a.q = q; a.k = k; a.v = v; a.dtype = dtype;
+  a.B = B; a.Hkv = Hkv; a.G = G; a.D = D; a.T_cap = T_cap; a.NB_cap = ceil_div(T_cap, blk);
+  a.seqlens = seqlens; a.summ = summ; a.idx_in = idx; a.nsel_in = nsel;
+  a.topk = topk; a.n_sink = n_sink; a.n_local = n_local;
+  a.scale = resolve_scale(scale, D);
+  a.idx_out = fused ? idx_out : nullptr;
+  a.o = o; a.lse = lse;
+  a.mode = fused ? lsa::MODE_FUSED : lsa::MODE_ATTEND;
+  return cuda_status(lsa::launch_decode(a, stream));
+}
+
+int lsa_sparse_attn_blockquery(const void* q, const void* k, const void* v, int dtype,
+                               int B, int Hkv, int G, int D, int Tq, int T_prefix,
+                               int T_cap, const float* summ, int blk, int topk_per_query,
+                               int n_sink, int n_local, float scale, const uint8_t* active,
+                               const void* o_cache, const float* lse_cache, void* o,
+                               float* lse, int32_t* union_idx, int32_t* union_cnt,
+                               cudaStream_t stream) {
+  (void)q; (void)k; (void)v; (void)dtype; (void)B; (void)Hkv; (void)G; (void)D; (void)Tq;
+  (void)T_prefix; (void)T_cap; (void)summ; (void)blk; (void)topk_per_query; (void)n_sink;
+  (void)n_local; (void)scale; (void)active; (void)o_cache; (void)lse_cache; (void)o;
+  (void)lse; (void)union_idx; (void)union_cnt; (void)stream;
+  return LSA_ERR_UNSUPPORTED;
+}
+
+int lsa_blasst_prefill(const void* q, const void* k, const void* v, int dtype, int B, int Hq,
+                       int Hkv, int L, int D, float scale, float lambda, void* o, float* lse,
+                       uint32_t* skip_bits, unsigned long long* skipped_tiles,
+                       cudaStream_t stream) {
+  (void)q; (void)k; (void)v; (void)dtype; (void)B; (void)Hq; (void)Hkv; (void)L; (void)D;
+  (void)scale; (void)lambda; (void)o; (void)lse; (void)skip_bits; (void)skipped_tiles;
+  (void)stream;
+  return LSA_ERR_UNSUPPORTED;
+}
+
+}  // extern "C"

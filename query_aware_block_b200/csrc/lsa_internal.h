@@ -1,0 +1,41 @@
+// lsa_internal.h -- launchers behind the C ABI (host side, not exported).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace lsa {
+
+enum { DT_F32 = 0, DT_BF16 = 1 };
+
+cudaError_t launch_build_summaries(const void* k, int dtype, int B, int Hkv, int T_cap, int D,
+                                   const int32_t* seqlens, int nb_begin, int nb_end,
+                                   int range_max, float* summ, cudaStream_t stream);
+
+// The decode family: one thread-block cluster per (sequence, KV head).
+enum DecodeMode { MODE_SELECT = 0, MODE_ATTEND = 1, MODE_FUSED = 2 };
+
+struct DecodeArgs {
+  const void* q;
+  const void* k;
+  const void* v;
+  int dtype;
+  int B, Hkv, G, D, T_cap;
+  const int32_t* seqlens;
+  const float* summ;
+  int NB_cap;
+  const int32_t* idx_in;   // MODE_ATTEND
+  const int32_t* nsel_in;  // MODE_ATTEND
+  int topk, n_sink, n_local;
+  float scale;
+  int32_t* idx_out;        // MODE_SELECT / MODE_FUSED (may be NULL in fused mode)
+  int32_t* nsel_out;       // MODE_SELECT
+  float* scores_out;       // MODE_SELECT, optional
+  void* o;                 // MODE_ATTEND / MODE_FUSED
+  float* lse;              // optional
+  int mode;
+};
+
+cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream);
+
+}  // namespace lsa

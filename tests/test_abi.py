@@ -1,0 +1,89 @@
+"""The C ABI boundary on the CPU: liblsa.so loads, exports every entry point that
+include/lsa.h declares, and rejects bad arguments on the host before any launch (so these
+calls are safe without a GPU: none of them reaches a CUDA call)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "lsa.h")
+
+
+def _declared():
+    text = open(HEADER).read()
+    return re.findall(r"LSA_API\s+[\w\s\*]+?\b(lsa_\w+)\s*\(", text)
+
+
+def test_header_declares_the_five_entry_points():
+    names = _declared()
+    for n in ("lsa_build_summaries", "lsa_select_blocks", "lsa_sparse_attn_decode",
+              "lsa_sparse_attn_blockquery", "lsa_blasst_prefill"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol():
+    import query_aware_block_b200 as lsa
+    lib = ctypes.CDLL(lsa.LIB_PATH)
+    for n in _declared():
+        assert hasattr(lib, n), n
+    assert set(lsa.EXPORTED) == set(_declared())
+
+
+def test_status_strings_and_version():
+    import query_aware_block_b200 as lsa
+    lib = lsa.library()
+    assert lib.lsa_status_string(0) == b"LSA_OK"
+    for s in (1, 2, 3, 4):
+        assert lib.lsa_status_string(s).startswith(b"LSA_ERR")
+    assert lib.lsa_status_string(99) == b"unknown lsa status"
+    assert lsa.lsa_version() >= 100
+
+
+NULL = None
+
+
+def test_build_summaries_validation():
+    import query_aware_block_b200 as lsa
+    f = lsa.library().lsa_build_summaries
+    good = ctypes.c_void_p(4096)
+    # dtype, head dim, block size
+    assert f(good, 7, 1, 1, 64, 128, good, 64, 0, -1, good, NULL) == lsa.LSA_ERR_UNSUPPORTED
+    assert f(good, 1, 1, 1, 64, 96, good, 64, 0, -1, good, NULL) == lsa.LSA_ERR_UNSUPPORTED
+    assert f(good, 1, 1, 1, 64, 128, good, 32, 0, -1, good, NULL) == lsa.LSA_ERR_UNSUPPORTED
+    # null / misaligned pointers
+    assert f(NULL, 1, 1, 1, 64, 128, good, 64, 0, -1, good, NULL) == lsa.LSA_ERR_INVALID_ARG
+    assert f(ctypes.c_void_p(4098), 1, 1, 1, 64, 128, good, 64, 0, -1, good, NULL) == lsa.LSA_ERR_INVALID_ARG
+    assert f(good, 1, -1, 1, 64, 128, good, 64, 0, -1, good, NULL) == lsa.LSA_ERR_INVALID_ARG
+    # empty problems are a successful no-op, nothing launched
+    assert f(NULL, 1, 0, 1, 64, 128, NULL, 64, 0, -1, NULL, NULL) == lsa.LSA_OK
+    assert f(good, 1, 1, 1, 64, 128, good, 64, 5, 3, good, NULL) == lsa.LSA_OK  # empty range
+
+
+def test_select_and_decode_validation():
+    import query_aware_block_b200 as lsa
+    lib = lsa.library()
+    g = ctypes.c_void_p(4096)
+    sel = lib.lsa_select_blocks
+    # topk range, forced count larger than topk, G > 16
+    assert sel(g, 1, g, 1, 8, 8, 128, 1024, g, 64, 0, 1, 2, 0.0, g, g, NULL, NULL) == lsa.LSA_ERR_INVALID_ARG
+    assert sel(g, 1, g, 1, 8, 8, 128, 1024, g, 64, 65, 1, 2, 0.0, g, g, NULL, NULL) == lsa.LSA_ERR_INVALID_ARG
+    assert sel(g, 1, g, 1, 8, 8, 128, 1024, g, 64, 2, 1, 2, 0.0, g, g, NULL, NULL) == lsa.LSA_ERR_INVALID_ARG
+    assert sel(g, 1, g, 1, 8, 17, 128, 1024, g, 64, 16, 1, 2, 0.0, g, g, NULL, NULL) == lsa.LSA_ERR_UNSUPPORTED
+    assert sel(g, 1, g, 1, 8, 8, 128, 1024, g, 64, 16, 1, 2, 0.0, NULL, g, NULL, NULL) == lsa.LSA_ERR_INVALID_ARG
+    dec = lib.lsa_sparse_attn_decode
+    # fused mode (idx NULL) needs summaries; given mode needs nsel
+    assert dec(g, g, g, 1, 1, 8, 8, 128, 65536, g, 64, NULL, NULL, 16, 0.0, NULL, 1, 2, NULL, g, NULL, NULL) == lsa.LSA_ERR_INVALID_ARG
+    assert dec(g, g, g, 1, 1, 8, 8, 128, 65536, g, 64, g, NULL, 16, 0.0, NULL, 1, 2, NULL, g, NULL, NULL) == lsa.LSA_ERR_INVALID_ARG
+    assert dec(g, g, g, 1, 1, 8, 8, 128, 1 << 22, g, 64, g, g, 16, 0.0, NULL, 1, 2, NULL, g, NULL, NULL) == lsa.LSA_ERR_UNSUPPORTED
+    assert dec(g, g, NULL, 1, 1, 8, 8, 128, 65536, g, 64, g, g, 16, 0.0, NULL, 1, 2, NULL, g, NULL, NULL) == lsa.LSA_ERR_INVALID_ARG
+
+
+def test_binding_raises_lsa_error_on_bad_arguments():
+    import torch
+    import query_aware_block_b200 as lsa
+    k = torch.zeros(1, 1, 64, 96)  # D = 96 unsupported; rejected before any launch
+    with pytest.raises(lsa.LsaError) as e:
+        lsa.lsa_build_summaries(k, torch.zeros(1, dtype=torch.int32), torch.zeros(1, 1, 1, 96), stream=0)
+    assert e.value.status == lsa.LSA_ERR_UNSUPPORTED
