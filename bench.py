@@ -1,0 +1,527 @@
+#!/usr/bin/env python
+"""Benchmark of the query-aware block-sparse attention hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload gqa_decode_64k|batched_decode|tiny_decode]
+
+Default workload: 64K-context GQA decode, bf16 (1 sequence, 8 KV heads x 8 query heads,
+head dim 128, 65,536 cached tokens = 1,024 blocks of 64, top-16 blocks per KV head with
+block 0 and the last 2 blocks forced, 16 planted needle blocks per group).
+
+One step = one decode step of the whole hot path: refresh the summary of the block that
+holds the newest token (lsa_build_summaries on the last block) and one fused launch of
+block scoring + top-k selection + sparse attention over the selected blocks
+(lsa_sparse_attn_decode with idx == NULL).  Inputs are resident in HBM; R distinct input
+copies are rotated so that R x (bytes a step touches) exceeds 4x the L2 size, i.e. every
+step reads cold data.  The K timed steps are replayed from a CUDA graph of one rotation
+cycle, bracketed by barrier + synchronize, timed with CUDA events (max over ranks).
+
+Reported: value = tokens/s over all ranks (1 token per sequence per step), the effective
+HBM GB/s of the algorithmic bytes, the roofline of the dominant kernel (fused decode) with
+its own CUDA-event launch duration, e2e through the C ABI with pinned host buffers (q and
+the new token's k, v copied in; o, lse, idx copied out every step), SM clocks sampled
+during the timed region, and the fp64 CPU oracle on a bounded sample as the CPU baseline.
+Multi-GPU (torchrun): every rank decodes its own independent sequence (the path shards by
+sequence with no collective): weak scaling.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import re
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+METRIC = "64K-ctx sparse decode tokens/s and effective KV GB/s (% of B200 HBM roofline)"
+UNIT = "tokens/s"
+KERNEL_SOURCES = ["query_aware_block_b200/csrc/decode.cu", "query_aware_block_b200/csrc/lsa_common.cuh"]
+PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "decode_fused_gqa_decode_64k.md")
+
+WORKLOADS = {
+    "gqa_decode_64k": dict(B=1, Hkv=8, G=8, D=128, T_cap=65536, T=65536, topk=16, n_sink=1,
+                           n_local=2, n_needles=16, dtype="bf16"),
+    "batched_decode": dict(B=16, Hkv=8, G=4, D=128, T_cap=32768, T=None, topk=16, n_sink=1,
+                           n_local=2, n_needles=8, dtype="bf16"),
+    "tiny_decode": dict(B=1, Hkv=1, G=4, D=64, T_cap=2048, T=2048, topk=8, n_sink=1,
+                        n_local=2, n_needles=0, dtype="f32"),
+}
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200000)
+    ap.add_argument("--warmup", type=int, default=600)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="gqa_decode_64k")
+    ap.add_argument("--rotate", type=int, default=0, help="input copies (0 = auto, > 4x L2)")
+    ap.add_argument("--e2e-steps", type=int, default=2000)
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile-small", action="store_true",
+                    help="a few launches on 2 input copies, for ncu captures")
+    return ap.parse_args()
+
+
+# ---------------------------------------------------------------------------- helpers --
+
+def _dtype(name):
+    return torch.bfloat16 if name == "bf16" else torch.float32
+
+
+def make_case(wl, seed, device):
+    import synth
+    w = WORKLOADS[wl]
+    if wl == "batched_decode":
+        return synth.batched_decode(seed=seed, device=device)
+    return synth.decode_case(B=w["B"], Hkv=w["Hkv"], G=w["G"], D=w["D"], T_cap=w["T_cap"],
+                             seqlens=w["T"], dtype=_dtype(w["dtype"]), topk=w["topk"],
+                             n_sink=w["n_sink"], n_local=w["n_local"], n_needles=w["n_needles"],
+                             theta=1e4, seed=seed, device=device)
+
+
+def algorithmic_bytes(case):
+    """Bytes the method must move in one step (per kernel), from the definitions:
+    fused decode: summaries of the candidate blocks + K and V of the selected blocks' valid
+    tokens + q + o + lse + idx; summary refresh: the last block's valid keys + its summary."""
+    B, Hkv, G, D, T_cap = case.shape
+    esz = case.k.element_size()
+    dec = 0
+    ref = 0
+    for b in range(B):
+        T = int(case.seqlens[b])
+        NB = -(-T // 64)
+        if NB > case.topk:
+            nf = case.n_sink + case.n_local
+            dec += Hkv * (NB - nf) * D * 4                      # candidate summaries
+            nsel = case.topk
+            # selected tokens: all full blocks except possibly the (forced) partial last one
+            toks = (nsel - 1) * 64 + (T - (NB - 1) * 64) if case.n_local > 0 else nsel * 64
+        else:
+            toks = T
+        dec += Hkv * toks * D * esz * 2                            # K and V
+        last = T - (NB - 1) * 64 if NB else 0
+        ref += Hkv * (last * D * esz + D * 4)
+    Hq = Hkv * G
+    dec += B * Hq * D * esz * 2 + B * Hq * 4 + B * Hkv * case.topk * 4  # q, o, lse, idx
+    return dec, ref
+
+
+class ClockSampler:
+    """nvidia-smi samples of the SM clock and throttle reasons during the timed region."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *a):
+        time.sleep(0.2)
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": [], "samples": 0}
+        sm.sort()
+        return {"sm_mhz": sm[len(sm) // 2], "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def source_hash():
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic():
+    """DRAM bytes per launch of the fused decode from the committed ncu summary, if it was
+    taken on the current kernel source; else None."""
+    try:
+        text = open(PROFILE_SUMMARY).read()
+    except OSError:
+        return None
+    m_hash = re.search(r"kernel source hash:\s*([0-9a-f]+)", text)
+    m_tr = re.search(r"dram bytes per launch \(read \+ write\):\s*([0-9]+)", text)
+    if not (m_hash and m_tr) or m_hash.group(1) != source_hash():
+        return None
+    return int(m_tr.group(1))
+
+
+def measured_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return 6650.0, "fallback"
+
+
+# ----------------------------------------------------------------------- our arm ----
+
+def run_ours(args, rank, world, local_rank):
+    import query_aware_block_b200 as lsa
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    wl = args.workload
+    # one step's algorithmic bytes set the rotation depth
+    base = make_case(wl, 1000 + 2 + 7919 * rank, "cpu" if wl == "tiny_decode" else dev)
+    dec_bytes, ref_bytes = algorithmic_bytes(base)
+    step_bytes = dec_bytes + ref_bytes
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    R = args.rotate or max(4, min(128, math.ceil(4 * l2 / step_bytes)))
+    if args.profile_small:
+        R = 2
+    B, Hkv, G, D, T_cap = base.shape
+    copies = []
+    for r in range(R):
+        c = base if r == 0 else make_case(wl, 1000 + 2 + 7919 * rank + 101 * r, dev)
+        q, k, v, sl = (t.to(dev) for t in (c.q, c.k, c.v, c.seqlens))
+        summ = torch.zeros(B, Hkv, -(-T_cap // 64), D, device=dev)
+        lsa.lsa_build_summaries(k, sl, summ)  # prefill-time summaries (not timed)
+        o = torch.empty_like(q)
+        lse = torch.empty(B, Hkv * G, device=dev)
+        idx = torch.empty(B, Hkv, base.topk, device=dev, dtype=torch.int32)
+        copies.append(dict(q=q, k=k, v=v, sl=sl, summ=summ, o=o, lse=lse, idx=idx))
+        del c
+    torch.cuda.synchronize()
+    topk, ns, nl = base.topk, base.n_sink, base.n_local
+
+    def step(c, stream=None):
+        lsa.lsa_build_summaries(c["k"], c["sl"], c["summ"], -1, -1, stream=stream)
+        lsa.lsa_sparse_attn_decode(c["q"], c["k"], c["v"], c["sl"], c["o"], topk, summ=c["summ"],
+                                   n_sink=ns, n_local=nl, idx_out=c["idx"], lse=c["lse"],
+                                   stream=stream)
+
+    def decode_only(c, stream=None):
+        lsa.lsa_sparse_attn_decode(c["q"], c["k"], c["v"], c["sl"], c["o"], topk, summ=c["summ"],
+                                   n_sink=ns, n_local=nl, idx_out=c["idx"], lse=c["lse"],
+                                   stream=stream)
+
+    # eager warm-up (also sets kernel attributes before any capture)
+    for i in range(max(3, min(args.warmup, 4 * R))):
+        step(copies[i % R])
+    torch.cuda.synchronize()
+
+    # graph of one rotation cycle: R steps, 2 kernels each
+    g_step = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_step):
+        for c in copies:
+            step(c)
+    # graph of the dominant kernel alone, with an event pair around every launch
+    ev_pairs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                for _ in range(R)]
+    g_dec = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_dec):
+        for c, (e0, e1) in zip(copies, ev_pairs):
+            e0.record()
+            decode_only(c)
+            e1.record()
+    torch.cuda.synchronize()
+
+    K, W = args.steps, args.warmup
+    if args.profile_small:
+        K, W = 2 * R, R
+    reps = max(1, K // R)
+    rem = K - reps * R
+    rem_graph = None
+    if rem:
+        rem_graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(rem_graph):
+            for c in copies[:rem]:
+                step(c)
+    # warm-up steps (untimed)
+    for _ in range(max(1, W // R)):
+        g_step.replay()
+    torch.cuda.synchronize()
+
+    def barrier():
+        if world > 1:
+            torch.distributed.barrier()
+
+    stream = torch.cuda.current_stream()
+    e_start = torch.cuda.Event(enable_timing=True)
+    e_stop = torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local_rank) as clocks:
+        barrier()
+        torch.cuda.synchronize()
+        e_start.record(stream)
+        for _ in range(reps):
+            g_step.replay()
+        if rem_graph is not None:
+            rem_graph.replay()
+        e_stop.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+    ms_total = e_start.elapsed_time(e_stop)
+    t = torch.tensor([ms_total], device=dev, dtype=torch.float64)
+    if world > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    ms_total = float(t.item())
+    ms_step = ms_total / K
+    tokens = world * B * K
+    value = tokens / (ms_total / 1e3)
+
+    # dominant kernel alone: per-launch CUDA-event durations
+    durs = []
+    for _ in range(max(1, min(50, 4096 // R))):
+        g_dec.replay()
+        torch.cuda.synchronize()
+        durs += [e0.elapsed_time(e1) for (e0, e1) in ev_pairs]
+    durs.sort()
+    dec_ms = sum(durs) / len(durs)
+    dec_ms_med = durs[len(durs) // 2]
+    peak, peak_kind = measured_peaks()
+    achieved = dec_bytes / (dec_ms * 1e-3) / 1e9
+    roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                "frac": round(achieved / peak, 4), "traffic": profiled_traffic(),
+                "kernel": "decode_cluster_kernel<bf16,128,FUSED>" if base.k.dtype == torch.bfloat16
+                else "decode_cluster_kernel<f32,FUSED>",
+                "peak_source": f"MEASURED_PEAKS.json hbm_gbs ({peak_kind})",
+                "algorithmic_bytes_per_launch": dec_bytes,
+                "launch_us_mean": round(dec_ms * 1e3, 3), "launch_us_median": round(dec_ms_med * 1e3, 3)}
+
+    # end to end through the C ABI with pinned host buffers
+    e2e = run_e2e(args, lsa, copies, base, dev, topk, ns, nl)
+    if world > 1:
+        te = torch.tensor([e2e["value"]], device=dev, dtype=torch.float64)
+        torch.distributed.all_reduce(te, op=torch.distributed.ReduceOp.MIN)  # slowest rank
+        e2e["value"] = float(te.item()) * world
+
+    result = {
+        "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": K,
+        "warmup": W, "ms_per_step": round(ms_step, 6), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16" if base.k.dtype == torch.bfloat16 else "f32",
+        "data": "synthetic (seeded N(0,1) q/k/v with RoPE theta 1e4 and planted needle blocks)",
+        "config": {"workload": wl, "batch": B, "kv_heads": Hkv, "q_heads_per_kv": G,
+                   "head_dim": D, "context": T_cap, "block": 64, "topk": topk,
+                   "forced": {"sink": ns, "local": nl},
+                   "l2": f"rotating {R} input copies ({R * step_bytes / 1e6:.0f} MB touched per "
+                         f"cycle, > 4x the {l2 / 1e6:.0f} MB L2)",
+                   "parallelism": f"replicas x{world} (independent sequences, no collective)"},
+        "effective_gbs": round(step_bytes / (ms_step * 1e-3) / 1e9, 1),
+        "bytes_per_step": step_bytes,
+        "roofline": roofline,
+        "e2e": e2e,
+        "gpu_launches": 2 * K,
+        "clocks": clocks.summary(),
+    }
+    return result
+
+
+def run_e2e(args, lsa, copies, base, dev, topk, ns, nl):
+    """Same metric through the public API, eager launches, pinned host buffers: every step
+    copies in q and the newest token's k and v and copies out o, lse and idx."""
+    R = len(copies)
+    B, Hkv, G, D, T_cap = base.shape
+    n = max(R, min(args.e2e_steps, args.steps))
+    hq = [copies[r]["q"].cpu().pin_memory() for r in range(R)]
+    last = [int(x) - 1 for x in base.seqlens.tolist()]
+    hk = [torch.stack([copies[r]["k"][b, :, last[b]] for b in range(B)]).cpu().pin_memory() for r in range(R)]
+    hv = [torch.stack([copies[r]["v"][b, :, last[b]] for b in range(B)]).cpu().pin_memory() for r in range(R)]
+    ho = torch.empty_like(copies[0]["o"], device="cpu").pin_memory()
+    hl = torch.empty_like(copies[0]["lse"], device="cpu").pin_memory()
+    hi = torch.empty_like(copies[0]["idx"], device="cpu").pin_memory()
+    kv_stage = torch.empty_like(hk[0], device=dev)
+    h2d = hq[0].numel() * hq[0].element_size() + 2 * hk[0].numel() * hk[0].element_size()
+    d2h = ho.numel() * ho.element_size() + hl.numel() * 4 + hi.numel() * 4
+
+    def one(i):
+        c = copies[i % R]
+        c["q"].copy_(hq[i % R], non_blocking=True)
+        kv_stage.copy_(hk[i % R], non_blocking=True)
+        for b in range(B):
+            c["k"][b, :, last[b]].copy_(kv_stage[b])
+        kv_stage.copy_(hv[i % R], non_blocking=True)
+        for b in range(B):
+            c["v"][b, :, last[b]].copy_(kv_stage[b])
+        lsa.lsa_build_summaries(c["k"], c["sl"], c["summ"], -1, -1)
+        lsa.lsa_sparse_attn_decode(c["q"], c["k"], c["v"], c["sl"], c["o"], topk, summ=c["summ"],
+                                   n_sink=ns, n_local=nl, idx_out=c["idx"], lse=c["lse"])
+        ho.copy_(c["o"], non_blocking=True)
+        hl.copy_(c["lse"], non_blocking=True)
+        hi.copy_(c["idx"], non_blocking=True)
+
+    for i in range(min(n, 3 * R)):
+        one(i)
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    t0 = time.perf_counter()
+    e0.record()
+    for i in range(n):
+        one(i)
+    e1.record()
+    torch.cuda.synchronize()
+    wall = time.perf_counter() - t0
+    ms = e0.elapsed_time(e1)
+    return {"value": round(B * n / (ms / 1e3), 1), "unit": UNIT, "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "steps": n, "host_wall_s": round(wall, 3),
+            "path": "python ctypes -> lsa_build_summaries + lsa_sparse_attn_decode, eager"}
+
+
+# ------------------------------------------------------------------ CPU (oracle) arm ----
+
+def oracle_step_runner(wl, seed=1002):
+    """The fp64 oracle's decode step on the same workload (inputs on the host): refresh the
+    last block's summary, score every block, select, attend.  Returns (run(units), meta)."""
+    import oracle
+    case = make_case(wl, seed, "cpu")
+    B, Hkv, G, D, T_cap = case.shape
+    summ = oracle.summaries(case.k, case.seqlens)  # prefill-time, not timed
+
+    def run(heads=None):
+        heads = heads or list(range(Hkv))
+        for b in range(B):
+            T = int(case.seqlens[b])
+            if T == 0:
+                continue
+            j = (T - 1) // 64
+            kb = case.k[b:b + 1, :, j * 64:T].contiguous()
+            summ[b:b + 1, :, j] = oracle.summaries(kb, torch.tensor([T - j * 64]))[:, :, 0]
+        hs = heads
+        q = case.q.view(B, Hkv, G, D)[:, hs].reshape(B, len(hs) * G, D).contiguous()
+        k = case.k[:, hs].contiguous() if len(hs) < Hkv else case.k
+        v = case.v[:, hs].contiguous() if len(hs) < Hkv else case.v
+        s = oracle.block_scores(q, summ[:, hs].contiguous(), case.seqlens)
+        idx, nsel = oracle.select(s, case.seqlens, case.topk, case.n_sink, case.n_local)
+        return oracle.decode_attn(q, k, v, case.seqlens, idx, nsel)
+
+    return run, dict(B=B, Hkv=Hkv)
+
+
+def cpu_baseline(wl, seconds):
+    import oracle
+    run, meta = oracle_step_runner(wl)
+    run()  # warm
+    n, t0 = 0, time.perf_counter()
+    while time.perf_counter() - t0 < seconds or n < 3:
+        run()
+        n += 1
+    dt = time.perf_counter() - t0
+    return {"value": round(meta["B"] * n / dt, 2), "unit": UNIT, "cores": oracle.num_threads(),
+            "kind": "oracle",
+            "sample": f"{n} full decode steps of the {wl} workload (last-block summary refresh, "
+                      f"scores of every block, selection, attention) in fp64 over {dt:.1f} s"}
+
+
+def run_reference(args):
+    import oracle
+    wl = args.workload
+    run, meta = oracle_step_runner(wl)
+    Hkv = meta["Hkv"]
+    t0 = time.perf_counter()
+    run()
+    t_full = time.perf_counter() - t0
+    budget = 150.0
+    K, W = args.steps, args.warmup
+    heads = Hkv
+    while heads > 1 and (K + W) * t_full * heads / Hkv > budget:
+        heads -= 1
+    hs = list(range(heads))
+    for _ in range(W):
+        run(hs)
+    timed = K
+    t0 = time.perf_counter()
+    done = 0
+    for i in range(K):
+        run(hs)
+        done += 1
+        if time.perf_counter() - t0 > budget:
+            break
+    dt = time.perf_counter() - t0
+    timed = done
+    frac = heads / Hkv
+    value = meta["B"] * frac * timed / dt
+    sample = (f"{timed} steps of the {wl} decode step restricted to {heads} of {Hkv} KV heads "
+              f"(heads are independent; tokens counted as {frac:.3f} per sequence per step)")
+    return {
+        "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": 1, "steps": timed,
+        "warmup": W, "ms_per_step": round(dt / timed * 1e3, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": wl}, "impl": "reference",
+        "cpu_baseline": {"value": round(value, 3), "unit": UNIT, "cores": oracle.num_threads(),
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(value, 3), "unit": UNIT, "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    args = parse()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args)), flush=True)
+        return
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local_rank))
+    res = run_ours(args, rank, world, local_rank)
+    if rank == 0 and not args.no_cpu_baseline and not args.profile_small:
+        res["cpu_baseline"] = cpu_baseline(args.workload, args.cpu_seconds)
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(res), flush=True)
+
+
+if __name__ == "__main__":
+    main()
