@@ -260,7 +260,8 @@ def run_ours(args, rank, world, local_rank):
         for c in copies:
             step(c)
     # graph of the dominant kernel alone, with an event pair around every launch
-    ev_pairs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+    ev_pairs = [(torch.cuda.Event(enable_timing=True, external=True),
+                 torch.cuda.Event(enable_timing=True, external=True))
                 for _ in range(R)]
     g_dec = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g_dec):
