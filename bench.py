@@ -8,10 +8,10 @@ Default workload: 64K-context GQA decode, bf16 (1 sequence, 8 KV heads x 8 query
 head dim 128, 65,536 cached tokens = 1,024 blocks of 64, top-16 blocks per KV head with
 block 0 and the last 2 blocks forced, 16 planted needle blocks per group).
 
-One step = one decode step of the whole hot path: refresh the summary of the block that
-holds the newest token (lsa_build_summaries on the last block) and one fused launch of
-block scoring + top-k selection + sparse attention over the selected blocks
-(lsa_sparse_attn_decode with idx == NULL).  Inputs are resident in HBM; R distinct input
+One step = one decode step of the whole hot path in one launch of lsa_sparse_attn_decode
+(idx == NULL, refresh_last_summary = 1): refresh of the summary of the block that holds the
+newest token, block scoring + top-k selection, and sparse attention over the selected
+blocks.  Inputs are resident in HBM; R distinct input
 copies are rotated so that R x (bytes a step touches) exceeds 4x the L2 size, i.e. every
 step reads cold data.  The K timed steps are replayed from a CUDA graph of one rotation
 cycle, bracketed by barrier + synchronize, timed with CUDA events (max over ranks).
@@ -68,6 +68,8 @@ def parse():
     ap.add_argument("--e2e-steps", type=int, default=2000)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-overlap", dest="overlap", action="store_false",
+                    help="launch steps without programmatic dependent launch")
     ap.add_argument("--profile-small", action="store_true",
                     help="a few launches on 2 input copies, for ncu captures")
     return ap.parse_args()
@@ -91,9 +93,10 @@ def make_case(wl, seed, device):
 
 
 def algorithmic_bytes(case):
-    """Bytes the method must move in one step (per kernel), from the definitions:
-    fused decode: summaries of the candidate blocks + K and V of the selected blocks' valid
-    tokens + q + o + lse + idx; summary refresh: the last block's valid keys + its summary."""
+    """Bytes the method must move in one decode step, from the definitions: summaries of
+    the candidate blocks + K and V of the selected blocks' valid tokens + q + o + lse + idx
+    + the refreshed summary of the newest block (its keys are among the selected ones).
+    Returns (bytes of the fused launch, bytes a separate summary refresh would add)."""
     B, Hkv, G, D, T_cap = case.shape
     esz = case.k.element_size()
     dec = 0
@@ -111,7 +114,8 @@ def algorithmic_bytes(case):
             toks = T
         dec += Hkv * toks * D * esz * 2                            # K and V
         last = T - (NB - 1) * 64 if NB else 0
-        ref += Hkv * (last * D * esz + D * 4)
+        dec += Hkv * D * 4 if NB else 0                            # refreshed summary
+        ref += Hkv * last * D * esz
     Hq = Hkv * G
     dec += B * Hq * D * esz * 2 + B * Hq * 4 + B * Hkv * case.topk * 4  # q, o, lse, idx
     return dec, ref
@@ -217,8 +221,8 @@ def run_ours(args, rank, world, local_rank):
     wl = args.workload
     # one step's algorithmic bytes set the rotation depth
     base = make_case(wl, 1000 + 2 + 7919 * rank, "cpu" if wl == "tiny_decode" else dev)
-    dec_bytes, ref_bytes = algorithmic_bytes(base)
-    step_bytes = dec_bytes + ref_bytes
+    dec_bytes, _ = algorithmic_bytes(base)
+    step_bytes = dec_bytes
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
     R = args.rotate or max(4, min(128, math.ceil(4 * l2 / step_bytes)))
     if args.profile_small:
@@ -238,23 +242,23 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.synchronize()
     topk, ns, nl = base.topk, base.n_sink, base.n_local
 
-    def step(c, stream=None):
-        lsa.lsa_build_summaries(c["k"], c["sl"], c["summ"], -1, -1, stream=stream)
+    flags = lsa.LSA_FLAG_PDL if args.overlap else 0
+
+    def step(c, stream=None, flags=flags):
+        # one launch: refresh of the newest block's summary + scoring + selection + attention
         lsa.lsa_sparse_attn_decode(c["q"], c["k"], c["v"], c["sl"], c["o"], topk, summ=c["summ"],
-                                   n_sink=ns, n_local=nl, idx_out=c["idx"], lse=c["lse"],
-                                   stream=stream)
+                                   n_sink=ns, n_local=nl, refresh_last_summary=True,
+                                   idx_out=c["idx"], lse=c["lse"], flags=flags, stream=stream)
 
     def decode_only(c, stream=None):
-        lsa.lsa_sparse_attn_decode(c["q"], c["k"], c["v"], c["sl"], c["o"], topk, summ=c["summ"],
-                                   n_sink=ns, n_local=nl, idx_out=c["idx"], lse=c["lse"],
-                                   stream=stream)
+        step(c, stream, flags=0)  # timed alone: no overlap with a neighbour
 
     # eager warm-up (also sets kernel attributes before any capture)
     for i in range(max(3, min(args.warmup, 4 * R))):
         step(copies[i % R])
     torch.cuda.synchronize()
 
-    # graph of one rotation cycle: R steps, 2 kernels each
+    # graph of one rotation cycle: R steps, one kernel each
     g_step = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g_step):
         for c in copies:
@@ -334,7 +338,8 @@ def run_ours(args, rank, world, local_rank):
                 "launch_us_mean": round(dec_ms * 1e3, 3), "launch_us_median": round(dec_ms_med * 1e3, 3)}
 
     # end to end through the C ABI with pinned host buffers
-    e2e = run_e2e(args, lsa, copies, base, dev, topk, ns, nl)
+    flags = lsa.LSA_FLAG_PDL if args.overlap else 0
+    e2e = run_e2e(args, lsa, copies, base, dev, topk, ns, nl, flags)
     if world > 1:
         te = torch.tensor([e2e["value"]], device=dev, dtype=torch.float64)
         torch.distributed.all_reduce(te, op=torch.distributed.ReduceOp.MIN)  # slowest rank
@@ -351,18 +356,19 @@ def run_ours(args, rank, world, local_rank):
                    "forced": {"sink": ns, "local": nl},
                    "l2": f"rotating {R} input copies ({R * step_bytes / 1e6:.0f} MB touched per "
                          f"cycle, > 4x the {l2 / 1e6:.0f} MB L2)",
-                   "parallelism": f"replicas x{world} (independent sequences, no collective)"},
+                   "parallelism": f"replicas x{world} (independent sequences, no collective)",
+                   "overlapped_launch": bool(args.overlap)},
         "effective_gbs": round(step_bytes / (ms_step * 1e-3) / 1e9, 1),
         "bytes_per_step": step_bytes,
         "roofline": roofline,
         "e2e": e2e,
-        "gpu_launches": 2 * K,
+        "gpu_launches": K,
         "clocks": clocks.summary(),
     }
     return result
 
 
-def run_e2e(args, lsa, copies, base, dev, topk, ns, nl):
+def run_e2e(args, lsa, copies, base, dev, topk, ns, nl, flags):
     """Same metric through the public API, eager launches, pinned host buffers: every step
     copies in q and the newest token's k and v and copies out o, lse and idx."""
     R = len(copies)
@@ -388,9 +394,9 @@ def run_e2e(args, lsa, copies, base, dev, topk, ns, nl):
         kv_stage.copy_(hv[i % R], non_blocking=True)
         for b in range(B):
             c["v"][b, :, last[b]].copy_(kv_stage[b])
-        lsa.lsa_build_summaries(c["k"], c["sl"], c["summ"], -1, -1)
         lsa.lsa_sparse_attn_decode(c["q"], c["k"], c["v"], c["sl"], c["o"], topk, summ=c["summ"],
-                                   n_sink=ns, n_local=nl, idx_out=c["idx"], lse=c["lse"])
+                                   n_sink=ns, n_local=nl, refresh_last_summary=True,
+                                   idx_out=c["idx"], lse=c["lse"], flags=flags)
         ho.copy_(c["o"], non_blocking=True)
         hl.copy_(c["lse"], non_blocking=True)
         hi.copy_(c["idx"], non_blocking=True)
@@ -410,7 +416,7 @@ def run_e2e(args, lsa, copies, base, dev, topk, ns, nl):
     ms = e0.elapsed_time(e1)
     return {"value": round(B * n / (ms / 1e3), 1), "unit": UNIT, "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": d2h, "steps": n, "host_wall_s": round(wall, 3),
-            "path": "python ctypes -> lsa_build_summaries + lsa_sparse_attn_decode, eager"}
+            "path": "python ctypes -> lsa_sparse_attn_decode (fused, with summary refresh), eager"}
 
 
 # ------------------------------------------------------------------ CPU (oracle) arm ----

@@ -58,6 +58,9 @@ extern "C" {
 #define LSA_F32 0
 #define LSA_BF16 1
 
+/* lsa_sparse_attn_decode flags */
+#define LSA_FLAG_PDL 1
+
 /* Human-readable name of a status code (static storage). */
 LSA_API const char* lsa_status_string(int status);
 
@@ -135,14 +138,27 @@ LSA_API int lsa_select_blocks(const void* q, int dtype, const float* summ, int B
  *   fused selection (idx == NULL): selection as in lsa_select_blocks is computed inside
  *       the same launch from summ (required) with n_sink / n_local; the selected indices
  *       are written to idx_out [B, Hkv, topk] (ascending, -1 padded) when it is non-NULL.
+ *       With refresh_last_summary != 0 (requires n_local >= 1) the launch also rewrites
+ *       summ[b, g, NB_b - 1, :] as the mean of that block's valid keys, i.e. the summary
+ *       update a decode step owes after appending a token, from the keys it loads anyway.
  * q [B, Hq, D]; k, v [B, Hkv, T_cap, D]; o [B, Hq, D] (dtype); lse [B, Hq] float32 or NULL.
+ * summ [B, Hkv, NB_cap, D] float32 (fused mode; written only by the refresh).
  * K/V rows at or beyond seqlens[b] are never used (they may hold any bits, NaN included).
+ * refresh_last_summary must be 0 in given-selection mode.
+ * flags: 0, or LSA_FLAG_PDL (fused mode only): launch with programmatic dependent launch,
+ *     so the kernel may start while the previous kernel of the stream still runs.  It then
+ *     reads seqlens, the summaries and the K/V of the forced blocks other than each
+ *     sequence's last block BEFORE that kernel completes; q and the last block's K/V are
+ *     read after it.  The caller guarantees the previous kernel writes none of the former
+ *     (true for a decode loop, where the previous kernel produces q and appends the newest
+ *     token; the summary a previous decode step refreshed is forced when n_local >= 2).
  */
 LSA_API int lsa_sparse_attn_decode(const void* q, const void* k, const void* v, int dtype, int B,
                            int Hkv, int G, int D, int T_cap, const int32_t* seqlens,
                            int blk, const int32_t* idx, const int32_t* nsel, int topk,
-                           float scale, const float* summ, int n_sink, int n_local,
-                           int32_t* idx_out, void* o, float* lse, cudaStream_t stream);
+                           float scale, float* summ, int n_sink, int n_local,
+                           int refresh_last_summary, int32_t* idx_out, void* o, float* lse,
+                           int flags, cudaStream_t stream);
 
 /*
  * lsa_sparse_attn_blockquery -- one denoising step of a block of Tq query tokens

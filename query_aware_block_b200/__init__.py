@@ -23,6 +23,7 @@ _lib = ctypes.CDLL(LIB_PATH)
 
 LSA_OK, LSA_ERR_INVALID_ARG, LSA_ERR_UNSUPPORTED, LSA_ERR_CUDA, LSA_ERR_DEVICE_STATUS = 0, 1, 2, 3, 4
 LSA_F32, LSA_BF16 = 0, 1
+LSA_FLAG_PDL = 1
 BLK = 64
 
 EXPORTED = ("lsa_status_string", "lsa_last_cuda_error", "lsa_version", "lsa_build_summaries",
@@ -38,7 +39,7 @@ _lib.lsa_build_summaries.argtypes = [_vp, _i, _i, _i, _i, _i, _vp, _i, _i, _i, _
 _lib.lsa_select_blocks.argtypes = [_vp, _i, _vp, _i, _i, _i, _i, _i, _vp, _i, _i, _i, _i, _f,
                                    _vp, _vp, _vp, _vp]
 _lib.lsa_sparse_attn_decode.argtypes = [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp, _i, _vp, _vp,
-                                        _i, _f, _vp, _i, _i, _vp, _vp, _vp, _vp]
+                                        _i, _f, _vp, _i, _i, _i, _vp, _vp, _vp, _i, _vp]
 _lib.lsa_sparse_attn_blockquery.argtypes = [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _vp,
                                             _i, _i, _i, _i, _f, _vp, _vp, _vp, _vp, _vp, _vp,
                                             _vp, _vp]
@@ -111,15 +112,17 @@ def lsa_select_blocks(q, summ, seqlens, topk, n_sink, n_local, idx, nsel, scale=
 
 
 def lsa_sparse_attn_decode(q, k, v, seqlens, o, topk, idx=None, nsel=None, summ=None,
-                           n_sink=0, n_local=0, idx_out=None, lse=None, scale=0.0, blk=BLK,
-                           stream=None):
-    """Sparse decode attention.  Given selection: idx, nsel.  Fused selection: summ."""
+                           n_sink=0, n_local=0, refresh_last_summary=False, idx_out=None,
+                           lse=None, scale=0.0, blk=BLK, flags=0, stream=None):
+    """Sparse decode attention.  Given selection: idx, nsel.  Fused selection: summ (and,
+    with refresh_last_summary, the last block's summary is rewritten in the same launch)."""
     B, Hq, D = q.shape
     _, Hkv, T_cap, _ = k.shape
     _check(_lib.lsa_sparse_attn_decode(_ptr(q), _ptr(k), _ptr(v), _dtype(q), B, Hkv, Hq // Hkv,
                                        D, T_cap, _ptr(seqlens), blk, _ptr(idx), _ptr(nsel),
                                        topk, float(scale), _ptr(summ), n_sink, n_local,
-                                       _ptr(idx_out), _ptr(o), _ptr(lse), _stream(stream)),
+                                       int(bool(refresh_last_summary)), _ptr(idx_out), _ptr(o),
+                                       _ptr(lse), int(flags), _stream(stream)),
            "lsa_sparse_attn_decode")
     return o
 

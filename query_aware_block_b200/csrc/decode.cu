@@ -8,30 +8,37 @@
 //               (ties to the lower block index); all blocks when NB <= topk
 //   o_h, lse_h = softmax attention of q_h over the tokens of the selected blocks
 //
-// How (B200):
-//   * A cluster of CL CTAs (16, 8 or 4) owns one (b, g).  Each CTA scores a contiguous
-//     slice of the NB block summaries with coalesced float4 loads (a warp per summary
-//     row), keeps its local top-m (m = topk - |F|) as 64-bit keys, and the CTAs exchange
-//     their sorted lists through distributed shared memory (DSMEM).  Every CTA derives the
-//     same global top-m from the gathered lists by binary-search ranking.
-//   * The selected blocks are dealt round-robin to the CTAs.  Forced blocks are known
-//     before any score is read, so in fused mode their K/V copies are issued before the
-//     summary scan and overlap it.
-//   * A 64-token block of K and V (16 KB each at D = 128, bf16) is staged with 16-byte
-//     cp.async into XOR-swizzled shared memory (2-stage pipeline).  For bf16 the G <= 16
-//     query heads form the M = 16 rows of mma.sync m16n8k16 for S = Q K^T and O += P V;
-//     the fp32 path uses CUDA-core FMA.  Online softmax in base 2, fp32 statistics.
-//   * The per-CTA partial (m, l, acc) is merged across the cluster by log-sum-exp over
-//     DSMEM; each CTA merges a 1/CL slice of the G x D outputs.
-// No global scratch memory, no spin-waits: cross-CTA ordering uses cluster barriers only.
-#include <cooperative_groups.h>
-
+// How (B200).  A decode step moves only a few MB, so the kernel is built for latency:
+//   * A cluster of CL CTAs (16, 8 or 4) owns one (b, g); 2 CTAs fit per SM, so a 16-CTA
+//     cluster per KV head fits in one wave.  At launch every CTA issues its slice of the
+//     summary rows (a warp per row, coalesced float4) and the group's query rows together;
+//     CTAs that own a forced block also start its K/V copy, so that copy overlaps the scan.
+//   * Each CTA ranks its candidates (64-bit keys: score, then lower index) and PUSHES its
+//     sorted local top-m list into every peer's shared memory (st.shared::cluster); after
+//     one release/acquire cluster barrier every CTA merges the CL sorted lists with a tree
+//     of warp-wide bitonic merges (shuffles only) and derives the same global top-m.
+//     DSMEM is touched only after a split arrive(relaxed)/wait barrier that proves every
+//     CTA of the cluster has started.
+//   * Overlapped launch (optional, programmatic dependent launch): the summary rows and the
+//     K/V of the forced blocks other than the newest one are requested before the kernel
+//     waits for the previous kernel of the stream; q and the newest block after it.
+//   * The selected blocks are dealt round-robin.  A 64-token block of K and V (16 KB each
+//     at D = 128, bf16) is staged with 16-byte cp.async into XOR-swizzled shared memory
+//     (2-stage pipeline).  For bf16 the G <= 16 query heads are the M = 16 rows of
+//     mma.sync m16n8k16 for S = Q K^T and O += P V; the fp32 path uses CUDA-core FMA.
+//     Online softmax in base 2 with fp32 statistics.
+//   * Each CTA pushes its partial (m, l) and the slices of its accumulator to the CTAs
+//     that own those output elements; after a second cluster barrier every CTA merges its
+//     1/CL slice by log-sum-exp from its own shared memory and writes it.  No CTA reads a
+//     peer's shared memory, so no trailing barrier is needed.
+//   * Optionally the CTA that attends the sequence's last block (always a forced local
+//     block) also refreshes that block's summary from the keys it staged: the summary
+//     update of a decode step costs no extra launch and no extra HBM read.
+// No global scratch memory and no spin-waits: cross-CTA ordering uses cluster barriers.
 #include <math.h>
 
 #include "lsa_common.cuh"
 #include "lsa_internal.h"
-
-namespace cg = cooperative_groups;
 
 namespace lsa {
 namespace {
@@ -40,11 +47,12 @@ typedef unsigned long long u64;
 
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
-constexpr int kRows = 16;      // query-head rows per group (G <= 16): the mma M dimension
+constexpr int kRows = 16;       // query-head rows per group (G <= 16): the mma M dimension
 constexpr int kMaxTopk = 64;
 constexpr int kMaxCluster = 16;
 constexpr int kStages = 2;
-constexpr int kSStride = 72;   // fp32 row stride of the score tile (bank spread)
+constexpr int kSStride = 72;    // fp32 row stride of the score tile (bank spread)
+constexpr int kRowsPerWarp = 8; // summary rows a warp has in flight per pass
 
 struct Params {
   const void* q;
@@ -53,57 +61,103 @@ struct Params {
   int Hkv, G, T_cap, NB_cap;
   const int32_t* seqlens;
   const float* summ;
+  float* summ_w;          // refresh target (fused mode), or null
   const int32_t* idx_in;
   const int32_t* nsel_in;
   int topk, n_sink, n_local;
-  float scale;       // natural-log softmax scale
+  float scale;            // natural-log softmax scale
   int32_t* idx_out;
   int32_t* nsel_out;
   float* scores_out;
   void* o;
   float* lse;
-  int per_max;       // max summary rows scored by one CTA
-  int m_pad;         // power of two >= topk
+  int per_max;            // max summary rows scored by one CTA
+  int m_pad;              // power of two >= topk
+  int lp;                 // length of an exchanged candidate list: max(16, m_pad)
+  int chunk;              // output elements merged by one CTA (even)
 };
+
+// ---- cluster primitives (PTX ISA: barrier.cluster, mapa, st.shared::cluster) ----------
+__device__ __forceinline__ int cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return (int)r;
+}
+__device__ __forceinline__ int cluster_size() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(r));
+  return (int)r;
+}
+__device__ __forceinline__ void cluster_arrive_relaxed() {
+  asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_arrive_release() {
+  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait() {
+  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ uint32_t map_rank(const void* p, int r) {
+  const uint32_t a = (uint32_t)__cvta_generic_to_shared(p);
+  uint32_t out;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(out) : "r"(a), "r"(r));
+  return out;
+}
+__device__ __forceinline__ void st_cluster(uint32_t addr, u64 v) {
+  asm volatile("st.shared::cluster.u64 [%0], %1;" ::"r"(addr), "l"(v) : "memory");
+}
+__device__ __forceinline__ void st_cluster(uint32_t addr, float2 v) {
+  asm volatile("st.shared::cluster.v2.f32 [%0], {%1, %2};" ::"r"(addr), "f"(v.x), "f"(v.y)
+               : "memory");
+}
+__device__ __forceinline__ void st_cluster(uint32_t addr, float v) {
+  asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
+}
+
+// Programmatic dependent launch (PTX griddepcontrol): with the launch attribute set, the
+// grid may start while the previous kernel of the stream still runs; `wait` blocks until
+// that kernel has completed and its memory is visible.  Without the attribute both are
+// no-ops in effect.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
 __host__ __device__ inline size_t align128(size_t x) { return (x + 127) & ~(size_t)127; }
 
 // Shared-memory carve-up (byte offsets), identical on host and device.
 struct Layout {
-  size_t qs, qsum, keys, top, work, all, gtop, order, kv, ss, ps, alpha, pm, pl, pacc, total;
+  size_t qs, keys, top, work, all, order, kv, ss, ps, alpha, ml_in, pacc_in, total;
   size_t kv_row, kv_tile;  // bytes per K/V row in smem, bytes per 64-row tile
 };
 
 __host__ __device__ inline Layout make_layout(int elem_bytes, int D, int per_max, int m_pad) {
   Layout L;
   size_t off = 0;
+  const int lp = m_pad < 16 ? 16 : m_pad;
+  const int nwork = (m_pad + kThreads) > (kMaxCluster / 2) * lp ? (m_pad + kThreads) : (kMaxCluster / 2) * lp;
   const bool f32 = elem_bytes == 4;
   L.kv_row = f32 ? (size_t)(D + 4) * 4 : (size_t)D * 2;
   L.kv_tile = L.kv_row * kBlk;
-  L.qs = off;    off = align128(off + (size_t)kRows * D * elem_bytes);
-  L.qsum = off;  off = align128(off + (size_t)D * 4);
-  L.keys = off;  off = align128(off + (size_t)per_max * 8);
-  L.top = off;   off = align128(off + (size_t)m_pad * 8);
-  L.work = off;  off = align128(off + (size_t)(m_pad + kThreads) * 8);
-  L.all = off;   off = align128(off + (size_t)kMaxCluster * m_pad * 8);
-  L.gtop = off;  off = align128(off + (size_t)m_pad * 8);
-  L.order = off; off = align128(off + (size_t)kMaxTopk * 4);
-  L.kv = off;    off = align128(off + (size_t)kStages * 2 * L.kv_tile);
-  L.ss = off;    off = align128(off + (size_t)kRows * kSStride * 4);
-  L.ps = off;    off = align128(off + (size_t)kRows * kBlk * 4);
-  L.alpha = off; off = align128(off + (size_t)kRows * 4);
-  L.pm = off;    off = align128(off + (size_t)kRows * 4);
-  L.pl = off;    off = align128(off + (size_t)kRows * 4);
-  L.pacc = off;  off = align128(off + (size_t)kRows * D * 4);
+  L.qs = off;      off = align128(off + (size_t)kRows * D * elem_bytes);
+  L.keys = off;    off = align128(off + (size_t)per_max * 8);
+  L.top = off;     off = align128(off + (size_t)lp * 8);
+  L.work = off;    off = align128(off + (size_t)nwork * 8);
+  L.all = off;     off = align128(off + (size_t)kMaxCluster * lp * 8);
+  L.order = off;   off = align128(off + (size_t)kMaxTopk * 4);
+  L.kv = off;      off = align128(off + (size_t)kStages * 2 * L.kv_tile);
+  L.ss = off;      off = align128(off + (size_t)kRows * kSStride * 4);
+  L.ps = off;      off = align128(off + (size_t)kRows * kBlk * 4);
+  L.alpha = off;   off = align128(off + (size_t)kRows * 4);
+  L.ml_in = off;   off = align128(off + (size_t)kMaxCluster * kRows * 8);
+  L.pacc_in = off; off = align128(off + (size_t)(kRows * D + 2 * kMaxCluster) * 4);
   L.total = off;
   return L;
 }
 
 // ---- selection helpers ------------------------------------------------------------------
 
-// Top-m of n keys (0 = not a candidate) into top[0..min(m, #valid)), descending.
-// top[] must be zero on entry.  Candidates are taken kThreads at a time together with the
-// current top list; each candidate's rank is the count of larger keys (keys are unique).
+// Top-m of n keys (0 = not a candidate) into top[0..min(m, #valid)), descending; top[]
+// must be zero on entry.  Candidates are taken kThreads at a time together with the
+// current list; a candidate's rank is the number of larger keys (keys are unique).
 __device__ void block_topm(const u64* keys, int n, int m, u64* top, u64* work) {
   int cur = 0;
   for (int base = 0; base < n; base += kThreads) {
@@ -117,7 +171,12 @@ __device__ void block_topm(const u64* keys, int n, int m, u64* top, u64* work) {
       const u64 x = (i < w) ? work[i] : 0ull;
       if (x != 0ull) {
         int r = 0;
-        for (int u = 0; u < w; ++u) r += work[u] > x;
+        int u = 0;
+        for (; u + 8 <= w; u += 8) {
+#pragma unroll
+          for (int k2 = 0; k2 < 8; ++k2) r += work[u + k2] > x;
+        }
+        for (; u < w; ++u) r += work[u] > x;
         if (r < m) top[r] = x;
       }
       nvalid += __syncthreads_count(x != 0ull);
@@ -127,19 +186,101 @@ __device__ void block_topm(const u64* keys, int n, int m, u64* top, u64* work) {
   __syncthreads();
 }
 
-// Number of entries greater than x in a descending, zero-padded list of n (power of 2).
-__device__ __forceinline__ int count_greater(const u64* L, int n, u64 x) {
-  int lo = 0;
-  for (int step = n >> 1; step > 0; step >>= 1)
-    if (L[lo + step - 1] > x) lo += step;
-  if (L[lo] > x) ++lo;
-  return lo;
+// Bitonic merge, descending, of the 32E-long sequence held by a warp (lane l holds
+// positions l*E .. l*E+E-1): positions [0, 16E) are a descending list and [16E, 32E) a
+// list in ascending order, so the whole is bitonic.  Afterwards the sequence is sorted
+// descending; the top 16E keys sit in lanes 0..15.
+template <int E>
+__device__ __forceinline__ void warp_merge_desc(u64 (&x)[E]) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int dist = 16 * E; dist >= 1; dist >>= 1) {
+    if (dist >= E) {
+      const int ld = dist / E;
+      const bool lower = (lane & ld) == 0;
+#pragma unroll
+      for (int e = 0; e < E; ++e) {
+        const u64 y = __shfl_xor_sync(0xffffffffu, x[e], ld);
+        x[e] = lower ? (x[e] > y ? x[e] : y) : (x[e] < y ? x[e] : y);
+      }
+    } else {
+#pragma unroll
+      for (int e = 0; e < E; ++e) {
+        if ((e & dist) == 0) {
+          const u64 a = x[e], b = x[e ^ dist];
+          x[e] = a > b ? a : b;
+          x[e ^ dist] = a > b ? b : a;
+        }
+      }
+    }
+  }
+}
+
+// Top list of the union of CL descending lists of 16E keys (zero padded) stored at
+// lists[c * 16E]: pairs are merged one warp each, level by level, ping-ponging between
+// `lists` and `work`.  Returns the buffer that holds the final list.
+template <int E>
+__device__ const u64* merge_lists(u64* lists, u64* work, int CL) {
+  constexpr int LP = 16 * E;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  u64* src = lists;
+  u64* dst = work;
+  for (int n = CL; n > 1; n >>= 1) {
+    for (int pr = warp; pr < (n >> 1); pr += kWarps) {
+      const u64* A = src + (2 * pr) * LP;
+      const u64* Bl = src + (2 * pr + 1) * LP;
+      u64 x[E];
+#pragma unroll
+      for (int e = 0; e < E; ++e) {
+        const int pos = lane * E + e;
+        x[e] = pos < LP ? A[pos] : Bl[2 * LP - 1 - pos];
+      }
+      warp_merge_desc<E>(x);
+      if (lane < 16) {
+#pragma unroll
+        for (int e = 0; e < E; ++e) dst[pr * LP + lane * E + e] = x[e];
+      }
+    }
+    __syncthreads();
+    u64* t = src;
+    src = dst;
+    dst = t;
+  }
+  return src;
+}
+
+// N consecutive elements as float.  kL2 = true reads through L2 only (ld.global.cg), for
+// data the previous kernel of the stream may have produced.
+template <typename T, int N, bool kL2 = false>
+__device__ __forceinline__ void load_f32(const T* p, float (&out)[N]) {
+  if constexpr (sizeof(T) == 4) {
+    if constexpr (N == 4) {
+      const float4 v = kL2 ? __ldcg(reinterpret_cast<const float4*>(p)) : __ldg(reinterpret_cast<const float4*>(p));
+      out[0] = v.x; out[1] = v.y; out[2] = v.z; out[3] = v.w;
+    } else {
+      const float2 v = kL2 ? __ldcg(reinterpret_cast<const float2*>(p)) : __ldg(reinterpret_cast<const float2*>(p));
+      out[0] = v.x; out[1] = v.y;
+    }
+  } else {
+    if constexpr (N == 4) {
+      const uint2 v = kL2 ? __ldcg(reinterpret_cast<const uint2*>(p)) : __ldg(reinterpret_cast<const uint2*>(p));
+      const __nv_bfloat162 a = *reinterpret_cast<const __nv_bfloat162*>(&v.x);
+      const __nv_bfloat162 b = *reinterpret_cast<const __nv_bfloat162*>(&v.y);
+      out[0] = __low2float(a); out[1] = __high2float(a);
+      out[2] = __low2float(b); out[3] = __high2float(b);
+    } else {
+      const uint32_t v = kL2 ? __ldcg(reinterpret_cast<const unsigned int*>(p)) : __ldg(reinterpret_cast<const unsigned int*>(p));
+      const __nv_bfloat162 a = *reinterpret_cast<const __nv_bfloat162*>(&v);
+      out[0] = __low2float(a); out[1] = __high2float(a);
+    }
+  }
 }
 
 // ---- K/V block staging ----------------------------------------------------------------
 
-// Copy the K and V rows of block j into a stage (rows >= Tb are zero-filled and never
-// read from global memory).  bf16 rows are chunk-swizzled; fp32 rows are padded.
+// Copy the K and V rows of block j into a stage (rows >= Tb, and every row of an invalid
+// j < 0, are zero-filled and never read from global memory).  bf16 rows are
+// chunk-swizzled; fp32 rows are padded by 16 bytes.
 template <typename T, int D>
 __device__ __forceinline__ void stage_block(unsigned char* dst_k, unsigned char* dst_v,
                                             const T* kbase, const T* vbase, int j, int Tb,
@@ -164,10 +305,13 @@ __device__ __forceinline__ void stage_block(unsigned char* dst_k, unsigned char*
 // ---- the kernel ---------------------------------------------------------------------
 
 template <typename T, int D, int MODE>
-__global__ void __launch_bounds__(kThreads, 1) decode_cluster_kernel(const Params p) {
-  cg::cluster_group cluster = cg::this_cluster();
-  const int CL = (int)cluster.num_blocks();
-  const int rank = (int)cluster.block_rank();
+__global__ void __launch_bounds__(kThreads, 2) decode_cluster_kernel(const Params p) {
+  const int CL = cluster_size();
+  const int rank = cluster_rank();
+  // DSMEM may be written only once every CTA of the cluster runs: arrive now, wait late
+  cluster_arrive_relaxed();
+  bool started = false;  // uniform: the start barrier has been waited on
+
   const int g = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int G = p.G;
@@ -179,20 +323,17 @@ __global__ void __launch_bounds__(kThreads, 1) decode_cluster_kernel(const Param
   extern __shared__ __align__(1024) unsigned char smem[];
   const Layout Lo = make_layout((int)sizeof(T), D, p.per_max, p.m_pad);
   unsigned char* Qs = smem + Lo.qs;
-  float* qsum = reinterpret_cast<float*>(smem + Lo.qsum);
   u64* keys = reinterpret_cast<u64*>(smem + Lo.keys);
   u64* top = reinterpret_cast<u64*>(smem + Lo.top);
   u64* work = reinterpret_cast<u64*>(smem + Lo.work);
   u64* all = reinterpret_cast<u64*>(smem + Lo.all);
-  u64* gtop = reinterpret_cast<u64*>(smem + Lo.gtop);
   int* order = reinterpret_cast<int*>(smem + Lo.order);
   unsigned char* kv = smem + Lo.kv;
   float* Ss = reinterpret_cast<float*>(smem + Lo.ss);
   unsigned char* Ps = smem + Lo.ps;
   float* alpha_s = reinterpret_cast<float*>(smem + Lo.alpha);
-  float* pm = reinterpret_cast<float*>(smem + Lo.pm);
-  float* pl = reinterpret_cast<float*>(smem + Lo.pl);
-  float* pacc = reinterpret_cast<float*>(smem + Lo.pacc);
+  float2* ml_in = reinterpret_cast<float2*>(smem + Lo.ml_in);
+  float* pacc_in = reinterpret_cast<float*>(smem + Lo.pacc_in);
   const int kv_row = (int)Lo.kv_row;
   const int kv_tile = (int)Lo.kv_tile;
 
@@ -201,97 +342,101 @@ __global__ void __launch_bounds__(kThreads, 1) decode_cluster_kernel(const Param
   const T* kbase = static_cast<const T*>(p.k) + unit * (size_t)p.T_cap * D;
   const T* vbase = static_cast<const T*>(p.v) + unit * (size_t)p.T_cap * D;
 
-  // ---- the forced set and the block order ------------------------------------------------
-  // order[0..n_order) lists the blocks to attend; order[i] is handled by CTA i % CL.
+  // ---- which blocks: forced / all known up front; order[i] is handled by CTA i % CL ----
   const bool select = MODE != MODE_ATTEND;
   const bool all_blocks = select && NB <= p.topk;
-  int nf = 0, n_order = 0;
+  const int nf = (select && !all_blocks) ? p.n_sink + p.n_local : 0;  // disjoint: NB > topk
+  int n_order;
   if (select) {
-    if (all_blocks) {
-      for (int i = tid; i < NB; i += kThreads) order[i] = i;
-      n_order = NB;
-    } else {
-      // NB > topk >= n_sink + n_local: the two forced ranges are disjoint
-      nf = p.n_sink + p.n_local;
-      for (int i = tid; i < nf; i += kThreads) order[i] = i < p.n_sink ? i : NB - p.n_local + (i - p.n_sink);
-      n_order = p.topk;
-    }
+    n_order = all_blocks ? NB : p.topk;
+    const int known = all_blocks ? NB : nf;
+    for (int i = tid; i < known; i += kThreads)
+      order[i] = all_blocks ? i : (i < p.n_sink ? i : NB - p.n_local + (i - p.n_sink));
   } else {
-    const int ns = max(0, min(p.nsel_in[unit], p.topk));  // never past order[kMaxTopk]
-    for (int i = tid; i < ns; i += kThreads) order[i] = p.idx_in[unit * p.topk + i];
-    n_order = ns;
+    n_order = max(0, min(__ldcg(p.nsel_in + unit), p.topk));  // never past order[kMaxTopk]
+    for (int i = tid; i < n_order; i += kThreads) order[i] = __ldcg(p.idx_in + unit * p.topk + i);
   }
-  // query rows (zero rows beyond G): bf16 swizzled for ldmatrix, fp32 plain
+  auto known_block = [&](int i) {
+    const int o = rank + i * CL;
+    return all_blocks ? o : (o < p.n_sink ? o : NB - p.n_local + (o - p.n_sink));
+  };
+  for (int i = tid; i < p.lp; i += kThreads) top[i] = 0ull;
+
+  // ---- before waiting on the previous kernel of the stream: copies of data that kernel
+  // cannot have written (the K/V of the known blocks except the sequence's newest one, and
+  // the first pass of summary rows).  With overlapped launch the caller vouches for this.
+  int issued = 0;  // my blocks whose copies were committed, in processing order
+  const int known = all_blocks ? NB : nf;
+  const int n_known = (MODE == MODE_FUSED && known > rank) ? (known - rank + CL - 1) / CL : 0;
+  if (MODE == MODE_FUSED) {
+    while (issued < kStages && issued < n_known && known_block(issued) != NB - 1) {
+      unsigned char* st = kv + (size_t)(issued % kStages) * 2 * kv_tile;
+      stage_block<T, D>(st, st + kv_tile, kbase, vbase, known_block(issued), Tb, kv_row);
+      cp_async_commit();
+      ++issued;
+    }
+  }
+  constexpr int VEC = D / 32;  // elements per lane of a D-row
+  const bool scan = select && !all_blocks;
+  const int per = (NB + CL - 1) / CL;
+  const int j0 = rank * per;
+  const int nloc = scan ? max(0, min(NB, j0 + per) - j0) : 0;
+  const float* sb = p.summ + unit * (size_t)p.NB_cap * D + lane * VEC;
+  float vals[kRowsPerWarp][VEC];
+  auto load_pass = [&](int o0) {
+#pragma unroll
+    for (int u = 0; u < kRowsPerWarp; ++u) {
+      const int oo = o0 + u * kWarps;
+      if (oo < nloc) {
+        load_f32<float, VEC>(sb + (size_t)(j0 + oo) * D, vals[u]);
+      } else {
+#pragma unroll
+        for (int e = 0; e < VEC; ++e) vals[u][e] = 0.f;
+      }
+    }
+  };
+  if (scan) load_pass(warp);
+  pdl_trigger();
+  pdl_wait();
+
+  // ---- query rows (staged for the mma) and the newest block, after the wait ------------
   if (MODE != MODE_SELECT) {
     constexpr int kQChunks = kRows * kRowBytesQ / 16;
     for (int id = tid; id < kQChunks; id += kThreads) {
       const int row = id / (kRowBytesQ / 16), c = id % (kRowBytesQ / 16);
-      const bool valid = row < G;
-      const T* src = qg + (size_t)(valid ? row : 0) * D + c * (16 / sizeof(T));
-      unsigned char* dst = Qs + (kF32 ? row * kRowBytesQ + c * 16 : swz(row, c, kRowBytesQ));
-      cp_async16(dst, src, valid);
+      uint4 v4 = make_uint4(0u, 0u, 0u, 0u);
+      if (row < G) v4 = __ldcg(reinterpret_cast<const uint4*>(qg + (size_t)row * D) + c);
+      *reinterpret_cast<uint4*>(Qs + (kF32 ? row * kRowBytesQ + c * 16 : swz(row, c, kRowBytesQ))) = v4;
     }
-    cp_async_commit();
   }
-  __syncthreads();
-
-  // ---- prefetch the blocks already known (forced, or all) ------------------------------
-  int issued = 0;  // number of my blocks whose copies were committed
-  auto my_block = [&](int i) { return order[rank + i * CL]; };
-  int n_my_known = 0;
   if (MODE == MODE_FUSED) {
-    const int known = all_blocks ? n_order : nf;
-    n_my_known = known > rank ? (known - rank + CL - 1) / CL : 0;
-    while (issued < kStages && issued < n_my_known) {
-      const int j = my_block(issued);
+    while (issued < kStages && issued < n_known) {
       unsigned char* st = kv + (size_t)(issued % kStages) * 2 * kv_tile;
-      stage_block<T, D>(st, st + kv_tile, kbase, vbase, j, Tb, kv_row);
+      stage_block<T, D>(st, st + kv_tile, kbase, vbase, known_block(issued), Tb, kv_row);
       cp_async_commit();
       ++issued;
     }
   }
 
-  // ---- selection ----------------------------------------------------------------------
-  if (select && !all_blocks) {
+  // ---- selection --------------------------------------------------------------------
+  if (scan) {
     const int m = p.topk - nf;
-    // summed, scaled query of the group
-    for (int d = tid; d < D; d += kThreads) {
-      float s = 0.f;
-      for (int h = 0; h < G; ++h) s += to_f32(qg[(size_t)h * D + d]);
-      qsum[d] = s * p.scale;
-    }
-    for (int i = tid; i < p.m_pad; i += kThreads) top[i] = 0ull;
-    __syncthreads();
-    constexpr int VEC = D / 32;  // floats per lane per summary row
+    // summed, scaled query of the group, per warp in registers
     float qv[VEC];
 #pragma unroll
-    for (int e = 0; e < VEC; ++e) qv[e] = qsum[lane * VEC + e];
-    const int per = (NB + CL - 1) / CL;
-    const int j0 = rank * per;
-    const int nloc = max(0, min(NB, j0 + per) - j0);
-    const float* sb = p.summ + unit * (size_t)p.NB_cap * D + lane * VEC;
-    constexpr int kUnroll = 8;
-    for (int o0 = warp; o0 < nloc; o0 += kWarps * kUnroll) {
-      float vals[kUnroll][VEC];
+    for (int e = 0; e < VEC; ++e) qv[e] = 0.f;
+    for (int h = 0; h < G; ++h) {
+      float t[VEC];
+      load_f32<T, VEC, true>(qg + (size_t)h * D + lane * VEC, t);
 #pragma unroll
-      for (int u = 0; u < kUnroll; ++u) {
-        const int oo = o0 + u * kWarps;
-        if (oo < nloc) {
-          const float* src = sb + (size_t)(j0 + oo) * D;
-          if constexpr (VEC == 4) {
-            const float4 t4 = __ldg(reinterpret_cast<const float4*>(src));
-            vals[u][0] = t4.x; vals[u][1] = t4.y; vals[u][2] = t4.z; vals[u][3] = t4.w;
-          } else {
-            const float2 t2 = __ldg(reinterpret_cast<const float2*>(src));
-            vals[u][0] = t2.x; vals[u][1] = t2.y;
-          }
-        } else {
+      for (int e = 0; e < VEC; ++e) qv[e] += t[e];
+    }
 #pragma unroll
-          for (int e = 0; e < VEC; ++e) vals[u][e] = 0.f;
-        }
-      }
+    for (int e = 0; e < VEC; ++e) qv[e] *= p.scale;
+    for (int o0 = warp;; o0 += kWarps * kRowsPerWarp) {
+      if (o0 != warp) load_pass(o0);
 #pragma unroll
-      for (int u = 0; u < kUnroll; ++u) {
+      for (int u = 0; u < kRowsPerWarp; ++u) {
         const int oo = o0 + u * kWarps;
         float dot = 0.f;
 #pragma unroll
@@ -304,30 +449,43 @@ __global__ void __launch_bounds__(kThreads, 1) decode_cluster_kernel(const Param
           if (p.scores_out) p.scores_out[unit * p.NB_cap + j] = dot;
         }
       }
+      if (o0 + kWarps * kRowsPerWarp >= nloc) break;
     }
     __syncthreads();
-    block_topm(keys, nloc, m, top, work);
-    cluster.sync();  // every CTA's local list is complete
-    // gather all lists and rank every candidate among them
-    const int nall = CL * p.m_pad;
-    for (int t = tid; t < nall; t += kThreads) {
-      const u64* peer = cluster.map_shared_rank(top, t / p.m_pad);
-      all[t] = peer[t % p.m_pad];
+    // local top-m, sorted, zero padded to lp
+    if (nloc <= kThreads) {
+      const u64 x = tid < nloc ? keys[tid] : 0ull;
+      if (x != 0ull) {
+        int r = 0, u = 0;
+        for (; u + 8 <= nloc; u += 8) {
+          const ulonglong2* k2 = reinterpret_cast<const ulonglong2*>(keys + u);
+#pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4) {
+            const ulonglong2 kk = k2[q4];
+            r += (kk.x > x) + (kk.y > x);
+          }
+        }
+        for (; u < nloc; ++u) r += keys[u] > x;
+        if (r < m) top[r] = x;
+      }
+      __syncthreads();
+    } else {
+      block_topm(keys, nloc, m, top, work);
     }
-    __syncthreads();
-    for (int t = tid; t < nall; t += kThreads) {
-      const u64 x = all[t];
-      if (x == 0ull) continue;
-      const int c = t / p.m_pad;
-      int r = t % p.m_pad;
-      for (int l = 0; l < CL; ++l)
-        if (l != c) r += count_greater(all + l * p.m_pad, p.m_pad, x);
-      if (r < m) gtop[r] = x;
+    // push the list into every peer (all[rank][*] on each CTA), then merge all lists
+    cluster_wait();
+    started = true;
+    for (int t = tid; t < CL * p.lp; t += kThreads) {
+      const int peer = t / p.lp, pos = t - peer * p.lp;
+      st_cluster(map_rank(all + rank * p.lp + pos, peer), top[pos]);
     }
-    __syncthreads();
-    for (int r = tid; r < m; r += kThreads) order[nf + r] = key_block(gtop[r]);
-    __syncthreads();
+    cluster_arrive_release();
+    cluster_wait();
+    const u64* fin = p.lp == 16 ? merge_lists<1>(all, work, CL)
+                   : (p.lp == 32 ? merge_lists<2>(all, work, CL) : merge_lists<4>(all, work, CL));
+    for (int r = tid; r < m; r += kThreads) order[nf + r] = key_block(fin[r]);
   }
+  __syncthreads();
 
   // selected indices, ascending (written by rank 0)
   if (select && rank == 0) {
@@ -337,6 +495,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_cluster_kernel(const Param
         if (i < n_order) {
           const int v = order[i];
           int pos = 0;
+#pragma unroll 8
           for (int u = 0; u < n_order; ++u) pos += order[u] < v;
           out[pos] = v;
         } else {
@@ -347,30 +506,24 @@ __global__ void __launch_bounds__(kThreads, 1) decode_cluster_kernel(const Param
     if (MODE == MODE_SELECT && tid == 0) p.nsel_out[unit] = n_order;
   }
   if (MODE == MODE_SELECT) {
-    cluster.sync();  // peers may still be reading this CTA's list
-    return;
+    if (!started) cluster_wait();
+    return;  // no CTA reads a peer's shared memory: no trailing barrier
   }
 
   // ---- attention over my share of the blocks ------------------------------------------
   const int n_my = n_order > rank ? (n_order - rank + CL - 1) / CL : 0;
   while (issued < kStages && issued < n_my) {
-    const int j = my_block(issued);
     unsigned char* st = kv + (size_t)(issued % kStages) * 2 * kv_tile;
-    stage_block<T, D>(st, st + kv_tile, kbase, vbase, j, Tb, kv_row);
+    stage_block<T, D>(st, st + kv_tile, kbase, vbase, order[rank + issued * CL], Tb, kv_row);
     cp_async_commit();
     ++issued;
   }
-  // the query copy was committed before every K/V copy: wait for it alone
-  if (issued >= 2) cp_async_wait<2>();
-  else if (issued == 1) cp_async_wait<1>();
-  else cp_async_wait<0>();
-  __syncthreads();
+  __syncthreads();  // (the staged query rows are visible)
 
   const float scale2 = p.scale * kLog2e;
   float m_run = -INFINITY, l_run = 0.f;  // softmax row state (row = tid >> 4)
   const int srow = tid >> 4, ssub = tid & 15;
-  // bf16 path: query A fragments and output accumulators in registers
-  constexpr int NT = kF32 ? 1 : D / 64;  // n8 tiles of the output per warp
+  constexpr int NT = kF32 ? 1 : D / 64;  // n8 tiles of the output per warp (bf16)
   uint32_t qa[kF32 ? 1 : D / 16][4];
   float acc[kF32 ? D / 16 : NT][kF32 ? 1 : 4];
   if constexpr (kF32) {
@@ -393,7 +546,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_cluster_kernel(const Param
   for (int i = 0; i < n_my; ++i) {
     if (issued > i + 1) cp_async_wait<1>(); else cp_async_wait<0>();
     __syncthreads();
-    const int j = my_block(i);
+    const int j = order[rank + i * CL];
     const unsigned char* Ks = kv + (size_t)(i % kStages) * 2 * kv_tile;
     const unsigned char* Vs = Ks + kv_tile;
 
@@ -500,51 +653,83 @@ __global__ void __launch_bounds__(kThreads, 1) decode_cluster_kernel(const Param
         }
       }
     }
+    // the summary of the sequence's last block, from the keys staged here
+    if (p.summ_w != nullptr && j == NB - 1) {
+      const int n = Tb - j * kBlk;
+      for (int d = tid; d < D; d += kThreads) {
+        float s = 0.f;
+        if constexpr (kF32) {
+#pragma unroll 8
+          for (int t = 0; t < n; ++t) s += reinterpret_cast<const float*>(Ks + t * kv_row)[d];
+        } else {
+          const int c = d >> 3, wd = d & 7;
+#pragma unroll 8
+          for (int t = 0; t < n; ++t)
+            s += __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(Ks + swz(t, c, kv_row))[wd]);
+        }
+        p.summ_w[(unit * p.NB_cap + j) * D + d] = s / (float)n;
+      }
+    }
     __syncthreads();  // the stage may now be refilled
     if (issued < n_my) {
-      const int jn = my_block(issued);
       unsigned char* st = kv + (size_t)(issued % kStages) * 2 * kv_tile;
-      stage_block<T, D>(st, st + kv_tile, kbase, vbase, jn, Tb, kv_row);
+      stage_block<T, D>(st, st + kv_tile, kbase, vbase, order[rank + issued * CL], Tb, kv_row);
       cp_async_commit();
       ++issued;
     }
   }
 
-  // ---- partial (m, l, acc) of this CTA -> shared memory ---------------------------------
-  if (ssub == 0) {
-    pm[srow] = m_run;
-    pl[srow] = l_run;
+  // ---- push the partial (m, l, acc) to the CTAs that merge each output slice -----------
+  if (!started) {
+    cluster_wait();
+    started = true;
   }
+  const int E = G * D;
+  const int chunk = p.chunk;
+  if (ssub < CL) st_cluster(map_rank(ml_in + rank * kRows + srow, ssub), make_float2(m_run, l_run));
   if constexpr (kF32) {
+    if (srow < G) {
 #pragma unroll
-    for (int e = 0; e < D / 16; ++e) pacc[srow * D + ssub + 16 * e] = acc[e][0];
+      for (int e2 = 0; e2 < D / 16; ++e2) {
+        const int e = srow * D + ssub + 16 * e2;
+        const int owner = e / chunk;
+        st_cluster(map_rank(pacc_in + rank * chunk + (e - owner * chunk), owner), acc[e2][0]);
+      }
+    }
   } else {
     const int r0 = lane >> 2;
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
       const int d = (D == 128 ? 16 * warp : 8 * warp) + 8 * nt + 2 * (lane & 3);
-      *reinterpret_cast<float2*>(pacc + r0 * D + d) = make_float2(acc[nt][0], acc[nt][1]);
-      *reinterpret_cast<float2*>(pacc + (r0 + 8) * D + d) = make_float2(acc[nt][2], acc[nt][3]);
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        const int row = r0 + 8 * half;
+        if (row < G) {
+          const int e = row * D + d;
+          const int owner = e / chunk;
+          st_cluster(map_rank(pacc_in + rank * chunk + (e - owner * chunk), owner),
+                     make_float2(acc[nt][2 * half], acc[nt][2 * half + 1]));
+        }
+      }
     }
   }
-  cluster.sync();
+  cluster_arrive_release();
+  cluster_wait();
 
-  // ---- log-sum-exp merge of the CL partials; this CTA writes a 1/CL slice -----------
+  // ---- log-sum-exp merge of this CTA's slice, from its own shared memory ---------------
   {
-    const int E = G * D;
-    const int chunk = (E + CL - 1) / CL;
-    const int e_end = min(E, (rank + 1) * chunk);
     T* og = static_cast<T*>(p.o) + ((size_t)b * p.Hkv * G + (size_t)g * G) * D;
-    for (int e = rank * chunk + tid; e < e_end; e += kThreads) {
-      const int h = e / D, d = e % D;
-      float mp[kMaxCluster];
+    const int e0 = rank * chunk;
+    const int e_end = min(E, e0 + chunk);
+    for (int e = e0 + tid; e < e_end; e += kThreads) {
+      const int h = e / D, d = e - h * D;
+      float2 ml[kMaxCluster];
       float M = -INFINITY;
 #pragma unroll
       for (int r = 0; r < kMaxCluster; ++r) {
-        mp[r] = -INFINITY;
         if (r < CL) {
-          mp[r] = *cluster.map_shared_rank(pm + h, r);
-          M = fmaxf(M, mp[r]);
+          ml[r] = ml_in[r * kRows + h];
+          M = fmaxf(M, ml[r].x);
         }
       }
       float Lsum = 0.f, O = 0.f;
@@ -552,9 +737,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_cluster_kernel(const Param
 #pragma unroll
         for (int r = 0; r < kMaxCluster; ++r) {
           if (r < CL) {
-            const float w = ex2(mp[r] - M);
-            Lsum = fmaf(*cluster.map_shared_rank(pl + h, r), w, Lsum);
-            O = fmaf(*cluster.map_shared_rank(pacc + h * D + d, r), w, O);
+            const float w = ex2(ml[r].x - M);
+            Lsum = fmaf(ml[r].y, w, Lsum);
+            O = fmaf(pacc_in[r * chunk + (e - e0)], w, O);
           }
         }
       }
@@ -564,7 +749,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_cluster_kernel(const Param
             M == -INFINITY ? -INFINITY : (M + log2f(Lsum)) * kLn2;
     }
   }
-  cluster.sync();  // keep this CTA's shared memory alive until every peer has read it
 }
 
 // ---- host side --------------------------------------------------------------------------
@@ -584,11 +768,13 @@ cudaError_t launch_t(const DecodeArgs& a, cudaStream_t stream) {
   Params p;
   p.q = a.q; p.k = a.k; p.v = a.v;
   p.Hkv = a.Hkv; p.G = a.G; p.T_cap = a.T_cap; p.NB_cap = a.NB_cap;
-  p.seqlens = a.seqlens; p.summ = a.summ; p.idx_in = a.idx_in; p.nsel_in = a.nsel_in;
+  p.seqlens = a.seqlens; p.summ = a.summ; p.summ_w = a.summ_w;
+  p.idx_in = a.idx_in; p.nsel_in = a.nsel_in;
   p.topk = a.topk; p.n_sink = a.n_sink; p.n_local = a.n_local; p.scale = a.scale;
   p.idx_out = a.idx_out; p.nsel_out = a.nsel_out; p.scores_out = a.scores_out;
   p.o = a.o; p.lse = a.lse;
   p.m_pad = next_pow2(a.topk < 2 ? 2 : a.topk);
+  p.lp = p.m_pad < 16 ? 16 : p.m_pad;
   // per template instance: the largest dynamic smem size set so far, and the last
   // (cluster size, smem) pair whose occupancy was checked
   static int smem_set = 0;
@@ -596,6 +782,8 @@ cudaError_t launch_t(const DecodeArgs& a, cudaStream_t stream) {
   cudaError_t err;
   for (;;) {
     p.per_max = (a.NB_cap + CL - 1) / CL;
+    const int E = a.G * D;
+    p.chunk = ((E + CL - 1) / CL + 1) & ~1;
     const Layout Lo = make_layout((int)sizeof(T), D, p.per_max, p.m_pad);
     const int smem = (int)Lo.total;
     if (smem > smem_set) {
@@ -610,13 +798,15 @@ cudaError_t launch_t(const DecodeArgs& a, cudaStream_t stream) {
     cfg.blockDim = dim3(kThreads, 1, 1);
     cfg.dynamicSmemBytes = (size_t)smem;
     cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = CL;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = (MODE == MODE_FUSED && a.pdl) ? 2 : 1;
     if (!(CL == last_cl && smem == last_smem)) {
       int nclusters = 0;
       err = cudaOccupancyMaxActiveClusters(&nclusters, kernel, &cfg);

@@ -102,12 +102,13 @@ int lsa_select_blocks(const void* q, int dtype, const float* summ, int B, int Hk
 int lsa_sparse_attn_decode(const void* q, const void* k, const void* v, int dtype, int B,
                            int Hkv, int G, int D, int T_cap, const int32_t* seqlens,
                            int blk, const int32_t* idx, const int32_t* nsel, int topk,
-                           float scale, const float* summ, int n_sink, int n_local,
-                           int32_t* idx_out, void* o, float* lse, cudaStream_t stream) {
+                           float scale, float* summ, int n_sink, int n_local,
+                           int refresh_last_summary, int32_t* idx_out, void* o, float* lse,
+                           int flags, cudaStream_t stream) {
   int st = check_common(dtype, B, Hkv, G, D, blk);
   if (st != LSA_OK) return st;
   if (topk < 1 || topk > 64) return LSA_ERR_INVALID_ARG;
-  if (T_cap < 0) return LSA_ERR_INVALID_ARG;
+  if (T_cap < 0 || (flags & ~LSA_FLAG_PDL) != 0) return LSA_ERR_INVALID_ARG;
   if (T_cap > kMaxTcap) return LSA_ERR_UNSUPPORTED;
   if (B == 0 || Hkv == 0) return LSA_OK;
   if (!q || !k || !v || !seqlens || !o) return LSA_ERR_INVALID_ARG;
@@ -116,18 +117,22 @@ int lsa_sparse_attn_decode(const void* q, const void* k, const void* v, int dtyp
   if (fused) {
     if (!summ || !aligned16(summ)) return LSA_ERR_INVALID_ARG;
     if (n_sink < 0 || n_local < 0 || n_sink + n_local > topk) return LSA_ERR_INVALID_ARG;
-  } else if (!nsel) {
+    // the refreshed block must be a forced one, so that no CTA scores it meanwhile
+    if (refresh_last_summary && n_local < 1) return LSA_ERR_INVALID_ARG;
+  } else if (!nsel || refresh_last_summary || (flags & LSA_FLAG_PDL)) {
     return LSA_ERR_INVALID_ARG;
   }
   lsa::DecodeArgs a = {};
   a.q = q; a.k = k; a.v = v; a.dtype = dtype;
   a.B = B; a.Hkv = Hkv; a.G = G; a.D = D; a.T_cap = T_cap; a.NB_cap = ceil_div(T_cap, blk);
-  a.seqlens = seqlens; a.summ = summ; a.idx_in = idx; a.nsel_in = nsel;
+  a.seqlens = seqlens; a.summ = summ; a.summ_w = refresh_last_summary ? summ : nullptr;
+  a.idx_in = idx; a.nsel_in = nsel;
   a.topk = topk; a.n_sink = n_sink; a.n_local = n_local;
   a.scale = resolve_scale(scale, D);
   a.idx_out = fused ? idx_out : nullptr;
   a.o = o; a.lse = lse;
   a.mode = fused ? lsa::MODE_FUSED : lsa::MODE_ATTEND;
+  a.pdl = (flags & LSA_FLAG_PDL) != 0;
   return cuda_status(lsa::launch_decode(a, stream));
 }
 

@@ -23,6 +23,7 @@ struct DecodeArgs {
   int B, Hkv, G, D, T_cap;
   const int32_t* seqlens;
   const float* summ;
+  float* summ_w;           // MODE_FUSED: refresh the last block's summary here, or NULL
   int NB_cap;
   const int32_t* idx_in;   // MODE_ATTEND
   const int32_t* nsel_in;  // MODE_ATTEND
@@ -34,6 +35,7 @@ struct DecodeArgs {
   void* o;                 // MODE_ATTEND / MODE_FUSED
   float* lse;              // optional
   int mode;
+  int pdl;                 // MODE_FUSED: launch with programmatic stream serialization
 };
 
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream);

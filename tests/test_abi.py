@@ -71,13 +71,19 @@ def test_select_and_decode_validation():
     assert sel(g, 1, g, 1, 8, 8, 128, 1024, g, 64, 65, 1, 2, 0.0, g, g, NULL, NULL) == lsa.LSA_ERR_INVALID_ARG
     assert sel(g, 1, g, 1, 8, 8, 128, 1024, g, 64, 2, 1, 2, 0.0, g, g, NULL, NULL) == lsa.LSA_ERR_INVALID_ARG
     assert sel(g, 1, g, 1, 8, 17, 128, 1024, g, 64, 16, 1, 2, 0.0, g, g, NULL, NULL) == lsa.LSA_ERR_UNSUPPORTED
-    assert sel(g, 1, g, 1, 8, 8, 128, 1024, g, 64, 16, 1, 2, 0.0, NULL, g, NULL, NULL) == lsa.LSA_ERR_INVALID_ARG
+    assert sel(g, 1, g, 1, 8, 8, 128, 1024, g, 64, 16, 1, 2, 0.0, NULL, g, NULL, 0, NULL) == lsa.LSA_ERR_INVALID_ARG
     dec = lib.lsa_sparse_attn_decode
     # fused mode (idx NULL) needs summaries; given mode needs nsel
-    assert dec(g, g, g, 1, 1, 8, 8, 128, 65536, g, 64, NULL, NULL, 16, 0.0, NULL, 1, 2, NULL, g, NULL, NULL) == lsa.LSA_ERR_INVALID_ARG
-    assert dec(g, g, g, 1, 1, 8, 8, 128, 65536, g, 64, g, NULL, 16, 0.0, NULL, 1, 2, NULL, g, NULL, NULL) == lsa.LSA_ERR_INVALID_ARG
-    assert dec(g, g, g, 1, 1, 8, 8, 128, 1 << 22, g, 64, g, g, 16, 0.0, NULL, 1, 2, NULL, g, NULL, NULL) == lsa.LSA_ERR_UNSUPPORTED
-    assert dec(g, g, NULL, 1, 1, 8, 8, 128, 65536, g, 64, g, g, 16, 0.0, NULL, 1, 2, NULL, g, NULL, NULL) == lsa.LSA_ERR_INVALID_ARG
+    assert dec(g, g, g, 1, 1, 8, 8, 128, 65536, g, 64, NULL, NULL, 16, 0.0, NULL, 1, 2, 0, NULL, g, NULL, 0, NULL) == lsa.LSA_ERR_INVALID_ARG
+    assert dec(g, g, g, 1, 1, 8, 8, 128, 65536, g, 64, g, NULL, 16, 0.0, NULL, 1, 2, 0, NULL, g, NULL, 0, NULL) == lsa.LSA_ERR_INVALID_ARG
+    assert dec(g, g, g, 1, 1, 8, 8, 128, 1 << 22, g, 64, g, g, 16, 0.0, NULL, 1, 2, 0, NULL, g, NULL, 0, NULL) == lsa.LSA_ERR_UNSUPPORTED
+    assert dec(g, g, NULL, 1, 1, 8, 8, 128, 65536, g, 64, g, g, 16, 0.0, NULL, 1, 2, 0, NULL, g, NULL, 0, NULL) == lsa.LSA_ERR_INVALID_ARG
+    # the refreshed last block must be forced (n_local >= 1), and only in fused mode
+    assert dec(g, g, g, 1, 1, 8, 8, 128, 65536, g, 64, NULL, NULL, 16, 0.0, g, 1, 0, 1, NULL, g, NULL, 0, NULL) == lsa.LSA_ERR_INVALID_ARG
+    assert dec(g, g, g, 1, 1, 8, 8, 128, 65536, g, 64, g, g, 16, 0.0, g, 1, 2, 1, NULL, g, NULL, 0, NULL) == lsa.LSA_ERR_INVALID_ARG
+    # overlapped launch only in fused mode; unknown flags rejected
+    assert dec(g, g, g, 1, 1, 8, 8, 128, 65536, g, 64, g, g, 16, 0.0, NULL, 1, 2, 0, NULL, g, NULL, 1, NULL) == lsa.LSA_ERR_INVALID_ARG
+    assert dec(g, g, g, 1, 1, 8, 8, 128, 65536, g, 64, NULL, NULL, 16, 0.0, g, 1, 2, 0, NULL, g, NULL, 2, NULL) == lsa.LSA_ERR_INVALID_ARG
 
 
 def test_binding_raises_lsa_error_on_bad_arguments():

@@ -139,13 +139,28 @@ def _run_both_modes(lsa, case, dtype, check_sel=True):
     lsa.lsa_sparse_attn_decode(q, k, v, sl, o, topk, idx=r["idx"].cuda(), nsel=r["nsel"].cuda(),
                                lse=lse)
     _check_attention(case, o, lse, r["idx"], dtype, "given")
-    # fused selection + attention
+    # fused selection + attention; when the last block is forced, also refresh its summary
+    # (poisoned first, so a refresh that did not happen or was read by the scan shows)
+    refresh = nl >= 1
+    summ_ref = oracle.summaries(case.k, case.seqlens)
+    if refresh:
+        for b in range(B):
+            NB = -(-int(case.seqlens[b]) // 64)
+            if NB:
+                summ[b, :, NB - 1] = float("nan")
     o2 = torch.empty_like(q)
     lse2 = torch.empty(B, Hkv * G, device="cuda")
     idx2 = torch.full((B, Hkv, topk), -7, device="cuda", dtype=torch.int32)
     lsa.lsa_sparse_attn_decode(q, k, v, sl, o2, topk, summ=summ, n_sink=ns, n_local=nl,
-                               idx_out=idx2, lse=lse2)
+                               refresh_last_summary=refresh, idx_out=idx2, lse=lse2)
     idx2c = idx2.cpu()
+    if refresh:
+        sc = summ.cpu()
+        for b in range(B):
+            NB = -(-int(case.seqlens[b]) // 64)
+            if NB:
+                assert max_abs(sc[b, :, NB - 1], summ_ref[b, :, NB - 1]) < 1e-5, "refresh"
+                assert max_abs(sc[b, :, :NB - 1], summ_ref[b, :, :NB - 1]) < 1e-5
     if check_sel:
         for b in range(B):
             NB = -(-int(case.seqlens[b]) // 64)
