@@ -184,15 +184,21 @@ LSA_API int lsa_sparse_attn_decode(const void* q, const void* k, const void* v, 
  * o_cache [B, Hq, Tq, D] bf16; lse_cache [B, Hq, Tq] float32; o, lse: same shapes, out.
  * union_idx [B, Hkv, NBp] int32 out or NULL (ascending, -1 padded);
  * union_cnt [B, Hkv] int32 out or NULL.
- * Requires 1 <= Tq <= 64, 1 <= topk_per_query <= 64.
+ * workspace: device scratch of at least lsa_blockquery_workspace_size(B, Hkv, G, D, Tq)
+ *     bytes (16-byte aligned, contents need no initialisation), for the per-CTA partial
+ *     results of the split over the union; calls that overlap on the GPU need their own.
+ * Requires bf16, 1 <= Tq <= 64, 1 <= topk_per_query <= 16, n_sink + n_local <=
+ * topk_per_query.
  */
+LSA_API size_t lsa_blockquery_workspace_size(int B, int Hkv, int G, int D, int Tq);
+
 LSA_API int lsa_sparse_attn_blockquery(const void* q, const void* k, const void* v, int dtype,
                                int B, int Hkv, int G, int D, int Tq, int T_prefix,
                                int T_cap, const float* summ, int blk, int topk_per_query,
                                int n_sink, int n_local, float scale, const uint8_t* active,
                                const void* o_cache, const float* lse_cache, void* o,
                                float* lse, int32_t* union_idx, int32_t* union_cnt,
-                               cudaStream_t stream);
+                               void* workspace, size_t ws_bytes, cudaStream_t stream);
 
 /*
  * lsa_blasst_prefill -- causal softmax attention that skips whole KV tiles whose

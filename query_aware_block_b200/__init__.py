@@ -4,7 +4,7 @@ The functions carry the names of the C ABI in include/lsa.h and only marshal arg
 shapes are read from the torch tensors, pointers and the current CUDA stream are passed
 through ctypes, and a non-zero status raises LsaError.  Every step of the computation runs
 in the library's CUDA kernels; there is no fallback of any kind.  If liblsa.so has not been
-built (``python -m query_aware_block_b200._build``), importing this package raises.
+built (``python query_aware_block_b200/_build.py``), importing this package raises.
 """
 from __future__ import annotations
 
@@ -17,7 +17,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "liblsa.so")
 
 if not os.path.exists(LIB_PATH):
-    raise ImportError(f"{LIB_PATH} is missing: build it with `python -m query_aware_block_b200._build`")
+    raise ImportError(f"{LIB_PATH} is missing: build it with `python query_aware_block_b200/_build.py`")
 
 _lib = ctypes.CDLL(LIB_PATH)
 
@@ -27,8 +27,8 @@ LSA_FLAG_PDL = 1
 BLK = 64
 
 EXPORTED = ("lsa_status_string", "lsa_last_cuda_error", "lsa_version", "lsa_build_summaries",
-            "lsa_select_blocks", "lsa_sparse_attn_decode", "lsa_sparse_attn_blockquery",
-            "lsa_blasst_prefill")
+            "lsa_select_blocks", "lsa_sparse_attn_decode", "lsa_blockquery_workspace_size",
+            "lsa_sparse_attn_blockquery", "lsa_blasst_prefill")
 
 _vp, _i, _f = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
 _lib.lsa_status_string.restype = ctypes.c_char_p
@@ -40,13 +40,16 @@ _lib.lsa_select_blocks.argtypes = [_vp, _i, _vp, _i, _i, _i, _i, _i, _vp, _i, _i
                                    _vp, _vp, _vp, _vp]
 _lib.lsa_sparse_attn_decode.argtypes = [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp, _i, _vp, _vp,
                                         _i, _f, _vp, _i, _i, _i, _vp, _vp, _vp, _i, _vp]
+_lib.lsa_blockquery_workspace_size.argtypes = [_i, _i, _i, _i, _i]
+_lib.lsa_blockquery_workspace_size.restype = ctypes.c_size_t
 _lib.lsa_sparse_attn_blockquery.argtypes = [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _vp,
                                             _i, _i, _i, _i, _f, _vp, _vp, _vp, _vp, _vp, _vp,
-                                            _vp, _vp]
+                                            _vp, _vp, _vp, ctypes.c_size_t, _vp]
 _lib.lsa_blasst_prefill.argtypes = [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _f, _vp, _vp, _vp,
                                     _vp, _vp]
 for _n in EXPORTED[3:]:
-    getattr(_lib, _n).restype = _i
+    if _n != "lsa_blockquery_workspace_size":
+        getattr(_lib, _n).restype = _i
 
 
 class LsaError(RuntimeError):
@@ -127,10 +130,16 @@ def lsa_sparse_attn_decode(q, k, v, seqlens, o, topk, idx=None, nsel=None, summ=
     return o
 
 
+def lsa_blockquery_workspace_size(B, Hkv, G, D, Tq) -> int:
+    return int(_lib.lsa_blockquery_workspace_size(B, Hkv, G, D, Tq))
+
+
 def lsa_sparse_attn_blockquery(q, k, v, summ, T_prefix, topk_per_query, active, o_cache,
-                               lse_cache, o, lse, n_sink=0, n_local=0, union_idx=None,
-                               union_cnt=None, scale=0.0, blk=BLK, stream=None):
-    """Block-query step: q [B,Hq,Tq,D] against the prefix of k, v [B,Hkv,T_cap,D]."""
+                               lse_cache, o, lse, workspace, n_sink=0, n_local=0,
+                               union_idx=None, union_cnt=None, scale=0.0, blk=BLK,
+                               stream=None):
+    """Block-query step: q [B,Hq,Tq,D] against the prefix of k, v [B,Hkv,T_cap,D].
+    workspace: a device buffer of at least lsa_blockquery_workspace_size(...) bytes."""
     B, Hq, Tq, D = q.shape
     _, Hkv, T_cap, _ = k.shape
     _check(_lib.lsa_sparse_attn_blockquery(_ptr(q), _ptr(k), _ptr(v), _dtype(q), B, Hkv,
@@ -138,6 +147,8 @@ def lsa_sparse_attn_blockquery(q, k, v, summ, T_prefix, topk_per_query, active, 
                                            topk_per_query, n_sink, n_local, float(scale),
                                            _ptr(active), _ptr(o_cache), _ptr(lse_cache),
                                            _ptr(o), _ptr(lse), _ptr(union_idx), _ptr(union_cnt),
+                                           _ptr(workspace),
+                                           workspace.numel() * workspace.element_size(),
                                            _stream(stream)),
            "lsa_sparse_attn_blockquery")
     return o, lse

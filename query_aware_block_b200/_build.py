@@ -1,6 +1,9 @@
 """Build liblsa.so in-tree with nvcc for sm_100a (B200).
 
-    python -m query_aware_block_b200._build [--verbose-ptxas] [--force]
+    python query_aware_block_b200/_build.py [--verbose-ptxas] [--force]
+
+Run it as a script (or load it by path, as __graft_entry__.build() does): importing the
+package itself loads liblsa.so, which is what this script produces.
 
 Every .cu file under csrc/ is compiled to an object in _build/ (parallel nvcc processes),
 then linked into query_aware_block_b200/liblsa.so with a static CUDA runtime.  Only the

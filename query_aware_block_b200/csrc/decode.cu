@@ -37,6 +37,7 @@
 // No global scratch memory and no spin-waits: cross-CTA ordering uses cluster barriers.
 #include <math.h>
 
+#include "cluster.cuh"
 #include "lsa_common.cuh"
 #include "lsa_internal.h"
 
@@ -76,50 +77,6 @@ struct Params {
   int lp;                 // length of an exchanged candidate list: max(16, m_pad)
   int chunk;              // output elements merged by one CTA (even)
 };
-
-// ---- cluster primitives (PTX ISA: barrier.cluster, mapa, st.shared::cluster) ----------
-__device__ __forceinline__ int cluster_rank() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-  return (int)r;
-}
-__device__ __forceinline__ int cluster_size() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(r));
-  return (int)r;
-}
-__device__ __forceinline__ void cluster_arrive_relaxed() {
-  asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
-}
-__device__ __forceinline__ void cluster_arrive_release() {
-  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
-}
-__device__ __forceinline__ void cluster_wait() {
-  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
-__device__ __forceinline__ uint32_t map_rank(const void* p, int r) {
-  const uint32_t a = (uint32_t)__cvta_generic_to_shared(p);
-  uint32_t out;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(out) : "r"(a), "r"(r));
-  return out;
-}
-__device__ __forceinline__ void st_cluster(uint32_t addr, u64 v) {
-  asm volatile("st.shared::cluster.u64 [%0], %1;" ::"r"(addr), "l"(v) : "memory");
-}
-__device__ __forceinline__ void st_cluster(uint32_t addr, float2 v) {
-  asm volatile("st.shared::cluster.v2.f32 [%0], {%1, %2};" ::"r"(addr), "f"(v.x), "f"(v.y)
-               : "memory");
-}
-__device__ __forceinline__ void st_cluster(uint32_t addr, float v) {
-  asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
-}
-
-// Programmatic dependent launch (PTX griddepcontrol): with the launch attribute set, the
-// grid may start while the previous kernel of the stream still runs; `wait` blocks until
-// that kernel has completed and its memory is visible.  Without the attribute both are
-// no-ops in effect.
-__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
-__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
 __host__ __device__ inline size_t align128(size_t x) { return (x + 127) & ~(size_t)127; }
 
@@ -186,36 +143,6 @@ __device__ void block_topm(const u64* keys, int n, int m, u64* top, u64* work) {
   __syncthreads();
 }
 
-// Bitonic merge, descending, of the 32E-long sequence held by a warp (lane l holds
-// positions l*E .. l*E+E-1): positions [0, 16E) are a descending list and [16E, 32E) a
-// list in ascending order, so the whole is bitonic.  Afterwards the sequence is sorted
-// descending; the top 16E keys sit in lanes 0..15.
-template <int E>
-__device__ __forceinline__ void warp_merge_desc(u64 (&x)[E]) {
-  const int lane = threadIdx.x & 31;
-#pragma unroll
-  for (int dist = 16 * E; dist >= 1; dist >>= 1) {
-    if (dist >= E) {
-      const int ld = dist / E;
-      const bool lower = (lane & ld) == 0;
-#pragma unroll
-      for (int e = 0; e < E; ++e) {
-        const u64 y = __shfl_xor_sync(0xffffffffu, x[e], ld);
-        x[e] = lower ? (x[e] > y ? x[e] : y) : (x[e] < y ? x[e] : y);
-      }
-    } else {
-#pragma unroll
-      for (int e = 0; e < E; ++e) {
-        if ((e & dist) == 0) {
-          const u64 a = x[e], b = x[e ^ dist];
-          x[e] = a > b ? a : b;
-          x[e ^ dist] = a > b ? b : a;
-        }
-      }
-    }
-  }
-}
-
 // Top list of the union of CL descending lists of 16E keys (zero padded) stored at
 // lists[c * 16E]: pairs are merged one warp each, level by level, ping-ponging between
 // `lists` and `work`.  Returns the buffer that holds the final list.
@@ -273,32 +200,6 @@ __device__ __forceinline__ void load_f32(const T* p, float (&out)[N]) {
       const __nv_bfloat162 a = *reinterpret_cast<const __nv_bfloat162*>(&v);
       out[0] = __low2float(a); out[1] = __high2float(a);
     }
-  }
-}
-
-// ---- K/V block staging ----------------------------------------------------------------
-
-// Copy the K and V rows of block j into a stage (rows >= Tb, and every row of an invalid
-// j < 0, are zero-filled and never read from global memory).  bf16 rows are
-// chunk-swizzled; fp32 rows are padded by 16 bytes.
-template <typename T, int D>
-__device__ __forceinline__ void stage_block(unsigned char* dst_k, unsigned char* dst_v,
-                                            const T* kbase, const T* vbase, int j, int Tb,
-                                            int kv_row) {
-  constexpr int kChunks = D * (int)sizeof(T) / 16;  // 16-byte chunks per row
-  constexpr int kTotal = 2 * kBlk * kChunks;
-  constexpr bool kF32 = sizeof(T) == 4;
-#pragma unroll
-  for (int it = 0; it < kTotal / kThreads; ++it) {
-    const int id = threadIdx.x + it * kThreads;
-    const int tensor = id / (kBlk * kChunks);
-    const int rem = id % (kBlk * kChunks);
-    const int row = rem / kChunks, c = rem % kChunks;
-    const int t = j * kBlk + row;
-    const bool valid = j >= 0 && t < Tb;
-    const T* src = (tensor ? vbase : kbase) + (size_t)(valid ? t : 0) * D + c * (16 / sizeof(T));
-    unsigned char* dst = (tensor ? dst_v : dst_k) + (kF32 ? row * kv_row + c * 16 : swz(row, c, kv_row));
-    cp_async16(dst, src, valid);
   }
 }
 
@@ -371,7 +272,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_cluster_kernel(const Param
   if (MODE == MODE_FUSED) {
     while (issued < kStages && issued < n_known && known_block(issued) != NB - 1) {
       unsigned char* st = kv + (size_t)(issued % kStages) * 2 * kv_tile;
-      stage_block<T, D>(st, st + kv_tile, kbase, vbase, known_block(issued), Tb, kv_row);
+      stage_block<T, D, kThreads>(st, st + kv_tile, kbase, vbase, known_block(issued), Tb, kv_row);
       cp_async_commit();
       ++issued;
     }
@@ -412,7 +313,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_cluster_kernel(const Param
   if (MODE == MODE_FUSED) {
     while (issued < kStages && issued < n_known) {
       unsigned char* st = kv + (size_t)(issued % kStages) * 2 * kv_tile;
-      stage_block<T, D>(st, st + kv_tile, kbase, vbase, known_block(issued), Tb, kv_row);
+      stage_block<T, D, kThreads>(st, st + kv_tile, kbase, vbase, known_block(issued), Tb, kv_row);
       cp_async_commit();
       ++issued;
     }
@@ -514,7 +415,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_cluster_kernel(const Param
   const int n_my = n_order > rank ? (n_order - rank + CL - 1) / CL : 0;
   while (issued < kStages && issued < n_my) {
     unsigned char* st = kv + (size_t)(issued % kStages) * 2 * kv_tile;
-    stage_block<T, D>(st, st + kv_tile, kbase, vbase, order[rank + issued * CL], Tb, kv_row);
+    stage_block<T, D, kThreads>(st, st + kv_tile, kbase, vbase, order[rank + issued * CL], Tb, kv_row);
     cp_async_commit();
     ++issued;
   }
@@ -673,7 +574,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_cluster_kernel(const Param
     __syncthreads();  // the stage may now be refilled
     if (issued < n_my) {
       unsigned char* st = kv + (size_t)(issued % kStages) * 2 * kv_tile;
-      stage_block<T, D>(st, st + kv_tile, kbase, vbase, order[rank + issued * CL], Tb, kv_row);
+      stage_block<T, D, kThreads>(st, st + kv_tile, kbase, vbase, order[rank + issued * CL], Tb, kv_row);
       cp_async_commit();
       ++issued;
     }

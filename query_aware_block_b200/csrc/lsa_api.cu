@@ -136,18 +136,41 @@ int lsa_sparse_attn_decode(const void* q, const void* k, const void* v, int dtyp
   return cuda_status(lsa::launch_decode(a, stream));
 }
 
+size_t lsa_blockquery_workspace_size(int B, int Hkv, int G, int D, int Tq) {
+  if (B <= 0 || Hkv <= 0 || G <= 0 || D <= 0 || Tq <= 0) return 0;
+  return lsa::blockquery_workspace_bytes(B, Hkv, G, D, Tq);
+}
+
 int lsa_sparse_attn_blockquery(const void* q, const void* k, const void* v, int dtype,
                                int B, int Hkv, int G, int D, int Tq, int T_prefix,
                                int T_cap, const float* summ, int blk, int topk_per_query,
                                int n_sink, int n_local, float scale, const uint8_t* active,
                                const void* o_cache, const float* lse_cache, void* o,
                                float* lse, int32_t* union_idx, int32_t* union_cnt,
-                               cudaStream_t stream) {
-  (void)q; (void)k; (void)v; (void)dtype; (void)B; (void)Hkv; (void)G; (void)D; (void)Tq;
-  (void)T_prefix; (void)T_cap; (void)summ; (void)blk; (void)topk_per_query; (void)n_sink;
-  (void)n_local; (void)scale; (void)active; (void)o_cache; (void)lse_cache; (void)o;
-  (void)lse; (void)union_idx; (void)union_cnt; (void)stream;
-  return LSA_ERR_UNSUPPORTED;
+                               void* workspace, size_t ws_bytes, cudaStream_t stream) {
+  int st = check_common(dtype, B, Hkv, G, D, blk);
+  if (st != LSA_OK) return st;
+  if (dtype != LSA_BF16) return LSA_ERR_UNSUPPORTED;
+  if (Tq < 1 || Tq > 64 || T_prefix < 0 || T_cap < T_prefix) return LSA_ERR_INVALID_ARG;
+  if (T_cap > kMaxTcap) return LSA_ERR_UNSUPPORTED;
+  if (topk_per_query < 1 || topk_per_query > 16 || n_sink < 0 || n_local < 0 ||
+      n_sink + n_local > topk_per_query)
+    return LSA_ERR_INVALID_ARG;
+  if (B == 0 || Hkv == 0) return LSA_OK;
+  if (!q || !k || !v || !summ || !active || !o_cache || !lse_cache || !o || !lse || !workspace)
+    return LSA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(summ) || !aligned16(o) ||
+      !aligned16(o_cache) || !aligned16(workspace))
+    return LSA_ERR_INVALID_ARG;
+  if (ws_bytes < lsa::blockquery_workspace_bytes(B, Hkv, G, D, Tq)) return LSA_ERR_INVALID_ARG;
+  lsa::BlockQueryArgs a = {};
+  a.q = q; a.k = k; a.v = v;
+  a.B = B; a.Hkv = Hkv; a.G = G; a.D = D; a.Tq = Tq; a.T_prefix = T_prefix; a.T_cap = T_cap;
+  a.summ = summ; a.topk = topk_per_query; a.n_sink = n_sink; a.n_local = n_local;
+  a.scale = resolve_scale(scale, D);
+  a.active = active; a.o_cache = o_cache; a.lse_cache = lse_cache; a.o = o; a.lse = lse;
+  a.union_idx = union_idx; a.union_cnt = union_cnt; a.workspace = workspace;
+  return cuda_status(lsa::launch_blockquery(a, stream));
 }
 
 int lsa_blasst_prefill(const void* q, const void* k, const void* v, int dtype, int B, int Hq,

@@ -110,4 +110,30 @@ __device__ __forceinline__ int swz(int r, int c, int row_bytes) {
   return r * row_bytes + ((c ^ (r & 7)) << 4);
 }
 
+// ---- K/V block staging ----------------------------------------------------------------
+
+// Copy the K and V rows of block j (64 tokens) into a stage with 16-byte cp.async: rows
+// >= Tb, and every row of an invalid j < 0, are zero-filled and never read from global
+// memory.  bf16 rows are chunk-swizzled; fp32 rows are padded by 16 bytes.
+template <typename T, int D, int kThreads>
+__device__ __forceinline__ void stage_block(unsigned char* dst_k, unsigned char* dst_v,
+                                            const T* kbase, const T* vbase, int j, int Tb,
+                                            int kv_row) {
+  constexpr int kChunks = D * (int)sizeof(T) / 16;  // 16-byte chunks per row
+  constexpr int kTotal = 2 * kBlk * kChunks;
+  constexpr bool kF32 = sizeof(T) == 4;
+#pragma unroll
+  for (int it = 0; it < kTotal / kThreads; ++it) {
+    const int id = threadIdx.x + it * kThreads;
+    const int tensor = id / (kBlk * kChunks);
+    const int rem = id % (kBlk * kChunks);
+    const int row = rem / kChunks, c = rem % kChunks;
+    const int t = j * kBlk + row;
+    const bool valid = j >= 0 && t < Tb;
+    const T* src = (tensor ? vbase : kbase) + (size_t)(valid ? t : 0) * D + c * (16 / sizeof(T));
+    unsigned char* dst = (tensor ? dst_v : dst_k) + (kF32 ? row * kv_row + c * 16 : swz(row, c, kv_row));
+    cp_async16(dst, src, valid);
+  }
+}
+
 }  // namespace lsa

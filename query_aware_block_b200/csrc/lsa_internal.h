@@ -40,4 +40,26 @@ struct DecodeArgs {
 
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream);
 
+// The block-query step: one cluster per (sequence, KV head); partials in a workspace.
+struct BlockQueryArgs {
+  const void* q;
+  const void* k;
+  const void* v;
+  int B, Hkv, G, D, Tq, T_prefix, T_cap;
+  const float* summ;
+  int topk, n_sink, n_local;
+  float scale;
+  const uint8_t* active;
+  const void* o_cache;
+  const float* lse_cache;
+  void* o;
+  float* lse;
+  int32_t* union_idx;
+  int32_t* union_cnt;
+  void* workspace;
+};
+
+size_t blockquery_workspace_bytes(int B, int Hkv, int G, int D, int Tq);
+cudaError_t launch_blockquery(const BlockQueryArgs& a, cudaStream_t stream);
+
 }  // namespace lsa
