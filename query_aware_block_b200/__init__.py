@@ -34,7 +34,9 @@ _vp, _i, _f = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
 _lib.lsa_status_string.restype = ctypes.c_char_p
 _lib.lsa_status_string.argtypes = [_i]
 _lib.lsa_last_cuda_error.restype = _i
+_lib.lsa_last_cuda_error.argtypes = []
 _lib.lsa_version.restype = _i
+_lib.lsa_version.argtypes = []
 _lib.lsa_build_summaries.argtypes = [_vp, _i, _i, _i, _i, _i, _vp, _i, _i, _i, _vp, _vp]
 _lib.lsa_select_blocks.argtypes = [_vp, _i, _vp, _i, _i, _i, _i, _i, _vp, _i, _i, _i, _i, _f,
                                    _vp, _vp, _vp, _vp]
@@ -44,7 +46,7 @@ _lib.lsa_blockquery_workspace_size.argtypes = [_i, _i, _i, _i, _i]
 _lib.lsa_blockquery_workspace_size.restype = ctypes.c_size_t
 _lib.lsa_sparse_attn_blockquery.argtypes = [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _vp,
                                             _i, _i, _i, _i, _f, _vp, _vp, _vp, _vp, _vp, _vp,
-                                            _vp, _vp, _vp, ctypes.c_size_t, _vp]
+                                            _vp, _vp, ctypes.c_size_t, _vp]
 _lib.lsa_blasst_prefill.argtypes = [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _f, _vp, _vp, _vp,
                                     _vp, _vp]
 for _n in EXPORTED[3:]:

@@ -93,3 +93,16 @@ def test_binding_raises_lsa_error_on_bad_arguments():
     with pytest.raises(lsa.LsaError) as e:
         lsa.lsa_build_summaries(k, torch.zeros(1, dtype=torch.int32), torch.zeros(1, 1, 1, 96), stream=0)
     assert e.value.status == lsa.LSA_ERR_UNSUPPORTED
+
+
+def test_binding_argtypes_match_header_parameter_counts():
+    # every ctypes prototype has exactly as many arguments as the C declaration
+    import query_aware_block_b200 as lsa
+    text = open(HEADER).read()
+    lib = lsa.library()
+    for name in _declared():
+        m = re.search(r"\b" + name + r"\s*\(([^)]*)\)", text)
+        params = m.group(1).strip()
+        n = 0 if params in ("", "void") else len(params.split(","))
+        argt = getattr(lib, name).argtypes
+        assert argt is not None and len(argt) == n, (name, n, argt and len(argt))
