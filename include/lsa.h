@@ -201,6 +201,35 @@ LSA_API int lsa_sparse_attn_blockquery(const void* q, const void* k, const void*
                                void* workspace, size_t ws_bytes, cudaStream_t stream);
 
 /*
+ * lsa_sparse_attn_blockquery_noalloc -- lsa_sparse_attn_blockquery for callers that may
+ * not allocate device memory at all (nothing of theirs may call cudaMalloc, for example
+ * code that runs where allocation is not allowed or must keep a fixed memory footprint).
+ *
+ * The pages have no counterpart of this entry point: it only changes where the scratch
+ * of the block-query split lives.  Arguments, outputs and errors are those of
+ * lsa_sparse_attn_blockquery without the workspace: the library uses one fixed device
+ * array of 16 MiB instead, which every GPU that loads the library holds until the
+ * process exits.  It allocates nothing and calls no allocating routine.
+ *   - Shapes whose lsa_blockquery_workspace_size(B, Hkv, G, D, Tq) exceeds 16 MiB are
+ *     rejected with LSA_ERR_UNSUPPORTED.
+ *   - All calls share the array: calls that overlap on the GPU (different streams or host
+ *     threads) race and must be serialised by the caller.  Its contents are left from the
+ *     previous call; none of them needs to start at zero.
+ *   - The first call on each device looks the array's device address up (the host-side
+ *     name of a __device__ array is not a device address) and caches it; make that first
+ *     call before any stream capture.
+ */
+LSA_API int lsa_sparse_attn_blockquery_noalloc(const void* q, const void* k, const void* v,
+                                               int dtype, int B, int Hkv, int G, int D,
+                                               int Tq, int T_prefix, int T_cap,
+                                               const float* summ, int blk, int topk_per_query,
+                                               int n_sink, int n_local, float scale,
+                                               const uint8_t* active, const void* o_cache,
+                                               const float* lse_cache, void* o, float* lse,
+                                               int32_t* union_idx, int32_t* union_cnt,
+                                               cudaStream_t stream);
+
+/*
  * lsa_blasst_prefill -- causal softmax attention that skips whole KV tiles whose
  * softmax weight is negligible (BLASST).
  *

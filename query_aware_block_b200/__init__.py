@@ -28,7 +28,8 @@ BLK = 64
 
 EXPORTED = ("lsa_status_string", "lsa_last_cuda_error", "lsa_version", "lsa_build_summaries",
             "lsa_select_blocks", "lsa_sparse_attn_decode", "lsa_blockquery_workspace_size",
-            "lsa_sparse_attn_blockquery", "lsa_blasst_prefill")
+            "lsa_sparse_attn_blockquery", "lsa_sparse_attn_blockquery_noalloc",
+            "lsa_blasst_prefill")
 
 _vp, _i, _f = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
 _lib.lsa_status_string.restype = ctypes.c_char_p
@@ -47,6 +48,9 @@ _lib.lsa_blockquery_workspace_size.restype = ctypes.c_size_t
 _lib.lsa_sparse_attn_blockquery.argtypes = [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _vp,
                                             _i, _i, _i, _i, _f, _vp, _vp, _vp, _vp, _vp, _vp,
                                             _vp, _vp, ctypes.c_size_t, _vp]
+_lib.lsa_sparse_attn_blockquery_noalloc.argtypes = [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i,
+                                                    _i, _vp, _i, _i, _i, _i, _f, _vp, _vp, _vp,
+                                                    _vp, _vp, _vp, _vp, _vp]
 _lib.lsa_blasst_prefill.argtypes = [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _f, _vp, _vp, _vp,
                                     _vp, _vp]
 for _n in EXPORTED[3:]:

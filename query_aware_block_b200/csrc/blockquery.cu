@@ -28,6 +28,8 @@
 //     CTAs exchange over DSMEM.
 #include <math.h>
 
+#include <mutex>
+
 #include "cluster.cuh"
 #include "lsa_common.cuh"
 #include "lsa_internal.h"
@@ -608,6 +610,45 @@ cudaError_t launch_blockquery(const BlockQueryArgs& a, cudaStream_t stream) {
     }
     return cudaLaunchKernelEx(&cfg, kernel, p);
   }
+}
+
+
+// ---- fixed scratch for callers that cannot allocate device memory -----------------------
+// Some callers may not allocate device memory at all (for instance code that runs where
+// allocation is forbidden or must not change the memory footprint).  For them the
+// block-query partials live in one statically sized device array instead of a caller
+// workspace.  The array exists once per GPU that loads this library and stays allocated
+// until the process exits; every call shares it, so calls that overlap on the GPU (other
+// streams, or other host threads) race on its contents.  Nothing in it has to start at
+// zero: each call writes every partial it reads back.
+constexpr size_t kStaticWorkspaceBytes = (size_t)16 << 20;  // 16 MiB
+static __device__ __align__(256) unsigned char g_blockquery_scratch[kStaticWorkspaceBytes];
+
+namespace {
+constexpr int kMaxDevices = 64;
+std::mutex g_scratch_mutex;
+void* g_scratch_ptr[kMaxDevices] = {};
+}  // namespace
+
+size_t blockquery_static_workspace_bytes() { return kStaticWorkspaceBytes; }
+
+// Device address of the fixed scratch on the current device.  The first call on a device
+// looks it up with cudaGetSymbolAddress (the host-side name of the array is not a device
+// address); later calls reuse the cached pointer.
+cudaError_t blockquery_static_workspace(void** ptr) {
+  int dev = 0;
+  cudaError_t err = cudaGetDevice(&dev);
+  if (err != cudaSuccess) return err;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(g_scratch_mutex);
+  if (g_scratch_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    err = cudaGetSymbolAddress(&p, g_blockquery_scratch);
+    if (err != cudaSuccess) return err;
+    g_scratch_ptr[dev] = p;
+  }
+  *ptr = g_scratch_ptr[dev];
+  return cudaSuccess;
 }
 
 }  // namespace lsa

@@ -173,6 +173,26 @@ int lsa_sparse_attn_blockquery(const void* q, const void* k, const void* v, int 
   return cuda_status(lsa::launch_blockquery(a, stream));
 }
 
+int lsa_sparse_attn_blockquery_noalloc(const void* q, const void* k, const void* v, int dtype,
+                                       int B, int Hkv, int G, int D, int Tq, int T_prefix,
+                                       int T_cap, const float* summ, int blk,
+                                       int topk_per_query, int n_sink, int n_local,
+                                       float scale, const uint8_t* active,
+                                       const void* o_cache, const float* lse_cache, void* o,
+                                       float* lse, int32_t* union_idx, int32_t* union_cnt,
+                                       cudaStream_t stream) {
+  if (B > 0 && Hkv > 0 && G > 0 && D > 0 && Tq > 0 &&
+      lsa::blockquery_workspace_bytes(B, Hkv, G, D, Tq) > lsa::blockquery_static_workspace_bytes())
+    return LSA_ERR_UNSUPPORTED;  // larger than the fixed scratch: use the workspace variant
+  void* ws = nullptr;
+  const cudaError_t err = lsa::blockquery_static_workspace(&ws);
+  if (err != cudaSuccess) return cuda_status(err);
+  return lsa_sparse_attn_blockquery(q, k, v, dtype, B, Hkv, G, D, Tq, T_prefix, T_cap, summ,
+                                    blk, topk_per_query, n_sink, n_local, scale, active,
+                                    o_cache, lse_cache, o, lse, union_idx, union_cnt, ws,
+                                    lsa::blockquery_static_workspace_bytes(), stream);
+}
+
 int lsa_blasst_prefill(const void* q, const void* k, const void* v, int dtype, int B, int Hq,
                        int Hkv, int L, int D, float scale, float lambda, void* o, float* lse,
                        uint32_t* skip_bits, unsigned long long* skipped_tiles,

@@ -62,4 +62,8 @@ struct BlockQueryArgs {
 size_t blockquery_workspace_bytes(int B, int Hkv, int G, int D, int Tq);
 cudaError_t launch_blockquery(const BlockQueryArgs& a, cudaStream_t stream);
 
+// The fixed device scratch used by lsa_sparse_attn_blockquery_noalloc.
+size_t blockquery_static_workspace_bytes();
+cudaError_t blockquery_static_workspace(void** ptr);
+
 }  // namespace lsa
