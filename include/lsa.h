@@ -252,12 +252,22 @@ LSA_API int lsa_sparse_attn_blockquery_noalloc(const void* q, const void* k, con
  *     (b, h, a) row is set iff tile c was skipped;
  * skipped_tiles: one uint64 counter or NULL, incremented by the number of skipped tiles
  *     (the caller zeroes it).
- * Requires D == 128, Hq % Hkv == 0, L >= 1.
+ * Requires bf16, D == 128, Hq % Hkv == 0, 0 <= lambda < 1.
+ * Every wait of the kernel on its own pipeline is bounded in time; should one ever run
+ * out, the kernel stops cleanly and lsa_device_status() reports LSA_DEVICE_TIMEOUT.
  */
 LSA_API int lsa_blasst_prefill(const void* q, const void* k, const void* v, int dtype, int B, int Hq,
                        int Hkv, int L, int D, float scale, float lambda, void* o, float* lse,
                        uint32_t* skip_bits, unsigned long long* skipped_tiles,
                        cudaStream_t stream);
+
+/*
+ * lsa_device_status -- the device-side status word the kernels set when a bounded wait
+ * runs out (LSA_DEVICE_TIMEOUT), 0 otherwise.  Synchronises with the device (it is a
+ * debugging and failure-detection aid, not for the hot loop).  reset != 0 clears it.
+ */
+#define LSA_DEVICE_TIMEOUT 1
+LSA_API int lsa_device_status(int* status, int reset);
 
 #ifdef __cplusplus
 }

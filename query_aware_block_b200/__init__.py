@@ -29,7 +29,7 @@ BLK = 64
 EXPORTED = ("lsa_status_string", "lsa_last_cuda_error", "lsa_version", "lsa_build_summaries",
             "lsa_select_blocks", "lsa_sparse_attn_decode", "lsa_blockquery_workspace_size",
             "lsa_sparse_attn_blockquery", "lsa_sparse_attn_blockquery_noalloc",
-            "lsa_blasst_prefill")
+            "lsa_blasst_prefill", "lsa_device_status")
 
 _vp, _i, _f = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
 _lib.lsa_status_string.restype = ctypes.c_char_p
@@ -53,6 +53,7 @@ _lib.lsa_sparse_attn_blockquery_noalloc.argtypes = [_vp, _vp, _vp, _i, _i, _i, _
                                                     _vp, _vp, _vp, _vp, _vp]
 _lib.lsa_blasst_prefill.argtypes = [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _f, _vp, _vp, _vp,
                                     _vp, _vp]
+_lib.lsa_device_status.argtypes = [_vp, _i]
 for _n in EXPORTED[3:]:
     if _n != "lsa_blockquery_workspace_size":
         getattr(_lib, _n).restype = _i
@@ -170,3 +171,13 @@ def lsa_blasst_prefill(q, k, v, o, lam, lse=None, skip_bits=None, skipped_tiles=
                                    _ptr(skipped_tiles), _stream(stream)),
            "lsa_blasst_prefill")
     return o
+
+
+def lsa_device_status(reset=False) -> int:
+    """The device status word (0, or LSA_DEVICE_TIMEOUT after a bounded wait ran out)."""
+    out = ctypes.c_int(0)
+    _check(_lib.lsa_device_status(ctypes.byref(out), int(bool(reset))), "lsa_device_status")
+    return out.value
+
+
+LSA_DEVICE_TIMEOUT = 1

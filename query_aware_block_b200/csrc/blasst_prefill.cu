@@ -1,0 +1,416 @@
+// blasst_prefill.cu -- causal prefill that skips whole KV tiles by a softmax threshold
+// (BLASST), on the sm_100a tensor cores (tcgen05, accumulators in tensor memory).
+//
+// What is computed (BLASST, "2. 방법론": "핵심 아이디어: 온라인 Softmax 통계 활용",
+// "알고리즘 및 커널 설계"): for each query head and 128-row query tile, the 64-key KV tiles
+// up to the causal diagonal are visited in ascending order with an online softmax; a tile
+// is skipped -- no exponentials, no P.V product -- when every row's tile maximum trails its
+// running maximum by more than -ln(lambda):  max_i (r_i - m_i) < ln(lambda).
+//
+// How (B200): one CTA per (b, h, query tile), heaviest tiles first; 8 warps.
+//   warp 0    TMA producer: Q once (2 boxes of 128 x 64 bf16, 128-byte swizzle), then K and
+//             V tiles into a 4-stage shared-memory ring (3-D tensor maps, no multicast).
+//   warp 1    MMA issuer (one thread): S_j = Q K_j^T (M 128, N 64, K 128) into a
+//             double-buffered TMEM tile; O += P_j V_j (M 128, N 128, K 64) with P read from
+//             tensor memory; tcgen05.commit signals S ready, O updated, stage free.
+//   warp 2    allocates / frees 256 TMEM columns: S0 [0,64), S1 [64,128), O [128,256).
+//   warps 4-7 softmax: thread = query row = TMEM lane.  Loads its S row, masks, takes the
+//             row max, votes on the skip with one bar.red.and over the 128 rows, writes
+//             P (bf16) back over its S columns, rescales its O row only when its running
+//             max grew by more than 2^8 since the exponent base was last set (exact: the
+//             final normalisation uses the same base), and stores o and lse at the end.
+// The MMA for S_{j+2} is issued as soon as P_j is consumed, so Q K^T of the next tiles
+// overlaps the softmax of the current one.  Every mbarrier wait is clock-bounded; a
+// timeout raises a CTA-wide abort, every role leaves its loop, the TMEM is freed and the
+// device status word records the failure.
+#include <cuda.h>
+#include <math.h>
+#include <string.h>
+
+#include "lsa_common.cuh"
+#include "lsa_internal.h"
+#include "tcgen05.cuh"
+
+namespace lsa {
+
+// 0 = no error; LSA_DEVICE_TIMEOUT when a bounded wait of a kernel ran out.
+__device__ int g_device_status = 0;
+
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kBM = 128;          // query rows per tile
+constexpr int kBN = 64;           // keys per KV tile
+constexpr int kD = 128;           // head dim
+constexpr int kStages = 4;
+constexpr uint32_t kTmemCols = 256;
+constexpr uint32_t kColO = 128;
+constexpr int kQBytes = kBM * kD * 2;        // 32 KB
+constexpr int kKVTileBytes = kBN * kD * 2;   // 16 KB per tensor
+constexpr int kStageBytes = 2 * kKVTileBytes;
+constexpr long long kWaitBudget = 4000000000LL;  // clock cycles (about 2 s)
+constexpr float kRescaleLog2 = 8.0f;             // rescale O when the max grew by > 2^8
+constexpr int kDeviceTimeout = 1;
+
+struct alignas(64) PrefillParams {
+  CUtensorMap tq;  // [B*Hq][L][D]
+  CUtensorMap tk;  // [B*Hkv][L][D]
+  CUtensorMap tv;
+  __nv_bfloat16* o;
+  float* lse;
+  uint32_t* skip_bits;
+  unsigned long long* skipped;
+  int Hq, Hkv, L, nqt, words;
+  float scale2;    // softmax scale * log2(e)
+  float log2lam;   // log2(lambda), -inf for lambda = 0
+};
+
+struct Bars {
+  uint64_t q_full;
+  uint64_t kv_full[kStages];
+  uint64_t kv_empty[kStages];
+  uint64_t s_full[2];
+  uint64_t p_full[2];
+  uint64_t o_done;
+  uint32_t tmem;
+  int skip[2];
+  int abort;
+};
+
+constexpr size_t kSmemBytes = 1024 /*alignment slack*/ + kQBytes + kStages * kStageBytes + 256;
+
+__global__ void __launch_bounds__(kThreads, 1) blasst_prefill_kernel(const __grid_constant__ PrefillParams p) {
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  unsigned char* Qs = smem;
+  unsigned char* KV = smem + kQBytes;
+  Bars* bars = reinterpret_cast<Bars*>(smem + kQBytes + kStages * kStageBytes);
+  volatile int* abort = &bars->abort;
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int bh = blockIdx.x;                       // b * Hq + h
+  const int a = p.nqt - 1 - (int)blockIdx.y;       // heaviest query tiles first
+  const int G = p.Hq / p.Hkv;
+  const int b = bh / p.Hq, h = bh - b * p.Hq;
+  const int bg = b * p.Hkv + h / G;
+  const int i0 = a * kBM;
+  const int i1 = min(i0 + kBM, p.L);
+  const int n_visit = (i1 - 1) / kBN + 1;
+
+  if (tid == 0) {
+    tc::mbar_init(&bars->q_full, 1);
+    for (int s = 0; s < kStages; ++s) {
+      tc::mbar_init(&bars->kv_full[s], 1);
+      tc::mbar_init(&bars->kv_empty[s], 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      tc::mbar_init(&bars->s_full[s], 1);
+      tc::mbar_init(&bars->p_full[s], 128);
+      bars->skip[s] = 0;
+    }
+    tc::mbar_init(&bars->o_done, 1);
+    bars->abort = 0;
+    tc::fence_mbar_init();
+  }
+  if (warp == 2) {
+    tc::tmem_alloc(&bars->tmem, kTmemCols);
+    tc::tmem_relinquish();
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem = bars->tmem;
+
+  if (warp == 0 && lane == 0) {
+    // ---------------------------------------------------------------- TMA producer ----
+    tc::prefetch_tmap(&p.tq);
+    tc::prefetch_tmap(&p.tk);
+    tc::prefetch_tmap(&p.tv);
+    tc::mbar_arrive_expect_tx(&bars->q_full, kQBytes);
+    tc::tma_load_3d(Qs, &p.tq, 0, i0, bh, &bars->q_full);
+    tc::tma_load_3d(Qs + kQBytes / 2, &p.tq, 64, i0, bh, &bars->q_full);
+    for (int j = 0; j < n_visit; ++j) {
+      const int s = j % kStages;
+      if (j >= kStages && !tc::mbar_wait(&bars->kv_empty[s], ((j / kStages) - 1) & 1, abort, kWaitBudget))
+        break;
+      unsigned char* Ks = KV + s * kStageBytes;
+      unsigned char* Vs = Ks + kKVTileBytes;
+      tc::mbar_arrive_expect_tx(&bars->kv_full[s], kStageBytes);
+      tc::tma_load_3d(Ks, &p.tk, 0, j * kBN, bg, &bars->kv_full[s]);
+      tc::tma_load_3d(Ks + kKVTileBytes / 2, &p.tk, 64, j * kBN, bg, &bars->kv_full[s]);
+      tc::tma_load_3d(Vs, &p.tv, 0, j * kBN, bg, &bars->kv_full[s]);
+      tc::tma_load_3d(Vs + kKVTileBytes / 2, &p.tv, 64, j * kBN, bg, &bars->kv_full[s]);
+    }
+  } else if (warp == 1 && lane == 0) {
+    // ----------------------------------------------------------------- MMA issuer ----
+    constexpr uint32_t idesc_qk = tc::idesc_bf16_f32(kBM, kBN, false);
+    constexpr uint32_t idesc_pv = tc::idesc_bf16_f32(kBM, kD, true);
+    const uint32_t q_addr = tc::smem_u32(Qs);
+    const uint32_t kv_addr = tc::smem_u32(KV);
+    auto issue_s = [&](int j) -> bool {
+      const int s = j % kStages;
+      if (!tc::mbar_wait(&bars->kv_full[s], (j / kStages) & 1, abort, kWaitBudget)) return false;
+      const uint32_t k_addr = kv_addr + s * kStageBytes;
+      const uint32_t d = tmem + (uint32_t)(j & 1) * 64u;
+#pragma unroll
+      for (int ks = 0; ks < kD / 16; ++ks) {
+        // K-major, 128-byte swizzle: 64-element boxes; a K step of 16 is 32 bytes in a box
+        const uint64_t ad = tc::smem_desc_sw128(q_addr + (ks >> 2) * (kQBytes / 2) + (ks & 3) * 32, 16, 1024);
+        const uint64_t bd = tc::smem_desc_sw128(k_addr + (ks >> 2) * (kKVTileBytes / 2) + (ks & 3) * 32, 16, 1024);
+        tc::mma_ss(d, ad, bd, idesc_qk, ks > 0 ? 1u : 0u);
+      }
+      tc::mma_commit(&bars->s_full[j & 1]);
+      return true;
+    };
+    bool ok = tc::mbar_wait(&bars->q_full, 0, abort, kWaitBudget);
+    if (ok) ok = issue_s(0);
+    if (ok && n_visit > 1) ok = issue_s(1);
+    int pv_count = 0;
+    for (int j = 0; ok && j < n_visit; ++j) {
+      const int buf = j & 1, s = j % kStages;
+      if (!tc::mbar_wait(&bars->p_full[buf], (j >> 1) & 1, abort, kWaitBudget)) break;
+      tc::fence_after_sync();
+      if (!bars->skip[buf]) {
+        const uint32_t v_addr = kv_addr + s * kStageBytes + kKVTileBytes;
+#pragma unroll
+        for (int kk = 0; kk < kBN / 16; ++kk) {
+          // V as B (K = keys, N = dims): MN-major, 128-byte swizzle; the two 64-dim boxes are
+          // LBO = 8 KB apart, 8-key groups SBO = 1 KB apart; P from TMEM (8 columns per K 16)
+          const uint64_t bd = tc::smem_desc_sw128(v_addr + kk * 16 * 128, kKVTileBytes / 2, 1024);
+          tc::mma_ts(tmem + kColO, tmem + (uint32_t)buf * 64u + (uint32_t)kk * 8u, bd, idesc_pv,
+                     (pv_count > 0 || kk > 0) ? 1u : 0u);
+        }
+        tc::mma_commit(&bars->o_done);
+        ++pv_count;
+      }
+      tc::mma_commit(&bars->kv_empty[s]);
+      if (j + 2 < n_visit && !issue_s(j + 2)) break;
+    }
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------------- softmax ----
+    const int row = tid - 128;
+    const int i = i0 + row;
+    const bool row_ok = i < p.L;
+    const uint32_t lane_addr = tmem + ((uint32_t)(32 * (warp - 4)) << 16);
+    float m_run = -INFINITY, m_used = -INFINITY, l = 0.f;
+    int pv_issued = 0, pv_observed = 0;
+    uint32_t skipmask = 0;
+    int nskipped = 0;
+    bool failed = false;
+    uint32_t* bits_row = p.skip_bits ? p.skip_bits + ((size_t)bh * p.nqt + a) * p.words : nullptr;
+    for (int j = 0; j < n_visit; ++j) {
+      const int buf = j & 1;
+      const bool ok = tc::mbar_wait(&bars->s_full[buf], (j >> 1) & 1, abort, kWaitBudget);
+      if (tc::named_or(1, 128, !ok)) {
+        failed = true;
+        break;
+      }
+      tc::fence_after_sync();
+      uint32_t sr[64];
+      {
+        uint32_t lo[32], hi[32];
+        tc::tmem_ld32(lane_addr + (uint32_t)buf * 64u, lo);
+        tc::tmem_ld32(lane_addr + (uint32_t)buf * 64u + 32u, hi);
+        tc::tmem_ld_wait();
+#pragma unroll
+        for (int c = 0; c < 32; ++c) {
+          sr[c] = lo[c];
+          sr[32 + c] = hi[c];
+        }
+      }
+      // scaled logits (log2 units) with the causal / length mask, and the row max
+      const int t0 = j * kBN;
+      const int lim = min(i, p.L - 1) - t0;  // keys t0 + c with c <= lim are visible
+      float r = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < kBN; ++c) {
+        const float v = (row_ok && c <= lim) ? __uint_as_float(sr[c]) * p.scale2 : -INFINITY;
+        sr[c] = __float_as_uint(v);
+        r = fmaxf(r, v);
+      }
+      // the skip vote: every row negligible (absent rows and rows without a visible key agree)
+      const bool negligible = !row_ok || r == -INFINITY || (m_run != -INFINITY && (r - m_run) < p.log2lam);
+      const bool skip = tc::named_and(1, 128, negligible);
+      if (skip) {
+        if (row == 0) {
+          bars->skip[buf] = 1;
+          skipmask |= 1u << (j & 31);
+          ++nskipped;
+        }
+        tc::mbar_arrive(&bars->p_full[buf]);
+      } else {
+        m_run = fmaxf(m_run, r);
+        float base = m_used;
+        bool resc = false;
+        if (m_used == -INFINITY) {
+          base = m_run;
+        } else if (m_run > m_used + kRescaleLog2) {
+          base = m_run;
+          resc = true;
+        }
+        const float alpha = resc ? ex2(m_used - base) : 1.f;
+        m_used = base;
+        uint32_t pk[32];
+        float rs = 0.f;
+#pragma unroll
+        for (int c = 0; c < 32; ++c) {
+          const float p0 = base == -INFINITY ? 0.f : ex2(__uint_as_float(sr[2 * c]) - base);
+          const float p1 = base == -INFINITY ? 0.f : ex2(__uint_as_float(sr[2 * c + 1]) - base);
+          rs += p0 + p1;
+          pk[c] = pack_bf16x2(p0, p1);
+        }
+        l = l * alpha + rs;
+        tc::tmem_st32(lane_addr + (uint32_t)buf * 64u, pk);
+        tc::tmem_st_wait();
+        if (row == 0) bars->skip[buf] = 0;
+        // the previous P.V must be complete: O is then stable, and at most one O update is
+        // ever outstanding, which keeps the o_done phase parity unambiguous
+        if (pv_issued > pv_observed) {
+          const bool ok2 = tc::mbar_wait(&bars->o_done, pv_observed & 1, abort, kWaitBudget);
+          if (tc::named_or(1, 128, !ok2)) {
+            failed = true;
+            break;
+          }
+          ++pv_observed;
+        }
+        if (__any_sync(0xffffffffu, resc) && pv_issued > 0) {
+          tc::fence_after_sync();
+#pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4) {
+            uint32_t ov[32];
+            tc::tmem_ld32(lane_addr + kColO + 32u * q4, ov);
+            tc::tmem_ld_wait();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
+            tc::tmem_st32(lane_addr + kColO + 32u * q4, ov);
+          }
+          tc::tmem_st_wait();
+        }
+        tc::fence_before_sync();
+        tc::mbar_arrive(&bars->p_full[buf]);
+        ++pv_issued;
+      }
+      if (row == 0 && bits_row && ((j & 31) == 31 || j == n_visit - 1)) {
+        bits_row[j >> 5] = skipmask;
+        skipmask = 0;
+      }
+    }
+    if (!failed) {
+      while (pv_observed < pv_issued) {
+        const bool ok = tc::mbar_wait(&bars->o_done, pv_observed & 1, abort, kWaitBudget);
+        if (tc::named_or(1, 128, !ok)) {
+          failed = true;
+          break;
+        }
+        ++pv_observed;
+      }
+    }
+    if (!failed) {
+      tc::fence_after_sync();
+      const float inv_l = (pv_issued > 0 && l > 0.f) ? 1.f / l : 0.f;
+      __nv_bfloat16* orow = p.o + ((size_t)bh * p.L + (row_ok ? i : 0)) * kD;
+#pragma unroll
+      for (int q4 = 0; q4 < 4; ++q4) {
+        uint32_t ov[32];
+        tc::tmem_ld32(lane_addr + kColO + 32u * q4, ov);
+        tc::tmem_ld_wait();
+        if (row_ok) {
+          uint4* dst = reinterpret_cast<uint4*>(orow + 32 * q4);
+#pragma unroll
+          for (int c8 = 0; c8 < 4; ++c8) {
+            uint4 w;
+            w.x = pack_bf16x2(__uint_as_float(ov[8 * c8 + 0]) * inv_l, __uint_as_float(ov[8 * c8 + 1]) * inv_l);
+            w.y = pack_bf16x2(__uint_as_float(ov[8 * c8 + 2]) * inv_l, __uint_as_float(ov[8 * c8 + 3]) * inv_l);
+            w.z = pack_bf16x2(__uint_as_float(ov[8 * c8 + 4]) * inv_l, __uint_as_float(ov[8 * c8 + 5]) * inv_l);
+            w.w = pack_bf16x2(__uint_as_float(ov[8 * c8 + 6]) * inv_l, __uint_as_float(ov[8 * c8 + 7]) * inv_l);
+            dst[c8] = w;
+          }
+        }
+      }
+      if (row_ok && p.lse) p.lse[(size_t)bh * p.L + i] = (m_used + log2f(l)) * kLn2;
+      if (row == 0 && bits_row)
+        for (int w = (n_visit + 31) >> 5; w < p.words; ++w) bits_row[w] = 0u;
+      if (row == 0 && p.skipped && nskipped) atomicAdd(p.skipped, (unsigned long long)nskipped);
+    }
+    tc::fence_before_sync();
+  }
+
+  __syncthreads();
+  if (tid == 0 && bars->abort) g_device_status = kDeviceTimeout;
+  if (warp == 2) {
+    tc::fence_after_sync();
+    tc::tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// ---- host: tensor maps through the driver entry point (no link against libcuda) --------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (fn == nullptr) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  }
+  return fn;
+}
+
+// 3-D map over [planes][rows][D] bf16, box {64, box_rows, 1}, 128-byte swizzle, zero fill.
+bool make_map(CUtensorMap* map, const void* base, int planes, int rows, int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[3] = {(cuuint64_t)kD, (cuuint64_t)rows, (cuuint64_t)planes};
+  const cuuint64_t strides[2] = {(cuuint64_t)kD * 2, (cuuint64_t)rows * kD * 2};
+  const cuuint32_t box[3] = {64u, (cuuint32_t)box_rows, 1u};
+  const cuuint32_t estr[3] = {1u, 1u, 1u};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+cudaError_t launch_blasst_prefill(const PrefillArgs& a, cudaStream_t stream) {
+  PrefillParams p;
+  memset(&p, 0, sizeof(p));
+  if (!make_map(&p.tq, a.q, a.B * a.Hq, a.L, kBM) || !make_map(&p.tk, a.k, a.B * a.Hkv, a.L, kBN) ||
+      !make_map(&p.tv, a.v, a.B * a.Hkv, a.L, kBN))
+    return cudaErrorInvalidValue;
+  p.o = static_cast<__nv_bfloat16*>(a.o);
+  p.lse = a.lse;
+  p.skip_bits = a.skip_bits;
+  p.skipped = a.skipped_tiles;
+  p.Hq = a.Hq;
+  p.Hkv = a.Hkv;
+  p.L = a.L;
+  p.nqt = (a.L + kBM - 1) / kBM;
+  p.words = ((a.L + kBN - 1) / kBN + 31) / 32;
+  p.scale2 = a.scale * kLog2e;
+  p.log2lam = a.lambda > 0.f ? log2f(a.lambda) : -INFINITY;
+  static bool attr_done = false;
+  if (!attr_done) {
+    const cudaError_t err =
+        cudaFuncSetAttribute(blasst_prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
+    if (err != cudaSuccess) return err;
+    attr_done = true;
+  }
+  dim3 grid(a.B * a.Hq, p.nqt, 1);
+  blasst_prefill_kernel<<<grid, kThreads, kSmemBytes, stream>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t read_device_status(int* status, bool reset) {
+  cudaError_t err = cudaMemcpyFromSymbol(status, g_device_status, sizeof(int));
+  if (err == cudaSuccess && reset) {
+    const int zero = 0;
+    err = cudaMemcpyToSymbol(g_device_status, &zero, sizeof(int));
+  }
+  return err;
+}
+
+}  // namespace lsa

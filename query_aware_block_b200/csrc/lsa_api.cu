@@ -197,10 +197,26 @@ int lsa_blasst_prefill(const void* q, const void* k, const void* v, int dtype, i
                        int Hkv, int L, int D, float scale, float lambda, void* o, float* lse,
                        uint32_t* skip_bits, unsigned long long* skipped_tiles,
                        cudaStream_t stream) {
-  (void)q; (void)k; (void)v; (void)dtype; (void)B; (void)Hq; (void)Hkv; (void)L; (void)D;
-  (void)scale; (void)lambda; (void)o; (void)lse; (void)skip_bits; (void)skipped_tiles;
-  (void)stream;
-  return LSA_ERR_UNSUPPORTED;
+  if (B < 0 || Hq < 1 || Hkv < 1 || L < 0) return LSA_ERR_INVALID_ARG;
+  if (dtype != LSA_BF16 || D != 128) return LSA_ERR_UNSUPPORTED;
+  if (Hq % Hkv != 0 || !(lambda >= 0.f) || !(lambda < 1.f)) return LSA_ERR_INVALID_ARG;
+  if (L > kMaxTcap || (long long)B * Hq > 65535LL * 65535LL) return LSA_ERR_UNSUPPORTED;
+  if (B == 0 || L == 0) return LSA_OK;
+  if (!q || !k || !v || !o) return LSA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return LSA_ERR_INVALID_ARG;
+  if ((L + 127) / 128 > 65535) return LSA_ERR_UNSUPPORTED;
+  lsa::PrefillArgs a = {};
+  a.q = q; a.k = k; a.v = v;
+  a.B = B; a.Hq = Hq; a.Hkv = Hkv; a.L = L;
+  a.scale = resolve_scale(scale, D);
+  a.lambda = lambda;
+  a.o = o; a.lse = lse; a.skip_bits = skip_bits; a.skipped_tiles = skipped_tiles;
+  return cuda_status(lsa::launch_blasst_prefill(a, stream));
+}
+
+int lsa_device_status(int* status, int reset) {
+  if (!status) return LSA_ERR_INVALID_ARG;
+  return cuda_status(lsa::read_device_status(status, reset != 0));
 }
 
 }  // extern "C"

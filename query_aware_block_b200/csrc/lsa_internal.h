@@ -62,6 +62,21 @@ struct BlockQueryArgs {
 size_t blockquery_workspace_bytes(int B, int Hkv, int G, int D, int Tq);
 cudaError_t launch_blockquery(const BlockQueryArgs& a, cudaStream_t stream);
 
+// BLASST causal prefill on tcgen05.
+struct PrefillArgs {
+  const void* q;
+  const void* k;
+  const void* v;
+  int B, Hq, Hkv, L;
+  float scale, lambda;
+  void* o;
+  float* lse;
+  uint32_t* skip_bits;
+  unsigned long long* skipped_tiles;
+};
+cudaError_t launch_blasst_prefill(const PrefillArgs& a, cudaStream_t stream);
+cudaError_t read_device_status(int* status, bool reset);
+
 // The fixed device scratch used by lsa_sparse_attn_blockquery_noalloc.
 size_t blockquery_static_workspace_bytes();
 cudaError_t blockquery_static_workspace(void** ptr);

@@ -101,7 +101,7 @@ def test_binding_argtypes_match_header_parameter_counts():
     text = open(HEADER).read()
     lib = lsa.library()
     for name in _declared():
-        m = re.search(r"\b" + name + r"\s*\(([^)]*)\)", text)
+        m = re.search(r"LSA_API[^;]*?\b" + name + r"\s*\(([^)]*)\)", text)
         params = m.group(1).strip()
         n = 0 if params in ("", "void") else len(params.split(","))
         argt = getattr(lib, name).argtypes
