@@ -60,10 +60,14 @@ WORKLOADS = {
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200000)
-    ap.add_argument("--warmup", type=int, default=600)
+    ap.add_argument("--steps", type=int, default=None,
+                    help="timed steps (default: 200000 decode steps; 20 prefills; 20000 block-query steps)")
+    ap.add_argument("--warmup", type=int, default=None)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="gqa_decode_64k")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS) + ["blockquery", "blasst_prefill_32k"],
+                    default="gqa_decode_64k")
+    ap.add_argument("--prefill-sink", type=float, default=0.0,
+                    help="blasst_prefill_32k: plant an attention sink of this logit height")
     ap.add_argument("--rotate", type=int, default=0, help="input copies (0 = auto, > 4x L2)")
     ap.add_argument("--e2e-steps", type=int, default=2000)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
@@ -72,7 +76,13 @@ def parse():
                     help="launch steps without programmatic dependent launch")
     ap.add_argument("--profile-small", action="store_true",
                     help="a few launches on 2 input copies, for ncu captures")
-    return ap.parse_args()
+    a = ap.parse_args()
+    defaults = {"blockquery": (20000, 200), "blasst_prefill_32k": (20, 3)}.get(a.workload, (200000, 600))
+    if a.steps is None:
+        a.steps = defaults[0]
+    if a.warmup is None:
+        a.warmup = defaults[1]
+    return a
 
 
 # ---------------------------------------------------------------------------- helpers --
@@ -509,8 +519,185 @@ def run_reference(args):
     }
 
 
+# ------------------------------------------------------------ other workloads (extra lines) --
+
+def measured_tensor_peak():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            d = json.load(f)
+        return float(d["bf16_tflops_sustained"]), "measured, sustained"
+    except (OSError, KeyError, ValueError):
+        return 1400.0, "fallback, sustained"
+
+
+def prefill_tile_counts(L, tq=128, tk=64):
+    """Visited KV tiles of one head (causal, ascending up to the diagonal)."""
+    n = 0
+    for a in range(-(-L // tq)):
+        n += (min(a * tq + tq, L) - 1) // tk + 1
+    return n
+
+
+def run_prefill(args):
+    """BLASST causal prefill, 32 q heads / 8 KV heads, D 128, L 32768, lambda 1e-3: a step is
+    one whole prefill.  Inputs (q 256 MB, k/v 128 MB) exceed the L2, so every step reads
+    them from HBM."""
+    import query_aware_block_b200 as lsa
+    import synth
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    case = synth.prefill_case(B=1, Hq=32, Hkv=8, L=32768, D=128, lam=1e-3, sink=args.prefill_sink,
+                              seed=1005, device=dev)
+    B, Hq, L, D = case.q.shape
+    o = torch.empty_like(case.q)
+    lse = torch.empty(B, Hq, L, device=dev)
+    nqt, words = -(-L // 128), -(-(-(-L // 64)) // 32)
+    bits = torch.zeros(B, Hq, nqt, words, dtype=torch.int32, device=dev)
+    cnt = torch.zeros(1, dtype=torch.int64, device=dev)
+
+    def step():
+        lsa.lsa_blasst_prefill(case.q, case.k, case.v, o, case.lam, lse=lse, skip_bits=bits,
+                               skipped_tiles=cnt)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    cnt.zero_()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    K = args.steps
+    with ClockSampler(0) as clocks:
+        torch.cuda.synchronize()
+        e0.record()
+        for _ in range(K):
+            step()
+        e1.record()
+        torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / K
+    visited = B * Hq * prefill_tile_counts(L)
+    skipped = int(cnt.item()) / K
+    tile_flop = 2 * 128 * 64 * D
+    flops = visited * tile_flop + (visited - skipped) * tile_flop  # Q K^T always, P V if kept
+    tflops = flops / (ms * 1e-3) / 1e12
+    peak, kind = measured_tensor_peak()
+    return {
+        "metric": "BLASST causal prefill TFLOP/s (algorithmic: QK^T of every visited tile + PV of kept tiles)",
+        "value": round(tflops, 1), "unit": "TFLOP/s", "n_gpus": 1, "steps": K, "warmup": args.warmup,
+        "ms_per_step": round(ms, 4), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic (seeded N(0,1) q/k/v with RoPE theta 1e4"
+                                  + (f", attention sink {args.prefill_sink}" if args.prefill_sink else "") + ")",
+        "config": {"workload": "blasst_prefill_32k", "batch": B, "q_heads": Hq, "kv_heads": case.k.shape[1],
+                   "head_dim": D, "seq_len": L, "tiles": "128 x 64", "lambda": case.lam,
+                   "l2": "inputs (512 MB) larger than L2"},
+        "tokens_per_s": round(B * L / (ms * 1e-3), 1),
+        "skip_fraction": round(skipped / visited, 4),
+        "roofline": {"bound": "tensor", "achieved": round(tflops, 1), "peak": peak, "unit": "TFLOP/s",
+                     "frac": round(tflops / peak, 4), "traffic": None,
+                     "kernel": "blasst_prefill_kernel (tcgen05)",
+                     "peak_source": f"MEASURED_PEAKS.json bf16_tflops_sustained ({kind})",
+                     "algorithmic_flops_per_launch": flops},
+        "gpu_launches": K,
+        "clocks": clocks.summary(),
+    }
+
+
+def run_blockquery(args):
+    """Diffusion-LM block-query step (32 query tokens, 8 active, prefix 32768, top-8 blocks
+    per token and KV head).  A step is one call; R rotated input copies exceed 4x L2."""
+    import query_aware_block_b200 as lsa
+    import synth
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    base = synth.diffusion_blockquery(device=dev)
+    B, Hq, Tq, D = base.q.shape
+    Hkv = base.k.shape[1]
+    G = Hq // Hkv
+    T_cap = base.k.shape[2]
+    NBp = -(-base.T_prefix // 64)
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    ws = torch.empty(lsa.lsa_blockquery_workspace_size(B, Hkv, G, D, Tq), dtype=torch.uint8, device=dev)
+    copies = []
+    R = 4
+    for r in range(64):
+        c = base if r == 0 else synth.blockquery_case(seed=1004 + 101 * r, device=dev)
+        sl = torch.full((B,), T_cap, dtype=torch.int32, device=dev)
+        summ = torch.zeros(B, Hkv, -(-T_cap // 64), D, device=dev)
+        lsa.lsa_build_summaries(c.k, sl, summ)
+        copies.append(dict(c=c, summ=summ, o=torch.empty_like(c.o_cache), lse=torch.empty_like(c.lse_cache),
+                           ui=torch.empty(B, Hkv, NBp, dtype=torch.int32, device=dev),
+                           uc=torch.empty(B, Hkv, dtype=torch.int32, device=dev)))
+        if r == 0:
+            def one(x):
+                lsa.lsa_sparse_attn_blockquery(x["c"].q, x["c"].k, x["c"].v, x["summ"], x["c"].T_prefix,
+                                               x["c"].topk, x["c"].active, x["c"].o_cache, x["c"].lse_cache,
+                                               x["o"], x["lse"], ws, union_idx=x["ui"], union_cnt=x["uc"])
+            one(copies[0])
+            torch.cuda.synchronize()
+            U = int(copies[0]["uc"].sum())
+            A = int(base.active.sum())
+            step_bytes = (Hkv * NBp * D * 4 + U * 64 * D * 2 * 2 + 2 * A * G * Hkv * D * 2
+                          + (Tq - A) * G * Hkv * D * 2 * 2)
+            R = max(4, min(64, math.ceil(4 * l2 / step_bytes)))
+            if args.profile_small:
+                R = 4
+        if len(copies) >= R:
+            break
+    for x in copies:
+        one(x)
+    torch.cuda.synchronize()
+    U_mean = sum(int(x["uc"].sum()) for x in copies) / len(copies)
+    A = int(base.active.sum())
+    step_bytes = (Hkv * NBp * D * 4 + U_mean * 64 * D * 2 * 2 + 2 * A * G * Hkv * D * 2
+                  + (Tq - A) * G * Hkv * D * 2 * 2 + Hkv * NBp * 4)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for x in copies:
+            one(x)
+    K = args.steps
+    reps = max(1, K // R)
+    for _ in range(max(1, args.warmup // R)):
+        g.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(0) as clocks:
+        torch.cuda.synchronize()
+        e0.record()
+        for _ in range(reps):
+            g.replay()
+        e1.record()
+        torch.cuda.synchronize()
+    steps = reps * R
+    ms = e0.elapsed_time(e1) / steps
+    gbs = step_bytes / (ms * 1e-3) / 1e9
+    peak, kind = measured_peaks()
+    return {
+        "metric": "block-query denoising step: query tokens/s and effective GB/s (% of HBM roofline)",
+        "value": round(B * Tq / (ms * 1e-3), 1), "unit": "tokens/s", "n_gpus": 1, "steps": steps,
+        "warmup": args.warmup, "ms_per_step": round(ms, 6), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1), RoPE theta 1e4)",
+        "config": {"workload": "blockquery", "batch": B, "kv_heads": Hkv, "q_heads_per_kv": G,
+                   "head_dim": D, "query_tokens": Tq, "active": A, "prefix": base.T_prefix,
+                   "topk_per_token": base.topk,
+                   "l2": f"rotating {R} input copies ({R * step_bytes / 1e6:.0f} MB per cycle)"},
+        "mean_union_blocks_per_kv_head": round(U_mean / (B * Hkv), 2),
+        "kv_density": round(U_mean / (B * Hkv) / NBp, 4),
+        "effective_gbs": round(gbs, 1), "bytes_per_step": int(step_bytes),
+        "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peak, "unit": "GB/s",
+                     "frac": round(gbs / peak, 4), "traffic": None, "kernel": "blockquery_kernel<128>",
+                     "peak_source": f"MEASURED_PEAKS.json hbm_gbs ({kind})"},
+        "gpu_launches": steps,
+        "clocks": clocks.summary(),
+    }
+
+
 def main():
     args = parse()
+    if args.workload in ("blockquery", "blasst_prefill_32k"):
+        if args.impl == "reference":
+            print(json.dumps({"impl": "reference", "unavailable": "the oracle arm covers the decode workloads"}))
+            return
+        res = run_blockquery(args) if args.workload == "blockquery" else run_prefill(args)
+        print(json.dumps(res), flush=True)
+        return
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
