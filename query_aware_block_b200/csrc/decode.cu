@@ -53,7 +53,13 @@ constexpr int kMaxTopk = 64;
 constexpr int kMaxCluster = 16;
 constexpr int kStages = 2;
 constexpr int kSStride = 72;    // fp32 row stride of the score tile (bank spread)
-constexpr int kRowsPerWarp = 8; // summary rows a warp has in flight per pass
+// Scoring: 4 threads share a summary row's dot product, lane l of a warp taking row
+// 8 * warp + (l & 7) and quarter l >> 3, so that each quarter-warp (the unit of a 128-bit
+// shared-memory access) reads one quarter of 8 different rows: with the chunk swizzle below
+// that is 8 different bank groups, and the summed query it multiplies is one broadcast.
+constexpr int kLanesPerRow = 4;
+constexpr int kPassRows = kThreads / kLanesPerRow;  // summary rows scored per pass
+static_assert(kLanesPerRow == 4 && kPassRows == kWarps * 8, "the scoring's lane mapping");
 
 struct Params {
   const void* q;
@@ -82,7 +88,7 @@ __host__ __device__ inline size_t align128(size_t x) { return (x + 127) & ~(size
 
 // Shared-memory carve-up (byte offsets), identical on host and device.
 struct Layout {
-  size_t qs, keys, top, work, all, order, kv, ss, ps, alpha, ml_in, pacc_in, total;
+  size_t qs, qsum, keys, top, work, all, order, kv, ss, ps, alpha, ml_in, pacc_in, total;
   size_t kv_row, kv_tile;  // bytes per K/V row in smem, bytes per 64-row tile
 };
 
@@ -95,6 +101,7 @@ __host__ __device__ inline Layout make_layout(int elem_bytes, int D, int per_max
   L.kv_row = f32 ? (size_t)(D + 4) * 4 : (size_t)D * 2;
   L.kv_tile = L.kv_row * kBlk;
   L.qs = off;      off = align128(off + (size_t)kRows * D * elem_bytes);
+  L.qsum = off;    off = align128(off + (size_t)D * 4);
   L.keys = off;    off = align128(off + (size_t)per_max * 8);
   L.top = off;     off = align128(off + (size_t)lp * 8);
   L.work = off;    off = align128(off + (size_t)nwork * 8);
@@ -176,37 +183,14 @@ __device__ const u64* merge_lists(u64* lists, u64* work, int CL) {
   return src;
 }
 
-// N consecutive elements as float.  kL2 = true reads through L2 only (ld.global.cg), for
-// data the previous kernel of the stream may have produced.
-template <typename T, int N, bool kL2 = false>
-__device__ __forceinline__ void load_f32(const T* p, float (&out)[N]) {
-  if constexpr (sizeof(T) == 4) {
-    if constexpr (N == 4) {
-      const float4 v = kL2 ? __ldcg(reinterpret_cast<const float4*>(p)) : __ldg(reinterpret_cast<const float4*>(p));
-      out[0] = v.x; out[1] = v.y; out[2] = v.z; out[3] = v.w;
-    } else {
-      const float2 v = kL2 ? __ldcg(reinterpret_cast<const float2*>(p)) : __ldg(reinterpret_cast<const float2*>(p));
-      out[0] = v.x; out[1] = v.y;
-    }
-  } else {
-    if constexpr (N == 4) {
-      const uint2 v = kL2 ? __ldcg(reinterpret_cast<const uint2*>(p)) : __ldg(reinterpret_cast<const uint2*>(p));
-      const __nv_bfloat162 a = *reinterpret_cast<const __nv_bfloat162*>(&v.x);
-      const __nv_bfloat162 b = *reinterpret_cast<const __nv_bfloat162*>(&v.y);
-      out[0] = __low2float(a); out[1] = __high2float(a);
-      out[2] = __low2float(b); out[3] = __high2float(b);
-    } else {
-      const uint32_t v = kL2 ? __ldcg(reinterpret_cast<const unsigned int*>(p)) : __ldg(reinterpret_cast<const unsigned int*>(p));
-      const __nv_bfloat162 a = *reinterpret_cast<const __nv_bfloat162*>(&v);
-      out[0] = __low2float(a); out[1] = __high2float(a);
-    }
-  }
-}
-
 // ---- the kernel ---------------------------------------------------------------------
 
 template <typename T, int D, int MODE>
 __global__ void __launch_bounds__(kThreads, 2) decode_cluster_kernel(const Params p) {
+  // the parameter block is fetched all at once here (fields spaced < 32 bytes apart), not
+  // one constant-cache miss after another on first use
+  asm volatile("" ::"l"(p.q), "r"(p.T_cap), "l"(p.summ_w), "r"(p.topk), "l"(p.nsel_out), "l"(p.lse),
+               "r"(p.chunk));
   const int CL = cluster_size();
   const int rank = cluster_rank();
   // DSMEM may be written only once every CTA of the cluster runs: arrive now, wait late
@@ -242,9 +226,29 @@ __global__ void __launch_bounds__(kThreads, 2) decode_cluster_kernel(const Param
   const T* qg = static_cast<const T*>(p.q) + ((size_t)b * p.Hkv * G + (size_t)g * G) * D;
   const T* kbase = static_cast<const T*>(p.k) + unit * (size_t)p.T_cap * D;
   const T* vbase = static_cast<const T*>(p.v) + unit * (size_t)p.T_cap * D;
+  const bool select = MODE != MODE_ATTEND;
+
+  // ---- the first pass of this CTA's summary rows, requested before anything else: the
+  // slice [j0, j0 + per) depends on the capacity only, so the copy need not wait for the
+  // sequence length.  Stage 1 of the K/V ring holds it while scanning.
+  // row r's 16-byte chunk c sits at chunk c ^ (r & 7): the 8 rows a warp scores at once
+  // then read 8 different bank groups
+  constexpr int kRowChunks = D / 4;
+  const int per = p.per_max;
+  const int j0 = rank * per;
+  float* sumbuf = reinterpret_cast<float*>(kv + 2 * (size_t)kv_tile);
+  const bool may_scan = select && p.NB_cap > p.topk;
+  if (may_scan) {  // asynchronous copies: the summary rows cannot be written by the previous kernel
+    const int staged_rows = max(0, min(min(per, p.NB_cap - j0), kPassRows));
+    const float* src0 = p.summ + (unit * (size_t)p.NB_cap + j0) * D;
+    for (int id = tid; id < staged_rows * kRowChunks; id += kThreads) {
+      const int r = id / kRowChunks, c = id % kRowChunks;
+      cp_async16(sumbuf + r * D + ((c ^ (r & 7)) << 2), src0 + id * 4, true);
+    }
+    cp_async_commit();
+  }
 
   // ---- which blocks: forced / all known up front; order[i] is handled by CTA i % CL ----
-  const bool select = MODE != MODE_ATTEND;
   const bool all_blocks = select && NB <= p.topk;
   const int nf = (select && !all_blocks) ? p.n_sink + p.n_local : 0;  // disjoint: NB > topk
   int n_order;
@@ -265,53 +269,49 @@ __global__ void __launch_bounds__(kThreads, 2) decode_cluster_kernel(const Param
 
   // ---- before waiting on the previous kernel of the stream: copies of data that kernel
   // cannot have written (the K/V of the known blocks except the sequence's newest one, and
-  // the first pass of summary rows).  With overlapped launch the caller vouches for this.
+  // the summary rows above).  With overlapped launch the caller vouches for this.
   int issued = 0;  // my blocks whose copies were committed, in processing order
   const int known = all_blocks ? NB : nf;
   const int n_known = (MODE == MODE_FUSED && known > rank) ? (known - rank + CL - 1) / CL : 0;
+  const bool scan = select && !all_blocks;
+  const int nloc = scan ? max(0, min(NB, j0 + per) - j0) : 0;
+  // while scanning, stage 1 holds the first pass of this CTA's summary rows
+  const int early_stages = scan ? 1 : kStages;
   if (MODE == MODE_FUSED) {
-    while (issued < kStages && issued < n_known && known_block(issued) != NB - 1) {
+    while (issued < early_stages && issued < n_known && known_block(issued) != NB - 1) {
+      // a short sequence that scans nothing reuses stage 1 once the summary copy has landed
+      if (may_scan && issued == 1) cp_async_wait<1>();
       unsigned char* st = kv + (size_t)(issued % kStages) * 2 * kv_tile;
       stage_block<T, D, kThreads>(st, st + kv_tile, kbase, vbase, known_block(issued), Tb, kv_row);
       cp_async_commit();
       ++issued;
     }
   }
-  constexpr int VEC = D / 32;  // elements per lane of a D-row
-  const bool scan = select && !all_blocks;
-  const int per = (NB + CL - 1) / CL;
-  const int j0 = rank * per;
-  const int nloc = scan ? max(0, min(NB, j0 + per) - j0) : 0;
-  const float* sb = p.summ + unit * (size_t)p.NB_cap * D + lane * VEC;
-  float vals[kRowsPerWarp][VEC];
-  auto load_pass = [&](int o0) {
-#pragma unroll
-    for (int u = 0; u < kRowsPerWarp; ++u) {
-      const int oo = o0 + u * kWarps;
-      if (oo < nloc) {
-        load_f32<float, VEC>(sb + (size_t)(j0 + oo) * D, vals[u]);
-      } else {
-#pragma unroll
-        for (int e = 0; e < VEC; ++e) vals[u][e] = 0.f;
-      }
-    }
-  };
-  if (scan) load_pass(warp);
   pdl_trigger();
   pdl_wait();
 
-  // ---- query rows (staged for the mma) and the newest block, after the wait ------------
-  if (MODE != MODE_SELECT) {
+  // ---- query rows (the mma's A tile; rows >= G zero), then the remaining known blocks ----
+  {
     constexpr int kQChunks = kRows * kRowBytesQ / 16;
     for (int id = tid; id < kQChunks; id += kThreads) {
       const int row = id / (kRowBytesQ / 16), c = id % (kRowBytesQ / 16);
-      uint4 v4 = make_uint4(0u, 0u, 0u, 0u);
-      if (row < G) v4 = __ldcg(reinterpret_cast<const uint4*>(qg + (size_t)row * D) + c);
-      *reinterpret_cast<uint4*>(Qs + (kF32 ? row * kRowBytesQ + c * 16 : swz(row, c, kRowBytesQ))) = v4;
+      cp_async16(Qs + (kF32 ? row * kRowBytesQ + c * 16 : swz(row, c, kRowBytesQ)),
+                 qg + (size_t)(row < G ? row : 0) * D + c * (16 / (int)sizeof(T)), row < G);
     }
+    cp_async_commit();
   }
-  if (MODE == MODE_FUSED) {
+  const int issued_before_q = issued;
+  bool newest_issued = false;
+  if (MODE == MODE_FUSED && scan && issued == 0 && n_known > 0) {  // the newest block, now
+    stage_block<T, D, kThreads>(kv, kv + kv_tile, kbase, vbase, known_block(0), Tb, kv_row);
+    cp_async_commit();
+    ++issued;
+    newest_issued = true;
+  }
+  if (MODE == MODE_FUSED && !scan) {
     while (issued < kStages && issued < n_known) {
+      // stage 1 is reused once the summary copy (two groups older) has landed
+      if (may_scan && issued == 1) cp_async_wait<2>();
       unsigned char* st = kv + (size_t)(issued % kStages) * 2 * kv_tile;
       stage_block<T, D, kThreads>(st, st + kv_tile, kbase, vbase, known_block(issued), Tb, kv_row);
       cp_async_commit();
@@ -321,40 +321,89 @@ __global__ void __launch_bounds__(kThreads, 2) decode_cluster_kernel(const Param
 
   // ---- selection --------------------------------------------------------------------
   if (scan) {
+    // the staged summary and query rows: only the newest block's copy may be in flight
+    if (newest_issued) cp_async_wait<1>(); else cp_async_wait<0>();
+    __syncthreads();
     const int m = p.topk - nf;
-    // summed, scaled query of the group, per warp in registers
-    float qv[VEC];
-#pragma unroll
-    for (int e = 0; e < VEC; ++e) qv[e] = 0.f;
-    for (int h = 0; h < G; ++h) {
-      float t[VEC];
-      load_f32<T, VEC, true>(qg + (size_t)h * D + lane * VEC, t);
-#pragma unroll
-      for (int e = 0; e < VEC; ++e) qv[e] += t[e];
+    // summed, scaled query row of the group (fp32, shared), from the staged query rows
+    float* qsum = reinterpret_cast<float*>(smem + Lo.qsum);
+    for (int d = tid; d < D; d += kThreads) {
+      float acc = 0.f;
+      for (int h = 0; h < G; ++h) {
+        if constexpr (kF32)
+          acc += reinterpret_cast<const float*>(Qs + h * kRowBytesQ)[d];
+        else
+          acc += __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(
+              Qs + swz(h, (2 * d) >> 4, kRowBytesQ) + ((2 * d) & 15)));
+      }
+      qsum[d] = acc * p.scale;
     }
+    __syncthreads();
+    // kLanesPerRow threads per summary row, each a contiguous quarter of the row
+    constexpr int kSeg = D / kLanesPerRow;  // floats per thread
+    const int part = lane >> 3;
+    float qv[kSeg];
 #pragma unroll
-    for (int e = 0; e < VEC; ++e) qv[e] *= p.scale;
-    for (int o0 = warp;; o0 += kWarps * kRowsPerWarp) {
-      if (o0 != warp) load_pass(o0);
+    for (int k = 0; k < kSeg / 4; ++k) {
+      const float4 v = reinterpret_cast<const float4*>(qsum + part * kSeg)[k];
+      qv[4 * k] = v.x; qv[4 * k + 1] = v.y; qv[4 * k + 2] = v.z; qv[4 * k + 3] = v.w;
+    }
+    const float* grow = p.summ + (unit * (size_t)p.NB_cap + j0) * D + part * kSeg;
+    for (int base = 0; base < nloc; base += kPassRows) {  // uniform trip count
+      const int oo = base + warp * 8 + (lane & 7);
+      float a4[4] = {0.f, 0.f, 0.f, 0.f};
+      if (oo < nloc) {
 #pragma unroll
-      for (int u = 0; u < kRowsPerWarp; ++u) {
-        const int oo = o0 + u * kWarps;
-        float dot = 0.f;
-#pragma unroll
-        for (int e = 0; e < VEC; ++e) dot = fmaf(vals[u][e], qv[e], dot);
-        dot = warp_sum(dot);
-        if (oo < nloc && lane == 0) {
+        for (int k = 0; k < kSeg / 4; ++k) {
+          float4 v;
+          if (base == 0) {  // staged (swizzled) first pass
+            const int c = part * (kSeg / 4) + k;
+            v = *reinterpret_cast<const float4*>(sumbuf + oo * D + ((c ^ (oo & 7)) << 2));
+          } else {
+            v = __ldg(reinterpret_cast<const float4*>(grow + (size_t)oo * D) + k);
+          }
+          a4[k & 3] = fmaf(v.x, qv[4 * k], a4[k & 3]);
+          a4[k & 3] = fmaf(v.y, qv[4 * k + 1], a4[k & 3]);
+          a4[k & 3] = fmaf(v.z, qv[4 * k + 2], a4[k & 3]);
+          a4[k & 3] = fmaf(v.w, qv[4 * k + 3], a4[k & 3]);
+        }
+      }
+      float dot = (a4[0] + a4[1]) + (a4[2] + a4[3]);
+      dot += __shfl_xor_sync(0xffffffffu, dot, 8);
+      dot += __shfl_xor_sync(0xffffffffu, dot, 16);
+      if (part == 0) {
+        if (oo < nloc) {
           const int j = j0 + oo;
           const bool forced = j < p.n_sink || j >= NB - p.n_local;
           keys[oo] = forced ? 0ull : make_key(dot, j);
           if (p.scores_out) p.scores_out[unit * p.NB_cap + j] = dot;
+        } else if (oo < kPassRows && oo < per) {
+          keys[oo] = 0ull;  // the rank count below reads a full pass
         }
       }
-      if (o0 + kWarps * kRowsPerWarp >= nloc) break;
+    }
+    if (nloc == 0) {  // no pass ran: the rank count below still reads a full pass
+      for (int i = tid; i < min(kPassRows, per); i += kThreads) keys[i] = 0ull;
     }
     __syncthreads();
     // local top-m, sorted, zero padded to lp
-    if (nloc <= kThreads) {
+    if (nloc <= kPassRows && per >= kPassRows) {
+      // 4 threads per key (the lane mapping of the scoring), each counting the larger keys
+      // in a quarter of the pass
+      const int i = warp * 8 + (lane & 7), part = lane >> 3;
+      const u64 x = keys[i];
+      const ulonglong2* k2 = reinterpret_cast<const ulonglong2*>(keys + part * (kPassRows / 4));
+      int r = 0;
+#pragma unroll
+      for (int q4 = 0; q4 < kPassRows / 8; ++q4) {
+        const ulonglong2 kk = k2[q4];
+        r += (kk.x > x) + (kk.y > x);
+      }
+      r += __shfl_xor_sync(0xffffffffu, r, 8);
+      r += __shfl_xor_sync(0xffffffffu, r, 16);
+      if (part == 0 && x != 0ull && r < m) top[r] = x;
+      __syncthreads();
+    } else if (nloc <= kThreads) {
       const u64 x = tid < nloc ? keys[tid] : 0ull;
       if (x != 0ull) {
         int r = 0, u = 0;
@@ -407,6 +456,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_cluster_kernel(const Param
     if (MODE == MODE_SELECT && tid == 0) p.nsel_out[unit] = n_order;
   }
   if (MODE == MODE_SELECT) {
+    cp_async_wait<0>();  // no copy into shared memory outlives the CTA
     if (!started) cluster_wait();
     return;  // no CTA reads a peer's shared memory: no trailing barrier
   }
@@ -418,6 +468,10 @@ __global__ void __launch_bounds__(kThreads, 2) decode_cluster_kernel(const Param
     stage_block<T, D, kThreads>(st, st + kv_tile, kbase, vbase, order[rank + issued * CL], Tb, kv_row);
     cp_async_commit();
     ++issued;
+  }
+  if (!scan) {  // the query rows' copy, followed by at most kStages block copies
+    const int after_q = issued - issued_before_q;
+    if (after_q >= 2) cp_async_wait<2>(); else if (after_q == 1) cp_async_wait<1>(); else cp_async_wait<0>();
   }
   __syncthreads();  // (the staged query rows are visible)
 
@@ -580,6 +634,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_cluster_kernel(const Param
     }
   }
 
+  cp_async_wait<0>();  // (a CTA with no block may still have its query copy in flight)
   // ---- push the partial (m, l, acc) to the CTAs that merge each output slice -----------
   if (!started) {
     cluster_wait();
