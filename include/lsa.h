@@ -30,7 +30,9 @@
  *           error nothing is enqueued and the status is returned.  LSA_ERR_CUDA means a
  *           launch failed; lsa_last_cuda_error() returns that cudaError_t for the
  *           calling thread.  Device-side values (seqlens, idx) are trusted: they must obey
- *           the documented ranges.
+ *           the documented ranges.  Waits between the CTAs of one launch are bounded in
+ *           time (about 2 s); should one ever run out, the launch's outputs are undefined
+ *           and lsa_device_status() reports LSA_DEVICE_TIMEOUT.
  */
 #ifndef LSA_H_
 #define LSA_H_

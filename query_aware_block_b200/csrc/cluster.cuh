@@ -1,5 +1,5 @@
 // cluster.cuh -- thread-block-cluster and launch primitives shared by the kernels
-// (PTX ISA: barrier.cluster, mapa, st.shared::cluster, griddepcontrol), and the warp-wide
+// (PTX ISA: barrier.cluster, mapa, st.shared::cluster, st.async, griddepcontrol), and the warp-wide
 // bitonic merge used to combine sorted candidate lists.
 #pragma once
 
@@ -45,6 +45,26 @@ __device__ __forceinline__ void st_cluster_u32(uint32_t addr, uint32_t v) {
 }
 __device__ __forceinline__ void st_cluster(uint32_t addr, float v) {
   asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
+}
+
+// st.async: a store into a peer CTA's shared memory whose bytes count toward the
+// transaction count of an mbarrier in that CTA (both addresses from mapa).  The receiver
+// learns that the data has landed by waiting on its own mbarrier; no cluster barrier.
+__device__ __forceinline__ void st_async(uint32_t addr, unsigned long long v, uint32_t mbar) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.b64 [%0], %1, [%2];" ::"r"(addr),
+               "l"(v), "r"(mbar)
+               : "memory");
+}
+__device__ __forceinline__ void st_async(uint32_t addr, float2 v, uint32_t mbar) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v2.f32 [%0], {%1, %2}, [%3];" ::"r"(
+                   addr),
+               "f"(v.x), "f"(v.y), "r"(mbar)
+               : "memory");
+}
+__device__ __forceinline__ void st_async(uint32_t addr, float v, uint32_t mbar) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.f32 [%0], %1, [%2];" ::"r"(addr),
+               "f"(v), "r"(mbar)
+               : "memory");
 }
 
 // Programmatic dependent launch (PTX griddepcontrol): with the launch attribute set, the

@@ -10,15 +10,19 @@
 //
 // How (B200).  A decode step moves only a few MB, so the kernel is built for latency:
 //   * A cluster of CL CTAs (16, 8 or 4) owns one (b, g); 2 CTAs fit per SM, so a 16-CTA
-//     cluster per KV head fits in one wave.  At launch every CTA issues its slice of the
-//     summary rows (a warp per row, coalesced float4) and the group's query rows together;
-//     CTAs that own a forced block also start its K/V copy, so that copy overlaps the scan.
+//     cluster per KV head fits in one wave.  At launch every CTA copies its slice of the
+//     summary rows into shared memory with cp.async (the slice is fixed by the capacity, so
+//     the copy does not wait for the sequence length); CTAs that own a forced block also
+//     start its K/V copy, so that copy overlaps the scan.  The group's query rows follow.
+//   * Scoring: 4 threads per summary row (quarter-warp-uniform lane mapping, XOR-swizzled
+//     rows: conflict-free 128-bit shared loads) against the summed query in shared memory.
 //   * Each CTA ranks its candidates (64-bit keys: score, then lower index) and PUSHES its
-//     sorted local top-m list into every peer's shared memory (st.shared::cluster); after
-//     one release/acquire cluster barrier every CTA merges the CL sorted lists with a tree
-//     of warp-wide bitonic merges (shuffles only) and derives the same global top-m.
+//     sorted local top-m list into every peer's shared memory with st.async, whose bytes
+//     count toward an mbarrier in the receiving CTA: each CTA waits only until the CL lists
+//     have landed (no cluster-wide barrier), then merges them with a tree of warp-wide
+//     bitonic merges (shuffles only) and derives the same global top-m as its peers.
 //     DSMEM is touched only after a split arrive(relaxed)/wait barrier that proves every
-//     CTA of the cluster has started.
+//     CTA of the cluster has started and initialised its mbarriers.
 //   * Overlapped launch (optional, programmatic dependent launch): the summary rows and the
 //     K/V of the forced blocks other than the newest one are requested before the kernel
 //     waits for the previous kernel of the stream; q and the newest block after it.
@@ -28,23 +32,31 @@
 //     mma.sync m16n8k16 for S = Q K^T and O += P V; the fp32 path uses CUDA-core FMA.
 //     Online softmax in base 2 with fp32 statistics.
 //   * Each CTA pushes its partial (m, l) and the slices of its accumulator to the CTAs
-//     that own those output elements; after a second cluster barrier every CTA merges its
-//     1/CL slice by log-sum-exp from its own shared memory and writes it.  No CTA reads a
-//     peer's shared memory, so no trailing barrier is needed.
+//     that own those output elements (st.async again, second mbarrier); each CTA waits for
+//     its CL partials and merges its 1/CL slice by log-sum-exp from its own shared memory.
+//     Every byte a CTA receives is counted by its own mbarriers and waited for before it
+//     ends, so no CTA leaves while a peer may still write into it; no trailing barrier.
 //   * Optionally the CTA that attends the sequence's last block (always a forced local
 //     block) also refreshes that block's summary from the keys it staged: the summary
 //     update of a decode step costs no extra launch and no extra HBM read.
-// No global scratch memory and no spin-waits: cross-CTA ordering uses cluster barriers.
+// No global scratch memory.  The two mbarrier waits are bounded (about 2 s of clock); if
+// one runs out the launch's outputs are undefined and a device status word records it.
 #include <math.h>
 
 #include "cluster.cuh"
 #include "lsa_common.cuh"
 #include "lsa_internal.h"
+#include "tcgen05.cuh"
 
 namespace lsa {
 namespace {
 
 typedef unsigned long long u64;
+
+// Set when a bounded wait on a cross-CTA exchange runs out (the outputs of that launch are
+// then undefined); read and cleared by the host.
+__device__ int g_decode_status = 0;
+constexpr long long kWaitBudget = 4000000000LL;  // clock cycles (about 2 s)
 
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
@@ -53,13 +65,9 @@ constexpr int kMaxTopk = 64;
 constexpr int kMaxCluster = 16;
 constexpr int kStages = 2;
 constexpr int kSStride = 72;    // fp32 row stride of the score tile (bank spread)
-// Scoring: 4 threads share a summary row's dot product, lane l of a warp taking row
-// 8 * warp + (l & 7) and quarter l >> 3, so that each quarter-warp (the unit of a 128-bit
-// shared-memory access) reads one quarter of 8 different rows: with the chunk swizzle below
-// that is 8 different bank groups, and the summed query it multiplies is one broadcast.
-constexpr int kLanesPerRow = 4;
-constexpr int kPassRows = kThreads / kLanesPerRow;  // summary rows scored per pass
-static_assert(kLanesPerRow == 4 && kPassRows == kWarps * 8, "the scoring's lane mapping");
+// A scoring pass covers kPassRows summary rows, 8 per warp; the local rank count after it
+// gives each key 4 threads (lane l of warp w: key 8w + (l & 7), quarter l >> 3 of the keys).
+constexpr int kPassRows = kWarps * 8;
 
 struct Params {
   const void* q;
@@ -193,10 +201,6 @@ __global__ void __launch_bounds__(kThreads, 2) decode_cluster_kernel(const Param
                "r"(p.chunk));
   const int CL = cluster_size();
   const int rank = cluster_rank();
-  // DSMEM may be written only once every CTA of the cluster runs: arrive now, wait late
-  cluster_arrive_relaxed();
-  bool started = false;  // uniform: the start barrier has been waited on
-
   const int g = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int G = p.G;
@@ -205,6 +209,10 @@ __global__ void __launch_bounds__(kThreads, 2) decode_cluster_kernel(const Param
   constexpr bool kF32 = sizeof(T) == 4;
   constexpr int kRowBytesQ = D * (int)sizeof(T);
 
+  // mbarriers, one phase each: [0] and [1] count the bytes of the two cross-CTA exchanges,
+  // [2] the bulk copy of this CTA's summary rows
+  __shared__ __align__(8) uint64_t xbar[3];
+  __shared__ int xabort;
   extern __shared__ __align__(1024) unsigned char smem[];
   const Layout Lo = make_layout((int)sizeof(T), D, p.per_max, p.m_pad);
   unsigned char* Qs = smem + Lo.qs;
@@ -228,25 +236,31 @@ __global__ void __launch_bounds__(kThreads, 2) decode_cluster_kernel(const Param
   const T* vbase = static_cast<const T*>(p.v) + unit * (size_t)p.T_cap * D;
   const bool select = MODE != MODE_ATTEND;
 
-  // ---- the first pass of this CTA's summary rows, requested before anything else: the
-  // slice [j0, j0 + per) depends on the capacity only, so the copy need not wait for the
-  // sequence length.  Stage 1 of the K/V ring holds it while scanning.
-  // row r's 16-byte chunk c sits at chunk c ^ (r & 7): the 8 rows a warp scores at once
-  // then read 8 different bank groups
-  constexpr int kRowChunks = D / 4;
+  // ---- the first pass of this CTA's summary rows, requested before anything else with one
+  // bulk copy (the copy engine, not the load/store unit): the slice [j0, j0 + per) depends
+  // on the capacity only, so it need not wait for the sequence length, and the previous
+  // kernel of the stream cannot write it.  Stage 1 of the K/V ring holds it while scanning.
   const int per = p.per_max;
   const int j0 = rank * per;
   float* sumbuf = reinterpret_cast<float*>(kv + 2 * (size_t)kv_tile);
   const bool may_scan = select && p.NB_cap > p.topk;
-  if (may_scan) {  // asynchronous copies: the summary rows cannot be written by the previous kernel
-    const int staged_rows = max(0, min(min(per, p.NB_cap - j0), kPassRows));
-    const float* src0 = p.summ + (unit * (size_t)p.NB_cap + j0) * D;
-    for (int id = tid; id < staged_rows * kRowChunks; id += kThreads) {
-      const int r = id / kRowChunks, c = id % kRowChunks;
-      cp_async16(sumbuf + r * D + ((c ^ (r & 7)) << 2), src0 + id * 4, true);
+  const int staged_rows = may_scan ? max(0, min(min(per, p.NB_cap - j0), kPassRows)) : 0;
+  if (tid == 0) {
+    tc::mbar_init(&xbar[0], 1);
+    tc::mbar_init(&xbar[1], 1);
+    tc::mbar_init(&xbar[2], 1);
+    xabort = 0;
+    tc::fence_mbar_init();
+    if (staged_rows > 0) {
+      const uint32_t bytes = (uint32_t)(staged_rows * D * 4);
+      tc::mbar_arrive_expect_tx(&xbar[2], bytes);
+      tc::bulk_load(sumbuf, p.summ + (unit * (size_t)p.NB_cap + j0) * D, bytes, &xbar[2]);
     }
-    cp_async_commit();
   }
+  // DSMEM may be written only once every CTA of the cluster runs (and has initialised its
+  // barriers): arrive now, wait late
+  cluster_arrive_relaxed();
+  bool started = false;  // uniform: the start barrier has been waited on
 
   // ---- which blocks: forced / all known up front; order[i] is handled by CTA i % CL ----
   const bool all_blocks = select && NB <= p.topk;
@@ -277,10 +291,14 @@ __global__ void __launch_bounds__(kThreads, 2) decode_cluster_kernel(const Param
   const int nloc = scan ? max(0, min(NB, j0 + per) - j0) : 0;
   // while scanning, stage 1 holds the first pass of this CTA's summary rows
   const int early_stages = scan ? 1 : kStages;
+  // a short sequence that scans nothing reuses stage 1 once the summary copy has landed
+  // (the barrier makes thread 0's mbarrier initialisation visible first)
+  if (!scan && staged_rows > 0) {
+    __syncthreads();
+    tc::mbar_wait(&xbar[2], 0, &xabort, kWaitBudget);
+  }
   if (MODE == MODE_FUSED) {
     while (issued < early_stages && issued < n_known && known_block(issued) != NB - 1) {
-      // a short sequence that scans nothing reuses stage 1 once the summary copy has landed
-      if (may_scan && issued == 1) cp_async_wait<1>();
       unsigned char* st = kv + (size_t)(issued % kStages) * 2 * kv_tile;
       stage_block<T, D, kThreads>(st, st + kv_tile, kbase, vbase, known_block(issued), Tb, kv_row);
       cp_async_commit();
@@ -310,8 +328,6 @@ __global__ void __launch_bounds__(kThreads, 2) decode_cluster_kernel(const Param
   }
   if (MODE == MODE_FUSED && !scan) {
     while (issued < kStages && issued < n_known) {
-      // stage 1 is reused once the summary copy (two groups older) has landed
-      if (may_scan && issued == 1) cp_async_wait<2>();
       unsigned char* st = kv + (size_t)(issued % kStages) * 2 * kv_tile;
       stage_block<T, D, kThreads>(st, st + kv_tile, kbase, vbase, known_block(issued), Tb, kv_row);
       cp_async_commit();
@@ -321,7 +337,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_cluster_kernel(const Param
 
   // ---- selection --------------------------------------------------------------------
   if (scan) {
-    // the staged summary and query rows: only the newest block's copy may be in flight
+    // the staged query rows: only the newest block's copy may be in flight after them
     if (newest_issued) cp_async_wait<1>(); else cp_async_wait<0>();
     __syncthreads();
     const int m = p.topk - nf;
@@ -339,46 +355,58 @@ __global__ void __launch_bounds__(kThreads, 2) decode_cluster_kernel(const Param
       qsum[d] = acc * p.scale;
     }
     __syncthreads();
-    // kLanesPerRow threads per summary row, each a contiguous quarter of the row
-    constexpr int kSeg = D / kLanesPerRow;  // floats per thread
-    const int part = lane >> 3;
-    float qv[kSeg];
+    // the summary rows (the barriers above ordered thread 0's mbarrier initialisation first)
+    if (staged_rows > 0) tc::mbar_wait(&xbar[2], 0, &xabort, kWaitBudget);
+    // lane l of warp w scores rows 8w + (l >> 3) and 8w + 4 + (l >> 3) of a pass, taking
+    // 16-byte chunks cs, cs + 8, ... (cs = l & 7): a quarter-warp reads 128 contiguous bytes
+    // of one row (conflict-free), and every lane needs the same D / 8 summed-query values
+    // for both of its rows
+    constexpr int kCPL = D / 32;  // chunks of a row per lane
+    const int cs = lane & 7;
+    float qv[4 * kCPL];
 #pragma unroll
-    for (int k = 0; k < kSeg / 4; ++k) {
-      const float4 v = reinterpret_cast<const float4*>(qsum + part * kSeg)[k];
-      qv[4 * k] = v.x; qv[4 * k + 1] = v.y; qv[4 * k + 2] = v.z; qv[4 * k + 3] = v.w;
+    for (int m = 0; m < kCPL; ++m) {
+      const float4 v = reinterpret_cast<const float4*>(qsum)[cs + 8 * m];
+      qv[4 * m] = v.x; qv[4 * m + 1] = v.y; qv[4 * m + 2] = v.z; qv[4 * m + 3] = v.w;
     }
-    const float* grow = p.summ + (unit * (size_t)p.NB_cap + j0) * D + part * kSeg;
+    const float* grow = p.summ + (unit * (size_t)p.NB_cap + j0) * D;
     for (int base = 0; base < nloc; base += kPassRows) {  // uniform trip count
-      const int oo = base + warp * 8 + (lane & 7);
-      float a4[4] = {0.f, 0.f, 0.f, 0.f};
-      if (oo < nloc) {
+      float dot[2];
 #pragma unroll
-        for (int k = 0; k < kSeg / 4; ++k) {
-          float4 v;
-          if (base == 0) {  // staged (swizzled) first pass
-            const int c = part * (kSeg / 4) + k;
-            v = *reinterpret_cast<const float4*>(sumbuf + oo * D + ((c ^ (oo & 7)) << 2));
-          } else {
-            v = __ldg(reinterpret_cast<const float4*>(grow + (size_t)oo * D) + k);
-          }
-          a4[k & 3] = fmaf(v.x, qv[4 * k], a4[k & 3]);
-          a4[k & 3] = fmaf(v.y, qv[4 * k + 1], a4[k & 3]);
-          a4[k & 3] = fmaf(v.z, qv[4 * k + 2], a4[k & 3]);
-          a4[k & 3] = fmaf(v.w, qv[4 * k + 3], a4[k & 3]);
-        }
-      }
-      float dot = (a4[0] + a4[1]) + (a4[2] + a4[3]);
-      dot += __shfl_xor_sync(0xffffffffu, dot, 8);
-      dot += __shfl_xor_sync(0xffffffffu, dot, 16);
-      if (part == 0) {
+      for (int i = 0; i < 2; ++i) {
+        const int oo = base + warp * 8 + (lane >> 3) + 4 * i;
+        float a0 = 0.f, a1 = 0.f;
         if (oo < nloc) {
-          const int j = j0 + oo;
-          const bool forced = j < p.n_sink || j >= NB - p.n_local;
-          keys[oo] = forced ? 0ull : make_key(dot, j);
-          if (p.scores_out) p.scores_out[unit * p.NB_cap + j] = dot;
-        } else if (oo < kPassRows && oo < per) {
-          keys[oo] = 0ull;  // the rank count below reads a full pass
+#pragma unroll
+          for (int m = 0; m < kCPL; ++m) {
+            const float4 v = base == 0
+                ? reinterpret_cast<const float4*>(sumbuf + oo * D)[cs + 8 * m]
+                : __ldg(reinterpret_cast<const float4*>(grow + (size_t)oo * D) + cs + 8 * m);
+            a0 = fmaf(v.x, qv[4 * m], a0);
+            a1 = fmaf(v.y, qv[4 * m + 1], a1);
+            a0 = fmaf(v.z, qv[4 * m + 2], a0);
+            a1 = fmaf(v.w, qv[4 * m + 3], a1);
+          }
+        }
+        dot[i] = a0 + a1;
+      }
+#pragma unroll
+      for (int o = 1; o < 8; o <<= 1) {
+        dot[0] += __shfl_xor_sync(0xffffffffu, dot[0], o);
+        dot[1] += __shfl_xor_sync(0xffffffffu, dot[1], o);
+      }
+      if (cs == 0) {
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+          const int oo = base + warp * 8 + (lane >> 3) + 4 * i;
+          if (oo < nloc) {
+            const int j = j0 + oo;
+            const bool forced = j < p.n_sink || j >= NB - p.n_local;
+            keys[oo] = forced ? 0ull : make_key(dot[i], j);
+            if (p.scores_out) p.scores_out[unit * p.NB_cap + j] = dot[i];
+          } else if (oo < kPassRows && oo < per) {
+            keys[oo] = 0ull;  // the rank count below reads a full pass
+          }
         }
       }
     }
@@ -422,15 +450,16 @@ __global__ void __launch_bounds__(kThreads, 2) decode_cluster_kernel(const Param
     } else {
       block_topm(keys, nloc, m, top, work);
     }
-    // push the list into every peer (all[rank][*] on each CTA), then merge all lists
+    // push the list into every peer (all[rank][*] on each CTA), wait until all CL lists
+    // have landed here, then merge them
     cluster_wait();
     started = true;
+    if (tid == 0) tc::mbar_arrive_expect_tx(&xbar[0], (uint32_t)(CL * p.lp * 8));
     for (int t = tid; t < CL * p.lp; t += kThreads) {
       const int peer = t / p.lp, pos = t - peer * p.lp;
-      st_cluster(map_rank(all + rank * p.lp + pos, peer), top[pos]);
+      st_async(map_rank(all + rank * p.lp + pos, peer), top[pos], map_rank(&xbar[0], peer));
     }
-    cluster_arrive_release();
-    cluster_wait();
+    tc::mbar_wait(&xbar[0], 0, &xabort, kWaitBudget);
     const u64* fin = p.lp == 16 ? merge_lists<1>(all, work, CL)
                    : (p.lp == 32 ? merge_lists<2>(all, work, CL) : merge_lists<4>(all, work, CL));
     for (int r = tid; r < m; r += kThreads) order[nf + r] = key_block(fin[r]);
@@ -457,8 +486,9 @@ __global__ void __launch_bounds__(kThreads, 2) decode_cluster_kernel(const Param
   }
   if (MODE == MODE_SELECT) {
     cp_async_wait<0>();  // no copy into shared memory outlives the CTA
+    if (tid == 0 && xabort) g_decode_status = 1;
     if (!started) cluster_wait();
-    return;  // no CTA reads a peer's shared memory: no trailing barrier
+    return;  // every byte this CTA receives has landed: no trailing barrier
   }
 
   // ---- attention over my share of the blocks ------------------------------------------
@@ -642,14 +672,20 @@ __global__ void __launch_bounds__(kThreads, 2) decode_cluster_kernel(const Param
   }
   const int E = G * D;
   const int chunk = p.chunk;
-  if (ssub < CL) st_cluster(map_rank(ml_in + rank * kRows + srow, ssub), make_float2(m_run, l_run));
+  if (tid == 0) {  // from every CTA: kRows (m, l) pairs and this CTA's slice of the accumulator
+    const int own = max(0, min(E, (rank + 1) * chunk) - rank * chunk);
+    tc::mbar_arrive_expect_tx(&xbar[1], (uint32_t)(CL * (kRows * 8 + own * 4)));
+  }
+  if (ssub < CL)
+    st_async(map_rank(ml_in + rank * kRows + srow, ssub), make_float2(m_run, l_run), map_rank(&xbar[1], ssub));
   if constexpr (kF32) {
     if (srow < G) {
 #pragma unroll
       for (int e2 = 0; e2 < D / 16; ++e2) {
         const int e = srow * D + ssub + 16 * e2;
         const int owner = e / chunk;
-        st_cluster(map_rank(pacc_in + rank * chunk + (e - owner * chunk), owner), acc[e2][0]);
+        st_async(map_rank(pacc_in + rank * chunk + (e - owner * chunk), owner), acc[e2][0],
+                 map_rank(&xbar[1], owner));
       }
     }
   } else {
@@ -663,14 +699,14 @@ __global__ void __launch_bounds__(kThreads, 2) decode_cluster_kernel(const Param
         if (row < G) {
           const int e = row * D + d;
           const int owner = e / chunk;
-          st_cluster(map_rank(pacc_in + rank * chunk + (e - owner * chunk), owner),
-                     make_float2(acc[nt][2 * half], acc[nt][2 * half + 1]));
+          st_async(map_rank(pacc_in + rank * chunk + (e - owner * chunk), owner),
+                   make_float2(acc[nt][2 * half], acc[nt][2 * half + 1]), map_rank(&xbar[1], owner));
         }
       }
     }
   }
-  cluster_arrive_release();
-  cluster_wait();
+  tc::mbar_wait(&xbar[1], 0, &xabort, kWaitBudget);
+  if (tid == 0 && xabort) g_decode_status = 1;
 
   // ---- log-sum-exp merge of this CTA's slice, from its own shared memory ---------------
   {
@@ -791,6 +827,15 @@ cudaError_t launch_mode(const DecodeArgs& a, cudaStream_t s) {
 }
 
 }  // namespace
+
+cudaError_t read_decode_status(int* status, bool reset) {
+  cudaError_t err = cudaMemcpyFromSymbol(status, g_decode_status, sizeof(int));
+  if (err == cudaSuccess && reset) {
+    const int zero = 0;
+    err = cudaMemcpyToSymbol(g_decode_status, &zero, sizeof(int));
+  }
+  return err;
+}
 
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream) {
   if (a.B == 0 || a.Hkv == 0) return cudaSuccess;

@@ -216,7 +216,13 @@ int lsa_blasst_prefill(const void* q, const void* k, const void* v, int dtype, i
 
 int lsa_device_status(int* status, int reset) {
   if (!status) return LSA_ERR_INVALID_ARG;
-  return cuda_status(lsa::read_device_status(status, reset != 0));
+  int prefill = 0, decode = 0;
+  int st = cuda_status(lsa::read_device_status(&prefill, reset != 0));
+  if (st != LSA_OK) return st;
+  st = cuda_status(lsa::read_decode_status(&decode, reset != 0));
+  if (st != LSA_OK) return st;
+  *status = prefill | decode;
+  return LSA_OK;
 }
 
 }  // extern "C"

@@ -76,6 +76,7 @@ struct PrefillArgs {
 };
 cudaError_t launch_blasst_prefill(const PrefillArgs& a, cudaStream_t stream);
 cudaError_t read_device_status(int* status, bool reset);
+cudaError_t read_decode_status(int* status, bool reset);
 
 // The fixed device scratch used by lsa_sparse_attn_blockquery_noalloc.
 size_t blockquery_static_workspace_bytes();

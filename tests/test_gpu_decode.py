@@ -167,6 +167,7 @@ def _run_both_modes(lsa, case, dtype, check_sel=True):
             for g in range(Hkv):
                 check_selection(idx2c[b, g], r["scores"][b, g], NB, topk, ns, nl, f"fused b{b}g{g}")
     _check_attention(case, o2, lse2, idx2c, dtype, "fused")
+    assert lsa.lsa_device_status() == 0, "a bounded cross-CTA wait ran out"
     return r, idx2c
 
 
