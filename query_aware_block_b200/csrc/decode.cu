@@ -191,6 +191,33 @@ __device__ const u64* merge_lists(u64* lists, u64* work, int CL) {
   return src;
 }
 
+// Global top list of the union of CL (a power of two, 2..16) descending lists of 16 keys
+// at lists[c * 16] (zero padded), as a tree of warp-wide bitonic merges: warp w first
+// merges lists 2w and 2w + 1; at each later level a warp keeps its result in registers and
+// takes its partner warp's from shared memory after a pairwise named barrier (ids 1..7, one
+// per producing warp), so no level waits for the whole block.  Writes order[nf + r] for
+// r < m (m <= 16) from warp 0; the caller synchronises the block afterwards.
+__device__ __forceinline__ void merge_tree16(const u64* lists, u64* work, int CL, int m, int nf, int* order) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int npairs = CL >> 1;
+  if (warp >= npairs) return;
+  u64 x[1];
+  x[0] = lane < 16 ? lists[(2 * warp) * 16 + lane] : lists[(2 * warp + 1) * 16 + 31 - lane];
+  warp_merge_desc<1>(x);
+  for (int s = 1; s < npairs; s <<= 1) {
+    if (warp & s) {  // producer at this level: hand the top 16 to warp - s and leave
+      if (lane < 16) work[warp * 16 + lane] = x[0];
+      asm volatile("bar.arrive %0, 64;" ::"r"(warp) : "memory");
+      return;
+    }
+    if (warp + s >= npairs) continue;  // no partner at this level
+    asm volatile("bar.sync %0, 64;" ::"r"(warp + s) : "memory");
+    if (lane >= 16) x[0] = work[(warp + s) * 16 + 31 - lane];
+    warp_merge_desc<1>(x);
+  }
+  if (lane < m) order[nf + lane] = key_block(x[0]);
+}
+
 // ---- the kernel ---------------------------------------------------------------------
 
 template <typename T, int D, int MODE>
@@ -460,9 +487,13 @@ __global__ void __launch_bounds__(kThreads, 2) decode_cluster_kernel(const Param
       st_async(map_rank(all + rank * p.lp + pos, peer), top[pos], map_rank(&xbar[0], peer));
     }
     tc::mbar_wait(&xbar[0], 0, &xabort, kWaitBudget);
-    const u64* fin = p.lp == 16 ? merge_lists<1>(all, work, CL)
-                   : (p.lp == 32 ? merge_lists<2>(all, work, CL) : merge_lists<4>(all, work, CL));
-    for (int r = tid; r < m; r += kThreads) order[nf + r] = key_block(fin[r]);
+    if (p.lp == 16 && CL >= 2) {
+      merge_tree16(all, work, CL, m, nf, order);
+    } else {
+      const u64* fin = p.lp == 16 ? merge_lists<1>(all, work, CL)
+                     : (p.lp == 32 ? merge_lists<2>(all, work, CL) : merge_lists<4>(all, work, CL));
+      for (int r = tid; r < m; r += kThreads) order[nf + r] = key_block(fin[r]);
+    }
   }
   __syncthreads();
 
@@ -655,8 +686,8 @@ __global__ void __launch_bounds__(kThreads, 2) decode_cluster_kernel(const Param
         p.summ_w[(unit * p.NB_cap + j) * D + d] = s / (float)n;
       }
     }
-    __syncthreads();  // the stage may now be refilled
     if (issued < n_my) {
+      __syncthreads();  // the stage may now be refilled
       unsigned char* st = kv + (size_t)(issued % kStages) * 2 * kv_tile;
       stage_block<T, D, kThreads>(st, st + kv_tile, kbase, vbase, order[rank + issued * CL], Tb, kv_row);
       cp_async_commit();
