@@ -45,7 +45,7 @@ import torch  # noqa: E402
 METRIC = "64K-ctx sparse decode tokens/s and effective KV GB/s (% of B200 HBM roofline)"
 UNIT = "tokens/s"
 KERNEL_SOURCES = ["query_aware_block_b200/csrc/decode.cu", "query_aware_block_b200/csrc/lsa_common.cuh",
-                  "query_aware_block_b200/csrc/cluster.cuh"]
+                  "query_aware_block_b200/csrc/cluster.cuh", "query_aware_block_b200/csrc/tcgen05.cuh"]
 PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "decode_fused_gqa_decode_64k.md")
 
 WORKLOADS = {

@@ -69,7 +69,10 @@ constexpr int kSStride = 72;    // fp32 row stride of the score tile (bank sprea
 // gives each key 4 threads (lane l of warp w: key 8w + (l & 7), quarter l >> 3 of the keys).
 constexpr int kPassRows = kWarps * 8;
 
-struct Params {
+struct alignas(64) Params {
+  // bf16 K and V as [B * Hkv][T_cap][D], box {64, 64, 1}, 128-byte swizzle (unused for fp32)
+  CUtensorMap tmk;
+  CUtensorMap tmv;
   const void* q;
   const void* k;
   const void* v;
@@ -94,6 +97,13 @@ struct Params {
 
 __host__ __device__ inline size_t align128(size_t x) { return (x + 127) & ~(size_t)127; }
 
+// Byte offset of 16-byte chunk c of row r in a bf16 K/V tile of 64 rows: [c / 8][r][128 B]
+// with the chunk index XOR-swizzled by (r & 7), i.e. where 128-byte-swizzled TMA boxes of
+// 64 elements x 64 rows land; ldmatrix over 8 consecutive rows is conflict-free.
+__device__ __forceinline__ int kv_off(int r, int c) {
+  return ((c >> 3) << 13) + (r << 7) + ((((c & 7) ^ (r & 7))) << 4);
+}
+
 // Shared-memory carve-up (byte offsets), identical on host and device.
 struct Layout {
   size_t qs, qsum, keys, top, work, all, order, kv, ss, ps, alpha, ml_in, pacc_in, total;
@@ -115,7 +125,9 @@ __host__ __device__ inline Layout make_layout(int elem_bytes, int D, int per_max
   L.work = off;    off = align128(off + (size_t)nwork * 8);
   L.all = off;     off = align128(off + (size_t)kMaxCluster * lp * 8);
   L.order = off;   off = align128(off + (size_t)kMaxTopk * 4);
-  L.kv = off;      off = align128(off + (size_t)kStages * 2 * L.kv_tile);
+  // (the K/V ring is placed at the first 1024-byte boundary inside this range: a 128-byte
+  // swizzled TMA box must land 1024-byte aligned)
+  L.kv = off;      off = align128(off + (size_t)kStages * 2 * L.kv_tile + 1024);
   L.ss = off;      off = align128(off + (size_t)kRows * kSStride * 4);
   L.ps = off;      off = align128(off + (size_t)kRows * kBlk * 4);
   L.alpha = off;   off = align128(off + (size_t)kRows * 4);
@@ -221,7 +233,7 @@ __device__ __forceinline__ void merge_tree16(const u64* lists, u64* work, int CL
 // ---- the kernel ---------------------------------------------------------------------
 
 template <typename T, int D, int MODE>
-__global__ void __launch_bounds__(kThreads, 2) decode_cluster_kernel(const Params p) {
+__global__ void __launch_bounds__(kThreads, 2) decode_cluster_kernel(const __grid_constant__ Params p) {
   // the parameter block is fetched all at once here (fields spaced < 32 bytes apart), not
   // one constant-cache miss after another on first use
   asm volatile("" ::"l"(p.q), "r"(p.T_cap), "l"(p.summ_w), "r"(p.topk), "l"(p.nsel_out), "l"(p.lse),
@@ -236,9 +248,10 @@ __global__ void __launch_bounds__(kThreads, 2) decode_cluster_kernel(const Param
   constexpr bool kF32 = sizeof(T) == 4;
   constexpr int kRowBytesQ = D * (int)sizeof(T);
 
-  // mbarriers, one phase each: [0] and [1] count the bytes of the two cross-CTA exchanges,
-  // [2] the bulk copy of this CTA's summary rows
-  __shared__ __align__(8) uint64_t xbar[3];
+  // mbarriers: [0] and [1] count the bytes of the two cross-CTA exchanges and [2] the bulk
+  // copy of this CTA's summary rows (one phase each); [3 + s] the TMA loads into K/V stage s
+  // (bf16; one phase per use of the stage)
+  __shared__ __align__(8) uint64_t xbar[3 + kStages];
   __shared__ int xabort;
   extern __shared__ __align__(1024) unsigned char smem[];
   const Layout Lo = make_layout((int)sizeof(T), D, p.per_max, p.m_pad);
@@ -248,7 +261,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_cluster_kernel(const Param
   u64* work = reinterpret_cast<u64*>(smem + Lo.work);
   u64* all = reinterpret_cast<u64*>(smem + Lo.all);
   int* order = reinterpret_cast<int*>(smem + Lo.order);
-  unsigned char* kv = smem + Lo.kv;
+  unsigned char* kv = smem + Lo.kv + ((1024u - ((tc::smem_u32(smem) + (uint32_t)Lo.kv) & 1023u)) & 1023u);
   float* Ss = reinterpret_cast<float*>(smem + Lo.ss);
   unsigned char* Ps = smem + Lo.ps;
   float* alpha_s = reinterpret_cast<float*>(smem + Lo.alpha);
@@ -276,8 +289,13 @@ __global__ void __launch_bounds__(kThreads, 2) decode_cluster_kernel(const Param
     tc::mbar_init(&xbar[0], 1);
     tc::mbar_init(&xbar[1], 1);
     tc::mbar_init(&xbar[2], 1);
+    for (int st = 0; st < kStages; ++st) tc::mbar_init(&xbar[3 + st], 1);
     xabort = 0;
     tc::fence_mbar_init();
+    if constexpr (!kF32) {
+      tc::prefetch_tmap(&p.tmk);
+      tc::prefetch_tmap(&p.tmv);
+    }
     if (staged_rows > 0) {
       const uint32_t bytes = (uint32_t)(staged_rows * D * 4);
       tc::mbar_arrive_expect_tx(&xbar[2], bytes);
@@ -311,7 +329,34 @@ __global__ void __launch_bounds__(kThreads, 2) decode_cluster_kernel(const Param
   // ---- before waiting on the previous kernel of the stream: copies of data that kernel
   // cannot have written (the K/V of the known blocks except the sequence's newest one, and
   // the summary rows above).  With overlapped launch the caller vouches for this.
-  int issued = 0;  // my blocks whose copies were committed, in processing order
+  int issued = 0;  // my blocks whose copies were started, in processing order
+  // Start the copy of block j's K and V into stage issued % kStages (every thread calls
+  // this).  bf16: TMA boxes issued by thread 0 that land on the stage's mbarrier; fp32:
+  // 16-byte cp.async by every thread, one commit group per block.
+  auto issue_block = [&](int j) {
+    const int stg = issued % kStages;
+    unsigned char* st = kv + (size_t)stg * 2 * kv_tile;
+    if constexpr (kF32) {
+      stage_block<T, D, kThreads>(st, st + kv_tile, kbase, vbase, j, Tb, kv_row);
+      cp_async_commit();
+    } else {
+      if (tid == 0) {
+        tc::fence_proxy_async();  // earlier generic accesses to this stage come first
+        uint64_t* bar = &xbar[3 + stg];
+        if (j >= 0) {
+          tc::mbar_arrive_expect_tx(bar, (uint32_t)(2 * kv_tile));
+#pragma unroll
+          for (int h = 0; h < D / 64; ++h) {
+            tc::tma_load_3d(st + h * 8192, &p.tmk, h * 64, j * kBlk, (int)unit, bar);
+            tc::tma_load_3d(st + kv_tile + h * 8192, &p.tmv, h * 64, j * kBlk, (int)unit, bar);
+          }
+        } else {
+          tc::mbar_arrive(bar);  // nothing to copy: the phase completes empty
+        }
+      }
+    }
+    ++issued;
+  };
   const int known = all_blocks ? NB : nf;
   const int n_known = (MODE == MODE_FUSED && known > rank) ? (known - rank + CL - 1) / CL : 0;
   const bool scan = select && !all_blocks;
@@ -326,10 +371,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_cluster_kernel(const Param
   }
   if (MODE == MODE_FUSED) {
     while (issued < early_stages && issued < n_known && known_block(issued) != NB - 1) {
-      unsigned char* st = kv + (size_t)(issued % kStages) * 2 * kv_tile;
-      stage_block<T, D, kThreads>(st, st + kv_tile, kbase, vbase, known_block(issued), Tb, kv_row);
-      cp_async_commit();
-      ++issued;
+      issue_block(known_block(issued));
     }
   }
   pdl_trigger();
@@ -348,24 +390,19 @@ __global__ void __launch_bounds__(kThreads, 2) decode_cluster_kernel(const Param
   const int issued_before_q = issued;
   bool newest_issued = false;
   if (MODE == MODE_FUSED && scan && issued == 0 && n_known > 0) {  // the newest block, now
-    stage_block<T, D, kThreads>(kv, kv + kv_tile, kbase, vbase, known_block(0), Tb, kv_row);
-    cp_async_commit();
-    ++issued;
+    issue_block(known_block(0));
     newest_issued = true;
   }
   if (MODE == MODE_FUSED && !scan) {
     while (issued < kStages && issued < n_known) {
-      unsigned char* st = kv + (size_t)(issued % kStages) * 2 * kv_tile;
-      stage_block<T, D, kThreads>(st, st + kv_tile, kbase, vbase, known_block(issued), Tb, kv_row);
-      cp_async_commit();
-      ++issued;
+      issue_block(known_block(issued));
     }
   }
 
   // ---- selection --------------------------------------------------------------------
   if (scan) {
     // the staged query rows: only the newest block's copy may be in flight after them
-    if (newest_issued) cp_async_wait<1>(); else cp_async_wait<0>();
+    if (kF32 && newest_issued) cp_async_wait<1>(); else cp_async_wait<0>();
     __syncthreads();
     const int m = p.topk - nf;
     // summed, scaled query row of the group (fp32, shared), from the staged query rows
@@ -497,8 +534,10 @@ __global__ void __launch_bounds__(kThreads, 2) decode_cluster_kernel(const Param
   }
   __syncthreads();
 
-  // selected indices, ascending (written by rank 0)
-  if (select && rank == 0) {
+  // selected indices, ascending (written by rank 0; in fused mode after its attention
+  // copies have been started)
+  auto write_indices = [&]() {
+    if (!(select && rank == 0)) return;
     int32_t* out = p.idx_out ? p.idx_out + unit * p.topk : nullptr;
     if (out) {
       for (int i = tid; i < p.topk; i += kThreads) {
@@ -514,7 +553,8 @@ __global__ void __launch_bounds__(kThreads, 2) decode_cluster_kernel(const Param
       }
     }
     if (MODE == MODE_SELECT && tid == 0) p.nsel_out[unit] = n_order;
-  }
+  };
+  if (MODE == MODE_SELECT) write_indices();
   if (MODE == MODE_SELECT) {
     cp_async_wait<0>();  // no copy into shared memory outlives the CTA
     if (tid == 0 && xabort) g_decode_status = 1;
@@ -524,14 +564,10 @@ __global__ void __launch_bounds__(kThreads, 2) decode_cluster_kernel(const Param
 
   // ---- attention over my share of the blocks ------------------------------------------
   const int n_my = n_order > rank ? (n_order - rank + CL - 1) / CL : 0;
-  while (issued < kStages && issued < n_my) {
-    unsigned char* st = kv + (size_t)(issued % kStages) * 2 * kv_tile;
-    stage_block<T, D, kThreads>(st, st + kv_tile, kbase, vbase, order[rank + issued * CL], Tb, kv_row);
-    cp_async_commit();
-    ++issued;
-  }
-  if (!scan) {  // the query rows' copy, followed by at most kStages block copies
-    const int after_q = issued - issued_before_q;
+  while (issued < kStages && issued < n_my) issue_block(order[rank + issued * CL]);
+  if (MODE == MODE_FUSED) write_indices();
+  if (!scan) {  // the query rows' copy, followed (fp32) by at most kStages block copies
+    const int after_q = kF32 ? issued - issued_before_q : 0;
     if (after_q >= 2) cp_async_wait<2>(); else if (after_q == 1) cp_async_wait<1>(); else cp_async_wait<0>();
   }
   __syncthreads();  // (the staged query rows are visible)
@@ -560,11 +596,25 @@ __global__ void __launch_bounds__(kThreads, 2) decode_cluster_kernel(const Param
   }
 
   for (int i = 0; i < n_my; ++i) {
-    if (issued > i + 1) cp_async_wait<1>(); else cp_async_wait<0>();
+    if constexpr (kF32) {
+      if (issued > i + 1) cp_async_wait<1>(); else cp_async_wait<0>();
+    } else {
+      tc::mbar_wait(&xbar[3 + i % kStages], (uint32_t)((i / kStages) & 1), &xabort, kWaitBudget);
+    }
     __syncthreads();
     const int j = order[rank + i * CL];
     const unsigned char* Ks = kv + (size_t)(i % kStages) * 2 * kv_tile;
     const unsigned char* Vs = Ks + kv_tile;
+    if constexpr (!kF32) {
+      // V rows past the sequence (or all rows of an invalid j) hold whatever the cache
+      // holds there: zero them, so that P = 0 never meets a NaN (ordered before P V by the
+      // barrier after S)
+      const int nv = j < 0 ? 0 : min(kBlk, Tb - j * kBlk);
+      for (int id = tid; id < (kBlk - nv) * (D / 8); id += kThreads) {
+        const int r = nv + id / (D / 8), c = id % (D / 8);
+        *reinterpret_cast<uint4*>(const_cast<unsigned char*>(Vs) + kv_off(r, c)) = make_uint4(0u, 0u, 0u, 0u);
+      }
+    }
 
     // S = scale2 * Q K^T (masked past Tb) -> Ss
     if constexpr (kF32) {
@@ -589,7 +639,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_cluster_kernel(const Param
 #pragma unroll
       for (int ks = 0; ks < D / 16; ks += 2) {
         uint32_t kb[4];
-        ldsm_x4(kb, Ks + swz(8 * warp + (lane & 7), 2 * ks + (lane >> 3), kv_row));
+        ldsm_x4(kb, Ks + kv_off(8 * warp + (lane & 7), 2 * ks + (lane >> 3)));
         mma_bf16(s, qa[ks], kb[0], kb[1]);
         mma_bf16(s, qa[ks + 1], kb[2], kb[3]);
       }
@@ -659,12 +709,12 @@ __global__ void __launch_bounds__(kThreads, 2) decode_cluster_kernel(const Param
         const int vrow = 16 * ks + (lane & 7) + 8 * ((lane >> 3) & 1);
         if constexpr (D == 128) {
           uint32_t vb[4];
-          ldsm_x4_t(vb, Vs + swz(vrow, 2 * warp + (lane >> 4), kv_row));
+          ldsm_x4_t(vb, Vs + kv_off(vrow, 2 * warp + (lane >> 4)));
           mma_bf16(acc[0], pa, vb[0], vb[1]);
           mma_bf16(acc[1], pa, vb[2], vb[3]);
         } else {
           uint32_t vb[2];
-          ldsm_x2_t(vb, Vs + swz(vrow, warp, kv_row));
+          ldsm_x2_t(vb, Vs + kv_off(vrow, warp));
           mma_bf16(acc[0], pa, vb[0], vb[1]);
         }
       }
@@ -681,17 +731,14 @@ __global__ void __launch_bounds__(kThreads, 2) decode_cluster_kernel(const Param
           const int c = d >> 3, wd = d & 7;
 #pragma unroll 8
           for (int t = 0; t < n; ++t)
-            s += __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(Ks + swz(t, c, kv_row))[wd]);
+            s += __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(Ks + kv_off(t, c))[wd]);
         }
         p.summ_w[(unit * p.NB_cap + j) * D + d] = s / (float)n;
       }
     }
     if (issued < n_my) {
       __syncthreads();  // the stage may now be refilled
-      unsigned char* st = kv + (size_t)(issued % kStages) * 2 * kv_tile;
-      stage_block<T, D, kThreads>(st, st + kv_tile, kbase, vbase, order[rank + issued * CL], Tb, kv_row);
-      cp_async_commit();
-      ++issued;
+      issue_block(order[rank + issued * CL]);
     }
   }
 
@@ -776,6 +823,30 @@ __global__ void __launch_bounds__(kThreads, 2) decode_cluster_kernel(const Param
 
 // ---- host side --------------------------------------------------------------------------
 
+// The K and V tensor maps of the last bf16 call on this host thread: a decode loop calls
+// with the same cache tensors every step, so the maps are encoded once.
+struct MapCache {
+  const void* k = nullptr;
+  const void* v = nullptr;
+  int D = 0, T_cap = 0, planes = 0;
+  CUtensorMap mk, mv;
+};
+
+bool kv_maps(const DecodeArgs& a, CUtensorMap* mk, CUtensorMap* mv) {
+  static thread_local MapCache c;
+  const int planes = a.B * a.Hkv;
+  if (!(c.k == a.k && c.v == a.v && c.D == a.D && c.T_cap == a.T_cap && c.planes == planes)) {
+    c.k = nullptr;
+    if (!encode_rows_bf16(&c.mk, a.k, a.D, a.T_cap, planes, kBlk) ||
+        !encode_rows_bf16(&c.mv, a.v, a.D, a.T_cap, planes, kBlk))
+      return false;
+    c.k = a.k; c.v = a.v; c.D = a.D; c.T_cap = a.T_cap; c.planes = planes;
+  }
+  *mk = c.mk;
+  *mv = c.mv;
+  return true;
+}
+
 int next_pow2(int x) {
   int p = 1;
   while (p < x) p <<= 1;
@@ -788,7 +859,8 @@ cudaError_t launch_t(const DecodeArgs& a, cudaStream_t stream) {
   // cluster size: many CTAs per unit when there are few units
   const int units = a.B * a.Hkv;
   int CL = units <= 18 ? 16 : (units <= 74 ? 8 : 4);
-  Params p;
+  Params p{};
+  if (sizeof(T) == 2 && MODE != MODE_SELECT && !kv_maps(a, &p.tmk, &p.tmv)) return cudaErrorInvalidValue;
   p.q = a.q; p.k = a.k; p.v = a.v;
   p.Hkv = a.Hkv; p.G = a.G; p.T_cap = a.T_cap; p.NB_cap = a.NB_cap;
   p.seqlens = a.seqlens; p.summ = a.summ; p.summ_w = a.summ_w;

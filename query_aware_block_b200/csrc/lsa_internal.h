@@ -1,6 +1,7 @@
 // lsa_internal.h -- launchers behind the C ABI (host side, not exported).
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -77,6 +78,11 @@ struct PrefillArgs {
 cudaError_t launch_blasst_prefill(const PrefillArgs& a, cudaStream_t stream);
 cudaError_t read_device_status(int* status, bool reset);
 cudaError_t read_decode_status(int* status, bool reset);
+
+// 3-D TMA map over a row-major bf16 tensor [planes][rows][D]: box {64, box_rows, 1} (one
+// 128-byte swizzled row segment per box row), rows past `rows` read as zero.  False when
+// the driver entry point is missing or rejects the map.
+bool encode_rows_bf16(CUtensorMap* map, const void* base, int D, int rows, int planes, int box_rows);
 
 // The fixed device scratch used by lsa_sparse_attn_blockquery_noalloc.
 size_t blockquery_static_workspace_bytes();
