@@ -33,11 +33,17 @@
 #include "cluster.cuh"
 #include "lsa_common.cuh"
 #include "lsa_internal.h"
+#include "tcgen05.cuh"
 
 namespace lsa {
 namespace {
 
 typedef unsigned long long u64;
+
+// Set when a bounded wait on a cross-CTA exchange or a bulk copy runs out (the launch's
+// outputs are then undefined); read and cleared by the host.
+__device__ int g_blockquery_status = 0;
+constexpr long long kWaitBudget = 4000000000LL;  // clock cycles (about 2 s)
 
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
@@ -48,8 +54,15 @@ constexpr int kMaxCluster = 16;
 constexpr int kMaxTq = 64;
 constexpr int kStages = 2;
 constexpr int kSStride = 68;    // fp32 row stride of the score tile
+constexpr int kQStride = 132;   // fp32 row stride of the summed queries (bank spread)
+constexpr int kStageRows = 64;  // summary rows of a CTA's slice staged by one bulk copy
+constexpr int kMaxUnion = kMaxTq * kLP;  // a union holds at most Tq * topk blocks
+static_assert(kTokChunk == 8, "the scoring maps lane l to token l & 7");
 
-struct BQParams {
+struct alignas(64) BQParams {
+  // K and V as [B * Hkv][T_cap][D], box {64, 64, 1}, 128-byte swizzle
+  CUtensorMap tmk;
+  CUtensorMap tmv;
   const __nv_bfloat16* q;
   const __nv_bfloat16* k;
   const __nv_bfloat16* v;
@@ -67,62 +80,64 @@ struct BQParams {
   float* ws;       // [B][Hkv][kMaxCluster][rows_max][D + 2]
   int rows_max;    // Tq * G
   int per_max;     // max prefix blocks in one CTA's slice
+  int NBp;         // prefix blocks
+  FastDiv g_div;   // division by G
+  FastDiv per_div; // division by per_max
 };
 
 __host__ __device__ inline size_t al128(size_t x) { return (x + 127) & ~(size_t)127; }
 
 struct BQLayout {
-  size_t act, stab, ulist, cnt_in, thr, qs, ss, ps, alpha, region, total;
+  size_t act, stab, ulist, ubits, qs, ss, ps, alpha, region, total;
   // selection buffers, inside `region` (dead once the attention starts)
-  size_t qsum, keys, top, recv, work, inu;
+  size_t qsum, keys, top, recv, work, sumbuf, qrows;
   size_t kv_tile;
 };
 
-__host__ __device__ inline BQLayout bq_layout(int D, int per_max) {
+__host__ __device__ inline BQLayout bq_layout(int D, int per_max, int NBp, int G) {
   BQLayout L;
   size_t off = 0;
+  const int ucap = NBp < kMaxUnion ? NBp : kMaxUnion;
+  const int stage_rows = per_max < kStageRows ? per_max : kStageRows;
   L.act = off;    off = al128(off + kMaxTq * 4);
   L.stab = off;   off = al128(off + kMaxTq * 4);
-  L.ulist = off;  off = al128(off + (size_t)per_max * 4);
-  L.cnt_in = off; off = al128(off + kMaxCluster * 4);
-  L.thr = off;    off = al128(off + kTokChunk * 8);
+  L.ulist = off;  off = al128(off + (size_t)(ucap > 0 ? ucap : 1) * 4);
+  L.ubits = off;  off = al128(off + (size_t)((NBp + 31) / 32 + 1) * 4);
   L.qs = off;     off = al128(off + (size_t)kRowChunk * D * 2);
   L.ss = off;     off = al128(off + (size_t)kRowChunk * kSStride * 4);
   L.ps = off;     off = al128(off + (size_t)kRowChunk * kBlk * 2);
   L.alpha = off;  off = al128(off + kRowChunk * 4);
   L.region = off;
   L.kv_tile = (size_t)kBlk * D * 2;
-  const size_t kv_bytes = kStages * 2 * L.kv_tile;
+  // the K/V ring starts at the first 1024-byte boundary of the region (TMA 128-byte swizzle)
+  const size_t kv_bytes = kStages * 2 * L.kv_tile + 1024;
   size_t r = 0;
-  L.qsum = r; r = al128(r + (size_t)kTokChunk * D * 4);
+  L.qsum = r; r = al128(r + (size_t)kTokChunk * kQStride * 4);
   L.keys = r; r = al128(r + (size_t)kTokChunk * per_max * 8);
   L.top = r;  r = al128(r + (size_t)kTokChunk * kLP * 8);
-  L.recv = r; r = al128(r + (size_t)kMaxCluster * kTokChunk * kLP * 8);
+  L.recv = r; r = al128(r + (size_t)2 * kMaxCluster * kTokChunk * kLP * 8);  // two buffers
   L.work = r; r = al128(r + (size_t)kTokChunk * (kMaxCluster / 2) * kLP * 8);
-  L.inu = r;  r = al128(r + (size_t)per_max);
+  L.sumbuf = r; r = al128(r + (size_t)stage_rows * D * 4);
+  L.qrows = r; r = al128(r + (size_t)kTokChunk * G * D * 2);  // a token chunk's query rows
   L.total = off + (r > kv_bytes ? r : kv_bytes);
   return L;
 }
 
 template <int D>
-__global__ void __launch_bounds__(kThreads, 2) blockquery_kernel(const BQParams p) {
+__global__ void __launch_bounds__(kThreads, 2) blockquery_kernel(const __grid_constant__ BQParams p) {
   const int CL = cluster_size();
   const int rank = cluster_rank();
-  cluster_arrive_relaxed();  // DSMEM is written only after every CTA has started
-  bool started = false;
-
   const int g = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int G = p.G, Tq = p.Tq, Hq = p.Hkv * G;
   const size_t unit = (size_t)b * p.Hkv + g;
 
   extern __shared__ __align__(1024) unsigned char smem[];
-  const BQLayout Lo = bq_layout(D, p.per_max);
+  const BQLayout Lo = bq_layout(D, p.per_max, p.NBp, p.G);
   int* act = reinterpret_cast<int*>(smem + Lo.act);
   int* stab = reinterpret_cast<int*>(smem + Lo.stab);
   int* ulist = reinterpret_cast<int*>(smem + Lo.ulist);
-  int* cnt_in = reinterpret_cast<int*>(smem + Lo.cnt_in);
-  u64* thr = reinterpret_cast<u64*>(smem + Lo.thr);
+  uint32_t* ubits = reinterpret_cast<uint32_t*>(smem + Lo.ubits);
   unsigned char* Qs = smem + Lo.qs;
   float* Ss = reinterpret_cast<float*>(smem + Lo.ss);
   unsigned char* Ps = smem + Lo.ps;
@@ -133,10 +148,37 @@ __global__ void __launch_bounds__(kThreads, 2) blockquery_kernel(const BQParams 
   u64* top = reinterpret_cast<u64*>(region + Lo.top);
   u64* recv = reinterpret_cast<u64*>(region + Lo.recv);
   u64* work = reinterpret_cast<u64*>(region + Lo.work);
-  unsigned char* inu = region + Lo.inu;
-  unsigned char* kv = region;
+  float* sumbuf = reinterpret_cast<float*>(region + Lo.sumbuf);
+  unsigned char* qrows = region + Lo.qrows;
+  unsigned char* kv = region + ((1024u - (tc::smem_u32(region) & 1023u)) & 1023u);
   const int kv_tile = (int)Lo.kv_tile;
   constexpr int kRowBytes = D * 2;
+
+  const int NBp = p.NBp;
+  const int per = p.per_max;
+  const int j0 = rank * per;
+  const int nloc = max(0, min(NBp, j0 + per) - j0);
+  const bool all_blocks = NBp <= p.topk;
+  // mbarriers: [0], [1] count the bytes of the candidate-list exchange (two buffers, one
+  // phase per token chunk that uses the buffer); [2] the bulk copy of the summary slice;
+  // [3 + s] the TMA loads into K/V stage s (one phase per use of the stage)
+  __shared__ __align__(8) uint64_t xbar[3 + kStages];
+  __shared__ int xabort;
+  const int staged_rows = all_blocks ? 0 : min(nloc, kStageRows);
+  if (tid == 0) {
+    for (int i = 0; i < 3 + kStages; ++i) tc::mbar_init(&xbar[i], 1);
+    xabort = 0;
+    tc::fence_mbar_init();
+    tc::prefetch_tmap(&p.tmk);
+    tc::prefetch_tmap(&p.tmv);
+    if (staged_rows > 0) {  // the slice's first summary rows, one bulk copy
+      const uint32_t bytes = (uint32_t)(staged_rows * D * 4);
+      tc::mbar_arrive_expect_tx(&xbar[2], bytes);
+      tc::bulk_load(sumbuf, p.summ + (unit * (size_t)p.NB_cap + j0) * D, bytes, &xbar[2]);
+    }
+  }
+  cluster_arrive_relaxed();  // DSMEM is written only after every CTA has started
+  bool started = false;
 
   // ---- active / stable token lists (ascending) ----------------------------------------
   __shared__ int counts[2];
@@ -160,103 +202,170 @@ __global__ void __launch_bounds__(kThreads, 2) blockquery_kernel(const BQParams 
   }
   __syncthreads();
   const int A = counts[0], S = counts[1];
-
-  const int NBp = (p.T_prefix + kBlk - 1) / kBlk;
-  const int per = (NBp + CL - 1) / CL;
-  const int j0 = rank * per;
-  const int nloc = max(0, min(NBp, j0 + per) - j0);
-  const bool all_blocks = NBp <= p.topk;
   const int nf = all_blocks ? 0 : p.n_sink + p.n_local;  // disjoint when NBp > topk
   const int m = p.topk - nf;
-  auto forced = [&](int j) { return j < p.n_sink || j >= NBp - p.n_local; };
+  const bool selecting = A > 0 && !all_blocks && m > 0;  // (m == 0: every slot is forced)
+  const int rows = A * G;
 
-  // ---- the union over this CTA's slice --------------------------------------------------
-  for (int i = tid; i < nloc; i += kThreads) inu[i] = (A > 0 && (all_blocks || forced(j0 + i))) ? 1 : 0;
+  // ---- query rows by cp.async, requested as soon as the active tokens are known: those of
+  // a token chunk (scoring) into qrows, those of an attention row chunk into Qs (row r is
+  // token act[r / G], head r % G; rows past the end are zero)
+  auto load_token_rows = [&](int tc0) {
+    const int na = min(kTokChunk, A - tc0);
+    constexpr int kC = kRowBytes / 16;
+    for (int id = tid; id < na * G * kC; id += kThreads) {
+      const int rr = id / kC, cc = id - rr * kC, a2 = fdiv(rr, p.g_div), hh = rr - a2 * G;
+      cp_async16(qrows + (size_t)rr * kRowBytes + cc * 16,
+                 p.q + (((size_t)b * Hq + (size_t)g * G + hh) * Tq + act[tc0 + a2]) * D + cc * 8, true);
+    }
+  };
+  auto load_attn_rows = [&](int c0) {
+    constexpr int kC = kRowBytes / 16;
+    for (int id = tid; id < kRowChunk * kC; id += kThreads) {
+      const int r = id / kC, cc = id - r * kC, rr = c0 + r;
+      const bool ok = rr < rows;
+      const int a2 = ok ? fdiv(rr, p.g_div) : 0, hh = ok ? rr - a2 * G : 0;
+      cp_async16(Qs + swz(r, cc, kRowBytes),
+                 p.q + (((size_t)b * Hq + (size_t)g * G + hh) * Tq + act[ok ? a2 : 0]) * D + cc * 8, ok);
+    }
+  };
+  if (A > 0) {
+    if (selecting) load_token_rows(0);
+    load_attn_rows(0);
+    cp_async_commit();
+  }
+
+  auto forced = [&](int j) { return j < p.n_sink || j >= NBp - p.n_local; };
+  const int nwords = (NBp + 31) / 32;
+
+  // ---- the union U(b, g) as a bitmap over the prefix blocks, the same on every CTA --------
+  for (int w = tid; w < nwords; w += kThreads) ubits[w] = 0u;
   __syncthreads();
-  if (A > 0 && !all_blocks && m > 0) {  // (m == 0: every slot is a forced block)
-    constexpr int VEC = D / 32;
-    const float* sb = p.summ + unit * (size_t)p.NB_cap * D + lane * VEC;
+  if (A > 0) {
+    for (int j = tid; j < NBp; j += kThreads)
+      if (all_blocks || forced(j)) atomicOr(&ubits[j >> 5], 1u << (j & 31));
+  }
+  if (selecting) {
+    if (staged_rows > 0) tc::mbar_wait(&xbar[2], 0, &xabort, kWaitBudget);
+    constexpr int kSeg = D / 4;  // summary floats per lane: lane l takes quarter l >> 3
+    const int ta = lane & 7, q4 = lane >> 3;
+    const float* grow = p.summ + (unit * (size_t)p.NB_cap + j0) * D + q4 * kSeg;
     for (int tc0 = 0; tc0 < A; tc0 += kTokChunk) {
+      const int chunk_id = tc0 / kTokChunk, buf = chunk_id & 1;
       const int na = min(kTokChunk, A - tc0);
-      // summed, scaled queries of the chunk's tokens
-      for (int i = tid; i < na * D; i += kThreads) {
-        const int a = i / D, d = i - a * D;
-        const __nv_bfloat16* qrow = p.q + (((size_t)b * Hq + (size_t)g * G) * Tq + act[tc0 + a]) * D + d;
-        float s = 0.f;
-        for (int h = 0; h < G; ++h) s += __bfloat162float(qrow[(size_t)h * Tq * D]);
-        qsum[a * D + d] = s * p.scale;
+      if (tc0 > 0) {
+        load_token_rows(tc0);
+        cp_async_commit();
+      }
+      cp_async_wait<0>();
+      __syncthreads();
+      // summed, scaled queries of the chunk's tokens (rows past na are zero)
+      for (int i = tid; i < kTokChunk * D; i += kThreads) {
+        const int a2 = i / D, d = i - a2 * D;
+        float sum = 0.f;
+        if (a2 < na) {
+          const __nv_bfloat16* qr = reinterpret_cast<const __nv_bfloat16*>(qrows) + (size_t)a2 * G * D + d;
+          for (int h = 0; h < G; ++h) sum += __bfloat162float(qr[(size_t)h * D]);
+        }
+        qsum[a2 * kQStride + d] = sum * p.scale;
       }
       for (int i = tid; i < kTokChunk * kLP; i += kThreads) top[i] = 0ull;
       __syncthreads();
-      // scores of the slice for every token: a warp per summary row, 8 rows in flight
-      constexpr int kRowsPerWarp = 8;
-      for (int o0 = warp; o0 < nloc; o0 += kWarps * kRowsPerWarp) {
-        float vals[kRowsPerWarp][VEC];
+      // scores of the slice: lane (token ta, quarter q4) keeps its token's quarter of the
+      // summed query in registers; a quarter-warp reads one 16-byte chunk of a summary
+      // row (a broadcast), and the 4 quarters are summed with two shuffles
+      float qv[kSeg];
 #pragma unroll
-        for (int u = 0; u < kRowsPerWarp; ++u) {
-          const int oo = o0 + u * kWarps;
-          const float* src = sb + (size_t)(j0 + (oo < nloc ? oo : 0)) * D;
-          if constexpr (VEC == 4) {
-            const float4 t4 = __ldg(reinterpret_cast<const float4*>(src));
-            vals[u][0] = t4.x; vals[u][1] = t4.y; vals[u][2] = t4.z; vals[u][3] = t4.w;
-          } else {
-            const float2 t2 = __ldg(reinterpret_cast<const float2*>(src));
-            vals[u][0] = t2.x; vals[u][1] = t2.y;
+      for (int k4 = 0; k4 < kSeg / 4; ++k4) {
+        const float4 v = *reinterpret_cast<const float4*>(qsum + ta * kQStride + q4 * kSeg + 4 * k4);
+        qv[4 * k4] = v.x; qv[4 * k4 + 1] = v.y; qv[4 * k4 + 2] = v.z; qv[4 * k4 + 3] = v.w;
+      }
+      constexpr int kRU = 4;  // rows per warp at a time (independent chains)
+      for (int r0 = warp; r0 < nloc; r0 += kWarps * kRU) {  // warp-uniform
+        float dot[kRU];
+#pragma unroll
+        for (int u = 0; u < kRU; ++u) {
+          const int r = r0 + u * kWarps;
+          float a0 = 0.f, a1 = 0.f;
+          if (r < nloc) {
+            const float* row = r < staged_rows ? sumbuf + r * D + q4 * kSeg : grow + (size_t)r * D;
+#pragma unroll
+            for (int k4 = 0; k4 < kSeg / 4; ++k4) {
+              const float4 v = r < staged_rows ? reinterpret_cast<const float4*>(row)[k4]
+                                               : __ldg(reinterpret_cast<const float4*>(row) + k4);
+              a0 = fmaf(v.x, qv[4 * k4], a0);
+              a1 = fmaf(v.y, qv[4 * k4 + 1], a1);
+              a0 = fmaf(v.z, qv[4 * k4 + 2], a0);
+              a1 = fmaf(v.w, qv[4 * k4 + 3], a1);
+            }
           }
+          dot[u] = a0 + a1;
         }
 #pragma unroll
-        for (int u = 0; u < kRowsPerWarp; ++u) {
-          const int oo = o0 + u * kWarps;
-          if (oo >= nloc) break;
-          const int j = j0 + oo;
-          const bool fj = forced(j);
-          for (int a = 0; a < na; ++a) {
-            float dot = 0.f;
+        for (int u = 0; u < kRU; ++u) dot[u] += __shfl_xor_sync(0xffffffffu, dot[u], 8);
 #pragma unroll
-            for (int e = 0; e < VEC; ++e) dot = fmaf(vals[u][e], qsum[a * D + lane * VEC + e], dot);
-            dot = warp_sum(dot);
-            if (lane == 0) keys[a * p.per_max + oo] = fj ? 0ull : make_key(dot, j);
+        for (int u = 0; u < kRU; ++u) dot[u] += __shfl_xor_sync(0xffffffffu, dot[u], 16);
+        if (q4 == 0 && ta < na) {
+#pragma unroll
+          for (int u = 0; u < kRU; ++u) {
+            const int r = r0 + u * kWarps;
+            if (r < nloc) {
+              const int j = j0 + r;
+              keys[ta * per + r] = forced(j) ? 0ull : make_key(dot[u], j);
+            }
           }
         }
       }
       __syncthreads();
       // local top-m of every token (rank = number of larger keys; keys are unique)
-      for (int i = tid; i < na * nloc; i += kThreads) {
-        const int a = i / nloc, jj = i - a * nloc;
-        const u64* ka = keys + a * p.per_max;
+      for (int i = tid; i < na * per; i += kThreads) {
+        const int a2 = fdiv(i, p.per_div), jj = i - a2 * per;
+        if (jj >= nloc) continue;
+        const u64* ka = keys + a2 * per;
         const u64 x = ka[jj];
         if (x == 0ull) continue;
         int r = 0;
         for (int u = 0; u < nloc; ++u) r += ka[u] > x;
-        if (r < m) top[a * kLP + r] = x;
+        if (r < m) top[a2 * kLP + r] = x;
       }
       __syncthreads();
-      // push the lists: recv[rank][a][*] on every CTA
+      // push the lists into every peer's buffer `buf` (recv[buf][rank][a][*]); each CTA
+      // waits only until the CL lists of the chunk have landed on its own mbarrier
       if (!started) {
         cluster_wait();
         started = true;
       }
+      u64* rb = recv + (size_t)buf * kMaxCluster * kTokChunk * kLP;
+      if (tid == 0) tc::mbar_arrive_expect_tx(&xbar[buf], (uint32_t)(CL * kTokChunk * kLP * 8));
       for (int i = tid; i < CL * kTokChunk * kLP; i += kThreads) {
         const int peer = i / (kTokChunk * kLP), rem = i - peer * (kTokChunk * kLP);
-        st_cluster(map_rank(recv + (size_t)rank * kTokChunk * kLP + rem, peer), top[rem]);
+        st_async(map_rank(rb + (size_t)rank * kTokChunk * kLP + rem, peer), top[rem], map_rank(&xbar[buf], peer));
       }
-      cluster_arrive_release();
-      cluster_wait();
-      // batched merge trees: token a's lists are recv[c][a][*], c < CL
+      tc::mbar_wait(&xbar[buf], (uint32_t)((chunk_id >> 1) & 1), &xabort, kWaitBudget);
+      // batched merge trees: token a's lists are rb[c][a][*], c < CL; the result is the
+      // token's global top list, whose first m keys are its selected blocks
       {
-        u64* src = recv;
+        u64* src = rb;
         u64* dst = work;
         int cs = kTokChunk * kLP, as = kLP;
         for (int n = CL; n > 1; n >>= 1) {
           const int pairs = n >> 1;
-          for (int t = warp; t < na * pairs; t += kWarps) {
-            const int a = t / pairs, pr = t - a * pairs;
-            const u64* LA = src + (size_t)(2 * pr) * cs + a * as;
-            const u64* LB = src + (size_t)(2 * pr + 1) * cs + a * as;
-            u64 x[1];
-            x[0] = lane < kLP ? LA[lane] : LB[2 * kLP - 1 - lane];
-            warp_merge_desc<1>(x);
-            if (lane < kLP) dst[(size_t)a * (kMaxCluster / 2) * kLP + pr * kLP + lane] = x[0];
+          const int nm = na * pairs;
+          const int pl2 = __ffs(pairs) - 1;  // pairs is a power of two
+          // 4 independent merges per warp at a time (interleaved shared-memory searches)
+          for (int t0 = 4 * warp; t0 < nm; t0 += 4 * kWarps) {
+            const u64* LA[4];
+            const u64* LB[4];
+            u64* LC[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const int t = min(t0 + q, nm - 1);
+              const int a2 = t >> pl2, pr = t & (pairs - 1);
+              LA[q] = src + (size_t)(2 * pr) * cs + a2 * as;
+              LB[q] = src + (size_t)(2 * pr + 1) * cs + a2 * as;
+              LC[q] = dst + (size_t)a2 * (kMaxCluster / 2) * kLP + pr * kLP;
+            }
+            warp_merge_rank16<4>(LA, LB, LC, min(4, nm - t0));
           }
           __syncthreads();
           u64* t2 = src;
@@ -265,57 +374,74 @@ __global__ void __launch_bounds__(kThreads, 2) blockquery_kernel(const BQParams 
           cs = kLP;
           as = (kMaxCluster / 2) * kLP;
         }
-        if (tid < na) thr[tid] = src[(size_t)tid * as + (m - 1)];  // the token's m-th best key
-      }
-      __syncthreads();
-      for (int i = tid; i < nloc; i += kThreads) {
-        bool in = false;
-        for (int a = 0; a < na; ++a) {
-          const u64 x = keys[a * p.per_max + i];
-          in |= (x != 0ull && x >= thr[a]);
+        for (int a2 = warp; a2 < na; a2 += kWarps) {
+          const u64 x = lane < m ? src[(size_t)a2 * as + lane] : 0ull;  // m <= 16
+          if (x != 0ull) {
+            const int j = key_block(x);
+            atomicOr(&ubits[j >> 5], 1u << (j & 31));
+          }
         }
-        if (in) inu[i] = 1;
       }
-      if (tc0 + kTokChunk < A) {  // peers must finish reading recv before the next push
-        cluster_arrive_release();
-        cluster_wait();
-      }
-      __syncthreads();
+      __syncthreads();  // (qsum, top, keys and work are rewritten by the next chunk)
     }
+  } else if (staged_rows > 0) {
+    __syncthreads();  // (thread 0's mbarrier initialisation first)
+    tc::mbar_wait(&xbar[2], 0, &xabort, kWaitBudget);  // no copy outlives its buffer's reuse
   }
-  // compact this slice's union flags into an ascending list (block-wide ballot scan)
+  __syncthreads();
+  // the union as an ascending list (block-wide scan of the bitmap's popcounts)
   __shared__ int warp_tot[kWarps];
-  int n_my = 0;
-  for (int base = 0; base < nloc; base += kThreads) {
-    const int i = base + tid;
-    const bool on = i < nloc && inu[i];
-    const unsigned mk = __ballot_sync(0xffffffffu, on);
-    if (lane == 0) warp_tot[warp] = __popc(mk);
+  int U = 0;
+  for (int base = 0; base < nwords; base += kThreads) {
+    const int w = base + tid;
+    const uint32_t bits = w < nwords ? ubits[w] : 0u;
+    const int cnt = __popc(bits);
+    int incl = cnt;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    if (lane == 31) warp_tot[warp] = incl;
     __syncthreads();
-    int off = n_my;
-    for (int w = 0; w < warp; ++w) off += warp_tot[w];
-    if (on) ulist[off + __popc(mk & ((1u << lane) - 1u))] = j0 + i;
-    int tot = 0;
-    for (int w = 0; w < kWarps; ++w) tot += warp_tot[w];
-    n_my += tot;
+    int off = U + incl - cnt;
+    for (int w2 = 0; w2 < warp; ++w2) off += warp_tot[w2];
+    uint32_t rest = bits;
+    while (rest) {
+      const int bit = __ffs(rest) - 1;
+      ulist[off++] = w * 32 + bit;
+      rest &= rest - 1u;
+    }
+    for (int w2 = 0; w2 < kWarps; ++w2) U += warp_tot[w2];
     __syncthreads();
   }
+  // this CTA attends union entries rank, rank + CL, ... (balanced over the cluster)
+  const int cl_log2 = __ffs(CL) - 1;  // CL is a power of two
+  const int n_my = U > rank ? (U - rank + CL - 1) >> cl_log2 : 0;
 
   // ---- attention: rows (active token x head) in chunks of 32, my union blocks -----------
-  const int rows = A * G;
   const int nchunks = (rows + kRowChunk - 1) / kRowChunk;
   const int total = nchunks * n_my;
-  const __nv_bfloat16* kbase = p.k + unit * (size_t)p.T_cap * D;
-  const __nv_bfloat16* vbase = p.v + unit * (size_t)p.T_cap * D;
   float* wsu = p.ws + (unit * kMaxCluster + rank) * (size_t)p.rows_max * (D + 2);
   int issued = 0;
+  // the next block in processing order: K and V as TMA boxes (128-byte swizzled tiles)
+  // issued by thread 0, landing on the stage's mbarrier
   auto issue = [&]() {
-    unsigned char* st = kv + (size_t)(issued % kStages) * 2 * kv_tile;
-    stage_block<__nv_bfloat16, D, kThreads>(st, st + kv_tile, kbase, vbase, ulist[issued % n_my],
-                                            p.T_prefix, kRowBytes);
-    cp_async_commit();
+    const int stg = issued % kStages;
+    if (tid == 0) {
+      unsigned char* st = kv + (size_t)stg * 2 * kv_tile;
+      const int j = ulist[rank + (issued % n_my) * CL];
+      tc::fence_proxy_async();  // earlier generic accesses to this stage come first
+      tc::mbar_arrive_expect_tx(&xbar[3 + stg], (uint32_t)(2 * kv_tile));
+#pragma unroll
+      for (int h = 0; h < D / 64; ++h) {
+        tc::tma_load_3d(st + h * 8192, &p.tmk, h * 64, j * kBlk, (int)unit, &xbar[3 + stg]);
+        tc::tma_load_3d(st + kv_tile + h * 8192, &p.tmv, h * 64, j * kBlk, (int)unit, &xbar[3 + stg]);
+      }
+    }
     ++issued;
   };
+  __syncthreads();  // (the selection buffers that share the ring are dead)
   while (issued < kStages && issued < total) issue();
 
   constexpr int NT = D / 64;  // n8 tiles of the output per warp
@@ -327,16 +453,12 @@ __global__ void __launch_bounds__(kThreads, 2) blockquery_kernel(const BQParams 
   for (int c = 0; c < nchunks; ++c) {
     const int c0 = c * kRowChunk;
     const int nr = min(kRowChunk, rows - c0);
-    // query rows of the chunk (row r: token act[r / G], head r % G), zero beyond nr
-    for (int id = tid; id < kRowChunk * (kRowBytes / 16); id += kThreads) {
-      const int r = id / (kRowBytes / 16), cc = id - r * (kRowBytes / 16);
-      uint4 v4 = make_uint4(0u, 0u, 0u, 0u);
-      if (r < nr) {
-        const int rr = c0 + r, a = rr / G, hh = rr - a * G;
-        v4 = __ldg(reinterpret_cast<const uint4*>(p.q + (((size_t)b * Hq + (size_t)g * G + hh) * Tq + act[a]) * D) + cc);
-      }
-      *reinterpret_cast<uint4*>(Qs + swz(r, cc, kRowBytes)) = v4;
+    // query rows of the chunk (chunk 0 was requested at the start)
+    if (c > 0) {
+      load_attn_rows(c0);
+      cp_async_commit();
     }
+    cp_async_wait<0>();
     m_run = -INFINITY;
     l_run = 0.f;
 #pragma unroll
@@ -349,18 +471,25 @@ __global__ void __launch_bounds__(kThreads, 2) blockquery_kernel(const BQParams 
 
     for (int i = 0; i < n_my; ++i) {
       const int it = c * n_my + i;
-      if (issued > it + 1) cp_async_wait<1>(); else cp_async_wait<0>();
+      tc::mbar_wait(&xbar[3 + it % kStages], (uint32_t)((it / kStages) & 1), &xabort, kWaitBudget);
       __syncthreads();
-      const int j = ulist[i];
+      const int j = ulist[rank + i * CL];
       const unsigned char* Ks = kv + (size_t)(it % kStages) * 2 * kv_tile;
       const unsigned char* Vs = Ks + kv_tile;
+      {  // V rows past the prefix hold other tokens: zero them (P is 0 there, V must be finite)
+        const int nv = min(kBlk, p.T_prefix - j * kBlk);
+        for (int id = tid; id < (kBlk - nv) * (D / 8); id += kThreads) {
+          const int r = nv + id / (D / 8), cc = id % (D / 8);
+          *reinterpret_cast<uint4*>(const_cast<unsigned char*>(Vs) + kv_off(r, cc)) = make_uint4(0u, 0u, 0u, 0u);
+        }
+      }
       // S = Q K^T: warp w -> tokens 8w .. 8w+7, both m-tiles
       {
         float s[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
 #pragma unroll
         for (int ks = 0; ks < D / 16; ks += 2) {
           uint32_t kb[4];
-          ldsm_x4(kb, Ks + swz(8 * warp + (lane & 7), 2 * ks + (lane >> 3), kRowBytes));
+          ldsm_x4(kb, Ks + kv_off(8 * warp + (lane & 7), 2 * ks + (lane >> 3)));
 #pragma unroll
           for (int mt = 0; mt < 2; ++mt) {
             const int row = 16 * mt + (lane & 7) + 8 * ((lane >> 3) & 1);
@@ -426,10 +555,10 @@ __global__ void __launch_bounds__(kThreads, 2) blockquery_kernel(const BQParams 
         const int vrow = 16 * ks + (lane & 7) + 8 * ((lane >> 3) & 1);
         uint32_t vb[4];
         if constexpr (D == 128) {
-          ldsm_x4_t(vb, Vs + swz(vrow, 2 * warp + (lane >> 4), kRowBytes));
+          ldsm_x4_t(vb, Vs + kv_off(vrow, 2 * warp + (lane >> 4)));
         } else {
           uint32_t v2[2];
-          ldsm_x2_t(v2, Vs + swz(vrow, warp, kRowBytes));
+          ldsm_x2_t(v2, Vs + kv_off(vrow, warp));
           vb[0] = v2[0]; vb[1] = v2[1]; vb[2] = 0u; vb[3] = 0u;
         }
 #pragma unroll
@@ -464,45 +593,47 @@ __global__ void __launch_bounds__(kThreads, 2) blockquery_kernel(const BQParams 
     __syncthreads();  // Qs / stats are rewritten by the next chunk
   }
 
-  // ---- exchange union counts, barrier, then merge my output slice ------------------------
+  // ---- barrier (the partials are in the workspace), then merge my output slice ----------
   if (!started) {
     cluster_wait();
     started = true;
   }
-  if (tid < CL) st_cluster_u32(map_rank(cnt_in + rank, tid), (uint32_t)n_my);
   cluster_arrive_release();
   cluster_wait();
+  if (tid == 0 && xabort) g_blockquery_status = 1;
 
   const int E = rows * D;
-  const int chunk = (E + CL - 1) / CL;
+  const int chunk = (E + CL - 1) >> cl_log2;
   const float* wsg = p.ws + unit * kMaxCluster * (size_t)p.rows_max * (D + 2);
   for (int e = rank * chunk + tid; e < min(E, (rank + 1) * chunk); e += kThreads) {
     const int r = e / D, d = e - r * D;
-    float M = -INFINITY;
-    float mm[kMaxCluster], ll[kMaxCluster];
+    // every partial's (m, l) and value first (independent loads, one round trip), then
+    // the log-sum-exp weights
+    float2 ml[kMaxCluster];
+    float ov[kMaxCluster];
 #pragma unroll
     for (int c2 = 0; c2 < kMaxCluster; ++c2) {
-      mm[c2] = -INFINITY;
-      ll[c2] = 0.f;
+      ml[c2] = make_float2(-INFINITY, 0.f);
+      ov[c2] = 0.f;
       if (c2 < CL) {
-        const float2 ml = __ldcg(reinterpret_cast<const float2*>(wsg + ((size_t)c2 * p.rows_max + r) * (D + 2) + D));
-        mm[c2] = ml.x;
-        ll[c2] = ml.y;
-        M = fmaxf(M, ml.x);
+        const float* part = wsg + ((size_t)c2 * p.rows_max + r) * (D + 2);
+        ml[c2] = __ldcg(reinterpret_cast<const float2*>(part + D));
+        ov[c2] = __ldcg(part + d);
       }
     }
+    float M = -INFINITY;
+#pragma unroll
+    for (int c2 = 0; c2 < kMaxCluster; ++c2) M = fmaxf(M, ml[c2].x);
     float Lsum = 0.f, O = 0.f;
     if (M != -INFINITY) {
 #pragma unroll
       for (int c2 = 0; c2 < kMaxCluster; ++c2) {
-        if (c2 < CL && mm[c2] != -INFINITY) {
-          const float w = ex2(mm[c2] - M);
-          Lsum = fmaf(ll[c2], w, Lsum);
-          O = fmaf(__ldcg(wsg + ((size_t)c2 * p.rows_max + r) * (D + 2) + d), w, O);
-        }
+        const float w = ml[c2].x == -INFINITY ? 0.f : ex2(ml[c2].x - M);
+        Lsum = fmaf(ml[c2].y, w, Lsum);
+        O = fmaf(ov[c2], w, O);
       }
     }
-    const int a = r / G, hh = r - a * G;
+    const int a = fdiv(r, p.g_div), hh = r - a * G;
     const size_t orow = ((size_t)b * Hq + (size_t)g * G + hh) * Tq + act[a];
     p.o[orow * D + d] = __float2bfloat16_rn(M == -INFINITY ? 0.f : O / Lsum);
     if (d == 0) p.lse[orow] = M == -INFINITY ? -INFINITY : (M + log2f(Lsum)) * kLn2;
@@ -513,40 +644,43 @@ __global__ void __launch_bounds__(kThreads, 2) blockquery_kernel(const BQParams 
   if (p.o_cache != p.o && srows > 0) {
     const int per_row = kRowBytes / 16;
     const int n16 = srows * per_row;
-    const int c16 = (n16 + CL - 1) / CL;
+    const int c16 = (n16 + CL - 1) >> cl_log2;
     for (int i = rank * c16 + tid; i < min(n16, (rank + 1) * c16); i += kThreads) {
       const int r = i / per_row, cc = i - r * per_row;
-      const int s_i = r / G, hh = r - s_i * G;
+      const int s_i = fdiv(r, p.g_div), hh = r - s_i * G;
       const size_t orow = ((size_t)b * Hq + (size_t)g * G + hh) * Tq + stab[s_i];
       reinterpret_cast<uint4*>(p.o + orow * D)[cc] = reinterpret_cast<const uint4*>(p.o_cache + orow * D)[cc];
     }
   }
   if (p.lse_cache != p.lse && srows > 0) {
-    const int c1 = (srows + CL - 1) / CL;
+    const int c1 = (srows + CL - 1) >> cl_log2;
     for (int r = rank * c1 + tid; r < min(srows, (rank + 1) * c1); r += kThreads) {
-      const int s_i = r / G, hh = r - s_i * G;
+      const int s_i = fdiv(r, p.g_div), hh = r - s_i * G;
       const size_t orow = ((size_t)b * Hq + (size_t)g * G + hh) * Tq + stab[s_i];
       p.lse[orow] = p.lse_cache[orow];
     }
   }
 
-  // ---- the union list, by the offsets of the slices -------------------------------------
-  int off = 0, tot = 0;
-  for (int c2 = 0; c2 < CL; ++c2) {
-    const int cnt = cnt_in[c2];
-    if (c2 < rank) off += cnt;
-    tot += cnt;
+  // ---- the union list (every CTA holds it; rank 0 writes it) ----------------------------
+  if (rank == 0) {
+    if (p.union_idx) {
+      int32_t* ui = p.union_idx + unit * (size_t)NBp;
+      for (int i = tid; i < NBp; i += kThreads) ui[i] = i < U ? ulist[i] : -1;
+    }
+    if (p.union_cnt && tid == 0) p.union_cnt[unit] = U;
   }
-  if (p.union_idx) {
-    int32_t* ui = p.union_idx + unit * (size_t)NBp;
-    for (int i = tid; i < n_my; i += kThreads) ui[off + i] = ulist[i];
-    if (rank == CL - 1)
-      for (int i = tot + tid; i < NBp; i += kThreads) ui[i] = -1;
-  }
-  if (p.union_cnt && rank == 0 && tid == 0) p.union_cnt[unit] = tot;
 }
 
 }  // namespace
+
+cudaError_t read_blockquery_status(int* status, bool reset) {
+  cudaError_t err = cudaMemcpyFromSymbol(status, g_blockquery_status, sizeof(int));
+  if (err == cudaSuccess && reset) {
+    const int zero = 0;
+    err = cudaMemcpyToSymbol(g_blockquery_status, &zero, sizeof(int));
+  }
+  return err;
+}
 
 size_t blockquery_workspace_bytes(int B, int Hkv, int G, int D, int Tq) {
   return (size_t)B * Hkv * kMaxCluster * (size_t)Tq * G * (D + 2) * sizeof(float);
@@ -556,7 +690,8 @@ cudaError_t launch_blockquery(const BlockQueryArgs& a, cudaStream_t stream) {
   const int units = a.B * a.Hkv;
   int CL = units <= 14 ? 16 : (units <= 37 ? 8 : 4);
   const int NBp = (a.T_prefix + kBlk - 1) / kBlk;
-  BQParams p;
+  BQParams p{};
+  if (!kv_tensor_maps(a.k, a.v, a.D, a.T_cap, a.B * a.Hkv, &p.tmk, &p.tmv)) return cudaErrorInvalidValue;
   p.q = static_cast<const __nv_bfloat16*>(a.q);
   p.k = static_cast<const __nv_bfloat16*>(a.k);
   p.v = static_cast<const __nv_bfloat16*>(a.v);
@@ -569,13 +704,16 @@ cudaError_t launch_blockquery(const BlockQueryArgs& a, cudaStream_t stream) {
   p.union_idx = a.union_idx; p.union_cnt = a.union_cnt;
   p.ws = static_cast<float*>(a.workspace);
   p.rows_max = a.Tq * a.G;
+  p.NBp = NBp;
+  p.g_div = make_fastdiv((uint32_t)a.G);
   auto kernel = a.D == 128 ? blockquery_kernel<128> : blockquery_kernel<64>;
   static int smem_set128 = 0, smem_set64 = 0;
   int& smem_set = a.D == 128 ? smem_set128 : smem_set64;
   for (;;) {
     p.per_max = (NBp + CL - 1) / CL;
     if (p.per_max < 1) p.per_max = 1;
-    const BQLayout Lo = bq_layout(a.D, p.per_max);
+    p.per_div = make_fastdiv((uint32_t)p.per_max);
+    const BQLayout Lo = bq_layout(a.D, p.per_max, NBp, a.G);
     const int smem = (int)Lo.total;
     if (smem > 227 * 1024) return cudaErrorInvalidValue;
     cudaError_t err;

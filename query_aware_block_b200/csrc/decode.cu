@@ -93,16 +93,11 @@ struct alignas(64) Params {
   int m_pad;              // power of two >= topk
   int lp;                 // length of an exchanged candidate list: max(16, m_pad)
   int chunk;              // output elements merged by one CTA (even)
+  FastDiv chunk_div;      // division by chunk
 };
 
 __host__ __device__ inline size_t align128(size_t x) { return (x + 127) & ~(size_t)127; }
 
-// Byte offset of 16-byte chunk c of row r in a bf16 K/V tile of 64 rows: [c / 8][r][128 B]
-// with the chunk index XOR-swizzled by (r & 7), i.e. where 128-byte-swizzled TMA boxes of
-// 64 elements x 64 rows land; ldmatrix over 8 consecutive rows is conflict-free.
-__device__ __forceinline__ int kv_off(int r, int c) {
-  return ((c >> 3) << 13) + (r << 7) + ((((c & 7) ^ (r & 7))) << 4);
-}
 
 // Shared-memory carve-up (byte offsets), identical on host and device.
 struct Layout {
@@ -358,7 +353,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_cluster_kernel(const __gri
     ++issued;
   };
   const int known = all_blocks ? NB : nf;
-  const int n_known = (MODE == MODE_FUSED && known > rank) ? (known - rank + CL - 1) / CL : 0;
+  const int n_known = (MODE == MODE_FUSED && known > rank) ? (known - rank + CL - 1) >> (__ffs(CL) - 1) : 0;
   const bool scan = select && !all_blocks;
   const int nloc = scan ? max(0, min(NB, j0 + per) - j0) : 0;
   // while scanning, stage 1 holds the first pass of this CTA's summary rows
@@ -519,8 +514,9 @@ __global__ void __launch_bounds__(kThreads, 2) decode_cluster_kernel(const __gri
     cluster_wait();
     started = true;
     if (tid == 0) tc::mbar_arrive_expect_tx(&xbar[0], (uint32_t)(CL * p.lp * 8));
+    const int lp_log2 = __ffs(p.lp) - 1;  // lp is a power of two
     for (int t = tid; t < CL * p.lp; t += kThreads) {
-      const int peer = t / p.lp, pos = t - peer * p.lp;
+      const int peer = t >> lp_log2, pos = t & (p.lp - 1);
       st_async(map_rank(all + rank * p.lp + pos, peer), top[pos], map_rank(&xbar[0], peer));
     }
     tc::mbar_wait(&xbar[0], 0, &xabort, kWaitBudget);
@@ -563,7 +559,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_cluster_kernel(const __gri
   }
 
   // ---- attention over my share of the blocks ------------------------------------------
-  const int n_my = n_order > rank ? (n_order - rank + CL - 1) / CL : 0;
+  const int n_my = n_order > rank ? (n_order - rank + CL - 1) >> (__ffs(CL) - 1) : 0;  // CL: power of two
   while (issued < kStages && issued < n_my) issue_block(order[rank + issued * CL]);
   if (MODE == MODE_FUSED) write_indices();
   if (!scan) {  // the query rows' copy, followed (fp32) by at most kStages block copies
@@ -761,7 +757,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_cluster_kernel(const __gri
 #pragma unroll
       for (int e2 = 0; e2 < D / 16; ++e2) {
         const int e = srow * D + ssub + 16 * e2;
-        const int owner = e / chunk;
+        const int owner = fdiv(e, p.chunk_div);
         st_async(map_rank(pacc_in + rank * chunk + (e - owner * chunk), owner), acc[e2][0],
                  map_rank(&xbar[1], owner));
       }
@@ -776,7 +772,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_cluster_kernel(const __gri
         const int row = r0 + 8 * half;
         if (row < G) {
           const int e = row * D + d;
-          const int owner = e / chunk;
+          const int owner = fdiv(e, p.chunk_div);
           st_async(map_rank(pacc_in + rank * chunk + (e - owner * chunk), owner),
                    make_float2(acc[nt][2 * half], acc[nt][2 * half + 1]), map_rank(&xbar[1], owner));
         }
@@ -823,30 +819,6 @@ __global__ void __launch_bounds__(kThreads, 2) decode_cluster_kernel(const __gri
 
 // ---- host side --------------------------------------------------------------------------
 
-// The K and V tensor maps of the last bf16 call on this host thread: a decode loop calls
-// with the same cache tensors every step, so the maps are encoded once.
-struct MapCache {
-  const void* k = nullptr;
-  const void* v = nullptr;
-  int D = 0, T_cap = 0, planes = 0;
-  CUtensorMap mk, mv;
-};
-
-bool kv_maps(const DecodeArgs& a, CUtensorMap* mk, CUtensorMap* mv) {
-  static thread_local MapCache c;
-  const int planes = a.B * a.Hkv;
-  if (!(c.k == a.k && c.v == a.v && c.D == a.D && c.T_cap == a.T_cap && c.planes == planes)) {
-    c.k = nullptr;
-    if (!encode_rows_bf16(&c.mk, a.k, a.D, a.T_cap, planes, kBlk) ||
-        !encode_rows_bf16(&c.mv, a.v, a.D, a.T_cap, planes, kBlk))
-      return false;
-    c.k = a.k; c.v = a.v; c.D = a.D; c.T_cap = a.T_cap; c.planes = planes;
-  }
-  *mk = c.mk;
-  *mv = c.mv;
-  return true;
-}
-
 int next_pow2(int x) {
   int p = 1;
   while (p < x) p <<= 1;
@@ -860,7 +832,9 @@ cudaError_t launch_t(const DecodeArgs& a, cudaStream_t stream) {
   const int units = a.B * a.Hkv;
   int CL = units <= 18 ? 16 : (units <= 74 ? 8 : 4);
   Params p{};
-  if (sizeof(T) == 2 && MODE != MODE_SELECT && !kv_maps(a, &p.tmk, &p.tmv)) return cudaErrorInvalidValue;
+  if (sizeof(T) == 2 && MODE != MODE_SELECT &&
+      !kv_tensor_maps(a.k, a.v, a.D, a.T_cap, a.B * a.Hkv, &p.tmk, &p.tmv))
+    return cudaErrorInvalidValue;
   p.q = a.q; p.k = a.k; p.v = a.v;
   p.Hkv = a.Hkv; p.G = a.G; p.T_cap = a.T_cap; p.NB_cap = a.NB_cap;
   p.seqlens = a.seqlens; p.summ = a.summ; p.summ_w = a.summ_w;
@@ -879,6 +853,7 @@ cudaError_t launch_t(const DecodeArgs& a, cudaStream_t stream) {
     p.per_max = (a.NB_cap + CL - 1) / CL;
     const int E = a.G * D;
     p.chunk = ((E + CL - 1) / CL + 1) & ~1;
+    p.chunk_div = make_fastdiv((uint32_t)p.chunk);
     const Layout Lo = make_layout((int)sizeof(T), D, p.per_max, p.m_pad);
     const int smem = (int)Lo.total;
     if (smem > smem_set) {

@@ -221,7 +221,10 @@ int lsa_device_status(int* status, int reset) {
   if (st != LSA_OK) return st;
   st = cuda_status(lsa::read_decode_status(&decode, reset != 0));
   if (st != LSA_OK) return st;
-  *status = prefill | decode;
+  int bq = 0;
+  st = cuda_status(lsa::read_blockquery_status(&bq, reset != 0));
+  if (st != LSA_OK) return st;
+  *status = prefill | decode | bq;
   return LSA_OK;
 }
 

@@ -16,6 +16,28 @@ constexpr int kBlk = 64;            // KV block (selection unit) in tokens
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 
+// ---- division by a divisor known only at launch -----------------------------------------
+// floor(n / d) for 0 <= n < 2^31 as one 32x32->64 multiply and a shift: m = ceil(2^(31+l)/d)
+// with l = ceil(log2 d) (the round-up method of Granlund and Montgomery, "Division by
+// invariant integers using multiplication", 1994).  An integer division by a run-time
+// value costs tens of instructions on the GPU; the constants are computed on the host.
+struct FastDiv {
+  uint32_t m;
+  uint32_t sh;
+};
+inline FastDiv make_fastdiv(uint32_t d) {
+  uint32_t l = 0;
+  while ((1ull << l) < d) ++l;
+  const unsigned long long num = 1ull << (31 + l);
+  FastDiv f;
+  f.m = (uint32_t)((num + d - 1) / d);
+  f.sh = 31 + l;
+  return f;
+}
+__device__ __forceinline__ int fdiv(int n, FastDiv f) {
+  return (int)(((unsigned long long)(uint32_t)n * f.m) >> f.sh);
+}
+
 // ---- element conversion ------------------------------------------------------------
 __device__ __forceinline__ float to_f32(float x) { return x; }
 __device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
@@ -108,6 +130,13 @@ __device__ __forceinline__ void mma_bf16(float (&c)[4], const uint32_t (&a)[4], 
 // are XOR-swizzled by (r & 7): conflict-free for ldmatrix and for row-wise cp.async.
 __device__ __forceinline__ int swz(int r, int c, int row_bytes) {
   return r * row_bytes + ((c ^ (r & 7)) << 4);
+}
+
+// Byte offset of 16-byte chunk c of row r in a bf16 K/V tile of 64 rows: [c / 8][r][128 B]
+// with the chunk index XOR-swizzled by (r & 7), i.e. where 128-byte-swizzled TMA boxes of
+// 64 elements x 64 rows land; ldmatrix over 8 consecutive rows is conflict-free.
+__device__ __forceinline__ int kv_off(int r, int c) {
+  return ((c >> 3) << 13) + (r << 7) + ((((c & 7) ^ (r & 7))) << 4);
 }
 
 // ---- K/V block staging ----------------------------------------------------------------

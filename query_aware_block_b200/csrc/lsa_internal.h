@@ -78,11 +78,16 @@ struct PrefillArgs {
 cudaError_t launch_blasst_prefill(const PrefillArgs& a, cudaStream_t stream);
 cudaError_t read_device_status(int* status, bool reset);
 cudaError_t read_decode_status(int* status, bool reset);
+cudaError_t read_blockquery_status(int* status, bool reset);
 
 // 3-D TMA map over a row-major bf16 tensor [planes][rows][D]: box {64, box_rows, 1} (one
 // 128-byte swizzled row segment per box row), rows past `rows` read as zero.  False when
 // the driver entry point is missing or rejects the map.
 bool encode_rows_bf16(CUtensorMap* map, const void* base, int D, int rows, int planes, int box_rows);
+// Maps of a bf16 K/V cache pair [planes][T_cap][D] with 64-row boxes, cached per host
+// thread for the last (k, v, D, T_cap, planes).
+bool kv_tensor_maps(const void* k, const void* v, int D, int T_cap, int planes, CUtensorMap* mk,
+                    CUtensorMap* mv);
 
 // The fixed device scratch used by lsa_sparse_attn_blockquery_noalloc.
 size_t blockquery_static_workspace_bytes();

@@ -38,4 +38,29 @@ bool encode_rows_bf16(CUtensorMap* map, const void* base, int D, int rows, int p
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+namespace {
+// The K and V maps of the last call on this host thread: decode and block-query loops call
+// with the same cache tensors every step, so the maps are encoded once.
+struct KVMapCache {
+  const void* k = nullptr;
+  const void* v = nullptr;
+  int D = 0, T_cap = 0, planes = 0;
+  CUtensorMap mk, mv;
+};
+}  // namespace
+
+bool kv_tensor_maps(const void* k, const void* v, int D, int T_cap, int planes, CUtensorMap* mk,
+                    CUtensorMap* mv) {
+  static thread_local KVMapCache c;
+  if (!(c.k == k && c.v == v && c.D == D && c.T_cap == T_cap && c.planes == planes)) {
+    c.k = nullptr;
+    if (!encode_rows_bf16(&c.mk, k, D, T_cap, planes, 64) || !encode_rows_bf16(&c.mv, v, D, T_cap, planes, 64))
+      return false;
+    c.k = k; c.v = v; c.D = D; c.T_cap = T_cap; c.planes = planes;
+  }
+  *mk = c.mk;
+  *mv = c.mv;
+  return true;
+}
+
 }  // namespace lsa
