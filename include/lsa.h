@@ -254,7 +254,7 @@ LSA_API int lsa_sparse_attn_blockquery_noalloc(const void* q, const void* k, con
  *     (b, h, a) row is set iff tile c was skipped;
  * skipped_tiles: one uint64 counter or NULL, incremented by the number of skipped tiles
  *     (the caller zeroes it).
- * Requires bf16, D == 128, Hq % Hkv == 0, 0 <= lambda < 1.
+ * Requires bf16, D == 128, Hq % Hkv == 0, B * Hq <= 65535, 0 <= lambda < 1.
  * Every wait of the kernel on its own pipeline is bounded in time; should one ever run
  * out, the kernel stops cleanly and lsa_device_status() reports LSA_DEVICE_TIMEOUT.
  */

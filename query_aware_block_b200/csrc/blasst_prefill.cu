@@ -7,9 +7,12 @@
 // is skipped -- no exponentials, no P.V product -- when every row's tile maximum trails its
 // running maximum by more than -ln(lambda):  max_i (r_i - m_i) < ln(lambda).
 //
-// How (B200): one CTA per (b, h, query tile), heaviest tiles first; 8 warps.
+// How (B200): one CTA per (b, h, query tile), heaviest tiles first, the query tiles of one
+// head launched together (their KV group stays in L2); 8 warps, 2 CTAs per SM so that one
+// CTA's softmax overlaps the other's tensor-core work (each holds 256 of the 512 TMEM
+// columns).
 //   warp 0    TMA producer: Q once (2 boxes of 128 x 64 bf16, 128-byte swizzle), then K and
-//             V tiles into a 4-stage shared-memory ring (3-D tensor maps, no multicast).
+//             V tiles into a 2-stage shared-memory ring (3-D tensor maps, no multicast).
 //   warp 1    MMA issuer (one thread): S_j = Q K_j^T (M 128, N 64, K 128) into a
 //             double-buffered TMEM tile; O += P_j V_j (M 128, N 128, K 64) with P read from
 //             tensor memory; tcgen05.commit signals S ready, O updated, stage free.
@@ -42,7 +45,7 @@ constexpr int kThreads = 256;
 constexpr int kBM = 128;          // query rows per tile
 constexpr int kBN = 64;           // keys per KV tile
 constexpr int kD = 128;           // head dim
-constexpr int kStages = 4;
+constexpr int kStages = 2;       // (2 CTAs per SM: their softmax and MMA phases interleave)
 constexpr uint32_t kTmemCols = 256;
 constexpr uint32_t kColO = 128;
 constexpr int kQBytes = kBM * kD * 2;        // 32 KB
@@ -79,7 +82,7 @@ struct Bars {
 
 constexpr size_t kSmemBytes = 1024 /*alignment slack*/ + kQBytes + kStages * kStageBytes + 256;
 
-__global__ void __launch_bounds__(kThreads, 1) blasst_prefill_kernel(const __grid_constant__ PrefillParams p) {
+__global__ void __launch_bounds__(kThreads, 2) blasst_prefill_kernel(const __grid_constant__ PrefillParams p) {
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   unsigned char* Qs = smem;
@@ -88,8 +91,10 @@ __global__ void __launch_bounds__(kThreads, 1) blasst_prefill_kernel(const __gri
   volatile int* abort = &bars->abort;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int bh = blockIdx.x;                       // b * Hq + h
-  const int a = p.nqt - 1 - (int)blockIdx.y;       // heaviest query tiles first
+  // grid x: query tiles, heaviest first; y: b * Hq + h, so that the CTAs running together
+  // share one KV group's K/V in L2
+  const int bh = blockIdx.y;
+  const int a = p.nqt - 1 - (int)blockIdx.x;
   const int G = p.Hq / p.Hkv;
   const int b = bh / p.Hq, h = bh - b * p.Hq;
   const int bg = b * p.Hkv + h / G;
@@ -375,7 +380,7 @@ cudaError_t launch_blasst_prefill(const PrefillArgs& a, cudaStream_t stream) {
     if (err != cudaSuccess) return err;
     attr_done = true;
   }
-  dim3 grid(a.B * a.Hq, p.nqt, 1);
+  dim3 grid(p.nqt, a.B * a.Hq, 1);
   blasst_prefill_kernel<<<grid, kThreads, kSmemBytes, stream>>>(p);
   return cudaGetLastError();
 }

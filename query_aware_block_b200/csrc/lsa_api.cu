@@ -204,7 +204,7 @@ int lsa_blasst_prefill(const void* q, const void* k, const void* v, int dtype, i
   if (B == 0 || L == 0) return LSA_OK;
   if (!q || !k || !v || !o) return LSA_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return LSA_ERR_INVALID_ARG;
-  if ((L + 127) / 128 > 65535) return LSA_ERR_UNSUPPORTED;
+  if ((long long)B * Hq > 65535) return LSA_ERR_UNSUPPORTED;
   lsa::PrefillArgs a = {};
   a.q = q; a.k = k; a.v = v;
   a.B = B; a.Hq = Hq; a.Hkv = Hkv; a.L = L;
