@@ -55,22 +55,6 @@ constexpr long long kWaitBudget = 4000000000LL;  // clock cycles (about 2 s)
 constexpr float kRescaleLog2 = 8.0f;             // rescale O when the max grew by > 2^8
 constexpr int kDeviceTimeout = 1;
 
-// 2^x on the FMA/ALU pipes, for a share of the softmax exponentials (the MUFU unit issues
-// ex2 at a quarter of the FMA rate and limits the softmax).  x = n + f with n = round(x)
-// taken through the float adder (adding 1.5 * 2^23 leaves round(x) in the low mantissa
-// bits), f in [-1/2, 1/2]; 2^f by a degree-3 polynomial whose coefficients were fitted for
-// this kernel by iteratively reweighted least squares on [-1/2, 1/2] (largest relative
-// error 7.5e-5, far below the bf16 rounding of P); 2^n added into the exponent field.
-// x >= -126 keeps the result normal; in this kernel x <= 2^8 (the lazy rescale bound).
-__device__ __forceinline__ float exp2_fma(float x) {
-  x = fmaxf(x, -126.0f);
-  const float t = x + 12582912.0f;
-  const float f = x - (t - 12582912.0f);
-  const float p = fmaf(fmaf(fmaf(0.055171458847100355f, f, 0.24261086198506535f), f, 0.6932609924097385f), f,
-                       0.9999280895314314f);
-  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
-}
-
 struct alignas(64) PrefillParams {
   CUtensorMap tq;  // [B*Hq][L][D]
   CUtensorMap tk;  // [B*Hkv][L][D]
@@ -284,14 +268,12 @@ __global__ void __launch_bounds__(kThreads, 2) blasst_prefill_kernel(const __gri
 #pragma unroll
           for (int c = 0; c < 32; ++c) pk[c] = 0u;
         } else {
-          // p = 2^(scale2 * s - base); one exponential in four on the FMA pipes
+          // p = 2^(scale2 * s - base), the scale folded into one FMA per element
           const float nb = -base;
 #pragma unroll
           for (int c = 0; c < 32; ++c) {
-            const float x0 = fmaf(__uint_as_float(sr[2 * c]), p.scale2, nb);
-            const float x1 = fmaf(__uint_as_float(sr[2 * c + 1]), p.scale2, nb);
-            const float p0 = ex2(x0);
-            const float p1 = (c & 1) ? exp2_fma(x1) : ex2(x1);
+            const float p0 = ex2(fmaf(__uint_as_float(sr[2 * c]), p.scale2, nb));
+            const float p1 = ex2(fmaf(__uint_as_float(sr[2 * c + 1]), p.scale2, nb));
             rs += p0 + p1;
             pk[c] = pack_bf16x2(p0, p1);
           }
