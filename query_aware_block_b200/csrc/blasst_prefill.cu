@@ -11,8 +11,10 @@
 // head launched together (their KV group stays in L2); 8 warps, 2 CTAs per SM so that one
 // CTA's softmax overlaps the other's tensor-core work (each holds 256 of the 512 TMEM
 // columns).
-//   warp 0    TMA producer: Q once (2 boxes of 128 x 64 bf16, 128-byte swizzle), then K and
-//             V tiles into a 2-stage shared-memory ring (3-D tensor maps, no multicast).
+//   warp 0    TMA producers: lane 0 loads Q once (2 boxes of 128 x 64 bf16, 128-byte
+//             swizzle) and then the K tiles, lane 1 the V tiles, each into its own 2-stage
+//             ring (3-D tensor maps, no multicast): K_j is released when S_j is done, V_j
+//             when P_j V_j is, so the next K tiles arrive while P V is still pending.
 //   warp 1    MMA issuer (one thread): S_j = Q K_j^T (M 128, N 64, K 128) into a
 //             double-buffered TMEM tile; O += P_j V_j (M 128, N 128, K 64) with P read from
 //             tensor memory; tcgen05.commit signals S ready, O updated, stage free.
@@ -70,8 +72,10 @@ struct alignas(64) PrefillParams {
 
 struct Bars {
   uint64_t q_full;
-  uint64_t kv_full[kStages];
-  uint64_t kv_empty[kStages];
+  uint64_t k_full[kStages];   // K and V have separate rings: K_j is free once S_j is done,
+  uint64_t k_empty[kStages];  // long before P_j V_j frees V_j
+  uint64_t v_full[kStages];
+  uint64_t v_empty[kStages];
   uint64_t s_full[2];
   uint64_t p_full[2];
   uint64_t o_done;
@@ -86,7 +90,8 @@ __global__ void __launch_bounds__(kThreads, 2) blasst_prefill_kernel(const __gri
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   unsigned char* Qs = smem;
-  unsigned char* KV = smem + kQBytes;
+  unsigned char* Kring = smem + kQBytes;                        // kStages K tiles
+  unsigned char* Vring = Kring + kStages * kKVTileBytes;        // kStages V tiles
   Bars* bars = reinterpret_cast<Bars*>(smem + kQBytes + kStages * kStageBytes);
   volatile int* abort = &bars->abort;
 
@@ -105,8 +110,10 @@ __global__ void __launch_bounds__(kThreads, 2) blasst_prefill_kernel(const __gri
   if (tid == 0) {
     tc::mbar_init(&bars->q_full, 1);
     for (int s = 0; s < kStages; ++s) {
-      tc::mbar_init(&bars->kv_full[s], 1);
-      tc::mbar_init(&bars->kv_empty[s], 1);
+      tc::mbar_init(&bars->k_full[s], 1);
+      tc::mbar_init(&bars->k_empty[s], 1);
+      tc::mbar_init(&bars->v_full[s], 1);
+      tc::mbar_init(&bars->v_empty[s], 1);
     }
     for (int s = 0; s < 2; ++s) {
       tc::mbar_init(&bars->s_full[s], 1);
@@ -126,36 +133,41 @@ __global__ void __launch_bounds__(kThreads, 2) blasst_prefill_kernel(const __gri
   tc::fence_after_sync();
   const uint32_t tmem = bars->tmem;
 
-  if (warp == 0 && lane == 0) {
-    // ---------------------------------------------------------------- TMA producer ----
-    tc::prefetch_tmap(&p.tq);
-    tc::prefetch_tmap(&p.tk);
-    tc::prefetch_tmap(&p.tv);
-    tc::mbar_arrive_expect_tx(&bars->q_full, kQBytes);
-    tc::tma_load_3d(Qs, &p.tq, 0, i0, bh, &bars->q_full);
-    tc::tma_load_3d(Qs + kQBytes / 2, &p.tq, 64, i0, bh, &bars->q_full);
+  if (warp == 0 && lane < 2) {
+    // --------------------------------------------------------------- TMA producers ----
+    // lane 0: Q, then the K tiles; lane 1: the V tiles (each ring on its own barriers)
+    if (lane == 0) {
+      tc::prefetch_tmap(&p.tq);
+      tc::prefetch_tmap(&p.tk);
+      tc::mbar_arrive_expect_tx(&bars->q_full, kQBytes);
+      tc::tma_load_3d(Qs, &p.tq, 0, i0, bh, &bars->q_full);
+      tc::tma_load_3d(Qs + kQBytes / 2, &p.tq, 64, i0, bh, &bars->q_full);
+    } else {
+      tc::prefetch_tmap(&p.tv);
+    }
+    const CUtensorMap* map = lane == 0 ? &p.tk : &p.tv;
+    unsigned char* ring = lane == 0 ? Kring : Vring;
+    uint64_t* full = lane == 0 ? bars->k_full : bars->v_full;
+    uint64_t* empty = lane == 0 ? bars->k_empty : bars->v_empty;
     for (int j = 0; j < n_visit; ++j) {
       const int s = j % kStages;
-      if (j >= kStages && !tc::mbar_wait(&bars->kv_empty[s], ((j / kStages) - 1) & 1, abort, kWaitBudget))
-        break;
-      unsigned char* Ks = KV + s * kStageBytes;
-      unsigned char* Vs = Ks + kKVTileBytes;
-      tc::mbar_arrive_expect_tx(&bars->kv_full[s], kStageBytes);
-      tc::tma_load_3d(Ks, &p.tk, 0, j * kBN, bg, &bars->kv_full[s]);
-      tc::tma_load_3d(Ks + kKVTileBytes / 2, &p.tk, 64, j * kBN, bg, &bars->kv_full[s]);
-      tc::tma_load_3d(Vs, &p.tv, 0, j * kBN, bg, &bars->kv_full[s]);
-      tc::tma_load_3d(Vs + kKVTileBytes / 2, &p.tv, 64, j * kBN, bg, &bars->kv_full[s]);
+      if (j >= kStages && !tc::mbar_wait(&empty[s], ((j / kStages) - 1) & 1, abort, kWaitBudget)) break;
+      unsigned char* dst = ring + s * kKVTileBytes;
+      tc::mbar_arrive_expect_tx(&full[s], kKVTileBytes);
+      tc::tma_load_3d(dst, map, 0, j * kBN, bg, &full[s]);
+      tc::tma_load_3d(dst + kKVTileBytes / 2, map, 64, j * kBN, bg, &full[s]);
     }
   } else if (warp == 1 && lane == 0) {
     // ----------------------------------------------------------------- MMA issuer ----
     constexpr uint32_t idesc_qk = tc::idesc_bf16_f32(kBM, kBN, false);
     constexpr uint32_t idesc_pv = tc::idesc_bf16_f32(kBM, kD, true);
     const uint32_t q_addr = tc::smem_u32(Qs);
-    const uint32_t kv_addr = tc::smem_u32(KV);
+    const uint32_t kring_addr = tc::smem_u32(Kring);
+    const uint32_t vring_addr = tc::smem_u32(Vring);
     auto issue_s = [&](int j) -> bool {
       const int s = j % kStages;
-      if (!tc::mbar_wait(&bars->kv_full[s], (j / kStages) & 1, abort, kWaitBudget)) return false;
-      const uint32_t k_addr = kv_addr + s * kStageBytes;
+      if (!tc::mbar_wait(&bars->k_full[s], (j / kStages) & 1, abort, kWaitBudget)) return false;
+      const uint32_t k_addr = kring_addr + s * kKVTileBytes;
       const uint32_t d = tmem + (uint32_t)(j & 1) * 64u;
 #pragma unroll
       for (int ks = 0; ks < kD / 16; ++ks) {
@@ -165,6 +177,7 @@ __global__ void __launch_bounds__(kThreads, 2) blasst_prefill_kernel(const __gri
         tc::mma_ss(d, ad, bd, idesc_qk, ks > 0 ? 1u : 0u);
       }
       tc::mma_commit(&bars->s_full[j & 1]);
+      tc::mma_commit(&bars->k_empty[s]);  // K_j is no longer needed once S_j is done
       return true;
     };
     bool ok = tc::mbar_wait(&bars->q_full, 0, abort, kWaitBudget);
@@ -176,7 +189,8 @@ __global__ void __launch_bounds__(kThreads, 2) blasst_prefill_kernel(const __gri
       if (!tc::mbar_wait(&bars->p_full[buf], (j >> 1) & 1, abort, kWaitBudget)) break;
       tc::fence_after_sync();
       if (!bars->skip[buf]) {
-        const uint32_t v_addr = kv_addr + s * kStageBytes + kKVTileBytes;
+        if (!tc::mbar_wait(&bars->v_full[s], (j / kStages) & 1, abort, kWaitBudget)) break;
+        const uint32_t v_addr = vring_addr + s * kKVTileBytes;
 #pragma unroll
         for (int kk = 0; kk < kBN / 16; ++kk) {
           // V as B (K = keys, N = dims): MN-major, 128-byte swizzle; the two 64-dim boxes are
@@ -187,8 +201,10 @@ __global__ void __launch_bounds__(kThreads, 2) blasst_prefill_kernel(const __gri
         }
         tc::mma_commit(&bars->o_done);
         ++pv_count;
+      } else if (!tc::mbar_wait(&bars->v_full[s], (j / kStages) & 1, abort, kWaitBudget)) {
+        break;
       }
-      tc::mma_commit(&bars->kv_empty[s]);
+      tc::mma_commit(&bars->v_empty[s]);  // (a skipped tile's V is released unread)
       if (j + 2 < n_visit && !issue_s(j + 2)) break;
     }
   } else if (warp >= 4) {
@@ -227,18 +243,24 @@ __global__ void __launch_bounds__(kThreads, 2) blasst_prefill_kernel(const __gri
       // cuts this tile; scaled to log2 units after the max (scale2 > 0 commutes with it)
       const int t0 = j * kBN;
       const int lim = min(i, p.L - 1) - t0;  // keys t0 + c with c <= lim are visible
-      float rmax = -INFINITY;
+      // (8 independent partial maxima: a single chain of 64 dependent max operations would
+      // dominate the softmax latency)
+      float mx8[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) mx8[e] = -INFINITY;
       if (row_ok && lim >= kBN - 1) {
 #pragma unroll
-        for (int c = 0; c < kBN; ++c) rmax = fmaxf(rmax, __uint_as_float(sr[c]));
+        for (int c = 0; c < kBN; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], __uint_as_float(sr[c]));
       } else {
 #pragma unroll
         for (int c = 0; c < kBN; ++c) {
           const float v = (row_ok && c <= lim) ? __uint_as_float(sr[c]) : -INFINITY;
           sr[c] = __float_as_uint(v);
-          rmax = fmaxf(rmax, v);
+          mx8[c & 7] = fmaxf(mx8[c & 7], v);
         }
       }
+      const float rmax = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                               fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
       const float r = rmax * p.scale2;
       // the skip vote: every row negligible (absent rows and rows without a visible key agree)
       const bool negligible = !row_ok || r == -INFINITY || (m_run != -INFINITY && (r - m_run) < p.log2lam);
@@ -268,15 +290,18 @@ __global__ void __launch_bounds__(kThreads, 2) blasst_prefill_kernel(const __gri
 #pragma unroll
           for (int c = 0; c < 32; ++c) pk[c] = 0u;
         } else {
-          // p = 2^(scale2 * s - base), the scale folded into one FMA per element
+          // p = 2^(scale2 * s - base), the scale folded into one FMA per element; the row
+          // sum in 4 independent partial sums
           const float nb = -base;
+          float rs4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
           for (int c = 0; c < 32; ++c) {
             const float p0 = ex2(fmaf(__uint_as_float(sr[2 * c]), p.scale2, nb));
             const float p1 = ex2(fmaf(__uint_as_float(sr[2 * c + 1]), p.scale2, nb));
-            rs += p0 + p1;
+            rs4[c & 3] += p0 + p1;
             pk[c] = pack_bf16x2(p0, p1);
           }
+          rs = (rs4[0] + rs4[1]) + (rs4[2] + rs4[3]);
         }
         l = l * alpha + rs;
         tc::tmem_st32(lane_addr + (uint32_t)buf * 64u, pk);
