@@ -369,7 +369,8 @@ def run_ours(args, rank, world, local_rank):
                    "head_dim": D, "context": T_cap, "block": 64, "topk": topk,
                    "forced": {"sink": ns, "local": nl},
                    "l2": f"rotating {R} input copies ({R * step_bytes / 1e6:.0f} MB touched per "
-                         f"cycle, > 4x the {l2 / 1e6:.0f} MB L2)",
+                         f"cycle, " + (f"> 4x the {l2 / 1e6:.0f} MB L2)" if R * step_bytes > 4 * l2 else
+                                       f"within the {l2 / 1e6:.0f} MB L2: a profiling run, not a measurement)"),
                    "parallelism": f"replicas x{world} (independent sequences, no collective)",
                    "overlapped_launch": bool(args.overlap)},
         "effective_gbs": round(step_bytes / (ms_step * 1e-3) / 1e9, 1),
