@@ -20,7 +20,8 @@
 //             tensor memory; tcgen05.commit signals S ready, O updated, stage free.
 //   warp 2    allocates / frees 256 TMEM columns: S0 [0,64), S1 [64,128), O [128,256).
 //   warps 4-7 softmax: thread = query row = TMEM lane.  Loads its S row, masks, takes the
-//             row max, votes on the skip with one bar.red.and over the 128 rows, writes
+//             row max, votes on the skip (a warp with a non-negligible row marks the tile
+//             kept and goes on; only an all-negligible warp waits on the vote mbarrier), writes
 //             P (bf16) back over its S columns, rescales its O row only when its running
 //             max grew by more than 2^8 since the exponent base was last set (exact: the
 //             final normalisation uses the same base), and stores o and lse at the end.
@@ -78,9 +79,10 @@ struct Bars {
   uint64_t v_empty[kStages];
   uint64_t s_full[2];
   uint64_t p_full[2];
+  uint64_t vote[2];           // one arrival per softmax warp and tile: the skip vote is in
   uint64_t o_done;
   uint32_t tmem;
-  int skip[2];
+  int nonneg[2];              // the last tile (of this buffer) some softmax warp kept
   int abort;
 };
 
@@ -118,7 +120,8 @@ __global__ void __launch_bounds__(kThreads, 2) blasst_prefill_kernel(const __gri
     for (int s = 0; s < 2; ++s) {
       tc::mbar_init(&bars->s_full[s], 1);
       tc::mbar_init(&bars->p_full[s], 128);
-      bars->skip[s] = 0;
+      tc::mbar_init(&bars->vote[s], 4);
+      bars->nonneg[s] = -1;
     }
     tc::mbar_init(&bars->o_done, 1);
     bars->abort = 0;
@@ -188,7 +191,8 @@ __global__ void __launch_bounds__(kThreads, 2) blasst_prefill_kernel(const __gri
       const int buf = j & 1, s = j % kStages;
       if (!tc::mbar_wait(&bars->p_full[buf], (j >> 1) & 1, abort, kWaitBudget)) break;
       tc::fence_after_sync();
-      if (!bars->skip[buf]) {
+      const bool kept = reinterpret_cast<volatile int*>(bars->nonneg)[buf] == j;
+      if (kept) {
         if (!tc::mbar_wait(&bars->v_full[s], (j / kStages) & 1, abort, kWaitBudget)) break;
         const uint32_t v_addr = vring_addr + s * kKVTileBytes;
 #pragma unroll
@@ -219,10 +223,11 @@ __global__ void __launch_bounds__(kThreads, 2) blasst_prefill_kernel(const __gri
     int nskipped = 0;
     bool failed = false;
     uint32_t* bits_row = p.skip_bits ? p.skip_bits + ((size_t)bh * p.nqt + a) * p.words : nullptr;
+    // No block-wide barrier inside the loop: every wait is a bounded mbarrier wait whose
+    // outcome is made warp-uniform, so a failure lets each warp leave on its own.
     for (int j = 0; j < n_visit; ++j) {
       const int buf = j & 1;
-      const bool ok = tc::mbar_wait(&bars->s_full[buf], (j >> 1) & 1, abort, kWaitBudget);
-      if (tc::named_or(1, 128, !ok)) {
+      if (!__all_sync(0xffffffffu, tc::mbar_wait(&bars->s_full[buf], (j >> 1) & 1, abort, kWaitBudget))) {
         failed = true;
         break;
       }
@@ -264,10 +269,24 @@ __global__ void __launch_bounds__(kThreads, 2) blasst_prefill_kernel(const __gri
       const float r = rmax * p.scale2;
       // the skip vote: every row negligible (absent rows and rows without a visible key agree)
       const bool negligible = !row_ok || r == -INFINITY || (m_run != -INFINITY && (r - m_run) < p.log2lam);
-      const bool skip = tc::named_and(1, 128, negligible);
+      // The vote, without a block barrier: a warp holding a non-negligible row marks the
+      // tile kept and goes on (the tile cannot be skipped any more); a warp whose rows are
+      // all negligible waits for the four warps' votes.  The MMA thread reads the mark after
+      // all 128 rows have released the tile.
+      const bool warp_neg = __all_sync(0xffffffffu, negligible);
+      if (!warp_neg && lane == 0) reinterpret_cast<volatile int*>(bars->nonneg)[buf] = j;
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(&bars->vote[buf]);
+      bool skip = false;
+      if (warp_neg) {
+        if (!__all_sync(0xffffffffu, tc::mbar_wait(&bars->vote[buf], (j >> 1) & 1, abort, kWaitBudget))) {
+          failed = true;
+          break;
+        }
+        skip = reinterpret_cast<volatile int*>(bars->nonneg)[buf] != j;
+      }
       if (skip) {
         if (row == 0) {
-          bars->skip[buf] = 1;
           skipmask |= 1u << (j & 31);
           ++nskipped;
         }
@@ -306,12 +325,10 @@ __global__ void __launch_bounds__(kThreads, 2) blasst_prefill_kernel(const __gri
         l = l * alpha + rs;
         tc::tmem_st32(lane_addr + (uint32_t)buf * 64u, pk);
         tc::tmem_st_wait();
-        if (row == 0) bars->skip[buf] = 0;
         // the previous P.V must be complete: O is then stable, and at most one O update is
         // ever outstanding, which keeps the o_done phase parity unambiguous
         if (pv_issued > pv_observed) {
-          const bool ok2 = tc::mbar_wait(&bars->o_done, pv_observed & 1, abort, kWaitBudget);
-          if (tc::named_or(1, 128, !ok2)) {
+          if (!__all_sync(0xffffffffu, tc::mbar_wait(&bars->o_done, pv_observed & 1, abort, kWaitBudget))) {
             failed = true;
             break;
           }
@@ -341,8 +358,7 @@ __global__ void __launch_bounds__(kThreads, 2) blasst_prefill_kernel(const __gri
     }
     if (!failed) {
       while (pv_observed < pv_issued) {
-        const bool ok = tc::mbar_wait(&bars->o_done, pv_observed & 1, abort, kWaitBudget);
-        if (tc::named_or(1, 128, !ok)) {
+        if (!__all_sync(0xffffffffu, tc::mbar_wait(&bars->o_done, pv_observed & 1, abort, kWaitBudget))) {
           failed = true;
           break;
         }
