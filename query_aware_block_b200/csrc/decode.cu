@@ -395,6 +395,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_cluster_kernel(const __gri
   }
 
   // ---- selection --------------------------------------------------------------------
+  bool early = false;  // (uniform) the first block's copy was started by warp 0 after the merge
   if (scan) {
     // the staged query rows: only the newest block's copy may be in flight after them
     if (kF32 && newest_issued) cp_async_wait<1>(); else cp_async_wait<0>();
@@ -522,6 +523,22 @@ __global__ void __launch_bounds__(kThreads, 2) decode_cluster_kernel(const __gri
     tc::mbar_wait(&xbar[0], 0, &xabort, kWaitBudget);
     if (p.lp == 16 && CL >= 2) {
       merge_tree16(all, work, CL, m, nf, order);
+      // warp 0 ends the tree holding the final list: when this CTA's first block is a scored
+      // one (bf16, nothing staged yet), its TMA starts here, before the block barrier
+      early = !kF32 && MODE == MODE_FUSED && rank >= nf && rank - nf < m && issued == 0;
+      if (early && warp == 0) {
+        __syncwarp();  // (order[] was written by warp 0's lanes)
+        if (lane == 0) {
+          const int jb = order[rank];
+          tc::fence_proxy_async();
+          tc::mbar_arrive_expect_tx(&xbar[3], (uint32_t)(2 * kv_tile));
+#pragma unroll
+          for (int h = 0; h < D / 64; ++h) {
+            tc::tma_load_3d(kv + h * 8192, &p.tmk, h * 64, jb * kBlk, (int)unit, &xbar[3]);
+            tc::tma_load_3d(kv + kv_tile + h * 8192, &p.tmv, h * 64, jb * kBlk, (int)unit, &xbar[3]);
+          }
+        }
+      }
     } else {
       const u64* fin = p.lp == 16 ? merge_lists<1>(all, work, CL)
                      : (p.lp == 32 ? merge_lists<2>(all, work, CL) : merge_lists<4>(all, work, CL));
@@ -529,6 +546,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_cluster_kernel(const __gri
     }
   }
   __syncthreads();
+  if (early) ++issued;
 
   // selected indices, ascending (written by rank 0; in fused mode after its attention
   // copies have been started)
@@ -718,18 +736,42 @@ __global__ void __launch_bounds__(kThreads, 2) decode_cluster_kernel(const __gri
     // the summary of the sequence's last block, from the keys staged here
     if (p.summ_w != nullptr && j == NB - 1) {
       const int n = Tb - j * kBlk;
-      for (int d = tid; d < D; d += kThreads) {
-        float s = 0.f;
-        if constexpr (kF32) {
+      if constexpr (kF32) {
+        for (int d = tid; d < D; d += kThreads) {
+          float s = 0.f;
 #pragma unroll 8
           for (int t = 0; t < n; ++t) s += reinterpret_cast<const float*>(Ks + t * kv_row)[d];
-        } else {
-          const int c = d >> 3, wd = d & 7;
-#pragma unroll 8
-          for (int t = 0; t < n; ++t)
-            s += __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(Ks + kv_off(t, c))[wd]);
+          p.summ_w[(unit * p.NB_cap + j) * D + d] = s / (float)n;
         }
-        p.summ_w[(unit * p.NB_cap + j) * D + d] = s / (float)n;
+      } else {
+        // every thread: one column pair over a slice of the rows, then the slices are
+        // added through the score tile (free after the softmax)
+        constexpr int kPairs = D / 2, kSlices = kThreads / kPairs, kRowsPer = kBlk / kSlices;
+        float* red = Ss;
+        const int cp = tid % kPairs, sl = tid / kPairs;
+        const int c = (2 * cp) >> 3, wd = (2 * cp) & 7;
+        const int t_end = min(n, (sl + 1) * kRowsPer);
+        float a0 = 0.f, a1 = 0.f, b0 = 0.f, b1 = 0.f;
+        int t = sl * kRowsPer;
+        for (; t + 1 < t_end; t += 2) {
+          const __nv_bfloat162 x = *reinterpret_cast<const __nv_bfloat162*>(Ks + kv_off(t, c) + 2 * wd);
+          const __nv_bfloat162 y = *reinterpret_cast<const __nv_bfloat162*>(Ks + kv_off(t + 1, c) + 2 * wd);
+          a0 += __low2float(x); a1 += __high2float(x);
+          b0 += __low2float(y); b1 += __high2float(y);
+        }
+        if (t < t_end) {
+          const __nv_bfloat162 x = *reinterpret_cast<const __nv_bfloat162*>(Ks + kv_off(t, c) + 2 * wd);
+          a0 += __low2float(x); a1 += __high2float(x);
+        }
+        red[sl * D + 2 * cp] = a0 + b0;
+        red[sl * D + 2 * cp + 1] = a1 + b1;
+        __syncthreads();
+        for (int d = tid; d < D; d += kThreads) {
+          float s = 0.f;
+#pragma unroll
+          for (int q = 0; q < kSlices; ++q) s += red[q * D + d];
+          p.summ_w[(unit * p.NB_cap + j) * D + d] = s / (float)n;
+        }
       }
     }
     if (issued < n_my) {
