@@ -224,6 +224,32 @@ def measured_peaks():
 
 # ----------------------------------------------------------------------- our arm ----
 
+# ---- the job across ranks (one process per GPU; replicas on independent sequences) ------
+
+def rank_seed(rank, r=0):
+    """Seed of rank `rank`'s r-th input copy: every rank decodes its own sequences."""
+    return 1000 + 2 + 7919 * rank + 101 * r
+
+
+def max_over_ranks(x, world, device):
+    """The slowest rank's value (step time of the whole job)."""
+    if world == 1:
+        return float(x)
+    t = torch.tensor([float(x)], device=device, dtype=torch.float64)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_rate(rate, world, device):
+    """A whole-job rate from per-rank rates: the slowest rank's rate times the rank count
+    (every rank does the same work)."""
+    if world == 1:
+        return float(rate)
+    t = torch.tensor([float(rate)], device=device, dtype=torch.float64)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MIN)
+    return float(t.item()) * world
+
+
 def run_ours(args, rank, world, local_rank):
     import query_aware_block_b200 as lsa
 
@@ -231,7 +257,7 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.set_device(dev)
     wl = args.workload
     # one step's algorithmic bytes set the rotation depth
-    base = make_case(wl, 1000 + 2 + 7919 * rank, "cpu" if wl == "tiny_decode" else dev)
+    base = make_case(wl, rank_seed(rank), "cpu" if wl == "tiny_decode" else dev)
     dec_bytes, _ = algorithmic_bytes(base)
     step_bytes = dec_bytes
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
@@ -241,7 +267,7 @@ def run_ours(args, rank, world, local_rank):
     B, Hkv, G, D, T_cap = base.shape
     copies = []
     for r in range(R):
-        c = base if r == 0 else make_case(wl, 1000 + 2 + 7919 * rank + 101 * r, dev)
+        c = base if r == 0 else make_case(wl, rank_seed(rank, r), dev)
         q, k, v, sl = (t.to(dev) for t in (c.q, c.k, c.v, c.seqlens))
         summ = torch.zeros(B, Hkv, -(-T_cap // 64), D, device=dev)
         lsa.lsa_build_summaries(k, sl, summ)  # prefill-time summaries (not timed)
@@ -316,11 +342,7 @@ def run_ours(args, rank, world, local_rank):
         e_stop.record(stream)
         torch.cuda.synchronize()
         barrier()
-    ms_total = e_start.elapsed_time(e_stop)
-    t = torch.tensor([ms_total], device=dev, dtype=torch.float64)
-    if world > 1:
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-    ms_total = float(t.item())
+    ms_total = max_over_ranks(e_start.elapsed_time(e_stop), world, dev)
     ms_step = ms_total / K
     tokens = world * B * K
     value = tokens / (ms_total / 1e3)
@@ -354,10 +376,7 @@ def run_ours(args, rank, world, local_rank):
     # end to end through the C ABI with pinned host buffers
     flags = lsa.LSA_FLAG_PDL if args.overlap else 0
     e2e = run_e2e(args, lsa, copies, base, dev, topk, ns, nl, flags)
-    if world > 1:
-        te = torch.tensor([e2e["value"]], device=dev, dtype=torch.float64)
-        torch.distributed.all_reduce(te, op=torch.distributed.ReduceOp.MIN)  # slowest rank
-        e2e["value"] = float(te.item()) * world
+    e2e["value"] = job_rate(e2e["value"], world, dev)
 
     result = {
         "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": K,
