@@ -9,23 +9,24 @@
 //   stable rows (active == 0) keep the cached output and log-sum-exp, bit-exactly.
 //
 // How (B200):
-//   * Each CTA of the cluster owns a contiguous slice of the prefix blocks.  It scores its
-//     slice for every active token (a warp per summary row, coalesced float4), keeps each
-//     token's local top-k as 64-bit keys, and pushes the lists to every peer through
-//     distributed shared memory.  After one cluster barrier a batched tree of warp-wide
-//     bitonic merges yields every token's global k-th best key: the token's threshold.
-//   * A block of this CTA's slice is in the union iff some active token's key for it
-//     clears that token's threshold, so every CTA decides its own part of the union from
-//     the scores it already holds and attends exactly those blocks: the union is loaded
-//     from HBM once, spread over the cluster, with no redistribution.
+//   * Each CTA of the cluster owns a contiguous slice of the prefix blocks, copied into
+//     shared memory by one bulk copy at launch.  It scores its slice for 8 active tokens
+//     at a time (lane = token x quarter of a summary row, the summed queries in registers,
+//     4 rows in flight per warp), keeps each token's local top-m as 64-bit keys, and
+//     pushes the lists to every peer with st.async into a double-buffered receive area
+//     whose bytes complete on an mbarrier (no cluster-wide barrier).
+//   * A warp per token runs a tournament over the token's CL sorted lists (the warp
+//     maximum of the list heads, m rounds): its selected blocks go into a bitmap of the
+//     union, so every CTA holds the same union U(b, g) and attends entries rank, rank + CL,
+//     ... of its ascending list (balanced over the cluster).
 //   * Attention rows (active token x head) are processed 32 at a time (two mma m-tiles):
-//     K/V blocks are staged with cp.async into swizzled shared memory (2 stages, prefetch
-//     across row chunks; later chunks re-read the blocks from L2), S = Q K^T and O += P V
-//     on mma.sync m16n8k16 bf16, online softmax in base 2.
+//     K/V blocks arrive as TMA boxes (128-byte swizzle) on a 2-stage ring with per-stage
+//     mbarriers, S = Q K^T and O += P V on mma.sync m16n8k16 bf16, online softmax in base 2.
 //   * Each CTA writes its per-row partial (acc, m, l) to the caller's workspace; after a
-//     second cluster barrier every CTA merges a 1/CL slice of the outputs by log-sum-exp.
-//     Stable rows are copied from the cache, the union list is written by offsets that the
-//     CTAs exchange over DSMEM.
+//     cluster barrier every CTA merges a 1/CL slice of the outputs by log-sum-exp (all
+//     loads issued before use).  Stable rows are copied from the cache; rank 0 writes the
+//     union list.
+//   Every mbarrier wait is bounded (about 2 s); a timeout sets a device status word.
 #include <math.h>
 
 #include <mutex>
@@ -90,7 +91,7 @@ __host__ __device__ inline size_t al128(size_t x) { return (x + 127) & ~(size_t)
 struct BQLayout {
   size_t act, stab, ulist, ubits, qs, ss, ps, alpha, region, total;
   // selection buffers, inside `region` (dead once the attention starts)
-  size_t qsum, keys, top, recv, work, sumbuf, qrows;
+  size_t qsum, keys, top, recv, sumbuf, qrows;
   size_t kv_tile;
 };
 
@@ -116,7 +117,6 @@ __host__ __device__ inline BQLayout bq_layout(int D, int per_max, int NBp, int G
   L.keys = r; r = al128(r + (size_t)kTokChunk * per_max * 8);
   L.top = r;  r = al128(r + (size_t)kTokChunk * kLP * 8);
   L.recv = r; r = al128(r + (size_t)2 * kMaxCluster * kTokChunk * kLP * 8);  // two buffers
-  L.work = r; r = al128(r + (size_t)kTokChunk * (kMaxCluster / 2) * kLP * 8);
   L.sumbuf = r; r = al128(r + (size_t)stage_rows * D * 4);
   L.qrows = r; r = al128(r + (size_t)kTokChunk * G * D * 2);  // a token chunk's query rows
   L.total = off + (r > kv_bytes ? r : kv_bytes);
@@ -147,7 +147,6 @@ __global__ void __launch_bounds__(kThreads, 2) blockquery_kernel(const __grid_co
   u64* keys = reinterpret_cast<u64*>(region + Lo.keys);
   u64* top = reinterpret_cast<u64*>(region + Lo.top);
   u64* recv = reinterpret_cast<u64*>(region + Lo.recv);
-  u64* work = reinterpret_cast<u64*>(region + Lo.work);
   float* sumbuf = reinterpret_cast<float*>(region + Lo.sumbuf);
   unsigned char* qrows = region + Lo.qrows;
   unsigned char* kv = region + ((1024u - (tc::smem_u32(region) & 1023u)) & 1023u);
@@ -342,47 +341,34 @@ __global__ void __launch_bounds__(kThreads, 2) blockquery_kernel(const __grid_co
         st_async(map_rank(rb + (size_t)rank * kTokChunk * kLP + rem, peer), top[rem], map_rank(&xbar[buf], peer));
       }
       tc::mbar_wait(&xbar[buf], (uint32_t)((chunk_id >> 1) & 1), &xabort, kWaitBudget);
-      // batched merge trees: token a's lists are rb[c][a][*], c < CL; the result is the
-      // token's global top list, whose first m keys are its selected blocks
-      {
-        u64* src = rb;
-        u64* dst = work;
-        int cs = kTokChunk * kLP, as = kLP;
-        for (int n = CL; n > 1; n >>= 1) {
-          const int pairs = n >> 1;
-          const int nm = na * pairs;
-          const int pl2 = __ffs(pairs) - 1;  // pairs is a power of two
-          // 4 independent merges per warp at a time (interleaved shared-memory searches)
-          for (int t0 = 4 * warp; t0 < nm; t0 += 4 * kWarps) {
-            const u64* LA[4];
-            const u64* LB[4];
-            u64* LC[4];
+      // every token's m best keys by a tournament over its CL sorted lists rb[c][a][*]: a
+      // warp per token, lane l (and l + 16) holds the head of list l & 15; each round the
+      // warp's maximum is a selected block and its list advances (keys are unique, so
+      // exactly one list holds it).  m rounds of 4 shuffle steps, no block barrier.
+      for (int a2 = warp; a2 < na; a2 += kWarps) {
+        const int c = lane & 15;
+        const u64* L = rb + (size_t)c * kTokChunk * kLP + a2 * kLP;
+        int ptr = 0;
+        u64 head = c < CL ? L[0] : 0ull;
+        for (int r = 0; r < m; ++r) {
+          u64 best = head;
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              const int t = min(t0 + q, nm - 1);
-              const int a2 = t >> pl2, pr = t & (pairs - 1);
-              LA[q] = src + (size_t)(2 * pr) * cs + a2 * as;
-              LB[q] = src + (size_t)(2 * pr + 1) * cs + a2 * as;
-              LC[q] = dst + (size_t)a2 * (kMaxCluster / 2) * kLP + pr * kLP;
-            }
-            warp_merge_rank16<4>(LA, LB, LC, min(4, nm - t0));
+          for (int o = 8; o >= 1; o >>= 1) {
+            const u64 y = __shfl_xor_sync(0xffffffffu, best, o);
+            best = y > best ? y : best;
           }
-          __syncthreads();
-          u64* t2 = src;
-          src = dst;
-          dst = t2;
-          cs = kLP;
-          as = (kMaxCluster / 2) * kLP;
-        }
-        for (int a2 = warp; a2 < na; a2 += kWarps) {
-          const u64 x = lane < m ? src[(size_t)a2 * as + lane] : 0ull;  // m <= 16
-          if (x != 0ull) {
-            const int j = key_block(x);
+          if (best == 0ull) break;  // (uniform: both half-warps hold the same heads)
+          if (head == best) {
+            ++ptr;
+            head = ptr < kLP ? L[ptr] : 0ull;
+          }
+          if (lane == 0) {
+            const int j = key_block(best);
             atomicOr(&ubits[j >> 5], 1u << (j & 31));
           }
         }
       }
-      __syncthreads();  // (qsum, top, keys and work are rewritten by the next chunk)
+      __syncthreads();  // (qsum, top and keys are rewritten by the next chunk)
     }
   } else if (staged_rows > 0) {
     __syncthreads();  // (thread 0's mbarrier initialisation first)
