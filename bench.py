@@ -463,6 +463,8 @@ def oracle_step_runner(wl, seed=1002):
     B, Hkv, G, D, T_cap = case.shape
     summ = oracle.summaries(case.k, case.seqlens)  # prefill-time, not timed
 
+    kv_cache = {}  # the K/V of a head subset, made contiguous once (outside any timing)
+
     def run(heads=None):
         heads = heads or list(range(Hkv))
         for b in range(B):
@@ -474,8 +476,13 @@ def oracle_step_runner(wl, seed=1002):
             summ[b:b + 1, :, j] = oracle.summaries(kb, torch.tensor([T - j * 64]))[:, :, 0]
         hs = heads
         q = case.q.view(B, Hkv, G, D)[:, hs].reshape(B, len(hs) * G, D).contiguous()
-        k = case.k[:, hs].contiguous() if len(hs) < Hkv else case.k
-        v = case.v[:, hs].contiguous() if len(hs) < Hkv else case.v
+        if len(hs) < Hkv:
+            key = tuple(hs)
+            if key not in kv_cache:
+                kv_cache[key] = (case.k[:, hs].contiguous(), case.v[:, hs].contiguous())
+            k, v = kv_cache[key]
+        else:
+            k, v = case.k, case.v
         s = oracle.block_scores(q, summ[:, hs].contiguous(), case.seqlens)
         idx, nsel = oracle.select(s, case.seqlens, case.topk, case.n_sink, case.n_local)
         return oracle.decode_attn(q, k, v, case.seqlens, idx, nsel)
@@ -512,6 +519,7 @@ def run_reference(args):
     while heads > 1 and (K + W) * t_full * heads / Hkv > budget:
         heads -= 1
     hs = list(range(heads))
+    run(hs)  # (makes the head subset's K/V contiguous before the timed steps)
     for _ in range(W):
         run(hs)
     timed = K
@@ -533,7 +541,9 @@ def run_reference(args):
         "warmup": W, "ms_per_step": round(dt / timed * 1e3, 3), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": wl}, "impl": "reference",
-        "cpu_baseline": {"value": round(value, 3), "unit": UNIT, "cores": oracle.num_threads(),
+        # (the oracle's OpenMP loops run over (sequence, KV head) units)
+        "cpu_baseline": {"value": round(value, 3), "unit": UNIT,
+                         "cores": min(oracle.num_threads(), meta["B"] * heads),
                          "kind": "oracle", "sample": sample},
         "e2e": {"value": round(value, 3), "unit": UNIT, "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
