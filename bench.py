@@ -402,38 +402,57 @@ def run_ours(args, rank, world, local_rank):
     return result
 
 
+def _carve(buf, specs):
+    """Views of one byte buffer: specs = [(dtype, shape), ...], each view 16-byte aligned."""
+    out, off = [], 0
+    for dt, shape in specs:
+        n = math.prod(shape) * torch.tensor([], dtype=dt).element_size()
+        out.append(buf[off:off + n].view(dt).view(shape))
+        off += (n + 15) // 16 * 16
+    return out, off
+
+
 def run_e2e(args, lsa, copies, base, dev, topk, ns, nl, flags):
     """Same metric through the public API, eager launches, pinned host buffers: every step
-    copies in q and the newest token's k and v and copies out o, lse and idx."""
+    copies in q and the newest token's k and v (one host-to-device copy of one packed
+    buffer, then the token's k and v are written into the cache) and copies out o, lse and
+    idx (one device-to-host copy of one packed buffer)."""
     R = len(copies)
     B, Hkv, G, D, T_cap = base.shape
+    dt = copies[0]["q"].dtype
     n = max(R, min(args.e2e_steps, args.steps))
-    hq = [copies[r]["q"].cpu().pin_memory() for r in range(R)]
     last = [int(x) - 1 for x in base.seqlens.tolist()]
-    hk = [torch.stack([copies[r]["k"][b, :, last[b]] for b in range(B)]).cpu().pin_memory() for r in range(R)]
-    hv = [torch.stack([copies[r]["v"][b, :, last[b]] for b in range(B)]).cpu().pin_memory() for r in range(R)]
-    ho = torch.empty_like(copies[0]["o"], device="cpu").pin_memory()
-    hl = torch.empty_like(copies[0]["lse"], device="cpu").pin_memory()
-    hi = torch.empty_like(copies[0]["idx"], device="cpu").pin_memory()
-    kv_stage = torch.empty_like(hk[0], device=dev)
-    h2d = hq[0].numel() * hq[0].element_size() + 2 * hk[0].numel() * hk[0].element_size()
-    d2h = ho.numel() * ho.element_size() + hl.numel() * 4 + hi.numel() * 4
+    in_specs = [(dt, tuple(copies[0]["q"].shape)), (dt, (B, Hkv, D)), (dt, (B, Hkv, D))]
+    out_specs = [(dt, tuple(copies[0]["o"].shape)), (torch.float32, tuple(copies[0]["lse"].shape)),
+                 (torch.int32, tuple(copies[0]["idx"].shape))]
+    _, in_bytes = _carve(torch.empty(1 << 20, dtype=torch.uint8), in_specs)
+    _, out_bytes = _carve(torch.empty(1 << 20, dtype=torch.uint8), out_specs)
+    in_host = []
+    for r in range(R):
+        hb = torch.empty(in_bytes, dtype=torch.uint8).pin_memory()
+        (hq, hk, hv), _ = _carve(hb, in_specs)
+        hq.copy_(copies[r]["q"].cpu())
+        hk.copy_(torch.stack([copies[r]["k"][b, :, last[b]] for b in range(B)]).cpu())
+        hv.copy_(torch.stack([copies[r]["v"][b, :, last[b]] for b in range(B)]).cpu())
+        in_host.append(hb)
+    in_dev = torch.empty(in_bytes, dtype=torch.uint8, device=dev)
+    (q_dev, k_new, v_new), _ = _carve(in_dev, in_specs)
+    out_dev = torch.empty(out_bytes, dtype=torch.uint8, device=dev)
+    (o_dev, lse_dev, idx_dev), _ = _carve(out_dev, out_specs)
+    out_host = torch.empty(out_bytes, dtype=torch.uint8).pin_memory()
+    h2d = sum(math.prod(sh) * torch.tensor([], dtype=d).element_size() for d, sh in in_specs)
+    d2h = sum(math.prod(sh) * torch.tensor([], dtype=d).element_size() for d, sh in out_specs)
 
     def one(i):
         c = copies[i % R]
-        c["q"].copy_(hq[i % R], non_blocking=True)
-        kv_stage.copy_(hk[i % R], non_blocking=True)
+        in_dev.copy_(in_host[i % R], non_blocking=True)
         for b in range(B):
-            c["k"][b, :, last[b]].copy_(kv_stage[b])
-        kv_stage.copy_(hv[i % R], non_blocking=True)
-        for b in range(B):
-            c["v"][b, :, last[b]].copy_(kv_stage[b])
-        lsa.lsa_sparse_attn_decode(c["q"], c["k"], c["v"], c["sl"], c["o"], topk, summ=c["summ"],
+            c["k"][b, :, last[b]].copy_(k_new[b])
+            c["v"][b, :, last[b]].copy_(v_new[b])
+        lsa.lsa_sparse_attn_decode(q_dev, c["k"], c["v"], c["sl"], o_dev, topk, summ=c["summ"],
                                    n_sink=ns, n_local=nl, refresh_last_summary=True,
-                                   idx_out=c["idx"], lse=c["lse"], flags=flags)
-        ho.copy_(c["o"], non_blocking=True)
-        hl.copy_(c["lse"], non_blocking=True)
-        hi.copy_(c["idx"], non_blocking=True)
+                                   idx_out=idx_dev, lse=lse_dev, flags=flags)
+        out_host.copy_(out_dev, non_blocking=True)
 
     for i in range(min(n, 3 * R)):
         one(i)
@@ -450,7 +469,8 @@ def run_e2e(args, lsa, copies, base, dev, topk, ns, nl, flags):
     ms = e0.elapsed_time(e1)
     return {"value": round(B * n / (ms / 1e3), 1), "unit": UNIT, "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": d2h, "steps": n, "host_wall_s": round(wall, 3),
-            "path": "python ctypes -> lsa_sparse_attn_decode (fused, with summary refresh), eager"}
+            "path": "python ctypes -> lsa_sparse_attn_decode (fused, with summary refresh), eager; "
+                    "one packed host-to-device and one packed device-to-host copy per step"}
 
 
 # ------------------------------------------------------------------ CPU (oracle) arm ----

@@ -180,6 +180,8 @@ def _run_both_modes(lsa, case, dtype, check_sel=True):
     (3, 2, 4, 128, [0, 100, 64 * 70 + 1], 16, 1, 2, torch.bfloat16),  # empty sequence
     (20, 3, 2, 64, 64 * 40, 4, 1, 1, torch.bfloat16),  # 60 units -> 8-CTA clusters, 1 CTA of work
     (80, 1, 4, 128, 64 * 20, 6, 1, 2, torch.float32),  # 80 units -> 4-CTA clusters, 2 blocks each
+    # 1,100 blocks: 69 summary rows per CTA, two scoring passes (the second from global memory)
+    (1, 1, 8, 128, 64 * 1100 + 7, 16, 1, 2, torch.bfloat16),
 ])
 def test_decode_matches_oracle(lsa, B, Hkv, G, D, T, topk, ns, nl, dtype):
     T_cap = max(T) if isinstance(T, list) else T
