@@ -104,46 +104,4 @@ __device__ __forceinline__ void warp_merge_desc(unsigned long long (&x)[E]) {
   }
 }
 
-// Merge by rank, without shuffles: Q independent merges of two descending lists of 16
-// unique keys (zero padded at the end), A[q] and B[q], into the top 16 of their union,
-// C[q] (zero padded), one merge per warp at a time.  Lane l takes key (l & 15) of A (l < 16)
-// or of B; its rank in the union is its own index plus the number of keys of the other
-// list above it (a 5-step binary search in shared memory), and it is stored at that rank
-// if the rank is below 16.  The Q searches are interleaved stage by stage.  Only the
-// first nq merges are done (nq uniform across the warp, nq <= Q).  C[q] must not overlap
-// A[q] or B[q]; the warp is synchronised on return.
-template <int Q>
-__device__ __forceinline__ void warp_merge_rank16(const unsigned long long* const (&A)[Q],
-                                                  const unsigned long long* const (&B)[Q],
-                                                  unsigned long long* const (&C)[Q], int nq) {
-  const int lane = threadIdx.x & 31, i = lane & 15;
-  unsigned long long x[Q];
-  const unsigned long long* other[Q];
-  int lo[Q];
-#pragma unroll
-  for (int q = 0; q < Q; ++q) {
-    const int qq = q < nq ? q : 0;
-    x[q] = (lane < 16 ? A[qq] : B[qq])[i];
-    other[q] = lane < 16 ? B[qq] : A[qq];
-    lo[q] = 0;
-  }
-#pragma unroll
-  for (int step = 8; step >= 1; step >>= 1) {
-#pragma unroll
-    for (int q = 0; q < Q; ++q) lo[q] += other[q][lo[q] + step - 1] > x[q] ? step : 0;
-  }
-#pragma unroll
-  for (int q = 0; q < Q; ++q) lo[q] += other[q][lo[q]] > x[q] ? 1 : 0;
-#pragma unroll
-  for (int q = 0; q < Q; ++q)
-    if (q < nq && lane < 16) C[q][lane] = 0ull;
-  __syncwarp();
-#pragma unroll
-  for (int q = 0; q < Q; ++q) {
-    const int r = i + lo[q];
-    if (q < nq && x[q] != 0ull && r < 16) C[q][r] = x[q];
-  }
-  __syncwarp();
-}
-
 }  // namespace lsa
