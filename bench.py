@@ -69,6 +69,8 @@ def parse():
                     default="gqa_decode_64k")
     ap.add_argument("--prefill-sink", type=float, default=0.0,
                     help="blasst_prefill_32k: plant an attention sink of this logit height")
+    ap.add_argument("--prefill-qscale", type=float, default=1.0,
+                    help="prefill: scale the queries (peakier softmax, more skippable tiles)")
     ap.add_argument("--rotate", type=int, default=0, help="input copies (0 = auto, > 4x L2)")
     ap.add_argument("--e2e-steps", type=int, default=2000)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
@@ -394,6 +396,7 @@ def run_ours(args, rank, world, local_rank):
                    "overlapped_launch": bool(args.overlap)},
         "effective_gbs": round(step_bytes / (ms_step * 1e-3) / 1e9, 1),
         "bytes_per_step": step_bytes,
+        "needle_recall": needle_recall(base, copies[0]["idx"]),
         "roofline": roofline,
         "e2e": e2e,
         "gpu_launches": K,
@@ -410,6 +413,16 @@ def _carve(buf, specs):
         out.append(buf[off:off + n].view(dt).view(shape))
         off += (n + 15) // 16 * 16
     return out, off
+
+
+def needle_recall(case, idx):
+    """Planted needle blocks (synth) found in the selected indices of the same inputs."""
+    planted = sum(len(blocks) for _, _, blocks in case.needles)
+    if planted == 0:
+        return None
+    sel = idx.cpu()
+    found = sum(int(j) in set(sel[b, g].tolist()) for b, g, blocks in case.needles for j in blocks)
+    return {"found": found, "planted": planted, "fraction": round(found / planted, 4)}
 
 
 def run_e2e(args, lsa, copies, base, dev, topk, ns, nl, flags):
@@ -598,7 +611,7 @@ def run_prefill(args):
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
     case = synth.prefill_case(B=1, Hq=32, Hkv=8, L=32768, D=128, lam=1e-3, sink=args.prefill_sink,
-                              seed=1005, device=dev)
+                              q_scale=args.prefill_qscale, seed=1005, device=dev)
     B, Hq, L, D = case.q.shape
     o = torch.empty_like(case.q)
     lse = torch.empty(B, Hq, L, device=dev)
@@ -635,7 +648,9 @@ def run_prefill(args):
         "value": round(tflops, 1), "unit": "TFLOP/s", "n_gpus": 1, "steps": K, "warmup": args.warmup,
         "ms_per_step": round(ms, 4), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16", "data": "synthetic (seeded N(0,1) q/k/v with RoPE theta 1e4"
-                                  + (f", attention sink {args.prefill_sink}" if args.prefill_sink else "") + ")",
+                                  + (f", attention sink {args.prefill_sink}" if args.prefill_sink else "")
+                                  + (f", q scaled by {args.prefill_qscale}" if args.prefill_qscale != 1.0 else "")
+                                  + ")",
         "config": {"workload": "blasst_prefill_32k", "batch": B, "q_heads": Hq, "kv_heads": case.k.shape[1],
                    "head_dim": D, "seq_len": L, "tiles": "128 x 64", "lambda": case.lam,
                    "l2": "inputs (512 MB) larger than L2"},
