@@ -8,8 +8,9 @@ the CUDA library in ``query_aware_block_b200``.
 
 Parity status of each function (what pins it is in tests/test_oracle_pins.py):
   summaries, block_scores, select, decode_attn, blockquery_select, blockquery_attn,
-  blasst_prefill -- all pinned (textbook special cases, brute force, library routines,
-  closed forms and invariants).
+  blasst_prefill, losa_classify, blockquery_intra_merge (and the losa_step composition)
+  -- all pinned (textbook special cases, brute force, library routines, closed forms and
+  invariants).
 """
 from __future__ import annotations
 
@@ -224,3 +225,60 @@ def blasst_prefill(q, k, v, units, lam, tq=128, tk=64, scale=None, forced_bits=N
                                   tq, tk, n, _p(units), _p(fb), words, _p(o), _p(lse),
                                   _p(bits), _p(gap))
     return dict(o=o, lse=lse, bits=bits.to(torch.int64) & 0xFFFFFFFF, gap=gap)
+
+
+def losa_classify(q, q_prev, tau=0.0, n_top=0):
+    """Active / stable tokens from the mean squared change of their queries.
+
+    q, q_prev [B,Hq,Tq,D] (same dtype).  Returns (mse fp64 [B,Tq], active uint8 [B,Tq]):
+    n_top > 0 marks the n_top largest changes (ties: lower index), else mse > tau."""
+    q, q_prev = q.contiguous(), q_prev.contiguous()
+    assert q.dtype == q_prev.dtype and q.shape == q_prev.shape
+    B, Hq, Tq, D = q.shape
+    mse = torch.empty(B, Tq, dtype=torch.float64)
+    act = torch.empty(B, Tq, dtype=torch.uint8)
+    _load().oracle_losa_classify(_p(q), _p(q_prev), _dt(q), B, Hq, Tq, D,
+                                 ctypes.c_double(float(tau)), int(n_top), _p(mse), _p(act))
+    return mse, act
+
+
+def blockquery_intra_merge(q, k, v, T_prefix, o_pre, lse_pre, scale=None):
+    """Bidirectional attention over the block's own tokens (rows T_prefix .. T_prefix+Tq-1
+    of k and v), merged with the prefix result (o_pre, lse_pre) by log-sum-exp.
+
+    The prefix result is widened exactly to fp64.  -> (o fp64 [B,Hq,Tq,D], lse fp64 [B,Hq,Tq])."""
+    q, k, v = q.contiguous(), k.contiguous(), v.contiguous()
+    assert q.dtype == k.dtype == v.dtype
+    B, Hq, Tq, D = q.shape
+    _, Hkv, T_cap, _ = k.shape
+    assert T_prefix + Tq <= T_cap
+    G = Hq // Hkv
+    op = o_pre.to(torch.float64).contiguous()
+    lp = lse_pre.to(torch.float64).contiguous()
+    o = torch.empty(B, Hq, Tq, D, dtype=torch.float64)
+    lse = torch.empty(B, Hq, Tq, dtype=torch.float64)
+    _load().oracle_blockquery_intra_merge(_p(q), _p(k), _p(v), _dt(q), B, Hkv, G, D, Tq,
+                                          T_prefix, T_cap, ctypes.c_double(_scale(scale, D)),
+                                          _p(op), _p(lp), _p(o), _p(lse))
+    return o, lse
+
+
+def losa_step(q, q_prev, k, v, summ, T_prefix, o_cache, lse_cache, topk, tau=0.0, n_top=0,
+              n_sink=0, n_local=0, blk=64, scale=None, union=None):
+    """One LoSA denoising step in the oracle, in the pages' order: classify the tokens,
+    select and attend the prefix for the active ones (stable ones keep the cache), attend
+    inside the block and merge.  `union` = (union_idx, union_cnt) replaces the oracle's own
+    union (to evaluate another implementation's choice among tied scores).
+
+    Returns dict(mse, active, union_idx, union_cnt, o_prefix, lse_prefix, o, lse); the
+    prefix part is fp64 (not rounded)."""
+    mse, active = losa_classify(q, q_prev, tau, n_top)
+    if union is None:
+        uidx, ucnt = blockquery_select(q, summ, active, T_prefix, topk, n_sink, n_local, blk, scale)
+    else:
+        uidx, ucnt = union
+    o_p, lse_p = blockquery_attn(q, k, v, active, o_cache, lse_cache, uidx, ucnt, T_prefix,
+                                 blk, scale)
+    o, lse = blockquery_intra_merge(q, k, v, T_prefix, o_p, lse_p, scale)
+    return dict(mse=mse, active=active, union_idx=uidx, union_cnt=ucnt, o_prefix=o_p,
+                lse_prefix=lse_p, o=o, lse=lse)

@@ -31,6 +31,14 @@
  *                            order, skipping a tile whose row maxima all trail the running
  *                            maxima by more than ln(lambda)
  *                            [BLASST, "2. 방법론", "핵심 아이디어" and "알고리즘 및 커널 설계"]
+ *   oracle_losa_classify     active / stable tokens by the mean squared change of their
+ *                            queries between denoising steps [LoSA, "2. 방법론": the query
+ *                            change (MSE) of every step sorts tokens into active and stable]
+ *   oracle_blockquery_intra_merge
+ *                            bidirectional attention inside the query block, merged with
+ *                            the prefix result by log-sum-exp [LoSA, "2. 방법론": stable
+ *                            tokens reuse the prefix statistics and output; the block
+ *                            itself is attended every step]
  *
  * Readings taken where the pages are silent (each also listed in the design doc):
  *   - a partial last block is averaged over its valid tokens only;
@@ -39,6 +47,11 @@
  *   - the forced blocks are counted inside the n selected blocks;
  *   - the BLASST test quantifies over rows: skip iff every row's
  *     (tile row max - running row max) < ln(lambda); strict '<' as printed.
+ *   - LoSA's query change is the mean over all query heads and dims of the squared
+ *     difference; active iff it exceeds tau (or: the n_top largest, ties to the lower
+ *     index);
+ *   - attention inside the query block is bidirectional over all of its tokens, computed
+ *     for every token each step, and joined with the prefix part by log-sum-exp.
  *
  * Parallelism: OpenMP over independent (batch, kv head) / (batch, head, q tile) units
  * only; each unit is computed by one thread exactly as a serial loop would.
@@ -505,5 +518,97 @@ void oracle_blasst_prefill(const void* q, const void* k, const void* v, int dtyp
     free(r);
     free(l);
     free(m);
+  }
+}
+
+/* ------------------------------------------------------------------------------------
+ * LoSA token activity between two denoising steps.
+ *   mse[b,i] = (1 / (Hq*D)) * sum over query heads h and dims d of
+ *              (q[b,h,i,d] - q_prev[b,h,i,d])^2
+ * i.e. the mean squared change of token i's query vectors (all heads).
+ * Rule: n_top > 0  -> the n_top tokens of largest mse are active (equal mse: the lower
+ *                     token index ranks first);
+ *       n_top == 0 -> token i is active iff mse[b,i] > tau (strict).
+ * q, q_prev [B,Hq,Tq,D]; mse [B,Tq] out (double); active [B,Tq] out (1 = active).
+ * ---------------------------------------------------------------------------------- */
+void oracle_losa_classify(const void* q, const void* q_prev, int dtype, int B, int Hq, int Tq,
+                          int D, double tau, int n_top, double* mse, uint8_t* active) {
+  for (int b = 0; b < B; ++b) {
+    for (int i = 0; i < Tq; ++i) {
+      double sum = 0.0;
+      for (int h = 0; h < Hq; ++h) {
+        const size_t row = (((size_t)b * Hq + h) * Tq + i) * D;
+        for (int d = 0; d < D; ++d) {
+          const double diff = elem(q, dtype, row + d) - elem(q_prev, dtype, row + d);
+          sum += diff * diff;
+        }
+      }
+      mse[(size_t)b * Tq + i] = sum / ((double)Hq * (double)D);
+    }
+    for (int i = 0; i < Tq; ++i) {
+      const double mi = mse[(size_t)b * Tq + i];
+      int on;
+      if (n_top > 0) {
+        int rank = 0; /* tokens ranked before i */
+        for (int j = 0; j < Tq; ++j) {
+          const double mj = mse[(size_t)b * Tq + j];
+          if (mj > mi || (mj == mi && j < i)) ++rank;
+        }
+        on = rank < n_top;
+      } else {
+        on = mi > tau;
+      }
+      active[(size_t)b * Tq + i] = (uint8_t)on;
+    }
+  }
+}
+
+/* ------------------------------------------------------------------------------------
+ * Attention inside the query block, merged with the prefix result.
+ * Row (b, h, i) with KV group g = h / G.  The block's own tokens are rows
+ * T_prefix .. T_prefix + Tq - 1 of k and v; the row attends over all of them with no mask
+ * (bidirectional inside the block), which gives (o_in, lse_in) as in attend_row.  The
+ * prefix part (o_pre, lse_pre) is the softmax attention of the same row over its prefix
+ * tokens.  Softmax over the disjoint union of the two token sets:
+ *   lse = log(exp(lse_pre) + exp(lse_in))
+ *   o   = exp(lse_pre - lse) * o_pre + exp(lse_in - lse) * o_in
+ * (lse_pre = -inf is an empty prefix part: o = o_in, lse = lse_in).
+ * q [B,Hq,Tq,D] (dtype); k, v [B,Hkv,T_cap,D] (dtype); o_pre [B,Hq,Tq,D] and
+ * lse_pre [B,Hq,Tq] double; o, lse: same shapes, double, out.
+ * ---------------------------------------------------------------------------------- */
+void oracle_blockquery_intra_merge(const void* q, const void* k, const void* v, int dtype, int B,
+                                   int Hkv, int G, int D, int Tq, int T_prefix, int T_cap,
+                                   double scale, const double* o_pre, const double* lse_pre,
+                                   double* o, double* lse) {
+  const int Hq = Hkv * G;
+#pragma omp parallel for collapse(2) schedule(dynamic)
+  for (int b = 0; b < B; ++b) {
+    for (int h = 0; h < Hq; ++h) {
+      const int g = h / G;
+      int* toks = (int*)malloc(sizeof(int) * (size_t)Tq);
+      double* logits = (double*)malloc(sizeof(double) * (size_t)Tq);
+      double* o_in = (double*)malloc(sizeof(double) * (size_t)D);
+      for (int t = 0; t < Tq; ++t) toks[t] = T_prefix + t;
+      const size_t kvbase = ((size_t)b * Hkv + g) * (size_t)T_cap * D;
+      for (int i = 0; i < Tq; ++i) {
+        const size_t row = ((size_t)b * Hq + h) * Tq + i;
+        double lse_in;
+        attend_row(q, k, v, dtype, row * D, kvbase, D, toks, Tq, scale, logits, o_in, &lse_in);
+        const double lp = lse_pre[row];
+        if (lp == -INFINITY) {
+          for (int d = 0; d < D; ++d) o[row * D + d] = o_in[d];
+          lse[row] = lse_in;
+          continue;
+        }
+        const double mx = lp > lse_in ? lp : lse_in;
+        const double tot = mx + log(exp(lp - mx) + exp(lse_in - mx));
+        const double wp = exp(lp - tot), wi = exp(lse_in - tot);
+        for (int d = 0; d < D; ++d) o[row * D + d] = wp * o_pre[row * D + d] + wi * o_in[d];
+        lse[row] = tot;
+      }
+      free(o_in);
+      free(logits);
+      free(toks);
+    }
   }
 }

@@ -201,6 +201,41 @@ def diffusion_blockquery(seed=1004, device="cpu") -> BlockQueryCase:
 
 
 @dataclass
+class LosaCase(BlockQueryCase):
+    q_prev: torch.Tensor = None  # [B, Hq, Tq, D]: the block's queries one denoising step earlier
+
+
+def losa_case(B=1, Hkv=8, G=4, D=128, Tq=32, T_prefix=32768, n_active=8, topk=8, n_sink=0,
+              n_local=0, dtype=torch.bfloat16, theta=1e4, stable_noise=0.02, seed=1006,
+              device="cpu") -> LosaCase:
+    """A LoSA denoising step: the block-query case with the block's own keys and values at
+    cache rows T_prefix .. T_prefix + Tq - 1 (T_cap = T_prefix + Tq), plus the previous
+    step's queries.  A stable token's previous query is its query plus
+    stable_noise * N(0, I); an active token's is an independent rotated N(0, 1) draw, so
+    that the change separates the two kinds (expected squared change per element
+    stable_noise^2 against 2).  `active` is the planted set."""
+    c = blockquery_case(B=B, Hkv=Hkv, G=G, D=D, Tq=Tq, T_prefix=T_prefix, T_cap=T_prefix + Tq,
+                        n_active=n_active, topk=topk, n_sink=n_sink, n_local=n_local,
+                        dtype=dtype, theta=theta, seed=seed, device=device)
+    gen = _gen(seed + 7919, device)
+    Hq = Hkv * G
+    fresh = rope(torch.randn(B, Hq, Tq, D, generator=gen, device=device),
+                 torch.arange(T_prefix, T_prefix + Tq, device=device), theta).float()
+    near = c.q.float() + stable_noise * torch.randn(B, Hq, Tq, D, generator=gen, device=device)
+    on = c.active.bool()[:, None, :, None]
+    q_prev = torch.where(on, fresh, near).to(dtype).contiguous()
+    return LosaCase(q=c.q, k=c.k, v=c.v, active=c.active, o_cache=c.o_cache,
+                    lse_cache=c.lse_cache, T_prefix=c.T_prefix, topk=c.topk, n_sink=c.n_sink,
+                    n_local=c.n_local, q_prev=q_prev)
+
+
+def diffusion_losa_step(seed=1006, device="cpu") -> LosaCase:
+    """The diffusion block-query workload as a whole LoSA step: 32 query tokens (8 of them
+    changing), 8 KV heads x 4 q heads, D 128, prefix 32768, per-token top-8 blocks."""
+    return losa_case(seed=seed, device=device)
+
+
+@dataclass
 class PrefillCase:
     q: torch.Tensor  # [B, Hq, L, D]
     k: torch.Tensor  # [B, Hkv, L, D]

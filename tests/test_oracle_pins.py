@@ -466,3 +466,148 @@ def test_blasst_forced_bits_follow_the_given_decisions():
     for u, (b, h, a) in enumerate(units):
         nvisit = (min(a * 128 + 128, 256) - 1) // 64 + 1
         assert int(r["bits"][u, 0]) == (0b0100 if nvisit > 2 else 0)
+
+
+# ------------------------------------------------------------- LoSA step (classify) ----
+
+def _grid_bf16(shape, gen, lim=64):
+    """Values k/8 with |k| <= lim: exact in bf16, and so are their sums with eighths."""
+    return (torch.randint(-lim, lim + 1, shape, generator=gen).double() / 8).to(torch.bfloat16)
+
+
+def test_losa_classify_unchanged_queries():
+    gen = torch.Generator().manual_seed(40)
+    q = torch.randn(2, 4, 6, 16, generator=gen).to(torch.bfloat16)
+    mse, act = oracle.losa_classify(q, q.clone(), tau=0.0)
+    assert torch.count_nonzero(mse) == 0 and torch.count_nonzero(act) == 0
+    _, act = oracle.losa_classify(q, q.clone(), tau=-1.0)
+    assert bool(act.all())
+    # every change ties at 0: the n_top lowest token indices rank first
+    _, act = oracle.losa_classify(q, q.clone(), n_top=3)
+    assert act.tolist() == [[1, 1, 1, 0, 0, 0]] * 2
+
+
+def test_losa_classify_constant_shift_closed_form():
+    # token i of sequence b moves by c[b, i] in every head and dim: its MSE is c^2 exactly
+    B, Hq, Tq, D = 2, 3, 7, 16
+    gen = torch.Generator().manual_seed(41)
+    q_prev = _grid_bf16((B, Hq, Tq, D), gen)
+    c = torch.randint(0, 9, (B, Tq), generator=gen).double() / 8
+    c[0, 0] = 0.5  # a token exactly at the threshold below
+    q = (q_prev.double() + c[:, None, :, None]).to(torch.bfloat16)
+    assert torch.equal(q.double() - q_prev.double(), c[:, None, :, None].expand(B, Hq, Tq, D))
+    mse, act = oracle.losa_classify(q, q_prev, tau=0.25)
+    assert torch.equal(mse, c * c)
+    assert torch.equal(act.bool(), c * c > 0.25)
+    assert int(act[0, 0]) == 0  # strict: a change equal to tau is stable
+
+
+def test_losa_classify_single_element_change():
+    # one element (head 3, token 2, dim 17) moves by 0.5: that token's MSE is
+    # 0.25 / (Hq * D), every other token's is 0
+    B, Hq, Tq, D = 1, 5, 4, 24
+    q_prev = torch.zeros(B, Hq, Tq, D, dtype=torch.bfloat16)
+    q = q_prev.clone()
+    q[0, 3, 2, 17] = 0.5
+    mse, act = oracle.losa_classify(q, q_prev, tau=0.0)
+    expect = torch.zeros(B, Tq, dtype=torch.float64)
+    expect[0, 2] = 0.25 / (Hq * D)
+    assert torch.allclose(mse, expect, rtol=1e-15, atol=0)
+    assert act.tolist() == [[0, 0, 1, 0]]
+
+
+def test_losa_classify_top_n_is_a_stable_descending_sort():
+    # library routine: a stable sort of the negated changes ranks the tokens (equal changes:
+    # lower index first); duplicated shifts plant exact ties
+    B, Hq, Tq, D = 3, 4, 16, 8
+    gen = torch.Generator().manual_seed(42)
+    q_prev = _grid_bf16((B, Hq, Tq, D), gen)
+    c = torch.randint(0, 5, (B, Tq), generator=gen).double() / 8  # many equal shifts
+    q = (q_prev.double() + c[:, None, :, None]).to(torch.bfloat16)
+    for n in (1, 5, 16):
+        mse, act = oracle.losa_classify(q, q_prev, n_top=n)
+        for b in range(B):
+            order = torch.sort(-c[b] * c[b], stable=True).indices
+            expect = torch.zeros(Tq, dtype=torch.uint8)
+            expect[order[:n]] = 1
+            assert torch.equal(act[b], expect), (n, b)
+        assert torch.equal(mse, c * c)
+
+
+# ---------------------------------------------------- LoSA step (intra-block + merge) ----
+
+def _dense_rows(q, k, v, scale):
+    """Library routines: fp64 SDPA with no mask and the log-sum-exp of the logits."""
+    o = F.scaled_dot_product_attention(q.double(), k.double(), v.double(), scale=scale)
+    lse = torch.logsumexp(scale * q.double() @ k.double().transpose(-1, -2), dim=-1)
+    return o, lse
+
+
+def test_losa_step_all_blocks_equals_dense_attention_over_prefix_and_block():
+    # every token active and every prefix block selected: the prefix part is dense, the
+    # block part is bidirectional, so the merged row is plain softmax attention over all
+    # T_prefix + Tq keys
+    case = synth.losa_case(B=1, Hkv=2, G=2, D=32, Tq=6, T_prefix=320, n_active=6, topk=16,
+                           dtype=torch.float32, seed=43)
+    T, Tq, D = case.T_prefix, 6, 32
+    sl = torch.full((1,), T, dtype=torch.int32)
+    summ = oracle.summaries(case.k[:, :, :T].contiguous(), sl)
+    r = oracle.losa_step(case.q, case.q_prev, case.k, case.v, summ, T, case.o_cache,
+                         case.lse_cache, topk=16, tau=0.1)
+    assert r["active"].tolist() == [[1] * 6]
+    assert r["union_cnt"].tolist() == [[5, 5]]
+    for h in range(4):
+        g = h // 2
+        o_ref, lse_ref = _dense_rows(case.q[0, h], case.k[0, g, :T + Tq], case.v[0, g, :T + Tq],
+                                     1 / math.sqrt(D))
+        assert torch.allclose(r["o"][0, h], o_ref, rtol=0, atol=1e-12)
+        assert torch.allclose(r["lse"][0, h], lse_ref, rtol=0, atol=1e-12)
+        # the prefix part alone is dense prefix attention
+        o_p, lse_p = _dense_rows(case.q[0, h], case.k[0, g, :T], case.v[0, g, :T], 1 / math.sqrt(D))
+        assert torch.allclose(r["o_prefix"][0, h], o_p, rtol=0, atol=1e-12)
+        assert torch.allclose(r["lse_prefix"][0, h], lse_p, rtol=0, atol=1e-12)
+
+
+def test_intra_merge_empty_prefix_and_single_token():
+    case = synth.losa_case(B=2, Hkv=1, G=3, D=16, Tq=5, T_prefix=128, n_active=5, topk=2,
+                           dtype=torch.float32, seed=44)
+    T = case.T_prefix
+    none_o = torch.zeros(2, 3, 5, 16, dtype=torch.float64)
+    none_l = torch.full((2, 3, 5), -math.inf, dtype=torch.float64)
+    o, lse = oracle.blockquery_intra_merge(case.q, case.k, case.v, T, none_o, none_l)
+    for b in range(2):
+        for h in range(3):
+            o_ref, lse_ref = _dense_rows(case.q[b, h], case.k[b, 0, T:T + 5], case.v[b, 0, T:T + 5], 0.25)
+            assert torch.allclose(o[b, h], o_ref, rtol=0, atol=1e-12)
+            assert torch.allclose(lse[b, h], lse_ref, rtol=0, atol=1e-12)
+    # one token in the block and no prefix: the row's output is that token's value
+    q1 = case.q[:, :, :1].contiguous()
+    o1, lse1 = oracle.blockquery_intra_merge(q1, case.k, case.v, T, none_o[:, :, :1], none_l[:, :, :1])
+    for b in range(2):
+        for h in range(3):
+            assert torch.equal(o1[b, h, 0], case.v[b, 0, T].double())
+            assert abs(float(lse1[b, h, 0]) - 0.25 * float(case.q[b, h, 0].double() @ case.k[b, 0, T].double())) < 1e-12
+
+
+def test_losa_step_stable_rows_with_exact_cache_match_recomputation():
+    # a stable token whose cache holds its exact prefix result ends where recomputing it
+    # would: dense attention over prefix and block (fp32 cache: ~1e-7)
+    case = synth.losa_case(B=1, Hkv=2, G=2, D=32, Tq=8, T_prefix=256, n_active=3, topk=16,
+                           dtype=torch.float32, seed=45)
+    T, Tq, D = case.T_prefix, 8, 32
+    sc = 1 / math.sqrt(D)
+    o_cache = torch.empty(1, 4, Tq, D)
+    lse_cache = torch.empty(1, 4, Tq)
+    for h in range(4):
+        o_p, lse_p = _dense_rows(case.q[0, h], case.k[0, h // 2, :T], case.v[0, h // 2, :T], sc)
+        o_cache[0, h], lse_cache[0, h] = o_p.float(), lse_p.float()
+    sl = torch.full((1,), T, dtype=torch.int32)
+    summ = oracle.summaries(case.k[:, :, :T].contiguous(), sl)
+    r = oracle.losa_step(case.q, case.q_prev, case.k, case.v, summ, T, o_cache, lse_cache,
+                         topk=16, n_top=3)
+    assert torch.equal(r["active"], case.active)
+    for h in range(4):
+        o_ref, lse_ref = _dense_rows(case.q[0, h], case.k[0, h // 2, :T + Tq],
+                                     case.v[0, h // 2, :T + Tq], sc)
+        assert torch.allclose(r["o"][0, h], o_ref, rtol=0, atol=1e-6)
+        assert torch.allclose(r["lse"][0, h], lse_ref, rtol=0, atol=1e-5)
