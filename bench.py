@@ -2,7 +2,8 @@
 """Benchmark of the query-aware block-sparse attention hot path on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload gqa_decode_64k|batched_decode|tiny_decode]
+                    [--workload gqa_decode_64k|batched_decode|tiny_decode|blockquery|
+                                losa_step|blasst_prefill_32k]
 
 Default workload: 64K-context GQA decode, bf16 (1 sequence, 8 KV heads x 8 query heads,
 head dim 128, 65,536 cached tokens = 1,024 blocks of 64, top-16 blocks per KV head with
@@ -65,7 +66,7 @@ def parse():
                     help="timed steps (default: 200000 decode steps; 20 prefills; 20000 block-query steps)")
     ap.add_argument("--warmup", type=int, default=None)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=sorted(WORKLOADS) + ["blockquery", "blasst_prefill_32k"],
+    ap.add_argument("--workload", choices=sorted(WORKLOADS) + ["blockquery", "blasst_prefill_32k", "losa_step"],
                     default="gqa_decode_64k")
     ap.add_argument("--prefill-sink", type=float, default=0.0,
                     help="blasst_prefill_32k: plant an attention sink of this logit height")
@@ -80,7 +81,8 @@ def parse():
     ap.add_argument("--profile-small", action="store_true",
                     help="a few launches on 2 input copies, for ncu captures")
     a = ap.parse_args()
-    defaults = {"blockquery": (20000, 200), "blasst_prefill_32k": (20, 3)}.get(a.workload, (200000, 600))
+    defaults = {"blockquery": (20000, 200), "blasst_prefill_32k": (20, 3),
+                "losa_step": (8000, 200)}.get(a.workload, (200000, 600))
     if a.steps is None:
         a.steps = defaults[0]
     if a.warmup is None:
@@ -755,13 +757,153 @@ def run_blockquery(args):
     }
 
 
+def run_losa_step(args):
+    """One LoSA denoising step of the diffusion workload (32 query tokens, prefix 32768,
+    8 KV heads x 4 query heads, top-8 blocks per active token): the tokens are classified
+    by the change of their queries (the 8 largest), the active ones select and attend the
+    prefix (the prefix cache is updated in place, stable rows keep theirs), and every token
+    attends the block itself, merged with its prefix result.  A step is three launches
+    (the last one overlapped with PDL); R rotated input copies exceed 4x L2."""
+    import query_aware_block_b200 as lsa
+    import synth
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    base = synth.diffusion_losa_step(device=dev)
+    B, Hq, Tq, D = base.q.shape
+    Hkv = base.k.shape[1]
+    G = Hq // Hkv
+    T_cap = base.k.shape[2]
+    T = base.T_prefix
+    NBp = -(-T // 64)
+    n_top = int(base.active[0].sum())
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    ws = torch.empty(lsa.lsa_blockquery_workspace_size(B, Hkv, G, D, Tq), dtype=torch.uint8, device=dev)
+
+    def make(r):
+        c = base if r == 0 else synth.losa_case(seed=1006 + 101 * r, device=dev)
+        sl = torch.full((B,), T, dtype=torch.int32, device=dev)
+        summ = torch.zeros(B, Hkv, -(-T_cap // 64), D, device=dev)
+        lsa.lsa_build_summaries(c.k, sl, summ)
+        return dict(c=c, summ=summ, act=torch.empty(B, Tq, dtype=torch.uint8, device=dev),
+                    co=c.o_cache.clone(), cl=c.lse_cache.clone(), o=torch.empty_like(c.o_cache),
+                    lse=torch.empty_like(c.lse_cache),
+                    ui=torch.empty(B, Hkv, NBp, dtype=torch.int32, device=dev),
+                    uc=torch.empty(B, Hkv, dtype=torch.int32, device=dev))
+
+    def classify(x):
+        lsa.lsa_losa_classify(x["c"].q, x["c"].q_prev, x["act"], n_top=n_top)
+
+    def prefix(x):
+        c = x["c"]
+        lsa.lsa_sparse_attn_blockquery(c.q, c.k, c.v, x["summ"], T, c.topk, x["act"], x["co"], x["cl"],
+                                       x["co"], x["cl"], ws, union_idx=x["ui"], union_cnt=x["uc"])
+
+    def intra(x, flags=lsa.LSA_FLAG_PDL):
+        c = x["c"]
+        lsa.lsa_blockquery_intra_merge(c.q, c.k, c.v, T, x["co"], x["cl"], x["o"], x["lse"], flags=flags)
+
+    def one(x):
+        classify(x)
+        prefix(x)
+        intra(x)
+
+    copies = [make(0)]
+    one(copies[0])
+    torch.cuda.synchronize()
+    A = int(copies[0]["act"].sum())
+    U0 = int(copies[0]["uc"].sum())
+    blk_bytes = lambda U: (Hkv * NBp * D * 4 + U * 64 * D * 2 * 2 + 2 * A * G * Hkv * D * 2 + Hkv * NBp * 4)
+    other_bytes = (2 * Tq * Hq * D * 2 + Tq * B                      # classify: q, q_prev; mask
+                   + Hkv * Tq * D * 2 * 2 + Tq * Hq * D * 2          # intra: block K/V, q
+                   + 2 * Tq * Hq * D * 2 + 2 * Tq * Hq * 4 * 2)     # o_pre in, o out, lse in/out
+    R = 4 if args.profile_small else max(4, min(64, math.ceil(4 * l2 / (blk_bytes(U0) + other_bytes))))
+    while len(copies) < R:
+        copies.append(make(len(copies)))
+    for x in copies:
+        one(x)
+    torch.cuda.synchronize()
+    U_mean = sum(int(x["uc"].sum()) for x in copies) / len(copies)
+    step_bytes = blk_bytes(U_mean) + other_bytes
+
+    def graph_of(fn):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for x in copies:
+                fn(x)
+        return g
+
+    def time_graph(g, reps, clocks=None):
+        for _ in range(max(1, args.warmup // R)):
+            g.replay()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(reps):
+            g.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / (reps * R)
+
+    g_step = graph_of(one)
+    reps = max(1, args.steps // R)
+    with ClockSampler(0) as clocks:
+        ms = time_graph(g_step, reps)
+    # per-kernel breakdown (each alone, back to back)
+    parts = {}
+    for name, fn in (("classify", classify), ("blockquery", prefix), ("intra_merge", lambda x: intra(x, 0))):
+        parts[name] = round(time_graph(graph_of(fn), max(1, reps // 4)) * 1e3, 2)
+    # the dense first step of a block: every token, every prefix block
+    x0 = copies[0]
+    ones = torch.ones(B, Tq, dtype=torch.uint8, device=dev)
+    c0 = x0["c"]
+    dense = lambda: lsa.lsa_sparse_attn_blockquery(c0.q, c0.k, c0.v, x0["summ"], T, NBp, ones, x0["co"], x0["cl"],
+                                                   x0["o"], x0["lse"], ws, union_idx=x0["ui"], union_cnt=x0["uc"])
+    for _ in range(3):
+        dense()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(10):
+        dense()
+    e1.record()
+    torch.cuda.synchronize()
+    dense_ms = e0.elapsed_time(e1) / 10
+    dense_bytes = 2 * Hkv * T * D * 2 + Tq * Hq * D * 2 * 2
+    gbs = step_bytes / (ms * 1e-3) / 1e9
+    peak, kind = measured_peaks()
+    return {
+        "metric": "LoSA denoising step (classify + sparse prefix + intra-block merge): query tokens/s and "
+                  "effective GB/s (% of HBM roofline)",
+        "value": round(B * Tq / (ms * 1e-3), 1), "unit": "tokens/s", "n_gpus": 1, "steps": reps * R,
+        "warmup": args.warmup, "ms_per_step": round(ms, 6), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1), RoPE theta 1e4; "
+        "previous queries: +0.02 N(0,1) for stable tokens, fresh draws for the 8 changing ones)",
+        "config": {"workload": "losa_step", "batch": B, "kv_heads": Hkv, "q_heads_per_kv": G,
+                   "head_dim": D, "query_tokens": Tq, "active": A, "prefix": T, "topk_per_token": base.topk,
+                   "l2": f"rotating {R} input copies ({R * step_bytes / 1e6:.0f} MB per cycle)"},
+        "mean_union_blocks_per_kv_head": round(U_mean / (B * Hkv), 2),
+        "effective_gbs": round(gbs, 1), "bytes_per_step": int(step_bytes),
+        "kernel_us_alone": parts,
+        "dense_first_step": {"us": round(dense_ms * 1e3, 1),
+                             "effective_gbs": round(dense_bytes / (dense_ms * 1e-3) / 1e9, 1),
+                             "bytes": int(dense_bytes),
+                             "note": "every token over every prefix block (same K/V each call)"},
+        "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peak, "unit": "GB/s",
+                     "frac": round(gbs / peak, 4), "traffic": None, "kernel": "whole step (3 launches)",
+                     "peak_source": f"MEASURED_PEAKS.json hbm_gbs ({kind})"},
+        "gpu_launches": 3 * reps * R,
+        "clocks": clocks.summary(),
+    }
+
+
 def main():
     args = parse()
-    if args.workload in ("blockquery", "blasst_prefill_32k"):
+    if args.workload in ("blockquery", "blasst_prefill_32k", "losa_step"):
         if args.impl == "reference":
             print(json.dumps({"impl": "reference", "unavailable": "the oracle arm covers the decode workloads"}))
             return
-        res = run_blockquery(args) if args.workload == "blockquery" else run_prefill(args)
+        res = {"blockquery": run_blockquery, "blasst_prefill_32k": run_prefill,
+               "losa_step": run_losa_step}[args.workload](args)
         print(json.dumps(res), flush=True)
         return
     world = int(os.environ.get("WORLD_SIZE", "1"))

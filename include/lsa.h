@@ -7,6 +7,16 @@
  * the tokens' selections) -> online-softmax attention over only the selected KV blocks;
  * plus a causal prefill that skips whole KV tiles by a softmax threshold (BLASST).
  *
+ * One LoSA denoising step of a block of Tq query tokens is three calls on one stream:
+ *   lsa_losa_classify           (queries now vs the previous step -> active mask)
+ *   lsa_sparse_attn_blockquery  (prefix part: active tokens select and attend, stable
+ *                                tokens keep it; o_cache/lse_cache = o/lse = the prefix
+ *                                cache, updated in place)
+ *   lsa_blockquery_intra_merge  (the block's own tokens, merged with the prefix cache into
+ *                                the step's output)
+ * The first step of a block passes topk_per_query >= ceil(T_prefix / blk) and an all-ones
+ * mask (dense prefix attention, which fills the cache).
+ *
  * Conventions shared by every entry point
  * ---------------------------------------
  * Memory.   Every tensor argument is a raw DEVICE pointer to a contiguous row-major array
@@ -60,7 +70,7 @@ extern "C" {
 #define LSA_F32 0
 #define LSA_BF16 1
 
-/* lsa_sparse_attn_decode flags */
+/* lsa_sparse_attn_decode / lsa_blockquery_intra_merge flags */
 #define LSA_FLAG_PDL 1
 
 /* Human-readable name of a status code (static storage). */
@@ -189,8 +199,11 @@ LSA_API int lsa_sparse_attn_decode(const void* q, const void* k, const void* v, 
  * workspace: device scratch of at least lsa_blockquery_workspace_size(B, Hkv, G, D, Tq)
  *     bytes (16-byte aligned, contents need no initialisation), for the per-CTA partial
  *     results of the split over the union; calls that overlap on the GPU need their own.
- * Requires bf16, 1 <= Tq <= 64, 1 <= topk_per_query <= 16, n_sink + n_local <=
- * topk_per_query.
+ * Requires bf16, 1 <= Tq <= 64, n_sink + n_local <= topk_per_query, and either
+ * 1 <= topk_per_query <= 16 or topk_per_query >= NBp.  The latter selects every prefix
+ * block: with every token active this is the dense first denoising step of a block
+ * (LoSA, "2. 방법론": the first step attends densely to build the cache, later steps
+ * are sparse).
  */
 LSA_API size_t lsa_blockquery_workspace_size(int B, int Hkv, int G, int D, int Tq);
 
@@ -230,6 +243,65 @@ LSA_API int lsa_sparse_attn_blockquery_noalloc(const void* q, const void* k, con
                                                const float* lse_cache, void* o, float* lse,
                                                int32_t* union_idx, int32_t* union_cnt,
                                                cudaStream_t stream);
+
+/*
+ * lsa_losa_classify -- active and stable tokens of a query block between two denoising
+ * steps.
+ *
+ * Defined by: LoSA, "2. 방법론" (each denoising step measures how much every token's query
+ * vector changed, by its mean squared error, and calls the tokens that changed much
+ * active and the others stable).
+ *
+ *   mse[b, i] = (1 / (Hq * D)) * sum over query heads h and dims d of
+ *               (q[b, h, i, d] - q_prev[b, h, i, d])^2          (fp64)
+ *   n_top > 0:  active[b, i] = 1 for the n_top tokens of largest mse (equal mse: the
+ *               lower token index first), 0 for the others;
+ *   n_top == 0: active[b, i] = (mse[b, i] > tau).
+ * The sums and the comparison are carried out in double precision.
+ *
+ * q, q_prev [B, Hq, Tq, D] bf16 (the block's queries this step and the previous one);
+ * active [B, Tq] uint8 out (the mask lsa_sparse_attn_blockquery reads);
+ * mse [B, Tq] double out, or NULL (8-byte aligned).
+ * Requires bf16, D in {64, 128}, 1 <= Tq <= 64, n_top >= 0, B <= 65535, tau not NaN.
+ */
+LSA_API int lsa_losa_classify(const void* q, const void* q_prev, int dtype, int B, int Hq,
+                              int Tq, int D, double tau, int n_top, uint8_t* active,
+                              double* mse, cudaStream_t stream);
+
+/*
+ * lsa_blockquery_intra_merge -- attention of a query block over its own tokens, joined
+ * with the prefix result: the last step of a LoSA denoising step.
+ *
+ * Defined by: LoSA, "2. 방법론" (active tokens attend sparsely to the prefix, stable tokens
+ * reuse their prefix result -- output and statistics -- from the previous step; the block's
+ * own tokens change every step and are attended every step).
+ *
+ * For query row (b, h, i), KV group g = h / G: the block's tokens are rows
+ * T_prefix .. T_prefix + Tq - 1 of k[b, g] and v[b, g] (the caller writes this step's keys
+ * and values of the block there).  The row attends over all Tq of them, with no mask
+ * (attention inside the block is bidirectional):
+ *   (o_in, lse_in) = softmax attention with logits scale * q . k_t
+ * and the result is merged with the prefix part (o_pre, lse_pre) -- the softmax attention
+ * of the same row over its prefix tokens, as lsa_sparse_attn_blockquery returns it -- by
+ * log-sum-exp, i.e. the softmax over the union of both token sets:
+ *   lse = log(exp(lse_pre) + exp(lse_in))
+ *   o   = exp(lse_pre - lse) * o_pre + exp(lse_in - lse) * o_in
+ * lse_pre = -inf means an empty prefix part (o = o_in).
+ *
+ * q [B, Hq, Tq, D] bf16; k, v [B, Hkv, T_cap, D] bf16 with T_prefix + Tq <= T_cap;
+ * o_pre [B, Hq, Tq, D] bf16, lse_pre [B, Hq, Tq] float32; o, lse: same shapes, out.
+ * o may be o_pre and lse may be lse_pre (updated in place); other overlaps are rejected.
+ * flags: 0, or LSA_FLAG_PDL: launch with programmatic dependent launch; the kernel reads
+ *     q, k and v at once and o_pre, lse_pre only after the previous kernel of the stream
+ *     has completed, so the previous kernel may produce o_pre / lse_pre (the block-query
+ *     step) but must not write q, k or v.
+ * Requires bf16, D in {64, 128}, 1 <= Tq <= 64, G <= 16.
+ */
+LSA_API int lsa_blockquery_intra_merge(const void* q, const void* k, const void* v, int dtype,
+                                       int B, int Hkv, int G, int D, int Tq, int T_prefix,
+                                       int T_cap, float scale, const void* o_pre,
+                                       const float* lse_pre, void* o, float* lse, int flags,
+                                       cudaStream_t stream);
 
 /*
  * lsa_blasst_prefill -- causal softmax attention that skips whole KV tiles whose

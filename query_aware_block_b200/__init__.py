@@ -29,7 +29,8 @@ BLK = 64
 EXPORTED = ("lsa_status_string", "lsa_last_cuda_error", "lsa_version", "lsa_build_summaries",
             "lsa_select_blocks", "lsa_sparse_attn_decode", "lsa_blockquery_workspace_size",
             "lsa_sparse_attn_blockquery", "lsa_sparse_attn_blockquery_noalloc",
-            "lsa_blasst_prefill", "lsa_device_status")
+            "lsa_blasst_prefill", "lsa_device_status", "lsa_losa_classify",
+            "lsa_blockquery_intra_merge")
 
 _vp, _i, _f = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
 _lib.lsa_status_string.restype = ctypes.c_char_p
@@ -54,6 +55,10 @@ _lib.lsa_sparse_attn_blockquery_noalloc.argtypes = [_vp, _vp, _vp, _i, _i, _i, _
 _lib.lsa_blasst_prefill.argtypes = [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _f, _vp, _vp, _vp,
                                     _vp, _vp]
 _lib.lsa_device_status.argtypes = [_vp, _i]
+_lib.lsa_losa_classify.argtypes = [_vp, _vp, _i, _i, _i, _i, _i, ctypes.c_double, _i, _vp, _vp,
+                                   _vp]
+_lib.lsa_blockquery_intra_merge.argtypes = [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _f,
+                                            _vp, _vp, _vp, _vp, _i, _vp]
 for _n in EXPORTED[3:]:
     if _n != "lsa_blockquery_workspace_size":
         getattr(_lib, _n).restype = _i
@@ -171,6 +176,32 @@ def lsa_blasst_prefill(q, k, v, o, lam, lse=None, skip_bits=None, skipped_tiles=
                                    _ptr(skipped_tiles), _stream(stream)),
            "lsa_blasst_prefill")
     return o
+
+
+def lsa_losa_classify(q, q_prev, active, tau=0.0, n_top=0, mse=None, stream=None):
+    """Active mask [B,Tq] uint8 (in place) from the change of q [B,Hq,Tq,D] since q_prev:
+    the n_top largest mean squared changes, or (n_top == 0) those above tau.
+    mse: optional float64 [B,Tq] out."""
+    B, Hq, Tq, D = q.shape
+    _check(_lib.lsa_losa_classify(_ptr(q), _ptr(q_prev), _dtype(q), B, Hq, Tq, D, float(tau),
+                                  int(n_top), _ptr(active), _ptr(mse), _stream(stream)),
+           "lsa_losa_classify")
+    return active
+
+
+def lsa_blockquery_intra_merge(q, k, v, T_prefix, o_pre, lse_pre, o, lse, scale=0.0, flags=0,
+                               stream=None):
+    """Bidirectional attention of q [B,Hq,Tq,D] over the block's own keys (rows
+    T_prefix .. T_prefix+Tq-1 of k, v [B,Hkv,T_cap,D]), merged with the prefix result
+    (o_pre, lse_pre) by log-sum-exp into o, lse (in place; o may be o_pre)."""
+    B, Hq, Tq, D = q.shape
+    _, Hkv, T_cap, _ = k.shape
+    _check(_lib.lsa_blockquery_intra_merge(_ptr(q), _ptr(k), _ptr(v), _dtype(q), B, Hkv,
+                                           Hq // Hkv, D, Tq, T_prefix, T_cap, float(scale),
+                                           _ptr(o_pre), _ptr(lse_pre), _ptr(o), _ptr(lse),
+                                           int(flags), _stream(stream)),
+           "lsa_blockquery_intra_merge")
+    return o, lse
 
 
 def lsa_device_status(reset=False) -> int:

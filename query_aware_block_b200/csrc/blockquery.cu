@@ -95,11 +95,15 @@ struct BQLayout {
   size_t kv_tile;
 };
 
-__host__ __device__ inline BQLayout bq_layout(int D, int per_max, int NBp, int G) {
+// dense: every prefix block is selected (topk_per_query >= NBp), the selection buffers are
+// not used and the union holds all NBp blocks
+__host__ __device__ inline BQLayout bq_layout(int D, int per_max, int NBp, int G, bool dense) {
   BQLayout L;
   size_t off = 0;
-  const int ucap = NBp < kMaxUnion ? NBp : kMaxUnion;
-  const int stage_rows = per_max < kStageRows ? per_max : kStageRows;
+  const int ucap = (dense || NBp < kMaxUnion) ? NBp : kMaxUnion;
+  const int stage_rows = dense ? 0 : (per_max < kStageRows ? per_max : kStageRows);
+  const int per_sel = dense ? 0 : per_max;
+  const int tok_sel = dense ? 0 : kTokChunk;
   L.act = off;    off = al128(off + kMaxTq * 4);
   L.stab = off;   off = al128(off + kMaxTq * 4);
   L.ulist = off;  off = al128(off + (size_t)(ucap > 0 ? ucap : 1) * 4);
@@ -113,12 +117,12 @@ __host__ __device__ inline BQLayout bq_layout(int D, int per_max, int NBp, int G
   // the K/V ring starts at the first 1024-byte boundary of the region (TMA 128-byte swizzle)
   const size_t kv_bytes = kStages * 2 * L.kv_tile + 1024;
   size_t r = 0;
-  L.qsum = r; r = al128(r + (size_t)kTokChunk * kQStride * 4);
-  L.keys = r; r = al128(r + (size_t)kTokChunk * per_max * 8);
-  L.top = r;  r = al128(r + (size_t)kTokChunk * kLP * 8);
-  L.recv = r; r = al128(r + (size_t)2 * kMaxCluster * kTokChunk * kLP * 8);  // two buffers
+  L.qsum = r; r = al128(r + (size_t)tok_sel * kQStride * 4);
+  L.keys = r; r = al128(r + (size_t)tok_sel * per_sel * 8);
+  L.top = r;  r = al128(r + (size_t)tok_sel * kLP * 8);
+  L.recv = r; r = al128(r + (size_t)2 * kMaxCluster * tok_sel * kLP * 8);  // two buffers
   L.sumbuf = r; r = al128(r + (size_t)stage_rows * D * 4);
-  L.qrows = r; r = al128(r + (size_t)kTokChunk * G * D * 2);  // a token chunk's query rows
+  L.qrows = r; r = al128(r + (size_t)tok_sel * G * D * 2);  // a token chunk's query rows
   L.total = off + (r > kv_bytes ? r : kv_bytes);
   return L;
 }
@@ -133,7 +137,7 @@ __global__ void __launch_bounds__(kThreads, 2) blockquery_kernel(const __grid_co
   const size_t unit = (size_t)b * p.Hkv + g;
 
   extern __shared__ __align__(1024) unsigned char smem[];
-  const BQLayout Lo = bq_layout(D, p.per_max, p.NBp, p.G);
+  const BQLayout Lo = bq_layout(D, p.per_max, p.NBp, p.G, p.NBp <= p.topk);
   int* act = reinterpret_cast<int*>(smem + Lo.act);
   int* stab = reinterpret_cast<int*>(smem + Lo.stab);
   int* ulist = reinterpret_cast<int*>(smem + Lo.ulist);
@@ -699,7 +703,7 @@ cudaError_t launch_blockquery(const BlockQueryArgs& a, cudaStream_t stream) {
     p.per_max = (NBp + CL - 1) / CL;
     if (p.per_max < 1) p.per_max = 1;
     p.per_div = make_fastdiv((uint32_t)p.per_max);
-    const BQLayout Lo = bq_layout(a.D, p.per_max, NBp, a.G);
+    const BQLayout Lo = bq_layout(a.D, p.per_max, NBp, a.G, NBp <= a.topk);
     const int smem = (int)Lo.total;
     if (smem > 227 * 1024) return cudaErrorInvalidValue;
     cudaError_t err;

@@ -153,8 +153,10 @@ int lsa_sparse_attn_blockquery(const void* q, const void* k, const void* v, int 
   if (dtype != LSA_BF16) return LSA_ERR_UNSUPPORTED;
   if (Tq < 1 || Tq > 64 || T_prefix < 0 || T_cap < T_prefix) return LSA_ERR_INVALID_ARG;
   if (T_cap > kMaxTcap) return LSA_ERR_UNSUPPORTED;
-  if (topk_per_query < 1 || topk_per_query > 16 || n_sink < 0 || n_local < 0 ||
-      n_sink + n_local > topk_per_query)
+  // topk_per_query <= 16 selects; topk_per_query >= ceil(T_prefix / blk) takes every prefix
+  // block (the dense first step of a block)
+  if (topk_per_query < 1 || (topk_per_query > 16 && topk_per_query < ceil_div(T_prefix, blk)) ||
+      n_sink < 0 || n_local < 0 || n_sink + n_local > topk_per_query)
     return LSA_ERR_INVALID_ARG;
   if (B == 0 || Hkv == 0) return LSA_OK;
   if (!q || !k || !v || !summ || !active || !o_cache || !lse_cache || !o || !lse || !workspace)
@@ -191,6 +193,48 @@ int lsa_sparse_attn_blockquery_noalloc(const void* q, const void* k, const void*
                                     blk, topk_per_query, n_sink, n_local, scale, active,
                                     o_cache, lse_cache, o, lse, union_idx, union_cnt, ws,
                                     lsa::blockquery_static_workspace_bytes(), stream);
+}
+
+int lsa_losa_classify(const void* q, const void* q_prev, int dtype, int B, int Hq, int Tq, int D,
+                      double tau, int n_top, uint8_t* active, double* mse, cudaStream_t stream) {
+  if (B < 0 || Hq < 1 || Tq < 1 || n_top < 0) return LSA_ERR_INVALID_ARG;
+  if (dtype != LSA_BF16 || (D != 64 && D != 128)) return LSA_ERR_UNSUPPORTED;
+  if (Tq > 64 || B > 65535 || !(tau == tau)) return Tq > 64 || B > 65535 ? LSA_ERR_UNSUPPORTED
+                                                                         : LSA_ERR_INVALID_ARG;
+  if (B == 0) return LSA_OK;
+  if (!q || !q_prev || !active) return LSA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(q_prev) || (mse && ((uintptr_t)mse & 7u) != 0))
+    return LSA_ERR_INVALID_ARG;
+  return cuda_status(lsa::launch_losa_classify(q, q_prev, B, Hq, Tq, D, tau, n_top, active, mse,
+                                               stream));
+}
+
+int lsa_blockquery_intra_merge(const void* q, const void* k, const void* v, int dtype, int B,
+                               int Hkv, int G, int D, int Tq, int T_prefix, int T_cap,
+                               float scale, const void* o_pre, const float* lse_pre, void* o,
+                               float* lse, int flags, cudaStream_t stream) {
+  int st = check_common(dtype, B, Hkv, G, D, 64);
+  if (st != LSA_OK) return st;
+  if (dtype != LSA_BF16) return LSA_ERR_UNSUPPORTED;
+  if (Tq < 1 || Tq > 64 || T_prefix < 0 || T_cap < T_prefix + Tq) return LSA_ERR_INVALID_ARG;
+  if (T_cap > kMaxTcap || B > 65535 || (long long)Hkv * G > 65535) return LSA_ERR_UNSUPPORTED;
+  if ((flags & ~LSA_FLAG_PDL) != 0) return LSA_ERR_INVALID_ARG;
+  if (B == 0 || Hkv == 0) return LSA_OK;
+  if (!q || !k || !v || !o_pre || !lse_pre || !o || !lse) return LSA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o_pre) || !aligned16(o))
+    return LSA_ERR_INVALID_ARG;
+  // o may be o_pre and lse may be lse_pre; a partial overlap is rejected
+  const size_t obytes = (size_t)B * Hkv * G * Tq * D * 2, lbytes = (size_t)B * Hkv * G * Tq * 4;
+  const uintptr_t o0 = (uintptr_t)o, p0 = (uintptr_t)o_pre, l0 = (uintptr_t)lse, lp0 = (uintptr_t)lse_pre;
+  if (o0 != p0 && o0 < p0 + obytes && p0 < o0 + obytes) return LSA_ERR_INVALID_ARG;
+  if (l0 != lp0 && l0 < lp0 + lbytes && lp0 < l0 + lbytes) return LSA_ERR_INVALID_ARG;
+  lsa::IntraMergeArgs a = {};
+  a.q = q; a.k = k; a.v = v;
+  a.B = B; a.Hkv = Hkv; a.G = G; a.D = D; a.Tq = Tq; a.T_prefix = T_prefix; a.T_cap = T_cap;
+  a.scale = resolve_scale(scale, D);
+  a.o_pre = o_pre; a.lse_pre = lse_pre; a.o = o; a.lse = lse;
+  a.pdl = (flags & LSA_FLAG_PDL) != 0;
+  return cuda_status(lsa::launch_intra_merge(a, stream));
 }
 
 int lsa_blasst_prefill(const void* q, const void* k, const void* v, int dtype, int B, int Hq,

@@ -63,6 +63,24 @@ struct BlockQueryArgs {
 size_t blockquery_workspace_bytes(int B, int Hkv, int G, int D, int Tq);
 cudaError_t launch_blockquery(const BlockQueryArgs& a, cudaStream_t stream);
 
+// LoSA: token activity and the attention inside the query block merged with the prefix.
+cudaError_t launch_losa_classify(const void* q, const void* q_prev, int B, int Hq, int Tq, int D,
+                                 double tau, int n_top, uint8_t* active, double* mse,
+                                 cudaStream_t stream);
+struct IntraMergeArgs {
+  const void* q;
+  const void* k;
+  const void* v;
+  int B, Hkv, G, D, Tq, T_prefix, T_cap;
+  float scale;
+  const void* o_pre;
+  const float* lse_pre;
+  void* o;
+  float* lse;
+  int pdl;
+};
+cudaError_t launch_intra_merge(const IntraMergeArgs& a, cudaStream_t stream);
+
 // BLASST causal prefill on tcgen05.
 struct PrefillArgs {
   const void* q;

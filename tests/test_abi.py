@@ -86,6 +86,36 @@ def test_select_and_decode_validation():
     assert dec(g, g, g, 1, 1, 8, 8, 128, 65536, g, 64, NULL, NULL, 16, 0.0, g, 1, 2, 0, NULL, g, NULL, 2, NULL) == lsa.LSA_ERR_INVALID_ARG
 
 
+def test_losa_entry_points_validation():
+    import query_aware_block_b200 as lsa
+    lib = lsa.library()
+    g = ctypes.c_void_p(4096)
+    cls = lib.lsa_losa_classify
+    assert cls(g, g, 0, 1, 32, 32, 128, 0.1, 0, g, NULL, NULL) == lsa.LSA_ERR_UNSUPPORTED  # fp32
+    assert cls(g, g, 1, 1, 32, 65, 128, 0.1, 0, g, NULL, NULL) == lsa.LSA_ERR_UNSUPPORTED  # Tq > 64
+    assert cls(g, g, 1, 1, 32, 32, 96, 0.1, 0, g, NULL, NULL) == lsa.LSA_ERR_UNSUPPORTED   # D
+    assert cls(g, g, 1, 1, 32, 32, 128, 0.1, -1, g, NULL, NULL) == lsa.LSA_ERR_INVALID_ARG  # n_top
+    assert cls(g, g, 1, 1, 32, 32, 128, float("nan"), 0, g, NULL, NULL) == lsa.LSA_ERR_INVALID_ARG
+    assert cls(g, NULL, 1, 1, 32, 32, 128, 0.1, 0, g, NULL, NULL) == lsa.LSA_ERR_INVALID_ARG
+    assert cls(g, g, 1, 1, 32, 32, 128, 0.1, 0, g, ctypes.c_void_p(4100), NULL) == lsa.LSA_ERR_INVALID_ARG
+    assert cls(NULL, NULL, 1, 0, 32, 32, 128, 0.1, 0, NULL, NULL, NULL) == lsa.LSA_OK  # empty batch
+    im = lib.lsa_blockquery_intra_merge
+    big = 1 << 30
+    # the block must fit behind the prefix: T_prefix + Tq <= T_cap
+    assert im(g, g, g, 1, 1, 8, 4, 128, 32, 100, 131, 0.0, g, g, ctypes.c_void_p(big), g, 0, NULL) == lsa.LSA_ERR_INVALID_ARG
+    assert im(g, g, g, 1, 1, 8, 4, 128, 65, 100, 1000, 0.0, g, g, ctypes.c_void_p(big), g, 0, NULL) == lsa.LSA_ERR_INVALID_ARG
+    assert im(g, g, g, 0, 1, 8, 4, 128, 32, 100, 1000, 0.0, g, g, ctypes.c_void_p(big), g, 0, NULL) == lsa.LSA_ERR_UNSUPPORTED
+    assert im(g, g, g, 1, 1, 8, 4, 128, 32, 100, 1000, 0.0, g, g, ctypes.c_void_p(big), g, 2, NULL) == lsa.LSA_ERR_INVALID_ARG
+    # o overlapping o_pre without being it
+    assert im(g, g, g, 1, 1, 8, 4, 128, 32, 100, 1000, 0.0, g, g, ctypes.c_void_p(4096 + 256), g, 0, NULL) == lsa.LSA_ERR_INVALID_ARG
+    assert im(g, g, g, 1, 0, 8, 4, 128, 32, 100, 1000, 0.0, NULL, NULL, NULL, NULL, 0, NULL) == lsa.LSA_OK
+    bq = lib.lsa_sparse_attn_blockquery
+    # topk_per_query in (16, NBp) is rejected (>= NBp, every prefix block, is the dense step)
+    args = lambda topk, T: (g, g, g, 1, 1, 8, 4, 128, 32, T, T + 32, g, 64, topk, 0, 0, 0.0, g, g, g, g, g, NULL, NULL, g, 0, NULL)
+    assert bq(*args(17, 64 * 100)) == lsa.LSA_ERR_INVALID_ARG
+    assert bq(*args(0, 64 * 100)) == lsa.LSA_ERR_INVALID_ARG
+
+
 def test_binding_raises_lsa_error_on_bad_arguments():
     import torch
     import query_aware_block_b200 as lsa

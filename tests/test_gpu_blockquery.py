@@ -52,12 +52,13 @@ def _run_gpu(lsa, case, alias=False):
     return o.cpu(), lse.cpu(), ui[..., :NBp].cpu(), uc.cpu()
 
 
-def _check_union(case, ui, uc, where):
-    """The GPU union against the per-token oracle selections under the gap rule."""
+def _check_union(case, ui, uc, where, summ_len=None):
+    """The GPU union against the per-token oracle selections under the gap rule
+    (summaries over the first summ_len cache rows, by default all of them)."""
     B, Hq, Tq, D = case.q.shape
     Hkv = case.k.shape[1]
     NBp = -(-case.T_prefix // 64)
-    sl = torch.full((B,), case.k.shape[2], dtype=torch.int32)
+    sl = torch.full((B,), summ_len or case.k.shape[2], dtype=torch.int32)
     summ = oracle.summaries(case.k, sl)
     k = case.topk
     for b in range(B):
