@@ -199,6 +199,12 @@ LSA_API int lsa_sparse_attn_decode(const void* q, const void* k, const void* v, 
  * workspace: device scratch of at least lsa_blockquery_workspace_size(B, Hkv, G, D, Tq)
  *     bytes (16-byte aligned, contents need no initialisation), for the per-CTA partial
  *     results of the split over the union; calls that overlap on the GPU need their own.
+ * Launch: programmatic dependent launch.  The kernel may start while the previous kernel
+ * of the stream still runs, but reads no input before that kernel has completed (so any
+ * previous kernel may produce any input), and it lets the next kernel of the stream start
+ * early; a next kernel launched with programmatic dependent launch must wait for this
+ * one's completion before reading its outputs (lsa_blockquery_intra_merge with
+ * LSA_FLAG_PDL does).
  * Requires bf16, 1 <= Tq <= 64, n_sink + n_local <= topk_per_query, and either
  * 1 <= topk_per_query <= 16 or topk_per_query >= NBp.  The latter selects every prefix
  * block: with every token active this is the dense first denoising step of a block
@@ -257,7 +263,9 @@ LSA_API int lsa_sparse_attn_blockquery_noalloc(const void* q, const void* k, con
  *   n_top > 0:  active[b, i] = 1 for the n_top tokens of largest mse (equal mse: the
  *               lower token index first), 0 for the others;
  *   n_top == 0: active[b, i] = (mse[b, i] > tau).
- * The sums and the comparison are carried out in double precision.
+ * The sums and the comparison are carried out in double precision.  The kernel lets the
+ * next kernel of the stream start early (the block-query step, which waits for it before
+ * reading the mask).
  *
  * q, q_prev [B, Hq, Tq, D] bf16 (the block's queries this step and the previous one);
  * active [B, Tq] uint8 out (the mask lsa_sparse_attn_blockquery reads);

@@ -174,12 +174,18 @@ __global__ void __launch_bounds__(kThreads, 2) blockquery_kernel(const __grid_co
     tc::fence_mbar_init();
     tc::prefetch_tmap(&p.tmk);
     tc::prefetch_tmap(&p.tmv);
-    if (staged_rows > 0) {  // the slice's first summary rows, one bulk copy
-      const uint32_t bytes = (uint32_t)(staged_rows * D * 4);
-      tc::mbar_arrive_expect_tx(&xbar[2], bytes);
-      tc::bulk_load(sumbuf, p.summ + (unit * (size_t)p.NB_cap + j0) * D, bytes, &xbar[2]);
-    }
   }
+  // The launch is a programmatic dependent one: nothing above reads an input, and every
+  // input may come from the previous kernel of the stream, which is complete (and its
+  // memory visible) once this wait returns.  The trigger then lets the next kernel start
+  // its own prologue; one that reads this grid's outputs waits for its completion first.
+  pdl_wait();
+  if (tid == 0 && staged_rows > 0) {  // the slice's first summary rows, one bulk copy
+    const uint32_t bytes = (uint32_t)(staged_rows * D * 4);
+    tc::mbar_arrive_expect_tx(&xbar[2], bytes);
+    tc::bulk_load(sumbuf, p.summ + (unit * (size_t)p.NB_cap + j0) * D, bytes, &xbar[2]);
+  }
+  pdl_trigger();
   cluster_arrive_relaxed();  // DSMEM is written only after every CTA has started
   bool started = false;
 
@@ -719,11 +725,13 @@ cudaError_t launch_blockquery(const BlockQueryArgs& a, cudaStream_t stream) {
     cfg.blockDim = dim3(kThreads, 1, 1);
     cfg.dynamicSmemBytes = (size_t)smem;
     cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = CL;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     int nclusters = 0;
@@ -736,6 +744,7 @@ cudaError_t launch_blockquery(const BlockQueryArgs& a, cudaStream_t stream) {
       }
       return err != cudaSuccess ? err : cudaErrorInvalidConfiguration;
     }
+    cfg.numAttrs = 2;  // launched as a programmatic dependent of the previous kernel
     return cudaLaunchKernelEx(&cfg, kernel, p);
   }
 }

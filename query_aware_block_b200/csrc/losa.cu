@@ -69,6 +69,7 @@ __global__ void __cluster_dims__(kClsCluster, 1, 1) __launch_bounds__(kClsThread
   constexpr int kWarps = kClsThreads / 32;
   __shared__ double all_mse[kMaxTq];  // rank 0: the change of every token of the block
   __shared__ double red[kWarps][kClsTok];
+  pdl_trigger();  // the next kernel (the block-query step) may start its prologue now
   cluster_arrive_relaxed();  // rank 0's shared memory is written only after all have started
 
   const int per = (Tq + kClsCluster - 1) / kClsCluster;
