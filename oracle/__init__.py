@@ -8,7 +8,8 @@ the CUDA library in ``query_aware_block_b200``.
 
 Parity status of each function (what pins it is in tests/test_oracle_pins.py):
   summaries, block_scores, select, decode_attn, blockquery_select, blockquery_attn,
-  blasst_prefill, losa_classify, blockquery_intra_merge (and the losa_step composition)
+  blasst_prefill, decode_blasst, losa_classify, blockquery_intra_merge (and the losa_step
+  composition)
   -- all pinned (textbook special cases, brute force, library routines, closed forms and
   invariants).
 """
@@ -282,3 +283,34 @@ def losa_step(q, q_prev, k, v, summ, T_prefix, o_cache, lse_cache, topk, tau=0.0
     o, lse = blockquery_intra_merge(q, k, v, T_prefix, o_p, lse_p, scale)
     return dict(mse=mse, active=active, union_idx=uidx, union_cnt=ucnt, o_prefix=o_p,
                 lse_prefix=lse_p, o=o, lse=lse)
+
+
+def decode_blasst(q, k, v, seqlens, idx, nsel, lam, blk=64, scale=None, forced_bits=None):
+    """Sparse decode attention over the listed blocks (visited in ascending order) with
+    BLASST's skip test over the group's heads.
+
+    Returns dict(o fp64 [B,Hq,D], lse fp64 [B,Hq], bits [B,Hkv] (int64, bit r = slot r
+    skipped), gap fp64 [B,Hkv,topk]); forced_bits [B,Hkv] replaces the decisions."""
+    q, k, v = q.contiguous(), k.contiguous(), v.contiguous()
+    assert q.dtype == k.dtype == v.dtype
+    B, Hq, D = q.shape
+    _, Hkv, T_cap, _ = k.shape
+    G = Hq // Hkv
+    idx = _i32(idx)
+    nsel = _i32(nsel)
+    topk = idx.shape[-1]
+    assert topk <= 32
+    o = torch.empty(B, Hq, D, dtype=torch.float64)
+    lse = torch.empty(B, Hq, dtype=torch.float64)
+    bits = torch.empty(B, Hkv, dtype=torch.int32)
+    gap = torch.empty(B, Hkv, topk, dtype=torch.float64)
+    fb = None
+    if forced_bits is not None:
+        fb = np.asarray(torch.as_tensor(forced_bits).to(torch.int64).reshape(B, Hkv))
+        fb = torch.from_numpy((fb & 0xFFFFFFFF).astype(np.uint32).view(np.int32).copy())
+    sl = _i32(seqlens)
+    _load().oracle_decode_blasst(_p(q), _p(k), _p(v), _dt(q), B, Hkv, G, D, T_cap, _p(sl), blk,
+                                 _p(idx), _p(nsel), topk, ctypes.c_double(_scale(scale, D)),
+                                 ctypes.c_double(float(lam)), _p(fb), _p(o), _p(lse), _p(bits),
+                                 _p(gap))
+    return dict(o=o, lse=lse, bits=bits.to(torch.int64) & 0xFFFFFFFF, gap=gap)

@@ -31,6 +31,11 @@
  *                            order, skipping a tile whose row maxima all trail the running
  *                            maxima by more than ln(lambda)
  *                            [BLASST, "2. 방법론", "핵심 아이디어" and "알고리즘 및 커널 설계"]
+ *   oracle_decode_blasst     sparse decode attention whose selected blocks are visited in
+ *                            ascending order with BLASST's skip test (a block every head of
+ *                            the group finds negligible is not read: no V load)
+ *                            [BLASST, "2. 방법론", "알고리즘 및 커널 설계": the decode kernel
+ *                             saves the V-block loads]
  *   oracle_losa_classify     active / stable tokens by the mean squared change of their
  *                            queries between denoising steps [LoSA, "2. 방법론": the query
  *                            change (MSE) of every step sorts tokens into active and stable]
@@ -47,6 +52,8 @@
  *   - the forced blocks are counted inside the n selected blocks;
  *   - the BLASST test quantifies over rows: skip iff every row's
  *     (tile row max - running row max) < ln(lambda); strict '<' as printed.
+ *   - in decode the rows of BLASST's tile are the query heads of a GQA group (they share
+ *     the block's V): skip iff every head's (block max - running max) < ln(lambda);
  *   - LoSA's query change is the mean over all query heads and dims of the squared
  *     difference; active iff it exceeds tau (or: the n_top largest, ties to the lower
  *     index);
@@ -609,6 +616,124 @@ void oracle_blockquery_intra_merge(const void* q, const void* k, const void* v, 
       free(o_in);
       free(logits);
       free(toks);
+    }
+  }
+}
+
+/* ------------------------------------------------------------------------------------
+ * Sparse decode attention with BLASST's skip test over the selected blocks.
+ * Group (b, g): the selected blocks idx[b,g,:nsel] (ascending, -1 = unused slot) are
+ * visited in order, as the KV blocks of a blockwise online softmax.  For each visited block:
+ *   S_ht = scale * q_h . k_t for every query head h of the group, t in the block, t < T_b;
+ *   r_h  = max_t S_ht (the block's max for head h); m_h = head h's running max (-inf
+ *          before the first block);
+ *   gap  = max over the group's heads of (r_h - m_h)          (m_h = -inf gives +inf)
+ *   skip iff the block is not the first visited and gap < ln(lambda)  (lambda = 0: never)
+ * The group's heads are the rows of the tile: the block's V is shared by them, so it is
+ * skipped (not read, no exponentials, no P.V) only when every head finds it negligible;
+ * otherwise every head takes the usual online-softmax update.
+ * o = acc / l and lse = m + ln l per head.
+ * forced_bits (optional, [B,Hkv]): bit r decides slot r instead of the test (the gap is
+ * still reported), so the output can be evaluated on another implementation's decisions.
+ * skip_bits [B,Hkv] out: bit r set iff slot r was skipped; gap [B,Hkv,topk] out (NaN for
+ * unused slots).  q [B,Hq,D]; k, v [B,Hkv,T_cap,D]; o [B,Hq,D]; lse [B,Hq].
+ * ---------------------------------------------------------------------------------- */
+void oracle_decode_blasst(const void* q, const void* k, const void* v, int dtype, int B, int Hkv,
+                          int G, int D, int T_cap, const int32_t* seqlens, int blk,
+                          const int32_t* idx, const int32_t* nsel, int topk, double scale,
+                          double lambda, const uint32_t* forced_bits, double* o, double* lse,
+                          uint32_t* skip_bits, double* gap_out) {
+  const int Hq = Hkv * G;
+  const double ln_lambda = (lambda > 0.0) ? log(lambda) : -INFINITY;
+#pragma omp parallel for collapse(2) schedule(dynamic)
+  for (int b = 0; b < B; ++b) {
+    for (int g = 0; g < Hkv; ++g) {
+      const size_t u = (size_t)b * Hkv + g;
+      const int T = seqlens[b];
+      const size_t kvbase = u * (size_t)T_cap * D;
+      double* m = (double*)malloc(sizeof(double) * (size_t)G);
+      double* l = (double*)malloc(sizeof(double) * (size_t)G);
+      double* r = (double*)malloc(sizeof(double) * (size_t)G);
+      double* S = (double*)malloc(sizeof(double) * (size_t)G * blk);
+      for (int hh = 0; hh < G; ++hh) {
+        m[hh] = -INFINITY;
+        l[hh] = 0.0;
+        double* acc = o + ((size_t)b * Hq + g * G + hh) * D;
+        for (int d = 0; d < D; ++d) acc[d] = 0.0;
+      }
+      skip_bits[u] = 0u;
+      for (int s = 0; s < topk; ++s) gap_out[u * topk + s] = NAN;
+      int visited = 0;
+      for (int s = 0; s < nsel[u] && s < topk; ++s) {
+        const int j = idx[u * topk + s];
+        if (j < 0) continue;
+        const int t0 = j * blk;
+        /* logits and block maxima of every head of the group */
+        for (int hh = 0; hh < G; ++hh) {
+          const size_t qrow = ((size_t)b * Hq + g * G + hh) * D;
+          r[hh] = -INFINITY;
+          for (int tt = 0; tt < blk; ++tt) {
+            const int t = t0 + tt;
+            double sv = -INFINITY;
+            if (t < T) {
+              double dot = 0.0;
+              for (int d = 0; d < D; ++d)
+                dot += elem(q, dtype, qrow + d) * elem(k, dtype, kvbase + (size_t)t * D + d);
+              sv = scale * dot;
+            }
+            S[(size_t)hh * blk + tt] = sv;
+            if (sv > r[hh]) r[hh] = sv;
+          }
+        }
+        double gap = -INFINITY;
+        for (int hh = 0; hh < G; ++hh) {
+          double gi;
+          if (r[hh] == -INFINITY) gi = -INFINITY;
+          else if (m[hh] == -INFINITY) gi = INFINITY;
+          else gi = r[hh] - m[hh];
+          if (gi > gap) gap = gi;
+        }
+        gap_out[u * topk + s] = gap;
+        int skip;
+        if (forced_bits) skip = (int)((forced_bits[u] >> s) & 1u);
+        else skip = visited > 0 && gap < ln_lambda;
+        ++visited;
+        if (skip) {
+          skip_bits[u] |= 1u << s;
+          continue;
+        }
+        for (int hh = 0; hh < G; ++hh) {
+          const double mn = (r[hh] > m[hh]) ? r[hh] : m[hh];
+          if (mn == -INFINITY) continue;
+          const double alpha = (m[hh] == -INFINITY) ? 0.0 : exp(m[hh] - mn);
+          double* acc = o + ((size_t)b * Hq + g * G + hh) * D;
+          l[hh] *= alpha;
+          for (int d = 0; d < D; ++d) acc[d] *= alpha;
+          for (int tt = 0; tt < blk; ++tt) {
+            const double sv = S[(size_t)hh * blk + tt];
+            if (sv == -INFINITY) continue;
+            const double p = exp(sv - mn);
+            l[hh] += p;
+            const size_t vrow = kvbase + (size_t)(t0 + tt) * D;
+            for (int d = 0; d < D; ++d) acc[d] += p * elem(v, dtype, vrow + d);
+          }
+          m[hh] = mn;
+        }
+      }
+      for (int hh = 0; hh < G; ++hh) {
+        const size_t row = (size_t)b * Hq + g * G + hh;
+        double* acc = o + row * D;
+        if (l[hh] > 0.0) {
+          for (int d = 0; d < D; ++d) acc[d] /= l[hh];
+          lse[row] = m[hh] + log(l[hh]);
+        } else {
+          lse[row] = -INFINITY;
+        }
+      }
+      free(S);
+      free(r);
+      free(l);
+      free(m);
     }
   }
 }

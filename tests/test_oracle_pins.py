@@ -611,3 +611,116 @@ def test_losa_step_stable_rows_with_exact_cache_match_recomputation():
                                      case.v[0, h // 2, :T + Tq], sc)
         assert torch.allclose(r["o"][0, h], o_ref, rtol=0, atol=1e-6)
         assert torch.allclose(r["lse"][0, h], lse_ref, rtol=0, atol=1e-5)
+
+
+# ------------------------------------------------------ BLASST inside sparse decode ----
+
+def _masked_rows(q, k, v, T, blocks, scale):
+    """Library routines: fp64 SDPA of the query rows over the tokens of `blocks` (t < T),
+    and the log-sum-exp of those logits."""
+    mask = torch.zeros(T, dtype=torch.bool)
+    for j in blocks:
+        mask[j * 64:min(j * 64 + 64, T)] = True
+    kk, vv = k[:T][mask].double(), v[:T][mask].double()
+    o = F.scaled_dot_product_attention(q.double()[None], kk[None], vv[None], scale=scale)[0]
+    lse = torch.logsumexp(scale * q.double() @ kk.T, dim=-1)
+    return o, lse
+
+
+def _decode_sel(case, topk, n_sink=1, n_local=2):
+    r = oracle.decode(case.q, case.k, case.v, case.seqlens, topk, n_sink, n_local)
+    return r["idx"], r["nsel"]
+
+
+def test_decode_blasst_lambda_zero_is_masked_dense():
+    B, Hkv, G, D, T = 2, 2, 3, 32, 1000
+    case = synth.decode_case(B, Hkv, G, D, T_cap=1024, seqlens=[T, 700], dtype=torch.float32,
+                             topk=6, n_sink=1, n_local=2, seed=81)
+    idx, nsel = _decode_sel(case, 6)
+    r = oracle.decode_blasst(case.q, case.k, case.v, case.seqlens, idx, nsel, 0.0)
+    assert int(r["bits"].sum()) == 0
+    for b in range(B):
+        Tb = int(case.seqlens[b])
+        for g in range(Hkv):
+            blocks = [int(j) for j in idx[b, g] if j >= 0]
+            qh = case.q[b, g * G:(g + 1) * G]
+            o_ref, lse_ref = _masked_rows(qh, case.k[b, g], case.v[b, g], Tb, blocks, 1 / math.sqrt(D))
+            assert torch.allclose(r["o"][b, g * G:(g + 1) * G], o_ref, rtol=0, atol=1e-12)
+            assert torch.allclose(r["lse"][b, g * G:(g + 1) * G], lse_ref, rtol=0, atol=1e-12)
+
+
+def _planted_case(seed):
+    """G = 2 heads with opposite queries; block 1 is negligible for both heads (keys
+    orthogonal-ish and far below), block 2 is negligible for head 0 only, block 3 for
+    neither; block 0 holds a key every head scores highly (it sets the running maxima)."""
+    D, G, T = 32, 2, 64 * 5
+    g = torch.Generator().manual_seed(seed)
+    u = torch.randn(D, generator=g, dtype=torch.float64)
+    u = u / u.norm()
+    w = torch.randn(D, generator=g, dtype=torch.float64)
+    w = w - (w @ u) * u
+    w = w / w.norm()
+    q = torch.stack([8 * u + 8 * w, -8 * u + 8 * w])[None].float()          # [1, 2, D]
+    k = 0.05 * torch.randn(1, 1, T, D, generator=g, dtype=torch.float64)
+    k[0, 0, 0:64] += 4 * w                  # block 0: logit ~ 8*4/sqrt(32) = 5.7 for both heads
+    k[0, 0, 64:128] -= 4 * w                # block 1: ~ -5.7 for both: gap ~ -11.3
+    k[0, 0, 128:192] += -4 * u - 4 * w      # block 2: head 0 ~ -11.3, head 1 ~ 0: gap ~ -5.7
+    k[0, 0, 192:256] += 0.0                 # block 3: ~ 0 for both: gap ~ -5.7
+    v = torch.randn(1, 1, T, D, generator=g)
+    return q, k.float(), v, T
+
+
+def test_decode_blasst_skips_only_blocks_every_head_finds_negligible():
+    q, k, v, T = _planted_case(82)
+    sl = torch.tensor([T], dtype=torch.int32)
+    idx = torch.tensor([[[0, 1, 2, 3, -1]]], dtype=torch.int32)
+    nsel = torch.tensor([[4]], dtype=torch.int32)
+    # ln(1e-4) = -9.2: block 1 (gap -11.3) is skipped; blocks 2 and 3 (gap -5.7) are kept
+    r = oracle.decode_blasst(q, k, v, sl, idx, nsel, 1e-4)
+    assert int(r["bits"][0, 0]) == 0b0010
+    gap = r["gap"][0, 0]
+    assert math.isinf(float(gap[0])) and float(gap[1]) < math.log(1e-4) < float(gap[2])
+    assert math.isnan(float(gap[4]))
+    o_ref, lse_ref = _masked_rows(q[0], k[0, 0], v[0, 0], T, [0, 2, 3], 1 / math.sqrt(32))
+    assert torch.allclose(r["o"][0], o_ref, rtol=0, atol=1e-12)
+    assert torch.allclose(r["lse"][0], lse_ref, rtol=0, atol=1e-12)
+    # ln(0.01) = -4.6: now blocks 2 and 3 are negligible for every head too
+    r = oracle.decode_blasst(q, k, v, sl, idx, nsel, 1e-2)
+    assert int(r["bits"][0, 0]) == 0b1110
+    # the first visited block is never skipped, however small: with block 1 first, its gap
+    # is +inf and block 0 (gap +11.3) is kept as well
+    idx2 = torch.tensor([[[1, 0, 2, 3, -1]]], dtype=torch.int32)
+    r = oracle.decode_blasst(q, k, v, sl, idx2, nsel, 1e-2)
+    assert int(r["bits"][0, 0]) & 0b0011 == 0
+
+
+def test_decode_blasst_output_is_dense_over_kept_blocks_within_the_error_bound():
+    # a sharpened query (x3) makes some selected blocks negligible at lambda = 1e-3
+    B, Hkv, G, D, T = 1, 2, 2, 64, 64 * 24
+    case = synth.decode_case(B, Hkv, G, D, T_cap=T, seqlens=T, dtype=torch.float32, topk=12,
+                             n_sink=1, n_local=2, n_needles=3, seed=83)
+    q = (case.q * 3).contiguous()
+    idx, nsel = _decode_sel(case, 12)
+    lam = 1e-3
+    r = oracle.decode_blasst(q, case.k, case.v, case.seqlens, idx, nsel, lam)
+    full = oracle.decode_blasst(q, case.k, case.v, case.seqlens, idx, nsel, 0.0)
+    assert int(r["bits"].sum()) > 0, "the case should skip something"
+    sc = 1 / math.sqrt(D)
+    for g in range(Hkv):
+        kept = [int(idx[0, g, s]) for s in range(12) if not (int(r["bits"][0, g]) >> s) & 1]
+        dropped = 64 * (12 - len(kept))
+        qh = q[0, g * G:(g + 1) * G]
+        o_ref, lse_ref = _masked_rows(qh, case.k[0, g], case.v[0, g], T, kept, sc)
+        assert torch.allclose(r["o"][0, g * G:(g + 1) * G], o_ref, rtol=0, atol=1e-12)
+        assert torch.allclose(r["lse"][0, g * G:(g + 1) * G], lse_ref, rtol=0, atol=1e-12)
+        # each dropped weight is < lambda relative to the final max, whose weight is 1
+        vmax = float(case.v[0, g].abs().max())
+        err = float((r["o"][0, g * G:(g + 1) * G] - full["o"][0, g * G:(g + 1) * G]).abs().max())
+        assert err <= 2 * vmax * dropped * lam
+        # forcing the same decisions reproduces the output; forcing none gives lambda = 0
+    forced = oracle.decode_blasst(q, case.k, case.v, case.seqlens, idx, nsel, 0.5,
+                                  forced_bits=r["bits"])
+    assert torch.equal(forced["o"], r["o"]) and torch.equal(forced["bits"], r["bits"])
+    none = oracle.decode_blasst(q, case.k, case.v, case.seqlens, idx, nsel, 0.5,
+                                forced_bits=torch.zeros(1, Hkv, dtype=torch.int64))
+    assert torch.equal(none["o"], full["o"])
