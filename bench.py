@@ -3,7 +3,7 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--workload gqa_decode_64k|batched_decode|tiny_decode|blockquery|
-                                losa_step|blasst_prefill_32k]
+                                losa_step|decode_blasst|blasst_prefill_32k]
 
 Default workload: 64K-context GQA decode, bf16 (1 sequence, 8 KV heads x 8 query heads,
 head dim 128, 65,536 cached tokens = 1,024 blocks of 64, top-16 blocks per KV head with
@@ -66,12 +66,16 @@ def parse():
                     help="timed steps (default: 200000 decode steps; 20 prefills; 20000 block-query steps)")
     ap.add_argument("--warmup", type=int, default=None)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=sorted(WORKLOADS) + ["blockquery", "blasst_prefill_32k", "losa_step"],
+    ap.add_argument("--workload", choices=sorted(WORKLOADS) + ["blockquery", "blasst_prefill_32k", "losa_step",
+                                                          "decode_blasst"],
                     default="gqa_decode_64k")
     ap.add_argument("--prefill-sink", type=float, default=0.0,
                     help="blasst_prefill_32k: plant an attention sink of this logit height")
     ap.add_argument("--prefill-qscale", type=float, default=1.0,
                     help="prefill: scale the queries (peakier softmax, more skippable tiles)")
+    ap.add_argument("--decode-qscale", type=float, default=4.0,
+                    help="decode_blasst: scale of the queries (1 = the plain 64K inputs)")
+    ap.add_argument("--decode-lambda", type=float, default=1e-3, help="decode_blasst: threshold")
     ap.add_argument("--rotate", type=int, default=0, help="input copies (0 = auto, > 4x L2)")
     ap.add_argument("--e2e-steps", type=int, default=2000)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
@@ -82,7 +86,7 @@ def parse():
                     help="a few launches on 2 input copies, for ncu captures")
     a = ap.parse_args()
     defaults = {"blockquery": (20000, 200), "blasst_prefill_32k": (20, 3),
-                "losa_step": (8000, 200)}.get(a.workload, (200000, 600))
+                "losa_step": (8000, 200), "decode_blasst": (80000, 600)}.get(a.workload, (200000, 600))
     if a.steps is None:
         a.steps = defaults[0]
     if a.warmup is None:
@@ -896,14 +900,94 @@ def run_losa_step(args):
     }
 
 
+def run_decode_blasst(args):
+    """BLASST inside sparse decode on the 64K GQA decode inputs: the selection of the fused
+    decode (16 blocks per KV head, its own kernels) is given to lsa_sparse_attn_decode_blasst,
+    which reads K of every selected block and V only of the blocks some head still needs.
+    The queries are scaled by --decode-qscale (a sharper softmax: 1 = the plain workload,
+    where no block is negligible).  Each launch is timed alone with CUDA events after an L2
+    flush (a 512 MB write), next to the plain given-selection decode on the same inputs."""
+    import query_aware_block_b200 as lsa
+    import synth
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    c = synth.gqa_decode_64k(device=dev)
+    B, Hq, D = c.q.shape
+    Hkv, T_cap = c.k.shape[1], c.k.shape[2]
+    G = Hq // Hkv
+    lam = args.decode_lambda
+    q = (c.q.float() * args.decode_qscale).to(torch.bfloat16)
+    summ = torch.zeros(B, Hkv, -(-T_cap // 64), D, device=dev)
+    lsa.lsa_build_summaries(c.k, c.seqlens, summ)
+    idx = torch.empty(B, Hkv, 16, dtype=torch.int32, device=dev)
+    o = torch.empty(B, Hq, D, dtype=torch.bfloat16, device=dev)
+    lse = torch.empty(B, Hq, device=dev)
+    lsa.lsa_sparse_attn_decode(c.q, c.k, c.v, c.seqlens, o, 16, summ=summ, n_sink=1, n_local=2,
+                               idx_out=idx, lse=lse)
+    nsel = (idx >= 0).sum(-1).to(torch.int32)
+    bits = torch.zeros(B, Hkv, dtype=torch.int32, device=dev)
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
+
+    def blasst():
+        lsa.lsa_sparse_attn_decode_blasst(q, c.k, c.v, c.seqlens, idx, nsel, o, lam, lse=lse, skip_bits=bits)
+
+    def plain():
+        lsa.lsa_sparse_attn_decode(q, c.k, c.v, c.seqlens, o, 16, idx=idx, nsel=nsel, lse=lse)
+
+    def cold_us(fn, n):
+        for _ in range(max(3, args.warmup // 100)):
+            flush.fill_(1)
+            fn()
+        torch.cuda.synchronize()
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+        for e0, e1 in evs:
+            flush.fill_(1)
+            e0.record()
+            fn()
+            e1.record()
+        torch.cuda.synchronize()
+        return sum(e0.elapsed_time(e1) for e0, e1 in evs) / n * 1e3
+
+    n = max(20, min(500, args.steps // 400))
+    with ClockSampler(0) as clocks:
+        t_blasst = cold_us(blasst, n)
+        t_plain = cold_us(plain, n)
+    blasst()
+    torch.cuda.synchronize()
+    skipped = sum(bin(int(x) & 0xFFFFFFFF).count("1") for x in bits.flatten().tolist())
+    slots = int(nsel.sum())
+    blk_bytes = 64 * D * 2
+    step_bytes = slots * blk_bytes + (slots - skipped) * blk_bytes + 2 * B * Hq * D * 2 + B * Hkv * 16 * 4
+    gbs = step_bytes / (t_blasst * 1e-6) / 1e9
+    peak, kind = measured_peaks()
+    return {
+        "metric": "BLASST sparse decode over a given selection (64K GQA decode inputs): tokens/s and effective GB/s",
+        "value": round(B / (t_blasst * 1e-6), 1), "unit": "tokens/s", "n_gpus": 1, "steps": n,
+        "warmup": args.warmup, "ms_per_step": round(t_blasst * 1e-3, 6), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": f"synthetic 64K GQA decode inputs (seeded), queries x{args.decode_qscale}",
+        "config": {"workload": "decode_blasst", "batch": B, "kv_heads": Hkv, "q_heads_per_kv": G,
+                   "head_dim": D, "context": T_cap, "topk": 16, "lambda": lam,
+                   "l2": "flushed before every launch (512 MB write)"},
+        "skip_fraction": round(skipped / max(1, slots), 4), "skipped_v_blocks": skipped, "selected_blocks": slots,
+        "plain_given_selection_decode_us": round(t_plain, 2), "blasst_decode_us": round(t_blasst, 2),
+        "bytes_per_step": int(step_bytes),
+        "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peak, "unit": "GB/s",
+                     "frac": round(gbs / peak, 4), "traffic": None, "kernel": "decode_blasst_kernel<128>",
+                     "peak_source": f"MEASURED_PEAKS.json hbm_gbs ({kind})"},
+        "gpu_launches": n,
+        "clocks": clocks.summary(),
+    }
+
+
 def main():
     args = parse()
-    if args.workload in ("blockquery", "blasst_prefill_32k", "losa_step"):
+    if args.workload in ("blockquery", "blasst_prefill_32k", "losa_step", "decode_blasst"):
         if args.impl == "reference":
             print(json.dumps({"impl": "reference", "unavailable": "the oracle arm covers the decode workloads"}))
             return
         res = {"blockquery": run_blockquery, "blasst_prefill_32k": run_prefill,
-               "losa_step": run_losa_step}[args.workload](args)
+               "losa_step": run_losa_step, "decode_blasst": run_decode_blasst}[args.workload](args)
         print(json.dumps(res), flush=True)
         return
     world = int(os.environ.get("WORLD_SIZE", "1"))

@@ -251,6 +251,37 @@ LSA_API int lsa_sparse_attn_blockquery_noalloc(const void* q, const void* k, con
                                                cudaStream_t stream);
 
 /*
+ * lsa_sparse_attn_decode_blasst -- sparse decode attention over a given block selection
+ * that drops, before reading their V, the selected blocks whose softmax weight is
+ * negligible (BLASST inside sparse decode).
+ *
+ * Defined by: BLASST, "2. 방법론" -- "핵심 아이디어: 온라인 Softmax 통계 활용" (a block whose
+ * local maximum trails the running maximum by more than the threshold contributes
+ * nothing after the softmax) and "알고리즘 및 커널 설계" (block_max - running_max < ln(lambda);
+ * the decode kernel, bound by memory, saves the V-block loads).
+ *
+ * For each (b, g) the selected blocks idx[b, g, :nsel] (ascending) are visited in order as
+ * the blocks of an online softmax.  For block s and query head h of the group:
+ *   r_h = max over the block's tokens t < seqlens[b] of scale * q_h . k_t
+ *   m_h = the running maximum over the blocks visited before s
+ *   skip block s  iff  s is not the first visited and max over h of (r_h - m_h) < ln(lambda)
+ * (the group's heads share the block's V, so it is dropped only when every head finds it
+ * negligible).  The output is softmax attention over the tokens of the kept blocks:
+ * o [B, Hq, D] bf16, lse [B, Hq] float32 or NULL.  lambda = 0 never skips (and equals
+ * lsa_sparse_attn_decode with the same selection).
+ * skip_bits [B, Hkv] uint32 out or NULL: bit s set iff slot s was skipped.
+ * q [B, Hq, D] bf16; k, v [B, Hkv, T_cap, D] bf16; seqlens [B]; idx [B, Hkv, topk]
+ * ascending, -1 padded; nsel [B, Hkv].
+ * Requires bf16, 1 <= topk <= 16, 0 <= lambda < 1.
+ */
+LSA_API int lsa_sparse_attn_decode_blasst(const void* q, const void* k, const void* v, int dtype,
+                                          int B, int Hkv, int G, int D, int T_cap,
+                                          const int32_t* seqlens, int blk, const int32_t* idx,
+                                          const int32_t* nsel, int topk, float scale,
+                                          float lambda, void* o, float* lse,
+                                          uint32_t* skip_bits, cudaStream_t stream);
+
+/*
  * lsa_losa_classify -- active and stable tokens of a query block between two denoising
  * steps.
  *

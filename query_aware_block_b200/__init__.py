@@ -30,7 +30,7 @@ EXPORTED = ("lsa_status_string", "lsa_last_cuda_error", "lsa_version", "lsa_buil
             "lsa_select_blocks", "lsa_sparse_attn_decode", "lsa_blockquery_workspace_size",
             "lsa_sparse_attn_blockquery", "lsa_sparse_attn_blockquery_noalloc",
             "lsa_blasst_prefill", "lsa_device_status", "lsa_losa_classify",
-            "lsa_blockquery_intra_merge")
+            "lsa_blockquery_intra_merge", "lsa_sparse_attn_decode_blasst")
 
 _vp, _i, _f = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
 _lib.lsa_status_string.restype = ctypes.c_char_p
@@ -55,6 +55,8 @@ _lib.lsa_sparse_attn_blockquery_noalloc.argtypes = [_vp, _vp, _vp, _i, _i, _i, _
 _lib.lsa_blasst_prefill.argtypes = [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _f, _vp, _vp, _vp,
                                     _vp, _vp]
 _lib.lsa_device_status.argtypes = [_vp, _i]
+_lib.lsa_sparse_attn_decode_blasst.argtypes = [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp, _i,
+                                               _vp, _vp, _i, _f, _f, _vp, _vp, _vp, _vp]
 _lib.lsa_losa_classify.argtypes = [_vp, _vp, _i, _i, _i, _i, _i, ctypes.c_double, _i, _vp, _vp,
                                    _vp]
 _lib.lsa_blockquery_intra_merge.argtypes = [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _f,
@@ -175,6 +177,21 @@ def lsa_blasst_prefill(q, k, v, o, lam, lse=None, skip_bits=None, skipped_tiles=
                                    float(scale), float(lam), _ptr(o), _ptr(lse), _ptr(skip_bits),
                                    _ptr(skipped_tiles), _stream(stream)),
            "lsa_blasst_prefill")
+    return o
+
+
+def lsa_sparse_attn_decode_blasst(q, k, v, seqlens, idx, nsel, o, lam, lse=None, skip_bits=None,
+                                  scale=0.0, blk=BLK, stream=None):
+    """Sparse decode over the given selection idx [B,Hkv,topk] with BLASST's skip: blocks
+    every head of the group finds negligible (below the running max by -ln(lam)) are not
+    read.  skip_bits: optional int32 [B,Hkv] out (bit s = slot s skipped)."""
+    B, Hq, D = q.shape
+    _, Hkv, T_cap, _ = k.shape
+    _check(_lib.lsa_sparse_attn_decode_blasst(_ptr(q), _ptr(k), _ptr(v), _dtype(q), B, Hkv,
+                                              Hq // Hkv, D, T_cap, _ptr(seqlens), blk, _ptr(idx),
+                                              _ptr(nsel), idx.shape[-1], float(scale), float(lam),
+                                              _ptr(o), _ptr(lse), _ptr(skip_bits), _stream(stream)),
+           "lsa_sparse_attn_decode_blasst")
     return o
 
 

@@ -705,6 +705,11 @@ cudaError_t launch_blockquery(const BlockQueryArgs& a, cudaStream_t stream) {
   auto kernel = a.D == 128 ? blockquery_kernel<128> : blockquery_kernel<64>;
   static int smem_set128 = 0, smem_set64 = 0;
   int& smem_set = a.D == 128 ? smem_set128 : smem_set64;
+  // the last (cluster size, shared memory) found schedulable, per head dim: the occupancy
+  // query is a host-side cost paid only when the configuration changes
+  static int ok_cl128 = 0, ok_smem128 = 0, ok_cl64 = 0, ok_smem64 = 0;
+  int& ok_cl = a.D == 128 ? ok_cl128 : ok_cl64;
+  int& ok_smem = a.D == 128 ? ok_smem128 : ok_smem64;
   for (;;) {
     p.per_max = (NBp + CL - 1) / CL;
     if (p.per_max < 1) p.per_max = 1;
@@ -734,15 +739,19 @@ cudaError_t launch_blockquery(const BlockQueryArgs& a, cudaStream_t stream) {
     attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    int nclusters = 0;
-    err = cudaOccupancyMaxActiveClusters(&nclusters, kernel, &cfg);
-    if (err != cudaSuccess || nclusters == 0) {
-      (void)cudaGetLastError();
-      if (CL > 2) {
-        CL >>= 1;
-        continue;
+    if (!(CL == ok_cl && smem == ok_smem)) {
+      int nclusters = 0;
+      err = cudaOccupancyMaxActiveClusters(&nclusters, kernel, &cfg);
+      if (err != cudaSuccess || nclusters == 0) {
+        (void)cudaGetLastError();
+        if (CL > 2) {
+          CL >>= 1;
+          continue;
+        }
+        return err != cudaSuccess ? err : cudaErrorInvalidConfiguration;
       }
-      return err != cudaSuccess ? err : cudaErrorInvalidConfiguration;
+      ok_cl = CL;
+      ok_smem = smem;
     }
     cfg.numAttrs = 2;  // launched as a programmatic dependent of the previous kernel
     return cudaLaunchKernelEx(&cfg, kernel, p);

@@ -136,6 +136,30 @@ int lsa_sparse_attn_decode(const void* q, const void* k, const void* v, int dtyp
   return cuda_status(lsa::launch_decode(a, stream));
 }
 
+int lsa_sparse_attn_decode_blasst(const void* q, const void* k, const void* v, int dtype, int B,
+                                  int Hkv, int G, int D, int T_cap, const int32_t* seqlens,
+                                  int blk, const int32_t* idx, const int32_t* nsel, int topk,
+                                  float scale, float lambda, void* o, float* lse,
+                                  uint32_t* skip_bits, cudaStream_t stream) {
+  int st = check_common(dtype, B, Hkv, G, D, blk);
+  if (st != LSA_OK) return st;
+  if (dtype != LSA_BF16) return LSA_ERR_UNSUPPORTED;
+  if (T_cap < 0 || topk < 1 || topk > 16 || !(lambda >= 0.f) || !(lambda < 1.f))
+    return LSA_ERR_INVALID_ARG;
+  if (T_cap > kMaxTcap || B > 65535 || Hkv > 65535) return LSA_ERR_UNSUPPORTED;
+  if (B == 0 || Hkv == 0) return LSA_OK;
+  if (!q || !k || !v || !seqlens || !idx || !nsel || !o) return LSA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return LSA_ERR_INVALID_ARG;
+  lsa::DecodeBlasstArgs a = {};
+  a.q = q; a.k = k; a.v = v;
+  a.B = B; a.Hkv = Hkv; a.G = G; a.D = D; a.T_cap = T_cap;
+  a.seqlens = seqlens; a.idx = idx; a.nsel = nsel; a.topk = topk;
+  a.scale = resolve_scale(scale, D);
+  a.lambda = lambda;
+  a.o = o; a.lse = lse; a.skip_bits = skip_bits;
+  return cuda_status(lsa::launch_decode_blasst(a, stream));
+}
+
 size_t lsa_blockquery_workspace_size(int B, int Hkv, int G, int D, int Tq) {
   if (B <= 0 || Hkv <= 0 || G <= 0 || D <= 0 || Tq <= 0) return 0;
   return lsa::blockquery_workspace_bytes(B, Hkv, G, D, Tq);

@@ -63,6 +63,23 @@ struct BlockQueryArgs {
 size_t blockquery_workspace_bytes(int B, int Hkv, int G, int D, int Tq);
 cudaError_t launch_blockquery(const BlockQueryArgs& a, cudaStream_t stream);
 
+// Sparse decode over a given selection with BLASST's skip (V not read for negligible blocks).
+struct DecodeBlasstArgs {
+  const void* q;
+  const void* k;
+  const void* v;
+  int B, Hkv, G, D, T_cap;
+  const int32_t* seqlens;
+  const int32_t* idx;
+  const int32_t* nsel;
+  int topk;
+  float scale, lambda;
+  void* o;
+  float* lse;
+  uint32_t* skip_bits;
+};
+cudaError_t launch_decode_blasst(const DecodeBlasstArgs& a, cudaStream_t stream);
+
 // LoSA: token activity and the attention inside the query block merged with the prefix.
 cudaError_t launch_losa_classify(const void* q, const void* q_prev, int B, int Hq, int Tq, int D,
                                  double tau, int n_top, uint8_t* active, double* mse,

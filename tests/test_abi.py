@@ -116,6 +116,25 @@ def test_losa_entry_points_validation():
     assert bq(*args(0, 64 * 100)) == lsa.LSA_ERR_INVALID_ARG
 
 
+def test_decode_blasst_validation():
+    import query_aware_block_b200 as lsa
+    f = lsa.library().lsa_sparse_attn_decode_blasst
+    g = ctypes.c_void_p(4096)
+    args = lambda dtype=1, D=128, topk=16, lam=1e-3, G=8: (g, g, g, dtype, 1, 8, G, D, 65536, g, 64, g, g, topk, 0.0, lam, g, NULL, NULL, NULL)
+    assert f(*args(dtype=0)) == lsa.LSA_ERR_UNSUPPORTED      # fp32
+    assert f(*args(D=96)) == lsa.LSA_ERR_UNSUPPORTED
+    assert f(*args(G=17)) == lsa.LSA_ERR_UNSUPPORTED
+    assert f(*args(topk=17)) == lsa.LSA_ERR_INVALID_ARG      # one cluster slot per block
+    assert f(*args(topk=0)) == lsa.LSA_ERR_INVALID_ARG
+    assert f(*args(lam=1.0)) == lsa.LSA_ERR_INVALID_ARG
+    assert f(*args(lam=-0.1)) == lsa.LSA_ERR_INVALID_ARG
+    assert f(*args(lam=float("nan"))) == lsa.LSA_ERR_INVALID_ARG
+    bad = list(args())
+    bad[11] = NULL  # idx
+    assert f(*bad) == lsa.LSA_ERR_INVALID_ARG
+    assert f(g, g, g, 1, 0, 8, 8, 128, 65536, NULL, 64, NULL, NULL, 16, 0.0, 1e-3, NULL, NULL, NULL, NULL) == lsa.LSA_OK
+
+
 def test_binding_raises_lsa_error_on_bad_arguments():
     import torch
     import query_aware_block_b200 as lsa
