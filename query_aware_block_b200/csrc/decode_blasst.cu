@@ -49,6 +49,8 @@ struct Smem {
   float rloc[kMaxG];                 // this CTA's block maxima
   float part_m[kMaxG], part_l[kMaxG];
   float part_acc[kMaxG * D];
+  int slot_block[kCL];               // the block of every slot, -1 if none
+  uint32_t valid;                    // bit s: slot s holds a block
 };
 
 // Launched with clusters of kCL CTAs along x (grid (kCL, Hkv, B)).
@@ -71,28 +73,36 @@ __global__ void __launch_bounds__(kThreads)
   const size_t unit = (size_t)b * Hkv + g;
   cluster_arrive_relaxed();  // peers' shared memory is written only after all have started
 
-  // which slots hold a block (the same on every CTA)
+  // which slots hold a block (the same on every CTA): one load per lane of warp 0, all in
+  // flight together; the q rows of the group start copying meanwhile
+  for (int id = tid; id < G * kC; id += kThreads) {
+    const int h = id / kC, c = id - h * kC;
+    cp_async16(sm.q + h * D + c * 8, q + ((size_t)b * Hq + (size_t)g * G + h) * D + c * 8, true);
+  }
+  cp_async_commit();
   const int T = seqlens[b];
-  const int ns = min(nsel[unit], topk);
-  uint32_t valid = 0u;
-  for (int s = 0; s < ns; ++s)
-    if (idx[unit * topk + s] >= 0) valid |= 1u << s;
+  if (warp == 0) {
+    const int ns = nsel[unit];
+    const int jj = lane < topk && lane < kCL ? idx[unit * topk + lane] : -1;
+    const bool on = lane < ns && jj >= 0;
+    const uint32_t bits = __ballot_sync(0xffffffffu, on);
+    if (lane < kCL) sm.slot_block[lane] = on ? jj : -1;
+    if (lane == 0) sm.valid = bits;
+  }
+  __syncthreads();
+  const uint32_t valid = sm.valid;
   const bool has = (valid >> rank) & 1u;
-  const int j = has ? idx[unit * topk + rank] : 0;
+  const int j = has ? sm.slot_block[rank] : 0;
   const int nv = has ? max(0, min(kBlk, T - j * kBlk)) : 0;  // valid rows of the block
   const size_t kvrow0 = unit * (size_t)T_cap + (size_t)j * kBlk;
 
-  // q rows of the group and the K block (rows past the sequence are not read)
-  for (int id = tid; id < G * kC; id += kThreads) {
-    const int h = id / kC, c = id - h * kC;
-    *reinterpret_cast<uint4*>(sm.q + h * D + c * 8) =
-        __ldg(reinterpret_cast<const uint4*>(q + ((size_t)b * Hq + (size_t)g * G + h) * D) + c);
-  }
+  // the K block (rows past the sequence are not read), every copy in flight at once
   for (int id = tid; id < nv * kC; id += kThreads) {
     const int r = id / kC, c = id - r * kC;
-    *reinterpret_cast<uint4*>(sm.kv + r * kKS + c * 8) =
-        __ldg(reinterpret_cast<const uint4*>(k + (kvrow0 + r) * D) + c);
+    cp_async16(sm.kv + r * kKS + c * 8, k + (kvrow0 + r) * D + c * 8, true);
   }
+  cp_async_commit();
+  cp_async_wait<0>();
   __syncthreads();
   // logits in base 2: pair (h, t) = (p >> 6, p & 63); a warp shares h (q reads broadcast)
   for (int p = tid; p < G * kBlk; p += kThreads) {
@@ -169,10 +179,10 @@ __global__ void __launch_bounds__(kThreads)
   if (keep) {
     for (int id = tid; id < nv * kC; id += kThreads) {
       const int r = id / kC, c = id - r * kC;
-      *reinterpret_cast<uint4*>(sm.kv + r * kKS + c * 8) =
-          __ldg(reinterpret_cast<const uint4*>(v + (kvrow0 + r) * D) + c);
+      cp_async16(sm.kv + r * kKS + c * 8, v + (kvrow0 + r) * D + c * 8, true);
     }
   }
+  cp_async_commit();
   for (int h = warp; h < G; h += kWarps) {  // probabilities and row sums (warp per head)
     const float r = sm.rmax[rank][h];
     float p0 = 0.f, p1 = 0.f;
@@ -188,6 +198,7 @@ __global__ void __launch_bounds__(kThreads)
       sm.part_l[h] = l;
     }
   }
+  cp_async_wait<0>();  // (the V copies overlapped the softmax above)
   __syncthreads();
   {
     // output element (h, d): thread takes d = tid % D and heads tid / D + k * (256 / D)
