@@ -9,7 +9,7 @@ the CUDA library in ``query_aware_block_b200``.
 Parity status of each function (what pins it is in tests/test_oracle_pins.py):
   summaries, block_scores, select, decode_attn, blockquery_select, blockquery_attn,
   blasst_prefill, decode_blasst, losa_classify, blockquery_intra_merge (and the losa_step
-  composition)
+  composition), nsa_compress, range_attn_f64, window_attn (and the nsa_decode composition)
   -- all pinned (textbook special cases, brute force, library routines, closed forms and
   invariants).
 """
@@ -314,3 +314,78 @@ def decode_blasst(q, k, v, seqlens, idx, nsel, lam, blk=64, scale=None, forced_b
                                  ctypes.c_double(float(lam)), _p(fb), _p(o), _p(lse), _p(bits),
                                  _p(gap))
     return dict(o=o, lse=lse, bits=bits.to(torch.int64) & 0xFFFFFFFF, gap=gap)
+
+
+def nsa_compress(x, seqlens, length=32, stride=16):
+    """Mean-pooled compressed tokens: x [B,Hkv,T_cap,D] -> fp64 [B,Hkv,ceil(T_cap/stride),D],
+    row i the mean of the valid tokens of [i*stride, i*stride + length) (zeros past
+    ceil(T_b/stride))."""
+    x = x.contiguous()
+    B, Hkv, T_cap, D = x.shape
+    out = torch.empty(B, Hkv, -(-T_cap // stride), D, dtype=torch.float64)
+    sl = _i32(seqlens)
+    _load().oracle_nsa_compress(_p(x), _dt(x), B, Hkv, T_cap, D, _p(sl), int(length), int(stride),
+                                _p(out))
+    return out
+
+
+def range_attn_f64(q, kc, vc, t0, t1, scale=None):
+    """Attention of q [B,Hq,D] over tokens [t0_b, t1_b) of fp64 kc, vc [B,Hkv,N_cap,D]."""
+    q = q.contiguous()
+    kc = kc.to(torch.float64).contiguous()
+    vc = vc.to(torch.float64).contiguous()
+    B, Hq, D = q.shape
+    _, Hkv, N_cap, _ = kc.shape
+    o = torch.empty(B, Hq, D, dtype=torch.float64)
+    lse = torch.empty(B, Hq, dtype=torch.float64)
+    _load().oracle_range_attn_f64(_p(q), _dt(q), _p(kc), _p(vc), B, Hkv, Hq // Hkv, D, N_cap,
+                                  _p(_i32(t0)), _p(_i32(t1)), ctypes.c_double(_scale(scale, D)),
+                                  _p(o), _p(lse))
+    return o, lse
+
+
+def window_attn(q, k, v, seqlens, w=512, scale=None):
+    """Attention of the decode query over the last w tokens of each sequence."""
+    q, k, v = q.contiguous(), k.contiguous(), v.contiguous()
+    B, Hq, D = q.shape
+    _, Hkv, T_cap, _ = k.shape
+    o = torch.empty(B, Hq, D, dtype=torch.float64)
+    lse = torch.empty(B, Hq, dtype=torch.float64)
+    _load().oracle_window_attn(_p(q), _p(k), _p(v), _dt(q), B, Hkv, Hq // Hkv, D, T_cap,
+                               _p(_i32(seqlens)), int(w), ctypes.c_double(_scale(scale, D)),
+                               _p(o), _p(lse))
+    return o, lse
+
+
+def nsa_decode(q, k, v, seqlens, topk=16, n_sink=1, n_local=2, gates=(1 / 3, 1 / 3, 1 / 3),
+               length=32, stride=16, window=512, blk=64, scale=None, idx=None):
+    """NSA's three parallel branches for one decode step, with fixed parts in place of the
+    learned ones: the compressed branch (attention over mean-pooled tokens of `length`
+    keys at `stride`), the selected branch (the query-aware block selection and sparse
+    attention of this oracle; `idx` replaces the oracle's own selection) and the sliding
+    window (the last `window` tokens), combined as
+        o = gates[0] * o_cmp + gates[1] * o_slc + gates[2] * o_win.
+    Returns the branches, the combined o and the tokens each branch reads."""
+    B = q.shape[0]
+    sl = _i32(seqlens)
+    kc = nsa_compress(k, sl, length, stride)
+    vc = nsa_compress(v, sl, length, stride)
+    nc = torch.tensor([-(-int(t) // stride) for t in sl], dtype=torch.int32)
+    o_cmp, lse_cmp = range_attn_f64(q, kc, vc, torch.zeros(B, dtype=torch.int32), nc, scale)
+    if idx is None:
+        r = decode(q, k, v, sl, topk, n_sink, n_local, blk, scale)
+        idx, nsel = r["idx"], r["nsel"]
+        o_slc, lse_slc = r["o"], r["lse"]
+    else:
+        idx = _i32(idx)
+        nsel = (idx >= 0).sum(-1).to(torch.int32)
+        o_slc, lse_slc = decode_attn(q, k, v, sl, idx, nsel, blk, scale)
+    o_win, lse_win = window_attn(q, k, v, sl, window, scale)
+    g = [float(x) for x in gates]
+    o = g[0] * o_cmp + g[1] * o_slc + g[2] * o_win
+    tokens = dict(compressed=[int(x) for x in nc],
+                  selected=[[min(blk, int(t) - int(j) * blk) if j >= 0 else 0 for j in row]
+                            for row, t in zip(idx[:, 0].tolist(), sl.tolist())],
+                  window=[min(window, int(t)) for t in sl])
+    return dict(o=o, o_cmp=o_cmp, lse_cmp=lse_cmp, o_slc=o_slc, lse_slc=lse_slc, o_win=o_win,
+                lse_win=lse_win, idx=idx, nsel=nsel, kc=kc, vc=vc, tokens=tokens)

@@ -36,6 +36,12 @@
  *                            the group finds negligible is not read: no V load)
  *                            [BLASST, "2. 방법론", "알고리즘 및 커널 설계": the decode kernel
  *                             saves the V-block loads]
+ *   oracle_nsa_compress,     NSA's other two branches with fixed, non-learned parts:
+ *   oracle_range_attn_f64,   mean-pooled compressed tokens (block l, stride d) and attention
+ *   oracle_window_attn       over them; attention over the sliding window of the last w
+ *                            tokens [NSA news article, "NSA 구조": three parallel paths --
+ *                            compressed coarse tokens, selected fine tokens, a sliding
+ *                            window -- with l = 32, d = 16, l' = 64, n = 16, w = 512]
  *   oracle_losa_classify     active / stable tokens by the mean squared change of their
  *                            queries between denoising steps [LoSA, "2. 방법론": the query
  *                            change (MSE) of every step sorts tokens into active and stable]
@@ -54,6 +60,9 @@
  *     (tile row max - running row max) < ln(lambda); strict '<' as printed.
  *   - in decode the rows of BLASST's tile are the query heads of a GQA group (they share
  *     the block's V): skip iff every head's (block max - running max) < ln(lambda);
+ *   - NSA's compressed token i is the mean over [i*d, i*d + l) of the valid tokens (a
+ *     fixed pool in place of the learned compression), ceil(T/d) of them; the window is
+ *     the last w tokens; the three branch outputs are combined with caller-given gates;
  *   - LoSA's query change is the mean over all query heads and dims of the squared
  *     difference; active iff it exceeds tau (or: the n_top largest, ties to the lower
  *     index);
@@ -734,6 +743,110 @@ void oracle_decode_blasst(const void* q, const void* k, const void* v, int dtype
       free(r);
       free(l);
       free(m);
+    }
+  }
+}
+
+/* ------------------------------------------------------------------------------------
+ * NSA's compressed tokens with a fixed (non-learned) compression: the mean pool.
+ *   out[b,g,i,:] = mean of x[b,g,t,:] over t in [i*stride, i*stride + len) and t < T_b,
+ * for i < NC_b = ceil(T_b / stride) (a block that runs past the sequence is averaged over
+ * its valid tokens, as a partial summary block is); rows i >= NC_b are zeros.
+ * x [B,Hkv,T_cap,D] (dtype); out [B,Hkv,ceil(T_cap/stride),D] double.
+ * ---------------------------------------------------------------------------------- */
+void oracle_nsa_compress(const void* x, int dtype, int B, int Hkv, int T_cap, int D,
+                         const int32_t* seqlens, int len, int stride, double* out) {
+  const int NC_cap = ceil_div(T_cap, stride);
+#pragma omp parallel for collapse(2) schedule(dynamic)
+  for (int b = 0; b < B; ++b) {
+    for (int g = 0; g < Hkv; ++g) {
+      const int T = seqlens[b];
+      const int NC = ceil_div(T, stride);
+      for (int i = 0; i < NC_cap; ++i) {
+        double* o = out + (((size_t)b * Hkv + g) * NC_cap + i) * D;
+        for (int d = 0; d < D; ++d) o[d] = 0.0;
+        if (i >= NC) continue;
+        const int t0 = i * stride;
+        const int t1 = (t0 + len < T) ? t0 + len : T;
+        for (int t = t0; t < t1; ++t) {
+          const size_t row = (((size_t)b * Hkv + g) * T_cap + t) * D;
+          for (int d = 0; d < D; ++d) o[d] += elem(x, dtype, row + d);
+        }
+        for (int d = 0; d < D; ++d) o[d] /= (double)(t1 - t0);
+      }
+    }
+  }
+}
+
+/* ------------------------------------------------------------------------------------
+ * Softmax attention of every decode query over a contiguous token range [t0_b, t1_b) of a
+ * cache (double values): logit = scale * q_h . kc[t]; o = sum softmax * vc[t]; lse.
+ * Used for NSA's compressed branch (range [0, NC_b) of the pooled cache) with
+ * kc, vc [B,Hkv,N_cap,D] double; an empty range gives o = 0, lse = -inf.
+ * ---------------------------------------------------------------------------------- */
+void oracle_range_attn_f64(const void* q, int dtype, const double* kc, const double* vc, int B,
+                           int Hkv, int G, int D, int N_cap, const int32_t* t0s,
+                           const int32_t* t1s, double scale, double* o, double* lse) {
+  const int Hq = Hkv * G;
+#pragma omp parallel for collapse(2) schedule(dynamic)
+  for (int b = 0; b < B; ++b) {
+    for (int h = 0; h < Hq; ++h) {
+      const int g = h / G;
+      const int t0 = t0s[b], t1 = t1s[b];
+      const size_t qrow = ((size_t)b * Hq + h) * D;
+      const size_t base = ((size_t)b * Hkv + g) * (size_t)N_cap * D;
+      double* out = o + qrow;
+      for (int d = 0; d < D; ++d) out[d] = 0.0;
+      if (t1 <= t0) {
+        lse[(size_t)b * Hq + h] = -INFINITY;
+        continue;
+      }
+      double* logit = (double*)malloc(sizeof(double) * (size_t)(t1 - t0));
+      double m = -INFINITY;
+      for (int t = t0; t < t1; ++t) {
+        double dot = 0.0;
+        for (int d = 0; d < D; ++d) dot += elem(q, dtype, qrow + d) * kc[base + (size_t)t * D + d];
+        logit[t - t0] = scale * dot;
+        if (logit[t - t0] > m) m = logit[t - t0];
+      }
+      double l = 0.0;
+      for (int t = t0; t < t1; ++t) {
+        const double p = exp(logit[t - t0] - m);
+        l += p;
+        for (int d = 0; d < D; ++d) out[d] += p * vc[base + (size_t)t * D + d];
+      }
+      for (int d = 0; d < D; ++d) out[d] /= l;
+      lse[(size_t)b * Hq + h] = m + log(l);
+      free(logit);
+    }
+  }
+}
+
+/* ------------------------------------------------------------------------------------
+ * NSA's sliding-window branch: softmax attention of the decode query over the last w
+ * tokens of its sequence, t in [max(0, T_b - w), T_b).  q [B,Hq,D]; k, v [B,Hkv,T_cap,D].
+ * ---------------------------------------------------------------------------------- */
+void oracle_window_attn(const void* q, const void* k, const void* v, int dtype, int B, int Hkv,
+                        int G, int D, int T_cap, const int32_t* seqlens, int w, double scale,
+                        double* o, double* lse) {
+  const int Hq = Hkv * G;
+#pragma omp parallel for collapse(2) schedule(dynamic)
+  for (int b = 0; b < B; ++b) {
+    for (int g = 0; g < Hkv; ++g) {
+      const int T = seqlens[b];
+      const int t0 = T - w > 0 ? T - w : 0;
+      const int n = T - t0;
+      int* toks = (int*)malloc(sizeof(int) * (size_t)(n > 0 ? n : 1));
+      double* logits = (double*)malloc(sizeof(double) * (size_t)(n > 0 ? n : 1));
+      for (int i = 0; i < n; ++i) toks[i] = t0 + i;
+      const size_t kvbase = ((size_t)b * Hkv + g) * (size_t)T_cap * D;
+      for (int hh = 0; hh < G; ++hh) {
+        const size_t row = (size_t)b * Hq + g * G + hh;
+        attend_row(q, k, v, dtype, row * D, kvbase, D, toks, n, scale, logits, o + row * D,
+                   lse + row);
+      }
+      free(logits);
+      free(toks);
     }
   }
 }

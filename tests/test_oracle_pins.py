@@ -724,3 +724,84 @@ def test_decode_blasst_output_is_dense_over_kept_blocks_within_the_error_bound()
     none = oracle.decode_blasst(q, case.k, case.v, case.seqlens, idx, nsel, 0.5,
                                 forced_bits=torch.zeros(1, Hkv, dtype=torch.int64))
     assert torch.equal(none["o"], full["o"])
+
+
+# ------------------------------------------ NSA's compressed and sliding-window branches ----
+
+def test_nsa_compress_is_avg_pool_with_clipped_tail():
+    # library routine: avg_pool1d (kernel 32, stride 16, ceil mode: a window that runs past
+    # the end is divided by its valid count) gives every window that starts at least one
+    # stride before the end; the last window (start 16 * (NC - 1)) has a closed form
+    B, Hkv, T_cap, D = 2, 2, 700, 8
+    g = torch.Generator().manual_seed(71)
+    k = torch.randn(B, Hkv, T_cap, D, generator=g)
+    sl = torch.tensor([700, 333], dtype=torch.int32)
+    kc = oracle.nsa_compress(k, sl, 32, 16)
+    assert kc.shape == (B, Hkv, 44, D)
+    for b in range(B):
+        T = int(sl[b])
+        NC = -(-T // 16)
+        x = k[b, :, :T].double().transpose(1, 2)  # [Hkv, D, T]
+        ref = F.avg_pool1d(x, kernel_size=32, stride=16, ceil_mode=True).transpose(1, 2)
+        n = ref.shape[1]
+        assert n in (NC, NC - 1)
+        assert torch.allclose(kc[b, :, :n], ref, rtol=0, atol=1e-12)
+        t0 = 16 * (NC - 1)
+        assert torch.allclose(kc[b, :, NC - 1], k[b, :, t0:T].double().mean(dim=1), rtol=0, atol=1e-12)
+        assert torch.count_nonzero(kc[b, :, NC:]) == 0
+    # a ramp k_t = t: window [16i, min(16i + 32, T)) has mean (t0 + t1 - 1) / 2
+    ramp = torch.arange(T_cap, dtype=torch.float32)[None, None, :, None].expand(1, 1, T_cap, 4).contiguous()
+    kr = oracle.nsa_compress(ramp, torch.tensor([T_cap]), 32, 16)
+    for i in range(44):
+        t0, t1 = 16 * i, min(16 * i + 32, T_cap)
+        assert float(kr[0, 0, i, 0]) == (t0 + t1 - 1) / 2
+
+
+def test_nsa_compress_with_block_length_equal_to_stride_is_the_block_summary():
+    case = synth.decode_case(1, 2, 2, 32, T_cap=300, seqlens=300, dtype=torch.bfloat16, topk=4,
+                             n_sink=1, n_local=2, seed=72)
+    kc = oracle.nsa_compress(case.k, case.seqlens, 64, 64)
+    assert torch.equal(kc, oracle.summaries(case.k, case.seqlens))
+
+
+def test_nsa_window_and_compressed_branches_are_sdpa():
+    B, Hkv, G, D = 2, 2, 2, 32
+    case = synth.decode_case(B, Hkv, G, D, T_cap=1200, seqlens=[1200, 300], dtype=torch.float32,
+                             topk=4, n_sink=1, n_local=2, seed=73)
+    o_w, lse_w = oracle.window_attn(case.q, case.k, case.v, case.seqlens, 512)
+    kc = oracle.nsa_compress(case.k, case.seqlens, 32, 16)
+    vc = oracle.nsa_compress(case.v, case.seqlens, 32, 16)
+    nc = torch.tensor([75, 19], dtype=torch.int32)
+    o_c, lse_c = oracle.range_attn_f64(case.q, kc, vc, torch.zeros(2, dtype=torch.int32), nc)
+    sc = 1 / math.sqrt(D)
+    for b, T in ((0, 1200), (1, 300)):
+        t0 = max(0, T - 512)  # sequence 1 is shorter than the window: all of it
+        for g in range(Hkv):
+            qh = case.q[b, g * G:(g + 1) * G]
+            o_ref, lse_ref = _dense_rows(qh, case.k[b, g, t0:T], case.v[b, g, t0:T], sc)
+            assert torch.allclose(o_w[b, g * G:(g + 1) * G], o_ref, rtol=0, atol=1e-12)
+            assert torch.allclose(lse_w[b, g * G:(g + 1) * G], lse_ref, rtol=0, atol=1e-12)
+            n = int(nc[b])
+            o_ref, lse_ref = _dense_rows(qh, kc[b, g, :n], vc[b, g, :n], sc)
+            assert torch.allclose(o_c[b, g * G:(g + 1) * G], o_ref, rtol=0, atol=1e-12)
+            assert torch.allclose(lse_c[b, g * G:(g + 1) * G], lse_ref, rtol=0, atol=1e-12)
+
+
+def test_nsa_decode_combines_the_three_branches_and_reproduces_the_64k_accounting():
+    # the NSA page's 64K decoding count: 5,632 of 65,536 tokens read (4,096 compressed
+    # tokens, 16 selected blocks of 64, a 512-token window)
+    with open(os.path.join(GOLDEN, "nsa_decode_token_accounting.json")) as f:
+        gold = json.load(f)
+    T = gold["context"]
+    case = synth.decode_case(1, 1, 2, 16, T_cap=T, seqlens=T, dtype=torch.bfloat16, topk=16,
+                             n_sink=1, n_local=2, seed=74)
+    r = oracle.nsa_decode(case.q, case.k, case.v, case.seqlens, topk=gold["selected_blocks"],
+                          n_sink=gold["forced_initial_blocks"], n_local=gold["forced_local_blocks"],
+                          length=gold["compression_block"], stride=gold["compression_stride"],
+                          window=gold["window"])
+    t = r["tokens"]
+    assert t["compressed"] == [4096] and sum(t["selected"][0]) == 1024 and t["window"] == [512]
+    assert t["compressed"][0] + sum(t["selected"][0]) + t["window"][0] == gold["tokens_accessed"]
+    assert torch.allclose(r["o"], (r["o_cmp"] + r["o_slc"] + r["o_win"]) / 3, rtol=0, atol=1e-15)
+    only = oracle.nsa_decode(case.q, case.k, case.v, case.seqlens, gates=(0.0, 1.0, 0.0), idx=r["idx"])
+    assert torch.equal(only["o"], r["o_slc"])
