@@ -282,6 +282,50 @@ LSA_API int lsa_sparse_attn_decode_blasst(const void* q, const void* k, const vo
                                           uint32_t* skip_bits, cudaStream_t stream);
 
 /*
+ * lsa_nsa_compress -- NSA's compressed tokens with a fixed compression: the mean pool of
+ * every `len` keys (and values) at stride `stride`.
+ *
+ * Defined by: NSA news article, "NSA 구조" (a compressed path of coarse tokens beside the
+ * selected path and the sliding window; compression block l = 32, stride d = 16).  The
+ * learned compression of the model is replaced by its plainest fixed form, the mean.
+ *
+ *   kc[b, g, i, :] = mean of k[b, g, t, :] over t in [i*stride, i*stride + len), t < T_b,
+ *                    for i < NC_b = ceil(T_b / stride); rows i >= NC_b in the range are 0
+ * (vc likewise from v), accumulated in fp32 and stored in bf16 (round to nearest even).
+ * Range: nc_begin >= 0 -> compressed tokens [nc_begin, nc_end) (nc_end = -1: all);
+ *        nc_begin < 0  -> the last -nc_begin compressed tokens of each sequence (a decode
+ *        step that appended one token changes only the last ceil(len / stride) of them).
+ * k, v [B, Hkv, T_cap, D] bf16; kc, vc [B, Hkv, ceil(T_cap / stride), D] bf16 out.
+ * Requires bf16, D in {64, 128}, len, stride >= 1.
+ */
+LSA_API int lsa_nsa_compress(const void* k, const void* v, int dtype, int B, int Hkv, int T_cap,
+                             int D, const int32_t* seqlens, int len, int stride, int nc_begin,
+                             int nc_end, void* kc, void* vc, cudaStream_t stream);
+
+/*
+ * lsa_nsa_branches -- NSA's compressed and sliding-window branches for a decode step,
+ * combined with the selected branch by constant gates.
+ *
+ * Defined by: NSA news article, "NSA 구조" (three parallel attention paths -- compressed
+ * coarse tokens, selected fine tokens, a sliding window of w = 512 -- joined by gates; the
+ * model's gates are learned, here they are constants chosen by the caller).
+ *
+ *   o_cmp = softmax attention of q over kc / vc rows [0, ceil(T_b / stride))
+ *   o_win = softmax attention of q over k / v rows [max(0, T_b - window), T_b)
+ *   o     = g_cmp * o_cmp + g_slc * o_slc + g_win * o_win      (logits scale * q . k)
+ * o_slc is the selected branch's output (lsa_sparse_attn_decode), or NULL for none.
+ * q [B, Hq, D] bf16; k, v [B, Hkv, T_cap, D] bf16; kc, vc [B, Hkv, ceil(T_cap / stride), D]
+ * bf16 (lsa_nsa_compress); o [B, Hq, D] bf16 out (may be o_slc); lse_win, lse_cmp
+ * [B, Hq] float32 out or NULL (-inf for an empty branch).
+ * Requires bf16, D in {64, 128}, G <= 16, stride >= 1, window >= 0.
+ */
+LSA_API int lsa_nsa_branches(const void* q, const void* k, const void* v, const void* kc,
+                             const void* vc, int dtype, int B, int Hkv, int G, int D, int T_cap,
+                             const int32_t* seqlens, int window, int stride, float scale,
+                             float g_cmp, float g_slc, float g_win, const void* o_slc, void* o,
+                             float* lse_win, float* lse_cmp, cudaStream_t stream);
+
+/*
  * lsa_losa_classify -- active and stable tokens of a query block between two denoising
  * steps.
  *

@@ -30,7 +30,8 @@ EXPORTED = ("lsa_status_string", "lsa_last_cuda_error", "lsa_version", "lsa_buil
             "lsa_select_blocks", "lsa_sparse_attn_decode", "lsa_blockquery_workspace_size",
             "lsa_sparse_attn_blockquery", "lsa_sparse_attn_blockquery_noalloc",
             "lsa_blasst_prefill", "lsa_device_status", "lsa_losa_classify",
-            "lsa_blockquery_intra_merge", "lsa_sparse_attn_decode_blasst")
+            "lsa_blockquery_intra_merge", "lsa_sparse_attn_decode_blasst", "lsa_nsa_compress",
+            "lsa_nsa_branches")
 
 _vp, _i, _f = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
 _lib.lsa_status_string.restype = ctypes.c_char_p
@@ -57,6 +58,9 @@ _lib.lsa_blasst_prefill.argtypes = [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _
 _lib.lsa_device_status.argtypes = [_vp, _i]
 _lib.lsa_sparse_attn_decode_blasst.argtypes = [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp, _i,
                                                _vp, _vp, _i, _f, _f, _vp, _vp, _vp, _vp]
+_lib.lsa_nsa_compress.argtypes = [_vp, _vp, _i, _i, _i, _i, _i, _vp, _i, _i, _i, _i, _vp, _vp, _vp]
+_lib.lsa_nsa_branches.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp, _i, _i, _f,
+                                  _f, _f, _f, _vp, _vp, _vp, _vp, _vp]
 _lib.lsa_losa_classify.argtypes = [_vp, _vp, _i, _i, _i, _i, _i, ctypes.c_double, _i, _vp, _vp,
                                    _vp]
 _lib.lsa_blockquery_intra_merge.argtypes = [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _f,
@@ -192,6 +196,33 @@ def lsa_sparse_attn_decode_blasst(q, k, v, seqlens, idx, nsel, o, lam, lse=None,
                                               _ptr(nsel), idx.shape[-1], float(scale), float(lam),
                                               _ptr(o), _ptr(lse), _ptr(skip_bits), _stream(stream)),
            "lsa_sparse_attn_decode_blasst")
+    return o
+
+
+def lsa_nsa_compress(k, v, seqlens, kc, vc, length=32, stride=16, nc_begin=0, nc_end=-1,
+                     stream=None):
+    """Mean-pooled compressed keys and values: kc, vc [B,Hkv,ceil(T_cap/stride),D] bf16 (in
+    place); nc_begin < 0 refreshes the last -nc_begin compressed tokens of each sequence."""
+    B, Hkv, T_cap, D = k.shape
+    _check(_lib.lsa_nsa_compress(_ptr(k), _ptr(v), _dtype(k), B, Hkv, T_cap, D, _ptr(seqlens),
+                                 int(length), int(stride), int(nc_begin), int(nc_end), _ptr(kc),
+                                 _ptr(vc), _stream(stream)),
+           "lsa_nsa_compress")
+    return kc, vc
+
+
+def lsa_nsa_branches(q, k, v, kc, vc, seqlens, o, gates=(1 / 3, 1 / 3, 1 / 3), o_slc=None,
+                     window=512, stride=16, lse_win=None, lse_cmp=None, scale=0.0, stream=None):
+    """NSA's compressed and window branches of a decode step, combined with the selected
+    branch output o_slc: o = gates[0] * o_cmp + gates[1] * o_slc + gates[2] * o_win."""
+    B, Hq, D = q.shape
+    _, Hkv, T_cap, _ = k.shape
+    g = [float(x) for x in gates]
+    _check(_lib.lsa_nsa_branches(_ptr(q), _ptr(k), _ptr(v), _ptr(kc), _ptr(vc), _dtype(q), B, Hkv,
+                                 Hq // Hkv, D, T_cap, _ptr(seqlens), int(window), int(stride),
+                                 float(scale), g[0], g[1], g[2], _ptr(o_slc), _ptr(o),
+                                 _ptr(lse_win), _ptr(lse_cmp), _stream(stream)),
+           "lsa_nsa_branches")
     return o
 
 

@@ -160,6 +160,56 @@ int lsa_sparse_attn_decode_blasst(const void* q, const void* k, const void* v, i
   return cuda_status(lsa::launch_decode_blasst(a, stream));
 }
 
+int lsa_nsa_compress(const void* k, const void* v, int dtype, int B, int Hkv, int T_cap, int D,
+                     const int32_t* seqlens, int len, int stride, int nc_begin, int nc_end,
+                     void* kc, void* vc, cudaStream_t stream) {
+  int st = check_common(dtype, B, Hkv, 1, D, 64);
+  if (st != LSA_OK) return st;
+  if (dtype != LSA_BF16) return LSA_ERR_UNSUPPORTED;
+  if (T_cap < 0 || len < 1 || stride < 1) return LSA_ERR_INVALID_ARG;
+  if (T_cap > kMaxTcap || len > 4096 || B > 32767 || Hkv > 65535) return LSA_ERR_UNSUPPORTED;
+  if (B == 0 || Hkv == 0 || T_cap == 0) return LSA_OK;
+  if (!k || !v || !seqlens || !kc || !vc) return LSA_ERR_INVALID_ARG;
+  if (!aligned16(k) || !aligned16(v) || !aligned16(kc) || !aligned16(vc)) return LSA_ERR_INVALID_ARG;
+  const int NC_cap = ceil_div(T_cap, stride);
+  int range_max;
+  if (nc_begin >= 0) {
+    const int hi = nc_end >= 0 ? (nc_end < NC_cap ? nc_end : NC_cap) : NC_cap;
+    range_max = hi - nc_begin;
+  } else {
+    range_max = -nc_begin < NC_cap ? -nc_begin : NC_cap;
+  }
+  if (range_max <= 0) return LSA_OK;
+  return cuda_status(lsa::launch_nsa_compress(k, v, B, Hkv, T_cap, D, seqlens, len, stride,
+                                              nc_begin, nc_end, range_max, kc, vc, stream));
+}
+
+int lsa_nsa_branches(const void* q, const void* k, const void* v, const void* kc, const void* vc,
+                     int dtype, int B, int Hkv, int G, int D, int T_cap, const int32_t* seqlens,
+                     int window, int stride, float scale, float g_cmp, float g_slc, float g_win,
+                     const void* o_slc, void* o, float* lse_win, float* lse_cmp,
+                     cudaStream_t stream) {
+  int st = check_common(dtype, B, Hkv, G, D, 64);
+  if (st != LSA_OK) return st;
+  if (dtype != LSA_BF16) return LSA_ERR_UNSUPPORTED;
+  if (T_cap < 0 || window < 0 || stride < 1) return LSA_ERR_INVALID_ARG;
+  if (!(g_cmp == g_cmp) || !(g_slc == g_slc) || !(g_win == g_win)) return LSA_ERR_INVALID_ARG;
+  if (T_cap > kMaxTcap || B > 65535 || Hkv > 65535) return LSA_ERR_UNSUPPORTED;
+  if (B == 0 || Hkv == 0) return LSA_OK;
+  if (!q || !k || !v || !kc || !vc || !seqlens || !o) return LSA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(kc) || !aligned16(vc) ||
+      !aligned16(o))
+    return LSA_ERR_INVALID_ARG;
+  lsa::NsaBranchArgs a = {};
+  a.q = q; a.k = k; a.v = v; a.kc = kc; a.vc = vc;
+  a.B = B; a.Hkv = Hkv; a.G = G; a.D = D; a.T_cap = T_cap;
+  a.seqlens = seqlens; a.window = window; a.stride = stride;
+  a.scale = resolve_scale(scale, D);
+  a.g_cmp = g_cmp; a.g_slc = g_slc; a.g_win = g_win;
+  a.o_slc = o_slc; a.o = o; a.lse_win = lse_win; a.lse_cmp = lse_cmp;
+  return cuda_status(lsa::launch_nsa_branches(a, stream));
+}
+
 size_t lsa_blockquery_workspace_size(int B, int Hkv, int G, int D, int Tq) {
   if (B <= 0 || Hkv <= 0 || G <= 0 || D <= 0 || Tq <= 0) return 0;
   return lsa::blockquery_workspace_bytes(B, Hkv, G, D, Tq);

@@ -80,6 +80,27 @@ struct DecodeBlasstArgs {
 };
 cudaError_t launch_decode_blasst(const DecodeBlasstArgs& a, cudaStream_t stream);
 
+// NSA's compressed and sliding-window branches (fixed pool, constant gates).
+cudaError_t launch_nsa_compress(const void* k, const void* v, int B, int Hkv, int T_cap, int D,
+                                const int32_t* seqlens, int len, int stride, int nc_begin,
+                                int nc_end, int range_max, void* kc, void* vc, cudaStream_t stream);
+struct NsaBranchArgs {
+  const void* q;
+  const void* k;
+  const void* v;
+  const void* kc;
+  const void* vc;
+  int B, Hkv, G, D, T_cap;
+  const int32_t* seqlens;
+  int window, stride;
+  float scale, g_cmp, g_slc, g_win;
+  const void* o_slc;
+  void* o;
+  float* lse_win;
+  float* lse_cmp;
+};
+cudaError_t launch_nsa_branches(const NsaBranchArgs& a, cudaStream_t stream);
+
 // LoSA: token activity and the attention inside the query block merged with the prefix.
 cudaError_t launch_losa_classify(const void* q, const void* q_prev, int B, int Hq, int Tq, int D,
                                  double tau, int n_top, uint8_t* active, double* mse,
