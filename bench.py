@@ -3,7 +3,7 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--workload gqa_decode_64k|batched_decode|tiny_decode|blockquery|
-                                losa_step|decode_blasst|blasst_prefill_32k]
+                                losa_step|decode_blasst|nsa_decode|blasst_prefill_32k]
 
 Default workload: 64K-context GQA decode, bf16 (1 sequence, 8 KV heads x 8 query heads,
 head dim 128, 65,536 cached tokens = 1,024 blocks of 64, top-16 blocks per KV head with
@@ -67,7 +67,7 @@ def parse():
     ap.add_argument("--warmup", type=int, default=None)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=sorted(WORKLOADS) + ["blockquery", "blasst_prefill_32k", "losa_step",
-                                                          "decode_blasst"],
+                                                          "decode_blasst", "nsa_decode"],
                     default="gqa_decode_64k")
     ap.add_argument("--prefill-sink", type=float, default=0.0,
                     help="blasst_prefill_32k: plant an attention sink of this logit height")
@@ -86,7 +86,8 @@ def parse():
                     help="a few launches on 2 input copies, for ncu captures")
     a = ap.parse_args()
     defaults = {"blockquery": (20000, 200), "blasst_prefill_32k": (20, 3),
-                "losa_step": (8000, 200), "decode_blasst": (80000, 600)}.get(a.workload, (200000, 600))
+                "losa_step": (8000, 200), "decode_blasst": (80000, 600),
+                "nsa_decode": (20000, 200)}.get(a.workload, (200000, 600))
     if a.steps is None:
         a.steps = defaults[0]
     if a.warmup is None:
@@ -980,14 +981,127 @@ def run_decode_blasst(args):
     }
 
 
+def run_nsa_decode(args):
+    """NSA's three branches for a 64K GQA decode step (the fixed-part variant): the fused
+    selected-branch decode (summary refresh, selection, sparse attention), the refresh of
+    the 2 compressed tokens the newest token changes (mean pool, block 32, stride 16) and
+    one launch for the compressed (4,096 tokens) and window (512 tokens) branches joined
+    with the selected one by gates of 1/3.  A step is three launches; R rotated input
+    copies exceed 4x L2; graph replays timed with CUDA events."""
+    import query_aware_block_b200 as lsa
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    wl = "gqa_decode_64k"
+    base = make_case(wl, rank_seed(0), dev)
+    B, Hkv, G, D, T_cap = base.shape
+    Hq = Hkv * G
+    stride, length, window = 16, 32, 512
+    NC_cap = -(-T_cap // stride)
+    dec_bytes, _ = algorithmic_bytes(base)
+    T = int(base.seqlens[0])
+    nc = -(-T // stride)
+    nsa_bytes = (B * Hkv * (min(window, T) + nc) * D * 2 * 2             # window + compressed K/V
+                 + B * Hkv * (length + stride) * D * 2 * 2                 # pool refresh reads
+                 + B * Hkv * 2 * D * 2 * 2                                 # pool refresh writes
+                 + B * Hq * D * 2 * 3)                                     # q, o_slc, o
+    step_bytes = dec_bytes + nsa_bytes
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    R = 2 if args.profile_small else max(4, min(64, math.ceil(4 * l2 / step_bytes)))
+    copies = []
+    for r in range(R):
+        c = base if r == 0 else make_case(wl, rank_seed(0, r), dev)
+        q, k, v, sl = (t.to(dev) for t in (c.q, c.k, c.v, c.seqlens))
+        summ = torch.zeros(B, Hkv, -(-T_cap // 64), D, device=dev)
+        lsa.lsa_build_summaries(k, sl, summ)
+        kc = torch.empty(B, Hkv, NC_cap, D, dtype=torch.bfloat16, device=dev)
+        vc = torch.empty_like(kc)
+        lsa.lsa_nsa_compress(k, v, sl, kc, vc, length=length, stride=stride)
+        copies.append(dict(q=q, k=k, v=v, sl=sl, summ=summ, kc=kc, vc=vc,
+                           o_slc=torch.empty(B, Hq, D, dtype=torch.bfloat16, device=dev),
+                           o=torch.empty(B, Hq, D, dtype=torch.bfloat16, device=dev),
+                           idx=torch.empty(B, Hkv, base.topk, dtype=torch.int32, device=dev)))
+        del c
+    torch.cuda.synchronize()
+
+    def selected(c):
+        lsa.lsa_sparse_attn_decode(c["q"], c["k"], c["v"], c["sl"], c["o_slc"], base.topk, summ=c["summ"],
+                                   n_sink=base.n_sink, n_local=base.n_local, refresh_last_summary=True,
+                                   idx_out=c["idx"])
+
+    def pool(c):
+        lsa.lsa_nsa_compress(c["k"], c["v"], c["sl"], c["kc"], c["vc"], length=length, stride=stride,
+                             nc_begin=-2)
+
+    def branches(c):
+        lsa.lsa_nsa_branches(c["q"], c["k"], c["v"], c["kc"], c["vc"], c["sl"], c["o"], o_slc=c["o_slc"],
+                             window=window, stride=stride)
+
+    def one(c):
+        selected(c)
+        pool(c)
+        branches(c)
+
+    for i in range(max(3, min(args.warmup, 2 * R))):
+        one(copies[i % R])
+    torch.cuda.synchronize()
+
+    def graph_of(fn):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for c in copies:
+                fn(c)
+        return g
+
+    def time_graph(g, reps):
+        for _ in range(max(1, args.warmup // R)):
+            g.replay()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(reps):
+            g.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / (reps * R)
+
+    reps = max(1, (args.steps or 20000) // R)
+    g_step = graph_of(one)
+    with ClockSampler(0) as clocks:
+        ms = time_graph(g_step, reps)
+    parts = {name: round(time_graph(graph_of(fn), max(1, reps // 4)) * 1e3, 2)
+             for name, fn in (("selected_decode", selected), ("pool_refresh", pool), ("branches", branches))}
+    gbs = step_bytes / (ms * 1e-3) / 1e9
+    peak, kind = measured_peaks()
+    return {
+        "metric": "NSA decode step, fixed parts (selected + compressed + window branches): tokens/s and "
+                  "effective GB/s",
+        "value": round(B / (ms * 1e-3), 1), "unit": "tokens/s", "n_gpus": 1, "steps": reps * R,
+        "warmup": args.warmup, "ms_per_step": round(ms, 6), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic 64K GQA decode inputs (seeded, needles)",
+        "config": {"workload": "nsa_decode", "batch": B, "kv_heads": Hkv, "q_heads_per_kv": G,
+                   "head_dim": D, "context": T_cap, "topk": base.topk, "compress": [length, stride],
+                   "window": window, "gates": [1 / 3, 1 / 3, 1 / 3],
+                   "l2": f"rotating {R} input copies ({R * step_bytes / 1e6:.0f} MB per cycle)"},
+        "tokens_read_per_kv_head": nc + base.topk * 64 + min(window, T),
+        "bytes_per_step": int(step_bytes), "effective_gbs": round(gbs, 1),
+        "kernel_us_alone": parts,
+        "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peak, "unit": "GB/s",
+                     "frac": round(gbs / peak, 4), "traffic": None, "kernel": "whole step (3 launches)",
+                     "peak_source": f"MEASURED_PEAKS.json hbm_gbs ({kind})"},
+        "gpu_launches": 3 * reps * R,
+        "clocks": clocks.summary(),
+    }
+
+
 def main():
     args = parse()
-    if args.workload in ("blockquery", "blasst_prefill_32k", "losa_step", "decode_blasst"):
+    if args.workload in ("blockquery", "blasst_prefill_32k", "losa_step", "decode_blasst", "nsa_decode"):
         if args.impl == "reference":
             print(json.dumps({"impl": "reference", "unavailable": "the oracle arm covers the decode workloads"}))
             return
         res = {"blockquery": run_blockquery, "blasst_prefill_32k": run_prefill,
-               "losa_step": run_losa_step, "decode_blasst": run_decode_blasst}[args.workload](args)
+               "losa_step": run_losa_step, "decode_blasst": run_decode_blasst,
+               "nsa_decode": run_nsa_decode}[args.workload](args)
         print(json.dumps(res), flush=True)
         return
     world = int(os.environ.get("WORLD_SIZE", "1"))

@@ -135,6 +135,34 @@ def test_decode_blasst_validation():
     assert f(g, g, g, 1, 0, 8, 8, 128, 65536, NULL, 64, NULL, NULL, 16, 0.0, 1e-3, NULL, NULL, NULL, NULL) == lsa.LSA_OK
 
 
+def test_nsa_entry_points_validation():
+    import query_aware_block_b200 as lsa
+    lib = lsa.library()
+    g = ctypes.c_void_p(4096)
+    cmp_ = lib.lsa_nsa_compress
+    assert cmp_(g, g, 0, 1, 8, 65536, 128, g, 32, 16, 0, -1, g, g, NULL) == lsa.LSA_ERR_UNSUPPORTED  # fp32
+    assert cmp_(g, g, 1, 1, 8, 65536, 96, g, 32, 16, 0, -1, g, g, NULL) == lsa.LSA_ERR_UNSUPPORTED  # D
+    assert cmp_(g, g, 1, 1, 8, 65536, 128, g, 0, 16, 0, -1, g, g, NULL) == lsa.LSA_ERR_INVALID_ARG  # len
+    assert cmp_(g, g, 1, 1, 8, 65536, 128, g, 32, 0, 0, -1, g, g, NULL) == lsa.LSA_ERR_INVALID_ARG  # stride
+    assert cmp_(g, g, 1, 1, 8, 65536, 128, g, 32, 16, 0, -1, NULL, g, NULL) == lsa.LSA_ERR_INVALID_ARG
+    assert cmp_(g, g, 1, 1, 8, 65536, 128, g, 32, 16, 5000, 4000, g, g, NULL) == lsa.LSA_OK  # empty range
+    assert cmp_(g, g, 1, 0, 8, 65536, 128, NULL, 32, 16, 0, -1, NULL, NULL, NULL) == lsa.LSA_OK
+    br = lib.lsa_nsa_branches
+    args = lambda **kw: [kw.get(n, d) for n, d in (
+        ("q", g), ("k", g), ("v", g), ("kc", g), ("vc", g), ("dtype", 1), ("B", 1), ("Hkv", 8),
+        ("G", 8), ("D", 128), ("T_cap", 65536), ("sl", g), ("window", 512), ("stride", 16),
+        ("scale", 0.0), ("gc", 1 / 3), ("gs", 1 / 3), ("gw", 1 / 3), ("oslc", NULL), ("o", g),
+        ("lw", NULL), ("lc", NULL), ("stream", NULL))]
+    assert br(*args(dtype=0)) == lsa.LSA_ERR_UNSUPPORTED
+    assert br(*args(G=17)) == lsa.LSA_ERR_UNSUPPORTED
+    assert br(*args(window=-1)) == lsa.LSA_ERR_INVALID_ARG
+    assert br(*args(stride=0)) == lsa.LSA_ERR_INVALID_ARG
+    assert br(*args(gc=float("nan"))) == lsa.LSA_ERR_INVALID_ARG
+    assert br(*args(kc=NULL)) == lsa.LSA_ERR_INVALID_ARG
+    assert br(*args(o=ctypes.c_void_p(4100))) == lsa.LSA_ERR_INVALID_ARG
+    assert br(*args(B=0, q=NULL, o=NULL)) == lsa.LSA_OK
+
+
 def test_binding_raises_lsa_error_on_bad_arguments():
     import torch
     import query_aware_block_b200 as lsa
