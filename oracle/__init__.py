@@ -9,7 +9,8 @@ the CUDA library in ``query_aware_block_b200``.
 Parity status of each function (what pins it is in tests/test_oracle_pins.py):
   summaries, block_scores, select, decode_attn, blockquery_select, blockquery_attn,
   blasst_prefill, decode_blasst, losa_classify, blockquery_intra_merge (and the losa_step
-  composition), nsa_compress, range_attn_f64, window_attn (and the nsa_decode composition)
+  composition), nsa_compress, range_attn_f64, window_attn (and the nsa_decode composition),
+  block_scores_weighted with the FASA / Prism weight builders
   -- all pinned (textbook special cases, brute force, library routines, closed forms and
   invariants).
 """
@@ -389,3 +390,61 @@ def nsa_decode(q, k, v, seqlens, topk=16, n_sink=1, n_local=2, gates=(1 / 3, 1 /
                   window=[min(window, int(t)) for t in sl])
     return dict(o=o, o_cmp=o_cmp, lse_cmp=lse_cmp, o_slc=o_slc, lse_slc=lse_slc, o_win=o_win,
                 lse_win=lse_win, idx=idx, nsel=nsel, kc=kc, vc=vc, tokens=tokens)
+
+
+def block_scores_weighted(q, summ, seqlens, w, blk=64, scale=None):
+    """Group block scores with per-dimension weights w [D]:
+    s[b,g,j] = scale * sum_{h in g} sum_d w_d q[b,h,d] summ[b,g,j,d]."""
+    q = q.contiguous()
+    summ = summ.to(torch.float64).contiguous()
+    w = torch.as_tensor(w, dtype=torch.float64).contiguous()
+    B, Hq, D = q.shape
+    _, Hkv, NB_cap, _ = summ.shape
+    assert w.shape == (D,)
+    out = torch.empty(B, Hkv, NB_cap, dtype=torch.float64)
+    _load().oracle_block_scores_weighted(_p(q), _dt(q), _p(summ), _p(w), B, Hkv, Hq // Hkv, D,
+                                         NB_cap, _p(_i32(seqlens)), blk,
+                                         ctypes.c_double(_scale(scale, D)), _p(out))
+    return out
+
+
+def rope_chunk_of_dim(D):
+    """Rotary frequency chunk of every head dimension under rotate-half pairing: dims j and
+    j + D/2 form chunk j, rotated at frequency theta^(-2j/D)."""
+    return torch.cat([torch.arange(D // 2), torch.arange(D // 2)])
+
+
+def rope_block_attenuation(D, theta=1e4, blk=64):
+    """Magnitude left of a unit vector of rotary chunk j after mean pooling over blk
+    consecutive positions: |sin(blk * w_j / 2) / (blk * sin(w_j / 2))|, w_j = theta^(-2j/D)
+    (the Dirichlet kernel: a constant vector rotating at w_j averaged over blk positions).
+    Returns a [D/2] fp64 tensor (1 for a chunk that does not rotate)."""
+    j = torch.arange(D // 2, dtype=torch.float64)
+    wj = theta ** (-2.0 * j / D)
+    half = torch.sin(wj / 2)
+    a = torch.abs(torch.sin(blk * wj / 2) / (blk * half))
+    return torch.where(half.abs() < 1e-300, torch.ones_like(a), a)
+
+
+def fasa_weights(D, chunks):
+    """0/1 weight per dimension keeping the given rotary chunks (both dims of each)."""
+    keep = set(int(c) for c in chunks)
+    return torch.tensor([1.0 if int(c) in keep else 0.0 for c in rope_chunk_of_dim(D)],
+                        dtype=torch.float64)
+
+
+def prism_weights(D, theta=1e4, blk=64):
+    """Dual-band weights: the high band holds the chunks that turn by more than a full
+    period inside one block (w_j > 2 pi / blk: mean pooling cancels them), the low band the
+    rest; each band's temperature is the mean attenuation of its chunks under the pool
+    (rope_block_attenuation), and every dim of a band is weighted by 1 / temperature, which
+    restores the band's pooled magnitude.  Returns (w [D], high-band chunk mask [D/2],
+    (tau_high, tau_low))."""
+    j = torch.arange(D // 2, dtype=torch.float64)
+    wj = theta ** (-2.0 * j / D)
+    high = wj > 2 * math.pi / blk
+    a = rope_block_attenuation(D, theta, blk)
+    tau_hi = float(a[high].mean()) if bool(high.any()) else 1.0
+    tau_lo = float(a[~high].mean()) if bool((~high).any()) else 1.0
+    per_chunk = torch.where(high, torch.full_like(a, 1 / tau_hi), torch.full_like(a, 1 / tau_lo))
+    return per_chunk[rope_chunk_of_dim(D)], high, (tau_hi, tau_lo)

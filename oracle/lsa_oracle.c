@@ -42,6 +42,12 @@
  *                            tokens [NSA news article, "NSA 구조": three parallel paths --
  *                            compressed coarse tokens, selected fine tokens, a sliding
  *                            window -- with l = 32, d = 16, l' = 64, n = 16, w = 512]
+ *   oracle_block_scores_weighted
+ *                            the group block score with a weight per head dimension: a
+ *                            subset of rotary frequency chunks [FASA, "2. 방법론": token
+ *                            importance from the dominant frequency chunks only] or one
+ *                            temperature per frequency band [Prism, "3. 제안 방법론":
+ *                            dual-band block importance, energy-based temperature]
  *   oracle_losa_classify     active / stable tokens by the mean squared change of their
  *                            queries between denoising steps [LoSA, "2. 방법론": the query
  *                            change (MSE) of every step sorts tokens into active and stable]
@@ -847,6 +853,42 @@ void oracle_window_attn(const void* q, const void* k, const void* v, int dtype, 
       }
       free(logits);
       free(toks);
+    }
+  }
+}
+
+/* ------------------------------------------------------------------------------------
+ * Group block scores with a weight per head dimension (decode):
+ *   scores[b,g,j] = scale * sum_{h in g} sum_d w[d] * q[b,h,d] * summ[b,g,j,d]   (j < NB_b)
+ * A 0/1 weight keeps a subset of the rotary frequency chunks (FASA's scoring with its
+ * dominant chunks only); one weight per frequency band is Prism's per-band temperature
+ * (the reciprocal of the band's temperature).  w = 1 everywhere is oracle_block_scores.
+ * q [B,Hq,D]; summ [B,Hkv,NB_cap,D] double; w [D] double; scores [B,Hkv,NB_cap] (-inf past NB_b).
+ * ---------------------------------------------------------------------------------- */
+void oracle_block_scores_weighted(const void* q, int dtype, const double* summ, const double* w,
+                                  int B, int Hkv, int G, int D, int NB_cap,
+                                  const int32_t* seqlens, int blk, double scale, double* scores) {
+  const int Hq = Hkv * G;
+#pragma omp parallel for collapse(2) schedule(dynamic)
+  for (int b = 0; b < B; ++b) {
+    for (int g = 0; g < Hkv; ++g) {
+      const int NB = ceil_div(seqlens[b], blk);
+      for (int j = 0; j < NB_cap; ++j) {
+        double* out = scores + ((size_t)b * Hkv + g) * NB_cap + j;
+        if (j >= NB) {
+          *out = -INFINITY;
+          continue;
+        }
+        const double* kb = summ + (((size_t)b * Hkv + g) * NB_cap + j) * D;
+        double acc = 0.0;
+        for (int hh = 0; hh < G; ++hh) {
+          const size_t qrow = ((size_t)b * Hq + g * G + hh) * D;
+          double dot = 0.0;
+          for (int d = 0; d < D; ++d) dot += w[d] * elem(q, dtype, qrow + d) * kb[d];
+          acc += dot;
+        }
+        *out = scale * acc;
+      }
     }
   }
 }

@@ -805,3 +805,91 @@ def test_nsa_decode_combines_the_three_branches_and_reproduces_the_64k_accountin
     assert torch.allclose(r["o"], (r["o_cmp"] + r["o_slc"] + r["o_win"]) / 3, rtol=0, atol=1e-15)
     only = oracle.nsa_decode(case.q, case.k, case.v, case.seqlens, gates=(0.0, 1.0, 0.0), idx=r["idx"])
     assert torch.equal(only["o"], r["o_slc"])
+
+
+# ------------------------------------- weighted block scores (FASA / Prism-style scorers) ----
+
+def _scorer_case(seed=75):
+    case = synth.decode_case(2, 2, 3, 64, T_cap=640, seqlens=[640, 400], dtype=torch.bfloat16,
+                             topk=4, n_sink=1, n_local=2, seed=seed)
+    summ = oracle.summaries(case.k, case.seqlens)
+    return case, summ
+
+
+def test_weighted_scores_reduce_to_the_plain_score_and_are_linear_in_the_weights():
+    case, summ = _scorer_case()
+    D = 64
+    plain = oracle.block_scores(case.q, summ, case.seqlens)
+    assert torch.equal(oracle.block_scores_weighted(case.q, summ, case.seqlens, torch.ones(D)), plain)
+    g = torch.Generator().manual_seed(76)
+    w1 = torch.rand(D, generator=g, dtype=torch.float64)
+    w2 = torch.rand(D, generator=g, dtype=torch.float64)
+    s1 = oracle.block_scores_weighted(case.q, summ, case.seqlens, w1)
+    s2 = oracle.block_scores_weighted(case.q, summ, case.seqlens, w2)
+    s12 = oracle.block_scores_weighted(case.q, summ, case.seqlens, w1 + 3 * w2)
+    fin = torch.isfinite(s12)
+    assert torch.allclose(s12[fin], (s1 + 3 * s2)[fin], rtol=1e-12, atol=1e-12)
+    assert torch.equal(torch.isinf(s12), torch.isinf(plain))
+
+
+def test_fasa_weights_score_with_the_kept_chunks_only():
+    # library routine: einsum over the sliced dims of the kept rotary chunks
+    case, summ = _scorer_case()
+    D, G = 64, 3
+    chunks = [2, 5, 17, 30]
+    w = oracle.fasa_weights(D, chunks)
+    dims = [d for d in range(D) if int(oracle.rope_chunk_of_dim(D)[d]) in chunks]
+    assert dims == [2, 5, 17, 30, 34, 37, 49, 62] and int(w.sum()) == 8
+    s = oracle.block_scores_weighted(case.q, summ, case.seqlens, w)
+    for b, T in ((0, 640), (1, 400)):
+        NB = -(-T // 64)
+        for g in range(2):
+            qs = case.q[b, g * G:(g + 1) * G][:, dims].double().sum(0)
+            ref = (summ[b, g, :NB][:, dims] @ qs) / math.sqrt(D)
+            assert torch.allclose(s[b, g, :NB], ref, rtol=1e-12, atol=1e-12)
+
+
+def test_rope_attenuation_is_the_measured_magnitude_of_a_pooled_rotating_constant():
+    # pool a constant unit vector of chunk j rotated over 64 positions (the generator's
+    # rotary embedding, the oracle's block mean): what is left is the closed form
+    D = 32
+    a = oracle.rope_block_attenuation(D, 1e4, 64)
+    for j in (0, 1, 3, 7, 15):
+        c = torch.zeros(1, 1, 64, D, dtype=torch.float64)
+        c[..., j] = 1.0
+        k = synth.rope(c[0, 0], torch.arange(64), 1e4)[None, None].float()
+        kbar = oracle.summaries(k, torch.tensor([64]))[0, 0, 0]
+        mag = float(torch.hypot(kbar[j], kbar[j + D // 2]))
+        assert abs(mag - float(a[j])) < 2e-6, (j, mag, float(a[j]))   # fp32 keys
+
+
+def test_prism_weights_split_the_bands_at_one_rotation_per_block():
+    D, blk = 128, 64
+    w, high, (t_hi, t_lo) = oracle.prism_weights(D, 1e4, blk)
+    j = torch.arange(D // 2, dtype=torch.float64)
+    period = 2 * math.pi / (1e4 ** (-2 * j / D))
+    assert torch.equal(high, period < blk)
+    a = oracle.rope_block_attenuation(D, 1e4, blk)
+    assert abs(t_hi - float(a[high].mean())) < 1e-15 and abs(t_lo - float(a[~high].mean())) < 1e-15
+    chunk = oracle.rope_chunk_of_dim(D)
+    for d in range(D):
+        assert float(w[d]) == (1 / t_hi if bool(high[chunk[d]]) else 1 / t_lo)
+    assert t_hi < 0.1 < 0.9 < t_lo  # pooling erases the fast chunks, keeps the slow ones
+
+
+def test_fasa_weighted_selection_ignores_a_decoy_in_the_dropped_chunks():
+    # block 5's summary matches the query strongly in chunk 0 only, block 9's moderately in
+    # chunk 20 only: the plain score picks block 5, the score on chunk 20 picks block 9
+    D, NB = 64, 16
+    q = torch.zeros(1, 1, D)
+    q[0, 0, 0] = 1.0
+    q[0, 0, 20] = 1.0
+    summ = torch.zeros(1, 1, NB, D, dtype=torch.float64)
+    summ[0, 0, 5, 0] = 3.0
+    summ[0, 0, 9, 20] = 1.0
+    sl = torch.tensor([NB * 64])
+    plain = oracle.block_scores(q, summ, sl)
+    idx_plain, _ = oracle.select(plain, sl, 1, 0, 0)
+    ws = oracle.block_scores_weighted(q, summ, sl, oracle.fasa_weights(D, [20]))
+    idx_w, _ = oracle.select(ws, sl, 1, 0, 0)
+    assert idx_plain.tolist() == [[[5]]] and idx_w.tolist() == [[[9]]]
