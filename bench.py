@@ -141,8 +141,26 @@ def algorithmic_bytes(case):
     return dec, ref
 
 
+def _nvtx_push(name):
+    """An NVTX range around a timed region (seen by nsys or ncu --nvtx); no-op without NVTX."""
+    try:
+        torch.cuda.nvtx.range_push(name)
+        return True
+    except (RuntimeError, AttributeError):
+        return False
+
+
+def _nvtx_pop(pushed):
+    if pushed:
+        try:
+            torch.cuda.nvtx.range_pop()
+        except (RuntimeError, AttributeError):
+            pass
+
+
 class ClockSampler:
-    """nvidia-smi samples of the SM clock and throttle reasons during the timed region."""
+    """nvidia-smi samples of the SM clock and throttle reasons during the timed region, which
+    is also marked as an NVTX range ("timed region")."""
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
@@ -163,6 +181,7 @@ class ClockSampler:
         except OSError:
             self.proc = None
         time.sleep(0.3)
+        self.nvtx = _nvtx_push("timed region")
         return self
 
     def _read(self):
@@ -170,6 +189,7 @@ class ClockSampler:
             self.lines.append(line.strip())
 
     def __exit__(self, *a):
+        _nvtx_pop(self.nvtx)
         time.sleep(0.2)
         if self.proc:
             self.proc.terminate()
@@ -480,11 +500,13 @@ def run_e2e(args, lsa, copies, base, dev, topk, ns, nl, flags):
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     t0 = time.perf_counter()
+    nv = _nvtx_push("e2e timed region")
     e0.record()
     for i in range(n):
         one(i)
     e1.record()
     torch.cuda.synchronize()
+    _nvtx_pop(nv)
     wall = time.perf_counter() - t0
     ms = e0.elapsed_time(e1)
     return {"value": round(B * n / (ms / 1e3), 1), "unit": UNIT, "h2d_bytes_per_step": h2d,
