@@ -456,6 +456,22 @@ def test_blasst_constructed_negligible_tile_is_skipped():
     assert int(r2["bits"][0, 0]) == 0
 
 
+def test_blasst_skip_needs_every_row_negligible():
+    # the tile above, but row 100's query points the other way: tile 1 is that row's best
+    # tile (gap +8), so the tile is kept although every other row finds it negligible
+    D, L = 16, 128
+    q = torch.zeros(1, 1, L, D)
+    q[..., 0] = 4.0
+    q[0, 0, 100, 0] = -4.0
+    k = torch.zeros(1, 1, L, D)
+    k[0, 0, :64, 0] = 4.0
+    k[0, 0, 64:, 0] = -4.0
+    v = torch.randn(1, 1, L, D)
+    r = oracle.blasst_prefill(q, k, v, [(0, 0, 0)], 1e-3, scale=0.25)
+    assert int(r["bits"][0, 0]) == 0
+    assert abs(float(r["gap"][0, 1]) - 8.0) < 1e-12
+
+
 def test_blasst_forced_bits_follow_the_given_decisions():
     case = _sharp_case(L=256, seed=33)
     units = _all_units(1, 2, 256)
