@@ -10,6 +10,7 @@ import os
 import subprocess
 
 import pytest
+import torch
 
 import oracle
 from tests import test_oracle_pins as pins
@@ -71,6 +72,32 @@ MUTANTS = [
     ("weighted score ignores the weights",
      "dot += w[d] * elem(q, dtype, qrow + d) * kb[d];", "dot += elem(q, dtype, qrow + d) * kb[d];",
      pins.test_fasa_weights_score_with_the_kept_chunks_only),
+    ("local forced blocks shifted by one",
+     "for (int j = NB - n_local; j < NB; ++j)", "for (int j = NB - n_local - 1; j < NB - 1; ++j)",
+     functools.partial(pins.test_select_matches_brute_force, NB=10, k=4, ns=1, nl=2)),
+    ("decode reads the query of another head",
+     "const size_t qrow = ((size_t)b * Hq + h) * D;\n        attend_row(q, k, v, dtype, qrow, kvbase",
+     "const size_t qrow = ((size_t)b * Hq + hh * Hkv + g) * D;\n        attend_row(q, k, v, dtype, qrow, kvbase",
+     functools.partial(pins.test_decode_with_all_blocks_equals_dense, dtype=torch.float32)),
+    ("prefill forgets to rescale the running sum",
+     "        l[ii] *= alpha;\n", "",
+     functools.partial(pins.test_blasst_lambda_zero_is_dense_causal, L=300)),
+    ("stable rows attend instead of keeping the cache",
+     "if (active[(size_t)b * Tq + i]) {", "if (1) {",
+     pins.test_blockquery_all_stable_is_cache_bit_exact),
+    ("activity ties to the higher token index",
+     "(mj == mi && j < i)", "(mj == mi && j > i)",
+     pins.test_losa_classify_unchanged_queries),
+    ("attention inside the block made causal",
+     "attend_row(q, k, v, dtype, row * D, kvbase, D, toks, Tq, scale, logits, o_in, &lse_in);",
+     "attend_row(q, k, v, dtype, row * D, kvbase, D, toks, i + 1, scale, logits, o_in, &lse_in);",
+     pins.test_losa_step_all_blocks_equals_dense_attention_over_prefix_and_block),
+    ("compressed block as long as the stride",
+     "const int t1 = (t0 + len < T) ? t0 + len : T;", "const int t1 = (t0 + stride < T) ? t0 + stride : T;",
+     pins.test_nsa_compress_is_avg_pool_with_clipped_tail),
+    ("sparse-decode rescale factor inverted",
+     "exp(m[hh] - mn)", "exp(mn - m[hh])",
+     pins.test_decode_blasst_lambda_zero_is_masked_dense),
 ]
 
 
