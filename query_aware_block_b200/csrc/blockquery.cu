@@ -710,6 +710,9 @@ cudaError_t launch_blockquery(const BlockQueryArgs& a, cudaStream_t stream) {
   static int ok_cl128 = 0, ok_smem128 = 0, ok_cl64 = 0, ok_smem64 = 0;
   int& ok_cl = a.D == 128 ? ok_cl128 : ok_cl64;
   int& ok_smem = a.D == 128 ? ok_smem128 : ok_smem64;
+  // these per-process caches are shared by every host thread that launches: one lock
+  // covers them (and the attribute and occupancy calls they guard), not the launch
+  static std::mutex cache_mutex;
   for (;;) {
     p.per_max = (NBp + CL - 1) / CL;
     if (p.per_max < 1) p.per_max = 1;
@@ -718,6 +721,7 @@ cudaError_t launch_blockquery(const BlockQueryArgs& a, cudaStream_t stream) {
     const int smem = (int)Lo.total;
     if (smem > 227 * 1024) return cudaErrorInvalidValue;
     cudaError_t err;
+    std::unique_lock<std::mutex> lock(cache_mutex);
     if (smem > smem_set) {
       err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
       if (err != cudaSuccess) return err;
@@ -753,6 +757,7 @@ cudaError_t launch_blockquery(const BlockQueryArgs& a, cudaStream_t stream) {
       ok_cl = CL;
       ok_smem = smem;
     }
+    lock.unlock();
     cfg.numAttrs = 2;  // launched as a programmatic dependent of the previous kernel
     return cudaLaunchKernelEx(&cfg, kernel, p);
   }

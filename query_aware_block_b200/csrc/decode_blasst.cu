@@ -262,10 +262,6 @@ __global__ void __launch_bounds__(kThreads)
 template <int D>
 cudaError_t launch_d(const DecodeBlasstArgs& a, cudaStream_t stream) {
   auto kernel = decode_blasst_kernel<D>;
-  // the cluster attribute and the occupancy check are per process (the configuration is
-  // fixed): done once, so that a launch costs only the launch
-  static int checked = 0;  // 0 = not yet, 1 = schedulable, -1 = a cudaError_t was returned
-  static cudaError_t check_err = cudaSuccess;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(kCL, a.Hkv, a.B);
   cfg.blockDim = dim3(kThreads, 1, 1);
@@ -278,15 +274,17 @@ cudaError_t launch_d(const DecodeBlasstArgs& a, cudaStream_t stream) {
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (checked == 0) {
+  // the cluster attribute and the occupancy check depend only on the kernel and its fixed
+  // block shape: done once per process (a function-local static is initialised once, also
+  // when host threads race), so that a launch costs only the launch
+  static const cudaError_t check_err = [&]() {
     cudaError_t err = cudaFuncSetAttribute(kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
     int nclusters = 0;
     if (err == cudaSuccess) err = cudaOccupancyMaxActiveClusters(&nclusters, kernel, &cfg);
     if (err == cudaSuccess && nclusters == 0) err = cudaErrorInvalidConfiguration;
-    check_err = err;
-    checked = err == cudaSuccess ? 1 : -1;
-  }
-  if (checked < 0) return check_err;
+    return err;
+  }();
+  if (check_err != cudaSuccess) return check_err;
   const float scale2 = a.scale * kLog2e;
   const float log2_lambda = a.lambda > 0.f ? log2f(a.lambda) : -INFINITY;
   return cudaLaunchKernelEx(&cfg, kernel, static_cast<const __nv_bfloat16*>(a.q),

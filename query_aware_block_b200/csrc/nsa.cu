@@ -315,8 +315,6 @@ template <int D>
 cudaError_t launch_branches(const NsaBranchArgs& a, cudaStream_t stream) {
   auto kernel = nsa_branches_kernel<D>;
   const int smem = (int)sizeof(BranchSmem<D>);
-  static int checked = 0;  // the attributes and the occupancy check, once per process
-  static cudaError_t check_err = cudaSuccess;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(kCL, a.Hkv, a.B);
   cfg.blockDim = dim3(kThreads, 1, 1);
@@ -329,16 +327,18 @@ cudaError_t launch_branches(const NsaBranchArgs& a, cudaStream_t stream) {
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (checked == 0) {
+  // the attributes and the occupancy check depend only on the kernel and its fixed block
+  // shape: done once per process (a function-local static is initialised once, also when
+  // host threads race)
+  static const cudaError_t check_err = [&]() {
     cudaError_t err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (err == cudaSuccess) err = cudaFuncSetAttribute(kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
     int nclusters = 0;
     if (err == cudaSuccess) err = cudaOccupancyMaxActiveClusters(&nclusters, kernel, &cfg);
     if (err == cudaSuccess && nclusters == 0) err = cudaErrorInvalidConfiguration;
-    check_err = err;
-    checked = err == cudaSuccess ? 1 : -1;
-  }
-  if (checked < 0) return check_err;
+    return err;
+  }();
+  if (check_err != cudaSuccess) return check_err;
   BranchParams p;
   p.q = static_cast<const __nv_bfloat16*>(a.q);
   p.k = static_cast<const __nv_bfloat16*>(a.k);
