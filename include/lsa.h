@@ -251,6 +251,30 @@ LSA_API int lsa_sparse_attn_blockquery_noalloc(const void* q, const void* k, con
                                                cudaStream_t stream);
 
 /*
+ * lsa_select_blocks_weighted -- lsa_select_blocks with a weight per head dimension in the
+ * group score (FASA- and Prism-style scorers).
+ *
+ * Defined by: FASA, "2. 방법론" (token importance estimated from the dominant rotary
+ * frequency chunks only) and Prism, "3. 제안 방법론" (block importance per frequency band,
+ * each band with its own temperature that restores what mean pooling attenuates).
+ *
+ *   s[b, g, j] = scale * sum_{h in g} sum_d dim_weights[d] * q[b, h, d] * summ[b, g, j, d]
+ * then the selection of lsa_select_blocks.  A 0/1 weight keeps a subset of the rotary
+ * chunks (dims j and j + D/2 form chunk j under rotate-half pairing); one weight per band,
+ * 1 / temperature, gives the dual-band score.  Choosing the chunks or temperatures is the
+ * caller's.  The reweighted queries w * q are formed in fp32 in q_weighted (scratch,
+ * [B, Hq, D] float32, 16-byte aligned; it may be q itself when q is float32) and scored by
+ * the selection kernel.  dim_weights: [D] float32, device.  Other arguments and outputs as
+ * lsa_select_blocks (scores_out holds the weighted scores).
+ */
+LSA_API int lsa_select_blocks_weighted(const void* q, int dtype, const float* summ,
+                                       const float* dim_weights, int B, int Hkv, int G, int D,
+                                       int NB_cap, const int32_t* seqlens, int blk, int topk,
+                                       int n_sink, int n_local, float scale, float* q_weighted,
+                                       int32_t* idx, int32_t* nsel, float* scores_out,
+                                       cudaStream_t stream);
+
+/*
  * lsa_sparse_attn_decode_blasst -- sparse decode attention over a given block selection
  * that drops, before reading their V, the selected blocks whose softmax weight is
  * negligible (BLASST inside sparse decode).

@@ -31,7 +31,7 @@ EXPORTED = ("lsa_status_string", "lsa_last_cuda_error", "lsa_version", "lsa_buil
             "lsa_sparse_attn_blockquery", "lsa_sparse_attn_blockquery_noalloc",
             "lsa_blasst_prefill", "lsa_device_status", "lsa_losa_classify",
             "lsa_blockquery_intra_merge", "lsa_sparse_attn_decode_blasst", "lsa_nsa_compress",
-            "lsa_nsa_branches")
+            "lsa_nsa_branches", "lsa_select_blocks_weighted")
 
 _vp, _i, _f = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
 _lib.lsa_status_string.restype = ctypes.c_char_p
@@ -58,6 +58,8 @@ _lib.lsa_blasst_prefill.argtypes = [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _
 _lib.lsa_device_status.argtypes = [_vp, _i]
 _lib.lsa_sparse_attn_decode_blasst.argtypes = [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp, _i,
                                                _vp, _vp, _i, _f, _f, _vp, _vp, _vp, _vp]
+_lib.lsa_select_blocks_weighted.argtypes = [_vp, _i, _vp, _vp, _i, _i, _i, _i, _i, _vp, _i, _i, _i,
+                                            _i, _f, _vp, _vp, _vp, _vp, _vp]
 _lib.lsa_nsa_compress.argtypes = [_vp, _vp, _i, _i, _i, _i, _i, _vp, _i, _i, _i, _i, _vp, _vp, _vp]
 _lib.lsa_nsa_branches.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp, _i, _i, _f,
                                   _f, _f, _f, _vp, _vp, _vp, _vp, _vp]
@@ -182,6 +184,23 @@ def lsa_blasst_prefill(q, k, v, o, lam, lse=None, skip_bits=None, skipped_tiles=
                                    _ptr(skipped_tiles), _stream(stream)),
            "lsa_blasst_prefill")
     return o
+
+
+def lsa_select_blocks_weighted(q, summ, seqlens, dim_weights, topk, n_sink, n_local, idx, nsel,
+                               q_weighted=None, scale=0.0, scores_out=None, blk=BLK, stream=None):
+    """Block selection with a weight per head dimension (FASA / Prism-style scorers):
+    dim_weights [D] float32 on the device; q_weighted: float32 [B,Hq,D] scratch (allocated
+    here when not given)."""
+    B, Hq, D = q.shape
+    _, Hkv, NB_cap, _ = summ.shape
+    if q_weighted is None:
+        q_weighted = torch.empty(B, Hq, D, dtype=torch.float32, device=q.device)
+    _check(_lib.lsa_select_blocks_weighted(_ptr(q), _dtype(q), _ptr(summ), _ptr(dim_weights), B, Hkv,
+                                           Hq // Hkv, D, NB_cap, _ptr(seqlens), blk, topk, n_sink,
+                                           n_local, float(scale), _ptr(q_weighted), _ptr(idx),
+                                           _ptr(nsel), _ptr(scores_out), _stream(stream)),
+           "lsa_select_blocks_weighted")
+    return idx, nsel
 
 
 def lsa_sparse_attn_decode_blasst(q, k, v, seqlens, idx, nsel, o, lam, lse=None, skip_bits=None,

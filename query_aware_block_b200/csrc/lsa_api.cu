@@ -99,6 +99,33 @@ int lsa_select_blocks(const void* q, int dtype, const float* summ, int B, int Hk
   return cuda_status(lsa::launch_decode(a, stream));
 }
 
+int lsa_select_blocks_weighted(const void* q, int dtype, const float* summ,
+                               const float* dim_weights, int B, int Hkv, int G, int D, int NB_cap,
+                               const int32_t* seqlens, int blk, int topk, int n_sink,
+                               int n_local, float scale, float* q_weighted, int32_t* idx,
+                               int32_t* nsel, float* scores_out, cudaStream_t stream) {
+  int st = check_common(dtype, B, Hkv, G, D, blk);
+  if (st != LSA_OK) return st;
+  if (topk < 1 || topk > 64 || n_sink < 0 || n_local < 0 || n_sink + n_local > topk)
+    return LSA_ERR_INVALID_ARG;
+  if (NB_cap < 0) return LSA_ERR_INVALID_ARG;
+  if (NB_cap > kMaxTcap / 64) return LSA_ERR_UNSUPPORTED;
+  if (B == 0 || Hkv == 0) return LSA_OK;
+  if (!q || !summ || !dim_weights || !seqlens || !q_weighted || !idx || !nsel)
+    return LSA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(summ) || !aligned16(q_weighted)) return LSA_ERR_INVALID_ARG;
+  cudaError_t err = lsa::launch_weight_queries(q, dtype, dim_weights, B, Hkv * G, D, q_weighted, stream);
+  if (err != cudaSuccess) return cuda_status(err);
+  lsa::DecodeArgs a = {};
+  a.q = q_weighted; a.dtype = LSA_F32; a.summ = summ;
+  a.B = B; a.Hkv = Hkv; a.G = G; a.D = D; a.T_cap = NB_cap * blk; a.NB_cap = NB_cap;
+  a.seqlens = seqlens; a.topk = topk; a.n_sink = n_sink; a.n_local = n_local;
+  a.scale = resolve_scale(scale, D);
+  a.idx_out = idx; a.nsel_out = nsel; a.scores_out = scores_out;
+  a.mode = lsa::MODE_SELECT;
+  return cuda_status(lsa::launch_decode(a, stream));
+}
+
 int lsa_sparse_attn_decode(const void* q, const void* k, const void* v, int dtype, int B,
                            int Hkv, int G, int D, int T_cap, const int32_t* seqlens,
                            int blk, const int32_t* idx, const int32_t* nsel, int topk,

@@ -63,6 +63,10 @@ struct BlockQueryArgs {
 size_t blockquery_workspace_bytes(int B, int Hkv, int G, int D, int Tq);
 cudaError_t launch_blockquery(const BlockQueryArgs& a, cudaStream_t stream);
 
+// Queries reweighted per head dimension (fp32 out) for the weighted block selection.
+cudaError_t launch_weight_queries(const void* q, int dtype, const float* w, int B, int Hq, int D,
+                                  float* out, cudaStream_t stream);
+
 // Sparse decode over a given selection with BLASST's skip (V not read for negligible blocks).
 struct DecodeBlasstArgs {
   const void* q;

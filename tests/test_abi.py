@@ -163,6 +163,24 @@ def test_nsa_entry_points_validation():
     assert br(*args(B=0, q=NULL, o=NULL)) == lsa.LSA_OK
 
 
+def test_weighted_select_validation():
+    import query_aware_block_b200 as lsa
+    f = lsa.library().lsa_select_blocks_weighted
+    g = ctypes.c_void_p(4096)
+    args = lambda **kw: [kw.get(n, d) for n, d in (
+        ("q", g), ("dtype", 1), ("summ", g), ("w", g), ("B", 1), ("Hkv", 8), ("G", 8), ("D", 128),
+        ("NB", 1024), ("sl", g), ("blk", 64), ("topk", 16), ("ns", 1), ("nl", 2), ("scale", 0.0),
+        ("qw", g), ("idx", g), ("nsel", g), ("sc", NULL), ("stream", NULL))]
+    assert f(*args(w=NULL)) == lsa.LSA_ERR_INVALID_ARG
+    assert f(*args(qw=NULL)) == lsa.LSA_ERR_INVALID_ARG
+    assert f(*args(qw=ctypes.c_void_p(4100))) == lsa.LSA_ERR_INVALID_ARG
+    assert f(*args(topk=0)) == lsa.LSA_ERR_INVALID_ARG
+    assert f(*args(ns=10, nl=10)) == lsa.LSA_ERR_INVALID_ARG
+    assert f(*args(D=96)) == lsa.LSA_ERR_UNSUPPORTED
+    assert f(*args(blk=32)) == lsa.LSA_ERR_UNSUPPORTED
+    assert f(*args(B=0, q=NULL, w=NULL, qw=NULL)) == lsa.LSA_OK
+
+
 def test_binding_raises_lsa_error_on_bad_arguments():
     import torch
     import query_aware_block_b200 as lsa
