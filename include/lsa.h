@@ -17,6 +17,14 @@
  * The first step of a block passes topk_per_query >= ceil(T_prefix / blk) and an all-ones
  * mask (dense prefix attention, which fills the cache).
  *
+ * One NSA decode step with fixed parts is three calls on one stream:
+ *   lsa_sparse_attn_decode      (the selected branch, fused selection)
+ *   lsa_nsa_compress            (nc_begin = -2: the compressed tokens the new token changes)
+ *   lsa_nsa_branches            (compressed and window branches, gated sum with the above)
+ * Variants: lsa_select_blocks_weighted scores with a weight per head dimension (FASA /
+ * Prism-style scorers); lsa_sparse_attn_decode_blasst drops, before reading their V, the
+ * selected blocks whose softmax weight is negligible (BLASST inside sparse decode).
+ *
  * Conventions shared by every entry point
  * ---------------------------------------
  * Memory.   Every tensor argument is a raw DEVICE pointer to a contiguous row-major array
