@@ -17,6 +17,9 @@ Recipes (the shapes are those of the five workloads the pages motivate):
   every key of a needle block is sqrt(D) * u_g + 0.5 * N(0, I) (so |key| ~ |N(0,1) key|);
   needle blocks are distinct, uniform over the non-forced blocks, independent per (b, g);
   they are planted after the rotation; v is left N(0, 1);
+* LoSA steps: the previous step's queries are the current ones plus 0.02 * N(0, I) for a
+  stable token and a fresh rotated N(0, 1) draw for an active one; the block's own keys
+  and values sit at cache rows T_prefix .. T_prefix + Tq - 1;
 * the result is rounded once (round-to-nearest-even) to the case dtype;
 * optional poison: cache positions at or beyond a sequence's length are filled with NaN,
   so that any kernel that lets them into a result is caught.

@@ -909,3 +909,15 @@ def test_fasa_weighted_selection_ignores_a_decoy_in_the_dropped_chunks():
     ws = oracle.block_scores_weighted(q, summ, sl, oracle.fasa_weights(D, [20]))
     idx_w, _ = oracle.select(ws, sl, 1, 0, 0)
     assert idx_plain.tolist() == [[[5]]] and idx_w.tolist() == [[[9]]]
+
+
+def test_losa_generator_plants_what_the_classification_finds():
+    # the synthetic previous queries separate the planted active tokens by a wide margin:
+    # both rules of the oracle recover them (stable change ~4e-4, active ~2 per element)
+    case = synth.losa_case(B=2, Hkv=2, G=4, D=64, Tq=32, T_prefix=128, n_active=8, topk=2, seed=46)
+    mse, act = oracle.losa_classify(case.q, case.q_prev, tau=0.1)
+    assert torch.equal(act, case.active)
+    _, act = oracle.losa_classify(case.q, case.q_prev, n_top=8)
+    assert torch.equal(act, case.active)
+    on = case.active.bool()
+    assert float(mse[~on].max()) < 1e-3 < 1.0 < float(mse[on].min())
