@@ -57,7 +57,7 @@
  *                            tokens reuse the prefix statistics and output; the block
  *                            itself is attended every step]
  *
- * Readings taken where the pages are silent (each also listed in the design doc):
+ * Readings taken where the pages are silent (the CUDA library takes the same ones):
  *   - a partial last block is averaged over its valid tokens only;
  *   - the GQA group score is the sum over the group's query heads of scale * q_h . kbar;
  *   - ties in the top-n go to the lower block index;
