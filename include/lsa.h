@@ -181,6 +181,24 @@ LSA_API int lsa_sparse_attn_decode(const void* q, const void* k, const void* v, 
                            int flags, cudaStream_t stream);
 
 /*
+ * lsa_append_kv -- writes the newest token's key and value into the KV cache, the first
+ * part of a decode step (the cache keeps every token; NSA news article, "NSA 구조": the
+ * selected, compressed and window branches all read the cache).
+ *
+ *   k[b, g, seqlens[b] - 1, :] = k_new[b, g, :]     v[b, g, seqlens[b] - 1, :] = v_new[b, g, :]
+ * seqlens[b] already counts the new token; a sequence with seqlens[b] == 0 is left alone.
+ * k_new, v_new [B, Hkv, D] (dtype); k, v [B, Hkv, T_cap, D] (dtype), written in place.
+ * flags: 0, or LSA_FLAG_PDL: launched as a programmatic dependent of the previous kernel of
+ *     the stream; it reads k_new, v_new and seqlens only after that kernel completes, and
+ *     lets the next kernel start at once (a decode call with LSA_FLAG_PDL then overlaps its
+ *     prologue with this copy; it reads the newest block only after this call completes).
+ * Support: D in {64, 128}; B * Hkv * D <= 2^24.
+ */
+LSA_API int lsa_append_kv(const void* k_new, const void* v_new, int dtype, int B, int Hkv,
+                          int T_cap, int D, const int32_t* seqlens, void* k, void* v, int flags,
+                          cudaStream_t stream);
+
+/*
  * lsa_sparse_attn_blockquery -- one denoising step of a block of Tq query tokens
  * (block-wise diffusion LM) against a cached prefix of T_prefix tokens.
  *
@@ -271,8 +289,9 @@ LSA_API int lsa_sparse_attn_blockquery_noalloc(const void* q, const void* k, con
  * chunks (dims j and j + D/2 form chunk j under rotate-half pairing); one weight per band,
  * 1 / temperature, gives the dual-band score.  Choosing the chunks or temperatures is the
  * caller's.  The reweighted queries w * q are formed in fp32 in q_weighted (scratch,
- * [B, Hq, D] float32, 16-byte aligned; it may be q itself when q is float32) and scored by
- * the selection kernel.  dim_weights: [D] float32, device.  Other arguments and outputs as
+ * [B, Hq, D] float32, 16-byte aligned; it may be q itself when q is float32, and any other
+ * overlap with q or dim_weights returns LSA_ERR_INVALID_ARG) and scored by the selection
+ * kernel.  dim_weights: [D] float32, device.  Other arguments and outputs as
  * lsa_select_blocks (scores_out holds the weighted scores).
  */
 LSA_API int lsa_select_blocks_weighted(const void* q, int dtype, const float* summ,

@@ -31,7 +31,7 @@ EXPORTED = ("lsa_status_string", "lsa_last_cuda_error", "lsa_version", "lsa_buil
             "lsa_sparse_attn_blockquery", "lsa_sparse_attn_blockquery_noalloc",
             "lsa_blasst_prefill", "lsa_device_status", "lsa_losa_classify",
             "lsa_blockquery_intra_merge", "lsa_sparse_attn_decode_blasst", "lsa_nsa_compress",
-            "lsa_nsa_branches", "lsa_select_blocks_weighted")
+            "lsa_nsa_branches", "lsa_select_blocks_weighted", "lsa_append_kv")
 
 _vp, _i, _f = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
 _lib.lsa_status_string.restype = ctypes.c_char_p
@@ -45,6 +45,7 @@ _lib.lsa_select_blocks.argtypes = [_vp, _i, _vp, _i, _i, _i, _i, _i, _vp, _i, _i
                                    _vp, _vp, _vp, _vp]
 _lib.lsa_sparse_attn_decode.argtypes = [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp, _i, _vp, _vp,
                                         _i, _f, _vp, _i, _i, _i, _vp, _vp, _vp, _i, _vp]
+_lib.lsa_append_kv.argtypes = [_vp, _vp, _i, _i, _i, _i, _i, _vp, _vp, _vp, _i, _vp]
 _lib.lsa_blockquery_workspace_size.argtypes = [_i, _i, _i, _i, _i]
 _lib.lsa_blockquery_workspace_size.restype = ctypes.c_size_t
 _lib.lsa_sparse_attn_blockquery.argtypes = [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _vp,
@@ -132,6 +133,14 @@ def lsa_select_blocks(q, summ, seqlens, topk, n_sink, n_local, idx, nsel, scale=
                                   _ptr(idx), _ptr(nsel), _ptr(scores_out), _stream(stream)),
            "lsa_select_blocks")
     return idx, nsel
+
+
+def lsa_append_kv(k_new, v_new, seqlens, k, v, flags=0, stream=None):
+    """k_new, v_new [B,Hkv,D] -> k, v [B,Hkv,T_cap,D] at row seqlens[b] - 1 (in place)."""
+    B, Hkv, T_cap, D = k.shape
+    _check(_lib.lsa_append_kv(_ptr(k_new), _ptr(v_new), _dtype(k), B, Hkv, T_cap, D, _ptr(seqlens),
+                              _ptr(k), _ptr(v), flags, _stream(stream)), "lsa_append_kv")
+    return k, v
 
 
 def lsa_sparse_attn_decode(q, k, v, seqlens, o, topk, idx=None, nsel=None, summ=None,

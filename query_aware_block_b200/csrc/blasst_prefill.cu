@@ -33,6 +33,7 @@
 #include <math.h>
 #include <string.h>
 
+#include "launch_cache.h"
 #include "lsa_common.cuh"
 #include "lsa_internal.h"
 #include "tcgen05.cuh"
@@ -428,13 +429,12 @@ cudaError_t launch_blasst_prefill(const PrefillArgs& a, cudaStream_t stream) {
   p.words = ((a.L + kBN - 1) / kBN + 31) / 32;
   p.scale2 = a.scale * kLog2e;
   p.log2lam = a.lambda > 0.f ? log2f(a.lambda) : -INFINITY;
-  static bool attr_done = false;
-  if (!attr_done) {
-    const cudaError_t err =
-        cudaFuncSetAttribute(blasst_prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
-    if (err != cudaSuccess) return err;
-    attr_done = true;
-  }
+  // the shared memory attribute applies to the current device: set once per device
+  static DeviceOnce attr_once;
+  const cudaError_t err = attr_once.run([] {
+    return cudaFuncSetAttribute(blasst_prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
+  });
+  if (err != cudaSuccess) return err;
   dim3 grid(p.nqt, a.B * a.Hq, 1);
   blasst_prefill_kernel<<<grid, kThreads, kSmemBytes, stream>>>(p);
   return cudaGetLastError();

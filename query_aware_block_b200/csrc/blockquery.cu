@@ -32,6 +32,7 @@
 #include <mutex>
 
 #include "cluster.cuh"
+#include "launch_cache.h"
 #include "lsa_common.cuh"
 #include "lsa_internal.h"
 #include "tcgen05.cuh"
@@ -703,16 +704,15 @@ cudaError_t launch_blockquery(const BlockQueryArgs& a, cudaStream_t stream) {
   p.NBp = NBp;
   p.g_div = make_fastdiv((uint32_t)a.G);
   auto kernel = a.D == 128 ? blockquery_kernel<128> : blockquery_kernel<64>;
-  static int smem_set128 = 0, smem_set64 = 0;
-  int& smem_set = a.D == 128 ? smem_set128 : smem_set64;
-  // the last (cluster size, shared memory) found schedulable, per head dim: the occupancy
-  // query is a host-side cost paid only when the configuration changes
-  static int ok_cl128 = 0, ok_smem128 = 0, ok_cl64 = 0, ok_smem64 = 0;
-  int& ok_cl = a.D == 128 ? ok_cl128 : ok_cl64;
-  int& ok_smem = a.D == 128 ? ok_smem128 : ok_smem64;
-  // these per-process caches are shared by every host thread that launches: one lock
-  // covers them (and the attribute and occupancy calls they guard), not the launch
-  static std::mutex cache_mutex;
+  // per head dim and device: the largest dynamic smem size set so far and the (cluster
+  // size, smem) pairs found schedulable (thread-safe; see launch_cache.h)
+  static LaunchRecord rec128, rec64;
+  LaunchRecord& rec = a.D == 128 ? rec128 : rec64;
+  int dev = 0;
+  {
+    const cudaError_t derr = current_device(&dev);
+    if (derr != cudaSuccess) return derr;
+  }
   for (;;) {
     p.per_max = (NBp + CL - 1) / CL;
     if (p.per_max < 1) p.per_max = 1;
@@ -721,14 +721,6 @@ cudaError_t launch_blockquery(const BlockQueryArgs& a, cudaStream_t stream) {
     const int smem = (int)Lo.total;
     if (smem > 227 * 1024) return cudaErrorInvalidValue;
     cudaError_t err;
-    std::unique_lock<std::mutex> lock(cache_mutex);
-    if (smem > smem_set) {
-      err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-      if (err != cudaSuccess) return err;
-      err = cudaFuncSetAttribute(kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-      if (err != cudaSuccess) return err;
-      smem_set = smem;
-    }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(CL, a.Hkv, a.B);
     cfg.blockDim = dim3(kThreads, 1, 1);
@@ -743,21 +735,24 @@ cudaError_t launch_blockquery(const BlockQueryArgs& a, cudaStream_t stream) {
     attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (!(CL == ok_cl && smem == ok_smem)) {
-      int nclusters = 0;
-      err = cudaOccupancyMaxActiveClusters(&nclusters, kernel, &cfg);
-      if (err != cudaSuccess || nclusters == 0) {
-        (void)cudaGetLastError();
-        if (CL > 2) {
-          CL >>= 1;
-          continue;
+    {
+      std::lock_guard<std::mutex> lock(rec.mu);
+      err = rec.ensure_smem(dev, kernel, smem, true);
+      if (err != cudaSuccess) return err;
+      if (!rec.shape_ok(dev, CL, smem)) {
+        int nclusters = 0;
+        err = cudaOccupancyMaxActiveClusters(&nclusters, kernel, &cfg);
+        if (err != cudaSuccess || nclusters == 0) {
+          (void)cudaGetLastError();
+          if (CL > 2) {
+            CL >>= 1;
+            continue;
+          }
+          return err != cudaSuccess ? err : cudaErrorInvalidConfiguration;
         }
-        return err != cudaSuccess ? err : cudaErrorInvalidConfiguration;
+        rec.remember_shape(dev, CL, smem);
       }
-      ok_cl = CL;
-      ok_smem = smem;
     }
-    lock.unlock();
     cfg.numAttrs = 2;  // launched as a programmatic dependent of the previous kernel
     return cudaLaunchKernelEx(&cfg, kernel, p);
   }
@@ -776,29 +771,40 @@ constexpr size_t kStaticWorkspaceBytes = (size_t)16 << 20;  // 16 MiB
 static __device__ __align__(256) unsigned char g_blockquery_scratch[kStaticWorkspaceBytes];
 
 namespace {
-constexpr int kMaxDevices = 64;
+// per device: the scratch's device address and the id of the context it was looked up in
+struct ScratchSlot {
+  void* ptr = nullptr;
+  unsigned long long ctx = 0;
+};
 std::mutex g_scratch_mutex;
-void* g_scratch_ptr[kMaxDevices] = {};
+ScratchSlot g_scratch[kMaxDevices];
 }  // namespace
 
 size_t blockquery_static_workspace_bytes() { return kStaticWorkspaceBytes; }
 
 // Device address of the fixed scratch on the current device.  The first call on a device
 // looks it up with cudaGetSymbolAddress (the host-side name of the array is not a device
-// address); later calls reuse the cached pointer.
+// address); later calls reuse it while the device's context is the same one.  A device
+// reset (cudaDeviceReset) destroys the context and reloads the module, so a call after it
+// sees a new context id and looks the address up again.
 cudaError_t blockquery_static_workspace(void** ptr) {
   int dev = 0;
-  cudaError_t err = cudaGetDevice(&dev);
+  cudaError_t err = current_device(&dev);
   if (err != cudaSuccess) return err;
-  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
   std::lock_guard<std::mutex> lock(g_scratch_mutex);
-  if (g_scratch_ptr[dev] == nullptr) {
+  ScratchSlot& slot = g_scratch[dev];
+  unsigned long long ctx = 0;
+  const bool known_ctx = current_context_id(&ctx);
+  if (slot.ptr == nullptr || !known_ctx || ctx != slot.ctx) {
     void* p = nullptr;
     err = cudaGetSymbolAddress(&p, g_blockquery_scratch);
     if (err != cudaSuccess) return err;
-    g_scratch_ptr[dev] = p;
+    // (the lookup made the device's primary context current on this thread)
+    unsigned long long now = 0;
+    slot.ctx = current_context_id(&now) ? now : 0;
+    slot.ptr = p;
   }
-  *ptr = g_scratch_ptr[dev];
+  *ptr = slot.ptr;
   return cudaSuccess;
 }
 

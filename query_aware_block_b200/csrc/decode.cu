@@ -45,6 +45,7 @@
 
 #include "cluster.cuh"
 #include "lsa_common.cuh"
+#include "launch_cache.h"
 #include "lsa_internal.h"
 #include "tcgen05.cuh"
 
@@ -886,11 +887,12 @@ cudaError_t launch_t(const DecodeArgs& a, cudaStream_t stream) {
   p.o = a.o; p.lse = a.lse;
   p.m_pad = next_pow2(a.topk < 2 ? 2 : a.topk);
   p.lp = p.m_pad < 16 ? 16 : p.m_pad;
-  // per template instance: the largest dynamic smem size set so far, and the last
-  // (cluster size, smem) pair whose occupancy was checked
-  static int smem_set = 0;
-  static int last_cl = 0, last_smem = -1;
-  cudaError_t err;
+  // per template instance and device: the largest dynamic smem size set so far and the
+  // (cluster size, smem) pairs found schedulable (thread-safe; see launch_cache.h)
+  static LaunchRecord rec;
+  int dev = 0;
+  cudaError_t err = current_device(&dev);
+  if (err != cudaSuccess) return err;
   for (;;) {
     p.per_max = (a.NB_cap + CL - 1) / CL;
     const int E = a.G * D;
@@ -898,13 +900,6 @@ cudaError_t launch_t(const DecodeArgs& a, cudaStream_t stream) {
     p.chunk_div = make_fastdiv((uint32_t)p.chunk);
     const Layout Lo = make_layout((int)sizeof(T), D, p.per_max, p.m_pad);
     const int smem = (int)Lo.total;
-    if (smem > smem_set) {
-      err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-      if (err != cudaSuccess) return err;
-      err = cudaFuncSetAttribute(kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-      if (err != cudaSuccess) return err;
-      smem_set = smem;
-    }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(CL, a.Hkv, a.B);
     cfg.blockDim = dim3(kThreads, 1, 1);
@@ -919,19 +914,23 @@ cudaError_t launch_t(const DecodeArgs& a, cudaStream_t stream) {
     attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = (MODE == MODE_FUSED && a.pdl) ? 2 : 1;
-    if (!(CL == last_cl && smem == last_smem)) {
-      int nclusters = 0;
-      err = cudaOccupancyMaxActiveClusters(&nclusters, kernel, &cfg);
-      if (err != cudaSuccess || nclusters == 0) {
-        (void)cudaGetLastError();
-        if (CL > 2) {
-          CL >>= 1;
-          continue;
+    {
+      std::lock_guard<std::mutex> lock(rec.mu);
+      err = rec.ensure_smem(dev, kernel, smem, true);
+      if (err != cudaSuccess) return err;
+      if (!rec.shape_ok(dev, CL, smem)) {
+        int nclusters = 0;
+        err = cudaOccupancyMaxActiveClusters(&nclusters, kernel, &cfg);
+        if (err != cudaSuccess || nclusters == 0) {
+          (void)cudaGetLastError();
+          if (CL > 2) {
+            CL >>= 1;
+            continue;
+          }
+          return err != cudaSuccess ? err : cudaErrorInvalidConfiguration;
         }
-        return err != cudaSuccess ? err : cudaErrorInvalidConfiguration;
+        rec.remember_shape(dev, CL, smem);
       }
-      last_cl = CL;
-      last_smem = smem;
     }
     return cudaLaunchKernelEx(&cfg, kernel, p);
   }

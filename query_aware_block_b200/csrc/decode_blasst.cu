@@ -16,12 +16,15 @@
 // and stores the maxima into every peer's shared memory (DSMEM); after one cluster barrier
 // every CTA knows every block's maxima and evaluates its own block's test (the maximum
 // over the earlier slots is the running maximum, so the sequential rule is decided in
-// parallel).  Only kept blocks load V.  The per-CTA partials (m, l, acc) are merged by
-// log-sum-exp with DSMEM loads, each CTA producing 1/16 of the outputs.  The only waits are
-// hardware cluster barriers that every thread of every CTA reaches.
+// parallel).  Only kept blocks load V.  Each CTA stores its partial (m, l, acc) into the
+// shared memory of the CTAs that own each slice of the outputs (DSMEM stores), and after
+// one more cluster barrier every CTA merges its 1/16 of the outputs by log-sum-exp from its
+// own shared memory.  The only waits are hardware cluster barriers that every thread of
+// every CTA reaches.
 #include <math.h>
 
 #include "cluster.cuh"
+#include "launch_cache.h"
 #include "lsa_common.cuh"
 #include "lsa_internal.h"
 
@@ -33,11 +36,6 @@ constexpr int kWarps = kThreads / 32;
 constexpr int kCL = 16;      // CTAs per cluster = maximum selection slots
 constexpr int kMaxG = 16;
 
-__device__ __forceinline__ float ld_cluster_f32(uint32_t addr) {
-  float v;
-  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
-  return v;
-}
 
 template <int D>
 struct Smem {
@@ -47,8 +45,8 @@ struct Smem {
   float s[kMaxG][kBlk];              // logits (base 2), then probabilities
   float rmax[kCL][kMaxG];            // every slot's block maxima (written by the peers)
   float rloc[kMaxG];                 // this CTA's block maxima
-  float part_m[kMaxG], part_l[kMaxG];
-  float part_acc[kMaxG * D];
+  float2 recv_ml[kCL][kMaxG];            // (m, l) of every CTA's partial, every head
+  float recv_acc[kCL][kMaxG * D / kCL];  // every CTA's partial of this CTA's output slice
   int slot_block[kCL];               // the block of every slot, -1 if none
   uint32_t valid;                    // bit s: slot s holds a block
 };
@@ -193,10 +191,8 @@ __global__ void __launch_bounds__(kThreads)
     sm.s[h][lane] = p0;
     sm.s[h][lane + 32] = p1;
     const float l = warp_sum(p0 + p1);
-    if (lane == 0) {
-      sm.part_m[h] = keep ? r : -INFINITY;
-      sm.part_l[h] = l;
-    }
+    if (lane < kCL)  // (m, l) of head h into every CTA's table, row `rank`
+      st_cluster(map_rank(&sm.recv_ml[rank][h], lane), make_float2(keep ? r : -INFINITY, l));
   }
   cp_async_wait<0>();  // (the V copies overlapped the softmax above)
   __syncthreads();
@@ -208,7 +204,26 @@ __global__ void __launch_bounds__(kThreads)
 #pragma unroll
     for (int i = 0; i < kMaxG / kHS; ++i) acc[i] = 0.f;
     if (keep) {
-      for (int t = 0; t < nv; ++t) {
+      // 4 keys at a time: one 16-byte read of each head's probabilities (a broadcast) per
+      // 4 value reads; rows at or past nv hold no loaded value and are never read
+      const int nv4 = nv & ~3;
+      for (int t = 0; t < nv4; t += 4) {
+        float vv[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) vv[u] = __bfloat162float(sm.kv[(t + u) * kKS + d]);
+#pragma unroll
+        for (int i = 0; i < kMaxG / kHS; ++i) {
+          const int h = h0 + i * kHS;
+          if (h < G) {
+            const float4 p4 = *reinterpret_cast<const float4*>(&sm.s[h][t]);
+            acc[i] = fmaf(p4.x, vv[0], acc[i]);
+            acc[i] = fmaf(p4.y, vv[1], acc[i]);
+            acc[i] = fmaf(p4.z, vv[2], acc[i]);
+            acc[i] = fmaf(p4.w, vv[3], acc[i]);
+          }
+        }
+      }
+      for (int t = nv4; t < nv; ++t) {
         const float vv = __bfloat162float(sm.kv[t * kKS + d]);
 #pragma unroll
         for (int i = 0; i < kMaxG / kHS; ++i) {
@@ -217,26 +232,32 @@ __global__ void __launch_bounds__(kThreads)
         }
       }
     }
+    // each output element's partial goes to the CTA that owns its slice of the outputs
+    const int per = G * D / kCL;  // (G * D is a multiple of 16: D is 64 or 128)
 #pragma unroll
     for (int i = 0; i < kMaxG / kHS; ++i) {
       const int h = h0 + i * kHS;
-      if (h < G) sm.part_acc[h * D + d] = acc[i];
+      if (h < G) {
+        const int e = h * D + d, owner = e / per;
+        st_cluster(map_rank(&sm.recv_acc[rank][e - owner * per], owner), acc[i]);
+      }
     }
   }
-  cluster_arrive_release();  // every CTA's partial is complete ...
-  cluster_wait();
+  cluster_arrive_release();  // every partial has been stored into its owner ...
+  cluster_wait();            // ... and after this no CTA touches another's shared memory
 
-  // merge: this CTA's 1/16 of the G x D outputs, every partial read over DSMEM
-  const int E = G * D;
-  const int per = (E + kCL - 1) / kCL;
-  for (int e = rank * per + tid; e < min(E, (rank + 1) * per); e += kThreads) {
+  // merge: this CTA's 1/16 of the G x D outputs, from its own shared memory
+  const int per = G * D / kCL;
+  for (int le = tid; le < per; le += kThreads) {
+    const int e = rank * per + le;
     const int h = e / D, d = e - h * D;
     float pm[kCL], pl[kCL], pa[kCL];
 #pragma unroll
-    for (int c = 0; c < kCL; ++c) {  // all loads first
-      pm[c] = ld_cluster_f32(map_rank(&sm.part_m[h], c));
-      pl[c] = ld_cluster_f32(map_rank(&sm.part_l[h], c));
-      pa[c] = ld_cluster_f32(map_rank(&sm.part_acc[h * D + d], c));
+    for (int c = 0; c < kCL; ++c) {
+      const float2 ml = sm.recv_ml[c][h];
+      pm[c] = ml.x;
+      pl[c] = ml.y;
+      pa[c] = sm.recv_acc[c][le];
     }
     float M = -INFINITY;
 #pragma unroll
@@ -255,8 +276,6 @@ __global__ void __launch_bounds__(kThreads)
     if (d == 0 && lse) lse[row] = L > 0.f ? (M + log2f(L)) * kLn2 : -INFINITY;
   }
   if (rank == 0 && tid == 0 && skip_bits) skip_bits[unit] = skipped;
-  cluster_arrive_release();  // no CTA leaves while a peer may still read its partial
-  cluster_wait();
 }
 
 template <int D>
@@ -275,15 +294,16 @@ cudaError_t launch_d(const DecodeBlasstArgs& a, cudaStream_t stream) {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   // the cluster attribute and the occupancy check depend only on the kernel and its fixed
-  // block shape: done once per process (a function-local static is initialised once, also
-  // when host threads race), so that a launch costs only the launch
-  static const cudaError_t check_err = [&]() {
+  // block shape: done once per device (the first launch on a device runs it, racing host
+  // threads wait for it), so that a launch costs only the launch
+  static DeviceOnce check_once;
+  const cudaError_t check_err = check_once.run([&]() {
     cudaError_t err = cudaFuncSetAttribute(kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
     int nclusters = 0;
     if (err == cudaSuccess) err = cudaOccupancyMaxActiveClusters(&nclusters, kernel, &cfg);
     if (err == cudaSuccess && nclusters == 0) err = cudaErrorInvalidConfiguration;
     return err;
-  }();
+  });
   if (check_err != cudaSuccess) return check_err;
   const float scale2 = a.scale * kLog2e;
   const float log2_lambda = a.lambda > 0.f ? log2f(a.lambda) : -INFINITY;

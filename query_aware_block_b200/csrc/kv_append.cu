@@ -1,0 +1,62 @@
+// kv_append.cu -- writes a decode step's new key and value rows into the KV cache.
+//
+// A decode step appends the newest token's key and value at cache row seqlens[b] - 1 (the
+// sequence length already counts it) before attending: NSA news article, "NSA 구조" (the
+// cache keeps every token; the selected, compressed and window branches read from it).
+// One thread moves 16 bytes; the launch is tiny and latency-bound, so it lets the next
+// kernel of the stream start at once (programmatic dependent launch): a decode step launched
+// with LSA_FLAG_PDL overlaps its prologue with this copy and waits for it before it reads
+// the newest block.  Launched itself with LSA_FLAG_PDL, it reads k_new / v_new only after
+// the previous kernel of the stream (the one that produced them) has completed.
+#include "cluster.cuh"
+#include "lsa_internal.h"
+
+namespace lsa {
+namespace {
+
+constexpr int kThreads = 128;
+
+// chunk c of the nb = B * Hkv * rows16 16-byte chunks of k_new (then of v_new): unit
+// u = c / rows16 = b * Hkv + g, column part c % rows16
+__global__ void __launch_bounds__(kThreads)
+    kv_append_kernel(const uint4* __restrict__ k_new, const uint4* __restrict__ v_new, int Hkv, int T_cap,
+                     int rows16, int n, const int32_t* __restrict__ seqlens, uint4* __restrict__ k,
+                     uint4* __restrict__ v) {
+  pdl_trigger();  // the next kernel may start its prologue now ...
+  pdl_wait();     // ... while this one waits for the kernel that produced k_new / v_new
+  const int c = blockIdx.x * kThreads + threadIdx.x;
+  if (c >= 2 * n) return;
+  const bool is_v = c >= n;
+  const int cc = is_v ? c - n : c;
+  const int u = cc / rows16, part = cc - u * rows16;
+  const int b = u / Hkv;
+  const int t = seqlens[b] - 1;
+  if (t < 0 || t >= T_cap) return;  // an empty sequence has no newest token
+  const uint4 x = is_v ? v_new[cc] : k_new[cc];
+  uint4* dst = (is_v ? v : k) + ((size_t)u * T_cap + t) * rows16 + part;
+  *dst = x;
+}
+
+}  // namespace
+
+cudaError_t launch_kv_append(const void* k_new, const void* v_new, int elem_bytes, int B, int Hkv,
+                             int T_cap, int D, const int32_t* seqlens, void* k, void* v, int pdl,
+                             cudaStream_t stream) {
+  const int rows16 = D * elem_bytes / 16;
+  const int n = B * Hkv * rows16;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((2 * n + kThreads - 1) / kThreads, 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kv_append_kernel, static_cast<const uint4*>(k_new),
+                            static_cast<const uint4*>(v_new), Hkv, T_cap, rows16, n, seqlens,
+                            static_cast<uint4*>(k), static_cast<uint4*>(v));
+}
+
+}  // namespace lsa

@@ -114,6 +114,18 @@ int lsa_select_blocks_weighted(const void* q, int dtype, const float* summ,
   if (!q || !summ || !dim_weights || !seqlens || !q_weighted || !idx || !nsel)
     return LSA_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(summ) || !aligned16(q_weighted)) return LSA_ERR_INVALID_ARG;
+  // q_weighted may be q itself only for float32 q (the same element is read, then written, by
+  // one thread); any other overlap would let a thread overwrite query elements that others
+  // have not read yet
+  {
+    const size_t n = (size_t)B * Hkv * G * D;
+    const uintptr_t w0 = (uintptr_t)q_weighted, q0 = (uintptr_t)q;
+    const size_t wbytes = n * 4, qbytes = n * (dtype == LSA_F32 ? 4 : 2);
+    const bool same = dtype == LSA_F32 && w0 == q0;
+    if (!same && w0 < q0 + qbytes && q0 < w0 + wbytes) return LSA_ERR_INVALID_ARG;
+    const uintptr_t d0 = (uintptr_t)dim_weights;
+    if (w0 < d0 + (size_t)D * 4 && d0 < w0 + wbytes) return LSA_ERR_INVALID_ARG;
+  }
   cudaError_t err = lsa::launch_weight_queries(q, dtype, dim_weights, B, Hkv * G, D, q_weighted, stream);
   if (err != cudaSuccess) return cuda_status(err);
   lsa::DecodeArgs a = {};
@@ -161,6 +173,19 @@ int lsa_sparse_attn_decode(const void* q, const void* k, const void* v, int dtyp
   a.mode = fused ? lsa::MODE_FUSED : lsa::MODE_ATTEND;
   a.pdl = (flags & LSA_FLAG_PDL) != 0;
   return cuda_status(lsa::launch_decode(a, stream));
+}
+
+int lsa_append_kv(const void* k_new, const void* v_new, int dtype, int B, int Hkv, int T_cap,
+                  int D, const int32_t* seqlens, void* k, void* v, int flags, cudaStream_t stream) {
+  int st = check_common(dtype, B, Hkv, 1, D, 64);
+  if (st != LSA_OK) return st;
+  if (T_cap < 0 || (flags & ~LSA_FLAG_PDL) != 0) return LSA_ERR_INVALID_ARG;
+  if (T_cap > kMaxTcap || (long long)B * Hkv * D > (1 << 24)) return LSA_ERR_UNSUPPORTED;
+  if (B == 0 || Hkv == 0 || T_cap == 0) return LSA_OK;
+  if (!k_new || !v_new || !seqlens || !k || !v) return LSA_ERR_INVALID_ARG;
+  if (!aligned16(k_new) || !aligned16(v_new) || !aligned16(k) || !aligned16(v)) return LSA_ERR_INVALID_ARG;
+  return cuda_status(lsa::launch_kv_append(k_new, v_new, dtype == LSA_BF16 ? 2 : 4, B, Hkv, T_cap, D,
+                                           seqlens, k, v, (flags & LSA_FLAG_PDL) != 0, stream));
 }
 
 int lsa_sparse_attn_decode_blasst(const void* q, const void* k, const void* v, int dtype, int B,

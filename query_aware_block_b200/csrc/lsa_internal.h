@@ -149,6 +149,15 @@ bool encode_rows_bf16(CUtensorMap* map, const void* base, int D, int rows, int p
 bool kv_tensor_maps(const void* k, const void* v, int D, int T_cap, int planes, CUtensorMap* mk,
                     CUtensorMap* mv);
 
+// The new token's key and value rows into the cache at row seqlens[b] - 1.
+cudaError_t launch_kv_append(const void* k_new, const void* v_new, int elem_bytes, int B, int Hkv,
+                             int T_cap, int D, const int32_t* seqlens, void* k, void* v, int pdl,
+                             cudaStream_t stream);
+
+// Unique id of the context current on this host thread (false when none is current or the
+// driver lacks the entry points).
+bool current_context_id(unsigned long long* id);
+
 // The fixed device scratch used by lsa_sparse_attn_blockquery_noalloc.
 size_t blockquery_static_workspace_bytes();
 cudaError_t blockquery_static_workspace(void** ptr);

@@ -26,6 +26,7 @@
 #include <math.h>
 
 #include "cluster.cuh"
+#include "launch_cache.h"
 #include "lsa_common.cuh"
 #include "lsa_internal.h"
 
@@ -328,16 +329,17 @@ cudaError_t launch_branches(const NsaBranchArgs& a, cudaStream_t stream) {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   // the attributes and the occupancy check depend only on the kernel and its fixed block
-  // shape: done once per process (a function-local static is initialised once, also when
-  // host threads race)
-  static const cudaError_t check_err = [&]() {
+  // shape: done once per device (the first launch on a device runs it, racing host threads
+  // wait for it)
+  static DeviceOnce check_once;
+  const cudaError_t check_err = check_once.run([&]() {
     cudaError_t err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (err == cudaSuccess) err = cudaFuncSetAttribute(kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
     int nclusters = 0;
     if (err == cudaSuccess) err = cudaOccupancyMaxActiveClusters(&nclusters, kernel, &cfg);
     if (err == cudaSuccess && nclusters == 0) err = cudaErrorInvalidConfiguration;
     return err;
-  }();
+  });
   if (check_err != cudaSuccess) return check_err;
   BranchParams p;
   p.q = static_cast<const __nv_bfloat16*>(a.q);

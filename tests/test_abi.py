@@ -179,6 +179,13 @@ def test_weighted_select_validation():
     assert f(*args(D=96)) == lsa.LSA_ERR_UNSUPPORTED
     assert f(*args(blk=32)) == lsa.LSA_ERR_UNSUPPORTED
     assert f(*args(B=0, q=NULL, w=NULL, qw=NULL)) == lsa.LSA_OK
+    # q_weighted (fp32, B*Hq*D*4 bytes) may not overlap a bf16 q, nor partly overlap an fp32
+    # q, nor overlap the weights (q and w far apart here; each call stops at the overlap check)
+    far = ctypes.c_void_p(1 << 30)
+    assert f(*args(q=g, qw=g, w=far)) == lsa.LSA_ERR_INVALID_ARG                       # bf16 q
+    assert f(*args(q=g, qw=ctypes.c_void_p(4096 + 4096), w=far)) == lsa.LSA_ERR_INVALID_ARG
+    assert f(*args(dtype=0, q=g, qw=ctypes.c_void_p(4096 + 256), w=far)) == lsa.LSA_ERR_INVALID_ARG
+    assert f(*args(q=far, qw=g, w=ctypes.c_void_p(4096 + 512))) == lsa.LSA_ERR_INVALID_ARG
 
 
 def test_binding_raises_lsa_error_on_bad_arguments():
@@ -201,3 +208,20 @@ def test_binding_argtypes_match_header_parameter_counts():
         n = 0 if params in ("", "void") else len(params.split(","))
         argt = getattr(lib, name).argtypes
         assert argt is not None and len(argt) == n, (name, n, argt and len(argt))
+
+
+def test_append_kv_validation():
+    import query_aware_block_b200 as lsa
+    f = lsa.library().lsa_append_kv
+    g = ctypes.c_void_p(4096)
+    args = lambda **kw: [kw.get(n, d) for n, d in (
+        ("kn", g), ("vn", g), ("dtype", 1), ("B", 1), ("Hkv", 8), ("T", 65536), ("D", 128),
+        ("sl", g), ("k", g), ("v", g), ("flags", 0), ("stream", NULL))]
+    assert f(*args(kn=NULL)) == lsa.LSA_ERR_INVALID_ARG
+    assert f(*args(v=ctypes.c_void_p(4104))) == lsa.LSA_ERR_INVALID_ARG
+    assert f(*args(flags=2)) == lsa.LSA_ERR_INVALID_ARG
+    assert f(*args(T=-1)) == lsa.LSA_ERR_INVALID_ARG
+    assert f(*args(D=96)) == lsa.LSA_ERR_UNSUPPORTED
+    assert f(*args(dtype=5)) == lsa.LSA_ERR_UNSUPPORTED
+    assert f(*args(B=0, kn=NULL, vn=NULL, k=NULL, v=NULL, sl=NULL)) == lsa.LSA_OK
+

@@ -224,3 +224,45 @@ def test_gqa_decode_64k(lsa):
 def test_batched_varlen_decode(lsa):
     case = synth.batched_decode(poison_tail=True)
     _run_both_modes(lsa, case, torch.bfloat16)
+
+
+# ------------------------------------------------------------ append + decode step ----
+
+@pytest.mark.parametrize("dtype,D", [(torch.bfloat16, 128), (torch.float32, 64)])
+def test_append_then_decode_step(lsa, dtype, D):
+    """A decode step as a serving loop runs it: the newest token's k/v appended by
+    lsa_append_kv (its cache row NaN before), then the fused decode launched with
+    LSA_FLAG_PDL (its prologue overlaps the append).  The cache must equal the original bit
+    for bit, and the outputs must match the oracle on the original inputs."""
+    case = synth.decode_case(B=3, Hkv=2, G=4, D=D, T_cap=64 * 60, seqlens=[64 * 60, 64 * 31 + 1, 0],
+                             dtype=dtype, topk=8, n_sink=1, n_local=2, seed=46, poison_tail=True)
+    q, k, v, sl = _dev(case)
+    B, Hkv, G, D, T_cap = case.shape
+    last = [int(t) - 1 for t in case.seqlens.tolist()]
+    k_new = torch.zeros(B, Hkv, D, device="cuda", dtype=dtype)
+    v_new = torch.zeros_like(k_new)
+    for b in range(B):
+        if last[b] >= 0:
+            k_new[b] = k[b, :, last[b]]
+            v_new[b] = v[b, :, last[b]]
+            k[b, :, last[b]] = float("nan")
+            v[b, :, last[b]] = float("nan")
+    summ = _gpu_summaries(lsa, case.k.cuda(), sl)  # the prefill's summaries of the true keys
+    o = torch.empty_like(q)
+    lse = torch.empty(B, Hkv * G, device="cuda")
+    idx = torch.empty(B, Hkv, case.topk, device="cuda", dtype=torch.int32)
+    lsa.lsa_append_kv(k_new, v_new, sl, k, v)
+    lsa.lsa_sparse_attn_decode(q, k, v, sl, o, case.topk, summ=summ, n_sink=1, n_local=2,
+                               refresh_last_summary=True, idx_out=idx, lse=lse,
+                               flags=lsa.LSA_FLAG_PDL)
+    torch.cuda.synchronize()
+    kc, vc = k.cpu(), v.cpu()
+    for b in range(B):
+        T = int(case.seqlens[b])
+        # bit-exact up to the sequence end (rows past it keep their poison)
+        assert torch.equal(kc[b, :, :T].view(torch.int16 if dtype == torch.bfloat16 else torch.int32),
+                           case.k[b, :, :T].view(torch.int16 if dtype == torch.bfloat16 else torch.int32))
+        assert torch.equal(vc[b, :, :T].view(torch.int16 if dtype == torch.bfloat16 else torch.int32),
+                           case.v[b, :, :T].view(torch.int16 if dtype == torch.bfloat16 else torch.int32))
+    _check_attention(case, o, lse, idx, dtype, "append + decode")
+    assert lsa.lsa_device_status() == 0
