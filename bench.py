@@ -76,6 +76,8 @@ def parse():
     ap.add_argument("--decode-qscale", type=float, default=4.0,
                     help="decode_blasst: scale of the queries (1 = the plain 64K inputs)")
     ap.add_argument("--decode-lambda", type=float, default=1e-3, help="decode_blasst: threshold")
+    ap.add_argument("--decode-batched", action="store_true",
+                    help="decode_blasst: the batched varlen decode inputs (16 sequences) instead of 64K")
     ap.add_argument("--rotate", type=int, default=0, help="input copies (0 = auto, > 4x L2)")
     ap.add_argument("--e2e-steps", type=int, default=2000)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
@@ -1133,77 +1135,118 @@ def run_decode_blasst(args):
     decode (16 blocks per KV head, its own kernels) is given to lsa_sparse_attn_decode_blasst,
     which reads K of every selected block and V only of the blocks some head still needs.
     The queries are scaled by --decode-qscale (a sharper softmax: 1 = the plain workload,
-    where no block is negligible).  Each launch is timed alone with CUDA events after an L2
-    flush (a 512 MB write), next to the plain given-selection decode on the same inputs."""
+    where no block is negligible).  R input copies (distinct caches, queries and
+    selections) are rotated so that a launch's data was last touched more than 4x the L2
+    size of traffic earlier; back-to-back launches over one rotation are captured in a CUDA
+    graph and timed with CUDA events, next to the plain given-selection decode on the same
+    inputs timed the same way."""
     import query_aware_block_b200 as lsa
     import synth
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
-    c = synth.gqa_decode_64k(device=dev)
-    B, Hq, D = c.q.shape
-    Hkv, T_cap = c.k.shape[1], c.k.shape[2]
-    G = Hq // Hkv
     lam = args.decode_lambda
-    q = (c.q.float() * args.decode_qscale).to(torch.bfloat16)
-    summ = torch.zeros(B, Hkv, -(-T_cap // 64), D, device=dev)
-    lsa.lsa_build_summaries(c.k, c.seqlens, summ)
-    idx = torch.empty(B, Hkv, 16, dtype=torch.int32, device=dev)
-    o = torch.empty(B, Hq, D, dtype=torch.bfloat16, device=dev)
-    lse = torch.empty(B, Hq, device=dev)
-    lsa.lsa_sparse_attn_decode(c.q, c.k, c.v, c.seqlens, o, 16, summ=summ, n_sink=1, n_local=2,
-                               idx_out=idx, lse=lse)
-    nsel = (idx >= 0).sum(-1).to(torch.int32)
-    bits = torch.zeros(B, Hkv, dtype=torch.int32, device=dev)
-    flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
-
-    def blasst():
-        lsa.lsa_sparse_attn_decode_blasst(q, c.k, c.v, c.seqlens, idx, nsel, o, lam, lse=lse, skip_bits=bits)
-
-    def plain():
-        lsa.lsa_sparse_attn_decode(q, c.k, c.v, c.seqlens, o, 16, idx=idx, nsel=nsel, lse=lse)
-
-    def cold_us(fn, n):
-        for _ in range(max(3, args.warmup // 100)):
-            flush.fill_(1)
-            fn()
-        torch.cuda.synchronize()
-        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
-        for e0, e1 in evs:
-            flush.fill_(1)
-            e0.record()
-            fn()
-            e1.record()
-        torch.cuda.synchronize()
-        return sum(e0.elapsed_time(e1) for e0, e1 in evs) / n * 1e3
-
-    n = max(20, min(500, args.steps // 400))
-    with ClockSampler(0) as clocks:
-        t_blasst = cold_us(blasst, n)
-        t_plain = cold_us(plain, n)
-    blasst()
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    if args.decode_batched:
+        B, Hkv, G, D, T_cap = 16, 8, 4, 128, 32768
+        make = lambda seed: synth.batched_decode(seed=seed, device=dev)
+        seed0, what = 1003, "batched varlen decode inputs (16 sequences, T ~ U[8K, 32K])"
+    else:
+        B, Hkv, G, D, T_cap = 1, 8, 8, 128, 65536
+        make = lambda seed: synth.gqa_decode_64k(seed=seed, device=dev)
+        seed0, what = 1002, "64K GQA decode inputs"
+    Hq = Hkv * G
+    approx_step = B * Hkv * 16 * 64 * D * 2 * 2
+    R = 4 if args.profile_small else (args.rotate or max(8, min(160, math.ceil(4 * l2 / approx_step))))
+    copies = []
+    for r in range(R):
+        c = make(seed0 + 7919 * r)
+        q = (c.q.float() * args.decode_qscale).to(torch.bfloat16)
+        summ = torch.zeros(B, Hkv, -(-T_cap // 64), D, device=dev)
+        lsa.lsa_build_summaries(c.k, c.seqlens, summ)
+        idx = torch.empty(B, Hkv, 16, dtype=torch.int32, device=dev)
+        o = torch.empty(B, Hq, D, dtype=torch.bfloat16, device=dev)
+        lse = torch.empty(B, Hq, device=dev)
+        lsa.lsa_sparse_attn_decode(c.q, c.k, c.v, c.seqlens, o, 16, summ=summ, n_sink=1, n_local=2,
+                                   idx_out=idx, lse=lse)
+        nsel = (idx >= 0).sum(-1).to(torch.int32)
+        bits = torch.zeros(B, Hkv, dtype=torch.int32, device=dev)
+        copies.append(dict(q=q, k=c.k, v=c.v, sl=c.seqlens, idx=idx, nsel=nsel, o=o, lse=lse, bits=bits))
+        del summ, c
     torch.cuda.synchronize()
-    skipped = sum(bin(int(x) & 0xFFFFFFFF).count("1") for x in bits.flatten().tolist())
-    slots = int(nsel.sum())
-    blk_bytes = 64 * D * 2
-    step_bytes = slots * blk_bytes + (slots - skipped) * blk_bytes + 2 * B * Hq * D * 2 + B * Hkv * 16 * 4
-    gbs = step_bytes / (t_blasst * 1e-6) / 1e9
+
+    def blasst(c):
+        lsa.lsa_sparse_attn_decode_blasst(c["q"], c["k"], c["v"], c["sl"], c["idx"], c["nsel"], c["o"], lam,
+                                          lse=c["lse"], skip_bits=c["bits"])
+
+    def plain(c):
+        lsa.lsa_sparse_attn_decode(c["q"], c["k"], c["v"], c["sl"], c["o"], 16, idx=c["idx"], nsel=c["nsel"],
+                                   lse=c["lse"])
+
+    def graph_of(fn):
+        for c in copies:
+            fn(c)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for c in copies:
+                fn(c)
+        g.replay()
+        torch.cuda.synchronize()
+        return g
+
+    stream = torch.cuda.current_stream()
+    g_b, g_p = graph_of(blasst), graph_of(plain)
+    reps = 2 if args.profile_small else max(5, min(50, args.steps // R))
+    with ClockSampler(0) as clocks:
+        t_blasst, med_b = _time_graph_launches(g_b, R, reps, stream)
+        t_plain, med_p = _time_graph_launches(g_p, R, reps, stream)
+    del g_b, g_p
+    torch.cuda.synchronize()
+    # per launch: K rows of every selected block and V rows of the kept ones (valid tokens
+    # only), q, o, lse, idx, nsel
+    k_tok = v_tok = skipped = slots = 0
+    for c in copies:
+        idx_c, bits_c, sl_c = c["idx"].cpu(), c["bits"].cpu(), c["sl"].cpu()
+        for b in range(B):
+            T = int(sl_c[b])
+            for g in range(Hkv):
+                word = int(bits_c[b, g]) & 0xFFFFFFFF
+                for s_, j in enumerate(idx_c[b, g].tolist()):
+                    if j < 0:
+                        continue
+                    n = max(0, min(64, T - 64 * j))
+                    slots += 1
+                    k_tok += n
+                    if (word >> s_) & 1:
+                        skipped += 1
+                    else:
+                        v_tok += n
+    row = D * 2
+    small = 2 * B * Hq * D * 2 + B * Hq * 4 + B * Hkv * 17 * 4
+    step_bytes = (k_tok + v_tok) * row / R + small
+    plain_bytes = 2 * k_tok * row / R + small
+    t_us, tp_us = t_blasst * 1e3, t_plain * 1e3
+    gbs = step_bytes / (t_us * 1e-6) / 1e9
     peak, kind = measured_peaks()
     return {
-        "metric": "BLASST sparse decode over a given selection (64K GQA decode inputs): tokens/s and effective GB/s",
-        "value": round(B / (t_blasst * 1e-6), 1), "unit": "tokens/s", "n_gpus": 1, "steps": n,
-        "warmup": args.warmup, "ms_per_step": round(t_blasst * 1e-3, 6), "higher_is_better": True,
+        "metric": f"BLASST sparse decode over a given selection ({what}): tokens/s and effective GB/s",
+        "value": round(B / (t_us * 1e-6), 1), "unit": "tokens/s", "n_gpus": 1, "steps": reps * R,
+        "warmup": R, "ms_per_step": round(t_us * 1e-3, 6), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-        "data": f"synthetic 64K GQA decode inputs (seeded), queries x{args.decode_qscale}",
-        "config": {"workload": "decode_blasst", "batch": B, "kv_heads": Hkv, "q_heads_per_kv": G,
+        "data": f"synthetic {what} (seeded), queries x{args.decode_qscale}",
+        "config": {"workload": "decode_blasst" + ("_batched" if args.decode_batched else ""), "batch": B, "kv_heads": Hkv, "q_heads_per_kv": G,
                    "head_dim": D, "context": T_cap, "topk": 16, "lambda": lam,
-                   "l2": "flushed before every launch (512 MB write)"},
+                   "l2": f"{R} input copies rotated ({R * step_bytes / 1e6:.0f} MB touched per rotation, "
+                         f"L2 {l2 / 1e6:.0f} MB); back-to-back launches of one rotation in a CUDA graph"},
         "skip_fraction": round(skipped / max(1, slots), 4), "skipped_v_blocks": skipped, "selected_blocks": slots,
-        "plain_given_selection_decode_us": round(t_plain, 2), "blasst_decode_us": round(t_blasst, 2),
-        "bytes_per_step": int(step_bytes),
+        "blasst_decode_us": round(t_us, 3), "blasst_decode_us_median": round(med_b * 1e3, 3),
+        "plain_given_selection_decode_us": round(tp_us, 3),
+        "plain_given_selection_decode_us_median": round(med_p * 1e3, 3),
+        "bytes_per_step": int(step_bytes), "plain_bytes_per_step": int(plain_bytes),
         "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peak, "unit": "GB/s",
                      "frac": round(gbs / peak, 4), "traffic": None, "kernel": "decode_blasst_kernel<128>",
-                     "peak_source": f"MEASURED_PEAKS.json hbm_gbs ({kind})"},
-        "gpu_launches": n,
+                     "peak_source": f"MEASURED_PEAKS.json hbm_gbs ({kind}, of measured)"},
+        "gpu_launches": reps * R * 2,
         "clocks": clocks.summary(),
     }
 

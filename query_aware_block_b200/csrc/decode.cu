@@ -10,26 +10,29 @@
 //
 // How (B200).  A decode step moves only a few MB, so the kernel is built for latency:
 //   * A cluster of CL CTAs (16, 8 or 4) owns one (b, g); 2 CTAs fit per SM, so a 16-CTA
-//     cluster per KV head fits in one wave.  At launch every CTA copies its slice of the
-//     summary rows into shared memory with cp.async (the slice is fixed by the capacity, so
-//     the copy does not wait for the sequence length); CTAs that own a forced block also
-//     start its K/V copy, so that copy overlaps the scan.  The group's query rows follow.
-//   * Scoring: 4 threads per summary row (quarter-warp-uniform lane mapping, XOR-swizzled
-//     rows: conflict-free 128-bit shared loads) against the summed query in shared memory.
+//     cluster per KV head fits in one wave.  At launch thread 0 of every CTA starts one bulk
+//     copy (cp.async.bulk, the copy engine) of its slice of the summary rows into shared
+//     memory (the slice is fixed by the capacity, so the copy does not wait for the sequence
+//     length); CTAs that own a forced block also start its K/V as TMA boxes, so that copy
+//     overlaps the scan.  The group's query rows follow (16-byte cp.async).
+//   * Scoring: 4 threads per summary row (quarter-warp-uniform lane mapping: conflict-free
+//     128-bit shared loads) against the summed query in shared memory.
 //   * Each CTA ranks its candidates (64-bit keys: score, then lower index) and PUSHES its
 //     sorted local top-m list into every peer's shared memory with st.async, whose bytes
 //     count toward an mbarrier in the receiving CTA: each CTA waits only until the CL lists
 //     have landed (no cluster-wide barrier), then merges them with a tree of warp-wide
-//     bitonic merges (shuffles only) and derives the same global top-m as its peers.
+//     bitonic merges (shuffles only; levels hand over through pairwise named barriers) and
+//     derives the same global top-m as its peers; warp 0 ends the tree holding the list and
+//     starts the TMA copy of this CTA's first scored block at once.
 //     DSMEM is touched only after a split arrive(relaxed)/wait barrier that proves every
 //     CTA of the cluster has started and initialised its mbarriers.
 //   * Overlapped launch (optional, programmatic dependent launch): the summary rows and the
 //     K/V of the forced blocks other than the newest one are requested before the kernel
 //     waits for the previous kernel of the stream; q and the newest block after it.
-//   * The selected blocks are dealt round-robin.  A 64-token block of K and V (16 KB each
-//     at D = 128, bf16) is staged with 16-byte cp.async into XOR-swizzled shared memory
-//     (2-stage pipeline).  For bf16 the G <= 16 query heads are the M = 16 rows of
-//     mma.sync m16n8k16 for S = Q K^T and O += P V; the fp32 path uses CUDA-core FMA.
+//   * The selected blocks are dealt round-robin.  bf16: a 64-token block of K and V (16 KB
+//     each at D = 128) arrives as TMA boxes (128-byte swizzle) on a per-stage mbarrier
+//     (2-stage ring); the G <= 16 query heads are the M = 16 rows of mma.sync m16n8k16 for
+//     S = Q K^T and O += P V.  fp32: 16-byte cp.async into padded rows and CUDA-core FMA.
 //     Online softmax in base 2 with fp32 statistics.
 //   * Each CTA pushes its partial (m, l) and the slices of its accumulator to the CTAs
 //     that own those output elements (st.async again, second mbarrier); each CTA waits for
@@ -39,9 +42,11 @@
 //   * Optionally the CTA that attends the sequence's last block (always a forced local
 //     block) also refreshes that block's summary from the keys it staged: the summary
 //     update of a decode step costs no extra launch and no extra HBM read.
-// No global scratch memory.  The two mbarrier waits are bounded (about 2 s of clock); if
-// one runs out the launch's outputs are undefined and a device status word records it.
+// No global scratch memory.  The mbarrier waits are bounded (about 2 s of clock); if one
+// runs out the launch's outputs are undefined and a device status word records it.
 #include <math.h>
+
+#include <type_traits>
 
 #include "cluster.cuh"
 #include "lsa_common.cuh"
@@ -94,6 +99,7 @@ struct alignas(64) Params {
   int m_pad;              // power of two >= topk
   int lp;                 // length of an exchanged candidate list: max(16, m_pad)
   int chunk;              // output elements merged by one CTA (even)
+  int pdl;                // launched as a programmatic dependent of the previous kernel
   FastDiv chunk_div;      // division by chunk
 };
 
@@ -303,6 +309,22 @@ __global__ void __launch_bounds__(kThreads, 2) decode_cluster_kernel(const __gri
   cluster_arrive_relaxed();
   bool started = false;  // uniform: the start barrier has been waited on
 
+  // The query rows (the mma's A tile; rows >= G zero) by 16-byte cp.async, one commit
+  // group.  Without overlapped launch (nothing to wait for) and with the K/V on TMA (bf16:
+  // no other cp.async group), they are requested here, before anything waits for the
+  // sequence length; otherwise after the wait for the previous kernel, which may write q.
+  auto stage_q = [&]() {
+    constexpr int kQChunks = kRows * kRowBytesQ / 16;
+    for (int id = tid; id < kQChunks; id += kThreads) {
+      const int row = id / (kRowBytesQ / 16), c = id % (kRowBytesQ / 16);
+      cp_async16(Qs + (kF32 ? row * kRowBytesQ + c * 16 : swz(row, c, kRowBytesQ)),
+                 qg + (size_t)(row < G ? row : 0) * D + c * (16 / (int)sizeof(T)), row < G);
+    }
+    cp_async_commit();
+  };
+  const bool q_early = !kF32 && !p.pdl;
+  if (q_early) stage_q();
+
   // ---- which blocks: forced / all known up front; order[i] is handled by CTA i % CL ----
   const bool all_blocks = select && NB <= p.topk;
   const int nf = (select && !all_blocks) ? p.n_sink + p.n_local : 0;  // disjoint: NB > topk
@@ -374,15 +396,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_cluster_kernel(const __gri
   pdl_wait();
 
   // ---- query rows (the mma's A tile; rows >= G zero), then the remaining known blocks ----
-  {
-    constexpr int kQChunks = kRows * kRowBytesQ / 16;
-    for (int id = tid; id < kQChunks; id += kThreads) {
-      const int row = id / (kRowBytesQ / 16), c = id % (kRowBytesQ / 16);
-      cp_async16(Qs + (kF32 ? row * kRowBytesQ + c * 16 : swz(row, c, kRowBytesQ)),
-                 qg + (size_t)(row < G ? row : 0) * D + c * (16 / (int)sizeof(T)), row < G);
-    }
-    cp_async_commit();
-  }
+  if (!q_early) stage_q();
   const int issued_before_q = issued;
   bool newest_issued = false;
   if (MODE == MODE_FUSED && scan && issued == 0 && n_known > 0) {  // the newest block, now
@@ -431,7 +445,10 @@ __global__ void __launch_bounds__(kThreads, 2) decode_cluster_kernel(const __gri
       qv[4 * m] = v.x; qv[4 * m + 1] = v.y; qv[4 * m + 2] = v.z; qv[4 * m + 3] = v.w;
     }
     const float* grow = p.summ + (unit * (size_t)p.NB_cap + j0) * D;
-    for (int base = 0; base < nloc; base += kPassRows) {  // uniform trip count
+    // one pass: rows base .. base + kPassRows - 1 of this CTA's slice, from the rows staged
+    // in shared memory (the first pass) or from global memory (any later one); the two
+    // sources are separate instantiations so that the staged rows are read with shared loads
+    auto score_pass = [&](int base, auto staged) {
       float dot[2];
 #pragma unroll
       for (int i = 0; i < 2; ++i) {
@@ -440,9 +457,11 @@ __global__ void __launch_bounds__(kThreads, 2) decode_cluster_kernel(const __gri
         if (oo < nloc) {
 #pragma unroll
           for (int m = 0; m < kCPL; ++m) {
-            const float4 v = base == 0
-                ? reinterpret_cast<const float4*>(sumbuf + oo * D)[cs + 8 * m]
-                : __ldg(reinterpret_cast<const float4*>(grow + (size_t)oo * D) + cs + 8 * m);
+            float4 v;
+            if constexpr (decltype(staged)::value)
+              v = reinterpret_cast<const float4*>(sumbuf + oo * D)[cs + 8 * m];
+            else
+              v = __ldg(reinterpret_cast<const float4*>(grow + (size_t)oo * D) + cs + 8 * m);
             a0 = fmaf(v.x, qv[4 * m], a0);
             a1 = fmaf(v.y, qv[4 * m + 1], a1);
             a0 = fmaf(v.z, qv[4 * m + 2], a0);
@@ -470,7 +489,9 @@ __global__ void __launch_bounds__(kThreads, 2) decode_cluster_kernel(const __gri
           }
         }
       }
-    }
+    };
+    if (nloc > 0) score_pass(0, std::true_type{});
+    for (int base = kPassRows; base < nloc; base += kPassRows) score_pass(base, std::false_type{});
     if (nloc == 0) {  // no pass ran: the rank count below still reads a full pass
       for (int i = tid; i < min(kPassRows, per); i += kThreads) keys[i] = 0ull;
     }
@@ -914,6 +935,7 @@ cudaError_t launch_t(const DecodeArgs& a, cudaStream_t stream) {
     attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = (MODE == MODE_FUSED && a.pdl) ? 2 : 1;
+    p.pdl = cfg.numAttrs == 2;
     {
       std::lock_guard<std::mutex> lock(rec.mu);
       err = rec.ensure_smem(dev, kernel, smem, true);

@@ -12,21 +12,27 @@
 // The output is softmax attention over the tokens of the kept blocks.
 //
 // How (B200): one thread-block cluster of 16 CTAs per (b, g), CTA r owning selection slot
-// r.  Each CTA loads q and its K block, computes the G x 64 logits and the G block maxima,
-// and stores the maxima into every peer's shared memory (DSMEM); after one cluster barrier
-// every CTA knows every block's maxima and evaluates its own block's test (the maximum
-// over the earlier slots is the running maximum, so the sequential rule is decided in
-// parallel).  Only kept blocks load V.  Each CTA stores its partial (m, l, acc) into the
-// shared memory of the CTAs that own each slice of the outputs (DSMEM stores), and after
-// one more cluster barrier every CTA merges its 1/16 of the outputs by log-sum-exp from its
-// own shared memory.  The only waits are hardware cluster barriers that every thread of
-// every CTA reaches.
+// r (topk <= 16).  Thread 0 reads the slot's block index and starts the K block as TMA
+// boxes (128-byte swizzle) on one mbarrier; q arrives by cp.async meanwhile.  S = Q K^T
+// runs on mma.sync m16n8k16 (the G <= 16 query heads are the 16 rows), the block maxima are
+// reduced across the warps, and each CTA stores its G maxima into every peer's shared
+// memory with st.async, completed on the receiver's mbarrier (no cluster barrier).  Every
+// CTA then evaluates the test for every slot (the maximum over the earlier slots is the
+// running maximum, so the sequential rule is decided in parallel); a kept block's CTA
+// starts its V block by TMA (second mbarrier), forms P = 2^(S - r) in bf16 and computes
+// P V on mma.sync.  Each CTA pushes its partial (m, l) and the slices of its accumulator
+// to the CTAs that own those output elements (st.async, third mbarrier), and every CTA
+// merges its 1/16 of the outputs by log-sum-exp from its own shared memory.  Every byte a
+// CTA receives is counted by its own mbarriers and waited for before it ends, so no CTA
+// leaves while a peer may still write into it.  Waits are bounded (about 2 s of clock); if
+// one runs out the launch's outputs are undefined and a status word records it.
 #include <math.h>
 
 #include "cluster.cuh"
 #include "launch_cache.h"
 #include "lsa_common.cuh"
 #include "lsa_internal.h"
+#include "tcgen05.cuh"
 
 namespace lsa {
 namespace {
@@ -34,257 +40,345 @@ namespace {
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
 constexpr int kCL = 16;      // CTAs per cluster = maximum selection slots
-constexpr int kMaxG = 16;
+constexpr int kRows = 16;    // query-head rows (G <= 16): the mma M dimension
+constexpr long long kWaitBudget = 4000000000LL;  // clock cycles (about 2 s)
 
+// Set when a bounded wait runs out (the outputs of that launch are then undefined); read
+// and cleared by the host.
+__device__ int g_blasst_decode_status = 0;
 
-template <int D>
-struct Smem {
-  static constexpr int kKS = D + 8;  // padded K/V row (bf16): conflict-free 16-byte reads
-  __nv_bfloat16 kv[kBlk * kKS];      // the K block, then (if kept) the V block
-  __nv_bfloat16 q[kMaxG * D];
-  float s[kMaxG][kBlk];              // logits (base 2), then probabilities
-  float rmax[kCL][kMaxG];            // every slot's block maxima (written by the peers)
-  float rloc[kMaxG];                 // this CTA's block maxima
-  float2 recv_ml[kCL][kMaxG];            // (m, l) of every CTA's partial, every head
-  float recv_acc[kCL][kMaxG * D / kCL];  // every CTA's partial of this CTA's output slice
-  int slot_block[kCL];               // the block of every slot, -1 if none
-  uint32_t valid;                    // bit s: slot s holds a block
+struct Params {
+  CUtensorMap tmk;  // bf16 K and V as [B * Hkv][T_cap][D], box {64, 64, 1}, 128-byte swizzle
+  CUtensorMap tmv;
+  const __nv_bfloat16* q;
+  int Hkv, G, T_cap;
+  const int32_t* seqlens;
+  const int32_t* idx;
+  const int32_t* nsel;
+  int topk;
+  float scale2;       // softmax scale times log2(e)
+  float log2_lambda;  // log2(lambda), -inf for lambda = 0
+  __nv_bfloat16* o;
+  float* lse;
+  uint32_t* skip_bits;
 };
 
-// Launched with clusters of kCL CTAs along x (grid (kCL, Hkv, B)).
+// Shared-memory carve-up (byte offsets from the first 1024-byte boundary of the dynamic buffer).
 template <int D>
-__global__ void __launch_bounds__(kThreads)
-    decode_blasst_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
-                         const __nv_bfloat16* __restrict__ v, int Hkv, int G, int T_cap,
-                         const int32_t* __restrict__ seqlens, const int32_t* __restrict__ idx,
-                         const int32_t* __restrict__ nsel, int topk, float scale2, float log2_lambda,
-                         __nv_bfloat16* __restrict__ o, float* __restrict__ lse,
-                         uint32_t* __restrict__ skip_bits) {
-  using S = Smem<D>;
-  constexpr int kKS = S::kKS;
-  constexpr int kC = D / 8;  // 16-byte chunks per row
-  __shared__ __align__(16) S sm;
+struct Lay {
+  static constexpr int kTile = kBlk * D * 2;            // one K or V block (bf16)
+  static constexpr int kK = 0;                          // TMA boxes: 1024-byte aligned
+  static constexpr int kV = kK + kTile;
+  static constexpr int kQ = kV + kTile;                 // [16][D] bf16, chunk-swizzled
+  static constexpr int kP = kQ + kRows * D * 2;         // [16][64] bf16, chunk-swizzled
+  static constexpr int kRed = kP + kRows * kBlk * 2;    // [8 warps][16] float
+  static constexpr int kRmax = kRed + kWarps * kRows * 4;        // [16 slots][16 heads] float
+  static constexpr int kMl = kRmax + kCL * kRows * 4;            // [16 CTAs][16 heads] float2
+  static constexpr int kAcc = kMl + kCL * kRows * 8;             // [16 CTAs][16 D / 16] float
+  static constexpr int kTotal = kAcc + kCL * (kRows * D / kCL) * 4;
+};
+
+template <int D>
+__global__ void __launch_bounds__(kThreads) decode_blasst_kernel(const __grid_constant__ Params p) {
+  using L = Lay<D>;
+  constexpr int kRowBytes = D * 2;
+  constexpr int NT = D / 64;  // n8 tiles of the output per warp
+  extern __shared__ __align__(1024) unsigned char smem[];
+  // mbarriers: [0] the K block, [1] the V block, [2] the block maxima of every slot, [3] the
+  // partials of every CTA (one phase each)
+  __shared__ __align__(8) uint64_t bar[4];
+  __shared__ int slot_block[kCL];
+  __shared__ uint32_t valid_bits, skip_word;
+  __shared__ float rloc[kRows], lloc[kRows];
+  __shared__ int xabort;
+  // the K/V boxes land 1024-byte aligned (128-byte swizzle): the layout starts at the first
+  // 1024-byte boundary of the dynamic buffer (1 KB of slack is allocated for it)
+  unsigned char* base = smem + ((1024u - (tc::smem_u32(smem) & 1023u)) & 1023u);
+  unsigned char* Ks = base + L::kK;
+  unsigned char* Vs = base + L::kV;
+  unsigned char* Qs = base + L::kQ;
+  unsigned char* Ps = base + L::kP;
+  float* red = reinterpret_cast<float*>(base + L::kRed);
+  float* rmax = reinterpret_cast<float*>(base + L::kRmax);
+  float2* ml_in = reinterpret_cast<float2*>(base + L::kMl);
+  float* acc_in = reinterpret_cast<float*>(base + L::kAcc);
+
   const int rank = cluster_rank();
   const int g = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int Hq = Hkv * G;
-  const size_t unit = (size_t)b * Hkv + g;
-  cluster_arrive_relaxed();  // peers' shared memory is written only after all have started
+  const int G = p.G;
+  const int Hq = p.Hkv * G;
+  const int unit = b * p.Hkv + g;
+  const int per = G * D / kCL;  // output elements merged by one CTA (G * D is a multiple of 16)
 
-  // which slots hold a block (the same on every CTA): one load per lane of warp 0, all in
-  // flight together; the q rows of the group start copying meanwhile
-  for (int id = tid; id < G * kC; id += kThreads) {
-    const int h = id / kC, c = id - h * kC;
-    cp_async16(sm.q + h * D + c * 8, q + ((size_t)b * Hq + (size_t)g * G + h) * D + c * 8, true);
+  // the slot's block and the sequence length first (the K copy waits only for them)
+  const int ns = __ldg(p.nsel + unit);
+  const int jj = rank < p.topk ? __ldg(p.idx + unit * p.topk + rank) : -1;
+  const int T = __ldg(p.seqlens + b);
+  if (tid == 0) {
+    for (int i = 0; i < 4; ++i) tc::mbar_init(&bar[i], 1);
+    xabort = 0;
+    tc::fence_mbar_init();
+    tc::prefetch_tmap(&p.tmk);
+    tc::prefetch_tmap(&p.tmv);
+    const bool has0 = rank < ns && jj >= 0;
+    if (has0 && jj * kBlk < T) {
+      tc::mbar_arrive_expect_tx(&bar[0], (uint32_t)L::kTile);
+#pragma unroll
+      for (int h = 0; h < D / 64; ++h) tc::tma_load_3d(Ks + h * 8192, &p.tmk, h * 64, jj * kBlk, unit, &bar[0]);
+    }
   }
-  cp_async_commit();
-  const int T = seqlens[b];
+  cluster_arrive_relaxed();  // DSMEM is written only after every CTA has started
+  // the query rows (rows >= G zero) by 16-byte cp.async
+  {
+    const __nv_bfloat16* qg = p.q + ((size_t)b * Hq + (size_t)g * G) * D;
+    constexpr int kQChunks = kRows * kRowBytes / 16;
+    for (int id = tid; id < kQChunks; id += kThreads) {
+      const int row = id / (kRowBytes / 16), c = id % (kRowBytes / 16);
+      cp_async16(Qs + swz(row, c, kRowBytes), qg + (size_t)(row < G ? row : 0) * D + c * 8, row < G);
+    }
+    cp_async_commit();
+  }
+  // which slots hold a block (the same on every CTA)
   if (warp == 0) {
-    const int ns = nsel[unit];
-    const int jj = lane < topk && lane < kCL ? idx[unit * topk + lane] : -1;
-    const bool on = lane < ns && jj >= 0;
+    const int j2 = lane < p.topk && lane < kCL ? __ldg(p.idx + unit * p.topk + lane) : -1;
+    const bool on = lane < ns && lane < kCL && j2 >= 0;
     const uint32_t bits = __ballot_sync(0xffffffffu, on);
-    if (lane < kCL) sm.slot_block[lane] = on ? jj : -1;
-    if (lane == 0) sm.valid = bits;
+    if (lane < kCL) slot_block[lane] = on ? j2 : -1;
+    if (lane == 0) valid_bits = bits;
   }
-  __syncthreads();
-  const uint32_t valid = sm.valid;
-  const bool has = (valid >> rank) & 1u;
-  const int j = has ? sm.slot_block[rank] : 0;
-  const int nv = has ? max(0, min(kBlk, T - j * kBlk)) : 0;  // valid rows of the block
-  const size_t kvrow0 = unit * (size_t)T_cap + (size_t)j * kBlk;
-
-  // the K block (rows past the sequence are not read), every copy in flight at once
-  for (int id = tid; id < nv * kC; id += kThreads) {
-    const int r = id / kC, c = id - r * kC;
-    cp_async16(sm.kv + r * kKS + c * 8, k + (kvrow0 + r) * D + c * 8, true);
-  }
-  cp_async_commit();
   cp_async_wait<0>();
   __syncthreads();
-  // logits in base 2: pair (h, t) = (p >> 6, p & 63); a warp shares h (q reads broadcast)
-  for (int p = tid; p < G * kBlk; p += kThreads) {
-    const int h = p >> 6, t = p & (kBlk - 1);
-    float acc = -INFINITY;
-    if (t < nv) {
-      float a0 = 0.f, a1 = 0.f;
-      const __nv_bfloat16* kr = sm.kv + t * kKS;
-      const __nv_bfloat16* qr = sm.q + h * D;
-#pragma unroll 4
-      for (int c = 0; c < kC; ++c) {
-        const uint4 kk = *reinterpret_cast<const uint4*>(kr + c * 8);
-        const uint4 qq = *reinterpret_cast<const uint4*>(qr + c * 8);
-        const uint32_t wk[4] = {kk.x, kk.y, kk.z, kk.w};
-        const uint32_t wq[4] = {qq.x, qq.y, qq.z, qq.w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          a0 = fmaf(__uint_as_float(wq[e] << 16), __uint_as_float(wk[e] << 16), a0);
-          a1 = fmaf(__uint_as_float(wq[e] & 0xffff0000u), __uint_as_float(wk[e] & 0xffff0000u), a1);
-        }
-      }
-      acc = (a0 + a1) * scale2;
-    }
-    sm.s[h][t] = acc;
-  }
-  __syncthreads();
-  // block maxima (warp per head)
-  for (int h = warp; h < G; h += kWarps) {
-    float mx = fmaxf(sm.s[h][lane], sm.s[h][lane + 32]);
-#pragma unroll
-    for (int o2 = 16; o2 > 0; o2 >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o2));
-    if (lane == 0) sm.rloc[h] = mx;
-  }
-  __syncthreads();
-  cluster_wait();  // (matches the arrive at the start) every CTA has started: DSMEM is live
-  if (has) {       // this block's maxima into every CTA's table, row `rank`
-    for (int i = tid; i < kCL * G; i += kThreads) {
-      const int peer = i / G, h = i - peer * G;
-      st_cluster(map_rank(&sm.rmax[rank][h], peer), sm.rloc[h]);
-    }
-  }
-  cluster_arrive_release();  // the stores above are visible to every peer ...
-  cluster_wait();            // ... once every CTA has passed here
+  const uint32_t valid = valid_bits;
+  const int nvalid = __popc(valid);
+  const bool has = (valid >> rank) & 1u;
+  const int j = has ? slot_block[rank] : 0;
+  const int nv = has ? max(0, min(kBlk, T - j * kBlk)) : 0;  // valid rows of the block
+  const bool loaded = nv > 0;
 
-  // the test for every slot (each CTA decides all of them; it acts on its own)
-  uint32_t skipped = 0u;
+  // ---- S = Q K^T (base-2 logits), the block maxima --------------------------------------
+  float s[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+  uint32_t qa[D / 16][4];
+  const int r0 = lane >> 2;
+  const int col = 8 * warp + 2 * (lane & 3);
+  if (loaded) {
+#pragma unroll
+    for (int ks = 0; ks < D / 16; ++ks) {
+      const int row = (lane & 7) + 8 * ((lane >> 3) & 1);
+      ldsm_x4(qa[ks], Qs + swz(row, 2 * ks + (lane >> 4), kRowBytes));
+    }
+    tc::mbar_wait(&bar[0], 0, &xabort, kWaitBudget);
+    float c4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int ks = 0; ks < D / 16; ks += 2) {
+      uint32_t kb[4];
+      ldsm_x4(kb, Ks + kv_off(8 * warp + (lane & 7), 2 * ks + (lane >> 3)));
+      mma_bf16(c4, qa[ks], kb[0], kb[1]);
+      mma_bf16(c4, qa[ks + 1], kb[2], kb[3]);
+    }
+    const bool v0 = col < nv, v1 = col + 1 < nv;
+    s[0] = v0 && r0 < G ? c4[0] * p.scale2 : -INFINITY;
+    s[1] = v1 && r0 < G ? c4[1] * p.scale2 : -INFINITY;
+    s[2] = v0 && r0 + 8 < G ? c4[2] * p.scale2 : -INFINITY;
+    s[3] = v1 && r0 + 8 < G ? c4[3] * p.scale2 : -INFINITY;
+  }
   {
-    float m_run[kMaxG];
+    float m_lo = fmaxf(s[0], s[1]), m_hi = fmaxf(s[2], s[3]);
 #pragma unroll
-    for (int h = 0; h < kMaxG; ++h) m_run[h] = -INFINITY;
-    bool first = true;
-    for (int s = 0; s < kCL; ++s) {
-      if (!((valid >> s) & 1u)) continue;
-      float gap = -INFINITY;
-#pragma unroll
-      for (int h = 0; h < kMaxG; ++h) {
-        if (h < G) {
-          const float r = sm.rmax[s][h];
-          const float gi = r == -INFINITY ? -INFINITY : (m_run[h] == -INFINITY ? INFINITY : r - m_run[h]);
-          gap = fmaxf(gap, gi);
-        }
-      }
-      if (!first && gap < log2_lambda) skipped |= 1u << s;
-      first = false;
-#pragma unroll
-      for (int h = 0; h < kMaxG; ++h)
-        if (h < G) m_run[h] = fmaxf(m_run[h], sm.rmax[s][h]);
+    for (int o2 = 1; o2 < 4; o2 <<= 1) {
+      m_lo = fmaxf(m_lo, __shfl_xor_sync(0xffffffffu, m_lo, o2));
+      m_hi = fmaxf(m_hi, __shfl_xor_sync(0xffffffffu, m_hi, o2));
+    }
+    if ((lane & 3) == 0) {
+      red[warp * kRows + r0] = m_lo;
+      red[warp * kRows + r0 + 8] = m_hi;
     }
   }
-  const bool keep = has && !((skipped >> rank) & 1u) && nv > 0;
+  __syncthreads();
+  if (tid < kRows) {
+    float mx = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) mx = fmaxf(mx, red[w * kRows + tid]);
+    rloc[tid] = mx;
+  }
+  cluster_wait();  // (matches the arrive at the start) every CTA runs: DSMEM is live
+  if (tid == 0) tc::mbar_arrive_expect_tx(&bar[2], (uint32_t)(nvalid * G * 4));
+  __syncthreads();  // (rloc is complete)
+  // this slot's maxima into every CTA's table, row `rank`
+  if (has && tid < kCL * G) {
+    const int peer = tid / G, h = tid - peer * G;
+    st_async(map_rank(rmax + rank * kRows + h, peer), rloc[h], map_rank(&bar[2], peer));
+  }
+  if (nvalid > 0) tc::mbar_wait(&bar[2], 0, &xabort, kWaitBudget);
 
-  // V of a kept block (into the K buffer: the logits are done), softmax, P.V
-  __syncthreads();
-  if (keep) {
-    for (int id = tid; id < nv * kC; id += kThreads) {
-      const int r = id / kC, c = id - r * kC;
-      cp_async16(sm.kv + r * kKS + c * 8, v + (kvrow0 + r) * D + c * 8, true);
-    }
-  }
-  cp_async_commit();
-  for (int h = warp; h < G; h += kWarps) {  // probabilities and row sums (warp per head)
-    const float r = sm.rmax[rank][h];
-    float p0 = 0.f, p1 = 0.f;
-    if (keep) {
-      p0 = lane < nv ? ex2(sm.s[h][lane] - r) : 0.f;
-      p1 = lane + 32 < nv ? ex2(sm.s[h][lane + 32] - r) : 0.f;
-    }
-    sm.s[h][lane] = p0;
-    sm.s[h][lane + 32] = p1;
-    const float l = warp_sum(p0 + p1);
-    if (lane < kCL)  // (m, l) of head h into every CTA's table, row `rank`
-      st_cluster(map_rank(&sm.recv_ml[rank][h], lane), make_float2(keep ? r : -INFINITY, l));
-  }
-  cp_async_wait<0>();  // (the V copies overlapped the softmax above)
-  __syncthreads();
-  {
-    // output element (h, d): thread takes d = tid % D and heads tid / D + k * (256 / D)
-    constexpr int kHS = kThreads / D;  // 2 (D 128) or 4 (D 64)
-    const int d = tid % D, h0 = tid / D;
-    float acc[kMaxG / kHS];
+  // ---- the test for every slot (each CTA decides all of them; it acts on its own) ----------
+  // Warp 0, lane s = slot s: per head, the running maximum before slot s is an exclusive
+  // prefix maximum over the lanes (slots without a block contribute -inf); the slot's gap is
+  // the maximum over the heads of (r_h - m_h).  The first slot holding a block is never
+  // skipped.  The decision reaches the other warps through shared memory.
+  if (warp == 0) {
+    const bool vs = lane < kCL && ((valid >> lane) & 1u);
+    float gap = -INFINITY;
 #pragma unroll
-    for (int i = 0; i < kMaxG / kHS; ++i) acc[i] = 0.f;
-    if (keep) {
-      // 4 keys at a time: one 16-byte read of each head's probabilities (a broadcast) per
-      // 4 value reads; rows at or past nv hold no loaded value and are never read
-      const int nv4 = nv & ~3;
-      for (int t = 0; t < nv4; t += 4) {
-        float vv[4];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) vv[u] = __bfloat162float(sm.kv[(t + u) * kKS + d]);
-#pragma unroll
-        for (int i = 0; i < kMaxG / kHS; ++i) {
-          const int h = h0 + i * kHS;
-          if (h < G) {
-            const float4 p4 = *reinterpret_cast<const float4*>(&sm.s[h][t]);
-            acc[i] = fmaf(p4.x, vv[0], acc[i]);
-            acc[i] = fmaf(p4.y, vv[1], acc[i]);
-            acc[i] = fmaf(p4.z, vv[2], acc[i]);
-            acc[i] = fmaf(p4.w, vv[3], acc[i]);
-          }
-        }
-      }
-      for (int t = nv4; t < nv; ++t) {
-        const float vv = __bfloat162float(sm.kv[t * kKS + d]);
-#pragma unroll
-        for (int i = 0; i < kMaxG / kHS; ++i) {
-          const int h = h0 + i * kHS;
-          if (h < G) acc[i] = fmaf(sm.s[h][t], vv, acc[i]);
-        }
-      }
-    }
-    // each output element's partial goes to the CTA that owns its slice of the outputs
-    const int per = G * D / kCL;  // (G * D is a multiple of 16: D is 64 or 128)
-#pragma unroll
-    for (int i = 0; i < kMaxG / kHS; ++i) {
-      const int h = h0 + i * kHS;
+    for (int h = 0; h < kRows; ++h) {
       if (h < G) {
-        const int e = h * D + d, owner = e / per;
-        st_cluster(map_rank(&sm.recv_acc[rank][e - owner * per], owner), acc[i]);
+        const float r = vs ? rmax[lane * kRows + h] : -INFINITY;
+        float m = r;  // inclusive prefix maximum over lanes 0 .. lane
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const float t = __shfl_up_sync(0xffffffffu, m, o);
+          if (lane >= o) m = fmaxf(m, t);
+        }
+        float before = __shfl_up_sync(0xffffffffu, m, 1);
+        if (lane == 0) before = -INFINITY;
+        const float gi = r == -INFINITY ? -INFINITY : (before == -INFINITY ? INFINITY : r - before);
+        gap = fmaxf(gap, gi);
+      }
+    }
+    const int first = valid ? __ffs(valid) - 1 : -1;
+    const uint32_t bits = __ballot_sync(0xffffffffu, vs && lane != first && gap < p.log2_lambda);
+    if (lane == 0) skip_word = bits;
+  }
+  __syncthreads();
+  const uint32_t skipped = skip_word;
+  const bool keep = loaded && !((skipped >> rank) & 1u);
+  if (keep && tid == 0) {
+    tc::mbar_arrive_expect_tx(&bar[1], (uint32_t)L::kTile);
+#pragma unroll
+    for (int h = 0; h < D / 64; ++h) tc::tma_load_3d(Vs + h * 8192, &p.tmv, h * 64, j * kBlk, unit, &bar[1]);
+  }
+
+  // ---- P = 2^(S - r) (bf16, into shared memory), the row sums, O = P V ---------------------
+  float acc[NT][4];
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) acc[nt][e] = 0.f;
+  if (keep) {  // (uniform)
+    const float rl = rloc[r0], rh = rloc[r0 + 8];
+    const float p0 = s[0] == -INFINITY ? 0.f : ex2(s[0] - rl);
+    const float p1 = s[1] == -INFINITY ? 0.f : ex2(s[1] - rl);
+    const float p2 = s[2] == -INFINITY ? 0.f : ex2(s[2] - rh);
+    const float p3 = s[3] == -INFINITY ? 0.f : ex2(s[3] - rh);
+    *reinterpret_cast<uint32_t*>(Ps + swz(r0, col >> 3, kBlk * 2) + (col & 7) * 2) = pack_bf16x2(p0, p1);
+    *reinterpret_cast<uint32_t*>(Ps + swz(r0 + 8, col >> 3, kBlk * 2) + (col & 7) * 2) = pack_bf16x2(p2, p3);
+    float l_lo = p0 + p1, l_hi = p2 + p3;
+#pragma unroll
+    for (int o2 = 1; o2 < 4; o2 <<= 1) {
+      l_lo += __shfl_xor_sync(0xffffffffu, l_lo, o2);
+      l_hi += __shfl_xor_sync(0xffffffffu, l_hi, o2);
+    }
+    // (red held the maxima, all read before the barrier after the rloc reduction)
+    if ((lane & 3) == 0) {
+      red[warp * kRows + r0] = l_lo;
+      red[warp * kRows + r0 + 8] = l_hi;
+    }
+    // V rows past the sequence hold whatever the cache holds there: zero them once they
+    // have landed, so that P = 0 never meets a NaN
+    tc::mbar_wait(&bar[1], 0, &xabort, kWaitBudget);
+    for (int id = tid; id < (kBlk - nv) * (D / 8); id += kThreads) {
+      const int r = nv + id / (D / 8), c = id % (D / 8);
+      *reinterpret_cast<uint4*>(Vs + kv_off(r, c)) = make_uint4(0u, 0u, 0u, 0u);
+    }
+    __syncthreads();
+    if (tid < kRows) {
+      float l = 0.f;
+#pragma unroll
+      for (int w = 0; w < kWarps; ++w) l += red[w * kRows + tid];
+      lloc[tid] = l;
+    }
+    // warp w takes output columns [w * D / 8, (w + 1) * D / 8)
+#pragma unroll
+    for (int ks = 0; ks < kBlk / 16; ++ks) {
+      uint32_t pa[4];
+      const int row = (lane & 7) + 8 * ((lane >> 3) & 1);
+      ldsm_x4(pa, Ps + swz(row, 2 * ks + (lane >> 4), kBlk * 2));
+      const int vrow = 16 * ks + (lane & 7) + 8 * ((lane >> 3) & 1);
+      if constexpr (D == 128) {
+        uint32_t vb[4];
+        ldsm_x4_t(vb, Vs + kv_off(vrow, 2 * warp + (lane >> 4)));
+        mma_bf16(acc[0], pa, vb[0], vb[1]);
+        mma_bf16(acc[1], pa, vb[2], vb[3]);
+      } else {
+        uint32_t vb[2];
+        ldsm_x2_t(vb, Vs + kv_off(vrow, warp));
+        mma_bf16(acc[0], pa, vb[0], vb[1]);
       }
     }
   }
-  cluster_arrive_release();  // every partial has been stored into its owner ...
-  cluster_wait();            // ... and after this no CTA touches another's shared memory
+  __syncthreads();  // (lloc is complete)
 
-  // merge: this CTA's 1/16 of the G x D outputs, from its own shared memory
-  const int per = G * D / kCL;
+  // ---- partials to the CTAs that own each output slice -------------------------------------
+  if (tid == 0) tc::mbar_arrive_expect_tx(&bar[3], (uint32_t)(kCL * (G * 8 + per * 4)));
+  if (tid < kCL * G) {  // (m, l) of every head into every CTA, row `rank`
+    const int peer = tid / G, h = tid - peer * G;
+    const float2 ml = keep ? make_float2(rloc[h], lloc[h]) : make_float2(-INFINITY, 0.f);
+    st_async(map_rank(ml_in + rank * kRows + h, peer), ml, map_rank(&bar[3], peer));
+  }
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) {
+    const int d = (D == 128 ? 16 * warp : 8 * warp) + 8 * nt + 2 * (lane & 3);
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+      const int row = r0 + 8 * half;
+      if (row < G) {
+        const int e = row * D + d;
+        const int owner = e / per;  // (per is even, so both elements share the owner)
+        st_async(map_rank(acc_in + rank * per + (e - owner * per), owner),
+                 make_float2(acc[nt][2 * half], acc[nt][2 * half + 1]), map_rank(&bar[3], owner));
+      }
+    }
+  }
+  tc::mbar_wait(&bar[3], 0, &xabort, kWaitBudget);
+  if (tid == 0 && xabort) g_blasst_decode_status = 1;
+
+  // ---- merge this CTA's slice by log-sum-exp ------------------------------------------------
   for (int le = tid; le < per; le += kThreads) {
     const int e = rank * per + le;
     const int h = e / D, d = e - h * D;
-    float pm[kCL], pl[kCL], pa[kCL];
-#pragma unroll
-    for (int c = 0; c < kCL; ++c) {
-      const float2 ml = sm.recv_ml[c][h];
-      pm[c] = ml.x;
-      pl[c] = ml.y;
-      pa[c] = sm.recv_acc[c][le];
-    }
     float M = -INFINITY;
 #pragma unroll
-    for (int c = 0; c < kCL; ++c) M = fmaxf(M, pm[c]);
-    float L = 0.f, O = 0.f;
+    for (int c = 0; c < kCL; ++c) M = fmaxf(M, ml_in[c * kRows + h].x);
+    float Lsum = 0.f, O = 0.f;
     if (M != -INFINITY) {
 #pragma unroll
       for (int c = 0; c < kCL; ++c) {
-        const float w = pm[c] == -INFINITY ? 0.f : ex2(pm[c] - M);
-        L = fmaf(pl[c], w, L);
-        O = fmaf(pa[c], w, O);
+        const float2 ml = ml_in[c * kRows + h];
+        const float w = ml.x == -INFINITY ? 0.f : ex2(ml.x - M);
+        Lsum = fmaf(ml.y, w, Lsum);
+        O = fmaf(acc_in[c * per + le], w, O);
       }
     }
     const size_t row = (size_t)b * Hq + (size_t)g * G + h;
-    o[row * D + d] = __float2bfloat16_rn(L > 0.f ? O / L : 0.f);
-    if (d == 0 && lse) lse[row] = L > 0.f ? (M + log2f(L)) * kLn2 : -INFINITY;
+    p.o[row * D + d] = __float2bfloat16_rn(Lsum > 0.f ? O / Lsum : 0.f);
+    if (d == 0 && p.lse) p.lse[row] = Lsum > 0.f ? (M + log2f(Lsum)) * kLn2 : -INFINITY;
   }
-  if (rank == 0 && tid == 0 && skip_bits) skip_bits[unit] = skipped;
+  if (rank == 0 && tid == 0 && p.skip_bits) p.skip_bits[unit] = skipped;
 }
 
 template <int D>
 cudaError_t launch_d(const DecodeBlasstArgs& a, cudaStream_t stream) {
   auto kernel = decode_blasst_kernel<D>;
+  Params p{};
+  if (!kv_tensor_maps(a.k, a.v, D, a.T_cap, a.B * a.Hkv, &p.tmk, &p.tmv)) return cudaErrorInvalidValue;
+  p.q = static_cast<const __nv_bfloat16*>(a.q);
+  p.Hkv = a.Hkv;
+  p.G = a.G;
+  p.T_cap = a.T_cap;
+  p.seqlens = a.seqlens;
+  p.idx = a.idx;
+  p.nsel = a.nsel;
+  p.topk = a.topk;
+  p.scale2 = a.scale * kLog2e;
+  p.log2_lambda = a.lambda > 0.f ? log2f(a.lambda) : -INFINITY;
+  p.o = static_cast<__nv_bfloat16*>(a.o);
+  p.lse = a.lse;
+  p.skip_bits = a.skip_bits;
+  const int smem = Lay<D>::kTotal + 1024;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(kCL, a.Hkv, a.B);
   cfg.blockDim = dim3(kThreads, 1, 1);
-  cfg.dynamicSmemBytes = 0;
+  cfg.dynamicSmemBytes = (size_t)smem;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -293,30 +387,35 @@ cudaError_t launch_d(const DecodeBlasstArgs& a, cudaStream_t stream) {
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  // the cluster attribute and the occupancy check depend only on the kernel and its fixed
-  // block shape: done once per device (the first launch on a device runs it, racing host
+  // the attributes and the occupancy check depend only on the kernel and its fixed block
+  // shape: done once per device (the first launch on a device runs it, racing host
   // threads wait for it), so that a launch costs only the launch
   static DeviceOnce check_once;
   const cudaError_t check_err = check_once.run([&]() {
-    cudaError_t err = cudaFuncSetAttribute(kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    cudaError_t err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (err == cudaSuccess) err = cudaFuncSetAttribute(kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
     int nclusters = 0;
     if (err == cudaSuccess) err = cudaOccupancyMaxActiveClusters(&nclusters, kernel, &cfg);
     if (err == cudaSuccess && nclusters == 0) err = cudaErrorInvalidConfiguration;
     return err;
   });
   if (check_err != cudaSuccess) return check_err;
-  const float scale2 = a.scale * kLog2e;
-  const float log2_lambda = a.lambda > 0.f ? log2f(a.lambda) : -INFINITY;
-  return cudaLaunchKernelEx(&cfg, kernel, static_cast<const __nv_bfloat16*>(a.q),
-                            static_cast<const __nv_bfloat16*>(a.k), static_cast<const __nv_bfloat16*>(a.v),
-                            a.Hkv, a.G, a.T_cap, a.seqlens, a.idx, a.nsel, a.topk, scale2, log2_lambda,
-                            static_cast<__nv_bfloat16*>(a.o), a.lse, a.skip_bits);
+  return cudaLaunchKernelEx(&cfg, kernel, p);
 }
 
 }  // namespace
 
 cudaError_t launch_decode_blasst(const DecodeBlasstArgs& a, cudaStream_t stream) {
   return a.D == 128 ? launch_d<128>(a, stream) : launch_d<64>(a, stream);
+}
+
+cudaError_t read_decode_blasst_status(int* status, bool reset) {
+  cudaError_t err = cudaMemcpyFromSymbol(status, g_blasst_decode_status, sizeof(int));
+  if (err == cudaSuccess && reset) {
+    const int zero = 0;
+    err = cudaMemcpyToSymbol(g_blasst_decode_status, &zero, sizeof(int));
+  }
+  return err;
 }
 
 }  // namespace lsa

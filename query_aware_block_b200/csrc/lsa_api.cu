@@ -394,7 +394,10 @@ int lsa_device_status(int* status, int reset) {
   int bq = 0;
   st = cuda_status(lsa::read_blockquery_status(&bq, reset != 0));
   if (st != LSA_OK) return st;
-  *status = prefill | decode | bq;
+  int dbl = 0;
+  st = cuda_status(lsa::read_decode_blasst_status(&dbl, reset != 0));
+  if (st != LSA_OK) return st;
+  *status = prefill | decode | bq | dbl;
   return LSA_OK;
 }
 

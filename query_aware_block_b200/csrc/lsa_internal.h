@@ -83,6 +83,7 @@ struct DecodeBlasstArgs {
   uint32_t* skip_bits;
 };
 cudaError_t launch_decode_blasst(const DecodeBlasstArgs& a, cudaStream_t stream);
+cudaError_t read_decode_blasst_status(int* status, bool reset);
 
 // NSA's compressed and sliding-window branches (fixed pool, constant gates).
 cudaError_t launch_nsa_compress(const void* k, const void* v, int B, int Hkv, int T_cap, int D,

@@ -74,5 +74,17 @@ def max_abs_beyond_bf16(gpu, ref):
     return float(d.max()) if d.numel() else 0.0
 
 
+def max_abs_vs_bf16(gpu, ref):
+    """max |gpu - RNE_bf16(ref)|: a bf16 output against the exact value rounded to bf16 the
+    way the kernels round (nearest even).  Where |ref| <= 1 a bf16 ulp is at most 2^-7, so
+    the plain 1e-2 bound still leaves room for one rounding step either way."""
+    a = gpu.double().cpu()
+    b = ref.to(torch.float32).to(torch.bfloat16).double().cpu()
+    both_inf = torch.isinf(a) & torch.isinf(b) & (torch.sign(a) == torch.sign(b))
+    d = (a - b).abs()
+    d[both_inf] = 0.0
+    return float(d.max()) if d.numel() else 0.0
+
+
 def nsel_of(idx):
     return (idx >= 0).sum(-1).to(torch.int32)

@@ -12,7 +12,7 @@ import torch
 
 import oracle
 import synth
-from tests.parity import LSE_TOL, TOL, max_abs, max_abs_beyond_bf16
+from tests.parity import LSE_TOL, TOL, max_abs, max_abs_vs_bf16
 
 pytestmark = pytest.mark.gpu
 
@@ -52,7 +52,7 @@ def _check(q, k, v, sl, idx, nsel, lam, o, lse, bits, where):
                     gap = float(ref["gap"][b, g, s])
                     assert abs(gap - ln_l) <= BAND, f"{where}: b{b} g{g} slot {s} gap {gap}"
     forced = oracle.decode_blasst(q, k, v, sl, idx, nsel, lam, forced_bits=bits)
-    assert max_abs_beyond_bf16(o, forced["o"]) <= TOL[torch.bfloat16], where
+    assert max_abs_vs_bf16(o, forced["o"]) <= TOL[torch.bfloat16], where
     assert max_abs(lse, forced["lse"]) <= LSE_TOL[torch.bfloat16], where
     return ref
 

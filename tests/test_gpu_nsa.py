@@ -10,7 +10,7 @@ import torch
 
 import oracle
 import synth
-from tests.parity import LSE_TOL, TOL, max_abs, max_abs_beyond_bf16
+from tests.parity import LSE_TOL, TOL, max_abs, max_abs_beyond_bf16, max_abs_vs_bf16
 
 pytestmark = pytest.mark.gpu
 
@@ -97,7 +97,7 @@ def _check(case, gates, window, o, lw, lc, idx, o_slc, with_slc=True, where=""):
     r = oracle.nsa_decode(case.q, case.k, case.v, case.seqlens, gates=gates, window=window,
                           idx=idx)
     ref = r["o"] if with_slc else gates[0] * r["o_cmp"] + gates[2] * r["o_win"]
-    assert max_abs_beyond_bf16(o, ref) <= TOL[torch.bfloat16], where
+    assert max_abs_vs_bf16(o, ref) <= TOL[torch.bfloat16], where
     assert max_abs(lw, r["lse_win"]) <= LSE_TOL[torch.bfloat16], where
     assert max_abs(lc, r["lse_cmp"]) <= LSE_TOL[torch.bfloat16], where
 
