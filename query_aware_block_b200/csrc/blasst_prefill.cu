@@ -81,7 +81,7 @@ struct Bars {
   uint64_t s_full[2];
   uint64_t p_full[2];
   uint64_t vote[2];           // one arrival per softmax warp and tile: the skip vote is in
-  uint64_t o_done;
+  uint64_t o_done[2];         // P.V number n completes on o_done[n & 1]
   uint32_t tmem;
   int nonneg[2];              // the last tile (of this buffer) some softmax warp kept
   int abort;
@@ -124,7 +124,8 @@ __global__ void __launch_bounds__(kThreads, 2) blasst_prefill_kernel(const __gri
       tc::mbar_init(&bars->vote[s], 4);
       bars->nonneg[s] = -1;
     }
-    tc::mbar_init(&bars->o_done, 1);
+    tc::mbar_init(&bars->o_done[0], 1);
+    tc::mbar_init(&bars->o_done[1], 1);
     bars->abort = 0;
     tc::fence_mbar_init();
   }
@@ -204,7 +205,7 @@ __global__ void __launch_bounds__(kThreads, 2) blasst_prefill_kernel(const __gri
           tc::mma_ts(tmem + kColO, tmem + (uint32_t)buf * 64u + (uint32_t)kk * 8u, bd, idesc_pv,
                      (pv_count > 0 || kk > 0) ? 1u : 0u);
         }
-        tc::mma_commit(&bars->o_done);
+        tc::mma_commit(&bars->o_done[pv_count & 1]);
         ++pv_count;
       } else if (!tc::mbar_wait(&bars->v_full[s], (j / kStages) & 1, abort, kWaitBudget)) {
         break;
@@ -219,7 +220,7 @@ __global__ void __launch_bounds__(kThreads, 2) blasst_prefill_kernel(const __gri
     const bool row_ok = i < p.L;
     const uint32_t lane_addr = tmem + ((uint32_t)(32 * (warp - 4)) << 16);
     float m_run = -INFINITY, m_used = -INFINITY, l = 0.f;
-    int pv_issued = 0, pv_observed = 0;
+    int pv_issued = 0;
     uint32_t skipmask = 0;
     int nskipped = 0;
     bool failed = false;
@@ -249,24 +250,22 @@ __global__ void __launch_bounds__(kThreads, 2) blasst_prefill_kernel(const __gri
       // cuts this tile; scaled to log2 units after the max (scale2 > 0 commutes with it)
       const int t0 = j * kBN;
       const int lim = min(i, p.L - 1) - t0;  // keys t0 + c with c <= lim are visible
-      // (8 independent partial maxima: a single chain of 64 dependent max operations would
-      // dominate the softmax latency)
+      // (8 independent chains of three-input maxima: a single chain of 64 dependent max
+      // operations would dominate the softmax latency)
+      if (!(row_ok && lim >= kBN - 1)) {
+#pragma unroll
+        for (int c = 0; c < kBN; ++c)
+          sr[c] = (row_ok && c <= lim) ? sr[c] : __float_as_uint(-INFINITY);
+      }
       float mx8[8];
 #pragma unroll
-      for (int e = 0; e < 8; ++e) mx8[e] = -INFINITY;
-      if (row_ok && lim >= kBN - 1) {
-#pragma unroll
-        for (int c = 0; c < kBN; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], __uint_as_float(sr[c]));
-      } else {
-#pragma unroll
-        for (int c = 0; c < kBN; ++c) {
-          const float v = (row_ok && c <= lim) ? __uint_as_float(sr[c]) : -INFINITY;
-          sr[c] = __float_as_uint(v);
-          mx8[c & 7] = fmaxf(mx8[c & 7], v);
-        }
+      for (int e = 0; e < 8; ++e) {
+        float mk = fmax3f(__uint_as_float(sr[e]), __uint_as_float(sr[e + 8]), __uint_as_float(sr[e + 16]));
+        mk = fmax3f(mk, __uint_as_float(sr[e + 24]), __uint_as_float(sr[e + 32]));
+        mk = fmax3f(mk, __uint_as_float(sr[e + 40]), __uint_as_float(sr[e + 48]));
+        mx8[e] = fmaxf(mk, __uint_as_float(sr[e + 56]));
       }
-      const float rmax = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                               fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+      const float rmax = fmaxf(fmax3f(mx8[0], mx8[1], mx8[2]), fmax3f(fmax3f(mx8[3], mx8[4], mx8[5]), mx8[6], mx8[7]));
       const float r = rmax * p.scale2;
       // the skip vote: every row negligible (absent rows and rows without a visible key agree)
       const bool negligible = !row_ok || r == -INFINITY || (m_run != -INFINITY && (r - m_run) < p.log2lam);
@@ -310,32 +309,40 @@ __global__ void __launch_bounds__(kThreads, 2) blasst_prefill_kernel(const __gri
 #pragma unroll
           for (int c = 0; c < 32; ++c) pk[c] = 0u;
         } else {
-          // p = 2^(scale2 * s - base), the scale folded into one FMA per element; the row
-          // sum in 4 independent partial sums
-          const float nb = -base;
-          float rs4[4] = {0.f, 0.f, 0.f, 0.f};
+          // p = 2^(scale2 * s - base): the scale folded into one two-wide FMA per pair of
+          // elements; the row sum in 4 independent two-wide partial sums
+          const unsigned long long sc2 = f2_pack(p.scale2, p.scale2), nb2 = f2_pack(-base, -base);
+          unsigned long long rs2[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) rs2[e] = 0ull;
 #pragma unroll
           for (int c = 0; c < 32; ++c) {
-            const float p0 = ex2(fmaf(__uint_as_float(sr[2 * c]), p.scale2, nb));
-            const float p1 = ex2(fmaf(__uint_as_float(sr[2 * c + 1]), p.scale2, nb));
-            rs4[c & 3] += p0 + p1;
+            float x0, x1;
+            f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[2 * c]), __uint_as_float(sr[2 * c + 1])), sc2, nb2), x0, x1);
+            const float p0 = ex2(x0), p1 = ex2(x1);
+            rs2[c & 3] = f2_add(rs2[c & 3], f2_pack(p0, p1));
             pk[c] = pack_bf16x2(p0, p1);
           }
-          rs = (rs4[0] + rs4[1]) + (rs4[2] + rs4[3]);
+          float a0, a1;
+          f2_unpack(f2_add(f2_add(rs2[0], rs2[1]), f2_add(rs2[2], rs2[3])), a0, a1);
+          rs = a0 + a1;
         }
         l = l * alpha + rs;
         tc::tmem_st32(lane_addr + (uint32_t)buf * 64u, pk);
         tc::tmem_st_wait();
-        // the previous P.V must be complete: O is then stable, and at most one O update is
-        // ever outstanding, which keeps the o_done phase parity unambiguous
-        if (pv_issued > pv_observed) {
-          if (!__all_sync(0xffffffffu, tc::mbar_wait(&bars->o_done, pv_observed & 1, abort, kWaitBudget))) {
+        const bool warp_resc = __any_sync(0xffffffffu, resc);
+        if (warp_resc && pv_issued > 0) {
+          // O is rescaled in place, so the last P.V issued (number pv_issued - 1) must be
+          // complete (tcgen05 work completes in issue order: so are all earlier ones).  It
+          // is the ((pv_issued - 1) >> 1)-th completion of o_done[(pv_issued - 1) & 1], and
+          // that barrier cannot complete again before this warp releases a later tile, so
+          // the parity wait is unambiguous.  Without a rescale nothing waits for O.
+          const int n = pv_issued - 1;
+          if (!__all_sync(0xffffffffu, tc::mbar_wait(&bars->o_done[n & 1], (uint32_t)((n >> 1) & 1), abort,
+                                                     kWaitBudget))) {
             failed = true;
             break;
           }
-          ++pv_observed;
-        }
-        if (__any_sync(0xffffffffu, resc) && pv_issued > 0) {
           tc::fence_after_sync();
 #pragma unroll
           for (int q4 = 0; q4 < 4; ++q4) {
@@ -357,14 +364,11 @@ __global__ void __launch_bounds__(kThreads, 2) blasst_prefill_kernel(const __gri
         skipmask = 0;
       }
     }
-    if (!failed) {
-      while (pv_observed < pv_issued) {
-        if (!__all_sync(0xffffffffu, tc::mbar_wait(&bars->o_done, pv_observed & 1, abort, kWaitBudget))) {
-          failed = true;
-          break;
-        }
-        ++pv_observed;
-      }
+    if (!failed && pv_issued > 0) {  // the last P.V (and with it every earlier one) is complete
+      const int n = pv_issued - 1;
+      if (!__all_sync(0xffffffffu, tc::mbar_wait(&bars->o_done[n & 1], (uint32_t)((n >> 1) & 1), abort,
+                                                 kWaitBudget)))
+        failed = true;
     }
     if (!failed) {
       tc::fence_after_sync();
