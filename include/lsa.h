@@ -471,11 +471,44 @@ LSA_API int lsa_blasst_prefill(const void* q, const void* k, const void* v, int 
 
 /*
  * lsa_device_status -- the device-side status word the kernels set when a bounded wait
- * runs out (LSA_DEVICE_TIMEOUT), 0 otherwise.  Synchronises with the device (it is a
+ * runs out (LSA_DEVICE_TIMEOUT; a debug-bounds build also ORs in LSA_DEVICE_BOUNDS), 0
+ * otherwise.  Synchronises with the device (it is a
  * debugging and failure-detection aid, not for the hot loop).  reset != 0 clears it.
  */
 #define LSA_DEVICE_TIMEOUT 1
+#define LSA_DEVICE_BOUNDS 2
 LSA_API int lsa_device_status(int* status, int reset);
+
+/*
+ * lsa_debug_bounds_code -- the first out-of-range device-side value found by a library built
+ * with LSA_DEBUG_BOUNDS (liblsa_debug.so), as (kind << 8) | site, 0 if none; reset != 0
+ * clears it.  Kinds: 1 a sequence length outside [0, T_cap], 2 a selection index outside
+ * [-1, NB_b), 3 a selection count outside [0, topk].  Sites: 1 summaries, 2 decode /
+ * selection, 3 BLASST decode, 4 NSA pool, 5 NSA branches, 6 KV append.  The debug build
+ * clamps such a value into range (every access stays in bounds, nothing traps) and also
+ * reports LSA_DEVICE_BOUNDS in lsa_device_status().  The release build checks nothing,
+ * sets *code = 0 and returns LSA_ERR_UNSUPPORTED.  Synchronises with the device.
+ */
+LSA_API int lsa_debug_bounds_code(int* code, int reset);
+
+/*
+ * Failure-handling controls, for tests of the bounded waits (no counterpart on the pages;
+ * they exist so that the timeout path can be exercised without faulting a GPU).
+ *
+ * lsa_debug_set_wait_budget -- the clock-cycle limit of every bounded wait inside the
+ *     kernels launched from now on (process-wide); cycles <= 0 restores the default
+ *     (4e9 cycles, about 2 s).  After a wait runs out a kernel leaves its loops, waits (with
+ *     a second, fixed 4e9-cycle limit) for its own copies and tensor-core work in flight and
+ *     for the bytes its cluster peers still owe it, frees its tensor memory, and sets the
+ *     status word; the launch's outputs are then undefined.
+ * lsa_debug_inject -- kind 0: normal operation (the default).  LSA_DEBUG_PREFILL_DROP_S:
+ *     the next lsa_blasst_prefill launches never signal their first S tile, so the softmax
+ *     warps' wait for it runs out and the timeout path above runs.  Process-wide.
+ * Both return LSA_OK, or LSA_ERR_INVALID_ARG for an unknown kind.
+ */
+#define LSA_DEBUG_PREFILL_DROP_S 1
+LSA_API int lsa_debug_set_wait_budget(long long cycles);
+LSA_API int lsa_debug_inject(int kind);
 
 #ifdef __cplusplus
 }

@@ -14,16 +14,19 @@ import os
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "liblsa.so")
+# LSA_LIBRARY=debug loads the bounds-checking build (liblsa_debug.so, see _build.py)
+LIB_PATH = os.path.join(_HERE, "liblsa_debug.so" if os.environ.get("LSA_LIBRARY") == "debug" else "liblsa.so")
 
 if not os.path.exists(LIB_PATH):
-    raise ImportError(f"{LIB_PATH} is missing: build it with `python query_aware_block_b200/_build.py`")
+    raise ImportError(f"{LIB_PATH} is missing: build it with `python query_aware_block_b200/_build.py`"
+                      + (" --debug-bounds" if LIB_PATH.endswith("_debug.so") else ""))
 
 _lib = ctypes.CDLL(LIB_PATH)
 
 LSA_OK, LSA_ERR_INVALID_ARG, LSA_ERR_UNSUPPORTED, LSA_ERR_CUDA, LSA_ERR_DEVICE_STATUS = 0, 1, 2, 3, 4
 LSA_F32, LSA_BF16 = 0, 1
 LSA_FLAG_PDL = 1
+LSA_DEBUG_PREFILL_DROP_S = 1
 BLK = 64
 
 EXPORTED = ("lsa_status_string", "lsa_last_cuda_error", "lsa_version", "lsa_build_summaries",
@@ -31,7 +34,8 @@ EXPORTED = ("lsa_status_string", "lsa_last_cuda_error", "lsa_version", "lsa_buil
             "lsa_sparse_attn_blockquery", "lsa_sparse_attn_blockquery_noalloc",
             "lsa_blasst_prefill", "lsa_device_status", "lsa_losa_classify",
             "lsa_blockquery_intra_merge", "lsa_sparse_attn_decode_blasst", "lsa_nsa_compress",
-            "lsa_nsa_branches", "lsa_select_blocks_weighted", "lsa_append_kv")
+            "lsa_nsa_branches", "lsa_select_blocks_weighted", "lsa_append_kv",
+            "lsa_debug_set_wait_budget", "lsa_debug_inject", "lsa_debug_bounds_code")
 
 _vp, _i, _f = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
 _lib.lsa_status_string.restype = ctypes.c_char_p
@@ -45,6 +49,9 @@ _lib.lsa_select_blocks.argtypes = [_vp, _i, _vp, _i, _i, _i, _i, _i, _vp, _i, _i
                                    _vp, _vp, _vp, _vp]
 _lib.lsa_sparse_attn_decode.argtypes = [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp, _i, _vp, _vp,
                                         _i, _f, _vp, _i, _i, _i, _vp, _vp, _vp, _i, _vp]
+_lib.lsa_debug_set_wait_budget.argtypes = [ctypes.c_longlong]
+_lib.lsa_debug_inject.argtypes = [_i]
+_lib.lsa_debug_bounds_code.argtypes = [_vp, _i]
 _lib.lsa_append_kv.argtypes = [_vp, _vp, _i, _i, _i, _i, _i, _vp, _vp, _vp, _i, _vp]
 _lib.lsa_blockquery_workspace_size.argtypes = [_i, _i, _i, _i, _i]
 _lib.lsa_blockquery_workspace_size.restype = ctypes.c_size_t
@@ -288,3 +295,21 @@ def lsa_device_status(reset=False) -> int:
 
 
 LSA_DEVICE_TIMEOUT = 1
+
+
+def lsa_debug_set_wait_budget(cycles: int) -> None:
+    """Clock-cycle limit of the kernels' bounded waits (tests only; <= 0 restores 4e9)."""
+    _check(_lib.lsa_debug_set_wait_budget(int(cycles)), "lsa_debug_set_wait_budget")
+
+
+def lsa_debug_bounds_code(reset=False) -> int:
+    """The first out-of-range device-side value a bounds-checking build found, as
+    (kind << 8) | site (0 if none); raises LsaError (LSA_ERR_UNSUPPORTED) in the release build."""
+    out = ctypes.c_int(0)
+    _check(_lib.lsa_debug_bounds_code(ctypes.byref(out), int(bool(reset))), "lsa_debug_bounds_code")
+    return out.value
+
+
+def lsa_debug_inject(kind: int) -> None:
+    """Fault injected into later launches (tests only; 0 = none)."""
+    _check(_lib.lsa_debug_inject(int(kind)), "lsa_debug_inject")

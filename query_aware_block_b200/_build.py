@@ -1,6 +1,11 @@
 """Build liblsa.so in-tree with nvcc for sm_100a (B200).
 
-    python query_aware_block_b200/_build.py [--verbose-ptxas] [--force]
+    python query_aware_block_b200/_build.py [--verbose-ptxas] [--force] [--debug-bounds]
+
+--debug-bounds builds liblsa_debug.so instead (objects in _build/debug, -DLSA_DEBUG_BOUNDS):
+the kernels check the device-side values that decide their addresses (sequence lengths,
+selection indices and counts), record the first one out of range in a status word
+(lsa_debug_bounds_code) and clamp it.  The package loads it when LSA_LIBRARY=debug.
 
 Run it as a script (or load it by path, as __graft_entry__.build() does): importing the
 package itself loads liblsa.so, which is what this script produces.
@@ -24,6 +29,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "liblsa.so")
+LIB_DEBUG = os.path.join(PKG, "liblsa_debug.so")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 
@@ -34,8 +40,8 @@ def _nvcc() -> str:
     raise RuntimeError("nvcc not found")
 
 
-def _flags(verbose_ptxas: bool):
-    f = ARCH + ["-O3", "-lineinfo", "-std=c++17", "--expt-relaxed-constexpr",
+def _flags(verbose_ptxas: bool, debug_bounds: bool = False):
+    f = ARCH + (["-DLSA_DEBUG_BOUNDS"] if debug_bounds else []) + ["-O3", "-lineinfo", "-std=c++17", "--expt-relaxed-constexpr",
                 "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",
                 "-I", os.path.join(ROOT, "include"), "-I", CSRC]
     if verbose_ptxas:
@@ -59,12 +65,15 @@ def _stale(obj: str, src: str) -> bool:
     return any(os.path.getmtime(d) > t for d in [src] + _headers())
 
 
-def build(force: bool = False, verbose_ptxas: bool = False, jobs: int | None = None) -> str:
-    os.makedirs(BUILD, exist_ok=True)
+def build(force: bool = False, verbose_ptxas: bool = False, jobs: int | None = None,
+          debug_bounds: bool = False) -> str:
+    build_dir = os.path.join(BUILD, "debug") if debug_bounds else BUILD
+    lib = LIB_DEBUG if debug_bounds else LIB
+    os.makedirs(build_dir, exist_ok=True)
     nvcc = _nvcc()
-    flags = _flags(verbose_ptxas)
+    flags = _flags(verbose_ptxas, debug_bounds)
     srcs = _sources()
-    objs = [os.path.join(BUILD, os.path.basename(s)[:-3] + ".o") for s in srcs]
+    objs = [os.path.join(build_dir, os.path.basename(s)[:-3] + ".o") for s in srcs]
     todo = [(s, o) for s, o in zip(srcs, objs) if force or verbose_ptxas or _stale(o, s)]
 
     def compile_one(so):
@@ -82,17 +91,18 @@ def build(force: bool = False, verbose_ptxas: bool = False, jobs: int | None = N
                 failed.append(s)
     if failed:
         raise RuntimeError("nvcc failed: " + ", ".join(os.path.basename(f) for f in failed))
-    if todo or not os.path.exists(LIB) or any(os.path.getmtime(o) > os.path.getmtime(LIB) for o in objs):
-        tmp = LIB + f".tmp{os.getpid()}"
+    if todo or not os.path.exists(lib) or any(os.path.getmtime(o) > os.path.getmtime(lib) for o in objs):
+        tmp = lib + f".tmp{os.getpid()}"
         subprocess.run([nvcc, *ARCH, "-shared", "-cudart", "static", "-o", tmp, *objs],
                        check=True)
-        os.replace(tmp, LIB)
-    return LIB
+        os.replace(tmp, lib)
+    return lib
 
 
 if __name__ == "__main__":
     ap = argparse.ArgumentParser()
     ap.add_argument("--force", action="store_true")
     ap.add_argument("--verbose-ptxas", action="store_true")
+    ap.add_argument("--debug-bounds", action="store_true")
     a = ap.parse_args()
-    print(build(force=a.force, verbose_ptxas=a.verbose_ptxas))
+    print(build(force=a.force, verbose_ptxas=a.verbose_ptxas, debug_bounds=a.debug_bounds))

@@ -27,7 +27,9 @@
 //             final normalisation uses the same base), and stores o and lse at the end.
 // The MMA for S_{j+2} is issued as soon as P_j is consumed, so Q K^T of the next tiles
 // overlaps the softmax of the current one.  Every mbarrier wait is clock-bounded; a
-// timeout raises a CTA-wide abort, every role leaves its loop, the TMEM is freed and the
+// timeout raises a CTA-wide abort and every role leaves its loop; the TMA producers then wait
+// (with a second bound) for the loads they issued, the MMA thread for the tensor-core work
+// it issued, so nothing lands in shared or tensor memory after the TMEM is freed, and the
 // device status word records the failure.
 #include <cuda.h>
 #include <math.h>
@@ -55,7 +57,6 @@ constexpr uint32_t kColO = 128;
 constexpr int kQBytes = kBM * kD * 2;        // 32 KB
 constexpr int kKVTileBytes = kBN * kD * 2;   // 16 KB per tensor
 constexpr int kStageBytes = 2 * kKVTileBytes;
-constexpr long long kWaitBudget = 4000000000LL;  // clock cycles (about 2 s)
 constexpr float kRescaleLog2 = 8.0f;             // rescale O when the max grew by > 2^8
 constexpr int kDeviceTimeout = 1;
 
@@ -70,6 +71,8 @@ struct alignas(64) PrefillParams {
   int Hq, Hkv, L, nqt, words;
   float scale2;    // softmax scale * log2(e)
   float log2lam;   // log2(lambda), -inf for lambda = 0
+  long long budget;  // clock-cycle limit of every bounded wait
+  int drop_s;        // test injection: the first S tile is never signalled
 };
 
 struct Bars {
@@ -82,6 +85,7 @@ struct Bars {
   uint64_t p_full[2];
   uint64_t vote[2];           // one arrival per softmax warp and tile: the skip vote is in
   uint64_t o_done[2];         // P.V number n completes on o_done[n & 1]
+  uint64_t drain;             // after a timeout: every tcgen05 operation issued has completed
   uint32_t tmem;
   int nonneg[2];              // the last tile (of this buffer) some softmax warp kept
   int abort;
@@ -126,6 +130,7 @@ __global__ void __launch_bounds__(kThreads, 2) blasst_prefill_kernel(const __gri
     }
     tc::mbar_init(&bars->o_done[0], 1);
     tc::mbar_init(&bars->o_done[1], 1);
+    tc::mbar_init(&bars->drain, 1);
     bars->abort = 0;
     tc::fence_mbar_init();
   }
@@ -138,6 +143,7 @@ __global__ void __launch_bounds__(kThreads, 2) blasst_prefill_kernel(const __gri
   tc::fence_after_sync();
   const uint32_t tmem = bars->tmem;
 
+  int kv_issued = 0;  // (TMA producer lanes) loads issued into the ring
   if (warp == 0 && lane < 2) {
     // --------------------------------------------------------------- TMA producers ----
     // lane 0: Q, then the K tiles; lane 1: the V tiles (each ring on its own barriers)
@@ -156,11 +162,12 @@ __global__ void __launch_bounds__(kThreads, 2) blasst_prefill_kernel(const __gri
     uint64_t* empty = lane == 0 ? bars->k_empty : bars->v_empty;
     for (int j = 0; j < n_visit; ++j) {
       const int s = j % kStages;
-      if (j >= kStages && !tc::mbar_wait(&empty[s], ((j / kStages) - 1) & 1, abort, kWaitBudget)) break;
+      if (j >= kStages && !tc::mbar_wait(&empty[s], ((j / kStages) - 1) & 1, abort, p.budget)) break;
       unsigned char* dst = ring + s * kKVTileBytes;
       tc::mbar_arrive_expect_tx(&full[s], kKVTileBytes);
       tc::tma_load_3d(dst, map, 0, j * kBN, bg, &full[s]);
       tc::tma_load_3d(dst + kKVTileBytes / 2, map, 64, j * kBN, bg, &full[s]);
+      ++kv_issued;
     }
   } else if (warp == 1 && lane == 0) {
     // ----------------------------------------------------------------- MMA issuer ----
@@ -171,7 +178,7 @@ __global__ void __launch_bounds__(kThreads, 2) blasst_prefill_kernel(const __gri
     const uint32_t vring_addr = tc::smem_u32(Vring);
     auto issue_s = [&](int j) -> bool {
       const int s = j % kStages;
-      if (!tc::mbar_wait(&bars->k_full[s], (j / kStages) & 1, abort, kWaitBudget)) return false;
+      if (!tc::mbar_wait(&bars->k_full[s], (j / kStages) & 1, abort, p.budget)) return false;
       const uint32_t k_addr = kring_addr + s * kKVTileBytes;
       const uint32_t d = tmem + (uint32_t)(j & 1) * 64u;
 #pragma unroll
@@ -181,21 +188,21 @@ __global__ void __launch_bounds__(kThreads, 2) blasst_prefill_kernel(const __gri
         const uint64_t bd = tc::smem_desc_sw128(k_addr + (ks >> 2) * (kKVTileBytes / 2) + (ks & 3) * 32, 16, 1024);
         tc::mma_ss(d, ad, bd, idesc_qk, ks > 0 ? 1u : 0u);
       }
-      tc::mma_commit(&bars->s_full[j & 1]);
+      if (!(p.drop_s && j == 0)) tc::mma_commit(&bars->s_full[j & 1]);
       tc::mma_commit(&bars->k_empty[s]);  // K_j is no longer needed once S_j is done
       return true;
     };
-    bool ok = tc::mbar_wait(&bars->q_full, 0, abort, kWaitBudget);
+    bool ok = tc::mbar_wait(&bars->q_full, 0, abort, p.budget);
     if (ok) ok = issue_s(0);
     if (ok && n_visit > 1) ok = issue_s(1);
     int pv_count = 0;
     for (int j = 0; ok && j < n_visit; ++j) {
       const int buf = j & 1, s = j % kStages;
-      if (!tc::mbar_wait(&bars->p_full[buf], (j >> 1) & 1, abort, kWaitBudget)) break;
+      if (!tc::mbar_wait(&bars->p_full[buf], (j >> 1) & 1, abort, p.budget)) break;
       tc::fence_after_sync();
       const bool kept = reinterpret_cast<volatile int*>(bars->nonneg)[buf] == j;
       if (kept) {
-        if (!tc::mbar_wait(&bars->v_full[s], (j / kStages) & 1, abort, kWaitBudget)) break;
+        if (!tc::mbar_wait(&bars->v_full[s], (j / kStages) & 1, abort, p.budget)) break;
         const uint32_t v_addr = vring_addr + s * kKVTileBytes;
 #pragma unroll
         for (int kk = 0; kk < kBN / 16; ++kk) {
@@ -207,12 +214,13 @@ __global__ void __launch_bounds__(kThreads, 2) blasst_prefill_kernel(const __gri
         }
         tc::mma_commit(&bars->o_done[pv_count & 1]);
         ++pv_count;
-      } else if (!tc::mbar_wait(&bars->v_full[s], (j / kStages) & 1, abort, kWaitBudget)) {
+      } else if (!tc::mbar_wait(&bars->v_full[s], (j / kStages) & 1, abort, p.budget)) {
         break;
       }
       tc::mma_commit(&bars->v_empty[s]);  // (a skipped tile's V is released unread)
       if (j + 2 < n_visit && !issue_s(j + 2)) break;
     }
+
   } else if (warp >= 4) {
     // ------------------------------------------------------------------- softmax ----
     const int row = tid - 128;
@@ -229,7 +237,7 @@ __global__ void __launch_bounds__(kThreads, 2) blasst_prefill_kernel(const __gri
     // outcome is made warp-uniform, so a failure lets each warp leave on its own.
     for (int j = 0; j < n_visit; ++j) {
       const int buf = j & 1;
-      if (!__all_sync(0xffffffffu, tc::mbar_wait(&bars->s_full[buf], (j >> 1) & 1, abort, kWaitBudget))) {
+      if (!__all_sync(0xffffffffu, tc::mbar_wait(&bars->s_full[buf], (j >> 1) & 1, abort, p.budget))) {
         failed = true;
         break;
       }
@@ -279,7 +287,7 @@ __global__ void __launch_bounds__(kThreads, 2) blasst_prefill_kernel(const __gri
       if (lane == 0) tc::mbar_arrive(&bars->vote[buf]);
       bool skip = false;
       if (warp_neg) {
-        if (!__all_sync(0xffffffffu, tc::mbar_wait(&bars->vote[buf], (j >> 1) & 1, abort, kWaitBudget))) {
+        if (!__all_sync(0xffffffffu, tc::mbar_wait(&bars->vote[buf], (j >> 1) & 1, abort, p.budget))) {
           failed = true;
           break;
         }
@@ -339,7 +347,7 @@ __global__ void __launch_bounds__(kThreads, 2) blasst_prefill_kernel(const __gri
           // the parity wait is unambiguous.  Without a rescale nothing waits for O.
           const int n = pv_issued - 1;
           if (!__all_sync(0xffffffffu, tc::mbar_wait(&bars->o_done[n & 1], (uint32_t)((n >> 1) & 1), abort,
-                                                     kWaitBudget))) {
+                                                     p.budget))) {
             failed = true;
             break;
           }
@@ -367,7 +375,7 @@ __global__ void __launch_bounds__(kThreads, 2) blasst_prefill_kernel(const __gri
     if (!failed && pv_issued > 0) {  // the last P.V (and with it every earlier one) is complete
       const int n = pv_issued - 1;
       if (!__all_sync(0xffffffffu, tc::mbar_wait(&bars->o_done[n & 1], (uint32_t)((n >> 1) & 1), abort,
-                                                 kWaitBudget)))
+                                                 p.budget)))
         failed = true;
     }
     if (!failed) {
@@ -401,7 +409,24 @@ __global__ void __launch_bounds__(kThreads, 2) blasst_prefill_kernel(const __gri
   }
 
   __syncthreads();
-  if (tid == 0 && bars->abort) g_device_status = kDeviceTimeout;
+  // every role has left its loop: after a timeout, nothing may land in shared or tensor
+  // memory once the CTA has gone, so the producers wait (bounded) for the last load issued
+  // into every stage of their ring (earlier ones into a stage completed before it was
+  // reused) and the MMA thread for all the tensor-core work it issued
+  const bool aborted = bars->abort != 0;
+  if (aborted) {
+    if (warp == 0 && lane < 2) {
+      uint64_t* full = lane == 0 ? bars->k_full : bars->v_full;
+      for (int j = kv_issued - kStages < 0 ? 0 : kv_issued - kStages; j < kv_issued; ++j)
+        tc::mbar_drain(&full[j % kStages], (uint32_t)((j / kStages) & 1), kDrainBudget);
+      if (lane == 0) tc::mbar_drain(&bars->q_full, 0, kDrainBudget);
+    } else if (warp == 1 && lane == 0) {
+      tc::mma_commit(&bars->drain);
+      tc::mbar_drain(&bars->drain, 0, kDrainBudget);
+    }
+    __syncthreads();
+  }
+  if (tid == 0 && aborted) g_device_status = kDeviceTimeout;
   if (warp == 2) {
     tc::fence_after_sync();
     tc::tmem_dealloc(tmem, kTmemCols);
@@ -433,6 +458,8 @@ cudaError_t launch_blasst_prefill(const PrefillArgs& a, cudaStream_t stream) {
   p.words = ((a.L + kBN - 1) / kBN + 31) / 32;
   p.scale2 = a.scale * kLog2e;
   p.log2lam = a.lambda > 0.f ? log2f(a.lambda) : -INFINITY;
+  p.budget = wait_budget();
+  p.drop_s = debug_inject() == 1 ? 1 : 0;
   // the shared memory attribute applies to the current device: set once per device
   static DeviceOnce attr_once;
   const cudaError_t err = attr_once.run([] {

@@ -26,7 +26,9 @@
 //     cluster barrier every CTA merges a 1/CL slice of the outputs by log-sum-exp (all
 //     loads issued before use).  Stable rows are copied from the cache; rank 0 writes the
 //     union list.
-//   Every mbarrier wait is bounded (about 2 s); a timeout sets a device status word.
+//   Every mbarrier wait is bounded (about 2 s); after a timeout the CTA waits (bounded) for
+//   its copies and its peers' list bytes still in flight before it exits, and a device status
+//   word records the failure.
 #include <math.h>
 
 #include <mutex>
@@ -45,7 +47,6 @@ typedef unsigned long long u64;
 // Set when a bounded wait on a cross-CTA exchange or a bulk copy runs out (the launch's
 // outputs are then undefined); read and cleared by the host.
 __device__ int g_blockquery_status = 0;
-constexpr long long kWaitBudget = 4000000000LL;  // clock cycles (about 2 s)
 
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
@@ -85,6 +86,7 @@ struct alignas(64) BQParams {
   int NBp;         // prefix blocks
   FastDiv g_div;   // division by G
   FastDiv per_div; // division by per_max
+  long long budget;  // clock-cycle limit of every bounded wait
 };
 
 __host__ __device__ inline size_t al128(size_t x) { return (x + 127) & ~(size_t)127; }
@@ -256,7 +258,7 @@ __global__ void __launch_bounds__(kThreads, 2) blockquery_kernel(const __grid_co
       if (all_blocks || forced(j)) atomicOr(&ubits[j >> 5], 1u << (j & 31));
   }
   if (selecting) {
-    if (staged_rows > 0) tc::mbar_wait(&xbar[2], 0, &xabort, kWaitBudget);
+    if (staged_rows > 0) tc::mbar_wait(&xbar[2], 0, &xabort, p.budget);
     constexpr int kSeg = D / 4;  // summary floats per lane: lane l takes quarter l >> 3
     const int ta = lane & 7, q4 = lane >> 3;
     const float* grow = p.summ + (unit * (size_t)p.NB_cap + j0) * D + q4 * kSeg;
@@ -351,7 +353,7 @@ __global__ void __launch_bounds__(kThreads, 2) blockquery_kernel(const __grid_co
         const int peer = i / (kTokChunk * kLP), rem = i - peer * (kTokChunk * kLP);
         st_async(map_rank(rb + (size_t)rank * kTokChunk * kLP + rem, peer), top[rem], map_rank(&xbar[buf], peer));
       }
-      tc::mbar_wait(&xbar[buf], (uint32_t)((chunk_id >> 1) & 1), &xabort, kWaitBudget);
+      tc::mbar_wait(&xbar[buf], (uint32_t)((chunk_id >> 1) & 1), &xabort, p.budget);
       // every token's m best keys by a tournament over its CL sorted lists rb[c][a][*]: a
       // warp per token, lane l (and l + 16) holds the head of list l & 15; each round the
       // warp's maximum is a selected block and its list advances (keys are unique, so
@@ -375,7 +377,9 @@ __global__ void __launch_bounds__(kThreads, 2) blockquery_kernel(const __grid_co
           }
           if (lane == 0) {
             const int j = key_block(best);
-            atomicOr(&ubits[j >> 5], 1u << (j & 31));
+            // (a key is always a prefix block; the check keeps even a corrupted list -- after
+            // a timed-out exchange -- inside the bitmap)
+            if (j >= 0 && j < NBp) atomicOr(&ubits[j >> 5], 1u << (j & 31));
           }
         }
       }
@@ -383,7 +387,7 @@ __global__ void __launch_bounds__(kThreads, 2) blockquery_kernel(const __grid_co
     }
   } else if (staged_rows > 0) {
     __syncthreads();  // (thread 0's mbarrier initialisation first)
-    tc::mbar_wait(&xbar[2], 0, &xabort, kWaitBudget);  // no copy outlives its buffer's reuse
+    tc::mbar_wait(&xbar[2], 0, &xabort, p.budget);  // no copy outlives its buffer's reuse
   }
   __syncthreads();
   // the union as an ascending list (block-wide scan of the bitmap's popcounts)
@@ -468,7 +472,7 @@ __global__ void __launch_bounds__(kThreads, 2) blockquery_kernel(const __grid_co
 
     for (int i = 0; i < n_my; ++i) {
       const int it = c * n_my + i;
-      tc::mbar_wait(&xbar[3 + it % kStages], (uint32_t)((it / kStages) & 1), &xabort, kWaitBudget);
+      tc::mbar_wait(&xbar[3 + it % kStages], (uint32_t)((it / kStages) & 1), &xabort, p.budget);
       __syncthreads();
       const int j = ulist[rank + i * CL];
       const unsigned char* Ks = kv + (size_t)(it % kStages) * 2 * kv_tile;
@@ -597,7 +601,6 @@ __global__ void __launch_bounds__(kThreads, 2) blockquery_kernel(const __grid_co
   }
   cluster_arrive_release();
   cluster_wait();
-  if (tid == 0 && xabort) g_blockquery_status = 1;
 
   const int E = rows * D;
   const int chunk = (E + CL - 1) >> cl_log2;
@@ -666,6 +669,20 @@ __global__ void __launch_bounds__(kThreads, 2) blockquery_kernel(const __grid_co
     }
     if (p.union_cnt && tid == 0) p.union_cnt[unit] = U;
   }
+  // after a timeout (the outputs are then undefined) the CTA must not exit while its own
+  // copies, or list bytes its peers owe it, are in flight: wait for each (bounded, ignoring
+  // the abort) and record the failure
+  if (*reinterpret_cast<volatile int*>(&xabort)) {
+    if (staged_rows > 0) tc::mbar_drain(&xbar[2], 0, kDrainBudget);
+    if (selecting) {
+      const int nsel_chunks = (A + kTokChunk - 1) / kTokChunk;
+      for (int c = nsel_chunks - 2 < 0 ? 0 : nsel_chunks - 2; c < nsel_chunks; ++c)
+        tc::mbar_drain(&xbar[c & 1], (uint32_t)((c >> 1) & 1), kDrainBudget);
+    }
+    for (int i = issued - kStages < 0 ? 0 : issued - kStages; i < issued; ++i)
+      tc::mbar_drain(&xbar[3 + i % kStages], (uint32_t)((i / kStages) & 1), kDrainBudget);
+    g_blockquery_status = 1;
+  }
 }
 
 }  // namespace
@@ -703,6 +720,7 @@ cudaError_t launch_blockquery(const BlockQueryArgs& a, cudaStream_t stream) {
   p.rows_max = a.Tq * a.G;
   p.NBp = NBp;
   p.g_div = make_fastdiv((uint32_t)a.G);
+  p.budget = wait_budget();
   auto kernel = a.D == 128 ? blockquery_kernel<128> : blockquery_kernel<64>;
   // per head dim and device: the largest dynamic smem size set so far and the (cluster
   // size, smem) pairs found schedulable (thread-safe; see launch_cache.h)

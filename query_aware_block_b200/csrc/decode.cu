@@ -62,7 +62,6 @@ typedef unsigned long long u64;
 // Set when a bounded wait on a cross-CTA exchange runs out (the outputs of that launch are
 // then undefined); read and cleared by the host.
 __device__ int g_decode_status = 0;
-constexpr long long kWaitBudget = 4000000000LL;  // clock cycles (about 2 s)
 
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
@@ -100,6 +99,7 @@ struct alignas(64) Params {
   int lp;                 // length of an exchanged candidate list: max(16, m_pad)
   int chunk;              // output elements merged by one CTA (even)
   int pdl;                // launched as a programmatic dependent of the previous kernel
+  long long budget;       // clock-cycle limit of every bounded wait
   FastDiv chunk_div;      // division by chunk
 };
 
@@ -245,7 +245,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_cluster_kernel(const __gri
   const int g = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int G = p.G;
-  const int Tb = p.seqlens[b];
+  const int Tb = checked_range(p.seqlens[b], 0, p.T_cap, kBoundsSeqlen, kSiteDecode);
   const int NB = (Tb + kBlk - 1) / kBlk;
   constexpr bool kF32 = sizeof(T) == 4;
   constexpr int kRowBytesQ = D * (int)sizeof(T);
@@ -335,8 +335,9 @@ __global__ void __launch_bounds__(kThreads, 2) decode_cluster_kernel(const __gri
     for (int i = tid; i < known; i += kThreads)
       order[i] = all_blocks ? i : (i < p.n_sink ? i : NB - p.n_local + (i - p.n_sink));
   } else {
-    n_order = max(0, min(__ldcg(p.nsel_in + unit), p.topk));  // never past order[kMaxTopk]
-    for (int i = tid; i < n_order; i += kThreads) order[i] = __ldcg(p.idx_in + unit * p.topk + i);
+    n_order = max(0, min(checked_range(__ldcg(p.nsel_in + unit), 0, p.topk, kBoundsCount, kSiteDecode), p.topk));
+    for (int i = tid; i < n_order; i += kThreads)
+      order[i] = checked_range(__ldcg(p.idx_in + unit * p.topk + i), -1, NB - 1, kBoundsIndex, kSiteDecode);
   }
   auto known_block = [&](int i) {
     const int o = rank + i * CL;
@@ -385,13 +386,28 @@ __global__ void __launch_bounds__(kThreads, 2) decode_cluster_kernel(const __gri
   // (the barrier makes thread 0's mbarrier initialisation visible first)
   if (!scan && staged_rows > 0) {
     __syncthreads();
-    tc::mbar_wait(&xbar[2], 0, &xabort, kWaitBudget);
+    tc::mbar_wait(&xbar[2], 0, &xabort, p.budget);
   }
   if (MODE == MODE_FUSED) {
     while (issued < early_stages && issued < n_known && known_block(issued) != NB - 1) {
       issue_block(known_block(issued));
     }
   }
+  // After a timeout (the launch's outputs are then undefined) the CTA must not exit while
+  // copies it issued, or bytes its cluster peers owe it, are still in flight: every thread
+  // that sees the abort waits for each of them (bounded, ignoring the abort) and records
+  // the failure in the status word.
+  auto drain_on_abort = [&](bool lists, bool partials) {
+    if (!*reinterpret_cast<volatile int*>(&xabort)) return;
+    if (staged_rows > 0) tc::mbar_drain(&xbar[2], 0, kDrainBudget);
+    if (lists) tc::mbar_drain(&xbar[0], 0, kDrainBudget);
+    if (partials) tc::mbar_drain(&xbar[1], 0, kDrainBudget);
+    if constexpr (!kF32) {
+      for (int i = issued - kStages < 0 ? 0 : issued - kStages; i < issued; ++i)
+        tc::mbar_drain(&xbar[3 + i % kStages], (uint32_t)((i / kStages) & 1), kDrainBudget);
+    }
+    g_decode_status = 1;
+  };
   pdl_trigger();
   pdl_wait();
 
@@ -431,7 +447,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_cluster_kernel(const __gri
     }
     __syncthreads();
     // the summary rows (the barriers above ordered thread 0's mbarrier initialisation first)
-    if (staged_rows > 0) tc::mbar_wait(&xbar[2], 0, &xabort, kWaitBudget);
+    if (staged_rows > 0) tc::mbar_wait(&xbar[2], 0, &xabort, p.budget);
     // lane l of warp w scores rows 8w + (l >> 3) and 8w + 4 + (l >> 3) of a pass, taking
     // 16-byte chunks cs, cs + 8, ... (cs = l & 7): a quarter-warp reads 128 contiguous bytes
     // of one row (conflict-free), and every lane needs the same D / 8 summed-query values
@@ -542,7 +558,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_cluster_kernel(const __gri
       const int peer = t >> lp_log2, pos = t & (p.lp - 1);
       st_async(map_rank(all + rank * p.lp + pos, peer), top[pos], map_rank(&xbar[0], peer));
     }
-    tc::mbar_wait(&xbar[0], 0, &xabort, kWaitBudget);
+    tc::mbar_wait(&xbar[0], 0, &xabort, p.budget);
     if (p.lp == 16 && CL >= 2) {
       merge_tree16(all, work, CL, m, nf, order);
       // warp 0 ends the tree holding the final list: when this CTA's first block is a scored
@@ -593,8 +609,8 @@ __global__ void __launch_bounds__(kThreads, 2) decode_cluster_kernel(const __gri
   if (MODE == MODE_SELECT) write_indices();
   if (MODE == MODE_SELECT) {
     cp_async_wait<0>();  // no copy into shared memory outlives the CTA
-    if (tid == 0 && xabort) g_decode_status = 1;
     if (!started) cluster_wait();
+    drain_on_abort(scan, false);
     return;  // every byte this CTA receives has landed: no trailing barrier
   }
 
@@ -635,7 +651,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_cluster_kernel(const __gri
     if constexpr (kF32) {
       if (issued > i + 1) cp_async_wait<1>(); else cp_async_wait<0>();
     } else {
-      tc::mbar_wait(&xbar[3 + i % kStages], (uint32_t)((i / kStages) & 1), &xabort, kWaitBudget);
+      tc::mbar_wait(&xbar[3 + i % kStages], (uint32_t)((i / kStages) & 1), &xabort, p.budget);
     }
     __syncthreads();
     const int j = order[rank + i * CL];
@@ -645,7 +661,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_cluster_kernel(const __gri
       // V rows past the sequence (or all rows of an invalid j) hold whatever the cache
       // holds there: zero them, so that P = 0 never meets a NaN (ordered before P V by the
       // barrier after S)
-      const int nv = j < 0 ? 0 : min(kBlk, Tb - j * kBlk);
+      const int nv = (j < 0 || j >= NB) ? 0 : min(kBlk, Tb - j * kBlk);
       for (int id = tid; id < (kBlk - nv) * (D / 8); id += kThreads) {
         const int r = nv + id / (D / 8), c = id % (D / 8);
         *reinterpret_cast<uint4*>(const_cast<unsigned char*>(Vs) + kv_off(r, c)) = make_uint4(0u, 0u, 0u, 0u);
@@ -667,7 +683,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_cluster_kernel(const __gri
           s[r] = fmaf(q4.x, k4.x, fmaf(q4.y, k4.y, fmaf(q4.z, k4.z, fmaf(q4.w, k4.w, s[r]))));
         }
       }
-      const bool valid = j >= 0 && j * kBlk + tok < Tb;
+      const bool valid = j >= 0 && j < NB && j * kBlk + tok < Tb;
 #pragma unroll
       for (int r = 0; r < 4; ++r) Ss[(rg * 4 + r) * kSStride + tok] = valid ? s[r] * scale2 : -INFINITY;
     } else {
@@ -681,7 +697,8 @@ __global__ void __launch_bounds__(kThreads, 2) decode_cluster_kernel(const __gri
       }
       const int col = 8 * warp + 2 * (lane & 3);
       const int r0 = lane >> 2;
-      const bool v0 = j >= 0 && j * kBlk + col < Tb, v1 = j >= 0 && j * kBlk + col + 1 < Tb;
+      const bool jin = j >= 0 && j < NB;
+      const bool v0 = jin && j * kBlk + col < Tb, v1 = jin && j * kBlk + col + 1 < Tb;
       *reinterpret_cast<float2*>(Ss + r0 * kSStride + col) =
           make_float2(v0 ? s[0] * scale2 : -INFINITY, v1 ? s[1] * scale2 : -INFINITY);
       *reinterpret_cast<float2*>(Ss + (r0 + 8) * kSStride + col) =
@@ -843,8 +860,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_cluster_kernel(const __gri
       }
     }
   }
-  tc::mbar_wait(&xbar[1], 0, &xabort, kWaitBudget);
-  if (tid == 0 && xabort) g_decode_status = 1;
+  tc::mbar_wait(&xbar[1], 0, &xabort, p.budget);
 
   // ---- log-sum-exp merge of this CTA's slice, from its own shared memory ---------------
   {
@@ -879,6 +895,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_cluster_kernel(const __gri
             M == -INFINITY ? -INFINITY : (M + log2f(Lsum)) * kLn2;
     }
   }
+  drain_on_abort(scan, true);
 }
 
 // ---- host side --------------------------------------------------------------------------
@@ -936,6 +953,7 @@ cudaError_t launch_t(const DecodeArgs& a, cudaStream_t stream) {
     cfg.attrs = attr;
     cfg.numAttrs = (MODE == MODE_FUSED && a.pdl) ? 2 : 1;
     p.pdl = cfg.numAttrs == 2;
+    p.budget = wait_budget();
     {
       std::lock_guard<std::mutex> lock(rec.mu);
       err = rec.ensure_smem(dev, kernel, smem, true);
@@ -987,5 +1005,7 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream) {
   if (a.D == 128) return launch_mode<float, 128>(a, stream);
   return launch_mode<float, 64>(a, stream);
 }
+
+LSA_BOUNDS_READER(decode)
 
 }  // namespace lsa

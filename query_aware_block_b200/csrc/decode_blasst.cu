@@ -25,7 +25,8 @@
 // merges its 1/16 of the outputs by log-sum-exp from its own shared memory.  Every byte a
 // CTA receives is counted by its own mbarriers and waited for before it ends, so no CTA
 // leaves while a peer may still write into it.  Waits are bounded (about 2 s of clock); if
-// one runs out the launch's outputs are undefined and a status word records it.
+// one runs out the launch's outputs are undefined, the CTA waits (bounded) for what is still
+// in flight before it exits, and a status word records the failure.
 #include <math.h>
 
 #include "cluster.cuh"
@@ -41,7 +42,6 @@ constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
 constexpr int kCL = 16;      // CTAs per cluster = maximum selection slots
 constexpr int kRows = 16;    // query-head rows (G <= 16): the mma M dimension
-constexpr long long kWaitBudget = 4000000000LL;  // clock cycles (about 2 s)
 
 // Set when a bounded wait runs out (the outputs of that launch are then undefined); read
 // and cleared by the host.
@@ -61,6 +61,7 @@ struct Params {
   __nv_bfloat16* o;
   float* lse;
   uint32_t* skip_bits;
+  long long budget;  // clock-cycle limit of every bounded wait
 };
 
 // Shared-memory carve-up (byte offsets from the first 1024-byte boundary of the dynamic buffer).
@@ -112,9 +113,10 @@ __global__ void __launch_bounds__(kThreads) decode_blasst_kernel(const __grid_co
   const int per = G * D / kCL;  // output elements merged by one CTA (G * D is a multiple of 16)
 
   // the slot's block and the sequence length first (the K copy waits only for them)
-  const int ns = __ldg(p.nsel + unit);
-  const int jj = rank < p.topk ? __ldg(p.idx + unit * p.topk + rank) : -1;
-  const int T = __ldg(p.seqlens + b);
+  const int T = checked_range(__ldg(p.seqlens + b), 0, p.T_cap, kBoundsSeqlen, kSiteDecodeBlasst);
+  const int NBq = (T + kBlk - 1) / kBlk;
+  const int ns = checked_range(__ldg(p.nsel + unit), 0, p.topk, kBoundsCount, kSiteDecodeBlasst);
+  const int jj = rank < p.topk ? checked_range(__ldg(p.idx + unit * p.topk + rank), -1, NBq - 1, kBoundsIndex, kSiteDecodeBlasst) : -1;
   if (tid == 0) {
     for (int i = 0; i < 4; ++i) tc::mbar_init(&bar[i], 1);
     xabort = 0;
@@ -141,7 +143,8 @@ __global__ void __launch_bounds__(kThreads) decode_blasst_kernel(const __grid_co
   }
   // which slots hold a block (the same on every CTA)
   if (warp == 0) {
-    const int j2 = lane < p.topk && lane < kCL ? __ldg(p.idx + unit * p.topk + lane) : -1;
+    const int j2 = lane < p.topk && lane < kCL
+        ? checked_range(__ldg(p.idx + unit * p.topk + lane), -1, NBq - 1, kBoundsIndex, kSiteDecodeBlasst) : -1;
     const bool on = lane < ns && lane < kCL && j2 >= 0;
     const uint32_t bits = __ballot_sync(0xffffffffu, on);
     if (lane < kCL) slot_block[lane] = on ? j2 : -1;
@@ -167,7 +170,7 @@ __global__ void __launch_bounds__(kThreads) decode_blasst_kernel(const __grid_co
       const int row = (lane & 7) + 8 * ((lane >> 3) & 1);
       ldsm_x4(qa[ks], Qs + swz(row, 2 * ks + (lane >> 4), kRowBytes));
     }
-    tc::mbar_wait(&bar[0], 0, &xabort, kWaitBudget);
+    tc::mbar_wait(&bar[0], 0, &xabort, p.budget);
     float c4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
     for (int ks = 0; ks < D / 16; ks += 2) {
@@ -209,7 +212,7 @@ __global__ void __launch_bounds__(kThreads) decode_blasst_kernel(const __grid_co
     const int peer = tid / G, h = tid - peer * G;
     st_async(map_rank(rmax + rank * kRows + h, peer), rloc[h], map_rank(&bar[2], peer));
   }
-  if (nvalid > 0) tc::mbar_wait(&bar[2], 0, &xabort, kWaitBudget);
+  if (nvalid > 0) tc::mbar_wait(&bar[2], 0, &xabort, p.budget);
 
   // ---- the test for every slot (each CTA decides all of them; it acts on its own) ----------
   // Warp 0, lane s = slot s: per head, the running maximum before slot s is an exclusive
@@ -275,7 +278,7 @@ __global__ void __launch_bounds__(kThreads) decode_blasst_kernel(const __grid_co
     }
     // V rows past the sequence hold whatever the cache holds there: zero them once they
     // have landed, so that P = 0 never meets a NaN
-    tc::mbar_wait(&bar[1], 0, &xabort, kWaitBudget);
+    tc::mbar_wait(&bar[1], 0, &xabort, p.budget);
     for (int id = tid; id < (kBlk - nv) * (D / 8); id += kThreads) {
       const int r = nv + id / (D / 8), c = id % (D / 8);
       *reinterpret_cast<uint4*>(Vs + kv_off(r, c)) = make_uint4(0u, 0u, 0u, 0u);
@@ -329,8 +332,7 @@ __global__ void __launch_bounds__(kThreads) decode_blasst_kernel(const __grid_co
       }
     }
   }
-  tc::mbar_wait(&bar[3], 0, &xabort, kWaitBudget);
-  if (tid == 0 && xabort) g_blasst_decode_status = 1;
+  tc::mbar_wait(&bar[3], 0, &xabort, p.budget);
 
   // ---- merge this CTA's slice by log-sum-exp ------------------------------------------------
   for (int le = tid; le < per; le += kThreads) {
@@ -354,6 +356,16 @@ __global__ void __launch_bounds__(kThreads) decode_blasst_kernel(const __grid_co
     if (d == 0 && p.lse) p.lse[row] = Lsum > 0.f ? (M + log2f(Lsum)) * kLn2 : -INFINITY;
   }
   if (rank == 0 && tid == 0 && p.skip_bits) p.skip_bits[unit] = skipped;
+  // after a timeout (the outputs are then undefined) the CTA must not exit while its own
+  // copies, or bytes its peers owe it, are in flight: wait for each (bounded, ignoring the
+  // abort) and record the failure
+  if (*reinterpret_cast<volatile int*>(&xabort)) {
+    if (loaded) tc::mbar_drain(&bar[0], 0, kDrainBudget);
+    if (keep) tc::mbar_drain(&bar[1], 0, kDrainBudget);
+    if (nvalid > 0) tc::mbar_drain(&bar[2], 0, kDrainBudget);
+    tc::mbar_drain(&bar[3], 0, kDrainBudget);
+    g_blasst_decode_status = 1;
+  }
 }
 
 template <int D>
@@ -374,6 +386,7 @@ cudaError_t launch_d(const DecodeBlasstArgs& a, cudaStream_t stream) {
   p.o = static_cast<__nv_bfloat16*>(a.o);
   p.lse = a.lse;
   p.skip_bits = a.skip_bits;
+  p.budget = wait_budget();
   const int smem = Lay<D>::kTotal + 1024;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(kCL, a.Hkv, a.B);
@@ -417,5 +430,7 @@ cudaError_t read_decode_blasst_status(int* status, bool reset) {
   }
   return err;
 }
+
+LSA_BOUNDS_READER(decode_blasst)
 
 }  // namespace lsa

@@ -9,6 +9,7 @@
 // the newest block.  Launched itself with LSA_FLAG_PDL, it reads k_new / v_new only after
 // the previous kernel of the stream (the one that produced them) has completed.
 #include "cluster.cuh"
+#include "lsa_common.cuh"
 #include "lsa_internal.h"
 
 namespace lsa {
@@ -30,7 +31,7 @@ __global__ void __launch_bounds__(kThreads)
   const int cc = is_v ? c - n : c;
   const int u = cc / rows16, part = cc - u * rows16;
   const int b = u / Hkv;
-  const int t = seqlens[b] - 1;
+  const int t = checked_range(seqlens[b], 0, T_cap, kBoundsSeqlen, kSiteKvAppend) - 1;
   if (t < 0 || t >= T_cap) return;  // an empty sequence has no newest token
   const uint4 x = is_v ? v_new[cc] : k_new[cc];
   uint4* dst = (is_v ? v : k) + ((size_t)u * T_cap + t) * rows16 + part;
@@ -58,5 +59,7 @@ cudaError_t launch_kv_append(const void* k_new, const void* v_new, int elem_byte
                             static_cast<const uint4*>(v_new), Hkv, T_cap, rows16, n, seqlens,
                             static_cast<uint4*>(k), static_cast<uint4*>(v));
 }
+
+LSA_BOUNDS_READER(kv_append)
 
 }  // namespace lsa

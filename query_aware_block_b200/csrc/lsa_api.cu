@@ -3,8 +3,19 @@
 #include <math.h>
 #include <stdint.h>
 
+#include <atomic>
+
 #include "../../include/lsa.h"
 #include "lsa_internal.h"
+
+namespace lsa {
+namespace {
+std::atomic<long long> g_wait_budget{kDefaultWaitBudget};
+std::atomic<int> g_inject{0};
+}  // namespace
+long long wait_budget() { return g_wait_budget.load(std::memory_order_relaxed); }
+int debug_inject() { return g_inject.load(std::memory_order_relaxed); }
+}  // namespace lsa
 
 namespace {
 
@@ -384,6 +395,49 @@ int lsa_blasst_prefill(const void* q, const void* k, const void* v, int dtype, i
   return cuda_status(lsa::launch_blasst_prefill(a, stream));
 }
 
+int lsa_debug_set_wait_budget(long long cycles) {
+  lsa::g_wait_budget.store(cycles > 0 ? cycles : lsa::kDefaultWaitBudget, std::memory_order_relaxed);
+  return LSA_OK;
+}
+
+int lsa_debug_inject(int kind) {
+  if (kind != 0 && kind != LSA_DEBUG_PREFILL_DROP_S) return LSA_ERR_INVALID_ARG;
+  lsa::g_inject.store(kind, std::memory_order_relaxed);
+  return LSA_OK;
+}
+
+// The first recorded bounds violation over the translation units (0 if none).
+static int bounds_code(bool reset, cudaError_t* err) {
+  cudaError_t (*readers[])(int*, bool) = {lsa::read_bounds_summaries, lsa::read_bounds_decode,
+                                          lsa::read_bounds_decode_blasst, lsa::read_bounds_nsa,
+                                          lsa::read_bounds_kv_append};
+  int first = 0;
+  *err = cudaSuccess;
+  for (auto rd : readers) {
+    int w = 0;
+    const cudaError_t e = rd(&w, reset);
+    if (e != cudaSuccess) {
+      *err = e;
+      return 0;
+    }
+    if (first == 0) first = w;
+  }
+  return first;
+}
+
+int lsa_debug_bounds_code(int* code, int reset) {
+  if (!code) return LSA_ERR_INVALID_ARG;
+#ifdef LSA_DEBUG_BOUNDS
+  cudaError_t err;
+  *code = bounds_code(reset != 0, &err);
+  return cuda_status(err);
+#else
+  (void)reset;
+  *code = 0;
+  return LSA_ERR_UNSUPPORTED;
+#endif
+}
+
 int lsa_device_status(int* status, int reset) {
   if (!status) return LSA_ERR_INVALID_ARG;
   int prefill = 0, decode = 0;
@@ -397,7 +451,15 @@ int lsa_device_status(int* status, int reset) {
   int dbl = 0;
   st = cuda_status(lsa::read_decode_blasst_status(&dbl, reset != 0));
   if (st != LSA_OK) return st;
-  *status = prefill | decode | bq | dbl;
+  int bounds = 0;
+#ifdef LSA_DEBUG_BOUNDS
+  {
+    cudaError_t err;
+    bounds = bounds_code(reset != 0, &err) != 0 ? LSA_DEVICE_BOUNDS : 0;
+    if (err != cudaSuccess) return cuda_status(err);
+  }
+#endif
+  *status = prefill | decode | bq | dbl | bounds;
   return LSA_OK;
 }
 

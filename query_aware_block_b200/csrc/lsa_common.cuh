@@ -38,6 +38,44 @@ __device__ __forceinline__ int fdiv(int n, FastDiv f) {
   return (int)(((unsigned long long)(uint32_t)n * f.m) >> f.sh);
 }
 
+// ---- debug bounds checks (a build with LSA_DEBUG_BOUNDS) -------------------------------
+// A value read from device memory that decides where a kernel reads or writes (a sequence
+// length, a selection index, a selection count) is trusted by the release build.  A build
+// with LSA_DEBUG_BOUNDS checks it instead: the first value out of its documented range is
+// recorded in this translation unit's status word as (kind << 8) | site, the value is
+// clamped into range so that every access stays in bounds, and nothing traps.
+enum { kBoundsSeqlen = 1, kBoundsIndex = 2, kBoundsCount = 3 };
+enum { kSiteSummaries = 1, kSiteDecode = 2, kSiteDecodeBlasst = 3, kSiteNsaCompress = 4,
+       kSiteNsaBranches = 5, kSiteKvAppend = 6 };
+#ifdef LSA_DEBUG_BOUNDS
+namespace {
+__device__ int g_bounds_word = 0;
+}
+__device__ __forceinline__ int checked_range(int v, int lo, int hi, int kind, int site) {
+  if (v < lo || v > hi) {
+    atomicCAS(&g_bounds_word, 0, (kind << 8) | site);
+    return v < lo ? lo : hi;
+  }
+  return v;
+}
+#define LSA_BOUNDS_READER(name)                                                   \
+  cudaError_t read_bounds_##name(int* word, bool reset) {                         \
+    cudaError_t err = cudaMemcpyFromSymbol(word, g_bounds_word, sizeof(int));     \
+    if (err == cudaSuccess && reset) {                                            \
+      const int zero = 0;                                                         \
+      err = cudaMemcpyToSymbol(g_bounds_word, &zero, sizeof(int));                \
+    }                                                                             \
+    return err;                                                                   \
+  }
+#else
+__device__ __forceinline__ int checked_range(int v, int, int, int, int) { return v; }
+#define LSA_BOUNDS_READER(name)                              \
+  cudaError_t read_bounds_##name(int* word, bool) {          \
+    *word = 0;                                               \
+    return cudaSuccess;                                      \
+  }
+#endif
+
 // ---- element conversion ------------------------------------------------------------
 __device__ __forceinline__ float to_f32(float x) { return x; }
 __device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
@@ -186,7 +224,7 @@ __device__ __forceinline__ void stage_block(unsigned char* dst_k, unsigned char*
     const int rem = id % (kBlk * kChunks);
     const int row = rem / kChunks, c = rem % kChunks;
     const int t = j * kBlk + row;
-    const bool valid = j >= 0 && t < Tb;
+    const bool valid = j >= 0 && j < (Tb + kBlk - 1) / kBlk && t < Tb;
     const T* src = (tensor ? vbase : kbase) + (size_t)(valid ? t : 0) * D + c * (16 / sizeof(T));
     unsigned char* dst = (tensor ? dst_v : dst_k) + (kF32 ? row * kv_row + c * 16 : swz(row, c, kv_row));
     cp_async16(dst, src, valid);

@@ -155,6 +155,21 @@ cudaError_t launch_kv_append(const void* k_new, const void* v_new, int elem_byte
                              int T_cap, int D, const int32_t* seqlens, void* k, void* v, int pdl,
                              cudaStream_t stream);
 
+// The debug bounds-check status word of each translation unit (always 0 in the release
+// build, which compiles no checks).
+cudaError_t read_bounds_summaries(int* word, bool reset);
+cudaError_t read_bounds_decode(int* word, bool reset);
+cudaError_t read_bounds_decode_blasst(int* word, bool reset);
+cudaError_t read_bounds_nsa(int* word, bool reset);
+cudaError_t read_bounds_kv_append(int* word, bool reset);
+
+// Bounded waits: the clock-cycle limit of the first wait (settable for tests) and of the
+// drain that follows a timeout; the fault injected for tests (0 = none).
+constexpr long long kDefaultWaitBudget = 4000000000LL;  // about 2 s of clock
+constexpr long long kDrainBudget = 4000000000LL;
+long long wait_budget();
+int debug_inject();
+
 // Unique id of the context current on this host thread (false when none is current or the
 // driver lacks the entry points).
 bool current_context_id(unsigned long long* id);

@@ -47,7 +47,7 @@ __global__ void __launch_bounds__(kPoolThreads) nsa_compress_kernel(
   constexpr int kTok = kPoolThreads / kC;
   const int b = blockIdx.z >> 1, which = blockIdx.z & 1, g = blockIdx.y;
   const int tl = threadIdx.x / kC, c = threadIdx.x % kC;
-  const int T = seqlens[b];
+  const int T = checked_range(seqlens[b], 0, T_cap, kBoundsSeqlen, kSiteNsaCompress);
   const int NC = (T + stride - 1) / stride;
   const int NC_cap = (T_cap + stride - 1) / stride;
   // the range of compressed tokens: [nc_begin, min(nc_end, NC)) or, for nc_begin < 0, the
@@ -141,7 +141,7 @@ __global__ void __launch_bounds__(kThreads) nsa_branches_kernel(const BranchPara
     cp_async16(sm.q + h * D + c * 8, p.q + ((size_t)b * Hq + (size_t)g * G + h) * D + c * 8, true);
   }
   cp_async_commit();
-  const int T = p.seqlens[b];
+  const int T = checked_range(p.seqlens[b], 0, p.T_cap, kBoundsSeqlen, kSiteNsaBranches);
   const int nw = min(p.window, T);                  // window rows
   const int nc = (T + p.stride - 1) / p.stride;     // compressed rows
   const int R = nw + nc;
@@ -383,5 +383,7 @@ cudaError_t launch_nsa_compress(const void* k, const void* v, int B, int Hkv, in
 cudaError_t launch_nsa_branches(const NsaBranchArgs& a, cudaStream_t stream) {
   return a.D == 128 ? launch_branches<128>(a, stream) : launch_branches<64>(a, stream);
 }
+
+LSA_BOUNDS_READER(nsa)
 
 }  // namespace lsa

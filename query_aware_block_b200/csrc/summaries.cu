@@ -34,7 +34,7 @@ build_summaries_kernel(const T* __restrict__ k, int Hkv, int T_cap, const int32_
   __shared__ float red[Geo::kRowGroups][D];
 
   const int g = blockIdx.y, b = blockIdx.z;
-  const int Tb = seqlens[b];
+  const int Tb = checked_range(seqlens[b], 0, T_cap, kBoundsSeqlen, kSiteSummaries);
   const int NB = (Tb + kBlk - 1) / kBlk;
   const int lo = nb_begin >= 0 ? nb_begin : max(0, NB + nb_begin);
   const int hi = nb_end >= 0 ? min(nb_end, NB) : NB;
@@ -111,5 +111,7 @@ cudaError_t launch_build_summaries(const void* k, int dtype, int B, int Hkv, int
     return launch_t<float, 128>(k, B, Hkv, T_cap, seqlens, nb_begin, nb_end, range_max, summ, stream);
   return launch_t<float, 64>(k, B, Hkv, T_cap, seqlens, nb_begin, nb_end, range_max, summ, stream);
 }
+
+LSA_BOUNDS_READER(summaries)
 
 }  // namespace lsa

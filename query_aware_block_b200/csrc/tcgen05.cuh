@@ -63,6 +63,18 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   }
 }
 
+// After a timeout: wait for the phase of the given parity, bounded by `budget` but not by the
+// abort flag, so that copies still in flight (or bytes a cluster peer still owes) land before
+// the CTA exits.  False if the budget runs out too.
+__device__ __forceinline__ bool mbar_drain(uint64_t* bar, uint32_t parity, long long budget) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const long long t0 = clock64();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((it & 255u) == 0u && clock64() - t0 > budget) return false;
+  }
+}
+
 // ---- TMA (non-multicast loads only) ---------------------------------------------------------
 __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, int x, int y, int z,
                                             uint64_t* bar) {

@@ -225,3 +225,11 @@ def test_append_kv_validation():
     assert f(*args(dtype=5)) == lsa.LSA_ERR_UNSUPPORTED
     assert f(*args(B=0, kn=NULL, vn=NULL, k=NULL, v=NULL, sl=NULL)) == lsa.LSA_OK
 
+
+
+def test_debug_controls_validate_without_a_gpu():
+    import query_aware_block_b200 as lsa
+    lib = lsa.library()
+    assert lib.lsa_debug_inject(7) == lsa.LSA_ERR_INVALID_ARG
+    assert lib.lsa_debug_inject(0) == lsa.LSA_OK
+    assert lib.lsa_debug_set_wait_budget(0) == lsa.LSA_OK  # restores the default
