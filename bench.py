@@ -822,12 +822,14 @@ def run_reference(args):
 # ------------------------------------------------------------ other workloads (extra lines) --
 
 def measured_tensor_peak():
+    """The bf16 burst peak: the prefill line times its kernel alone (a run of back-to-back
+    prefills, each a single launch), so the burst cuBLAS figure is the comparable one."""
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
             d = json.load(f)
-        return float(d["bf16_tflops_sustained"]), "measured, sustained"
+        return float(d["bf16_tflops"]), "measured, burst"
     except (OSError, KeyError, ValueError):
-        return 1400.0, "fallback, sustained"
+        return 1590.0, "fallback, burst"
 
 
 def prefill_tile_counts(L, tq=128, tk=64):
@@ -895,7 +897,7 @@ def run_prefill(args):
         "roofline": {"bound": "tensor", "achieved": round(tflops, 1), "peak": peak, "unit": "TFLOP/s",
                      "frac": round(tflops / peak, 4), "traffic": None,
                      "kernel": "blasst_prefill_kernel (tcgen05)",
-                     "peak_source": f"MEASURED_PEAKS.json bf16_tflops_sustained ({kind})",
+                     "peak_source": f"MEASURED_PEAKS.json bf16_tflops ({kind}, of measured)",
                      "algorithmic_flops_per_launch": flops},
         "gpu_launches": K,
         "clocks": clocks.summary(),
