@@ -368,6 +368,321 @@ __global__ void __launch_bounds__(kThreads) decode_blasst_kernel(const __grid_co
   }
 }
 
+// ---- many (b, g) units: one CTA per unit, the selected blocks walked in order --------------
+// With many units the step is bandwidth-bound and a cluster per unit only adds exchanges.
+// One CTA walks its unit's selected blocks in ascending order, exactly as the rule reads:
+// the running maximum is local.  K blocks stream through a 4-stage TMA ring ahead of the
+// walk; a block's V is requested right after its test, into a 3-stage ring, and its P V is
+// done two kept blocks later, so the V load overlaps the next blocks' S and tests.  O stays
+// in mma.sync accumulators; each kept block's rescale factor is applied, in order, when its
+// P V is done.  No cluster, no cross-CTA exchange.
+template <int D>
+struct SeqLay {
+  static constexpr int kTile = kBlk * D * 2;
+  static constexpr int kKS = 4;  // K stages
+  static constexpr int kVS = 3;  // V stages = P buffers (P V lags two kept blocks)
+  static constexpr int kK = 0;   // TMA boxes: 1024-byte aligned
+  static constexpr int kV = kK + kKS * kTile;
+  static constexpr int kQ = kV + kVS * kTile;
+  static constexpr int kP = kQ + kRows * D * 2;
+  static constexpr int kRed = kP + kVS * kRows * kBlk * 2;
+  static constexpr int kTotal = kRed + kWarps * kRows * 4;
+};
+
+template <int D>
+__global__ void __launch_bounds__(kThreads) decode_blasst_seq_kernel(const __grid_constant__ Params p) {
+  using L = SeqLay<D>;
+  constexpr int kRowBytes = D * 2;
+  constexpr int NT = D / 64;
+  constexpr int kLag = L::kVS - 1;
+  extern __shared__ __align__(1024) unsigned char smem[];
+  __shared__ __align__(8) uint64_t kfull[L::kKS], vfull[L::kVS];
+  __shared__ int slot_block[kCL], slot_id[kCL], nslots;
+  __shared__ float rblk[kRows], m_run[kRows], l_run[kRows];
+  __shared__ float alpha_p[L::kVS][kRows];
+  __shared__ int nv_p[L::kVS];
+  __shared__ int keep_flag, skip_flag;
+  __shared__ int xabort;
+  unsigned char* base = smem + ((1024u - (tc::smem_u32(smem) & 1023u)) & 1023u);
+  unsigned char* Kr = base + L::kK;
+  unsigned char* Vr = base + L::kV;
+  unsigned char* Qs = base + L::kQ;
+  unsigned char* Pb = base + L::kP;
+  float* red = reinterpret_cast<float*>(base + L::kRed);
+
+  const int g = blockIdx.x, b = blockIdx.y;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int G = p.G;
+  const int Hq = p.Hkv * G;
+  const int unit = b * p.Hkv + g;
+  const int T = checked_range(__ldg(p.seqlens + b), 0, p.T_cap, kBoundsSeqlen, kSiteDecodeBlasst);
+  const int NBq = (T + kBlk - 1) / kBlk;
+  if (tid == 0) {
+    for (int i = 0; i < L::kKS; ++i) tc::mbar_init(&kfull[i], 1);
+    for (int i = 0; i < L::kVS; ++i) tc::mbar_init(&vfull[i], 1);
+    xabort = 0;
+    tc::fence_mbar_init();
+    tc::prefetch_tmap(&p.tmk);
+    tc::prefetch_tmap(&p.tmv);
+  }
+  if (tid < kRows) {
+    m_run[tid] = -INFINITY;
+    l_run[tid] = 0.f;
+  }
+  // the slots holding a block, compacted in ascending slot order
+  if (warp == 0) {
+    const int ns = checked_range(__ldg(p.nsel + unit), 0, p.topk, kBoundsCount, kSiteDecodeBlasst);
+    const int j2 = lane < p.topk && lane < kCL
+        ? checked_range(__ldg(p.idx + unit * p.topk + lane), -1, NBq - 1, kBoundsIndex, kSiteDecodeBlasst) : -1;
+    const bool on = lane < ns && lane < kCL && j2 >= 0;
+    const uint32_t bits = __ballot_sync(0xffffffffu, on);
+    const int pos = __popc(bits & ((1u << lane) - 1u));
+    if (on) {
+      slot_block[pos] = j2;
+      slot_id[pos] = lane;
+    }
+    if (lane == 0) nslots = __popc(bits);
+  }
+  {
+    const __nv_bfloat16* qg = p.q + ((size_t)b * Hq + (size_t)g * G) * D;
+    constexpr int kQChunks = kRows * kRowBytes / 16;
+    for (int id = tid; id < kQChunks; id += kThreads) {
+      const int row = id / (kRowBytes / 16), c = id % (kRowBytes / 16);
+      cp_async16(Qs + swz(row, c, kRowBytes), qg + (size_t)(row < G ? row : 0) * D + c * 8, row < G);
+    }
+    cp_async_commit();
+  }
+  __syncthreads();  // (the slot list and the barriers are set up)
+  const int n = nslots;
+  int k_issued = 0;
+  auto issue_k = [&](int i) {  // thread 0: K of the i-th visited block into stage i % kKS
+    const int st = i % L::kKS;
+    tc::fence_proxy_async();  // earlier generic reads of the stage come first
+    tc::mbar_arrive_expect_tx(&kfull[st], (uint32_t)L::kTile);
+#pragma unroll
+    for (int h = 0; h < D / 64; ++h)
+      tc::tma_load_3d(Kr + st * L::kTile + h * 8192, &p.tmk, h * 64, slot_block[i] * kBlk, unit, &kfull[st]);
+  };
+  if (tid == 0)
+    for (int i = 0; i < n && i < L::kKS; ++i) issue_k(i);
+  k_issued = n < L::kKS ? n : L::kKS;
+  cp_async_wait<0>();
+  __syncthreads();
+  uint32_t qa[D / 16][4];
+#pragma unroll
+  for (int ks = 0; ks < D / 16; ++ks) {
+    const int row = (lane & 7) + 8 * ((lane >> 3) & 1);
+    ldsm_x4(qa[ks], Qs + swz(row, 2 * ks + (lane >> 4), kRowBytes));
+  }
+  float acc[NT][4];
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) acc[nt][e] = 0.f;
+  const int r0 = lane >> 2;
+  const int col = 8 * warp + 2 * (lane & 3);
+  uint32_t skipped = 0u;
+  int vk = 0, pv_done = 0;
+
+  // P V of the k-th kept block (in order): O = alpha_k O + P_k V_k
+  auto process_pv = [&](int k) {
+    const int st = k % L::kVS;
+    tc::mbar_wait(&vfull[st], (uint32_t)((k / L::kVS) & 1), &xabort, p.budget);
+    unsigned char* Vs = Vr + st * L::kTile;
+    const int nv = nv_p[st];
+    for (int id = tid; id < (kBlk - nv) * (D / 8); id += kThreads) {  // rows past the sequence
+      const int r = nv + id / (D / 8), c = id % (D / 8);
+      *reinterpret_cast<uint4*>(Vs + kv_off(r, c)) = make_uint4(0u, 0u, 0u, 0u);
+    }
+    __syncthreads();
+    const float a_lo = alpha_p[st][r0], a_hi = alpha_p[st][r0 + 8];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      acc[nt][0] *= a_lo; acc[nt][1] *= a_lo;
+      acc[nt][2] *= a_hi; acc[nt][3] *= a_hi;
+    }
+    const unsigned char* Ps = Pb + st * (kRows * kBlk * 2);
+#pragma unroll
+    for (int ks = 0; ks < kBlk / 16; ++ks) {
+      uint32_t pa[4];
+      const int row = (lane & 7) + 8 * ((lane >> 3) & 1);
+      ldsm_x4(pa, Ps + swz(row, 2 * ks + (lane >> 4), kBlk * 2));
+      const int vrow = 16 * ks + (lane & 7) + 8 * ((lane >> 3) & 1);
+      if constexpr (D == 128) {
+        uint32_t vb[4];
+        ldsm_x4_t(vb, Vs + kv_off(vrow, 2 * warp + (lane >> 4)));
+        mma_bf16(acc[0], pa, vb[0], vb[1]);
+        mma_bf16(acc[1], pa, vb[2], vb[3]);
+      } else {
+        uint32_t vb[2];
+        ldsm_x2_t(vb, Vs + kv_off(vrow, warp));
+        mma_bf16(acc[0], pa, vb[0], vb[1]);
+      }
+    }
+    __syncthreads();  // the stage and the P buffer may be reused
+    ++pv_done;
+  };
+
+  for (int i = 0; i < n; ++i) {
+    const int j = slot_block[i];
+    const int nv = max(0, min(kBlk, T - j * kBlk));
+    const int kst = i % L::kKS;
+    tc::mbar_wait(&kfull[kst], (uint32_t)((i / L::kKS) & 1), &xabort, p.budget);
+    // S = Q K^T (base-2 logits): warp w takes keys 8w .. 8w + 7
+    float s[4];
+    {
+      const unsigned char* Ks = Kr + kst * L::kTile;
+      float c4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int ks = 0; ks < D / 16; ks += 2) {
+        uint32_t kb[4];
+        ldsm_x4(kb, Ks + kv_off(8 * warp + (lane & 7), 2 * ks + (lane >> 3)));
+        mma_bf16(c4, qa[ks], kb[0], kb[1]);
+        mma_bf16(c4, qa[ks + 1], kb[2], kb[3]);
+      }
+      const bool v0 = col < nv, v1 = col + 1 < nv;
+      s[0] = v0 && r0 < G ? c4[0] * p.scale2 : -INFINITY;
+      s[1] = v1 && r0 < G ? c4[1] * p.scale2 : -INFINITY;
+      s[2] = v0 && r0 + 8 < G ? c4[2] * p.scale2 : -INFINITY;
+      s[3] = v1 && r0 + 8 < G ? c4[3] * p.scale2 : -INFINITY;
+    }
+    {  // the block maxima
+      float m_lo = fmaxf(s[0], s[1]), m_hi = fmaxf(s[2], s[3]);
+#pragma unroll
+      for (int o2 = 1; o2 < 4; o2 <<= 1) {
+        m_lo = fmaxf(m_lo, __shfl_xor_sync(0xffffffffu, m_lo, o2));
+        m_hi = fmaxf(m_hi, __shfl_xor_sync(0xffffffffu, m_hi, o2));
+      }
+      if ((lane & 3) == 0) {
+        red[warp * kRows + r0] = m_lo;
+        red[warp * kRows + r0 + 8] = m_hi;
+      }
+    }
+    __syncthreads();  // (every warp has read K_i: its stage may be refilled)
+    if (tid == 0 && k_issued < n) issue_k(k_issued);
+    k_issued = k_issued < n ? k_issued + 1 : n;
+    // the test (warp 0, lane h = head h): skip iff not the first visited block and every
+    // head's block maximum trails its running maximum by more than -log2(lambda)
+    if (warp == 0) {
+      float r = -INFINITY;
+      if (lane < kRows) {
+#pragma unroll
+        for (int w = 0; w < kWarps; ++w) r = fmaxf(r, red[w * kRows + lane]);
+        rblk[lane] = r;
+      }
+      float gi = -INFINITY;
+      if (lane < G) {
+        const float m = m_run[lane];
+        gi = r == -INFINITY ? -INFINITY : (m == -INFINITY ? INFINITY : r - m);
+      }
+#pragma unroll
+      for (int o2 = 16; o2 > 0; o2 >>= 1) gi = fmaxf(gi, __shfl_xor_sync(0xffffffffu, gi, o2));
+      if (lane == 0) {
+        const bool sk = i > 0 && gi < p.log2_lambda;
+        skip_flag = sk;
+        keep_flag = !sk && nv > 0;
+      }
+    }
+    __syncthreads();
+    if (skip_flag) skipped |= 1u << slot_id[i];
+    if (!keep_flag) continue;
+    // kept: V_i into stage vk % kVS (its previous occupant's P V is done), P_i, statistics
+    const int vst = vk % L::kVS;
+    if (tid == 0) {
+      tc::fence_proxy_async();
+      tc::mbar_arrive_expect_tx(&vfull[vst], (uint32_t)L::kTile);
+#pragma unroll
+      for (int h = 0; h < D / 64; ++h)
+        tc::tma_load_3d(Vr + vst * L::kTile + h * 8192, &p.tmv, h * 64, j * kBlk, unit, &vfull[vst]);
+      nv_p[vst] = nv;
+    }
+    {
+      const float ml = fmaxf(m_run[r0], rblk[r0]), mh = fmaxf(m_run[r0 + 8], rblk[r0 + 8]);
+      const float p0 = s[0] == -INFINITY ? 0.f : ex2(s[0] - ml);
+      const float p1 = s[1] == -INFINITY ? 0.f : ex2(s[1] - ml);
+      const float p2 = s[2] == -INFINITY ? 0.f : ex2(s[2] - mh);
+      const float p3 = s[3] == -INFINITY ? 0.f : ex2(s[3] - mh);
+      unsigned char* Ps = Pb + vst * (kRows * kBlk * 2);
+      *reinterpret_cast<uint32_t*>(Ps + swz(r0, col >> 3, kBlk * 2) + (col & 7) * 2) = pack_bf16x2(p0, p1);
+      *reinterpret_cast<uint32_t*>(Ps + swz(r0 + 8, col >> 3, kBlk * 2) + (col & 7) * 2) = pack_bf16x2(p2, p3);
+      float l_lo = p0 + p1, l_hi = p2 + p3;
+#pragma unroll
+      for (int o2 = 1; o2 < 4; o2 <<= 1) {
+        l_lo += __shfl_xor_sync(0xffffffffu, l_lo, o2);
+        l_hi += __shfl_xor_sync(0xffffffffu, l_hi, o2);
+      }
+      if ((lane & 3) == 0) {  // (red's maxima were read before the last barrier)
+        red[warp * kRows + r0] = l_lo;
+        red[warp * kRows + r0 + 8] = l_hi;
+      }
+    }
+    __syncthreads();
+    if (tid < kRows) {
+      const float mo = m_run[tid], mn = fmaxf(mo, rblk[tid]);
+      float ls = 0.f;
+#pragma unroll
+      for (int w = 0; w < kWarps; ++w) ls += red[w * kRows + tid];
+      const float a = mo == -INFINITY ? 0.f : ex2(mo - mn);
+      alpha_p[vst][tid] = a;
+      l_run[tid] = l_run[tid] * a + ls;
+      m_run[tid] = mn;
+    }
+    __syncthreads();  // (red, m_run and the block's statistics: the next block rewrites them)
+    ++vk;
+    if (vk - 1 - kLag >= 0) process_pv(vk - 1 - kLag);
+  }
+  while (pv_done < vk) process_pv(pv_done);
+  __syncthreads();  // (the statistics are final)
+
+  // outputs: rows r0, r0 + 8 of the group, columns of this warp's n-tiles
+  const size_t orow = (size_t)b * Hq + (size_t)g * G;
+#pragma unroll
+  for (int half = 0; half < 2; ++half) {
+    const int h = r0 + 8 * half;
+    if (h < G) {
+      const float l = l_run[h];
+      const float inv = l > 0.f ? 1.f / l : 0.f;
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        const int d = (D == 128 ? 16 * warp : 8 * warp) + 8 * nt + 2 * (lane & 3);
+        *reinterpret_cast<uint32_t*>(p.o + (orow + h) * D + d) =
+            pack_bf16x2(acc[nt][2 * half] * inv, acc[nt][2 * half + 1] * inv);
+      }
+    }
+  }
+  if (tid < G && p.lse) {
+    const float l = l_run[tid];
+    p.lse[orow + tid] = l > 0.f ? (m_run[tid] + log2f(l)) * kLn2 : -INFINITY;
+  }
+  if (tid == 0 && p.skip_bits) p.skip_bits[unit] = skipped;
+  // after a timeout (the outputs are then undefined): the copies still in flight land
+  // before the CTA exits
+  if (*reinterpret_cast<volatile int*>(&xabort)) {
+    for (int i = k_issued - L::kKS < 0 ? 0 : k_issued - L::kKS; i < k_issued; ++i)
+      tc::mbar_drain(&kfull[i % L::kKS], (uint32_t)((i / L::kKS) & 1), kDrainBudget);
+    for (int k = vk - L::kVS < 0 ? 0 : vk - L::kVS; k < vk; ++k)
+      tc::mbar_drain(&vfull[k % L::kVS], (uint32_t)((k / L::kVS) & 1), kDrainBudget);
+    g_blasst_decode_status = 1;
+  }
+}
+
+// Units from which one CTA per unit (walking its blocks in order) fills the GPU better
+// than a 16-CTA cluster per unit.
+constexpr int kSeqUnits = 64;
+
+template <int D>
+cudaError_t launch_seq(const DecodeBlasstArgs& a, const Params& p, cudaStream_t stream) {
+  auto kernel = decode_blasst_seq_kernel<D>;
+  const int smem = SeqLay<D>::kTotal + 1024;
+  static DeviceOnce attr_once;
+  const cudaError_t err = attr_once.run([&]() {
+    return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  });
+  if (err != cudaSuccess) return err;
+  kernel<<<dim3(a.Hkv, a.B, 1), kThreads, smem, stream>>>(p);
+  return cudaGetLastError();
+}
+
 template <int D>
 cudaError_t launch_d(const DecodeBlasstArgs& a, cudaStream_t stream) {
   auto kernel = decode_blasst_kernel<D>;
@@ -387,6 +702,7 @@ cudaError_t launch_d(const DecodeBlasstArgs& a, cudaStream_t stream) {
   p.lse = a.lse;
   p.skip_bits = a.skip_bits;
   p.budget = wait_budget();
+  if (a.B * a.Hkv >= kSeqUnits) return launch_seq<D>(a, p, stream);
   const int smem = Lay<D>::kTotal + 1024;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(kCL, a.Hkv, a.B);

@@ -13,7 +13,7 @@ import torch
 
 import oracle
 import synth
-from tests.parity import LSE_TOL, TOL, max_abs, max_abs_beyond_bf16
+from tests.parity import LSE_TOL, TOL, max_abs, max_abs_beyond_rounding
 
 pytestmark = pytest.mark.gpu
 
@@ -52,5 +52,5 @@ def test_prefill_wait_runs_out_and_the_context_survives(lsa):
     r = oracle.blasst_prefill(case.q, case.k, case.v, units, 0.0)
     for u, (b, h, a) in enumerate(units):
         rows = slice(128 * a, 128 * a + 128)
-        assert max_abs_beyond_bf16(o[b, h, rows].float(), r["o"][u]) <= TOL[torch.bfloat16]
+        assert max_abs_beyond_rounding(o[b, h, rows].float(), r["o"][u]) <= TOL[torch.bfloat16]
         assert max_abs(lse[b, h, rows], r["lse"][u]) <= LSE_TOL[torch.bfloat16]

@@ -10,7 +10,7 @@ import torch
 
 import oracle
 import synth
-from tests.parity import LSE_TOL, TOL, max_abs, max_abs_beyond_bf16, max_abs_vs_bf16
+from tests.parity import LSE_TOL, TOL, max_abs, max_abs_beyond_rounding
 
 pytestmark = pytest.mark.gpu
 
@@ -48,8 +48,8 @@ def test_nsa_compress_matches_oracle(lsa, kw):
     torch.cuda.synchronize()
     kr = oracle.nsa_compress(case.k, case.seqlens, length, stride)
     vr = oracle.nsa_compress(case.v, case.seqlens, length, stride)
-    assert max_abs_beyond_bf16(kc.cpu(), kr) <= 1e-5, kw
-    assert max_abs_beyond_bf16(vc.cpu(), vr) <= 1e-5, kw
+    assert max_abs_beyond_rounding(kc.cpu(), kr) <= 1e-5, kw
+    assert max_abs_beyond_rounding(vc.cpu(), vr) <= 1e-5, kw
 
 
 def test_nsa_compress_refresh_of_the_last_tokens(lsa):
@@ -97,7 +97,7 @@ def _check(case, gates, window, o, lw, lc, idx, o_slc, with_slc=True, where=""):
     r = oracle.nsa_decode(case.q, case.k, case.v, case.seqlens, gates=gates, window=window,
                           idx=idx)
     ref = r["o"] if with_slc else gates[0] * r["o_cmp"] + gates[2] * r["o_win"]
-    assert max_abs_vs_bf16(o, ref) <= TOL[torch.bfloat16], where
+    assert max_abs_beyond_rounding(o, ref) <= TOL[torch.bfloat16], where
     assert max_abs(lw, r["lse_win"]) <= LSE_TOL[torch.bfloat16], where
     assert max_abs(lc, r["lse_cmp"]) <= LSE_TOL[torch.bfloat16], where
 
