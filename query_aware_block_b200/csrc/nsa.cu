@@ -17,10 +17,10 @@
 // two compressed tokens only (the ones a new token changes).  The two branches are one
 // launch: a cluster of 16 CTAs per (sequence, KV head) splits the concatenated rows
 // [window | compressed] evenly, so a CTA may hold rows of both; each CTA runs an online
-// softmax over 64-row tiles (K and V by cp.async into padded rows, logits and P.V on the
-// FMA pipes: G <= 16 query rows are too few for a tensor-core tile), then stores each
-// branch's partial (m, l, acc) into the shared memory of the CTA that owns that part of
-// the output.  After one cluster barrier each CTA merges its slice from its own shared
+// softmax over 64-row tiles (K and V by cp.async into a two-stage ring, the next tile in
+// flight while the current one is used; logits and P.V on mma.sync m16n8k16 with the
+// G <= 16 query heads as the 16 rows, zero-padded), then stores each branch's partial
+// (m, l, acc) into the shared memory of the CTA that owns that part of the output.  After one cluster barrier each CTA merges its slice from its own shared
 // memory, adds the gated selected-branch output and writes o.  The only waits are
 // hardware cluster barriers that every thread reaches.
 #include <math.h>
@@ -91,14 +91,18 @@ constexpr int kCL = 16;
 constexpr int kMaxG = 16;
 constexpr int kTile = 64;
 
+constexpr int kSStride = 68;  // fp32 row stride of the logits tile
+
 template <int D>
 struct BranchSmem {
-  static constexpr int kKS = D + 8;  // padded bf16 rows: conflict-free 16-byte reads
-  __nv_bfloat16 kt[kTile * kKS];
-  __nv_bfloat16 vt[kTile * kKS];
-  __nv_bfloat16 q[kMaxG * D];
-  float s[kMaxG][kTile];              // logits (base 2), then probabilities
-  float m_run[kMaxG], l_run[kMaxG], alpha[kMaxG];
+  static constexpr int kTileBytes = kTile * D * 2;
+  // [stage][K, V]: 64 rows in the 128-byte-swizzled box layout of kv_off (ldmatrix over 8
+  // consecutive rows is conflict-free)
+  alignas(128) unsigned char kv[2][2][kTileBytes];
+  alignas(128) unsigned char q[16 * D * 2];   // [16 rows][D], chunk-swizzled; rows >= G zero
+  alignas(128) unsigned char pb[16 * kTile * 2];  // P (bf16) [16][64], chunk-swizzled
+  float s[16][kSStride];                      // logits (base 2)
+  float m_run[kMaxG], l_run[kMaxG], alpha[16];
   float2 recv_ml[2][kCL][kMaxG];      // [branch][source CTA][head] (m, l)
   float recv_acc[2][kCL][kMaxG * D / kCL];  // [branch][source CTA][element of my slice]
 };
@@ -123,11 +127,10 @@ struct BranchParams {
 template <int D>
 __global__ void __launch_bounds__(kThreads) nsa_branches_kernel(const BranchParams p) {
   using S = BranchSmem<D>;
-  constexpr int kKS = S::kKS;
-  constexpr int kC = D / 8;
-  constexpr int kHS = kThreads / D;     // heads interleaved per output column: 2 or 4
-  constexpr int kPH = kMaxG / kHS;      // heads per thread in P.V
-  extern __shared__ __align__(16) unsigned char smem_raw[];
+  constexpr int kC = D / 8;               // 16-byte chunks per row
+  constexpr int kRowBytes = D * 2;
+  constexpr int NT = D / 64;              // n8 tiles of the output per warp
+  extern __shared__ __align__(128) unsigned char smem_raw[];
   S& sm = *reinterpret_cast<S*>(smem_raw);
   const int rank = cluster_rank();
   const int g = blockIdx.y, b = blockIdx.z;
@@ -136,9 +139,13 @@ __global__ void __launch_bounds__(kThreads) nsa_branches_kernel(const BranchPara
   const size_t unit = (size_t)b * p.Hkv + g;
   cluster_arrive_relaxed();  // peers' shared memory is written only after all have started
 
-  for (int id = tid; id < G * kC; id += kThreads) {
+  for (int id = tid; id < 16 * kC; id += kThreads) {
     const int h = id / kC, c = id - h * kC;
-    cp_async16(sm.q + h * D + c * 8, p.q + ((size_t)b * Hq + (size_t)g * G + h) * D + c * 8, true);
+    unsigned char* dst = sm.q + swz(h, c, kRowBytes);
+    if (h < G)
+      cp_async16(dst, p.q + ((size_t)b * Hq + (size_t)g * G + h) * D + c * 8, true);
+    else
+      *reinterpret_cast<uint4*>(dst) = make_uint4(0u, 0u, 0u, 0u);
   }
   cp_async_commit();
   const int T = checked_range(p.seqlens[b], 0, p.T_cap, kBoundsSeqlen, kSiteNsaBranches);
@@ -147,10 +154,9 @@ __global__ void __launch_bounds__(kThreads) nsa_branches_kernel(const BranchPara
   const int R = nw + nc;
   const int per = (R + kCL - 1) / kCL;
   const int r0 = min(R, rank * per), r1 = min(R, r0 + per);
-  const int d = tid % D, h0 = tid / D;              // P.V mapping: column d, heads h0 + i*kHS
   const int per_out = G * D / kCL;                  // output elements each CTA merges
-  cp_async_wait<0>();  // (q; also when this CTA gets no rows)
-  cluster_wait();      // (matches the arrive at the start) DSMEM is live from here on
+  const int srow = tid >> 4, ssub = tid & 15;       // softmax: row srow, keys 4 ssub .. + 3
+  cluster_wait();  // (matches the arrive at the start) DSMEM is live from here on
 
   for (int part = 0; part < 2; ++part) {  // 0: window rows [0, nw), 1: compressed [nw, R)
     const int lo = part == 0 ? max(r0, 0) : max(r0, nw);
@@ -162,103 +168,121 @@ __global__ void __launch_bounds__(kThreads) nsa_branches_kernel(const BranchPara
                                           : p.kc + unit * p.NC_cap * D;
     const __nv_bfloat16* vsrc = part == 0 ? p.v + (unit * p.T_cap + (size_t)(T - nw)) * D
                                           : p.vc + unit * p.NC_cap * D;
-    __syncthreads();  // (the previous part's statistics have been pushed)
-    for (int h = tid; h < G; h += kThreads) {
-      sm.m_run[h] = -INFINITY;
-      sm.l_run[h] = 0.f;
-    }
-    float acc[kPH];
-#pragma unroll
-    for (int i = 0; i < kPH; ++i) acc[i] = 0.f;
-    for (int t0 = lo; t0 < hi; t0 += kTile) {
+    // rows t0 .. t0 + 63 of this part into stage st; rows past hi: K and V zero (P is 0
+    // there, V must be finite)
+    auto load_tile = [&](int t0, int st) {
       const int nt = min(kTile, hi - t0);
-      __syncthreads();  // (the previous tile's K/V/P are no longer read)
-      for (int id = tid; id < nt * kC; id += kThreads) {
+      for (int id = tid; id < kTile * kC; id += kThreads) {
         const int r = id / kC, c = id - r * kC;
-        const size_t src = (size_t)(t0 + r - roff) * D + c * 8;
-        cp_async16(sm.kt + r * kKS + c * 8, ksrc + src, true);
-        cp_async16(sm.vt + r * kKS + c * 8, vsrc + src, true);
+        const int off = kv_off(r, c);
+        if (r < nt) {
+          const size_t src = (size_t)(t0 + r - roff) * D + c * 8;
+          cp_async16(sm.kv[st][0] + off, ksrc + src, true);
+          cp_async16(sm.kv[st][1] + off, vsrc + src, true);
+        } else {
+          *reinterpret_cast<uint4*>(sm.kv[st][0] + off) = make_uint4(0u, 0u, 0u, 0u);
+          *reinterpret_cast<uint4*>(sm.kv[st][1] + off) = make_uint4(0u, 0u, 0u, 0u);
+        }
       }
       cp_async_commit();
-      cp_async_wait<0>();
-      __syncthreads();
-      // logits: pair (h, t) = (pp >> 6, pp & 63), a warp shares h
-      for (int pp = tid; pp < G * kTile; pp += kThreads) {
-        const int h = pp >> 6, t = pp & (kTile - 1);
-        float sv = -INFINITY;
-        if (t < nt) {
-          float a0 = 0.f, a1 = 0.f;
-          const __nv_bfloat16* kr = sm.kt + t * kKS;
-          const __nv_bfloat16* qr = sm.q + h * D;
-#pragma unroll 4
-          for (int c = 0; c < kC; ++c) {
-            const uint4 kk = *reinterpret_cast<const uint4*>(kr + c * 8);
-            const uint4 qq = *reinterpret_cast<const uint4*>(qr + c * 8);
-            const uint32_t wk[4] = {kk.x, kk.y, kk.z, kk.w};
-            const uint32_t wq[4] = {qq.x, qq.y, qq.z, qq.w};
+    };
+    __syncthreads();  // (the previous part's statistics have been pushed, its stages are free)
+    if (lo < hi) load_tile(lo, 0);
+    float m_run = -INFINITY, l_run = 0.f;  // (row srow; every thread of the row keeps them)
+    float acc[NT][4];
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              a0 = fmaf(__uint_as_float(wq[e] << 16), __uint_as_float(wk[e] << 16), a0);
-              a1 = fmaf(__uint_as_float(wq[e] & 0xffff0000u), __uint_as_float(wk[e] & 0xffff0000u), a1);
-            }
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc[nt][e] = 0.f;
+    int st = 0;
+    for (int t0 = lo; t0 < hi; t0 += kTile, st ^= 1) {
+      const int nt = min(kTile, hi - t0);
+      __syncthreads();  // (the other stage, P and the logits of the previous tile are free)
+      if (t0 + kTile < hi) {
+        load_tile(t0 + kTile, st ^ 1);
+        cp_async_wait<1>();  // this tile (and q) landed; the next one stays in flight
+      } else {
+        cp_async_wait<0>();
+      }
+      __syncthreads();
+      const unsigned char* Ks = sm.kv[st][0];
+      const unsigned char* Vs = sm.kv[st][1];
+      // logits S = q K^T (base 2): warp w -> keys 8w .. 8w + 7
+      {
+        float sc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int ks = 0; ks < D / 16; ks += 2) {
+          uint32_t kb[4], qa0[4], qa1[4];
+          ldsm_x4(kb, Ks + kv_off(8 * warp + (lane & 7), 2 * ks + (lane >> 3)));
+          const int row = (lane & 7) + 8 * ((lane >> 3) & 1);
+          ldsm_x4(qa0, sm.q + swz(row, 2 * ks + (lane >> 4), kRowBytes));
+          ldsm_x4(qa1, sm.q + swz(row, 2 * ks + 2 + (lane >> 4), kRowBytes));
+          mma_bf16(sc, qa0, kb[0], kb[1]);
+          mma_bf16(sc, qa1, kb[2], kb[3]);
+        }
+        const int col = 8 * warp + 2 * (lane & 3);
+        const bool v0 = col < nt, v1 = col + 1 < nt;
+        const int rr = lane >> 2;
+        *reinterpret_cast<float2*>(&sm.s[rr][col]) =
+            make_float2(v0 ? sc[0] * p.scale2 : -INFINITY, v1 ? sc[1] * p.scale2 : -INFINITY);
+        *reinterpret_cast<float2*>(&sm.s[rr + 8][col]) =
+            make_float2(v0 ? sc[2] * p.scale2 : -INFINITY, v1 ? sc[3] * p.scale2 : -INFINITY);
+      }
+      __syncthreads();
+      // online softmax: 16 threads per row (a half warp), 4 keys each; rows >= G get P = 0
+      {
+        const float4 x = *reinterpret_cast<const float4*>(&sm.s[srow][4 * ssub]);
+        float mx = fmaxf(fmaxf(x.x, x.y), fmaxf(x.z, x.w));
+#pragma unroll
+        for (int o2 = 8; o2 > 0; o2 >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o2));
+        const float m_new = fmaxf(m_run, mx);  // finite: the tile has at least one row
+        float p0 = 0.f, p1 = 0.f, p2 = 0.f, p3 = 0.f, alpha = 1.f;
+        if (srow < G) {
+          p0 = ex2(x.x - m_new);
+          p1 = ex2(x.y - m_new);
+          p2 = ex2(x.z - m_new);
+          p3 = ex2(x.w - m_new);
+          alpha = m_run == -INFINITY ? 0.f : ex2(m_run - m_new);
+        }
+        float ps = (p0 + p1) + (p2 + p3);
+#pragma unroll
+        for (int o2 = 8; o2 > 0; o2 >>= 1) ps += __shfl_xor_sync(0xffffffffu, ps, o2);
+        l_run = l_run * alpha + ps;
+        m_run = m_new;
+        *reinterpret_cast<uint2*>(sm.pb + swz(srow, ssub >> 1, kTile * 2) + 8 * (ssub & 1)) =
+            make_uint2(pack_bf16x2(p0, p1), pack_bf16x2(p2, p3));
+        if (ssub == 0) sm.alpha[srow] = alpha;
+      }
+      __syncthreads();
+      // acc = alpha * acc + P V: warp w -> output dims 8 NT w .. 8 NT w + 8 NT - 1
+      {
+        const float a_lo = sm.alpha[lane >> 2], a_hi = sm.alpha[(lane >> 2) + 8];
+#pragma unroll
+        for (int n2 = 0; n2 < NT; ++n2) {
+          acc[n2][0] *= a_lo; acc[n2][1] *= a_lo;
+          acc[n2][2] *= a_hi; acc[n2][3] *= a_hi;
+        }
+#pragma unroll
+        for (int ks = 0; ks < kTile / 16; ++ks) {
+          const int vrow = 16 * ks + (lane & 7) + 8 * ((lane >> 3) & 1);
+          uint32_t vb[4], pa[4];
+          if constexpr (NT == 2) {
+            ldsm_x4_t(vb, Vs + kv_off(vrow, 2 * warp + (lane >> 4)));
+          } else {
+            uint32_t v2[2];
+            ldsm_x2_t(v2, Vs + kv_off(vrow, warp));
+            vb[0] = v2[0]; vb[1] = v2[1]; vb[2] = 0u; vb[3] = 0u;
           }
-          sv = (a0 + a1) * p.scale2;
-        }
-        sm.s[h][t] = sv;
-      }
-      __syncthreads();
-      // online softmax per head (warp per head): new max, rescale factor, probabilities
-      for (int h = warp; h < G; h += kWarps) {
-        const float x0 = sm.s[h][lane], x1 = sm.s[h][lane + 32];
-        float mx = fmaxf(x0, x1);
-#pragma unroll
-        for (int o2 = 16; o2 > 0; o2 >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o2));
-        const float m_old = sm.m_run[h];
-        const float m_new = fmaxf(m_old, mx);  // finite: the tile has at least one row
-        const float p0 = lane < nt ? ex2(x0 - m_new) : 0.f;
-        const float p1 = lane + 32 < nt ? ex2(x1 - m_new) : 0.f;
-        sm.s[h][lane] = p0;
-        sm.s[h][lane + 32] = p1;
-        const float ps = warp_sum(p0 + p1);
-        if (lane == 0) {
-          const float a = m_old == -INFINITY ? 0.f : ex2(m_old - m_new);
-          sm.alpha[h] = a;
-          sm.l_run[h] = sm.l_run[h] * a + ps;
-          sm.m_run[h] = m_new;
+          const int row = (lane & 7) + 8 * ((lane >> 3) & 1);
+          ldsm_x4(pa, sm.pb + swz(row, 2 * ks + (lane >> 4), kTile * 2));
+          mma_bf16(acc[0], pa, vb[0], vb[1]);
+          if constexpr (NT == 2) mma_bf16(acc[1], pa, vb[2], vb[3]);
         }
       }
-      __syncthreads();
-      // acc = alpha * acc + P.V, 4 rows at a time (one 16-byte read of each head's P)
-#pragma unroll
-      for (int i = 0; i < kPH; ++i) {
-        const int h = h0 + i * kHS;
-        if (h < G) acc[i] *= sm.alpha[h];
-      }
-      const int nt4 = nt & ~3;
-      for (int t = 0; t < nt4; t += 4) {
-        float vv[4];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) vv[u] = __bfloat162float(sm.vt[(t + u) * kKS + d]);
-#pragma unroll
-        for (int i = 0; i < kPH; ++i) {
-          const int h = h0 + i * kHS;
-          if (h < G) {
-            const float4 p4 = *reinterpret_cast<const float4*>(&sm.s[h][t]);
-            acc[i] = fmaf(p4.x, vv[0], acc[i]);
-            acc[i] = fmaf(p4.y, vv[1], acc[i]);
-            acc[i] = fmaf(p4.z, vv[2], acc[i]);
-            acc[i] = fmaf(p4.w, vv[3], acc[i]);
-          }
-        }
-      }
-      for (int t = nt4; t < nt; ++t) {
-        const float vv = __bfloat162float(sm.vt[t * kKS + d]);
-#pragma unroll
-        for (int i = 0; i < kPH; ++i) {
-          const int h = h0 + i * kHS;
-          if (h < G) acc[i] = fmaf(sm.s[h][t], vv, acc[i]);
-        }
-      }
+    }
+    if (ssub == 0 && srow < G) {
+      sm.m_run[srow] = m_run;
+      sm.l_run[srow] = l_run;
     }
     __syncthreads();  // (m_run / l_run final)
     // this part's partial into the owners' tables (an empty range gives m = -inf, l = 0)
@@ -267,14 +291,19 @@ __global__ void __launch_bounds__(kThreads) nsa_branches_kernel(const BranchPara
       st_cluster(map_rank(&sm.recv_ml[part][rank][h], peer), make_float2(sm.m_run[h], sm.l_run[h]));
     }
 #pragma unroll
-    for (int i = 0; i < kPH; ++i) {
-      const int h = h0 + i * kHS;
-      if (h < G) {
-        const int e = h * D + d, owner = e / per_out;
-        st_cluster(map_rank(&sm.recv_acc[part][rank][e - owner * per_out], owner), acc[i]);
+    for (int n2 = 0; n2 < NT; ++n2) {
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        const int h = (lane >> 2) + 8 * half;
+        if (h < G) {
+          const int e = h * D + 8 * NT * warp + 8 * n2 + 2 * (lane & 3), owner = e / per_out;
+          st_cluster(map_rank(&sm.recv_acc[part][rank][e - owner * per_out], owner),
+                     make_float2(acc[n2][2 * half], acc[n2][2 * half + 1]));
+        }
       }
     }
   }
+  cp_async_wait<0>();        // (q, when this CTA had no rows)
   cluster_arrive_release();  // every partial is in its owner's shared memory ...
   cluster_wait();            // ... and no CTA touches another's shared memory after this
 
