@@ -89,7 +89,10 @@ def test_prefill_skips_match_oracle(lsa, B, Hq, Hkv, L, lam, sink):
 def test_blasst_prefill_32k_workload_sampled(lsa):
     case = synth.blasst_prefill_32k()
     o, lse, bits, cnt = _run(lsa, case)
-    units = [(0, h, a) for h in (0, 13, 31) for a in (0, 1, 97, 255)]
+    # every KV group (4 query heads each): the first tiles, a mid-diagonal tile that moves
+    # with the group, and the last (diagonal) tile; plus the heaviest tiles of three heads
+    units = [(0, 4 * g + g % 4, a) for g in range(8) for a in (0, 1 + 3 * g, 64 + 17 * g, 255)]
+    units += [(0, h, a) for h in (0, 13, 31) for a in (97, 254)]
     _check_units(case, o, lse, bits, units, "32K workload")
     total = sum(bin(int(w)).count("1") for w in bits.flatten())
     assert total == cnt
