@@ -29,6 +29,7 @@ struct LaunchRecord {
   int smem_set[kMaxDevices] = {};
   int n_ok[kMaxDevices] = {};
   long long ok[kMaxDevices][kShapes] = {};
+  int sms[kMaxDevices] = {};
 
   // Caller holds mu.  Raises the kernel's dynamic shared memory limit on `dev` to at least
   // `smem`; `cluster` also allows non-portable cluster sizes (up to 16 CTAs).
@@ -42,6 +43,15 @@ struct LaunchRecord {
       if (err != cudaSuccess) return err;
     }
     smem_set[dev] = smem;
+    return cudaSuccess;
+  }
+  // Caller holds mu.  The number of SMs of `dev` (asked once).
+  cudaError_t sm_count(int dev, int* n) {
+    if (sms[dev] == 0) {
+      const cudaError_t err = cudaDeviceGetAttribute(&sms[dev], cudaDevAttrMultiProcessorCount, dev);
+      if (err != cudaSuccess) return err;
+    }
+    *n = sms[dev];
     return cudaSuccess;
   }
   // Caller holds mu.  Whether (cl, smem) was found schedulable on `dev`.
