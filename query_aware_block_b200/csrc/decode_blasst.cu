@@ -27,6 +27,9 @@
 // leaves while a peer may still write into it.  Waits are bounded (about 2 s of clock); if
 // one runs out the launch's outputs are undefined, the CTA waits (bounded) for what is still
 // in flight before it exits, and a status word records the failure.
+// With many (b, g) units (64 and up) one CTA per unit does the same in phases instead
+// (decode_blasst_unit_kernel below): every block's S, every slot's test at once, then the
+// kept blocks' V and P V spread over its warps.
 #include <math.h>
 
 #include "cluster.cuh"
@@ -368,47 +371,49 @@ __global__ void __launch_bounds__(kThreads) decode_blasst_kernel(const __grid_co
   }
 }
 
-// ---- many (b, g) units: one CTA per unit, the selected blocks walked in order --------------
-// With many units the step is bandwidth-bound and a cluster per unit only adds exchanges.
-// One CTA walks its unit's selected blocks in ascending order, exactly as the rule reads:
-// the running maximum is local.  K blocks stream through a 4-stage TMA ring ahead of the
-// walk; a block's V is requested right after its test, into a 3-stage ring, and its P V is
-// done two kept blocks later, so the V load overlaps the next blocks' S and tests.  O stays
-// in mma.sync accumulators; each kept block's rescale factor is applied, in order, when its
-// P V is done.  No cluster, no cross-CTA exchange.
+// ---- many (b, g) units: one CTA per unit in three parallel phases -------------------------
+// The sequential rule needs, for each selected block, only the maximum of the earlier
+// blocks' maxima (a skipped block never raises it), so nothing has to run block by block:
+//   1. S = Q K^T of every selected block, warp w taking slots w and w + 8 on its own TMA
+//      stage (the next K requested as soon as the warp has read the first), the logits kept
+//      in shared memory and each block's per-head maximum;
+//   2. every slot's test at once (a thread per (slot, head): the exclusive prefix maximum
+//      over the earlier slots, then the maximum over the heads);
+//   3. the kept blocks' V, warp w taking kept blocks w and w + 8 on its own stage again, each
+//      warp an online softmax of its own (P from the logits in registers, straight into the
+//      mma A operand);
+//   4. the eight warps' (m, l, O) merged by log-sum-exp.
+// One CTA per unit (128 CTAs for 16 sequences x 8 KV heads: one wave, one per SM), no
+// cluster, no cross-CTA exchange; the V loads of all kept blocks are in flight together.
 template <int D>
-struct SeqLay {
-  static constexpr int kTile = kBlk * D * 2;
-  static constexpr int kKS = 4;  // K stages
-  static constexpr int kVS = 3;  // V stages = P buffers (P V lags two kept blocks)
-  static constexpr int kK = 0;   // TMA boxes: 1024-byte aligned
-  static constexpr int kV = kK + kKS * kTile;
-  static constexpr int kQ = kV + kVS * kTile;
-  static constexpr int kP = kQ + kRows * D * 2;
-  static constexpr int kRed = kP + kVS * kRows * kBlk * 2;
-  static constexpr int kTotal = kRed + kWarps * kRows * 4;
+struct UnitLay {
+  static constexpr int kTile = kBlk * D * 2;                 // one K or V block (bf16)
+  static constexpr int kSSt = kBlk + 4;                      // fp32 row stride of the logits
+  static constexpr int kRing = 0;                            // kWarps stages, 1024-byte aligned
+  static constexpr int kS = kRing + kWarps * kTile;          // [16 slots][16 rows][kSSt] fp32
+  static constexpr int kQ = kS + kCL * kRows * kSSt * 4;     // [16][D] bf16, chunk-swizzled
+  static constexpr int kRmax = kQ + kRows * D * 2;           // [16 slots][16 heads] fp32
+  static constexpr int kTotal = kRmax + kCL * kRows * 4;
+  static_assert(kWarps * kRows * D * 4 <= kWarps * kTile, "the warps' partials fit the ring");
 };
 
 template <int D>
-__global__ void __launch_bounds__(kThreads) decode_blasst_seq_kernel(const __grid_constant__ Params p) {
-  using L = SeqLay<D>;
+__global__ void __launch_bounds__(kThreads, 1) decode_blasst_unit_kernel(const __grid_constant__ Params p) {
+  using L = UnitLay<D>;
   constexpr int kRowBytes = D * 2;
-  constexpr int NT = D / 64;
-  constexpr int kLag = L::kVS - 1;
+  constexpr int NO = D / 8;  // n8 tiles of a warp's output (all D columns)
   extern __shared__ __align__(1024) unsigned char smem[];
-  __shared__ __align__(8) uint64_t kfull[L::kKS], vfull[L::kVS];
+  __shared__ __align__(8) uint64_t kbar[kWarps], vbar[kWarps];
   __shared__ int slot_block[kCL], slot_id[kCL], nslots;
-  __shared__ float rblk[kRows], m_run[kRows], l_run[kRows];
-  __shared__ float alpha_p[L::kVS][kRows];
-  __shared__ int nv_p[L::kVS];
-  __shared__ int keep_flag, skip_flag;
+  __shared__ int kept_slot[kCL], nkept;
+  __shared__ int skipf[kCL];
+  __shared__ float2 ml_w[kWarps][kRows];
   __shared__ int xabort;
   unsigned char* base = smem + ((1024u - (tc::smem_u32(smem) & 1023u)) & 1023u);
-  unsigned char* Kr = base + L::kK;
-  unsigned char* Vr = base + L::kV;
+  unsigned char* ring = base + L::kRing;
+  float* Sbuf = reinterpret_cast<float*>(base + L::kS);
   unsigned char* Qs = base + L::kQ;
-  unsigned char* Pb = base + L::kP;
-  float* red = reinterpret_cast<float*>(base + L::kRed);
+  float* rmax = reinterpret_cast<float*>(base + L::kRmax);
 
   const int g = blockIdx.x, b = blockIdx.y;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -418,16 +423,14 @@ __global__ void __launch_bounds__(kThreads) decode_blasst_seq_kernel(const __gri
   const int T = checked_range(__ldg(p.seqlens + b), 0, p.T_cap, kBoundsSeqlen, kSiteDecodeBlasst);
   const int NBq = (T + kBlk - 1) / kBlk;
   if (tid == 0) {
-    for (int i = 0; i < L::kKS; ++i) tc::mbar_init(&kfull[i], 1);
-    for (int i = 0; i < L::kVS; ++i) tc::mbar_init(&vfull[i], 1);
+    for (int i = 0; i < kWarps; ++i) {
+      tc::mbar_init(&kbar[i], 1);
+      tc::mbar_init(&vbar[i], 1);
+    }
     xabort = 0;
     tc::fence_mbar_init();
     tc::prefetch_tmap(&p.tmk);
     tc::prefetch_tmap(&p.tmv);
-  }
-  if (tid < kRows) {
-    m_run[tid] = -INFINITY;
-    l_run[tid] = 0.f;
   }
   // the slots holding a block, compacted in ascending slot order
   if (warp == 0) {
@@ -454,226 +457,251 @@ __global__ void __launch_bounds__(kThreads) decode_blasst_seq_kernel(const __gri
   }
   __syncthreads();  // (the slot list and the barriers are set up)
   const int n = nslots;
-  int k_issued = 0;
-  auto issue_k = [&](int i) {  // thread 0: K of the i-th visited block into stage i % kKS
-    const int st = i % L::kKS;
-    tc::fence_proxy_async();  // earlier generic reads of the stage come first
-    tc::mbar_arrive_expect_tx(&kfull[st], (uint32_t)L::kTile);
+  unsigned char* stage = ring + warp * L::kTile;  // this warp's TMA stage
+  // lane 0 of the warp: block j of `map` into this warp's stage, completing on `bar`
+  auto load_block = [&](const CUtensorMap* map, int j, uint64_t* bar) {
+    tc::fence_proxy_async();  // this warp's earlier reads of the stage come first
+    tc::mbar_arrive_expect_tx(bar, (uint32_t)L::kTile);
 #pragma unroll
-    for (int h = 0; h < D / 64; ++h)
-      tc::tma_load_3d(Kr + st * L::kTile + h * 8192, &p.tmk, h * 64, slot_block[i] * kBlk, unit, &kfull[st]);
+    for (int h = 0; h < D / 64; ++h) tc::tma_load_3d(stage + h * 8192, map, h * 64, j * kBlk, unit, bar);
   };
-  if (tid == 0)
-    for (int i = 0; i < n && i < L::kKS; ++i) issue_k(i);
-  k_issued = n < L::kKS ? n : L::kKS;
+  // loads issued on this warp's barriers and waited for: a load is issued only after the
+  // previous one on the same barrier was seen complete, so at most one is ever in flight
+  int k_issued = 0, k_seen = 0, v_issued = 0, v_seen = 0;
+  // lane 0 of the warp: block j of `map` pulled into L2 for a later load
+  auto prefetch_block = [&](const CUtensorMap* map, int j) {
+#pragma unroll
+    for (int h = 0; h < D / 64; ++h) tc::tma_prefetch_l2_3d(map, h * 64, j * kBlk, unit);
+  };
+  if (lane == 0 && warp < n) {
+    load_block(&p.tmk, slot_block[warp], &kbar[warp]);
+    k_issued = 1;
+    // the second round's K waits for this stage: bring it into L2 meanwhile
+    if (warp + kWarps < n) prefetch_block(&p.tmk, slot_block[warp + kWarps]);
+  }
   cp_async_wait<0>();
-  __syncthreads();
+  __syncthreads();  // (q)
   uint32_t qa[D / 16][4];
 #pragma unroll
   for (int ks = 0; ks < D / 16; ++ks) {
     const int row = (lane & 7) + 8 * ((lane >> 3) & 1);
     ldsm_x4(qa[ks], Qs + swz(row, 2 * ks + (lane >> 4), kRowBytes));
   }
-  float acc[NT][4];
+  const int r0 = lane >> 2, q2 = 2 * (lane & 3);
+
+  // ---- 1. logits and block maxima of every slot ---------------------------------------------
+  for (int round = 0; round < 2; ++round) {
+    const int i = warp + kWarps * round;
+    if (i >= n) break;
+    const bool ok = __all_sync(0xffffffffu, tc::mbar_wait(&kbar[warp], (uint32_t)round, &xabort, p.budget));
+    k_seen += ok ? 1 : 0;
+    const int nv = max(0, min(kBlk, T - slot_block[i] * kBlk));
+    float* Si = Sbuf + i * kRows * L::kSSt;
+    float mlo = -INFINITY, mhi = -INFINITY;
 #pragma unroll
-  for (int nt = 0; nt < NT; ++nt)
+    for (int nt = 0; nt < kBlk / 8; ++nt) {
+      float c4[4] = {0.f, 0.f, 0.f, 0.f};
+      if (ok) {
+#pragma unroll
+        for (int ks = 0; ks < D / 16; ks += 2) {
+          uint32_t kb[4];
+          ldsm_x4(kb, stage + kv_off(8 * nt + (lane & 7), 2 * ks + (lane >> 3)));
+          mma_bf16(c4, qa[ks], kb[0], kb[1]);
+          mma_bf16(c4, qa[ks + 1], kb[2], kb[3]);
+        }
+      }
+      const int col = 8 * nt + q2;
+      const bool v0 = col < nv, v1 = col + 1 < nv;
+      const float s0 = v0 && r0 < G ? c4[0] * p.scale2 : -INFINITY;
+      const float s1 = v1 && r0 < G ? c4[1] * p.scale2 : -INFINITY;
+      const float s2 = v0 && r0 + 8 < G ? c4[2] * p.scale2 : -INFINITY;
+      const float s3 = v1 && r0 + 8 < G ? c4[3] * p.scale2 : -INFINITY;
+      *reinterpret_cast<float2*>(Si + r0 * L::kSSt + col) = make_float2(s0, s1);
+      *reinterpret_cast<float2*>(Si + (r0 + 8) * L::kSSt + col) = make_float2(s2, s3);
+      mlo = fmaxf(mlo, fmaxf(s0, s1));
+      mhi = fmaxf(mhi, fmaxf(s2, s3));
+    }
+#pragma unroll
+    for (int o2 = 1; o2 < 4; o2 <<= 1) {
+      mlo = fmaxf(mlo, __shfl_xor_sync(0xffffffffu, mlo, o2));
+      mhi = fmaxf(mhi, __shfl_xor_sync(0xffffffffu, mhi, o2));
+    }
+    if ((lane & 3) == 0) {
+      rmax[i * kRows + r0] = mlo;
+      rmax[i * kRows + r0 + 8] = mhi;
+    }
+    __syncwarp();  // (every lane has read the stage)
+    if (!ok) break;
+    if (lane == 0 && round == 0 && i + kWarps < n) {
+      load_block(&p.tmk, slot_block[i + kWarps], &kbar[warp]);
+      k_issued = 2;
+    }
+  }
+  __syncthreads();
+
+  // ---- 2. the test of every slot: a thread per (slot, head) ---------------------------------
+  {
+    const int sl = tid >> 4, h = tid & 15;  // (kThreads = 16 slots x 16 heads)
+    float gi = -INFINITY;
+    if (sl < n && h < G) {
+      const float r = rmax[sl * kRows + h];
+      float m = -INFINITY;  // the maximum over the earlier slots = the running maximum
+      for (int e = 0; e < sl; ++e) m = fmaxf(m, rmax[e * kRows + h]);
+      gi = r == -INFINITY ? -INFINITY : (m == -INFINITY ? INFINITY : r - m);
+    }
+#pragma unroll
+    for (int o2 = 8; o2 > 0; o2 >>= 1) gi = fmaxf(gi, __shfl_xor_sync(0xffffffffu, gi, o2));
+    if (h == 0 && sl < kCL) skipf[sl] = sl > 0 && sl < n && gi < p.log2_lambda;
+  }
+  __syncthreads();
+  if (warp == 0) {  // the kept slots in order, and the skip bits by selection slot
+    const bool in = lane < n;
+    const bool keep = in && !skipf[lane];
+    const uint32_t kb2 = __ballot_sync(0xffffffffu, keep);
+    const uint32_t sb = __ballot_sync(0xffffffffu, in && skipf[lane]);
+    if (keep) kept_slot[__popc(kb2 & ((1u << lane) - 1u))] = lane;
+    if (lane == 0) nkept = __popc(kb2);
+    uint32_t bits = 0u;
+    for (int e = 0; e < 32; ++e)
+      if ((sb >> e) & 1u) bits |= 1u << slot_id[e];
+    if (lane == 0 && p.skip_bits) p.skip_bits[unit] = bits;
+  }
+  __syncthreads();
+  const int nk = nkept;
+
+  // ---- 3. the kept blocks: V, then P V in each warp's own online softmax --------------------
+  if (lane == 0 && warp < nk && *reinterpret_cast<volatile int*>(&xabort) == 0) {
+    load_block(&p.tmv, slot_block[kept_slot[warp]], &vbar[warp]);
+    v_issued = 1;
+    if (warp + kWarps < nk) prefetch_block(&p.tmv, slot_block[kept_slot[warp + kWarps]]);
+  }
+  float acc[NO][4];
+#pragma unroll
+  for (int nt = 0; nt < NO; ++nt)
 #pragma unroll
     for (int e = 0; e < 4; ++e) acc[nt][e] = 0.f;
-  const int r0 = lane >> 2;
-  const int col = 8 * warp + 2 * (lane & 3);
-  uint32_t skipped = 0u;
-  int vk = 0, pv_done = 0;
-
-  // P V of the k-th kept block (in order): O = alpha_k O + P_k V_k
-  auto process_pv = [&](int k) {
-    const int st = k % L::kVS;
-    tc::mbar_wait(&vfull[st], (uint32_t)((k / L::kVS) & 1), &xabort, p.budget);
-    unsigned char* Vs = Vr + st * L::kTile;
-    const int nv = nv_p[st];
-    for (int id = tid; id < (kBlk - nv) * (D / 8); id += kThreads) {  // rows past the sequence
+  float m_lo = -INFINITY, m_hi = -INFINITY, l_lo = 0.f, l_hi = 0.f;
+  for (int round = 0; round < 2; ++round) {
+    const int k = warp + kWarps * round;
+    if (k >= nk) break;
+    const int i = kept_slot[k];
+    const bool ok = __all_sync(0xffffffffu, tc::mbar_wait(&vbar[warp], (uint32_t)round, &xabort, p.budget));
+    v_seen += ok ? 1 : 0;
+    if (!ok) break;
+    const int nv = max(0, min(kBlk, T - slot_block[i] * kBlk));
+    // V rows past the sequence hold whatever the cache holds there: zero them (P is 0 there)
+    for (int id = lane; id < (kBlk - nv) * (D / 8); id += 32) {
       const int r = nv + id / (D / 8), c = id % (D / 8);
-      *reinterpret_cast<uint4*>(Vs + kv_off(r, c)) = make_uint4(0u, 0u, 0u, 0u);
+      *reinterpret_cast<uint4*>(stage + kv_off(r, c)) = make_uint4(0u, 0u, 0u, 0u);
     }
-    __syncthreads();
-    const float a_lo = alpha_p[st][r0], a_hi = alpha_p[st][r0 + 8];
+    __syncwarp();
+    const float* Si = Sbuf + i * kRows * L::kSSt;
+    const float rlo = rmax[i * kRows + r0], rhi = rmax[i * kRows + r0 + 8];
+    const float nlo = fmaxf(m_lo, rlo), nhi = fmaxf(m_hi, rhi);
+    const float alo = m_lo == -INFINITY ? 0.f : ex2(m_lo - nlo);
+    const float ahi = m_hi == -INFINITY ? 0.f : ex2(m_hi - nhi);
+    m_lo = nlo;
+    m_hi = nhi;
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-      acc[nt][0] *= a_lo; acc[nt][1] *= a_lo;
-      acc[nt][2] *= a_hi; acc[nt][3] *= a_hi;
+    for (int nt = 0; nt < NO; ++nt) {
+      acc[nt][0] *= alo; acc[nt][1] *= alo;
+      acc[nt][2] *= ahi; acc[nt][3] *= ahi;
     }
-    const unsigned char* Ps = Pb + st * (kRows * kBlk * 2);
+    float slo = 0.f, shi = 0.f;
 #pragma unroll
-    for (int ks = 0; ks < kBlk / 16; ++ks) {
+    for (int kk = 0; kk < kBlk / 16; ++kk) {
+      // P of keys 16 kk .. 16 kk + 15 as the mma A operand, from the logits (rows r0, r0 + 8)
       uint32_t pa[4];
-      const int row = (lane & 7) + 8 * ((lane >> 3) & 1);
-      ldsm_x4(pa, Ps + swz(row, 2 * ks + (lane >> 4), kBlk * 2));
-      const int vrow = 16 * ks + (lane & 7) + 8 * ((lane >> 3) & 1);
-      if constexpr (D == 128) {
-        uint32_t vb[4];
-        ldsm_x4_t(vb, Vs + kv_off(vrow, 2 * warp + (lane >> 4)));
-        mma_bf16(acc[0], pa, vb[0], vb[1]);
-        mma_bf16(acc[1], pa, vb[2], vb[3]);
-      } else {
-        uint32_t vb[2];
-        ldsm_x2_t(vb, Vs + kv_off(vrow, warp));
-        mma_bf16(acc[0], pa, vb[0], vb[1]);
+#pragma unroll
+      for (int hf = 0; hf < 2; ++hf) {
+        const int col = 16 * kk + 8 * hf + q2;
+        const float2 xl = *reinterpret_cast<const float2*>(Si + r0 * L::kSSt + col);
+        const float2 xh = *reinterpret_cast<const float2*>(Si + (r0 + 8) * L::kSSt + col);
+        const float p0 = xl.x == -INFINITY ? 0.f : ex2(xl.x - nlo);
+        const float p1 = xl.y == -INFINITY ? 0.f : ex2(xl.y - nlo);
+        const float p2 = xh.x == -INFINITY ? 0.f : ex2(xh.x - nhi);
+        const float p3 = xh.y == -INFINITY ? 0.f : ex2(xh.y - nhi);
+        slo += p0 + p1;
+        shi += p2 + p3;
+        pa[2 * hf] = pack_bf16x2(p0, p1);
+        pa[2 * hf + 1] = pack_bf16x2(p2, p3);
+      }
+      if (ok) {
+        const int vrow = 16 * kk + (lane & 7) + 8 * ((lane >> 3) & 1);
+#pragma unroll
+        for (int np = 0; np < D / 16; ++np) {
+          uint32_t vb[4];
+          ldsm_x4_t(vb, stage + kv_off(vrow, 2 * np + (lane >> 4)));
+          mma_bf16(acc[2 * np], pa, vb[0], vb[1]);
+          mma_bf16(acc[2 * np + 1], pa, vb[2], vb[3]);
+        }
       }
     }
-    __syncthreads();  // the stage and the P buffer may be reused
-    ++pv_done;
-  };
-
-  for (int i = 0; i < n; ++i) {
-    const int j = slot_block[i];
-    const int nv = max(0, min(kBlk, T - j * kBlk));
-    const int kst = i % L::kKS;
-    tc::mbar_wait(&kfull[kst], (uint32_t)((i / L::kKS) & 1), &xabort, p.budget);
-    // S = Q K^T (base-2 logits): warp w takes keys 8w .. 8w + 7
-    float s[4];
-    {
-      const unsigned char* Ks = Kr + kst * L::kTile;
-      float c4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int ks = 0; ks < D / 16; ks += 2) {
-        uint32_t kb[4];
-        ldsm_x4(kb, Ks + kv_off(8 * warp + (lane & 7), 2 * ks + (lane >> 3)));
-        mma_bf16(c4, qa[ks], kb[0], kb[1]);
-        mma_bf16(c4, qa[ks + 1], kb[2], kb[3]);
-      }
-      const bool v0 = col < nv, v1 = col + 1 < nv;
-      s[0] = v0 && r0 < G ? c4[0] * p.scale2 : -INFINITY;
-      s[1] = v1 && r0 < G ? c4[1] * p.scale2 : -INFINITY;
-      s[2] = v0 && r0 + 8 < G ? c4[2] * p.scale2 : -INFINITY;
-      s[3] = v1 && r0 + 8 < G ? c4[3] * p.scale2 : -INFINITY;
+    for (int o2 = 1; o2 < 4; o2 <<= 1) {
+      slo += __shfl_xor_sync(0xffffffffu, slo, o2);
+      shi += __shfl_xor_sync(0xffffffffu, shi, o2);
     }
-    {  // the block maxima
-      float m_lo = fmaxf(s[0], s[1]), m_hi = fmaxf(s[2], s[3]);
-#pragma unroll
-      for (int o2 = 1; o2 < 4; o2 <<= 1) {
-        m_lo = fmaxf(m_lo, __shfl_xor_sync(0xffffffffu, m_lo, o2));
-        m_hi = fmaxf(m_hi, __shfl_xor_sync(0xffffffffu, m_hi, o2));
-      }
-      if ((lane & 3) == 0) {
-        red[warp * kRows + r0] = m_lo;
-        red[warp * kRows + r0 + 8] = m_hi;
-      }
+    l_lo = l_lo * alo + slo;
+    l_hi = l_hi * ahi + shi;
+    __syncwarp();  // (every lane has read the stage)
+    if (lane == 0 && round == 0 && k + kWarps < nk) {
+      load_block(&p.tmv, slot_block[kept_slot[k + kWarps]], &vbar[warp]);
+      v_issued = 2;
     }
-    __syncthreads();  // (every warp has read K_i: its stage may be refilled)
-    if (tid == 0 && k_issued < n) issue_k(k_issued);
-    k_issued = k_issued < n ? k_issued + 1 : n;
-    // the test (warp 0, lane h = head h): skip iff not the first visited block and every
-    // head's block maximum trails its running maximum by more than -log2(lambda)
-    if (warp == 0) {
-      float r = -INFINITY;
-      if (lane < kRows) {
-#pragma unroll
-        for (int w = 0; w < kWarps; ++w) r = fmaxf(r, red[w * kRows + lane]);
-        rblk[lane] = r;
-      }
-      float gi = -INFINITY;
-      if (lane < G) {
-        const float m = m_run[lane];
-        gi = r == -INFINITY ? -INFINITY : (m == -INFINITY ? INFINITY : r - m);
-      }
-#pragma unroll
-      for (int o2 = 16; o2 > 0; o2 >>= 1) gi = fmaxf(gi, __shfl_xor_sync(0xffffffffu, gi, o2));
-      if (lane == 0) {
-        const bool sk = i > 0 && gi < p.log2_lambda;
-        skip_flag = sk;
-        keep_flag = !sk && nv > 0;
-      }
-    }
-    __syncthreads();
-    if (skip_flag) skipped |= 1u << slot_id[i];
-    if (!keep_flag) continue;
-    // kept: V_i into stage vk % kVS (its previous occupant's P V is done), P_i, statistics
-    const int vst = vk % L::kVS;
-    if (tid == 0) {
-      tc::fence_proxy_async();
-      tc::mbar_arrive_expect_tx(&vfull[vst], (uint32_t)L::kTile);
-#pragma unroll
-      for (int h = 0; h < D / 64; ++h)
-        tc::tma_load_3d(Vr + vst * L::kTile + h * 8192, &p.tmv, h * 64, j * kBlk, unit, &vfull[vst]);
-      nv_p[vst] = nv;
-    }
-    {
-      const float ml = fmaxf(m_run[r0], rblk[r0]), mh = fmaxf(m_run[r0 + 8], rblk[r0 + 8]);
-      const float p0 = s[0] == -INFINITY ? 0.f : ex2(s[0] - ml);
-      const float p1 = s[1] == -INFINITY ? 0.f : ex2(s[1] - ml);
-      const float p2 = s[2] == -INFINITY ? 0.f : ex2(s[2] - mh);
-      const float p3 = s[3] == -INFINITY ? 0.f : ex2(s[3] - mh);
-      unsigned char* Ps = Pb + vst * (kRows * kBlk * 2);
-      *reinterpret_cast<uint32_t*>(Ps + swz(r0, col >> 3, kBlk * 2) + (col & 7) * 2) = pack_bf16x2(p0, p1);
-      *reinterpret_cast<uint32_t*>(Ps + swz(r0 + 8, col >> 3, kBlk * 2) + (col & 7) * 2) = pack_bf16x2(p2, p3);
-      float l_lo = p0 + p1, l_hi = p2 + p3;
-#pragma unroll
-      for (int o2 = 1; o2 < 4; o2 <<= 1) {
-        l_lo += __shfl_xor_sync(0xffffffffu, l_lo, o2);
-        l_hi += __shfl_xor_sync(0xffffffffu, l_hi, o2);
-      }
-      if ((lane & 3) == 0) {  // (red's maxima were read before the last barrier)
-        red[warp * kRows + r0] = l_lo;
-        red[warp * kRows + r0 + 8] = l_hi;
-      }
-    }
-    __syncthreads();
-    if (tid < kRows) {
-      const float mo = m_run[tid], mn = fmaxf(mo, rblk[tid]);
-      float ls = 0.f;
-#pragma unroll
-      for (int w = 0; w < kWarps; ++w) ls += red[w * kRows + tid];
-      const float a = mo == -INFINITY ? 0.f : ex2(mo - mn);
-      alpha_p[vst][tid] = a;
-      l_run[tid] = l_run[tid] * a + ls;
-      m_run[tid] = mn;
-    }
-    __syncthreads();  // (red, m_run and the block's statistics: the next block rewrites them)
-    ++vk;
-    if (vk - 1 - kLag >= 0) process_pv(vk - 1 - kLag);
   }
-  while (pv_done < vk) process_pv(pv_done);
-  __syncthreads();  // (the statistics are final)
+  __syncthreads();  // (every stage has been read: the ring holds the partials now)
 
-  // outputs: rows r0, r0 + 8 of the group, columns of this warp's n-tiles
+  // ---- 4. the warps' partials, merged by log-sum-exp ---------------------------------------
+  float* part = reinterpret_cast<float*>(ring);  // [warp][16 rows][D]
+#pragma unroll
+  for (int nt = 0; nt < NO; ++nt) {
+    const int d = 8 * nt + q2;
+    *reinterpret_cast<float2*>(part + (warp * kRows + r0) * D + d) = make_float2(acc[nt][0], acc[nt][1]);
+    *reinterpret_cast<float2*>(part + (warp * kRows + r0 + 8) * D + d) = make_float2(acc[nt][2], acc[nt][3]);
+  }
+  if ((lane & 3) == 0) {
+    ml_w[warp][r0] = make_float2(m_lo, l_lo);
+    ml_w[warp][r0 + 8] = make_float2(m_hi, l_hi);
+  }
+  __syncthreads();
   const size_t orow = (size_t)b * Hq + (size_t)g * G;
+  for (int e = tid; e < G * D; e += kThreads) {
+    const int h = e / D, d = e - h * D;
+    float M = -INFINITY;
 #pragma unroll
-  for (int half = 0; half < 2; ++half) {
-    const int h = r0 + 8 * half;
-    if (h < G) {
-      const float l = l_run[h];
-      const float inv = l > 0.f ? 1.f / l : 0.f;
+    for (int w = 0; w < kWarps; ++w) M = fmaxf(M, ml_w[w][h].x);
+    float Lsum = 0.f, O = 0.f;
+    if (M != -INFINITY) {
 #pragma unroll
-      for (int nt = 0; nt < NT; ++nt) {
-        const int d = (D == 128 ? 16 * warp : 8 * warp) + 8 * nt + 2 * (lane & 3);
-        *reinterpret_cast<uint32_t*>(p.o + (orow + h) * D + d) =
-            pack_bf16x2(acc[nt][2 * half] * inv, acc[nt][2 * half + 1] * inv);
+      for (int w = 0; w < kWarps; ++w) {
+        const float2 ml = ml_w[w][h];
+        const float wt = ml.x == -INFINITY ? 0.f : ex2(ml.x - M);
+        Lsum = fmaf(ml.y, wt, Lsum);
+        O = fmaf(part[(w * kRows + h) * D + d], wt, O);
       }
     }
+    p.o[(orow + h) * D + d] = __float2bfloat16_rn(Lsum > 0.f ? O / Lsum : 0.f);
+    if (d == 0 && p.lse) p.lse[orow + h] = Lsum > 0.f ? (M + log2f(Lsum)) * kLn2 : -INFINITY;
   }
-  if (tid < G && p.lse) {
-    const float l = l_run[tid];
-    p.lse[orow + tid] = l > 0.f ? (m_run[tid] + log2f(l)) * kLn2 : -INFINITY;
-  }
-  if (tid == 0 && p.skip_bits) p.skip_bits[unit] = skipped;
-  // after a timeout (the outputs are then undefined): the copies still in flight land
-  // before the CTA exits
+  // after a timeout (the outputs are then undefined): this warp's copies still in flight
+  // land before the CTA exits
   if (*reinterpret_cast<volatile int*>(&xabort)) {
-    for (int i = k_issued - L::kKS < 0 ? 0 : k_issued - L::kKS; i < k_issued; ++i)
-      tc::mbar_drain(&kfull[i % L::kKS], (uint32_t)((i / L::kKS) & 1), kDrainBudget);
-    for (int k = vk - L::kVS < 0 ? 0 : vk - L::kVS; k < vk; ++k)
-      tc::mbar_drain(&vfull[k % L::kVS], (uint32_t)((k / L::kVS) & 1), kDrainBudget);
-    g_blasst_decode_status = 1;
+    if (lane == 0) {
+      if (k_issued > k_seen) tc::mbar_drain(&kbar[warp], (uint32_t)((k_issued - 1) & 1), kDrainBudget);
+      if (v_issued > v_seen) tc::mbar_drain(&vbar[warp], (uint32_t)((v_issued - 1) & 1), kDrainBudget);
+    }
+    if (tid == 0) g_blasst_decode_status = 1;
   }
 }
 
-// Units from which one CTA per unit (walking its blocks in order) fills the GPU better
-// than a 16-CTA cluster per unit.
-constexpr int kSeqUnits = 64;
+// Units from which one CTA per unit fills the GPU better than a 16-CTA cluster per unit.
+constexpr int kUnitKernelUnits = 64;
 
 template <int D>
-cudaError_t launch_seq(const DecodeBlasstArgs& a, const Params& p, cudaStream_t stream) {
-  auto kernel = decode_blasst_seq_kernel<D>;
-  const int smem = SeqLay<D>::kTotal + 1024;
+cudaError_t launch_unit(const DecodeBlasstArgs& a, const Params& p, cudaStream_t stream) {
+  auto kernel = decode_blasst_unit_kernel<D>;
+  const int smem = UnitLay<D>::kTotal + 1024;
   static DeviceOnce attr_once;
   const cudaError_t err = attr_once.run([&]() {
     return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
@@ -702,7 +730,7 @@ cudaError_t launch_d(const DecodeBlasstArgs& a, cudaStream_t stream) {
   p.lse = a.lse;
   p.skip_bits = a.skip_bits;
   p.budget = wait_budget();
-  if (a.B * a.Hkv >= kSeqUnits) return launch_seq<D>(a, p, stream);
+  if (a.B * a.Hkv >= kUnitKernelUnits) return launch_unit<D>(a, p, stream);
   const int smem = Lay<D>::kTotal + 1024;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(kCL, a.Hkv, a.B);

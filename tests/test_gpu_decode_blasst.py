@@ -148,7 +148,7 @@ def test_decode_blasst_64k_workload(lsa):
         _check(q, case.k, case.v, case.seqlens, idx, nsel, lam, o, lse, bits, f"64k x{qscale}")
 
 
-# ---- many (b, g) units: one CTA per unit walks its blocks in order (64 units and up) ----
+# ---- many (b, g) units: one CTA per unit, in phases (64 units and up) ----
 
 @pytest.mark.parametrize("kw,qscale,lam", [
     (dict(B=32, Hkv=2, G=4, D=128, T_cap=3000, seqlens=None, topk=8, n_needles=3), 4.0, 1e-2),
