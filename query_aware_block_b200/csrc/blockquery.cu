@@ -595,6 +595,38 @@ __global__ void __launch_bounds__(kThreads, 2) blockquery_kernel(const __grid_co
   }
 
   // ---- barrier (the partials are in the workspace), then merge my output slice ----------
+  // Stable rows: the cached output and log-sum-exp, unchanged.  Each thread loads its first
+  // chunk here, before the cluster barrier, and stores it after the merge, so that round
+  // trip overlaps the barrier and the merge's own loads; any further chunks (more stable
+  // rows than threads) are copied after the merge.
+  const int srows = S * G;
+  const bool copy_o = p.o_cache != p.o && srows > 0;
+  const bool copy_l = p.lse_cache != p.lse && srows > 0;
+  constexpr int kPerRow = kRowBytes / 16;  // 16-byte chunks of an output row
+  const int n16 = srows * kPerRow;
+  const int c16 = (n16 + CL - 1) >> cl_log2;
+  const int i16 = rank * c16 + tid, i16_end = min(n16, (rank + 1) * c16);
+  const int c1 = (srows + CL - 1) >> cl_log2;
+  const int li = rank * c1 + tid, l_end = min(srows, (rank + 1) * c1);
+  auto stable_row = [&](int r) {  // row r of the stable rows: token stab[r / G], head r % G
+    const int s_i = fdiv(r, p.g_div), hh = r - s_i * G;
+    return ((size_t)b * Hq + (size_t)g * G + hh) * Tq + stab[s_i];
+  };
+  const bool have_o = copy_o && i16 < i16_end;
+  const bool have_l = copy_l && li < l_end;
+  uint4 o_keep = make_uint4(0u, 0u, 0u, 0u);
+  size_t o_at = 0, l_at = 0;
+  float l_keep = 0.f;
+  if (have_o) {
+    const int r = i16 / kPerRow;
+    o_at = stable_row(r) * kPerRow + (i16 - r * kPerRow);
+    o_keep = reinterpret_cast<const uint4*>(p.o_cache)[o_at];
+  }
+  if (have_l) {
+    l_at = stable_row(li);
+    l_keep = p.lse_cache[l_at];
+  }
+
   if (!started) {
     cluster_wait();
     started = true;
@@ -639,25 +671,20 @@ __global__ void __launch_bounds__(kThreads, 2) blockquery_kernel(const __grid_co
     if (d == 0) p.lse[orow] = M == -INFINITY ? -INFINITY : (M + log2f(Lsum)) * kLn2;
   }
 
-  // ---- stable rows: the cached output and log-sum-exp, unchanged --------------------------
-  const int srows = S * G;
-  if (p.o_cache != p.o && srows > 0) {
-    const int per_row = kRowBytes / 16;
-    const int n16 = srows * per_row;
-    const int c16 = (n16 + CL - 1) >> cl_log2;
-    for (int i = rank * c16 + tid; i < min(n16, (rank + 1) * c16); i += kThreads) {
-      const int r = i / per_row, cc = i - r * per_row;
-      const int s_i = fdiv(r, p.g_div), hh = r - s_i * G;
-      const size_t orow = ((size_t)b * Hq + (size_t)g * G + hh) * Tq + stab[s_i];
-      reinterpret_cast<uint4*>(p.o + orow * D)[cc] = reinterpret_cast<const uint4*>(p.o_cache + orow * D)[cc];
+  // ---- stable rows: the chunks loaded before the barrier, then any further ones -----------
+  if (have_o) reinterpret_cast<uint4*>(p.o)[o_at] = o_keep;
+  if (copy_o) {
+    for (int i = i16 + kThreads; i < i16_end; i += kThreads) {
+      const int r = i / kPerRow;
+      const size_t at = stable_row(r) * kPerRow + (i - r * kPerRow);
+      reinterpret_cast<uint4*>(p.o)[at] = reinterpret_cast<const uint4*>(p.o_cache)[at];
     }
   }
-  if (p.lse_cache != p.lse && srows > 0) {
-    const int c1 = (srows + CL - 1) >> cl_log2;
-    for (int r = rank * c1 + tid; r < min(srows, (rank + 1) * c1); r += kThreads) {
-      const int s_i = fdiv(r, p.g_div), hh = r - s_i * G;
-      const size_t orow = ((size_t)b * Hq + (size_t)g * G + hh) * Tq + stab[s_i];
-      p.lse[orow] = p.lse_cache[orow];
+  if (have_l) p.lse[l_at] = l_keep;
+  if (copy_l) {
+    for (int r = li + kThreads; r < l_end; r += kThreads) {
+      const size_t at = stable_row(r);
+      p.lse[at] = p.lse_cache[at];
     }
   }
 
