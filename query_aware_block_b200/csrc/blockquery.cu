@@ -92,7 +92,7 @@ struct alignas(64) BQParams {
 __host__ __device__ inline size_t al128(size_t x) { return (x + 127) & ~(size_t)127; }
 
 struct BQLayout {
-  size_t act, stab, ulist, ubits, qs, ss, ps, alpha, region, total;
+  size_t act, stab, ulist, ubits, qs, ss, ps, alpha, pml, pacc, region, total;
   // selection buffers, inside `region` (dead once the attention starts)
   size_t qsum, keys, top, recv, sumbuf, qrows;
   size_t kv_tile;
@@ -115,6 +115,10 @@ __host__ __device__ inline BQLayout bq_layout(int D, int per_max, int NBp, int G
   L.ss = off;     off = al128(off + (size_t)kRowChunk * kSStride * 4);
   L.ps = off;     off = al128(off + (size_t)kRowChunk * kBlk * 2);
   L.alpha = off;  off = al128(off + kRowChunk * 4);
+  // the partials pushed by the cluster's CTAs when the rows fit one chunk: every CTA's
+  // (m, l) of every row and its part of this CTA's slice of the outputs
+  L.pml = off;    off = al128(off + (size_t)kMaxCluster * kRowChunk * 8);
+  L.pacc = off;   off = al128(off + (size_t)kRowChunk * D * 4 + kMaxCluster * 8);
   L.region = off;
   L.kv_tile = (size_t)kBlk * D * 2;
   // the K/V ring starts at the first 1024-byte boundary of the region (TMA 128-byte swizzle)
@@ -149,6 +153,8 @@ __global__ void __launch_bounds__(kThreads, 2) blockquery_kernel(const __grid_co
   float* Ss = reinterpret_cast<float*>(smem + Lo.ss);
   unsigned char* Ps = smem + Lo.ps;
   float* alpha_s = reinterpret_cast<float*>(smem + Lo.alpha);
+  float2* pml = reinterpret_cast<float2*>(smem + Lo.pml);
+  float* pacc = reinterpret_cast<float*>(smem + Lo.pacc);
   unsigned char* region = smem + Lo.region;
   float* qsum = reinterpret_cast<float*>(region + Lo.qsum);
   u64* keys = reinterpret_cast<u64*>(region + Lo.keys);
@@ -167,12 +173,13 @@ __global__ void __launch_bounds__(kThreads, 2) blockquery_kernel(const __grid_co
   const bool all_blocks = NBp <= p.topk;
   // mbarriers: [0], [1] count the bytes of the candidate-list exchange (two buffers, one
   // phase per token chunk that uses the buffer); [2] the bulk copy of the summary slice;
-  // [3 + s] the TMA loads into K/V stage s (one phase per use of the stage)
-  __shared__ __align__(8) uint64_t xbar[3 + kStages];
+  // [3 + s] the TMA loads into K/V stage s (one phase per use of the stage); [3 + kStages]
+  // the partials pushed into this CTA (one phase)
+  __shared__ __align__(8) uint64_t xbar[4 + kStages];
   __shared__ int xabort;
   const int staged_rows = all_blocks ? 0 : min(nloc, kStageRows);
   if (tid == 0) {
-    for (int i = 0; i < 3 + kStages; ++i) tc::mbar_init(&xbar[i], 1);
+    for (int i = 0; i < 4 + kStages; ++i) tc::mbar_init(&xbar[i], 1);
     xabort = 0;
     tc::fence_mbar_init();
     tc::prefetch_tmap(&p.tmk);
@@ -422,6 +429,10 @@ __global__ void __launch_bounds__(kThreads, 2) blockquery_kernel(const __grid_co
 
   // ---- attention: rows (active token x head) in chunks of 32, my union blocks -----------
   const int nchunks = (rows + kRowChunk - 1) / kRowChunk;
+  // one chunk of rows: the partials go straight into the shared memory of the CTAs that
+  // merge them (st.async, counted on the owner's mbarrier), with no workspace round trip and
+  // no cluster barrier; more rows go through the caller's workspace
+  const bool dsm = nchunks == 1;
   const int total = nchunks * n_my;
   float* wsu = p.ws + (unit * kMaxCluster + rank) * (size_t)p.rows_max * (D + 2);
   int issued = 0;
@@ -574,9 +585,10 @@ __global__ void __launch_bounds__(kThreads, 2) blockquery_kernel(const __grid_co
       __syncthreads();  // the stage may now be refilled
       if (issued < total) issue();
     }
-    // partial of this chunk -> workspace: acc rows, then (m, l)
+    // partial of this chunk -> workspace: acc rows, then (m, l) (rows that fit one chunk are
+    // pushed to the owners' shared memory instead, below)
 #pragma unroll
-    for (int mt = 0; mt < 2; ++mt) {
+    for (int mt = 0; mt < 2 && !dsm; ++mt) {
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
         const int d = (D == 128 ? 16 * warp : 8 * warp) + 8 * nt + 2 * (lane & 3);
@@ -589,7 +601,7 @@ __global__ void __launch_bounds__(kThreads, 2) blockquery_kernel(const __grid_co
         }
       }
     }
-    if (ssub == 0 && srow < nr)
+    if (!dsm && ssub == 0 && srow < nr)
       *reinterpret_cast<float2*>(wsu + (size_t)(c0 + srow) * (D + 2) + D) = make_float2(m_run, l_run);
     __syncthreads();  // Qs / stats are rewritten by the next chunk
   }
@@ -631,28 +643,10 @@ __global__ void __launch_bounds__(kThreads, 2) blockquery_kernel(const __grid_co
     cluster_wait();
     started = true;
   }
-  cluster_arrive_release();
-  cluster_wait();
-
   const int E = rows * D;
-  const int chunk = (E + CL - 1) >> cl_log2;
-  const float* wsg = p.ws + unit * kMaxCluster * (size_t)p.rows_max * (D + 2);
-  for (int e = rank * chunk + tid; e < min(E, (rank + 1) * chunk); e += kThreads) {
+  // an output row's (m, l) and values from the CL partials: the log-sum-exp merge
+  auto merge_out = [&](int e, const float2 (&ml)[kMaxCluster], const float (&ov)[kMaxCluster]) {
     const int r = e / D, d = e - r * D;
-    // every partial's (m, l) and value first (independent loads, one round trip), then
-    // the log-sum-exp weights
-    float2 ml[kMaxCluster];
-    float ov[kMaxCluster];
-#pragma unroll
-    for (int c2 = 0; c2 < kMaxCluster; ++c2) {
-      ml[c2] = make_float2(-INFINITY, 0.f);
-      ov[c2] = 0.f;
-      if (c2 < CL) {
-        const float* part = wsg + ((size_t)c2 * p.rows_max + r) * (D + 2);
-        ml[c2] = __ldcg(reinterpret_cast<const float2*>(part + D));
-        ov[c2] = __ldcg(part + d);
-      }
-    }
     float M = -INFINITY;
 #pragma unroll
     for (int c2 = 0; c2 < kMaxCluster; ++c2) M = fmaxf(M, ml[c2].x);
@@ -669,6 +663,69 @@ __global__ void __launch_bounds__(kThreads, 2) blockquery_kernel(const __grid_co
     const size_t orow = ((size_t)b * Hq + (size_t)g * G + hh) * Tq + act[a];
     p.o[orow * D + d] = __float2bfloat16_rn(M == -INFINITY ? 0.f : O / Lsum);
     if (d == 0) p.lse[orow] = M == -INFINITY ? -INFINITY : (M + log2f(Lsum)) * kLn2;
+  };
+  if (dsm) {
+    // slice of the outputs each CTA merges (even, so a pushed pair never straddles two)
+    const int chunk = ((E + CL - 1) / CL + 1) & ~1;
+    if (tid == 0) {
+      const int own = max(0, min(E, (rank + 1) * chunk) - rank * chunk);
+      tc::mbar_arrive_expect_tx(&xbar[3 + kStages], (uint32_t)(CL * (rows * 8 + own * 4)));
+    }
+    if (srow < rows)
+      for (int peer = ssub; peer < CL; peer += 8)
+        st_async(map_rank(pml + rank * kRowChunk + srow, peer), make_float2(m_run, l_run),
+                 map_rank(&xbar[3 + kStages], peer));
+#pragma unroll
+    for (int mt = 0; mt < 2; ++mt) {
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        const int d = (D == 128 ? 16 * warp : 8 * warp) + 8 * nt + 2 * (lane & 3);
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          const int r = 16 * mt + (lane >> 2) + 8 * half;
+          if (r < rows) {
+            const int e = r * D + d, owner = e / chunk;
+            st_async(map_rank(pacc + rank * chunk + (e - owner * chunk), owner),
+                     make_float2(acc[mt][nt][2 * half], acc[mt][nt][2 * half + 1]),
+                     map_rank(&xbar[3 + kStages], owner));
+          }
+        }
+      }
+    }
+    tc::mbar_wait(&xbar[3 + kStages], 0, &xabort, p.budget);
+    for (int e = rank * chunk + tid; e < min(E, (rank + 1) * chunk); e += kThreads) {
+      const int r = e / D;
+      float2 ml[kMaxCluster];
+      float ov[kMaxCluster];
+#pragma unroll
+      for (int c2 = 0; c2 < kMaxCluster; ++c2) {
+        ml[c2] = c2 < CL ? pml[c2 * kRowChunk + r] : make_float2(-INFINITY, 0.f);
+        ov[c2] = c2 < CL ? pacc[c2 * chunk + (e - rank * chunk)] : 0.f;
+      }
+      merge_out(e, ml, ov);
+    }
+  } else {
+    cluster_arrive_release();  // every partial is in the workspace ...
+    cluster_wait();            // ... for every CTA of the cluster
+    const int chunk = (E + CL - 1) >> cl_log2;
+    const float* wsg = p.ws + unit * kMaxCluster * (size_t)p.rows_max * (D + 2);
+    for (int e = rank * chunk + tid; e < min(E, (rank + 1) * chunk); e += kThreads) {
+      const int r = e / D, d = e - r * D;
+      // every partial's (m, l) and value first (independent loads, one round trip)
+      float2 ml[kMaxCluster];
+      float ov[kMaxCluster];
+#pragma unroll
+      for (int c2 = 0; c2 < kMaxCluster; ++c2) {
+        ml[c2] = make_float2(-INFINITY, 0.f);
+        ov[c2] = 0.f;
+        if (c2 < CL) {
+          const float* part = wsg + ((size_t)c2 * p.rows_max + r) * (D + 2);
+          ml[c2] = __ldcg(reinterpret_cast<const float2*>(part + D));
+          ov[c2] = __ldcg(part + d);
+        }
+      }
+      merge_out(e, ml, ov);
+    }
   }
 
   // ---- stable rows: the chunks loaded before the barrier, then any further ones -----------
@@ -708,6 +765,7 @@ __global__ void __launch_bounds__(kThreads, 2) blockquery_kernel(const __grid_co
     }
     for (int i = issued - kStages < 0 ? 0 : issued - kStages; i < issued; ++i)
       tc::mbar_drain(&xbar[3 + i % kStages], (uint32_t)((i / kStages) & 1), kDrainBudget);
+    if (dsm) tc::mbar_drain(&xbar[3 + kStages], 0, kDrainBudget);  // (the partials peers owe)
     g_blockquery_status = 1;
   }
 }
