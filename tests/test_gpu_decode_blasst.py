@@ -185,8 +185,11 @@ def test_decode_blasst_many_units_padded_selection(lsa):
             idx[b, h, :n] = torch.tensor(blocks, dtype=torch.int32)
             if n > 2:
                 idx[b, h, 1] = -1  # an unused slot inside the list
+    nsel[0, 0] = 0  # a unit with no block at all: o = 0, lse = -inf
+    idx[0, 0] = -1
     q = (case.q.float() * 4).to(torch.bfloat16)
     o, lse, bits = _gpu(lsa, q, case.k, case.v, case.seqlens, idx, nsel, 0.5)
+    assert float(o[0, :4].float().abs().max()) == 0.0 and bool(torch.isinf(lse[0, :4]).all())
     assert all(int(bits[b, h]) >> int(nsel[b, h]) == 0 for b in range(B) for h in range(Hkv))
     _check(q, case.k, case.v, case.seqlens, idx, nsel, 0.5, o, lse, bits, "padded, many units")
 
