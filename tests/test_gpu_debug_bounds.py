@@ -63,8 +63,13 @@ def _decode(lsa, lib, q, k, v, sl, summ, topk, idx=None, nsel=None):
 
 def test_release_build_reports_no_bounds_checks(libs):
     lsa, _ = libs
+    # (the release library by its path: with LSA_LIBRARY=debug the package itself loads the
+    # debug build)
+    rel = ctypes.CDLL(os.path.join(ROOT, "query_aware_block_b200", "liblsa.so"))
+    rel.lsa_debug_bounds_code.argtypes = [ctypes.POINTER(ctypes.c_int), ctypes.c_int]
+    rel.lsa_debug_bounds_code.restype = ctypes.c_int
     c = ctypes.c_int(7)
-    assert lsa.library().lsa_debug_bounds_code(ctypes.byref(c), 0) == lsa.LSA_ERR_UNSUPPORTED
+    assert rel.lsa_debug_bounds_code(ctypes.byref(c), 0) == lsa.LSA_ERR_UNSUPPORTED
     assert c.value == 0
 
 
