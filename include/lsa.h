@@ -17,6 +17,12 @@
  * The first step of a block passes topk_per_query >= ceil(T_prefix / blk) and an all-ones
  * mask (dense prefix attention, which fills the cache).
  *
+ * One decode step with the host on both ends (inputs in, outputs out through pinned host
+ * memory) is three calls on one stream, each a programmatic dependent of the one before:
+ *   lsa_copy_async              (q from pinned host memory to the device)
+ *   lsa_append_kv               (k_new, v_new read from pinned host memory into the cache)
+ *   lsa_sparse_attn_decode      (o, lse, idx_out written straight into pinned host memory)
+ *
  * One NSA decode step with fixed parts is three calls on one stream:
  *   lsa_sparse_attn_decode      (the selected branch, fused selection)
  *   lsa_nsa_compress            (nc_begin = -2: the compressed tokens the new token changes)
@@ -28,7 +34,9 @@
  * Conventions shared by every entry point
  * ---------------------------------------
  * Memory.   Every tensor argument is a raw DEVICE pointer to a contiguous row-major array
- *           in the stated layout, aligned to 16 bytes.  The caller owns all memory; the
+ *           in the stated layout, aligned to 16 bytes (except where a call states that
+ *           pinned host memory is accepted: lsa_copy_async, k_new / v_new of lsa_append_kv,
+ *           o / lse / idx_out of lsa_sparse_attn_decode).  The caller owns all memory; the
  *           library allocates nothing, keeps no per-call state and never frees.
  * Streams.  All work is enqueued on `stream` (a cudaStream_t; 0 = legacy default
  *           stream).  Calls return as soon as the work is enqueued; nothing synchronises
@@ -162,6 +170,7 @@ LSA_API int lsa_select_blocks(const void* q, int dtype, const float* summ, int B
  *       summ[b, g, NB_b - 1, :] as the mean of that block's valid keys, i.e. the summary
  *       update a decode step owes after appending a token, from the keys it loads anyway.
  * q [B, Hq, D]; k, v [B, Hkv, T_cap, D]; o [B, Hq, D] (dtype); lse [B, Hq] float32 or NULL.
+ * o, lse and idx_out may be pinned host memory (written with plain stores, over PCIe).
  * summ [B, Hkv, NB_cap, D] float32 (fused mode; written only by the refresh).
  * K/V rows at or beyond seqlens[b] are never used (they may hold any bits, NaN included).
  * refresh_last_summary must be 0 in given-selection mode.
@@ -187,7 +196,8 @@ LSA_API int lsa_sparse_attn_decode(const void* q, const void* k, const void* v, 
  *
  *   k[b, g, seqlens[b] - 1, :] = k_new[b, g, :]     v[b, g, seqlens[b] - 1, :] = v_new[b, g, :]
  * seqlens[b] already counts the new token; a sequence with seqlens[b] == 0 is left alone.
- * k_new, v_new [B, Hkv, D] (dtype); k, v [B, Hkv, T_cap, D] (dtype), written in place.
+ * k_new, v_new [B, Hkv, D] (dtype; device or pinned host memory, read with plain loads);
+ * k, v [B, Hkv, T_cap, D] (dtype), written in place.
  * flags: 0, or LSA_FLAG_PDL: launched as a programmatic dependent of the previous kernel of
  *     the stream; it reads k_new, v_new and seqlens only after that kernel completes, and
  *     lets the next kernel start at once (a decode call with LSA_FLAG_PDL then overlaps its
@@ -197,6 +207,22 @@ LSA_API int lsa_sparse_attn_decode(const void* q, const void* k, const void* v, 
 LSA_API int lsa_append_kv(const void* k_new, const void* v_new, int dtype, int B, int Hkv,
                           int T_cap, int D, const int32_t* seqlens, void* k, void* v, int flags,
                           cudaStream_t stream);
+
+/*
+ * lsa_copy_async -- copies `bytes` from src to dst with a kernel (16-byte loads and stores),
+ * enqueued on `stream`.  Either side may be pinned host memory (cudaHostAlloc / a pinned
+ * tensor: under unified addressing its pointer is valid in kernels, and the kernel's loads or
+ * stores cross PCIe), which moves a decode step's small inputs to the device without a
+ * copy-engine round trip.  The other library calls accept pinned host memory in the same
+ * way for k_new / v_new of lsa_append_kv and for the outputs o, lse and idx_out of
+ * lsa_sparse_attn_decode (plain loads and stores); every other pointer must be device memory.
+ * flags: 0, or LSA_FLAG_PDL: launched as a programmatic dependent of the previous kernel of
+ *     the stream; it touches src and dst only after that kernel completes, and lets the next
+ *     kernel start at once.
+ * Errors: LSA_ERR_INVALID_ARG for bytes not a multiple of 16, a pointer not 16-byte aligned,
+ * overlapping ranges, or unknown flags; bytes == 0 enqueues nothing.
+ */
+LSA_API int lsa_copy_async(void* dst, const void* src, size_t bytes, int flags, cudaStream_t stream);
 
 /*
  * lsa_sparse_attn_blockquery -- one denoising step of a block of Tq query tokens

@@ -34,7 +34,7 @@ EXPORTED = ("lsa_status_string", "lsa_last_cuda_error", "lsa_version", "lsa_buil
             "lsa_sparse_attn_blockquery", "lsa_sparse_attn_blockquery_noalloc",
             "lsa_blasst_prefill", "lsa_device_status", "lsa_losa_classify",
             "lsa_blockquery_intra_merge", "lsa_sparse_attn_decode_blasst", "lsa_nsa_compress",
-            "lsa_nsa_branches", "lsa_select_blocks_weighted", "lsa_append_kv",
+            "lsa_nsa_branches", "lsa_select_blocks_weighted", "lsa_append_kv", "lsa_copy_async",
             "lsa_debug_set_wait_budget", "lsa_debug_inject", "lsa_debug_bounds_code")
 
 _vp, _i, _f = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
@@ -53,6 +53,7 @@ _lib.lsa_debug_set_wait_budget.argtypes = [ctypes.c_longlong]
 _lib.lsa_debug_inject.argtypes = [_i]
 _lib.lsa_debug_bounds_code.argtypes = [_vp, _i]
 _lib.lsa_append_kv.argtypes = [_vp, _vp, _i, _i, _i, _i, _i, _vp, _vp, _vp, _i, _vp]
+_lib.lsa_copy_async.argtypes = [_vp, _vp, ctypes.c_size_t, _i, _vp]
 _lib.lsa_blockquery_workspace_size.argtypes = [_i, _i, _i, _i, _i]
 _lib.lsa_blockquery_workspace_size.restype = ctypes.c_size_t
 _lib.lsa_sparse_attn_blockquery.argtypes = [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _vp,
@@ -148,6 +149,14 @@ def lsa_append_kv(k_new, v_new, seqlens, k, v, flags=0, stream=None):
     _check(_lib.lsa_append_kv(_ptr(k_new), _ptr(v_new), _dtype(k), B, Hkv, T_cap, D, _ptr(seqlens),
                               _ptr(k), _ptr(v), flags, _stream(stream)), "lsa_append_kv")
     return k, v
+
+
+def lsa_copy_async(dst, src, flags=0, stream=None):
+    """dst <- src (same number of bytes) by a kernel; either may be a pinned host tensor."""
+    n = src.numel() * src.element_size()
+    assert dst.numel() * dst.element_size() == n, "lsa_copy_async: sizes differ"
+    _check(_lib.lsa_copy_async(_ptr(dst), _ptr(src), n, int(flags), _stream(stream)), "lsa_copy_async")
+    return dst
 
 
 def lsa_sparse_attn_decode(q, k, v, seqlens, o, topk, idx=None, nsel=None, summ=None,

@@ -1,4 +1,5 @@
-// kv_append.cu -- writes a decode step's new key and value rows into the KV cache.
+// kv_append.cu -- writes a decode step's new key and value rows into the KV cache; and a
+// plain kernel copy for a step's small inputs and outputs.
 //
 // A decode step appends the newest token's key and value at cache row seqlens[b] - 1 (the
 // sequence length already counts it) before attending: NSA news article, "NSA 구조" (the
@@ -38,7 +39,37 @@ __global__ void __launch_bounds__(kThreads)
   *dst = x;
 }
 
+// A copy by a kernel, 16 bytes per thread and iteration: either side may be pinned host
+// memory (every pinned allocation is mapped under unified addressing, and plain loads and
+// stores reach it over PCIe), so a decode step's small inputs and outputs need no copy-engine
+// round trip.  It lets the next kernel start at once and touches memory only after the
+// previous kernel of the stream has completed (programmatic dependent launch).
+__global__ void __launch_bounds__(kThreads) copy16_kernel(const uint4* __restrict__ src, uint4* __restrict__ dst,
+                                                          size_t n16) {
+  pdl_trigger();
+  pdl_wait();
+  for (size_t i = blockIdx.x * (size_t)kThreads + threadIdx.x; i < n16; i += (size_t)gridDim.x * kThreads)
+    dst[i] = src[i];
+}
+
 }  // namespace
+
+cudaError_t launch_copy16(void* dst, const void* src, size_t bytes, int pdl, cudaStream_t stream) {
+  const size_t n16 = bytes / 16;
+  size_t blocks = (n16 + kThreads - 1) / kThreads;
+  if (blocks > 1184) blocks = 1184;  // (8 per SM on 148 SMs; the loop strides over the rest)
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)blocks, 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, copy16_kernel, static_cast<const uint4*>(src), static_cast<uint4*>(dst), n16);
+}
 
 cudaError_t launch_kv_append(const void* k_new, const void* v_new, int elem_bytes, int B, int Hkv,
                              int T_cap, int D, const int32_t* seqlens, void* k, void* v, int pdl,

@@ -199,6 +199,16 @@ int lsa_append_kv(const void* k_new, const void* v_new, int dtype, int B, int Hk
                                            seqlens, k, v, (flags & LSA_FLAG_PDL) != 0, stream));
 }
 
+int lsa_copy_async(void* dst, const void* src, size_t bytes, int flags, cudaStream_t stream) {
+  if ((flags & ~LSA_FLAG_PDL) != 0 || bytes % 16 != 0) return LSA_ERR_INVALID_ARG;
+  if (bytes == 0) return LSA_OK;
+  if (!dst || !src || !aligned16(dst) || !aligned16(src)) return LSA_ERR_INVALID_ARG;
+  const char* s = static_cast<const char*>(src);
+  const char* d = static_cast<const char*>(dst);
+  if (s < d + bytes && d < s + bytes) return LSA_ERR_INVALID_ARG;  // overlapping ranges
+  return cuda_status(lsa::launch_copy16(dst, src, bytes, (flags & LSA_FLAG_PDL) != 0, stream));
+}
+
 int lsa_sparse_attn_decode_blasst(const void* q, const void* k, const void* v, int dtype, int B,
                                   int Hkv, int G, int D, int T_cap, const int32_t* seqlens,
                                   int blk, const int32_t* idx, const int32_t* nsel, int topk,

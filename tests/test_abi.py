@@ -227,6 +227,18 @@ def test_append_kv_validation():
 
 
 
+def test_copy_async_validation():
+    import query_aware_block_b200 as lsa
+    f = lsa.library().lsa_copy_async
+    a, b = ctypes.c_void_p(4096), ctypes.c_void_p(8192)
+    assert f(a, b, 0, 0, NULL) == lsa.LSA_OK  # nothing to copy: nothing enqueued
+    assert f(a, b, 24, 0, NULL) == lsa.LSA_ERR_INVALID_ARG  # not a multiple of 16 bytes
+    assert f(ctypes.c_void_p(4104), b, 32, 0, NULL) == lsa.LSA_ERR_INVALID_ARG  # misaligned
+    assert f(a, ctypes.c_void_p(4112), 32, 0, NULL) == lsa.LSA_ERR_INVALID_ARG  # overlapping
+    assert f(a, b, 32, 2, NULL) == lsa.LSA_ERR_INVALID_ARG  # unknown flag
+    assert f(NULL, b, 32, 0, NULL) == lsa.LSA_ERR_INVALID_ARG
+
+
 def test_debug_controls_validate_without_a_gpu():
     import query_aware_block_b200 as lsa
     lib = lsa.library()
