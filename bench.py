@@ -635,11 +635,10 @@ def needle_recall(case, idx):
 
 def run_e2e(args, lsa, copies, base, dev, topk, ns, nl, flags):
     """Same metric through the public API with pinned host buffers on both ends: every step
-    moves q from pinned host memory to the device (lsa_copy_async, a kernel whose loads cross
-    PCIe), appends the newest token's k and v read straight from pinned host memory
-    (lsa_append_kv), decodes (lsa_sparse_attn_decode, fused selection and summary refresh)
-    with o, lse and idx written straight into pinned host memory, each call a programmatic
-    dependent of the one before.  The steps of one rotation cycle are captured once in a
+    moves q to the device and appends the newest token's k and v, all three read straight
+    from pinned host memory by one kernel whose loads cross PCIe (lsa_append_kv_stage_q),
+    then decodes (lsa_sparse_attn_decode, fused selection and summary refresh, a programmatic
+    dependent of the staging) with o, lse and idx written straight into pinned host memory.  The steps of one rotation cycle are captured once in a
     CUDA graph and replayed, as a serving loop does; the same calls issued eagerly from
     Python are timed beside it."""
     R = len(copies)
@@ -671,8 +670,7 @@ def run_e2e(args, lsa, copies, base, dev, topk, ns, nl, flags):
     def one(i):
         c = copies[i % R]
         hq, hk, hv = in_views[i % R]
-        lsa.lsa_copy_async(q_dev, hq, flags=flags)
-        lsa.lsa_append_kv(hk, hv, c["sl"], c["k"], c["v"], flags=flags)
+        lsa.lsa_append_kv_stage_q(hq, q_dev, hk, hv, c["sl"], c["k"], c["v"], flags=flags)
         lsa.lsa_sparse_attn_decode(q_dev, c["k"], c["v"], c["sl"], o_host, topk, summ=c["summ"],
                                    n_sink=ns, n_local=nl, refresh_last_summary=True,
                                    idx_out=idx_host, lse=lse_host, flags=flags)
@@ -715,8 +713,8 @@ def run_e2e(args, lsa, copies, base, dev, topk, ns, nl, flags):
             "eager": {"value": round(B * n / (ms_eager / 1e3), 1), "us_per_step": round(ms_eager * 1e3 / n, 3),
                       "host_wall_s": round(wall_eager, 3)},
             "outputs_checked": ok,
-            "path": "python ctypes -> lsa_copy_async (q: pinned host -> device) + lsa_append_kv (k, v "
-                    "read from pinned host memory) + lsa_sparse_attn_decode (fused selection, summary "
+            "path": "python ctypes -> lsa_append_kv_stage_q (q, k, v read from pinned host memory by "
+                    "one kernel) + lsa_sparse_attn_decode (fused selection, summary "
                     "refresh; o, lse, idx written into pinned host memory), every byte crossing PCIe "
                     "each step; value: the steps of a rotation cycle captured once in a CUDA graph "
                     "and replayed; eager: the same calls issued from Python every step"}

@@ -18,9 +18,9 @@
  * mask (dense prefix attention, which fills the cache).
  *
  * One decode step with the host on both ends (inputs in, outputs out through pinned host
- * memory) is three calls on one stream, each a programmatic dependent of the one before:
- *   lsa_copy_async              (q from pinned host memory to the device)
- *   lsa_append_kv               (k_new, v_new read from pinned host memory into the cache)
+ * memory) is two calls on one stream, the second a programmatic dependent of the first:
+ *   lsa_append_kv_stage_q       (q to the device and k_new, v_new into the cache, all read
+ *                                from pinned host memory)
  *   lsa_sparse_attn_decode      (o, lse, idx_out written straight into pinned host memory)
  *
  * One NSA decode step with fixed parts is three calls on one stream:
@@ -35,8 +35,8 @@
  * ---------------------------------------
  * Memory.   Every tensor argument is a raw DEVICE pointer to a contiguous row-major array
  *           in the stated layout, aligned to 16 bytes (except where a call states that
- *           pinned host memory is accepted: lsa_copy_async, k_new / v_new of lsa_append_kv,
- *           o / lse / idx_out of lsa_sparse_attn_decode).  The caller owns all memory; the
+ *           pinned host memory is accepted: lsa_copy_async, q_src / q_dst / k_new / v_new
+ *           of lsa_append_kv(_stage_q), o / lse / idx_out of lsa_sparse_attn_decode).  The caller owns all memory; the
  *           library allocates nothing, keeps no per-call state and never frees.
  * Streams.  All work is enqueued on `stream` (a cudaStream_t; 0 = legacy default
  *           stream).  Calls return as soon as the work is enqueued; nothing synchronises
@@ -207,6 +207,19 @@ LSA_API int lsa_sparse_attn_decode(const void* q, const void* k, const void* v, 
 LSA_API int lsa_append_kv(const void* k_new, const void* v_new, int dtype, int B, int Hkv,
                           int T_cap, int D, const int32_t* seqlens, void* k, void* v, int flags,
                           cudaStream_t stream);
+
+/*
+ * lsa_append_kv_stage_q -- lsa_append_kv, and in the same launch the step's query rows:
+ * q_bytes (a multiple of 16) copied from q_src to q_dst with 16-byte loads and stores.  With
+ * q_src, k_new and v_new in pinned host memory, the inputs of a decode step reach the device
+ * in one launch, their PCIe round trips overlapping.  Arguments and flags as lsa_append_kv;
+ * q_src, q_dst 16-byte aligned and not overlapping (either may be pinned host memory);
+ * q_bytes == 0 appends only.  Support: q_bytes <= 2^28.
+ */
+LSA_API int lsa_append_kv_stage_q(const void* q_src, void* q_dst, size_t q_bytes, const void* k_new,
+                                  const void* v_new, int dtype, int B, int Hkv, int T_cap, int D,
+                                  const int32_t* seqlens, void* k, void* v, int flags,
+                                  cudaStream_t stream);
 
 /*
  * lsa_copy_async -- copies `bytes` from src to dst with a kernel (16-byte loads and stores),

@@ -34,7 +34,7 @@ EXPORTED = ("lsa_status_string", "lsa_last_cuda_error", "lsa_version", "lsa_buil
             "lsa_sparse_attn_blockquery", "lsa_sparse_attn_blockquery_noalloc",
             "lsa_blasst_prefill", "lsa_device_status", "lsa_losa_classify",
             "lsa_blockquery_intra_merge", "lsa_sparse_attn_decode_blasst", "lsa_nsa_compress",
-            "lsa_nsa_branches", "lsa_select_blocks_weighted", "lsa_append_kv", "lsa_copy_async",
+            "lsa_nsa_branches", "lsa_select_blocks_weighted", "lsa_append_kv", "lsa_append_kv_stage_q", "lsa_copy_async",
             "lsa_debug_set_wait_budget", "lsa_debug_inject", "lsa_debug_bounds_code")
 
 _vp, _i, _f = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
@@ -54,6 +54,8 @@ _lib.lsa_debug_inject.argtypes = [_i]
 _lib.lsa_debug_bounds_code.argtypes = [_vp, _i]
 _lib.lsa_append_kv.argtypes = [_vp, _vp, _i, _i, _i, _i, _i, _vp, _vp, _vp, _i, _vp]
 _lib.lsa_copy_async.argtypes = [_vp, _vp, ctypes.c_size_t, _i, _vp]
+_lib.lsa_append_kv_stage_q.argtypes = [_vp, _vp, ctypes.c_size_t, _vp, _vp, _i, _i, _i, _i, _i, _vp,
+                                       _vp, _vp, _i, _vp]
 _lib.lsa_blockquery_workspace_size.argtypes = [_i, _i, _i, _i, _i]
 _lib.lsa_blockquery_workspace_size.restype = ctypes.c_size_t
 _lib.lsa_sparse_attn_blockquery.argtypes = [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _vp,
@@ -148,6 +150,17 @@ def lsa_append_kv(k_new, v_new, seqlens, k, v, flags=0, stream=None):
     B, Hkv, T_cap, D = k.shape
     _check(_lib.lsa_append_kv(_ptr(k_new), _ptr(v_new), _dtype(k), B, Hkv, T_cap, D, _ptr(seqlens),
                               _ptr(k), _ptr(v), flags, _stream(stream)), "lsa_append_kv")
+    return k, v
+
+
+def lsa_append_kv_stage_q(q_src, q_dst, k_new, v_new, seqlens, k, v, flags=0, stream=None):
+    """lsa_append_kv and q_dst <- q_src in one launch; q_src, k_new, v_new may be pinned host."""
+    B, Hkv, T_cap, D = k.shape
+    n = q_src.numel() * q_src.element_size()
+    assert q_dst.numel() * q_dst.element_size() == n, "lsa_append_kv_stage_q: q sizes differ"
+    _check(_lib.lsa_append_kv_stage_q(_ptr(q_src), _ptr(q_dst), n, _ptr(k_new), _ptr(v_new), _dtype(k), B,
+                                      Hkv, T_cap, D, _ptr(seqlens), _ptr(k), _ptr(v), int(flags),
+                                      _stream(stream)), "lsa_append_kv_stage_q")
     return k, v
 
 

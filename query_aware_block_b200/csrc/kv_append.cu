@@ -18,15 +18,21 @@ namespace {
 
 constexpr int kThreads = 128;
 
-// chunk c of the nb = B * Hkv * rows16 16-byte chunks of k_new (then of v_new): unit
-// u = c / rows16 = b * Hkv + g, column part c % rows16
+// chunks [0, nq): the step's query rows, q_dst[c] = q_src[c]; then chunk c of the
+// n = B * Hkv * rows16 16-byte chunks of k_new (then of v_new): unit u = c / rows16 =
+// b * Hkv + g, column part c % rows16
 __global__ void __launch_bounds__(kThreads)
     kv_append_kernel(const uint4* __restrict__ k_new, const uint4* __restrict__ v_new, int Hkv, int T_cap,
                      int rows16, int n, const int32_t* __restrict__ seqlens, uint4* __restrict__ k,
-                     uint4* __restrict__ v) {
+                     uint4* __restrict__ v, const uint4* __restrict__ q_src, uint4* __restrict__ q_dst, int nq) {
   pdl_trigger();  // the next kernel may start its prologue now ...
   pdl_wait();     // ... while this one waits for the kernel that produced k_new / v_new
-  const int c = blockIdx.x * kThreads + threadIdx.x;
+  int c = blockIdx.x * kThreads + threadIdx.x;
+  if (c < nq) {
+    q_dst[c] = q_src[c];
+    return;
+  }
+  c -= nq;
   if (c >= 2 * n) return;
   const bool is_v = c >= n;
   const int cc = is_v ? c - n : c;
@@ -73,11 +79,12 @@ cudaError_t launch_copy16(void* dst, const void* src, size_t bytes, int pdl, cud
 
 cudaError_t launch_kv_append(const void* k_new, const void* v_new, int elem_bytes, int B, int Hkv,
                              int T_cap, int D, const int32_t* seqlens, void* k, void* v, int pdl,
-                             cudaStream_t stream) {
+                             cudaStream_t stream, const void* q_src, void* q_dst, size_t q_bytes) {
   const int rows16 = D * elem_bytes / 16;
   const int n = B * Hkv * rows16;
+  const int nq = (int)(q_bytes / 16);
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((2 * n + kThreads - 1) / kThreads, 1, 1);
+  cfg.gridDim = dim3((nq + 2 * n + kThreads - 1) / kThreads, 1, 1);
   cfg.blockDim = dim3(kThreads, 1, 1);
   cfg.dynamicSmemBytes = 0;
   cfg.stream = stream;
@@ -88,7 +95,8 @@ cudaError_t launch_kv_append(const void* k_new, const void* v_new, int elem_byte
   cfg.numAttrs = pdl ? 1 : 0;
   return cudaLaunchKernelEx(&cfg, kv_append_kernel, static_cast<const uint4*>(k_new),
                             static_cast<const uint4*>(v_new), Hkv, T_cap, rows16, n, seqlens,
-                            static_cast<uint4*>(k), static_cast<uint4*>(v));
+                            static_cast<uint4*>(k), static_cast<uint4*>(v), static_cast<const uint4*>(q_src),
+                            static_cast<uint4*>(q_dst), nq);
 }
 
 LSA_BOUNDS_READER(kv_append)

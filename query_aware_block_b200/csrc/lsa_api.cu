@@ -199,6 +199,31 @@ int lsa_append_kv(const void* k_new, const void* v_new, int dtype, int B, int Hk
                                            seqlens, k, v, (flags & LSA_FLAG_PDL) != 0, stream));
 }
 
+int lsa_append_kv_stage_q(const void* q_src, void* q_dst, size_t q_bytes, const void* k_new,
+                          const void* v_new, int dtype, int B, int Hkv, int T_cap, int D,
+                          const int32_t* seqlens, void* k, void* v, int flags, cudaStream_t stream) {
+  int st = check_common(dtype, B, Hkv, 1, D, 64);
+  if (st != LSA_OK) return st;
+  if (T_cap < 0 || (flags & ~LSA_FLAG_PDL) != 0 || q_bytes % 16 != 0) return LSA_ERR_INVALID_ARG;
+  if (T_cap > kMaxTcap || (long long)B * Hkv * D > (1 << 24) || q_bytes > ((size_t)1 << 28))
+    return LSA_ERR_UNSUPPORTED;
+  if (q_bytes > 0) {
+    if (!q_src || !q_dst || !aligned16(q_src) || !aligned16(q_dst)) return LSA_ERR_INVALID_ARG;
+    const char* s = static_cast<const char*>(q_src);
+    const char* d = static_cast<const char*>(q_dst);
+    if (s < d + q_bytes && d < s + q_bytes) return LSA_ERR_INVALID_ARG;  // overlapping ranges
+  }
+  const bool kv = B > 0 && Hkv > 0 && T_cap > 0;
+  if (kv) {
+    if (!k_new || !v_new || !seqlens || !k || !v) return LSA_ERR_INVALID_ARG;
+    if (!aligned16(k_new) || !aligned16(v_new) || !aligned16(k) || !aligned16(v)) return LSA_ERR_INVALID_ARG;
+  }
+  if (!kv && q_bytes == 0) return LSA_OK;
+  return cuda_status(lsa::launch_kv_append(k_new, v_new, dtype == LSA_BF16 ? 2 : 4, kv ? B : 0, Hkv, T_cap, D,
+                                           seqlens, k, v, (flags & LSA_FLAG_PDL) != 0, stream, q_src, q_dst,
+                                           q_bytes));
+}
+
 int lsa_copy_async(void* dst, const void* src, size_t bytes, int flags, cudaStream_t stream) {
   if ((flags & ~LSA_FLAG_PDL) != 0 || bytes % 16 != 0) return LSA_ERR_INVALID_ARG;
   if (bytes == 0) return LSA_OK;

@@ -239,6 +239,23 @@ def test_copy_async_validation():
     assert f(NULL, b, 32, 0, NULL) == lsa.LSA_ERR_INVALID_ARG
 
 
+def test_append_kv_stage_q_validation():
+    import query_aware_block_b200 as lsa
+    f = lsa.library().lsa_append_kv_stage_q
+    g = ctypes.c_void_p(4096)
+    args = lambda **kw: [kw.get(n, d) for n, d in (
+        ("qs", ctypes.c_void_p(1 << 20)), ("qd", ctypes.c_void_p(2 << 20)), ("qb", 4096), ("kn", g),
+        ("vn", g), ("dtype", 1), ("B", 1), ("Hkv", 8), ("T", 65536), ("D", 128), ("sl", g), ("k", g),
+        ("v", g), ("flags", 0), ("stream", NULL))]
+    assert f(*args(qb=24)) == lsa.LSA_ERR_INVALID_ARG           # not a multiple of 16 bytes
+    assert f(*args(qs=NULL)) == lsa.LSA_ERR_INVALID_ARG
+    assert f(*args(qd=ctypes.c_void_p((1 << 20) + 16))) == lsa.LSA_ERR_INVALID_ARG  # overlapping
+    assert f(*args(kn=NULL)) == lsa.LSA_ERR_INVALID_ARG
+    assert f(*args(flags=2)) == lsa.LSA_ERR_INVALID_ARG
+    assert f(*args(D=96)) == lsa.LSA_ERR_UNSUPPORTED
+    assert f(*args(qb=0, B=0, kn=NULL, vn=NULL, k=NULL, v=NULL, sl=NULL)) == lsa.LSA_OK
+
+
 def test_debug_controls_validate_without_a_gpu():
     import query_aware_block_b200 as lsa
     lib = lsa.library()

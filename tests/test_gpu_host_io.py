@@ -1,7 +1,7 @@
 """A decode step with the host on both ends: lsa_copy_async (a kernel copy; either side may be
-pinned host memory), lsa_append_kv reading k_new / v_new from pinned host memory, and
-lsa_sparse_attn_decode writing o, lse and idx_out straight into pinned host memory.  Every
-result must equal, bit for bit, the same calls on device buffers."""
+pinned host memory), lsa_append_kv / lsa_append_kv_stage_q reading q, k_new and v_new from
+pinned host memory, and lsa_sparse_attn_decode writing o, lse and idx_out straight into pinned
+host memory.  Every result must equal, bit for bit, the same calls on device buffers."""
 import pytest
 import torch
 
@@ -43,7 +43,7 @@ def test_decode_step_with_host_inputs_and_outputs(lsa):
     k_new = torch.stack([case.k[b, :, last[b]] for b in range(B)]) * 0.5  # a new token's k, v
     v_new = torch.stack([case.v[b, :, last[b]] for b in range(B)]) * 0.5
 
-    def run(host):
+    def run(host, staged=False):
         k, v = case.k.to(DEV), case.v.to(DEV)
         summ = torch.zeros(B, Hkv, T_cap // 64, D, device=DEV)
         lsa.lsa_build_summaries(k, sl, summ)
@@ -53,14 +53,18 @@ def test_decode_step_with_host_inputs_and_outputs(lsa):
             o = torch.full((B, Hq, D), 7.0, dtype=torch.bfloat16).pin_memory()
             lse = torch.full((B, Hq), 7.0).pin_memory()
             idx = torch.full((B, Hkv, 8), 99, dtype=torch.int32).pin_memory()
-            lsa.lsa_copy_async(q_d, q_h, flags=lsa.LSA_FLAG_PDL)
+            if not staged:
+                lsa.lsa_copy_async(q_d, q_h, flags=lsa.LSA_FLAG_PDL)
         else:
             kn, vn = k_new.to(DEV), v_new.to(DEV)
             o = torch.full((B, Hq, D), 7.0, dtype=torch.bfloat16, device=DEV)
             lse = torch.full((B, Hq), 7.0, device=DEV)
             idx = torch.full((B, Hkv, 8), 99, dtype=torch.int32, device=DEV)
             q_d.copy_(case.q.to(DEV))
-        lsa.lsa_append_kv(kn, vn, sl, k, v, flags=lsa.LSA_FLAG_PDL)
+        if staged:  # q, k_new, v_new in one launch
+            lsa.lsa_append_kv_stage_q(q_h, q_d, kn, vn, sl, k, v, flags=lsa.LSA_FLAG_PDL)
+        else:
+            lsa.lsa_append_kv(kn, vn, sl, k, v, flags=lsa.LSA_FLAG_PDL)
         lsa.lsa_sparse_attn_decode(q_d, k, v, sl, o, 8, summ=summ, n_sink=1, n_local=2,
                                    refresh_last_summary=True, idx_out=idx, lse=lse,
                                    flags=lsa.LSA_FLAG_PDL)
@@ -68,10 +72,22 @@ def test_decode_step_with_host_inputs_and_outputs(lsa):
         assert lsa.lsa_device_status() == 0
         return o.cpu(), lse.cpu(), idx.cpu(), k.cpu(), v.cpu(), summ.cpu()
 
-    dev_r, host_r = run(False), run(True)
-    for a, b in zip(dev_r, host_r):
+    dev_r, host_r, staged_r = run(False), run(True), run(True, staged=True)
+    for a, b, c in zip(dev_r, host_r, staged_r):
         assert torch.equal(a, b)
+        assert torch.equal(a, c)
     # the appended rows are the new token's
     for b in range(B):
         assert torch.equal(host_r[3][b, :, last[b]], k_new[b])
         assert torch.equal(host_r[4][b, :, last[b]], v_new[b])
+
+
+def test_stage_q_alone_copies_the_query(lsa):
+    src = torch.arange(4096, dtype=torch.float32).pin_memory()
+    dst = torch.zeros(4096, device=DEV)
+    # B = 0: nothing appended, only the query rows copied
+    st = lsa.library().lsa_append_kv_stage_q(src.data_ptr(), dst.data_ptr(), 4096 * 4, None, None,
+                                             lsa.LSA_BF16, 0, 1, 64, 128, None, None, None, 0, None)
+    assert st == lsa.LSA_OK
+    torch.cuda.synchronize()
+    assert torch.equal(dst.cpu(), src)
