@@ -188,15 +188,8 @@ int lsa_sparse_attn_decode(const void* q, const void* k, const void* v, int dtyp
 
 int lsa_append_kv(const void* k_new, const void* v_new, int dtype, int B, int Hkv, int T_cap,
                   int D, const int32_t* seqlens, void* k, void* v, int flags, cudaStream_t stream) {
-  int st = check_common(dtype, B, Hkv, 1, D, 64);
-  if (st != LSA_OK) return st;
-  if (T_cap < 0 || (flags & ~LSA_FLAG_PDL) != 0) return LSA_ERR_INVALID_ARG;
-  if (T_cap > kMaxTcap || (long long)B * Hkv * D > (1 << 24)) return LSA_ERR_UNSUPPORTED;
-  if (B == 0 || Hkv == 0 || T_cap == 0) return LSA_OK;
-  if (!k_new || !v_new || !seqlens || !k || !v) return LSA_ERR_INVALID_ARG;
-  if (!aligned16(k_new) || !aligned16(v_new) || !aligned16(k) || !aligned16(v)) return LSA_ERR_INVALID_ARG;
-  return cuda_status(lsa::launch_kv_append(k_new, v_new, dtype == LSA_BF16 ? 2 : 4, B, Hkv, T_cap, D,
-                                           seqlens, k, v, (flags & LSA_FLAG_PDL) != 0, stream));
+  return lsa_append_kv_stage_q(nullptr, nullptr, 0, k_new, v_new, dtype, B, Hkv, T_cap, D, seqlens, k, v,
+                               flags, stream);
 }
 
 int lsa_append_kv_stage_q(const void* q_src, void* q_dst, size_t q_bytes, const void* k_new,
