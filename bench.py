@@ -670,7 +670,9 @@ def run_e2e(args, lsa, copies, base, dev, topk, ns, nl, flags):
     def one(i):
         c = copies[i % R]
         hq, hk, hv = in_views[i % R]
-        lsa.lsa_append_kv_stage_q(hq, q_dev, hk, hv, c["sl"], c["k"], c["v"], flags=flags)
+        # (the host wrote this step's inputs before enqueueing it: they are read at once)
+        lsa.lsa_append_kv_stage_q(hq, q_dev, hk, hv, c["sl"], c["k"], c["v"],
+                                  flags=flags | (lsa.LSA_FLAG_INPUTS_READY if flags else 0))
         lsa.lsa_sparse_attn_decode(q_dev, c["k"], c["v"], c["sl"], o_host, topk, summ=c["summ"],
                                    n_sink=ns, n_local=nl, refresh_last_summary=True,
                                    idx_out=idx_host, lse=lse_host, flags=flags)

@@ -36,8 +36,9 @@
  * Memory.   Every tensor argument is a raw DEVICE pointer to a contiguous row-major array
  *           in the stated layout, aligned to 16 bytes (except where a call states that
  *           pinned host memory is accepted: lsa_copy_async, q_src / q_dst / k_new / v_new
- *           of lsa_append_kv(_stage_q), o / lse / idx_out of lsa_sparse_attn_decode).  The caller owns all memory; the
- *           library allocates nothing, keeps no per-call state and never frees.
+ *           of lsa_append_kv and lsa_append_kv_stage_q, o / lse / idx_out of
+ *           lsa_sparse_attn_decode).  The caller owns all memory; the library allocates
+ *           nothing, keeps no per-call state and never frees.
  * Streams.  All work is enqueued on `stream` (a cudaStream_t; 0 = legacy default
  *           stream).  Calls return as soon as the work is enqueued; nothing synchronises
  *           the host.  Calls are thread-safe.
@@ -86,8 +87,14 @@ extern "C" {
 #define LSA_F32 0
 #define LSA_BF16 1
 
-/* lsa_sparse_attn_decode / lsa_blockquery_intra_merge flags */
+/* lsa_sparse_attn_decode / lsa_blockquery_intra_merge / lsa_append_kv / lsa_append_kv_stage_q /
+ * lsa_copy_async flags */
 #define LSA_FLAG_PDL 1
+/* lsa_append_kv / lsa_append_kv_stage_q / lsa_copy_async, with LSA_FLAG_PDL: the call's
+ * inputs (q_src, k_new, v_new, seqlens; src) are complete when the call is enqueued (written
+ * by the host, say), so they are read at once; only the writes wait for the previous
+ * kernel. */
+#define LSA_FLAG_INPUTS_READY 2
 
 /* Human-readable name of a status code (static storage). */
 LSA_API const char* lsa_status_string(int status);
@@ -202,6 +209,8 @@ LSA_API int lsa_sparse_attn_decode(const void* q, const void* k, const void* v, 
  *     the stream; it reads k_new, v_new and seqlens only after that kernel completes, and
  *     lets the next kernel start at once (a decode call with LSA_FLAG_PDL then overlaps its
  *     prologue with this copy; it reads the newest block only after this call completes).
+ *     LSA_FLAG_PDL | LSA_FLAG_INPUTS_READY: the inputs are read at once (they do not depend
+ *     on the previous kernel), and only the writes into the cache wait for it.
  * Support: D in {64, 128}; B * Hkv * D <= 2^24.
  */
 LSA_API int lsa_append_kv(const void* k_new, const void* v_new, int dtype, int B, int Hkv,
@@ -231,7 +240,8 @@ LSA_API int lsa_append_kv_stage_q(const void* q_src, void* q_dst, size_t q_bytes
  * lsa_sparse_attn_decode (plain loads and stores); every other pointer must be device memory.
  * flags: 0, or LSA_FLAG_PDL: launched as a programmatic dependent of the previous kernel of
  *     the stream; it touches src and dst only after that kernel completes, and lets the next
- *     kernel start at once.
+ *     kernel start at once; with LSA_FLAG_INPUTS_READY as well, src is read at once and only
+ *     the writes wait.
  * Errors: LSA_ERR_INVALID_ARG for bytes not a multiple of 16, a pointer not 16-byte aligned,
  * overlapping ranges, or unknown flags; bytes == 0 enqueues nothing.
  */

@@ -26,6 +26,7 @@ _lib = ctypes.CDLL(LIB_PATH)
 LSA_OK, LSA_ERR_INVALID_ARG, LSA_ERR_UNSUPPORTED, LSA_ERR_CUDA, LSA_ERR_DEVICE_STATUS = 0, 1, 2, 3, 4
 LSA_F32, LSA_BF16 = 0, 1
 LSA_FLAG_PDL = 1
+LSA_FLAG_INPUTS_READY = 2
 LSA_DEBUG_PREFILL_DROP_S = 1
 BLK = 64
 

@@ -24,12 +24,17 @@ constexpr int kThreads = 128;
 __global__ void __launch_bounds__(kThreads)
     kv_append_kernel(const uint4* __restrict__ k_new, const uint4* __restrict__ v_new, int Hkv, int T_cap,
                      int rows16, int n, const int32_t* __restrict__ seqlens, uint4* __restrict__ k,
-                     uint4* __restrict__ v, const uint4* __restrict__ q_src, uint4* __restrict__ q_dst, int nq) {
+                     uint4* __restrict__ v, const uint4* __restrict__ q_src, uint4* __restrict__ q_dst, int nq,
+                     int inputs_ready) {
   pdl_trigger();  // the next kernel may start its prologue now ...
-  pdl_wait();     // ... while this one waits for the kernel that produced k_new / v_new
+  // ... while this one waits for the kernel that produced its inputs (or, when they are
+  // ready at enqueue, reads them first and waits only before writing)
+  if (!inputs_ready) pdl_wait();
   int c = blockIdx.x * kThreads + threadIdx.x;
   if (c < nq) {
-    q_dst[c] = q_src[c];
+    const uint4 x = q_src[c];
+    if (inputs_ready) pdl_wait();
+    q_dst[c] = x;
     return;
   }
   c -= nq;
@@ -42,6 +47,7 @@ __global__ void __launch_bounds__(kThreads)
   if (t < 0 || t >= T_cap) return;  // an empty sequence has no newest token
   const uint4 x = is_v ? v_new[cc] : k_new[cc];
   uint4* dst = (is_v ? v : k) + ((size_t)u * T_cap + t) * rows16 + part;
+  if (inputs_ready) pdl_wait();
   *dst = x;
 }
 
@@ -51,16 +57,24 @@ __global__ void __launch_bounds__(kThreads)
 // round trip.  It lets the next kernel start at once and touches memory only after the
 // previous kernel of the stream has completed (programmatic dependent launch).
 __global__ void __launch_bounds__(kThreads) copy16_kernel(const uint4* __restrict__ src, uint4* __restrict__ dst,
-                                                          size_t n16) {
+                                                          size_t n16, int inputs_ready) {
   pdl_trigger();
-  pdl_wait();
-  for (size_t i = blockIdx.x * (size_t)kThreads + threadIdx.x; i < n16; i += (size_t)gridDim.x * kThreads)
-    dst[i] = src[i];
+  if (!inputs_ready) pdl_wait();
+  const size_t i0 = blockIdx.x * (size_t)kThreads + threadIdx.x, step = (size_t)gridDim.x * kThreads;
+  if (inputs_ready && i0 < n16) {  // the first chunk read before the wait
+    const uint4 x = src[i0];
+    pdl_wait();
+    dst[i0] = x;
+    for (size_t i = i0 + step; i < n16; i += step) dst[i] = src[i];
+  } else {
+    for (size_t i = i0; i < n16; i += step) dst[i] = src[i];
+  }
 }
 
 }  // namespace
 
-cudaError_t launch_copy16(void* dst, const void* src, size_t bytes, int pdl, cudaStream_t stream) {
+cudaError_t launch_copy16(void* dst, const void* src, size_t bytes, int pdl, cudaStream_t stream,
+                          int inputs_ready) {
   const size_t n16 = bytes / 16;
   size_t blocks = (n16 + kThreads - 1) / kThreads;
   if (blocks > 1184) blocks = 1184;  // (8 per SM on 148 SMs; the loop strides over the rest)
@@ -74,12 +88,14 @@ cudaError_t launch_copy16(void* dst, const void* src, size_t bytes, int pdl, cud
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = pdl ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, copy16_kernel, static_cast<const uint4*>(src), static_cast<uint4*>(dst), n16);
+  return cudaLaunchKernelEx(&cfg, copy16_kernel, static_cast<const uint4*>(src), static_cast<uint4*>(dst), n16,
+                            pdl && inputs_ready ? 1 : 0);
 }
 
 cudaError_t launch_kv_append(const void* k_new, const void* v_new, int elem_bytes, int B, int Hkv,
                              int T_cap, int D, const int32_t* seqlens, void* k, void* v, int pdl,
-                             cudaStream_t stream, const void* q_src, void* q_dst, size_t q_bytes) {
+                             cudaStream_t stream, const void* q_src, void* q_dst, size_t q_bytes,
+                             int inputs_ready) {
   const int rows16 = D * elem_bytes / 16;
   const int n = B * Hkv * rows16;
   const int nq = (int)(q_bytes / 16);
@@ -96,7 +112,7 @@ cudaError_t launch_kv_append(const void* k_new, const void* v_new, int elem_byte
   return cudaLaunchKernelEx(&cfg, kv_append_kernel, static_cast<const uint4*>(k_new),
                             static_cast<const uint4*>(v_new), Hkv, T_cap, rows16, n, seqlens,
                             static_cast<uint4*>(k), static_cast<uint4*>(v), static_cast<const uint4*>(q_src),
-                            static_cast<uint4*>(q_dst), nq);
+                            static_cast<uint4*>(q_dst), nq, pdl && inputs_ready ? 1 : 0);
 }
 
 LSA_BOUNDS_READER(kv_append)

@@ -197,7 +197,8 @@ int lsa_append_kv_stage_q(const void* q_src, void* q_dst, size_t q_bytes, const 
                           const int32_t* seqlens, void* k, void* v, int flags, cudaStream_t stream) {
   int st = check_common(dtype, B, Hkv, 1, D, 64);
   if (st != LSA_OK) return st;
-  if (T_cap < 0 || (flags & ~LSA_FLAG_PDL) != 0 || q_bytes % 16 != 0) return LSA_ERR_INVALID_ARG;
+  if (T_cap < 0 || (flags & ~(LSA_FLAG_PDL | LSA_FLAG_INPUTS_READY)) != 0 || q_bytes % 16 != 0)
+    return LSA_ERR_INVALID_ARG;
   if (T_cap > kMaxTcap || (long long)B * Hkv * D > (1 << 24) || q_bytes > ((size_t)1 << 28))
     return LSA_ERR_UNSUPPORTED;
   if (q_bytes > 0) {
@@ -214,17 +215,18 @@ int lsa_append_kv_stage_q(const void* q_src, void* q_dst, size_t q_bytes, const 
   if (!kv && q_bytes == 0) return LSA_OK;
   return cuda_status(lsa::launch_kv_append(k_new, v_new, dtype == LSA_BF16 ? 2 : 4, kv ? B : 0, Hkv, T_cap, D,
                                            seqlens, k, v, (flags & LSA_FLAG_PDL) != 0, stream, q_src, q_dst,
-                                           q_bytes));
+                                           q_bytes, (flags & LSA_FLAG_INPUTS_READY) != 0));
 }
 
 int lsa_copy_async(void* dst, const void* src, size_t bytes, int flags, cudaStream_t stream) {
-  if ((flags & ~LSA_FLAG_PDL) != 0 || bytes % 16 != 0) return LSA_ERR_INVALID_ARG;
+  if ((flags & ~(LSA_FLAG_PDL | LSA_FLAG_INPUTS_READY)) != 0 || bytes % 16 != 0) return LSA_ERR_INVALID_ARG;
   if (bytes == 0) return LSA_OK;
   if (!dst || !src || !aligned16(dst) || !aligned16(src)) return LSA_ERR_INVALID_ARG;
   const char* s = static_cast<const char*>(src);
   const char* d = static_cast<const char*>(dst);
   if (s < d + bytes && d < s + bytes) return LSA_ERR_INVALID_ARG;  // overlapping ranges
-  return cuda_status(lsa::launch_copy16(dst, src, bytes, (flags & LSA_FLAG_PDL) != 0, stream));
+  return cuda_status(lsa::launch_copy16(dst, src, bytes, (flags & LSA_FLAG_PDL) != 0, stream,
+                                        (flags & LSA_FLAG_INPUTS_READY) != 0));
 }
 
 int lsa_sparse_attn_decode_blasst(const void* q, const void* k, const void* v, int dtype, int B,

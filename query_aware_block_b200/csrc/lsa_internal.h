@@ -151,11 +151,13 @@ bool kv_tensor_maps(const void* k, const void* v, int D, int T_cap, int planes, 
                     CUtensorMap* mv);
 
 // The new token's key and value rows into the cache at row seqlens[b] - 1.
-cudaError_t launch_copy16(void* dst, const void* src, size_t bytes, int pdl, cudaStream_t stream);
+cudaError_t launch_copy16(void* dst, const void* src, size_t bytes, int pdl, cudaStream_t stream,
+                          int inputs_ready = 0);
 cudaError_t launch_kv_append(const void* k_new, const void* v_new, int elem_bytes, int B, int Hkv,
                              int T_cap, int D, const int32_t* seqlens, void* k, void* v, int pdl,
                              cudaStream_t stream,
-                             const void* q_src = nullptr, void* q_dst = nullptr, size_t q_bytes = 0);
+                             const void* q_src = nullptr, void* q_dst = nullptr, size_t q_bytes = 0,
+                             int inputs_ready = 0);
 
 // The debug bounds-check status word of each translation unit (always 0 in the release
 // build, which compiles no checks).

@@ -219,7 +219,7 @@ def test_append_kv_validation():
         ("sl", g), ("k", g), ("v", g), ("flags", 0), ("stream", NULL))]
     assert f(*args(kn=NULL)) == lsa.LSA_ERR_INVALID_ARG
     assert f(*args(v=ctypes.c_void_p(4104))) == lsa.LSA_ERR_INVALID_ARG
-    assert f(*args(flags=2)) == lsa.LSA_ERR_INVALID_ARG
+    assert f(*args(flags=4)) == lsa.LSA_ERR_INVALID_ARG  # unknown flag
     assert f(*args(T=-1)) == lsa.LSA_ERR_INVALID_ARG
     assert f(*args(D=96)) == lsa.LSA_ERR_UNSUPPORTED
     assert f(*args(dtype=5)) == lsa.LSA_ERR_UNSUPPORTED
@@ -235,7 +235,7 @@ def test_copy_async_validation():
     assert f(a, b, 24, 0, NULL) == lsa.LSA_ERR_INVALID_ARG  # not a multiple of 16 bytes
     assert f(ctypes.c_void_p(4104), b, 32, 0, NULL) == lsa.LSA_ERR_INVALID_ARG  # misaligned
     assert f(a, ctypes.c_void_p(4112), 32, 0, NULL) == lsa.LSA_ERR_INVALID_ARG  # overlapping
-    assert f(a, b, 32, 2, NULL) == lsa.LSA_ERR_INVALID_ARG  # unknown flag
+    assert f(a, b, 32, 4, NULL) == lsa.LSA_ERR_INVALID_ARG  # unknown flag
     assert f(NULL, b, 32, 0, NULL) == lsa.LSA_ERR_INVALID_ARG
 
 
@@ -251,7 +251,7 @@ def test_append_kv_stage_q_validation():
     assert f(*args(qs=NULL)) == lsa.LSA_ERR_INVALID_ARG
     assert f(*args(qd=ctypes.c_void_p((1 << 20) + 16))) == lsa.LSA_ERR_INVALID_ARG  # overlapping
     assert f(*args(kn=NULL)) == lsa.LSA_ERR_INVALID_ARG
-    assert f(*args(flags=2)) == lsa.LSA_ERR_INVALID_ARG
+    assert f(*args(flags=4)) == lsa.LSA_ERR_INVALID_ARG  # unknown flag
     assert f(*args(D=96)) == lsa.LSA_ERR_UNSUPPORTED
     assert f(*args(qb=0, B=0, kn=NULL, vn=NULL, k=NULL, v=NULL, sl=NULL)) == lsa.LSA_OK
 

@@ -43,7 +43,7 @@ def test_decode_step_with_host_inputs_and_outputs(lsa):
     k_new = torch.stack([case.k[b, :, last[b]] for b in range(B)]) * 0.5  # a new token's k, v
     v_new = torch.stack([case.v[b, :, last[b]] for b in range(B)]) * 0.5
 
-    def run(host, staged=False):
+    def run(host, staged=False, ready=False):
         k, v = case.k.to(DEV), case.v.to(DEV)
         summ = torch.zeros(B, Hkv, T_cap // 64, D, device=DEV)
         lsa.lsa_build_summaries(k, sl, summ)
@@ -61,8 +61,9 @@ def test_decode_step_with_host_inputs_and_outputs(lsa):
             lse = torch.full((B, Hq), 7.0, device=DEV)
             idx = torch.full((B, Hkv, 8), 99, dtype=torch.int32, device=DEV)
             q_d.copy_(case.q.to(DEV))
-        if staged:  # q, k_new, v_new in one launch
-            lsa.lsa_append_kv_stage_q(q_h, q_d, kn, vn, sl, k, v, flags=lsa.LSA_FLAG_PDL)
+        if staged:  # q, k_new, v_new in one launch (read before the wait when ready)
+            f = lsa.LSA_FLAG_PDL | (lsa.LSA_FLAG_INPUTS_READY if ready else 0)
+            lsa.lsa_append_kv_stage_q(q_h, q_d, kn, vn, sl, k, v, flags=f)
         else:
             lsa.lsa_append_kv(kn, vn, sl, k, v, flags=lsa.LSA_FLAG_PDL)
         lsa.lsa_sparse_attn_decode(q_d, k, v, sl, o, 8, summ=summ, n_sink=1, n_local=2,
@@ -72,10 +73,11 @@ def test_decode_step_with_host_inputs_and_outputs(lsa):
         assert lsa.lsa_device_status() == 0
         return o.cpu(), lse.cpu(), idx.cpu(), k.cpu(), v.cpu(), summ.cpu()
 
-    dev_r, host_r, staged_r = run(False), run(True), run(True, staged=True)
-    for a, b, c in zip(dev_r, host_r, staged_r):
-        assert torch.equal(a, b)
-        assert torch.equal(a, c)
+    dev_r = run(False)
+    host_r = run(True)
+    for other in (host_r, run(True, staged=True), run(True, staged=True, ready=True)):
+        for a, b in zip(dev_r, other):
+            assert torch.equal(a, b)
     # the appended rows are the new token's
     for b in range(B):
         assert torch.equal(host_r[3][b, :, last[b]], k_new[b])
