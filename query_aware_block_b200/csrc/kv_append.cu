@@ -8,7 +8,10 @@
 // kernel of the stream start at once (programmatic dependent launch): a decode step launched
 // with LSA_FLAG_PDL overlaps its prologue with this copy and waits for it before it reads
 // the newest block.  Launched itself with LSA_FLAG_PDL, it reads k_new / v_new only after
-// the previous kernel of the stream (the one that produced them) has completed.
+// the previous kernel of the stream (the one that produced them) has completed -- unless
+// LSA_FLAG_INPUTS_READY says they were complete when the call was enqueued (written by the
+// host): then it reads them at once, over PCIe when they are in pinned host memory, and waits
+// only before writing.  The same launch may also copy the step's query rows.
 #include "cluster.cuh"
 #include "lsa_common.cuh"
 #include "lsa_internal.h"
@@ -55,7 +58,8 @@ __global__ void __launch_bounds__(kThreads)
 // memory (every pinned allocation is mapped under unified addressing, and plain loads and
 // stores reach it over PCIe), so a decode step's small inputs and outputs need no copy-engine
 // round trip.  It lets the next kernel start at once and touches memory only after the
-// previous kernel of the stream has completed (programmatic dependent launch).
+// previous kernel of the stream has completed (programmatic dependent launch), or, with
+// inputs ready at enqueue, reads its first chunk at once and waits only before writing.
 __global__ void __launch_bounds__(kThreads) copy16_kernel(const uint4* __restrict__ src, uint4* __restrict__ dst,
                                                           size_t n16, int inputs_ready) {
   pdl_trigger();
