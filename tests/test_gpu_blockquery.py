@@ -117,6 +117,7 @@ def _check_outputs(case, o, lse, ui, uc, where, alias=False):
     dict(B=1, Hkv=2, G=4, D=128, Tq=16, T_prefix=64 * 60, n_active=16, topk=8, n_sink=1, n_local=2),
     dict(B=1, Hkv=2, G=4, D=128, Tq=16, T_prefix=64 * 5 + 3, n_active=5, topk=8),  # NBp <= topk
     dict(B=1, Hkv=2, G=4, D=128, Tq=16, T_prefix=64 * 50, n_active=0, topk=8),    # nothing active
+    dict(B=1, Hkv=2, G=4, D=128, Tq=16, T_prefix=64 * 50, n_active=9, topk=8),    # 36 rows: just past one chunk
     dict(B=4, Hkv=8, G=2, D=128, Tq=16, T_prefix=64 * 64, n_active=4, topk=8),    # 32 units: 8-CTA clusters
     dict(B=1, Hkv=2, G=4, D=128, Tq=64, T_prefix=64 * 40, n_active=64, topk=4),   # all 64 tokens active
     # 1,100 blocks: a CTA's slice (69 rows) exceeds the 64 staged rows (the rest from global)
