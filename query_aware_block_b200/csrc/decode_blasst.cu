@@ -371,27 +371,29 @@ __global__ void __launch_bounds__(kThreads) decode_blasst_kernel(const __grid_co
   }
 }
 
-// ---- many (b, g) units: one CTA per unit in three parallel phases -------------------------
+// ---- many (b, g) units: one CTA per unit, the test taken in two halves --------------------
 // The sequential rule needs, for each selected block, only the maximum of the earlier
-// blocks' maxima (a skipped block never raises it), so nothing has to run block by block:
-//   1. S = Q K^T of every selected block, warp w taking slots w and w + 8 on its own TMA
-//      stage (the next K requested as soon as the warp has read the first), the logits kept
-//      in shared memory and each block's per-head maximum;
-//   2. every slot's test at once (a thread per (slot, head): the exclusive prefix maximum
-//      over the earlier slots, then the maximum over the heads);
-//   3. the kept blocks' V, warp w taking kept blocks w and w + 8 on its own stage again, each
-//      warp an online softmax of its own (P from the logits in registers, straight into the
-//      mma A operand);
+// blocks' maxima (a skipped block never raises it), so nothing has to run block by block,
+// and the first eight slots can be decided before the last eight are scored:
+//   1. warp w computes S of slot w on its own TMA stage, keeps the logits in registers and
+//      posts the block's per-head maxima, then requests slot w + 8's K into the same stage;
+//   2. slots 0..7 are tested (a thread per (slot, head): the exclusive prefix maximum over
+//      the earlier slots, then the maximum over the heads) and the V of up to four kept
+//      ones starts at once into four extra stages, while warp w computes S of slot w + 8;
+//   3. slots 8..15 are tested; each warp then loads the V of its kept slots that have no
+//      stage yet into its own stage (free again) and folds its kept slots into an online
+//      softmax of its own, P built from the logits in registers straight into the mma A
+//      operand;
 //   4. the eight warps' (m, l, O) merged by log-sum-exp.
 // One CTA per unit (128 CTAs for 16 sequences x 8 KV heads: one wave, one per SM), no
-// cluster, no cross-CTA exchange; the V loads of all kept blocks are in flight together.
+// cluster, no cross-CTA exchange.
 template <int D>
 struct UnitLay {
   static constexpr int kTile = kBlk * D * 2;                 // one K or V block (bf16)
-  static constexpr int kSSt = kBlk + 4;                      // fp32 row stride of the logits
+  static constexpr int kXS = 4;                              // extra V stages
   static constexpr int kRing = 0;                            // kWarps stages, 1024-byte aligned
-  static constexpr int kS = kRing + kWarps * kTile;          // [16 slots][16 rows][kSSt] fp32
-  static constexpr int kQ = kS + kCL * kRows * kSSt * 4;     // [16][D] bf16, chunk-swizzled
+  static constexpr int kX = kRing + kWarps * kTile;          // kXS extra V stages
+  static constexpr int kQ = kX + kXS * kTile;                // [16][D] bf16, chunk-swizzled
   static constexpr int kRmax = kQ + kRows * D * 2;           // [16 slots][16 heads] fp32
   static constexpr int kTotal = kRmax + kCL * kRows * 4;
   static_assert(kWarps * kRows * D * 4 <= kWarps * kTile, "the warps' partials fit the ring");
@@ -402,16 +404,16 @@ __global__ void __launch_bounds__(kThreads, 1) decode_blasst_unit_kernel(const _
   using L = UnitLay<D>;
   constexpr int kRowBytes = D * 2;
   constexpr int NO = D / 8;  // n8 tiles of a warp's output (all D columns)
+  constexpr int NS = kBlk / 8;  // n8 tiles of a block's logits
   extern __shared__ __align__(1024) unsigned char smem[];
-  __shared__ __align__(8) uint64_t kbar[kWarps], vbar[kWarps];
+  __shared__ __align__(8) uint64_t kbar[kWarps], vbar[kWarps], xbar[L::kXS];
   __shared__ int slot_block[kCL], slot_id[kCL], nslots;
-  __shared__ int kept_slot[kCL], nkept;
-  __shared__ int skipf[kCL];
+  __shared__ int skipf[kCL], xstage[kCL];
   __shared__ float2 ml_w[kWarps][kRows];
   __shared__ int xabort;
   unsigned char* base = smem + ((1024u - (tc::smem_u32(smem) & 1023u)) & 1023u);
   unsigned char* ring = base + L::kRing;
-  float* Sbuf = reinterpret_cast<float*>(base + L::kS);
+  unsigned char* xring = base + L::kX;
   unsigned char* Qs = base + L::kQ;
   float* rmax = reinterpret_cast<float*>(base + L::kRmax);
 
@@ -427,6 +429,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_blasst_unit_kernel(const _
       tc::mbar_init(&kbar[i], 1);
       tc::mbar_init(&vbar[i], 1);
     }
+    for (int i = 0; i < L::kXS; ++i) tc::mbar_init(&xbar[i], 1);
     xabort = 0;
     tc::fence_mbar_init();
     tc::prefetch_tmap(&p.tmk);
@@ -445,6 +448,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_blasst_unit_kernel(const _
       slot_id[pos] = lane;
     }
     if (lane == 0) nslots = __popc(bits);
+    if (lane < kCL) {
+      skipf[lane] = 0;
+      xstage[lane] = -1;
+    }
   }
   {
     const __nv_bfloat16* qg = p.q + ((size_t)b * Hq + (size_t)g * G) * D;
@@ -458,25 +465,25 @@ __global__ void __launch_bounds__(kThreads, 1) decode_blasst_unit_kernel(const _
   __syncthreads();  // (the slot list and the barriers are set up)
   const int n = nslots;
   unsigned char* stage = ring + warp * L::kTile;  // this warp's TMA stage
-  // lane 0 of the warp: block j of `map` into this warp's stage, completing on `bar`
-  auto load_block = [&](const CUtensorMap* map, int j, uint64_t* bar) {
+  // lane 0 of the warp: block j of `map` into `dst`, completing on `bar`
+  auto load_block = [&](const CUtensorMap* map, int j, unsigned char* dst, uint64_t* bar) {
     tc::fence_proxy_async();  // this warp's earlier reads of the stage come first
     tc::mbar_arrive_expect_tx(bar, (uint32_t)L::kTile);
 #pragma unroll
-    for (int h = 0; h < D / 64; ++h) tc::tma_load_3d(stage + h * 8192, map, h * 64, j * kBlk, unit, bar);
+    for (int h = 0; h < D / 64; ++h) tc::tma_load_3d(dst + h * 8192, map, h * 64, j * kBlk, unit, bar);
   };
-  // loads issued on this warp's barriers and waited for: a load is issued only after the
-  // previous one on the same barrier was seen complete, so at most one is ever in flight
-  int k_issued = 0, k_seen = 0, v_issued = 0, v_seen = 0;
-  // lane 0 of the warp: block j of `map` pulled into L2 for a later load
   auto prefetch_block = [&](const CUtensorMap* map, int j) {
 #pragma unroll
     for (int h = 0; h < D / 64; ++h) tc::tma_prefetch_l2_3d(map, h * 64, j * kBlk, unit);
   };
+  // loads issued on this warp's barriers and seen complete: a load into a stage is issued
+  // only after the previous one on the same barrier was seen complete, so at most one is in
+  // flight per barrier
+  int k_issued = 0, k_seen = 0, v_issued = 0, v_seen = 0, x_issued = 0, x_seen = 0, my_x = -1;
   if (lane == 0 && warp < n) {
-    load_block(&p.tmk, slot_block[warp], &kbar[warp]);
+    load_block(&p.tmk, slot_block[warp], stage, &kbar[warp]);
     k_issued = 1;
-    // the second round's K waits for this stage: bring it into L2 meanwhile
+    // the second slot's K waits for this stage: bring it into L2 meanwhile
     if (warp + kWarps < n) prefetch_block(&p.tmk, slot_block[warp + kWarps]);
   }
   cp_async_wait<0>();
@@ -489,17 +496,13 @@ __global__ void __launch_bounds__(kThreads, 1) decode_blasst_unit_kernel(const _
   }
   const int r0 = lane >> 2, q2 = 2 * (lane & 3);
 
-  // ---- 1. logits and block maxima of every slot ---------------------------------------------
-  for (int round = 0; round < 2; ++round) {
-    const int i = warp + kWarps * round;
-    if (i >= n) break;
-    const bool ok = __all_sync(0xffffffffu, tc::mbar_wait(&kbar[warp], (uint32_t)round, &xabort, p.budget));
-    k_seen += ok ? 1 : 0;
+  // logits of slot i (base 2, -inf where masked) from the stage into registers, and the
+  // block's per-head maxima into rmax[i][*]
+  auto logits = [&](int i, bool ok, float (&S)[NS][4]) {
     const int nv = max(0, min(kBlk, T - slot_block[i] * kBlk));
-    float* Si = Sbuf + i * kRows * L::kSSt;
     float mlo = -INFINITY, mhi = -INFINITY;
 #pragma unroll
-    for (int nt = 0; nt < kBlk / 8; ++nt) {
+    for (int nt = 0; nt < NS; ++nt) {
       float c4[4] = {0.f, 0.f, 0.f, 0.f};
       if (ok) {
 #pragma unroll
@@ -512,14 +515,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_blasst_unit_kernel(const _
       }
       const int col = 8 * nt + q2;
       const bool v0 = col < nv, v1 = col + 1 < nv;
-      const float s0 = v0 && r0 < G ? c4[0] * p.scale2 : -INFINITY;
-      const float s1 = v1 && r0 < G ? c4[1] * p.scale2 : -INFINITY;
-      const float s2 = v0 && r0 + 8 < G ? c4[2] * p.scale2 : -INFINITY;
-      const float s3 = v1 && r0 + 8 < G ? c4[3] * p.scale2 : -INFINITY;
-      *reinterpret_cast<float2*>(Si + r0 * L::kSSt + col) = make_float2(s0, s1);
-      *reinterpret_cast<float2*>(Si + (r0 + 8) * L::kSSt + col) = make_float2(s2, s3);
-      mlo = fmaxf(mlo, fmaxf(s0, s1));
-      mhi = fmaxf(mhi, fmaxf(s2, s3));
+      S[nt][0] = v0 && r0 < G ? c4[0] * p.scale2 : -INFINITY;
+      S[nt][1] = v1 && r0 < G ? c4[1] * p.scale2 : -INFINITY;
+      S[nt][2] = v0 && r0 + 8 < G ? c4[2] * p.scale2 : -INFINITY;
+      S[nt][3] = v1 && r0 + 8 < G ? c4[3] * p.scale2 : -INFINITY;
+      mlo = fmaxf(mlo, fmaxf(S[nt][0], S[nt][1]));
+      mhi = fmaxf(mhi, fmaxf(S[nt][2], S[nt][3]));
     }
 #pragma unroll
     for (int o2 = 1; o2 < 4; o2 <<= 1) {
@@ -530,20 +531,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_blasst_unit_kernel(const _
       rmax[i * kRows + r0] = mlo;
       rmax[i * kRows + r0 + 8] = mhi;
     }
-    __syncwarp();  // (every lane has read the stage)
-    if (!ok) break;
-    if (lane == 0 && round == 0 && i + kWarps < n) {
-      load_block(&p.tmk, slot_block[i + kWarps], &kbar[warp]);
-      k_issued = 2;
-    }
-  }
-  __syncthreads();
-
-  // ---- 2. the test of every slot: a thread per (slot, head) ---------------------------------
-  {
+  };
+  // the test of slots [lo, hi): a thread per (slot, head); skipf[slot] = skipped
+  auto test_slots = [&](int lo, int hi) {
     const int sl = tid >> 4, h = tid & 15;  // (kThreads = 16 slots x 16 heads)
     float gi = -INFINITY;
-    if (sl < n && h < G) {
+    if (sl >= lo && sl < hi && sl < n && h < G) {
       const float r = rmax[sl * kRows + h];
       float m = -INFINITY;  // the maximum over the earlier slots = the running maximum
       for (int e = 0; e < sl; ++e) m = fmaxf(m, rmax[e * kRows + h]);
@@ -551,51 +544,73 @@ __global__ void __launch_bounds__(kThreads, 1) decode_blasst_unit_kernel(const _
     }
 #pragma unroll
     for (int o2 = 8; o2 > 0; o2 >>= 1) gi = fmaxf(gi, __shfl_xor_sync(0xffffffffu, gi, o2));
-    if (h == 0 && sl < kCL) skipf[sl] = sl > 0 && sl < n && gi < p.log2_lambda;
+    if (h == 0 && sl >= lo && sl < hi) skipf[sl] = sl > 0 && sl < n && gi < p.log2_lambda;
+  };
+
+  // ---- 1. slot w's logits; slot w + 8's K requested into the same stage ----------------------
+  float S0[NS][4], S1[NS][4];
+  bool ok0 = false, ok1 = false;
+  if (warp < n) {
+    ok0 = __all_sync(0xffffffffu, tc::mbar_wait(&kbar[warp], 0, &xabort, p.budget));
+    k_seen += ok0 ? 1 : 0;
+    logits(warp, ok0, S0);
+    __syncwarp();  // (every lane has read the stage)
+    if (ok0 && lane == 0 && warp + kWarps < n) {
+      load_block(&p.tmk, slot_block[warp + kWarps], stage, &kbar[warp]);
+      k_issued = 2;
+    }
   }
   __syncthreads();
-  if (warp == 0) {  // the kept slots in order, and the skip bits by selection slot
-    const bool in = lane < n;
-    const bool keep = in && !skipf[lane];
+  // ---- 2. slots 0..7 decided; up to kXS of the kept ones get an extra stage, V at once -------
+  test_slots(0, kWarps);
+  __syncthreads();
+  if (warp == 0) {
+    const bool keep = lane < kWarps && lane < n && !skipf[lane];
     const uint32_t kb2 = __ballot_sync(0xffffffffu, keep);
-    const uint32_t sb = __ballot_sync(0xffffffffu, in && skipf[lane]);
-    if (keep) kept_slot[__popc(kb2 & ((1u << lane) - 1u))] = lane;
-    if (lane == 0) nkept = __popc(kb2);
+    const int rank = __popc(kb2 & ((1u << lane) - 1u));
+    if (keep && rank < L::kXS) xstage[lane] = rank;
+  }
+  __syncthreads();
+  if (warp < n && !skipf[warp] && xstage[warp] >= 0) {
+    my_x = xstage[warp];
+    if (lane == 0 && *reinterpret_cast<volatile int*>(&xabort) == 0) {
+      load_block(&p.tmv, slot_block[warp], xring + my_x * L::kTile, &xbar[my_x]);
+      x_issued = 1;
+    }
+  }
+  if (warp + kWarps < n) {
+    ok1 = __all_sync(0xffffffffu, tc::mbar_wait(&kbar[warp], 1, &xabort, p.budget));
+    k_seen += ok1 ? 1 : 0;
+    logits(warp + kWarps, ok1, S1);
+  }
+  __syncthreads();
+  // ---- 3. slots 8..15 decided; each warp folds in its kept slots ---------------------------
+  test_slots(kWarps, kCL);
+  __syncthreads();
+  if (warp == 0) {  // the skip bits by selection slot
+    const uint32_t sb = __ballot_sync(0xffffffffu, lane < n && skipf[lane & (kCL - 1)]);
     uint32_t bits = 0u;
-    for (int e = 0; e < 32; ++e)
+    for (int e = 0; e < kCL; ++e)
       if ((sb >> e) & 1u) bits |= 1u << slot_id[e];
     if (lane == 0 && p.skip_bits) p.skip_bits[unit] = bits;
   }
-  __syncthreads();
-  const int nk = nkept;
-
-  // ---- 3. the kept blocks: V, then P V in each warp's own online softmax --------------------
-  if (lane == 0 && warp < nk && *reinterpret_cast<volatile int*>(&xabort) == 0) {
-    load_block(&p.tmv, slot_block[kept_slot[warp]], &vbar[warp]);
-    v_issued = 1;
-    if (warp + kWarps < nk) prefetch_block(&p.tmv, slot_block[kept_slot[warp + kWarps]]);
-  }
+  const bool keep0 = warp < n && !skipf[warp];
+  const bool keep1 = warp + kWarps < n && !skipf[warp + kWarps];
   float acc[NO][4];
 #pragma unroll
   for (int nt = 0; nt < NO; ++nt)
 #pragma unroll
     for (int e = 0; e < 4; ++e) acc[nt][e] = 0.f;
   float m_lo = -INFINITY, m_hi = -INFINITY, l_lo = 0.f, l_hi = 0.f;
-  for (int round = 0; round < 2; ++round) {
-    const int k = warp + kWarps * round;
-    if (k >= nk) break;
-    const int i = kept_slot[k];
-    const bool ok = __all_sync(0xffffffffu, tc::mbar_wait(&vbar[warp], (uint32_t)round, &xabort, p.budget));
-    v_seen += ok ? 1 : 0;
-    if (!ok) break;
+  // one kept slot folded in: O = alpha O + P V, P from the logits S, V at `vs`
+  auto fold = [&](int i, const float (&S)[NS][4], const unsigned char* vs, bool ok) {
     const int nv = max(0, min(kBlk, T - slot_block[i] * kBlk));
     // V rows past the sequence hold whatever the cache holds there: zero them (P is 0 there)
     for (int id = lane; id < (kBlk - nv) * (D / 8); id += 32) {
       const int r = nv + id / (D / 8), c = id % (D / 8);
-      *reinterpret_cast<uint4*>(stage + kv_off(r, c)) = make_uint4(0u, 0u, 0u, 0u);
+      *reinterpret_cast<uint4*>(const_cast<unsigned char*>(vs) + kv_off(r, c)) = make_uint4(0u, 0u, 0u, 0u);
     }
     __syncwarp();
-    const float* Si = Sbuf + i * kRows * L::kSSt;
     const float rlo = rmax[i * kRows + r0], rhi = rmax[i * kRows + r0 + 8];
     const float nlo = fmaxf(m_lo, rlo), nhi = fmaxf(m_hi, rhi);
     const float alo = m_lo == -INFINITY ? 0.f : ex2(m_lo - nlo);
@@ -610,17 +625,14 @@ __global__ void __launch_bounds__(kThreads, 1) decode_blasst_unit_kernel(const _
     float slo = 0.f, shi = 0.f;
 #pragma unroll
     for (int kk = 0; kk < kBlk / 16; ++kk) {
-      // P of keys 16 kk .. 16 kk + 15 as the mma A operand, from the logits (rows r0, r0 + 8)
       uint32_t pa[4];
 #pragma unroll
       for (int hf = 0; hf < 2; ++hf) {
-        const int col = 16 * kk + 8 * hf + q2;
-        const float2 xl = *reinterpret_cast<const float2*>(Si + r0 * L::kSSt + col);
-        const float2 xh = *reinterpret_cast<const float2*>(Si + (r0 + 8) * L::kSSt + col);
-        const float p0 = xl.x == -INFINITY ? 0.f : ex2(xl.x - nlo);
-        const float p1 = xl.y == -INFINITY ? 0.f : ex2(xl.y - nlo);
-        const float p2 = xh.x == -INFINITY ? 0.f : ex2(xh.x - nhi);
-        const float p3 = xh.y == -INFINITY ? 0.f : ex2(xh.y - nhi);
+        const float* x = S[2 * kk + hf];
+        const float p0 = x[0] == -INFINITY ? 0.f : ex2(x[0] - nlo);
+        const float p1 = x[1] == -INFINITY ? 0.f : ex2(x[1] - nlo);
+        const float p2 = x[2] == -INFINITY ? 0.f : ex2(x[2] - nhi);
+        const float p3 = x[3] == -INFINITY ? 0.f : ex2(x[3] - nhi);
         slo += p0 + p1;
         shi += p2 + p3;
         pa[2 * hf] = pack_bf16x2(p0, p1);
@@ -631,7 +643,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_blasst_unit_kernel(const _
 #pragma unroll
         for (int np = 0; np < D / 16; ++np) {
           uint32_t vb[4];
-          ldsm_x4_t(vb, stage + kv_off(vrow, 2 * np + (lane >> 4)));
+          ldsm_x4_t(vb, vs + kv_off(vrow, 2 * np + (lane >> 4)));
           mma_bf16(acc[2 * np], pa, vb[0], vb[1]);
           mma_bf16(acc[2 * np + 1], pa, vb[2], vb[3]);
         }
@@ -644,11 +656,46 @@ __global__ void __launch_bounds__(kThreads, 1) decode_blasst_unit_kernel(const _
     }
     l_lo = l_lo * alo + slo;
     l_hi = l_hi * ahi + shi;
-    __syncwarp();  // (every lane has read the stage)
-    if (lane == 0 && round == 0 && k + kWarps < nk) {
-      load_block(&p.tmv, slot_block[kept_slot[k + kWarps]], &vbar[warp]);
-      v_issued = 2;
+  };
+  // the stage's V loads: slot w's when it has no extra stage, then slot w + 8's
+  const bool w_in_stage = keep0 && my_x < 0;
+  if (lane == 0 && *reinterpret_cast<volatile int*>(&xabort) == 0) {
+    if (w_in_stage) {
+      load_block(&p.tmv, slot_block[warp], stage, &vbar[warp]);
+      v_issued = 1;
+    } else if (keep1) {
+      load_block(&p.tmv, slot_block[warp + kWarps], stage, &vbar[warp]);
+      v_issued = 1;
     }
+  }
+  v_issued = __shfl_sync(0xffffffffu, v_issued, 0);
+  if (keep0) {
+    bool ok;
+    const unsigned char* vs;
+    if (my_x >= 0) {
+      ok = __all_sync(0xffffffffu, tc::mbar_wait(&xbar[my_x], 0, &xabort, p.budget));
+      x_seen += ok ? 1 : 0;
+      vs = xring + my_x * L::kTile;
+    } else {
+      ok = __all_sync(0xffffffffu, tc::mbar_wait(&vbar[warp], 0, &xabort, p.budget));
+      v_seen += ok ? 1 : 0;
+      vs = stage;
+    }
+    fold(warp, S0, vs, ok && ok0);
+  }
+  if (keep1) {
+    if (w_in_stage) {  // the stage held slot w's V: slot w + 8's now
+      __syncwarp();  // (every lane has read the stage)
+      if (lane == 0 && v_seen == 1 && *reinterpret_cast<volatile int*>(&xabort) == 0) {
+        load_block(&p.tmv, slot_block[warp + kWarps], stage, &vbar[warp]);
+        v_issued = 2;
+      }
+      v_issued = __shfl_sync(0xffffffffu, v_issued, 0);
+    }
+    const int ph = v_issued - 1;
+    bool ok = ph >= 0 && __all_sync(0xffffffffu, tc::mbar_wait(&vbar[warp], (uint32_t)(ph & 1), &xabort, p.budget));
+    v_seen += ok ? 1 : 0;
+    fold(warp + kWarps, S1, stage, ok && ok1);
   }
   __syncthreads();  // (every stage has been read: the ring holds the partials now)
 
@@ -690,6 +737,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_blasst_unit_kernel(const _
     if (lane == 0) {
       if (k_issued > k_seen) tc::mbar_drain(&kbar[warp], (uint32_t)((k_issued - 1) & 1), kDrainBudget);
       if (v_issued > v_seen) tc::mbar_drain(&vbar[warp], (uint32_t)((v_issued - 1) & 1), kDrainBudget);
+      if (x_issued > x_seen) tc::mbar_drain(&xbar[my_x], 0, kDrainBudget);
     }
     if (tid == 0) g_blasst_decode_status = 1;
   }
