@@ -19,13 +19,17 @@
 //     maximum of the list heads, m rounds): its selected blocks go into a bitmap of the
 //     union, so every CTA holds the same union U(b, g) and attends entries rank, rank + CL,
 //     ... of its ascending list (balanced over the cluster).
-//   * Attention rows (active token x head) are processed 32 at a time (two mma m-tiles):
-//     K/V blocks arrive as TMA boxes (128-byte swizzle) on a 2-stage ring with per-stage
-//     mbarriers, S = Q K^T and O += P V on mma.sync m16n8k16 bf16, online softmax in base 2.
-//   * Each CTA writes its per-row partial (acc, m, l) to the caller's workspace; after a
-//     cluster barrier every CTA merges a 1/CL slice of the outputs by log-sum-exp (all
-//     loads issued before use).  Stable rows are copied from the cache; rank 0 writes the
-//     union list.
+//   * Attention rows (active token x head) are processed 32 at a time: K/V blocks arrive
+//     as TMA boxes (128-byte swizzle) on a 2-stage ring with per-stage mbarriers; warp w
+//     owns 16 rows and a quarter (16 keys) of every block, computes S = Q K^T and
+//     O += P V on mma.sync m16n8k16 bf16 with the logits kept in registers (online softmax
+//     in base 2), and the last warp done with a stage refills it.  The four key quarters
+//     are merged by log-sum-exp once per row chunk, through the ring.
+//   * When the rows fit one chunk, each CTA pushes its per-row partial (acc, m, l) into the
+//     shared memory of the CTA that merges that slice of the outputs (st.async on the
+//     owner's mbarrier) and the owners merge by log-sum-exp; more rows go through the
+//     caller's workspace and one cluster barrier (all loads of a merge issued before use).
+//     Stable rows are copied from the cache; rank 0 writes the union list.
 //   Every mbarrier wait is bounded (about 2 s); after a timeout the CTA waits (bounded) for
 //   its copies and its peers' list bytes still in flight before it exits, and a device status
 //   word records the failure.
@@ -56,11 +60,13 @@ constexpr int kLP = 16;         // length of an exchanged list (topk_per_query <
 constexpr int kMaxCluster = 16;
 constexpr int kMaxTq = 64;
 constexpr int kStages = 2;
-constexpr int kSStride = 68;    // fp32 row stride of the score tile
 constexpr int kQStride = 132;   // fp32 row stride of the summed queries (bank spread)
 constexpr int kStageRows = 64;  // summary rows of a CTA's slice staged by one bulk copy
 constexpr int kMaxUnion = kMaxTq * kLP;  // a union holds at most Tq * topk blocks
 static_assert(kTokChunk == 8, "the scoring maps lane l to token l & 7");
+static_assert(kThreads == 256 && kRowChunk == 32, "attention: 8 warps = 2 row tiles x 4 key quarters");
+// the key quarters' partials of a row chunk (fp32) are merged in the K/V ring
+static_assert(kStages * 2 * kBlk * 2 >= (kWarps / 2) * kRowChunk * 4, "merge buffer exceeds the ring");
 
 struct alignas(64) BQParams {
   // K and V as [B * Hkv][T_cap][D], box {64, 64, 1}, 128-byte swizzle
@@ -89,10 +95,18 @@ struct alignas(64) BQParams {
   long long budget;  // clock-cycle limit of every bounded wait
 };
 
+// st.async of four floats into a peer CTA's shared memory, counted on its mbarrier
+__device__ __forceinline__ void st_async4(uint32_t addr, float4 v, uint32_t mbar) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.f32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(
+                   addr),
+               "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w), "r"(mbar)
+               : "memory");
+}
+
 __host__ __device__ inline size_t al128(size_t x) { return (x + 127) & ~(size_t)127; }
 
 struct BQLayout {
-  size_t act, stab, ulist, ubits, qs, ss, ps, alpha, pml, pacc, region, total;
+  size_t act, stab, ulist, ubits, qs, pml, pacc, region, total;
   // selection buffers, inside `region` (dead once the attention starts)
   size_t qsum, keys, top, recv, sumbuf, qrows;
   size_t kv_tile;
@@ -112,13 +126,10 @@ __host__ __device__ inline BQLayout bq_layout(int D, int per_max, int NBp, int G
   L.ulist = off;  off = al128(off + (size_t)(ucap > 0 ? ucap : 1) * 4);
   L.ubits = off;  off = al128(off + (size_t)((NBp + 31) / 32 + 1) * 4);
   L.qs = off;     off = al128(off + (size_t)kRowChunk * D * 2);
-  L.ss = off;     off = al128(off + (size_t)kRowChunk * kSStride * 4);
-  L.ps = off;     off = al128(off + (size_t)kRowChunk * kBlk * 2);
-  L.alpha = off;  off = al128(off + kRowChunk * 4);
   // the partials pushed by the cluster's CTAs when the rows fit one chunk: every CTA's
   // (m, l) of every row and its part of this CTA's slice of the outputs
   L.pml = off;    off = al128(off + (size_t)kMaxCluster * kRowChunk * 8);
-  L.pacc = off;   off = al128(off + (size_t)kRowChunk * D * 4 + kMaxCluster * 8);
+  L.pacc = off;   off = al128(off + (size_t)kRowChunk * D * 4 + kMaxCluster * 16);
   L.region = off;
   L.kv_tile = (size_t)kBlk * D * 2;
   // the K/V ring starts at the first 1024-byte boundary of the region (TMA 128-byte swizzle)
@@ -150,9 +161,6 @@ __global__ void __launch_bounds__(kThreads, 2) blockquery_kernel(const __grid_co
   int* ulist = reinterpret_cast<int*>(smem + Lo.ulist);
   uint32_t* ubits = reinterpret_cast<uint32_t*>(smem + Lo.ubits);
   unsigned char* Qs = smem + Lo.qs;
-  float* Ss = reinterpret_cast<float*>(smem + Lo.ss);
-  unsigned char* Ps = smem + Lo.ps;
-  float* alpha_s = reinterpret_cast<float*>(smem + Lo.alpha);
   float2* pml = reinterpret_cast<float2*>(smem + Lo.pml);
   float* pacc = reinterpret_cast<float*>(smem + Lo.pacc);
   unsigned char* region = smem + Lo.region;
@@ -428,39 +436,54 @@ __global__ void __launch_bounds__(kThreads, 2) blockquery_kernel(const __grid_co
   const int n_my = U > rank ? (U - rank + CL - 1) >> cl_log2 : 0;
 
   // ---- attention: rows (active token x head) in chunks of 32, my union blocks -----------
+  // Warp w owns rows 16 (w & 1) .. + 15 of the chunk and keys 16 (w >> 1) .. + 15 of every
+  // block: its logits stay in registers and become the A operand of P V directly, so a block
+  // costs no block-wide barrier.  The four key quarters of a row are merged once per chunk,
+  // by log-sum-exp, through the K/V ring (free once the chunk's blocks are done).
   const int nchunks = (rows + kRowChunk - 1) / kRowChunk;
   // one chunk of rows: the partials go straight into the shared memory of the CTAs that
   // merge them (st.async, counted on the owner's mbarrier), with no workspace round trip and
   // no cluster barrier; more rows go through the caller's workspace
   const bool dsm = nchunks == 1;
-  const int total = nchunks * n_my;
   float* wsu = p.ws + (unit * kMaxCluster + rank) * (size_t)p.rows_max * (D + 2);
-  int issued = 0;
-  // the next block in processing order: K and V as TMA boxes (128-byte swizzled tiles)
-  // issued by thread 0, landing on the stage's mbarrier
-  auto issue = [&]() {
-    const int stg = issued % kStages;
-    if (tid == 0) {
-      unsigned char* st = kv + (size_t)stg * 2 * kv_tile;
-      const int j = ulist[rank + (issued % n_my) * CL];
-      tc::fence_proxy_async();  // earlier generic accesses to this stage come first
-      tc::mbar_arrive_expect_tx(&xbar[3 + stg], (uint32_t)(2 * kv_tile));
+  __shared__ int stage_rel[kStages];  // warps done with the stage's current block (mod 8)
+  __shared__ int n_issued;             // block loads issued so far
+  // block `it` of the processing order (row chunk it / n_my, union entry it % n_my): K and V
+  // as TMA boxes (128-byte swizzled tiles) into stage it % kStages, landing on the stage's
+  // mbarrier; called by one thread
+  auto issue = [&](int it) {
+    unsigned char* st = kv + (size_t)(it % kStages) * 2 * kv_tile;
+    const int j = ulist[rank + (it % n_my) * CL];
+    tc::fence_proxy_async();  // earlier generic accesses to this stage come first
+    tc::mbar_arrive_expect_tx(&xbar[3 + it % kStages], (uint32_t)(2 * kv_tile));
 #pragma unroll
-      for (int h = 0; h < D / 64; ++h) {
-        tc::tma_load_3d(st + h * 8192, &p.tmk, h * 64, j * kBlk, (int)unit, &xbar[3 + stg]);
-        tc::tma_load_3d(st + kv_tile + h * 8192, &p.tmv, h * 64, j * kBlk, (int)unit, &xbar[3 + stg]);
-      }
+    for (int h = 0; h < D / 64; ++h) {
+      tc::tma_load_3d(st + h * 8192, &p.tmk, h * 64, j * kBlk, (int)unit, &xbar[3 + it % kStages]);
+      tc::tma_load_3d(st + kv_tile + h * 8192, &p.tmv, h * 64, j * kBlk, (int)unit, &xbar[3 + it % kStages]);
     }
-    ++issued;
+    atomicMax(&n_issued, it + 1);
   };
+  if (tid == 0) {
+    for (int s = 0; s < kStages; ++s) stage_rel[s] = 0;
+    n_issued = 0;
+  }
   __syncthreads();  // (the selection buffers that share the ring are dead)
-  while (issued < kStages && issued < total) issue();
+  if (tid == 0 && rows > 0)
+    for (int it = 0; it < kStages && it < n_my; ++it) issue(it);
 
-  constexpr int NT = D / 64;  // n8 tiles of the output per warp
+  constexpr int NA = D / 8;   // n8 tiles of the output: all of D in every warp
+  constexpr int KS = D / 16;  // k16 steps of Q K^T
+  const int mt = warp & 1, kq = warp >> 1;
   const float scale2 = p.scale * kLog2e;
-  const int srow = tid >> 3, ssub = tid & 7;  // softmax mapping: 32 rows x 8 threads
-  float m_run = -INFINITY, l_run = 0.f;
-  float acc[2][NT][4];
+  // (m, l) of every row per key quarter, posted for the merge at the end of a chunk
+  __shared__ float2 qml[kWarps / 2][kRowChunk];
+  // the merge buffer over the ring: [key quarter][row][D] fp32, 32-byte granules of a row
+  // XOR-swizzled by (row & 3) (the fragment stores and the float4 reads are conflict-free)
+  float* mb = reinterpret_cast<float*>(kv);
+  const int r_lo = 16 * mt + (lane >> 2), r_hi = r_lo + 8;  // this lane's rows in the chunk
+  const int mr = tid >> 3, mc = tid & 7;  // merge mapping: row mr, columns 32 i + 4 mc .. + 3
+  float M_row = -INFINITY, L_row = 0.f;
+  float4 o_row[D / 32];
 
   for (int c = 0; c < nchunks; ++c) {
     const int c0 = c * kRowChunk;
@@ -471,139 +494,165 @@ __global__ void __launch_bounds__(kThreads, 2) blockquery_kernel(const __grid_co
       cp_async_commit();
     }
     cp_async_wait<0>();
-    m_run = -INFINITY;
-    l_run = 0.f;
-#pragma unroll
-    for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-      for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) acc[mt][nt][e] = 0.f;
     __syncthreads();
+    const bool live = 16 * mt < nr;  // (a warp of padding rows only waits and releases)
+    float m_lo = -INFINITY, m_hi = -INFINITY, l_lo = 0.f, l_hi = 0.f;
+    float acc[NA][4];
+#pragma unroll
+    for (int n = 0; n < NA; ++n)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc[n][e] = 0.f;
+    const int q_row = 16 * mt + (lane & 7) + 8 * ((lane >> 3) & 1);  // ldmatrix row of the A tile
 
     for (int i = 0; i < n_my; ++i) {
       const int it = c * n_my + i;
       tc::mbar_wait(&xbar[3 + it % kStages], (uint32_t)((it / kStages) & 1), &xabort, p.budget);
-      __syncthreads();
       const int j = ulist[rank + i * CL];
       const unsigned char* Ks = kv + (size_t)(it % kStages) * 2 * kv_tile;
       const unsigned char* Vs = Ks + kv_tile;
-      {  // V rows past the prefix hold other tokens: zero them (P is 0 there, V must be finite)
-        const int nv = min(kBlk, p.T_prefix - j * kBlk);
-        for (int id = tid; id < (kBlk - nv) * (D / 8); id += kThreads) {
-          const int r = nv + id / (D / 8), cc = id % (D / 8);
-          *reinterpret_cast<uint4*>(const_cast<unsigned char*>(Vs) + kv_off(r, cc)) = make_uint4(0u, 0u, 0u, 0u);
-        }
-      }
-      // S = Q K^T: warp w -> tokens 8w .. 8w+7, both m-tiles
-      {
+      if (live) {
+        // S = Q K^T for my 16 rows x 16 keys: s[nt] = keys 8 nt .. 8 nt + 7 of my quarter
         float s[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
 #pragma unroll
-        for (int ks = 0; ks < D / 16; ks += 2) {
-          uint32_t kb[4];
-          ldsm_x4(kb, Ks + kv_off(8 * warp + (lane & 7), 2 * ks + (lane >> 3)));
-#pragma unroll
-          for (int mt = 0; mt < 2; ++mt) {
-            const int row = 16 * mt + (lane & 7) + 8 * ((lane >> 3) & 1);
-            uint32_t qa0[4], qa1[4];
-            ldsm_x4(qa0, Qs + swz(row, 2 * ks + (lane >> 4), kRowBytes));
-            ldsm_x4(qa1, Qs + swz(row, 2 * ks + 2 + (lane >> 4), kRowBytes));
-            mma_bf16(s[mt], qa0, kb[0], kb[1]);
-            mma_bf16(s[mt], qa1, kb[2], kb[3]);
-          }
+        for (int ks = 0; ks < KS; ++ks) {
+          uint32_t qa[4], kb[4];
+          ldsm_x4(qa, Qs + swz(q_row, 2 * ks + (lane >> 4), kRowBytes));
+          ldsm_x4(kb, Ks + kv_off(16 * kq + (lane & 7) + 8 * (lane >> 4), 2 * ks + ((lane >> 3) & 1)));
+          mma_bf16(s[0], qa, kb[0], kb[1]);
+          mma_bf16(s[1], qa, kb[2], kb[3]);
         }
-        const int col = 8 * warp + 2 * (lane & 3);
-        const bool v0 = j * kBlk + col < p.T_prefix, v1 = j * kBlk + col + 1 < p.T_prefix;
+        // online softmax in base 2 over my quarter (row maxima over the lane quad); keys
+        // past the prefix are -inf
+        const int key0 = j * kBlk + 16 * kq + 2 * (lane & 3);
+        float x[2][4];
 #pragma unroll
-        for (int mt = 0; mt < 2; ++mt) {
-          const int r0 = 16 * mt + (lane >> 2);
-          *reinterpret_cast<float2*>(Ss + r0 * kSStride + col) =
-              make_float2(v0 ? s[mt][0] * scale2 : -INFINITY, v1 ? s[mt][1] * scale2 : -INFINITY);
-          *reinterpret_cast<float2*>(Ss + (r0 + 8) * kSStride + col) =
-              make_float2(v0 ? s[mt][2] * scale2 : -INFINITY, v1 ? s[mt][3] * scale2 : -INFINITY);
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            x[nt][e] = key0 + 8 * nt + (e & 1) < p.T_prefix ? s[nt][e] * scale2 : -INFINITY;
+        float mx_lo = fmaxf(fmaxf(x[0][0], x[0][1]), fmaxf(x[1][0], x[1][1]));
+        float mx_hi = fmaxf(fmaxf(x[0][2], x[0][3]), fmaxf(x[1][2], x[1][3]));
+#pragma unroll
+        for (int o = 1; o <= 2; o <<= 1) {
+          mx_lo = fmaxf(mx_lo, __shfl_xor_sync(0xffffffffu, mx_lo, o));
+          mx_hi = fmaxf(mx_hi, __shfl_xor_sync(0xffffffffu, mx_hi, o));
         }
-      }
-      __syncthreads();
-      // online softmax: row srow, columns 8*ssub .. 8*ssub+7
-      {
-        const float4 sa = *reinterpret_cast<const float4*>(Ss + srow * kSStride + 8 * ssub);
-        const float4 sb4 = *reinterpret_cast<const float4*>(Ss + srow * kSStride + 8 * ssub + 4);
-        float mx = fmaxf(fmaxf(fmaxf(sa.x, sa.y), fmaxf(sa.z, sa.w)), fmaxf(fmaxf(sb4.x, sb4.y), fmaxf(sb4.z, sb4.w)));
+        const float mn_lo = fmaxf(m_lo, mx_lo), mn_hi = fmaxf(m_hi, mx_hi);
+        // a row with no valid key so far subtracts 0: its P is 0 and its (zero) state stays
+        const float base_lo = mn_lo == -INFINITY ? 0.f : mn_lo;
+        const float base_hi = mn_hi == -INFINITY ? 0.f : mn_hi;
+        const float a_lo = ex2(m_lo - base_lo), a_hi = ex2(m_hi - base_hi);
+        float pr[2][4];
 #pragma unroll
-        for (int o = 4; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-        const float m_new = fmaxf(m_run, mx);
-        float pv[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-        float alpha = 1.f;
-        if (m_new != -INFINITY) {
-          alpha = ex2(m_run - m_new);
-          pv[0] = ex2(sa.x - m_new); pv[1] = ex2(sa.y - m_new);
-          pv[2] = ex2(sa.z - m_new); pv[3] = ex2(sa.w - m_new);
-          pv[4] = ex2(sb4.x - m_new); pv[5] = ex2(sb4.y - m_new);
-          pv[6] = ex2(sb4.z - m_new); pv[7] = ex2(sb4.w - m_new);
+        for (int nt = 0; nt < 2; ++nt) {
+          pr[nt][0] = ex2(x[nt][0] - base_lo); pr[nt][1] = ex2(x[nt][1] - base_lo);
+          pr[nt][2] = ex2(x[nt][2] - base_hi); pr[nt][3] = ex2(x[nt][3] - base_hi);
         }
-        float ps = ((pv[0] + pv[1]) + (pv[2] + pv[3])) + ((pv[4] + pv[5]) + (pv[6] + pv[7]));
-#pragma unroll
-        for (int o = 4; o > 0; o >>= 1) ps += __shfl_xor_sync(0xffffffffu, ps, o);
-        l_run = l_run * alpha + ps;
-        m_run = m_new;
-        *reinterpret_cast<uint4*>(Ps + swz(srow, ssub, kBlk * 2)) =
-            make_uint4(pack_bf16x2(pv[0], pv[1]), pack_bf16x2(pv[2], pv[3]),
-                       pack_bf16x2(pv[4], pv[5]), pack_bf16x2(pv[6], pv[7]));
-        if (ssub == 0) alpha_s[srow] = alpha;
-      }
-      __syncthreads();
-      // O = alpha * O + P V: warp w -> output dims of its n-tiles, both m-tiles
-#pragma unroll
-      for (int mt = 0; mt < 2; ++mt) {
-        const float a_lo = alpha_s[16 * mt + (lane >> 2)], a_hi = alpha_s[16 * mt + (lane >> 2) + 8];
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-          acc[mt][nt][0] *= a_lo; acc[mt][nt][1] *= a_lo;
-          acc[mt][nt][2] *= a_hi; acc[mt][nt][3] *= a_hi;
+        l_lo = fmaf(l_lo, a_lo, (pr[0][0] + pr[0][1]) + (pr[1][0] + pr[1][1]));
+        l_hi = fmaf(l_hi, a_hi, (pr[0][2] + pr[0][3]) + (pr[1][2] + pr[1][3]));
+        m_lo = mn_lo;
+        m_hi = mn_hi;
+        // the S fragments are the A fragments of P (16 rows x 16 keys)
+        const uint32_t pa[4] = {pack_bf16x2(pr[0][0], pr[0][1]), pack_bf16x2(pr[0][2], pr[0][3]),
+                                pack_bf16x2(pr[1][0], pr[1][1]), pack_bf16x2(pr[1][2], pr[1][3])};
+        // V rows past the prefix hold other tokens: P is 0 there, and V is masked to 0 in
+        // the B fragments (lane: keys 2 (lane & 3) + {0, 1} in the low / high halves, + 8 in
+        // the second register) so that no NaN reaches the sum
+        const int nvk = p.T_prefix - (j * kBlk + 16 * kq);
+        uint32_t vm0 = 0xffffffffu, vm1 = 0xffffffffu;
+        if (nvk < 16) {
+          const int k0 = 2 * (lane & 3);
+          vm0 = (k0 < nvk ? 0x0000ffffu : 0u) | (k0 + 1 < nvk ? 0xffff0000u : 0u);
+          vm1 = (k0 + 8 < nvk ? 0x0000ffffu : 0u) | (k0 + 9 < nvk ? 0xffff0000u : 0u);
         }
-      }
+        // O = alpha O + P V over all of D
 #pragma unroll
-      for (int ks = 0; ks < kBlk / 16; ++ks) {
-        const int vrow = 16 * ks + (lane & 7) + 8 * ((lane >> 3) & 1);
-        uint32_t vb[4];
-        if constexpr (D == 128) {
-          ldsm_x4_t(vb, Vs + kv_off(vrow, 2 * warp + (lane >> 4)));
-        } else {
-          uint32_t v2[2];
-          ldsm_x2_t(v2, Vs + kv_off(vrow, warp));
-          vb[0] = v2[0]; vb[1] = v2[1]; vb[2] = 0u; vb[3] = 0u;
+        for (int n = 0; n < NA; ++n) {
+          acc[n][0] *= a_lo; acc[n][1] *= a_lo;
+          acc[n][2] *= a_hi; acc[n][3] *= a_hi;
         }
 #pragma unroll
-        for (int mt = 0; mt < 2; ++mt) {
-          uint32_t pa[4];
-          const int row = 16 * mt + (lane & 7) + 8 * ((lane >> 3) & 1);
-          ldsm_x4(pa, Ps + swz(row, 2 * ks + (lane >> 4), kBlk * 2));
-          mma_bf16(acc[mt][0], pa, vb[0], vb[1]);
-          if constexpr (NT == 2) mma_bf16(acc[mt][1], pa, vb[2], vb[3]);
+        for (int np = 0; np < NA / 2; ++np) {
+          uint32_t vb[4];
+          ldsm_x4_t(vb, Vs + kv_off(16 * kq + (lane & 7) + 8 * ((lane >> 3) & 1), 2 * np + (lane >> 4)));
+          mma_bf16(acc[2 * np], pa, vb[0] & vm0, vb[1] & vm1);
+          mma_bf16(acc[2 * np + 1], pa, vb[2] & vm0, vb[3] & vm1);
         }
       }
-      __syncthreads();  // the stage may now be refilled
-      if (issued < total) issue();
-    }
-    // partial of this chunk -> workspace: acc rows, then (m, l) (rows that fit one chunk are
-    // pushed to the owners' shared memory instead, below)
-#pragma unroll
-    for (int mt = 0; mt < 2 && !dsm; ++mt) {
-#pragma unroll
-      for (int nt = 0; nt < NT; ++nt) {
-        const int d = (D == 128 ? 16 * warp : 8 * warp) + 8 * nt + 2 * (lane & 3);
-#pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          const int r = 16 * mt + (lane >> 2) + 8 * half;
-          if (r < nr)
-            *reinterpret_cast<float2*>(wsu + (size_t)(c0 + r) * (D + 2) + d) =
-                make_float2(acc[mt][nt][2 * half], acc[mt][nt][2 * half + 1]);
+      // release the stage: the last of the eight warps refills it with the block kStages
+      // later in this chunk (after a timeout nothing more is loaded)
+      __syncwarp();
+      if (lane == 0) {
+        __threadfence_block();
+        const int old = atomicAdd(&stage_rel[it % kStages], 1);
+        if ((old & (kWarps - 1)) == kWarps - 1 && i + kStages < n_my) {
+          __threadfence_block();
+          if (!*reinterpret_cast<volatile int*>(&xabort)) issue(it + kStages);
         }
       }
     }
-    if (!dsm && ssub == 0 && srow < nr)
-      *reinterpret_cast<float2*>(wsu + (size_t)(c0 + srow) * (D + 2) + D) = make_float2(m_run, l_run);
-    __syncthreads();  // Qs / stats are rewritten by the next chunk
+
+    // ---- merge the four key quarters of every row by log-sum-exp ------------------------
+    l_lo += __shfl_xor_sync(0xffffffffu, l_lo, 1);
+    l_lo += __shfl_xor_sync(0xffffffffu, l_lo, 2);
+    l_hi += __shfl_xor_sync(0xffffffffu, l_hi, 1);
+    l_hi += __shfl_xor_sync(0xffffffffu, l_hi, 2);
+    if ((lane & 3) == 0) {
+      qml[kq][r_lo] = make_float2(m_lo, l_lo);
+      qml[kq][r_hi] = make_float2(m_hi, l_hi);
+    }
+    __syncthreads();  // (every warp is past the chunk's last block: the ring is free)
+    {
+      float Ml = -INFINITY, Mh = -INFINITY;
+#pragma unroll
+      for (int q2 = 0; q2 < kWarps / 2; ++q2) {
+        Ml = fmaxf(Ml, qml[q2][r_lo].x);
+        Mh = fmaxf(Mh, qml[q2][r_hi].x);
+      }
+      const float f_lo = Ml == -INFINITY ? 0.f : ex2(m_lo - Ml);
+      const float f_hi = Mh == -INFINITY ? 0.f : ex2(m_hi - Mh);
+      float* mrow = mb + (size_t)(kq * kRowChunk + r_lo) * D + 2 * (lane & 3);
+#pragma unroll
+      for (int n = 0; n < NA; ++n) {  // (rows r_lo and r_hi share r & 3)
+        const int gcol = (n ^ (r_lo & 3)) << 3;
+        *reinterpret_cast<float2*>(mrow + gcol) = make_float2(acc[n][0] * f_lo, acc[n][1] * f_lo);
+        *reinterpret_cast<float2*>(mrow + 8 * D + gcol) = make_float2(acc[n][2] * f_hi, acc[n][3] * f_hi);
+      }
+    }
+    __syncthreads();
+    M_row = -INFINITY;
+    L_row = 0.f;
+#pragma unroll
+    for (int q2 = 0; q2 < kWarps / 2; ++q2) M_row = fmaxf(M_row, qml[q2][mr].x);
+    if (M_row != -INFINITY) {
+#pragma unroll
+      for (int q2 = 0; q2 < kWarps / 2; ++q2) L_row = fmaf(qml[q2][mr].y, ex2(qml[q2][mr].x - M_row), L_row);
+    }
+#pragma unroll
+    for (int i = 0; i < D / 32; ++i) {
+      const int off = (((4 * i + (mc >> 1)) ^ (mr & 3)) << 3) + 4 * (mc & 1);
+      float4 t = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int q2 = 0; q2 < kWarps / 2; ++q2) {
+        const float4 u = *reinterpret_cast<const float4*>(mb + (size_t)(q2 * kRowChunk + mr) * D + off);
+        t.x += u.x; t.y += u.y; t.z += u.z; t.w += u.w;
+      }
+      o_row[i] = t;
+    }
+    // partial of this chunk -> workspace: row values, then (m, l) (rows that fit one chunk
+    // are pushed to the owners' shared memory instead, below)
+    if (!dsm && mr < nr) {
+      float* wrow = wsu + (size_t)(c0 + mr) * (D + 2);
+#pragma unroll
+      for (int i = 0; i < D / 32; ++i) {
+        *reinterpret_cast<float2*>(wrow + 32 * i + 4 * mc) = make_float2(o_row[i].x, o_row[i].y);
+        *reinterpret_cast<float2*>(wrow + 32 * i + 4 * mc + 2) = make_float2(o_row[i].z, o_row[i].w);
+      }
+      if (mc == 0) *reinterpret_cast<float2*>(wrow + D) = make_float2(M_row, L_row);
+    }
+    __syncthreads();  // (the merge buffer is read; Qs and qml are rewritten by the next chunk)
+    if (c + 1 < nchunks && tid == 0 && !*reinterpret_cast<volatile int*>(&xabort))
+      for (int it = (c + 1) * n_my; it < (c + 1) * n_my + min(kStages, n_my); ++it) issue(it);
   }
 
   // ---- barrier (the partials are in the workspace), then merge my output slice ----------
@@ -665,31 +714,22 @@ __global__ void __launch_bounds__(kThreads, 2) blockquery_kernel(const __grid_co
     if (d == 0) p.lse[orow] = M == -INFINITY ? -INFINITY : (M + log2f(Lsum)) * kLn2;
   };
   if (dsm) {
-    // slice of the outputs each CTA merges (even, so a pushed pair never straddles two)
-    const int chunk = ((E + CL - 1) / CL + 1) & ~1;
+    // slice of the outputs each CTA merges (a multiple of 4, so a pushed float4 never
+    // straddles two)
+    const int chunk = ((E + CL - 1) / CL + 3) & ~3;
     if (tid == 0) {
       const int own = max(0, min(E, (rank + 1) * chunk) - rank * chunk);
       tc::mbar_arrive_expect_tx(&xbar[3 + kStages], (uint32_t)(CL * (rows * 8 + own * 4)));
     }
-    if (srow < rows)
-      for (int peer = ssub; peer < CL; peer += 8)
-        st_async(map_rank(pml + rank * kRowChunk + srow, peer), make_float2(m_run, l_run),
+    if (mr < rows) {
+      for (int peer = mc; peer < CL; peer += 8)
+        st_async(map_rank(pml + rank * kRowChunk + mr, peer), make_float2(M_row, L_row),
                  map_rank(&xbar[3 + kStages], peer));
 #pragma unroll
-    for (int mt = 0; mt < 2; ++mt) {
-#pragma unroll
-      for (int nt = 0; nt < NT; ++nt) {
-        const int d = (D == 128 ? 16 * warp : 8 * warp) + 8 * nt + 2 * (lane & 3);
-#pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          const int r = 16 * mt + (lane >> 2) + 8 * half;
-          if (r < rows) {
-            const int e = r * D + d, owner = e / chunk;
-            st_async(map_rank(pacc + rank * chunk + (e - owner * chunk), owner),
-                     make_float2(acc[mt][nt][2 * half], acc[mt][nt][2 * half + 1]),
-                     map_rank(&xbar[3 + kStages], owner));
-          }
-        }
+      for (int i = 0; i < D / 32; ++i) {
+        const int e = mr * D + 32 * i + 4 * mc, owner = e / chunk;
+        st_async4(map_rank(pacc + rank * chunk + (e - owner * chunk), owner), o_row[i],
+                 map_rank(&xbar[3 + kStages], owner));
       }
     }
     tc::mbar_wait(&xbar[3 + kStages], 0, &xabort, p.budget);
@@ -763,7 +803,8 @@ __global__ void __launch_bounds__(kThreads, 2) blockquery_kernel(const __grid_co
       for (int c = nsel_chunks - 2 < 0 ? 0 : nsel_chunks - 2; c < nsel_chunks; ++c)
         tc::mbar_drain(&xbar[c & 1], (uint32_t)((c >> 1) & 1), kDrainBudget);
     }
-    for (int i = issued - kStages < 0 ? 0 : issued - kStages; i < issued; ++i)
+    const int n_iss = *reinterpret_cast<volatile int*>(&n_issued);
+    for (int i = n_iss - kStages < 0 ? 0 : n_iss - kStages; i < n_iss; ++i)
       tc::mbar_drain(&xbar[3 + i % kStages], (uint32_t)((i / kStages) & 1), kDrainBudget);
     if (dsm) tc::mbar_drain(&xbar[3 + kStages], 0, kDrainBudget);  // (the partials peers owe)
     g_blockquery_status = 1;
