@@ -1246,7 +1246,9 @@ def run_decode_blasst(args):
         "plain_given_selection_decode_us_median": round(med_p * 1e3, 3),
         "bytes_per_step": int(step_bytes), "plain_bytes_per_step": int(plain_bytes),
         "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peak, "unit": "GB/s",
-                     "frac": round(gbs / peak, 4), "traffic": None, "kernel": "decode_blasst_kernel<128>",
+                     "frac": round(gbs / peak, 4), "traffic": None,
+                     # (the library runs one CTA per (b, g) unit from 64 units up, else a cluster per unit)
+                     "kernel": "decode_blasst_unit_kernel<128>" if B * Hkv >= 64 else "decode_blasst_kernel<128>",
                      "peak_source": f"MEASURED_PEAKS.json hbm_gbs ({kind}, of measured)"},
         "gpu_launches": reps * R * 2,
         "clocks": clocks.summary(),
