@@ -264,7 +264,8 @@ LSA_API int lsa_copy_async(void* dst, const void* src, size_t bytes, int flags, 
  *   every active row (b, h in g, i) attends over all tokens t < T_prefix of the blocks in
  *   U(b, g) (no mask inside the prefix): o = softmax-weighted v, lse = log-sum-exp.
  * Stable rows (active == 0): o[b,h,i,:] = o_cache[b,h,i,:] and lse = lse_cache, bit-exact
- * (o_cache / lse_cache may alias o / lse, in which case stable rows are left as they are).
+ * (o_cache / lse_cache may alias o / lse, in which case stable rows are left as they are;
+ * a partial overlap of o with o_cache, or of lse with lse_cache, is LSA_ERR_INVALID_ARG).
  *
  * q [B, Hq, Tq, D] bf16; k, v [B, Hkv, T_cap, D] bf16 (T_prefix <= T_cap);
  * summ [B, Hkv, NB_cap, D] float32; active [B, Tq] uint8;
@@ -280,7 +281,7 @@ LSA_API int lsa_copy_async(void* dst, const void* src, size_t bytes, int flags, 
  * early; a next kernel launched with programmatic dependent launch must wait for this
  * one's completion before reading its outputs (lsa_blockquery_intra_merge with
  * LSA_FLAG_PDL does).
- * Requires bf16, 1 <= Tq <= 64, n_sink + n_local <= topk_per_query, and either
+ * Requires bf16, 1 <= Tq <= 64, B and Hkv <= 65535, n_sink + n_local <= topk_per_query, and either
  * 1 <= topk_per_query <= 16 or topk_per_query >= NBp.  The latter selects every prefix
  * block: with every token active this is the dense first denoising step of a block
  * (LoSA, "2. 방법론": the first step attends densely to build the cache, later steps

@@ -332,6 +332,16 @@ int lsa_sparse_attn_blockquery(const void* q, const void* k, const void* v, int 
       !aligned16(o_cache) || !aligned16(workspace))
     return LSA_ERR_INVALID_ARG;
   if (ws_bytes < lsa::blockquery_workspace_bytes(B, Hkv, G, D, Tq)) return LSA_ERR_INVALID_ARG;
+  if (B > 65535 || Hkv > 65535) return LSA_ERR_UNSUPPORTED;  // (grid y, z)
+  // o may be o_cache and lse may be lse_cache (stable rows are then left as they are); a
+  // partial overlap would let the copy of one stable row overwrite another's cached value
+  {
+    const size_t obytes = (size_t)B * Hkv * G * Tq * D * 2, lbytes = (size_t)B * Hkv * G * Tq * 4;
+    const uintptr_t o0 = (uintptr_t)o, c0 = (uintptr_t)o_cache, l0 = (uintptr_t)lse,
+                    lc0 = (uintptr_t)lse_cache;
+    if (o0 != c0 && o0 < c0 + obytes && c0 < o0 + obytes) return LSA_ERR_INVALID_ARG;
+    if (l0 != lc0 && l0 < lc0 + lbytes && lc0 < l0 + lbytes) return LSA_ERR_INVALID_ARG;
+  }
   lsa::BlockQueryArgs a = {};
   a.q = q; a.k = k; a.v = v;
   a.B = B; a.Hkv = Hkv; a.G = G; a.D = D; a.Tq = Tq; a.T_prefix = T_prefix; a.T_cap = T_cap;

@@ -114,6 +114,15 @@ def test_losa_entry_points_validation():
     args = lambda topk, T: (g, g, g, 1, 1, 8, 4, 128, 32, T, T + 32, g, 64, topk, 0, 0, 0.0, g, g, g, g, g, NULL, NULL, g, 0, NULL)
     assert bq(*args(17, 64 * 100)) == lsa.LSA_ERR_INVALID_ARG
     assert bq(*args(0, 64 * 100)) == lsa.LSA_ERR_INVALID_ARG
+    # o / lse may be o_cache / lse_cache, but must not overlap them partially
+    ws = 1 << 30
+    over = lambda o, lse: (g, g, g, 1, 1, 8, 4, 128, 32, 6400, 6432, g, 64, 8, 1, 2, 0.0, g,
+                           g, g, o, lse, NULL, NULL, g, ws, NULL)
+    assert bq(*over(ctypes.c_void_p(4096 + 256), ctypes.c_void_p(big))) == lsa.LSA_ERR_INVALID_ARG
+    assert bq(*over(ctypes.c_void_p(big), ctypes.c_void_p(4096 + 4))) == lsa.LSA_ERR_INVALID_ARG
+    # more sequences than a grid dimension holds
+    assert bq(g, g, g, 1, 65536, 1, 4, 128, 8, 6400, 6432, g, 64, 8, 1, 2, 0.0, g, g, g,
+              ctypes.c_void_p(big), ctypes.c_void_p(big), NULL, NULL, g, 1 << 62, NULL) == lsa.LSA_ERR_UNSUPPORTED
 
 
 def test_decode_blasst_validation():
