@@ -50,8 +50,9 @@
  *           Summaries summ: [B, Hkv, NB_cap, D] float32.
  * Types.    dtype = LSA_F32 or LSA_BF16 for q, k, v and o.  lse, summaries and scores are
  *           always float32; indices int32.
- * Support.  D in {64, 128}; blk == 64; G <= 16.  bf16 everywhere; fp32 in summaries,
- *           selection and decode.  Anything else returns LSA_ERR_UNSUPPORTED.
+ * Support.  D in {64, 128}; blk == 64; G <= 16; B and Hkv <= 65535 (grid dimensions).
+ *           bf16 everywhere; fp32 in summaries, selection and decode.  Anything else
+ *           returns LSA_ERR_UNSUPPORTED.
  * Scale.    scale <= 0 means 1/sqrt(D).
  * Errors.   Every argument is validated on the host before anything is launched; on
  *           error nothing is enqueued and the status is returned.  LSA_ERR_CUDA means a

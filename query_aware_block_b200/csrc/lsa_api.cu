@@ -40,6 +40,7 @@ int check_common(int dtype, int B, int Hkv, int G, int D, int blk) {
   if (D != 64 && D != 128) return LSA_ERR_UNSUPPORTED;
   if (blk != 64) return LSA_ERR_UNSUPPORTED;
   if (G > 16) return LSA_ERR_UNSUPPORTED;
+  if (B > 65535 || Hkv > 65535) return LSA_ERR_UNSUPPORTED;  // (grid y and z of the launches)
   return LSA_OK;
 }
 

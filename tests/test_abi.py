@@ -84,6 +84,10 @@ def test_select_and_decode_validation():
     # overlapped launch only in fused mode; unknown flags rejected
     assert dec(g, g, g, 1, 1, 8, 8, 128, 65536, g, 64, g, g, 16, 0.0, NULL, 1, 2, 0, NULL, g, NULL, 1, NULL) == lsa.LSA_ERR_INVALID_ARG
     assert dec(g, g, g, 1, 1, 8, 8, 128, 65536, g, 64, NULL, NULL, 16, 0.0, g, 1, 2, 0, NULL, g, NULL, 2, NULL) == lsa.LSA_ERR_INVALID_ARG
+    # B or Hkv past a grid dimension
+    assert dec(g, g, g, 1, 65536, 1, 8, 128, 4096, g, 64, NULL, NULL, 16, 0.0, g, 1, 2, 0, NULL, g, NULL, 0, NULL) == lsa.LSA_ERR_UNSUPPORTED
+    assert sel(g, 1, g, 1, 65536, 8, 128, 64, g, 64, 16, 1, 2, 0.0, g, g, NULL, NULL) == lsa.LSA_ERR_UNSUPPORTED
+    assert lib.lsa_build_summaries(g, 1, 1, 65536, 4096, 128, g, 64, 0, -1, g, NULL) == lsa.LSA_ERR_UNSUPPORTED
 
 
 def test_losa_entry_points_validation():
