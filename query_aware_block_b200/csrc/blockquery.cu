@@ -650,6 +650,9 @@ __global__ void __launch_bounds__(kThreads, 2) blockquery_kernel(const __grid_co
       }
       if (mc == 0) *reinterpret_cast<float2*>(wrow + D) = make_float2(M_row, L_row);
     }
+    // every thread's generic accesses to the ring (the merge buffer) before the next chunk's
+    // TMA writes into it
+    tc::fence_proxy_async();
     __syncthreads();  // (the merge buffer is read; Qs and qml are rewritten by the next chunk)
     if (c + 1 < nchunks && tid == 0 && !*reinterpret_cast<volatile int*>(&xabort))
       for (int it = (c + 1) * n_my; it < (c + 1) * n_my + min(kStages, n_my); ++it) issue(it);
