@@ -98,6 +98,16 @@ MUTANTS = [
     ("sparse-decode rescale factor inverted",
      "exp(m[hh] - mn)", "exp(mn - m[hh])",
      pins.test_decode_blasst_lambda_zero_is_masked_dense),
+    ("group score from the first head only",
+     "          acc += dot;\n        }\n        *s = scale * acc;",
+     "          acc += dot;\n          break;\n        }\n        *s = scale * acc;",
+     pins.test_group_score_is_sum_of_single_head_scores),
+    ("compressed-branch log-sum-exp without the max",
+     "      lse[(size_t)b * Hq + h] = m + log(l);", "      lse[(size_t)b * Hq + h] = log(l);",
+     pins.test_nsa_window_and_compressed_branches_are_sdpa),
+    ("compressed-branch logits without the softmax scale",
+     "        logit[t - t0] = scale * dot;", "        logit[t - t0] = dot;",
+     pins.test_nsa_window_and_compressed_branches_are_sdpa),
 ]
 
 
