@@ -447,6 +447,7 @@ int lsa_debug_inject(int kind) {
   return LSA_OK;
 }
 
+#ifdef LSA_DEBUG_BOUNDS
 // The first recorded bounds violation over the translation units (0 if none).
 static int bounds_code(bool reset, cudaError_t* err) {
   cudaError_t (*readers[])(int*, bool) = {lsa::read_bounds_summaries, lsa::read_bounds_decode,
@@ -465,6 +466,7 @@ static int bounds_code(bool reset, cudaError_t* err) {
   }
   return first;
 }
+#endif
 
 int lsa_debug_bounds_code(int* code, int reset) {
   if (!code) return LSA_ERR_INVALID_ARG;

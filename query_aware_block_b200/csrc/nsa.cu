@@ -86,7 +86,6 @@ __global__ void __launch_bounds__(kPoolThreads) nsa_compress_kernel(
 
 // ---- the window and compressed branches, merged and gated ------------------------------
 constexpr int kThreads = 256;
-constexpr int kWarps = kThreads / 32;
 constexpr int kCL = 16;
 constexpr int kMaxG = 16;
 constexpr int kTile = 64;
